@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""Throughput of the B200 audio-encoder forward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload tower|ragged|frontend|attention]
+    python bench.py --impl reference ...      # the CPU oracle on the same workload (bounded sample)
+
+A step is one ae_encode over one batch (default: 16 clips x 30 s, the
+12-layer tower plus the embedding head, bf16 tensor-core projections),
+inputs resident in device memory. K steps are timed with CUDA events on the
+launching stream after W warm-up steps, L2 flushed (256 MiB written)
+between steps, outside the events. With N > 1 (torchrun), every rank runs
+its own replica of the batch (weak scaling, no data-path collective); the
+step time is the max over ranks and the value counts every rank's audio.
+
+One JSON line on rank 0: the metric, the end-to-end figure through
+ae_encode_host (host buffers, copies inside the timed region), the roofline
+of the dominant kernel class from the library's per-launch event timing,
+the clocks seen during the timed region, and the oracle's CPU baseline.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "audio seconds encoded/sec (soft tokens/sec) on 1 B200; % HBM / % tensor peak"
+UNIT = "audio-s/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+
+class Clocks:
+    """nvidia-smi sampled every 200 ms during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        time.sleep(0.3)
+        if self.p:
+            self.p.terminate()
+            try:
+                self.p.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.p.kill()
+
+    def summary(self):
+        self.f.flush()
+        rows = []
+        for line in open(self.f.name):
+            c = [x.strip() for x in line.split(",")]
+            if len(c) < 10:
+                continue
+            try:
+                rows.append((float(c[1]), float(c[2]), float(c[4]), c[6], c[7], c[8], c[9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        busy = [r for r in rows if r[2] >= 30] or rows
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in busy for n, v in zip(names, r[3:]) if v.lower().startswith("active")})
+        return {"sm_mhz": float(np.median([r[0] for r in busy])), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(busy)}
+
+
+# ------------------------------------------------------------------ workloads
+
+def workload_desc(name: str, info: dict) -> dict:
+    base = {"tower": "16 clips x 30 s, 12 Conformer layers + embedding head, bf16 weights, f32 accumulation",
+            "ragged": "256 clips of 1-30 s (uniform whole samples), packed, 12 layers + head, bf16",
+            "frontend": "log-mel front-end only, 64 clips x 30 s, f32",
+            "attention": "local-attention core only, 32 x 8192 tokens, 8 heads x 128, bf16 q/k/v"}[name]
+    d = {"workload": f"{name}: {base}", "l2": "flushed between steps (256 MiB write)",
+         "model": "gemma4_audio tower shape (random init)"}
+    d.update(info)
+    return d
+
+
+class Ours:
+    def __init__(self, name: str):
+        import torch
+        import log_mel_front_b200 as ae
+        self.ae, self.torch, self.name = ae, torch, name
+        self.stream = torch.cuda.current_stream()
+        if name in ("tower", "ragged", "frontend"):
+            self.lens = synth.clip_lengths(name)
+            clips = synth.waves(name)
+            flat, self.off = synth.pack(clips)
+            self.h_wave = torch.from_numpy(flat).pin_memory()
+            self.d_wave = self.h_wave.cuda()
+            self.frames = sum(ae.ae_num_frames(n) for n in self.lens)
+            self.tokens = sum(ae.ae_num_tokens(n) for n in self.lens)
+            self.audio_s = sum(min(n, synth.MAX_SAMPLES) for n in self.lens) / synth.SAMPLE_RATE
+        if name in ("tower", "ragged"):
+            self.model = ae.Model(synth.model_weights(name), ae.AE_BF16)
+            self.ws_bytes = self.model.workspace_size(len(self.lens), self.frames, self.tokens)
+            self.d_out = torch.empty((self.tokens, 512), device="cuda")
+            self.h_out = torch.empty((self.tokens, 512)).pin_memory()
+            self.ws_host_bytes = ae.ae_encode_host_workspace_size(self.model, self.off)
+            self.ws = torch.empty(max(self.ws_bytes, self.ws_host_bytes), dtype=torch.uint8, device="cuda")
+            self.dominant = "gemm"
+        elif name == "frontend":
+            self.ws_bytes = ae.ae_workspace_size(None, len(self.lens), self.frames, 0)
+            self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
+            self.d_mel = torch.empty((self.frames, 128), device="cuda")
+            self.h_mel = torch.empty((self.frames, 128)).pin_memory()
+            self.dominant = "logmel"
+        elif name == "attention":
+            S, T = synth.ATT_SEQS, synth.ATT_T
+            p = synth.attention_params()
+            R, qs, self.ks = ae.ae_attention_tables(p["relk"], p["pds"])
+            self.R, self.qs = torch.from_numpy(R).cuda(), torch.from_numpy(qs).cuda()
+            g = torch.Generator(device="cuda").manual_seed(4)
+            self.q, self.k, self.v = (torch.randn((S * T, 1024), generator=g, device="cuda").to(torch.bfloat16)
+                                      for _ in range(3))
+            self.o = torch.empty_like(self.q)
+            self.tok_off = np.arange(S + 1, dtype=np.int64) * T
+            self.tokens = S * T
+            self.audio_s = self.tokens / 25.0
+            self.ws_bytes = ae.ae_workspace_size(None, S, 0, self.tokens)
+            self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
+            self.dominant = "attention"
+        self.flush = torch.empty(L2_FLUSH_BYTES // 4, device="cuda")
+
+    def step(self):
+        ae = self.ae
+        if self.name in ("tower", "ragged"):
+            ae.ae_encode(self.model, self.d_wave, self.off, self.d_out, self.ws, self.ws_bytes, self.stream)
+        elif self.name == "frontend":
+            ae.ae_logmel(self.d_wave, self.off, self.d_mel, self.ws, self.ws_bytes, self.stream)
+        else:
+            ae.ae_local_attention(self.q, self.k, self.v, 1024, ae.AE_BF16, self.R, self.qs, self.ks, 50.0,
+                                  self.tok_off, self.o, 1024, self.ws, self.ws_bytes, self.stream)
+
+    def step_e2e(self):
+        """One step through the host-buffer path; returns (h2d bytes, d2h bytes)."""
+        ae, torch = self.ae, self.torch
+        if self.name in ("tower", "ragged"):
+            ae.ae_encode_host(self.model, self.h_wave, self.off, self.h_out, self.ws, self.ws.numel(), self.stream)
+            return self.h_wave.numel() * 4, self.h_out.numel() * 4
+        if self.name == "frontend":
+            self.d_wave.copy_(self.h_wave, non_blocking=True)
+            self.step()
+            self.h_mel.copy_(self.d_mel, non_blocking=True)
+            self.stream.synchronize()
+            return self.h_wave.numel() * 4, self.h_mel.numel() * 4
+        return 0, 0
+
+    def timed(self, k: int, fn):
+        torch = self.torch
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k)]
+        for a, b in ev:
+            self.flush.zero_()
+            a.record(self.stream)
+            fn()
+            b.record(self.stream)
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in ev)
+
+
+class OracleRun:
+    """The oracle as it stands, timed on the host cores on a bounded sample of
+    the workload (inputs prepared outside the timing)."""
+
+    def __init__(self, name: str):
+        from oracle import oracle as O
+        self.O, self.name = O, name
+        try:
+            from threadpoolctl import threadpool_info
+            self.threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        except Exception:
+            self.threads = os.cpu_count() or 1
+        if name in ("tower", "ragged"):
+            self.W = synth.model_weights(name)
+            self.lens = synth.clip_lengths(name)
+            self.next = 0
+        elif name == "attention":
+            p = synth.attention_params()
+            q, k, v = synth.attention_qkv(0, T=2048)
+            self.qkv = [x.astype(np.float64) for x in (q, k, v)]
+            self.R = O.relative_keys(p["relk"], 12, 1024)
+            self.qd = O.softplus(p["pds"])
+
+    def step(self):
+        """One bounded unit of work; returns (seconds, audio seconds, description)."""
+        O = self.O
+        if self.name in ("tower", "ragged"):
+            i = self.next % len(self.lens)
+            self.next += 1
+            c = synth.waves(self.name, [i])[0]
+            t0 = time.perf_counter()
+            O.encode([c], self.W)
+            dt = time.perf_counter() - t0
+            return dt, min(len(c), synth.MAX_SAMPLES) / synth.SAMPLE_RATE, f"clip {i} of the {self.name} workload"
+        if self.name == "frontend":
+            c = synth.waves(self.name, [0])[0]
+            t0 = time.perf_counter()
+            O.log_mel(c)
+            return time.perf_counter() - t0, 30.0, "clip 0 of the frontend workload (log-mel)"
+        t0 = time.perf_counter()
+        O.local_attention_core(*self.qkv, np.arange(2048), self.R, self.qd, 8, 12, 50.0)
+        return time.perf_counter() - t0, 2048 / 25.0, "2048 tokens of one attention sequence"
+
+
+def oracle_baseline(name: str, budget_s: float = 20.0):
+    """(audio-s/s, sample description, threads) of the oracle within about budget_s."""
+    r = OracleRun(name)
+    t = a = 0.0
+    n = 0
+    while n == 0 or t < budget_s:
+        dt, au, _ = r.step()
+        t, a, n = t + dt, a + au, n + 1
+        if name == "tower" and n >= 16:
+            break
+    return a / t, f"{n} unit(s) of the {name} workload through the f64 oracle ({a:.1f} s of audio)", r.threads
+
+
+# ------------------------------------------------------------------ arms
+
+def run_ours(args, rank, world, dist):
+    import torch
+    ours = Ours(args.workload)
+    ae = ours.ae
+    for _ in range(args.warmup):
+        ours.step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    with Clocks(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                else int(os.environ.get("LOCAL_RANK", 0))) as clk:
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        ms = ours.timed(args.steps, ours.step)
+        if dist:
+            t = torch.tensor([ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+            dist.barrier()
+    clocks = clk.summary()
+    # per-kernel-class timing over a replica of the timed region (events around every launch)
+    ae.ae_profile_enable(True)
+    ae.ae_profile_read()
+    ms_prof = ours.timed(args.steps, ours.step)
+    prof = ae.ae_profile_read()
+    ae.ae_profile_enable(False)
+    # end to end through the host-buffer entry point
+    h2d = d2h = 0
+    ms_e2e = None
+    if args.workload != "attention":
+        ours.step_e2e()
+        torch.cuda.synchronize()
+        sizes = []
+
+        def e2e():
+            sizes.append(ours.step_e2e())
+        ms_e2e = ours.timed(args.steps, e2e)
+        if dist:
+            t = torch.tensor([ms_e2e], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        h2d, d2h = sizes[0]
+    if rank != 0:
+        return None
+    pk = peaks()
+    per_step = ms / args.steps
+    audio = ours.audio_s * world
+    value = audio / (per_step / 1e3)
+    launches = sum(v["launches"] for k, v in prof.items() if k != "dropped")
+    dom = prof[ours.dominant]
+    if ours.dominant in ("gemm",):
+        achieved = dom["flops"] / (dom["ms"] / 1e3) / 1e12
+        peak = pk["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "unit": "TFLOP/s", "peak_kind": "bf16 sustained (" + pk["source"] + ")"}
+    else:
+        achieved = dom["bytes"] / (dom["ms"] / 1e3) / 1e9
+        peak = pk["hbm_gbs"]
+        roof = {"bound": "hbm", "unit": "GB/s", "peak_kind": "HBM copy (" + pk["source"] + ")"}
+    roof.update({"kernel": {"gemm": "k_gemm_tc (all projections)", "logmel": "k_logmel",
+                            "attention": "k_attention"}[ours.dominant],
+                 "achieved": round(achieved, 2), "peak": peak, "frac": round(achieved / peak, 4),
+                 "traffic": None, "launches_per_step": dom["launches"] / args.steps,
+                 "share_of_step": round(dom["ms"] / max(ms_prof, 1e-9), 4)})
+    classes = {k: {"ms_per_step": round(v["ms"] / args.steps, 4), "launches_per_step": v["launches"] / args.steps,
+                   **({"tflops": round(v["flops"] / (v["ms"] / 1e3) / 1e12, 1)} if v["flops"] and v["ms"] else {}),
+                   **({"gbs": round(v["bytes"] / (v["ms"] / 1e3) / 1e9, 1)} if v["bytes"] and v["ms"] else {})}
+               for k, v in prof.items() if k != "dropped" and v["launches"]}
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(per_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if args.workload != "frontend" else "f32", "data": "synthetic",
+        "config": workload_desc(args.workload, {
+            "clips": len(getattr(ours, "lens", [])) or synth.ATT_SEQS, "tokens_per_replica": ours.tokens,
+            "audio_seconds_per_replica": round(ours.audio_s, 3), "parallelism": f"replicas x{world}",
+            "soft_tokens_per_s": round(ours.tokens * world / (per_step / 1e3), 1)}),
+        "e2e": None if ms_e2e is None else {
+            "value": round(audio / (ms_e2e / args.steps / 1e3), 2), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "api": "ae_encode_host" if args.workload in ("tower", "ragged") else "ae_logmel + copies"},
+        "gpu_launches": int(launches),
+        "roofline": roof,
+        "kernel_classes": classes,
+        "profiled_ms_per_step": round(ms_prof / args.steps, 4),
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        v, sample, threads = oracle_baseline(args.workload)
+        line["cpu_baseline"] = {"value": round(v, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": sample}
+    return line
+
+
+def run_reference(args):
+    """The base contract's reference arm: the oracle on the host cores, one
+    bounded unit of the workload per step (a 30 s clip for the tower)."""
+    r = OracleRun(args.workload)
+    for _ in range(args.warmup):
+        r.step()
+    t = a = 0.0
+    desc = ""
+    for _ in range(args.steps):
+        dt, au, desc = r.step()
+        t, a = t + dt, a + au
+    v = a / t
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * t / args.steps, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_desc(args.workload, {"parallelism": "cpu"}),
+            "cpu_baseline": {"value": round(v, 4), "unit": UNIT, "cores": r.threads, "kind": "oracle",
+                             "sample": f"one unit per step, e.g. {desc}"},
+            "e2e": {"value": round(v, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=("tower", "ragged", "frontend", "attention"), default="tower")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    import torch
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        line = run_ours(args, rank, world, dist)
+    finally:
+        if dist:
+            dist.barrier()
+            dist.destroy_process_group()
+    if rank == 0 and line:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

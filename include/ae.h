@@ -1,0 +1,264 @@
+/*
+ * ae.h -- C ABI of the B200 (sm_100a) audio-encoder forward: 16 kHz waveform
+ * -> log-mel -> two-conv subsampling stem -> Conformer layers with causal
+ * local attention -> 512-d embedding rows.
+ *
+ * The operations are those of the gemma4_audio tower as the docs.rs page of
+ * cortiq-engine 0.8.49, egemma2_audio.rs, states them (module doc items 1-5,
+ * and the functions named beside each call below).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Pointers named d_* are CUDA device pointers; h_* are host pointers.
+ * - The caller owns every buffer, the workspace and the stream. The library
+ *   owns only an ae_model (weights and load-time tables) until
+ *   ae_model_destroy.
+ * - Clips are packed back to back without padding. A batch of n_clips clips
+ *   is described by host int64 offsets [n_clips + 1], non-decreasing,
+ *   starting at 0 (samples, frames or tokens depending on the call).
+ * - Clips longer than 480000 samples are cut to their first 480000 samples
+ *   (the feature extractor's 30 s truncation). A clip of 160 samples or fewer
+ *   has no frames and no tokens; it is legal and produces no rows.
+ * - Calls are stream-ordered: they enqueue work on `stream` and return
+ *   without waiting for it, except ae_encode_host, which waits. They never
+ *   allocate device memory; all scratch space comes from the caller's
+ *   workspace (d_ws, ws_bytes), whose size ae_workspace_size returns. Two
+ *   calls that share a workspace must be ordered on one stream.
+ * - Every argument is checked on the host before anything is enqueued: null
+ *   pointers, a workspace below the required size, offsets that are not
+ *   monotone, sizes whose indices would not fit the kernels' 32-bit
+ *   arithmetic, and configurations the compiled kernels do not implement.
+ *   A refused call returns an error status, writes nothing and enqueues
+ *   nothing; ae_last_error() then names the offending argument.
+ * - AE_ECUDA reports a CUDA launch or API failure seen by the host when the
+ *   work was enqueued. Faults of kernels that already ran are reported by
+ *   the CUDA runtime on the next synchronising call, as for any kernel.
+ * - There is no CPU fallback: if no CUDA device is usable every compute
+ *   call returns AE_ECUDA.
+ */
+#ifndef AE_H
+#define AE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (NULL = the legacy default stream). */
+typedef struct CUstream_st *ae_stream;
+
+typedef enum {
+  AE_OK = 0,
+  AE_EINVAL = 1,        /* a bad argument (null pointer, bad offsets, bad layer index) */
+  AE_EUNSUPPORTED = 2,  /* a configuration the compiled kernels do not implement */
+  AE_EWORKSPACE = 3,    /* ws_bytes below ae_workspace_size */
+  AE_ECUDA = 4,         /* a CUDA API or launch error */
+  AE_ENOMEM = 5,        /* device memory for the model could not be allocated */
+  AE_EDEVICE = 6        /* a kernel gave up a bounded wait (see ae_device_status) */
+} ae_status;
+
+/* Arithmetic of the tower. AE_F32: float32 weights, activations and
+ * products (CUDA-core FMA). AE_BF16: bf16 weights and bf16 operands of
+ * every projection on the tcgen05 tensor cores with float32 accumulation;
+ * the residual stream, norms, attention and convolution arithmetic stay
+ * float32. The front-end is float32 in both. */
+typedef enum { AE_F32 = 0, AE_BF16 = 1 } ae_dtype;
+
+/* Hyper-parameters of the tower (egemma2_audio.rs, AudioTower::load reads
+ * them from audio_config). The kernels are compiled for the release shape:
+ * n_mels 128, c0 128, c1 32, hidden 1024, heads 8 (head_dim 128), left 12
+ * (attention_context_left 13 minus one), kernel 5; ffn, out_dim and
+ * embed_dim must be multiples of 256; n_layers >= 0. Anything else is
+ * refused with AE_EUNSUPPORTED. attention_context_right must be 0 in the
+ * release and is not a parameter here. */
+typedef struct {
+  int32_t n_mels, c0, c1, hidden, heads, ffn, left, kernel, out_dim, embed_dim, n_layers;
+  float softcap;          /* attention_logit_cap, 50 */
+  float residual_weight;  /* FFN half-residual, 0.5 */
+} ae_config;
+
+/* Input and output bounds of one clippable projection (Gemma4ClippableLinear,
+ * the page's ClipLin): y = clamp(clamp(x, lo_in, hi_in) W^T, lo_out, hi_out).
+ * +-INFINITY means unbounded. */
+typedef struct { float lo_in, hi_in, lo_out, hi_out; } ae_clip;
+
+/* One Conformer layer's weights as host float32 arrays in the checkpoint's
+ * layouts: matrices [out][in] row-major; norm weights [hidden];
+ * per_dim_scale [head_dim]; lc_dw [hidden][kernel]. For AE_BF16 every
+ * matrix is converted to bf16 by round-to-nearest-even at model creation.
+ * q, k and v must share their input bounds (they read the same normalised
+ * activations through one fused projection). */
+typedef struct {
+  const float *ff1_pre, *ff1_w1, *ff1_w2, *ff1_post;
+  const float *ff2_pre, *ff2_w1, *ff2_w2, *ff2_post;
+  const float *norm_pre_attn, *norm_post_attn, *norm_out;
+  const float *q, *k, *v, *post;
+  const float *per_dim_scale, *relative_k;
+  const float *lc_pre, *lc_start, *lc_dw, *lc_norm, *lc_end;
+  ae_clip clip_ff1_w1, clip_ff1_w2, clip_q, clip_k, clip_v, clip_post;
+  ae_clip clip_lc_start, clip_lc_end, clip_ff2_w1, clip_ff2_w2;
+} ae_host_layer;
+
+/* Stem and head weights (host float32): conv0 [c0][1][3][3], ln0 [c0],
+ * conv1 [c1][c0][3][3], ln1 [c1], in_proj [hidden][c1 * n_mels/4],
+ * out_proj [out_dim][hidden], out_bias [out_dim], embed [embed_dim][out_dim],
+ * layers [n_layers]. */
+typedef struct {
+  const float *conv0, *ln0, *conv1, *ln1, *in_proj;
+  const ae_host_layer *layers;
+  const float *out_proj, *out_bias, *embed;
+} ae_host_weights;
+
+typedef struct ae_model ae_model;
+
+/* --- sizes (egemma2_audio.rs, num_frames / num_tokens) --------------------- */
+
+/* Mel frames of a clip of n samples: 0 if min(n, 480000) <= 160, else
+ * ceil((min(n, 480000) - 160) / 160). Negative n gives 0. */
+int64_t ae_num_frames(int64_t n_samples);
+
+/* Soft tokens of a clip of n samples: ceil(ceil(frames / 2) / 2). */
+int64_t ae_num_tokens(int64_t n_samples);
+
+/* --- model ----------------------------------------------------------------- */
+
+/* Validates cfg and the weight pointers, converts and uploads the weights
+ * to the current CUDA device, and computes the load-time tables of each
+ * layer (AudioTower::load): softplus(per_dim_scale) with torch's threshold
+ * of 20, and the relative keys R = pe relative_k^T of distances
+ * 0..left-1 from the sinusoids [sin(d inv) | cos(d inv)],
+ * inv_i = exp(-i ln(1e4) / (hidden/2 - 1)), all in float64 on the host and
+ * stored as float32. Synchronous. On failure *out is NULL. */
+ae_status ae_model_create(const ae_config *cfg, const ae_host_weights *w, ae_dtype dtype,
+                          ae_model **out);
+void ae_model_destroy(ae_model *m);
+
+/* Bytes of workspace that any call below needs for a batch of n_clips clips
+ * holding total_frames mel frames and total_tokens soft tokens in all. With
+ * m == NULL: the workspace of ae_logmel and ae_local_attention. */
+size_t ae_workspace_size(const ae_model *m, int64_t n_clips, int64_t total_frames,
+                         int64_t total_tokens);
+
+/* --- the hot path ------------------------------------------------------------ */
+
+/* Log-mel features (MelFrontend::log_mel): per frame i of each clip,
+ * x_j = wave[160 i + j - 160] (0 before the clip) times the periodic Hann
+ * window 0.5 - 0.5 cos(2 pi j / 320), j < 320, zero-padded to 512; |rfft|;
+ * 128 HTK mel bands over 0-8 kHz without normalisation; ln(mel + 0.001).
+ * d_wave: float32 [h_sample_off[n_clips]]. d_mel: float32 [sum frames][128],
+ * clip after clip. Workspace: ae_workspace_size(NULL, ...). */
+ae_status ae_logmel(const float *d_wave, const int64_t *h_sample_off, int n_clips, float *d_mel,
+                    void *d_ws, size_t ws_bytes, ae_stream stream);
+
+/* Subsampling stem plus input projection (AudioTower::subsample and
+ * input_proj_linear), per clip: 3x3 stride-2 conv 1 -> c0 with zero pad 1,
+ * bias-free LayerNorm over channels (eps 1e-6), ReLU; 3x3 stride-2 conv
+ * c0 -> c1, LayerNorm, ReLU; flatten frequency-major (f * c1 + c); times
+ * in_proj^T (no bias, no clamp). d_mel: float32 [h_frame_off[n_clips]][128].
+ * d_h: float32 [sum tokens][hidden], the residual stream entering layer 0. */
+ae_status ae_subsample(const ae_model *m, const float *d_mel, const int64_t *h_frame_off,
+                       int n_clips, float *d_h, void *d_ws, size_t ws_bytes, ae_stream stream);
+
+/* One Conformer layer in place on the float32 residual stream d_h
+ * [h_tok_off[n_clips]][hidden] (the loop body of encode_locked):
+ * FFN1 (h += rw * rms_post(W2 silu(W1 rms_pre(h)))), local attention
+ * (h += rms_post_attn(post(attn(q, k, v of rms_pre_attn(h))))), where a
+ * token sees itself and the left-1 tokens before it in its own clip,
+ * q * log2(e)/sqrt(head_dim) * softplus(per_dim_scale), k * log2(1+e),
+ * logits q.k + q.R[d] capped by softcap * tanh(z / softcap) and a
+ * natural-exp softmax; light conv (h += lc_end(silu(rms(dwconv(glu(
+ * lc_start(rms(h)))))))) with a causal depthwise conv that does not reach
+ * before the clip start; FFN2; h = rms_norm_out(h). Every ClipLin clamps
+ * its input and output. */
+ae_status ae_conformer_layer(const ae_model *m, int layer, float *d_h, const int64_t *h_tok_off,
+                             int n_clips, void *d_ws, size_t ws_bytes, ae_stream stream);
+
+/* The whole forward (AudioTower::soft_tokens for one packed batch):
+ * log-mel, stem, in_proj, every layer, then out_proj + bias, a weightless
+ * RMS norm and embed. d_wave: float32 [h_sample_off[n_clips]]. d_out:
+ * float32 [sum tokens][embed_dim], clip after clip. */
+ae_status ae_encode(const ae_model *m, const float *d_wave, const int64_t *h_sample_off,
+                    int n_clips, float *d_out, void *d_ws, size_t ws_bytes, ae_stream stream);
+
+/* ae_encode from host memory to host memory: copies h_wave into the
+ * workspace, runs ae_encode, copies the rows back to h_out and waits for
+ * the stream. Pinned host buffers make the copies asynchronous DMA. The
+ * workspace must hold ae_workspace_size(...) plus the wave and output
+ * bytes, rounded up to 256 each: see ae_encode_host_workspace_size. */
+size_t ae_encode_host_workspace_size(const ae_model *m, const int64_t *h_sample_off, int n_clips);
+ae_status ae_encode_host(const ae_model *m, const float *h_wave, const int64_t *h_sample_off,
+                         int n_clips, float *h_out, void *d_ws, size_t ws_bytes, ae_stream stream);
+
+/* --- the attention core alone ------------------------------------------------ */
+
+/* Load-time tables of one attention layer on the host in float64, stored
+ * float32: h_R [left][hidden] = rows 0..left-1 of pe relative_k^T, and
+ * h_qscale [hidden/heads] = log2(e)/sqrt(head_dim) * softplus(per_dim_scale).
+ * *k_scale = log2(1 + e). */
+ae_status ae_attention_tables(const float *h_relative_k, const float *h_per_dim_scale, int hidden,
+                              int heads, int left, float *h_R, float *h_qscale, float *k_scale);
+
+/* The attention core of the page's `attention` on clamped projections:
+ * o_t = sum_{d <= min(pos_t, left-1)} softmax_d(cap tanh((q_t s) . (k_scale
+ * k_{t-d}) + (q_t s) . R[d]) / cap)) v_{t-d} per head, s = d_qscale.
+ * d_q/d_k/d_v: [total_tokens][hidden] rows with a stride of ld_qkv
+ * elements, bf16 (dtype AE_BF16) or float32 (AE_F32); d_out the same type,
+ * [total_tokens][ld_out]. d_R: float32 [left][hidden]; d_qscale: float32
+ * [head_dim]. Requires hidden 1024, heads 8, left 12. Token offsets per
+ * sequence h_tok_off [n_clips + 1]. Workspace: ae_workspace_size(NULL, ...). */
+ae_status ae_local_attention(const void *d_q, const void *d_k, const void *d_v, int64_t ld_qkv,
+                             ae_dtype dtype, const float *d_R, const float *d_qscale,
+                             float k_scale, float softcap, const int64_t *h_tok_off, int n_clips,
+                             void *d_out, int64_t ld_out, void *d_ws, size_t ws_bytes,
+                             ae_stream stream);
+
+/* --- kernel timing ------------------------------------------------------------ */
+
+/* Classes of the kernels the calls launch. */
+typedef enum {
+  AE_K_TABLES = 0,   /* per-call clip tables and token positions */
+  AE_K_LOGMEL = 1,   /* fused log-mel front-end */
+  AE_K_CONV0 = 2,    /* stem conv0 + LayerNorm + ReLU */
+  AE_K_CONV1 = 3,    /* stem conv1 + LayerNorm + ReLU (implicit GEMM) */
+  AE_K_GEMM = 4,     /* every projection (tcgen05 for AE_BF16) */
+  AE_K_ATTENTION = 5,
+  AE_K_LCONV = 6,    /* depthwise conv + RMS norm + SiLU */
+  AE_K_ROWOP = 7,    /* residual / RMS-norm row passes */
+  AE_K_COUNT = 8
+} ae_kernel_class;
+
+/* Kernel timing for measurement (the analogue of the page's
+ * CMF_EGEMMA2_PROF split). While enabled, every call records a CUDA event
+ * pair on its stream around each kernel it launches, together with the
+ * launch's algorithmic work: flops for the projections and conv1 (2 M N K),
+ * bytes that must cross DRAM for the others (inputs read once, outputs
+ * written once). Enabling allocates the event pool (up to 16384 launches
+ * between reads); the calls themselves still allocate nothing. Not
+ * thread-safe: enable, call and read from one thread. */
+ae_status ae_profile_enable(int on);
+
+/* Synchronises the device, then returns per class (arrays of AE_K_COUNT)
+ * the summed event milliseconds, launch counts, flops and bytes since the
+ * last read, and resets them. Any output pointer may be NULL. *dropped
+ * (if not NULL) receives the launches not timed because the pool was full. */
+ae_status ae_profile_read(double *ms, int64_t *launches, double *flops, double *bytes, int64_t *dropped);
+
+/* --- diagnostics ------------------------------------------------------------- */
+
+/* Message of the last failed call on this thread ("" if none). */
+const char *ae_last_error(void);
+
+/* Synchronises the current device and reports whether a kernel of this
+ * library gave up a bounded wait since the last call (AE_EDEVICE), or the
+ * device reported an error (AE_ECUDA); clears the library's flag. */
+ae_status ae_device_status(void);
+
+/* Version of the library, "major.minor.patch". */
+const char *ae_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* AE_H */

@@ -1,0 +1,168 @@
+// Internal declarations of the audio-encoder library: the device-resident
+// model, the workspace layout and the kernel launchers. Not part of the ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "../../include/ae.h"
+
+namespace ae {
+
+using bf16 = __nv_bfloat16;
+
+// Shapes the kernels are compiled for (the release tower).
+constexpr int kMels = 128;        // mel bands
+constexpr int kFrame = 320;       // window
+constexpr int kHop = 160;         // hop
+constexpr int kFft = 512;         // FFT size
+constexpr int kMaxSamples = 480000;
+constexpr int kC0 = 128;          // conv0 channels
+constexpr int kC1 = 32;           // conv1 channels
+constexpr int kF1 = 64;           // frequency rows after conv0
+constexpr int kF2 = 32;           // frequency rows after conv1
+constexpr int kHidden = 1024;
+constexpr int kHeads = 8;
+constexpr int kHeadDim = 128;
+constexpr int kLeft = 12;         // attention span (itself + 11 before)
+constexpr int kKernel = 5;        // depthwise taps
+
+// Output modes of the GEMM epilogue.
+enum EpiMode : int {
+  EPI_F32 = 0,        // v = clamp(acc + bias) -> float
+  EPI_BF16 = 1,       // v = clamp(acc) -> act
+  EPI_SILU = 2,       // v = clamp2(silu(clamp(acc))) -> act
+  EPI_GLU = 3,        // columns (2c, 2c+1) -> clamp, a * sigmoid(b) -> act column c
+};
+
+struct EpiArgs {
+  void *out;          // output base
+  int64_t ld;         // output row stride in elements
+  const float *bias;  // [N] or null
+  float lo, hi;       // first clamp
+  float lo2, hi2;     // clamp after the activation (EPI_SILU)
+  int seg_w;          // if > 0: columns [s*seg_w, (s+1)*seg_w) use seg_lo/hi[s] as the first clamp
+  float seg_lo[3], seg_hi[3];
+};
+
+// Device copy of one layer.
+struct LayerDev {
+  float *ff1_pre, *ff1_post, *ff2_pre, *ff2_post;
+  float *norm_pre_attn, *norm_post_attn, *norm_out, *lc_pre, *lc_norm;
+  float *lc_dw;               // [hidden][kernel]
+  float *R;                   // [left][hidden]
+  float *qscale;              // [head_dim]: q_scale * softplus(per_dim_scale)
+  void *ff1_w1, *ff1_w2, *ff2_w1, *ff2_w2;
+  void *qkv;                  // [3*hidden][hidden]: q, k, v rows stacked
+  void *post, *lc_end;
+  void *lc_start;             // [2*hidden][hidden], rows interleaved (a_0, b_0, a_1, b_1, ...)
+  ae_clip c_ff1_w1, c_ff1_w2, c_ff2_w1, c_ff2_w2, c_q, c_k, c_v, c_post, c_lc_start, c_lc_end;
+  // tensor maps of the weight operands (bf16 only)
+  CUtensorMap tm_ff1_w1, tm_ff1_w2, tm_ff2_w1, tm_ff2_w2, tm_qkv, tm_post, tm_lc_start, tm_lc_end;
+};
+
+}  // namespace ae
+
+struct ae_model {
+  ae_config cfg;
+  ae_dtype dtype;
+  int device;
+  float k_scale;
+  // stem
+  float *conv0c;    // [c0][9] taps minus their channel mean (the LayerNorm's mean is linear in the patch)
+  float *conv0cov;  // [9][9] channel covariance of the taps: LayerNorm variance = p^T C p
+  float *ln0, *ln1;
+  void *conv1;      // [c1][9 * c0], k = (dt * 3 + df) * c0 + c
+  void *in_proj;    // [hidden][1024]
+  void *out_proj;   // [out_dim][hidden]
+  float *out_bias;
+  void *embed;      // [embed_dim][out_dim]
+  CUtensorMap tm_conv1, tm_in_proj, tm_out_proj, tm_embed;
+  std::vector<ae::LayerDev> layers;
+  std::vector<void *> allocs;
+};
+
+namespace ae {
+
+// Per-call clip tables, computed on the host from the caller's offsets.
+struct ClipTables {
+  int n_clips = 0;
+  int64_t total_samples = 0, total_frames = 0, total_tokens = 0, stem_rows = 0;
+  int64_t mel_tiles = 0, conv1_tiles = 0;
+  std::vector<int64_t> sample_off;  // [B+1]
+  std::vector<int32_t> frame_off, tok_off, stem_off, mel_tile_off, conv1_tile_off;  // [B+1]
+};
+
+// Device view of the tables (inside the workspace).
+struct ClipTablesDev {
+  int n_clips;
+  const int64_t *sample_off;
+  const int32_t *frame_off, *tok_off, *stem_off, *mel_tile_off, *conv1_tile_off;
+  const int32_t *pos;  // [total_tokens]
+};
+
+// Workspace carve-up. Every region is 256-byte aligned.
+struct WsLayout {
+  size_t tables = 0, pos = 0, mel = 0, y0 = 0, xs = 0, h = 0, a = 0, big = 0, y = 0, o = 0;
+  size_t total = 0;
+};
+
+constexpr int kMelTile = 64;       // frames per log-mel work item
+constexpr int kConv1TileTok = 4;   // tokens per conv1 tile (4 x 32 frequency rows = 128 GEMM rows)
+
+WsLayout ws_layout(const ae_model *m, int64_t n_clips, int64_t frames, int64_t tokens, bool with_model);
+
+// launchers (return cudaError_t of the launch)
+cudaError_t launch_upload_tables(const ClipTables &t, void *ws, const WsLayout &L, ClipTablesDev *dev,
+                                 bool with_pos, cudaStream_t s);
+size_t tables_bytes(int64_t n_clips);
+cudaError_t launch_logmel(const float *wave, float *mel, const ClipTablesDev &t, int64_t mel_tiles,
+                          cudaStream_t s);
+cudaError_t launch_conv0(const ae_model *m, const float *mel, void *y0, const ClipTablesDev &t,
+                         int64_t stem_rows, cudaStream_t s);
+cudaError_t launch_conv1(const ae_model *m, const void *y0, int64_t stem_rows, void *xs,
+                         const ClipTablesDev &t, int64_t conv1_tiles, int64_t tokens, cudaStream_t s);
+
+// y = epilogue(x W^T); x [M][K] act, W [N][K]. For bf16 the caller passes
+// the weight's tensor map (or null to build one).
+cudaError_t gemm(const ae_model *m, const void *x, int64_t M, int K, const void *w, const CUtensorMap *tmW,
+                 int N, int mode, const EpiArgs &ep, cudaStream_t s);
+
+// Row update of the residual stream (one warp per row of `width` floats):
+//   if y:      h += s * (y_norm ? rms(y) * wy : y)
+//   if w_out:  h = rms(h) * w_out
+//   write h back if anything changed it
+//   if a_out:  a = clamp(rms(h) * w_next, lo, hi)  (act type of the model)
+struct RowArgs {
+  float *h; const float *y; const float *wy; float s; int y_norm;
+  const float *w_out;
+  void *a_out; const float *w_next; int a_rms; float lo, hi;
+  int width; int64_t rows;
+};
+cudaError_t launch_rowop(const ae_model *m, const RowArgs &r, cudaStream_t s);
+
+// Light-conv middle: c = clamp(silu(rms(dwconv(gl)) * w_norm), lo, hi).
+cudaError_t launch_lconv(const ae_model *m, const void *gl, const float *w_dw, const float *w_norm,
+                         float lo, float hi, void *out, const int32_t *pos, int64_t T, cudaStream_t s);
+
+// Attention core; q/k/v rows of `ld` elements; output clamped to [lo, hi].
+cudaError_t launch_attention(bool is_bf16, const void *q, const void *k, const void *v, int64_t ld,
+                             const float *R, const float *qscale, float k_scale, float cap, const int32_t *pos,
+                             int64_t T, void *out, int64_t ld_out, float lo, float hi, cudaStream_t s);
+
+// Tensor-map encoding (driver entry point looked up at run time).
+bool make_tmap_2d_bf16(CUtensorMap *tm, const void *base, uint64_t inner, uint64_t outer,
+                       uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
+bool make_tmap_stem_y0(CUtensorMap *tm, const void *y0, int64_t stem_rows);
+
+unsigned *device_status_word();
+unsigned read_and_clear_status();
+cudaError_t launch_pos(int32_t *pos, const int32_t *tok_off, int n_clips, cudaStream_t s);
+void set_error(const std::string &msg);
+
+}  // namespace ae

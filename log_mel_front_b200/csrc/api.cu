@@ -1,0 +1,881 @@
+// C ABI of the audio-encoder library: argument checks, model creation (weight
+// conversion, load-time tables), workspace layout and the stream-ordered
+// call sequences of the hot path. Every computation of a call runs in the
+// kernels of this library; the host only validates, lays out and launches.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "ae_internal.h"
+
+namespace ae {
+
+static thread_local std::string g_last_error;
+void set_error(const std::string &msg) { g_last_error = msg; }
+
+static size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static int64_t frames_of_samples(int64_t n) {
+  if (n < 0) n = 0;
+  if (n > kMaxSamples) n = kMaxSamples;
+  return n <= kHop ? 0 : (n - kHop + kHop - 1) / kHop;
+}
+static int64_t tokens_of_frames(int64_t f) { return ((f + 1) / 2 + 1) / 2; }
+
+// Limits that keep every index the kernels form inside their integer types.
+constexpr int64_t kMaxClips = 1 << 20;
+constexpr int64_t kMaxTokens = 4000000;
+constexpr int64_t kMaxFrames = 16000000;
+
+enum OffKind { kSamples, kFrames, kTokens };
+
+static ae_status fail(ae_status st, const std::string &msg) {
+  set_error(msg);
+  return st;
+}
+
+// ------------------------------------------------------------------ kernel timing
+
+struct Profiler {
+  bool on = false;
+  size_t cap = 0, n = 0;
+  int64_t dropped = 0;
+  std::vector<cudaEvent_t> ev;  // 2 per record
+  struct Rec {
+    int cls;
+    double flops, bytes;
+  };
+  std::vector<Rec> recs;
+};
+static Profiler g_prof;
+
+// Runs f (which enqueues kernels on s) between two recorded events.
+template <class F>
+static cudaError_t timed(int cls, double flops, double bytes, cudaStream_t s, F &&f) {
+  Profiler &P = g_prof;
+  const bool rec = P.on && P.n < P.cap;
+  if (P.on && !rec) ++P.dropped;
+  if (rec) cudaEventRecord(P.ev[2 * P.n], s);
+  const cudaError_t e = f();
+  if (rec) {
+    cudaEventRecord(P.ev[2 * P.n + 1], s);
+    P.recs[P.n] = {cls, flops, bytes};
+    ++P.n;
+  }
+  return e;
+}
+
+static size_t act_bytes(const ae_model *m) { return m->dtype == AE_BF16 ? 2 : 4; }
+
+// A projection with its algorithmic flops (2 M N K) and bytes (x, W, y once).
+static cudaError_t gemm_t(const ae_model *m, const void *x, int64_t M, int K, const void *w, const CUtensorMap *tmW,
+                          int N, int mode, const EpiArgs &ep, cudaStream_t s) {
+  const double a = (double)act_bytes(m);
+  const double out_cols = mode == EPI_GLU ? N / 2 : N;
+  const double out_b = mode == EPI_F32 ? 4.0 : a;
+  const double bytes = a * ((double)M * K + (double)N * K) + out_b * (double)M * out_cols;
+  return timed(AE_K_GEMM, 2.0 * (double)M * N * K, bytes, s, [&] { return gemm(m, x, M, K, w, tmW, N, mode, ep, s); });
+}
+
+static cudaError_t tables_t(const ClipTables &T, void *ws, const WsLayout &L, ClipTablesDev *td, bool pos,
+                            cudaStream_t s) {
+  return timed(AE_K_TABLES, 0.0, 0.0, s, [&] { return launch_upload_tables(T, ws, L, td, pos, s); });
+}
+
+static double samples_read(const ClipTables &T) {
+  double n = 0.0;
+  for (int c = 0; c < T.n_clips; ++c)
+    n += (double)std::min<int64_t>(T.sample_off[c + 1] - T.sample_off[c], kMaxSamples);
+  return n;
+}
+
+// log-mel: every sample read once (4 bytes), every frame's 128 floats written once
+static cudaError_t logmel_t(const float *wave, float *mel, const ClipTablesDev &td, const ClipTables &T,
+                            cudaStream_t s) {
+  const double bytes = 4.0 * samples_read(T) + 512.0 * (double)T.total_frames;
+  return timed(AE_K_LOGMEL, 0.0, bytes, s, [&] { return launch_logmel(wave, mel, td, T.mel_tiles, s); });
+}
+
+// conv0 reads the mel rows and writes every stem row (64 x 128 per row)
+static cudaError_t conv0_t(const ae_model *m, const float *mel, void *y0, const ClipTablesDev &td,
+                           const ClipTables &T, cudaStream_t s) {
+  const double bytes = 512.0 * (double)T.total_frames + (double)act_bytes(m) * kF1 * kC0 * (double)T.stem_rows;
+  const double flops = 2.0 * 9 * kC0 * kF1 * (double)T.stem_rows;
+  return timed(AE_K_CONV0, flops, bytes, s, [&] { return launch_conv0(m, mel, y0, td, T.stem_rows, s); });
+}
+
+// conv1 as a GEMM: M = tokens x 32 frequency rows, N = 32, K = 9 x 128
+static cudaError_t conv1_t(const ae_model *m, const void *y0, void *xs, const ClipTablesDev &td, const ClipTables &T,
+                           cudaStream_t s) {
+  const double M = (double)T.total_tokens * kF2;
+  const double a = (double)act_bytes(m);
+  const double bytes = a * kF1 * kC0 * (double)T.stem_rows + a * kHidden * (double)T.total_tokens;
+  return timed(AE_K_CONV1, 2.0 * M * kC1 * 9 * kC0, bytes, s,
+               [&] { return launch_conv1(m, y0, T.stem_rows, xs, td, T.conv1_tiles, T.total_tokens, s); });
+}
+
+static cudaError_t rowop_t(const ae_model *m, const RowArgs &r, cudaStream_t s) {
+  const double W = r.width;
+  const bool changed = r.y || r.w_out;
+  double per_row = 4.0 * W * (1.0 + (changed ? 1.0 : 0.0) + (r.y ? 1.0 : 0.0));
+  if (r.a_out) per_row += W * (double)act_bytes(m);
+  return timed(AE_K_ROWOP, 0.0, per_row * (double)r.rows, s, [&] { return launch_rowop(m, r, s); });
+}
+
+static ae_status build_tables(const int64_t *off, int n, OffKind kind, ClipTables &T, const char *name) {
+  if (n < 0) return fail(AE_EINVAL, "n_clips is negative");
+  if (n > kMaxClips) return fail(AE_EINVAL, "n_clips above 1048576");
+  if (!off) return fail(AE_EINVAL, std::string(name) + " is null");
+  if (off[0] != 0) return fail(AE_EINVAL, std::string(name) + "[0] must be 0");
+  T = ClipTables();
+  T.n_clips = n;
+  const size_t B1 = (size_t)n + 1;
+  T.sample_off.assign(B1, 0);
+  T.frame_off.assign(B1, 0);
+  T.tok_off.assign(B1, 0);
+  T.stem_off.assign(B1, 0);
+  T.mel_tile_off.assign(B1, 0);
+  T.conv1_tile_off.assign(B1, 0);
+  int64_t fr = 0, tk = 0, st = 0, mt = 0, ct = 0;
+  for (int c = 0; c < n; ++c) {
+    const int64_t len = off[c + 1] - off[c];
+    if (len < 0) return fail(AE_EINVAL, std::string(name) + " is not non-decreasing at clip " + std::to_string(c));
+    const int64_t F = kind == kSamples ? frames_of_samples(len) : (kind == kFrames ? len : 0);
+    if (kind == kFrames && F > frames_of_samples(kMaxSamples))
+      return fail(AE_EINVAL, "clip " + std::to_string(c) + " has more than 2999 frames");
+    const int64_t tok = kind == kTokens ? len : tokens_of_frames(F);
+    fr += F;
+    tk += tok;
+    st += 2 * tok + 2;
+    mt += (F + kMelTile - 1) / kMelTile;
+    ct += (tok + kConv1TileTok - 1) / kConv1TileTok;
+    if (fr > kMaxFrames || tk > kMaxTokens) return fail(AE_EINVAL, "batch too large for one call (frames or tokens)");
+    T.sample_off[c + 1] = kind == kSamples ? off[c + 1] : 0;
+    T.frame_off[c + 1] = (int32_t)fr;
+    T.tok_off[c + 1] = (int32_t)tk;
+    T.stem_off[c + 1] = (int32_t)st;
+    T.mel_tile_off[c + 1] = (int32_t)mt;
+    T.conv1_tile_off[c + 1] = (int32_t)ct;
+  }
+  T.total_samples = kind == kSamples ? off[n] : 0;
+  T.total_frames = fr;
+  T.total_tokens = tk;
+  T.stem_rows = st;
+  T.mel_tiles = mt;
+  T.conv1_tiles = ct;
+  return AE_OK;
+}
+
+// Workspace: [tables][pos][h][ union( stem: mel, y0, xs | layers: a, big, y, o ) ]
+WsLayout ws_layout(const ae_model *m, int64_t n_clips, int64_t frames, int64_t tokens, bool with_model) {
+  WsLayout L;
+  size_t off = 0;
+  L.tables = off;
+  off += al256(tables_bytes(n_clips));
+  L.pos = off;
+  off += al256((size_t)tokens * 4);
+  if (!with_model || !m) {
+    L.total = off;
+    return L;
+  }
+  const size_t act = m->dtype == AE_BF16 ? 2 : 4;
+  const int64_t H = m->cfg.hidden;
+  L.h = off;
+  off += al256((size_t)tokens * H * 4);
+  const size_t u = off;
+  size_t so = u;
+  L.mel = so;
+  so += al256((size_t)frames * kMels * 4);
+  L.y0 = so;
+  so += al256(act * (size_t)(2 * tokens + 2 * n_clips) * kF1 * kC0);
+  L.xs = so;
+  so += al256(act * (size_t)tokens * kHidden);
+  size_t lo_ = u;
+  const int64_t big_w = std::max<int64_t>({m->cfg.ffn, 3 * H, m->cfg.out_dim, 2 * H});
+  const int64_t y_w = std::max<int64_t>(H, m->cfg.out_dim);
+  L.a = lo_;
+  lo_ += al256(act * (size_t)tokens * H);
+  L.big = lo_;
+  lo_ += al256(act * (size_t)tokens * big_w);
+  L.y = lo_;
+  lo_ += al256((size_t)tokens * y_w * 4);
+  L.o = lo_;
+  lo_ += al256(act * (size_t)tokens * H);
+  L.total = std::max(so, lo_);
+  return L;
+}
+
+// ------------------------------------------------------------------ host-side load-time tables
+
+static double softplus_torch(double x) { return x > 20.0 ? x : std::log1p(std::exp(x)); }
+
+static void attention_tables_host(const float *relk, const float *pds, int hidden, int heads, int left, float *R,
+                                  float *qscale, float *k_scale) {
+  const int n_ts = hidden / 2;
+  const double incr = std::log(10000.0) / (double)(std::max(n_ts, 2) - 1);
+  std::vector<double> inv(n_ts), pe(hidden);
+  for (int i = 0; i < n_ts; ++i) inv[i] = std::exp(-(double)i * incr);
+  for (int d = 0; d < left; ++d) {
+    for (int i = 0; i < n_ts; ++i) {
+      pe[i] = std::sin(d * inv[i]);
+      pe[n_ts + i] = std::cos(d * inv[i]);
+    }
+    for (int j = 0; j < hidden; ++j) {
+      const float *w = relk + (size_t)j * hidden;
+      double acc = 0.0;
+      for (int i = 0; i < hidden; ++i) acc += pe[i] * (double)w[i];
+      R[(size_t)d * hidden + j] = (float)acc;
+    }
+  }
+  const int hd = hidden / heads;
+  const double qs = (1.0 / std::sqrt((double)hd)) / std::log(2.0);
+  for (int j = 0; j < hd; ++j) qscale[j] = (float)(qs * softplus_torch((double)pds[j]));
+  *k_scale = (float)(std::log(1.0 + std::exp(1.0)) / std::log(2.0));
+}
+
+static uint16_t f2bf(float f) {
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  if ((u & 0x7fffffffu) > 0x7f800000u) return 0x7fc0;
+  u += 0x7fffu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+
+struct Uploader {
+  ae_model *m;
+  bool ok = true;
+  template <typename T> T *alloc(size_t n) {
+    void *p = nullptr;
+    if (!ok || cudaMalloc(&p, std::max<size_t>(n, 1) * sizeof(T)) != cudaSuccess) {
+      ok = false;
+      return nullptr;
+    }
+    m->allocs.push_back(p);
+    return static_cast<T *>(p);
+  }
+  float *f32(const float *h, size_t n) {
+    float *d = alloc<float>(n);
+    if (d && cudaMemcpy(d, h, n * 4, cudaMemcpyHostToDevice) != cudaSuccess) ok = false;
+    return d;
+  }
+  // matrix in the model's GEMM operand type
+  void *mat(const std::vector<float> &h) {
+    if (m->dtype == AE_F32) return f32(h.data(), h.size());
+    std::vector<uint16_t> b(h.size());
+    for (size_t i = 0; i < h.size(); ++i) b[i] = f2bf(h[i]);
+    uint16_t *d = alloc<uint16_t>(b.size());
+    if (d && cudaMemcpy(d, b.data(), b.size() * 2, cudaMemcpyHostToDevice) != cudaSuccess) ok = false;
+    return d;
+  }
+  void *mat(const float *h, size_t n) { return mat(std::vector<float>(h, h + n)); }
+};
+
+static bool bad_clip(const ae_clip &c) {
+  return std::isnan(c.lo_in) || std::isnan(c.hi_in) || std::isnan(c.lo_out) || std::isnan(c.hi_out) ||
+         c.lo_in > c.hi_in || c.lo_out > c.hi_out;
+}
+
+// ------------------------------------------------------------------ one layer
+
+struct Bufs {
+  float *h;
+  void *a, *big, *o;
+  float *y;
+  const int32_t *pos;
+};
+
+static EpiArgs ep_of(void *out, int64_t ld, float lo, float hi) {
+  EpiArgs e;
+  std::memset(&e, 0, sizeof(e));
+  e.out = out;
+  e.ld = ld;
+  e.lo = lo;
+  e.hi = hi;
+  e.lo2 = -INFINITY;
+  e.hi2 = INFINITY;
+  return e;
+}
+
+static RowArgs row_of(float *h, int width, int64_t rows) {
+  RowArgs r;
+  std::memset(&r, 0, sizeof(r));
+  r.h = h;
+  r.width = width;
+  r.rows = rows;
+  r.a_rms = 1;
+  r.lo = -INFINITY;
+  r.hi = INFINITY;
+  return r;
+}
+
+#define AE_TRY(x)                            \
+  do {                                       \
+    cudaError_t e_ = (x);                    \
+    if (e_ != cudaSuccess) return e_;        \
+  } while (0)
+
+// What the layer's last row pass should also write into b.a.
+enum NextA { kNextNone, kNextLayer, kNextPlain };
+
+static cudaError_t run_layer(const ae_model *m, int li, const Bufs &b, int64_t T, bool a_ready, NextA next,
+                             cudaStream_t s) {
+  const LayerDev &L = m->layers[li];
+  const int H = m->cfg.hidden, F = m->cfg.ffn;
+  const float rw = m->cfg.residual_weight;
+  const size_t act = m->dtype == AE_BF16 ? 2 : 4;
+  const bool tc = m->dtype == AE_BF16;
+  if (!a_ready) {
+    RowArgs r = row_of(b.h, H, T);
+    r.a_out = b.a;
+    r.w_next = L.ff1_pre;
+    r.lo = L.c_ff1_w1.lo_in;
+    r.hi = L.c_ff1_w1.hi_in;
+    AE_TRY(rowop_t(m, r, s));
+  }
+  auto ffn = [&](void *w1, const CUtensorMap *t1, const ae_clip &c1, void *w2, const CUtensorMap *t2,
+                 const ae_clip &c2) -> cudaError_t {
+    EpiArgs e1 = ep_of(b.big, F, c1.lo_out, c1.hi_out);
+    e1.lo2 = c2.lo_in;
+    e1.hi2 = c2.hi_in;
+    AE_TRY(gemm_t(m,b.a, T, H, w1, tc ? t1 : nullptr, F, EPI_SILU, e1, s));
+    return gemm_t(m, b.big, T, F, w2, tc ? t2 : nullptr, H, EPI_F32, ep_of(b.y, H, c2.lo_out, c2.hi_out), s);
+  };
+  // ---- FFN1
+  AE_TRY(ffn(L.ff1_w1, &L.tm_ff1_w1, L.c_ff1_w1, L.ff1_w2, &L.tm_ff1_w2, L.c_ff1_w2));
+  {
+    RowArgs r = row_of(b.h, H, T);
+    r.y = b.y; r.wy = L.ff1_post; r.s = rw; r.y_norm = 1;
+    r.a_out = b.a; r.w_next = L.norm_pre_attn; r.lo = L.c_q.lo_in; r.hi = L.c_q.hi_in;
+    AE_TRY(rowop_t(m, r, s));
+  }
+  // ---- attention: fused q/k/v projection, core, post
+  {
+    EpiArgs e = ep_of(b.big, 3 * H, -INFINITY, INFINITY);
+    e.seg_w = H;
+    e.seg_lo[0] = L.c_q.lo_out; e.seg_hi[0] = L.c_q.hi_out;
+    e.seg_lo[1] = L.c_k.lo_out; e.seg_hi[1] = L.c_k.hi_out;
+    e.seg_lo[2] = L.c_v.lo_out; e.seg_hi[2] = L.c_v.hi_out;
+    AE_TRY(gemm_t(m,b.a, T, H, L.qkv, tc ? &L.tm_qkv : nullptr, 3 * H, EPI_BF16, e, s));
+    const uint8_t *qkv = static_cast<const uint8_t *>(b.big);
+    AE_TRY(timed(AE_K_ATTENTION, 0.0, (double)T * 4 * H * act, s, [&] {
+      return launch_attention(tc, qkv, qkv + act * H, qkv + 2 * act * H, 3 * H, L.R, L.qscale, m->k_scale,
+                              m->cfg.softcap, b.pos, T, b.o, H, L.c_post.lo_in, L.c_post.hi_in, s);
+    }));
+    AE_TRY(gemm_t(m,b.o, T, H, L.post, tc ? &L.tm_post : nullptr, H, EPI_F32,
+                ep_of(b.y, H, L.c_post.lo_out, L.c_post.hi_out), s));
+    RowArgs r = row_of(b.h, H, T);
+    r.y = b.y; r.wy = L.norm_post_attn; r.s = 1.0f; r.y_norm = 1;
+    r.a_out = b.a; r.w_next = L.lc_pre; r.lo = L.c_lc_start.lo_in; r.hi = L.c_lc_start.hi_in;
+    AE_TRY(rowop_t(m, r, s));
+  }
+  // ---- light conv
+  {
+    AE_TRY(gemm_t(m,b.a, T, H, L.lc_start, tc ? &L.tm_lc_start : nullptr, 2 * H, EPI_GLU,
+                ep_of(b.big, H, L.c_lc_start.lo_out, L.c_lc_start.hi_out), s));
+    AE_TRY(timed(AE_K_LCONV, 0.0, (double)T * 2 * H * act, s, [&] {
+      return launch_lconv(m, b.big, L.lc_dw, L.lc_norm, L.c_lc_end.lo_in, L.c_lc_end.hi_in, b.o, b.pos, T, s);
+    }));
+    AE_TRY(gemm_t(m,b.o, T, H, L.lc_end, tc ? &L.tm_lc_end : nullptr, H, EPI_F32,
+                ep_of(b.y, H, L.c_lc_end.lo_out, L.c_lc_end.hi_out), s));
+    RowArgs r = row_of(b.h, H, T);
+    r.y = b.y; r.s = 1.0f; r.y_norm = 0;
+    r.a_out = b.a; r.w_next = L.ff2_pre; r.lo = L.c_ff2_w1.lo_in; r.hi = L.c_ff2_w1.hi_in;
+    AE_TRY(rowop_t(m, r, s));
+  }
+  // ---- FFN2, norm_out, and the next consumer's input
+  AE_TRY(ffn(L.ff2_w1, &L.tm_ff2_w1, L.c_ff2_w1, L.ff2_w2, &L.tm_ff2_w2, L.c_ff2_w2));
+  {
+    RowArgs r = row_of(b.h, H, T);
+    r.y = b.y; r.wy = L.ff2_post; r.s = rw; r.y_norm = 1;
+    r.w_out = L.norm_out;
+    if (next == kNextLayer) {
+      const LayerDev &N = m->layers[li + 1];
+      r.a_out = b.a; r.w_next = N.ff1_pre; r.lo = N.c_ff1_w1.lo_in; r.hi = N.c_ff1_w1.hi_in;
+    } else if (next == kNextPlain) {
+      r.a_out = b.a; r.a_rms = 0;
+    }
+    AE_TRY(rowop_t(m, r, s));
+  }
+  return cudaSuccess;
+}
+
+// Head: out_proj + bias, weightless RMS norm, embed. b.a holds h in the operand type.
+static cudaError_t run_head(const ae_model *m, const Bufs &b, int64_t T, float *out, cudaStream_t s) {
+  const int H = m->cfg.hidden, OD = m->cfg.out_dim, ED = m->cfg.embed_dim;
+  const bool tc = m->dtype == AE_BF16;
+  EpiArgs e = ep_of(b.y, OD, -INFINITY, INFINITY);
+  e.bias = m->out_bias;
+  AE_TRY(gemm_t(m,b.a, T, H, m->out_proj, tc ? &m->tm_out_proj : nullptr, OD, EPI_F32, e, s));
+  RowArgs r = row_of(b.y, OD, T);
+  r.a_out = b.big;
+  AE_TRY(rowop_t(m, r, s));
+  return gemm_t(m, b.big, T, OD, m->embed, tc ? &m->tm_embed : nullptr, ED, EPI_F32,
+                ep_of(out, ED, -INFINITY, INFINITY), s);
+}
+
+static Bufs bufs_of(void *ws, const WsLayout &L, const ClipTablesDev &td) {
+  uint8_t *w = static_cast<uint8_t *>(ws);
+  Bufs b;
+  b.h = reinterpret_cast<float *>(w + L.h);
+  b.a = w + L.a;
+  b.big = w + L.big;
+  b.y = reinterpret_cast<float *>(w + L.y);
+  b.o = w + L.o;
+  b.pos = td.pos;
+  return b;
+}
+
+static ae_status cuda_fail(cudaError_t e, const char *where) {
+  return fail(AE_ECUDA, std::string(where) + ": " + cudaGetErrorString(e));
+}
+
+static ae_status check_model(const ae_model *m) {
+  if (!m) return fail(AE_EINVAL, "model is null");
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(AE_ECUDA, "no CUDA device");
+  if (dev != m->device) return fail(AE_EINVAL, "the current device is not the model's device");
+  return AE_OK;
+}
+
+static ae_status check_ws(void *ws, size_t have, size_t need) {
+  if (need > 0 && !ws) return fail(AE_EINVAL, "d_ws is null");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255) != 0) return fail(AE_EINVAL, "d_ws must be 256-byte aligned");
+  if (have < need)
+    return fail(AE_EWORKSPACE, "workspace of " + std::to_string(have) + " bytes, " + std::to_string(need) + " needed");
+  return AE_OK;
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// The encode sequence on device buffers (shared by ae_encode and ae_encode_host).
+static ae_status encode_dev(const ae_model *m, const float *d_wave, const ClipTables &T, float *d_out, void *d_ws,
+                            const WsLayout &L, cudaStream_t s) {
+  ClipTablesDev td;
+  cudaError_t e = tables_t(T, d_ws, L, &td, true, s);
+  if (e != cudaSuccess) return cuda_fail(e, "table upload");
+  if (T.total_tokens == 0) return AE_OK;
+  uint8_t *w = static_cast<uint8_t *>(d_ws);
+  float *mel = reinterpret_cast<float *>(w + L.mel);
+  Bufs b = bufs_of(d_ws, L, td);
+  if ((e = logmel_t(d_wave, mel, td, T, s)) != cudaSuccess) return cuda_fail(e, "logmel");
+  if ((e = conv0_t(m, mel, w + L.y0, td, T, s)) != cudaSuccess) return cuda_fail(e, "conv0");
+  if ((e = conv1_t(m, w + L.y0, w + L.xs, td, T, s)) != cudaSuccess)
+    return cuda_fail(e, "conv1");
+  if ((e = gemm_t(m, w + L.xs, T.total_tokens, kHidden, m->in_proj, m->dtype == AE_BF16 ? &m->tm_in_proj : nullptr,
+                m->cfg.hidden, EPI_F32, ep_of(b.h, m->cfg.hidden, -INFINITY, INFINITY), s)) != cudaSuccess)
+    return cuda_fail(e, "in_proj");
+  const int nl = m->cfg.n_layers;
+  for (int li = 0; li < nl; ++li) {
+    e = run_layer(m, li, b, T.total_tokens, li > 0, li + 1 < nl ? kNextLayer : kNextPlain, s);
+    if (e != cudaSuccess) return cuda_fail(e, "layer");
+  }
+  if (nl == 0) {
+    RowArgs r = row_of(b.h, m->cfg.hidden, T.total_tokens);
+    r.a_out = b.a;
+    r.a_rms = 0;
+    if ((e = rowop_t(m, r, s)) != cudaSuccess) return cuda_fail(e, "head input");
+  }
+  if ((e = run_head(m, b, T.total_tokens, d_out, s)) != cudaSuccess) return cuda_fail(e, "head");
+  return AE_OK;
+}
+
+}  // namespace ae
+
+using namespace ae;
+
+// ====================================================================== ABI
+
+extern "C" {
+
+int64_t ae_num_frames(int64_t n) { return frames_of_samples(n); }
+int64_t ae_num_tokens(int64_t n) { return tokens_of_frames(frames_of_samples(n)); }
+
+const char *ae_last_error(void) { return g_last_error.c_str(); }
+const char *ae_version(void) { return "0.1.0"; }
+
+ae_status ae_device_status(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return fail(AE_ECUDA, "device reported an error");
+  const unsigned v = read_and_clear_status();
+  if (v == ~0u) return fail(AE_ECUDA, "status word unreadable");
+  if (v) return fail(AE_EDEVICE, "a kernel gave up a bounded wait");
+  return AE_OK;
+}
+
+ae_status ae_attention_tables(const float *relk, const float *pds, int hidden, int heads, int left, float *R,
+                              float *qscale, float *k_scale) {
+  if (!relk || !pds || !R || !qscale || !k_scale) return fail(AE_EINVAL, "null pointer");
+  if (hidden <= 0 || heads <= 0 || hidden % heads || hidden % 2 || left <= 0)
+    return fail(AE_EINVAL, "bad hidden/heads/left");
+  attention_tables_host(relk, pds, hidden, heads, left, R, qscale, k_scale);
+  return AE_OK;
+}
+
+void ae_model_destroy(ae_model *m) {
+  if (!m) return;
+  for (void *p : m->allocs) cudaFree(p);
+  delete m;
+}
+
+ae_status ae_model_create(const ae_config *cfg, const ae_host_weights *w, ae_dtype dtype, ae_model **out) {
+  if (!out) return fail(AE_EINVAL, "out is null");
+  *out = nullptr;
+  if (!cfg || !w) return fail(AE_EINVAL, "cfg or weights is null");
+  const ae_config &c = *cfg;
+  if (c.n_mels != kMels || c.c0 != kC0 || c.c1 != kC1 || c.hidden != kHidden || c.heads != kHeads ||
+      c.left != kLeft || c.kernel != kKernel)
+    return fail(AE_EUNSUPPORTED, "kernels are built for n_mels 128, c0 128, c1 32, hidden 1024, heads 8, left 12, "
+                                 "kernel 5");
+  if (c.ffn <= 0 || c.ffn % 256 || c.embed_dim <= 0 || c.embed_dim % 256)
+    return fail(AE_EUNSUPPORTED, "ffn and embed_dim must be positive multiples of 256");
+  if (c.out_dim != 1024 && c.out_dim != 1536 && c.out_dim != 2048)
+    return fail(AE_EUNSUPPORTED, "out_dim must be 1024, 1536 or 2048");
+  if (c.n_layers < 0 || c.n_layers > 4096) return fail(AE_EINVAL, "n_layers out of range");
+  if (!(c.softcap > 0.f) || !std::isfinite(c.softcap) || !std::isfinite(c.residual_weight))
+    return fail(AE_EINVAL, "softcap must be positive and finite, residual_weight finite");
+  if (dtype != AE_F32 && dtype != AE_BF16) return fail(AE_EINVAL, "dtype");
+  if (!w->conv0 || !w->ln0 || !w->conv1 || !w->ln1 || !w->in_proj || !w->out_proj || !w->out_bias || !w->embed ||
+      (c.n_layers > 0 && !w->layers))
+    return fail(AE_EINVAL, "a stem or head weight pointer is null");
+  for (int i = 0; i < c.n_layers; ++i) {
+    const ae_host_layer &l = w->layers[i];
+    const void *ps[] = {l.ff1_pre, l.ff1_w1, l.ff1_w2, l.ff1_post, l.ff2_pre, l.ff2_w1, l.ff2_w2, l.ff2_post,
+                        l.norm_pre_attn, l.norm_post_attn, l.norm_out, l.q, l.k, l.v, l.post, l.per_dim_scale,
+                        l.relative_k, l.lc_pre, l.lc_start, l.lc_dw, l.lc_norm, l.lc_end};
+    for (const void *p : ps)
+      if (!p) return fail(AE_EINVAL, "a weight pointer of layer " + std::to_string(i) + " is null");
+    const ae_clip cs[] = {l.clip_ff1_w1, l.clip_ff1_w2, l.clip_q, l.clip_k, l.clip_v, l.clip_post,
+                          l.clip_lc_start, l.clip_lc_end, l.clip_ff2_w1, l.clip_ff2_w2};
+    for (const ae_clip &b : cs)
+      if (bad_clip(b)) return fail(AE_EINVAL, "a clamp bound of layer " + std::to_string(i) + " is NaN or inverted");
+    if (l.clip_q.lo_in != l.clip_k.lo_in || l.clip_q.lo_in != l.clip_v.lo_in || l.clip_q.hi_in != l.clip_k.hi_in ||
+        l.clip_q.hi_in != l.clip_v.hi_in)
+      return fail(AE_EUNSUPPORTED, "q, k and v input bounds differ in layer " + std::to_string(i));
+  }
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(AE_ECUDA, "no CUDA device");
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return fail(AE_ECUDA, "device properties");
+  if (prop.major != 10 || prop.minor != 0)
+    return fail(AE_EUNSUPPORTED, "this library is built for sm_100a (B200); device is sm_" +
+                                     std::to_string(prop.major) + std::to_string(prop.minor));
+
+  ae_model *m = new ae_model();
+  m->cfg = c;
+  m->dtype = dtype;
+  m->device = dev;
+  Uploader up{m};
+  const int H = c.hidden;
+  // conv0: taps minus their channel mean, and their channel covariance (float64)
+  {
+    std::vector<double> mean(9, 0.0);
+    for (int ch = 0; ch < kC0; ++ch)
+      for (int k = 0; k < 9; ++k) mean[k] += w->conv0[ch * 9 + k];
+    for (int k = 0; k < 9; ++k) mean[k] /= kC0;
+    std::vector<float> wc(kC0 * 9), cov(81);
+    std::vector<double> cd(81, 0.0);
+    for (int ch = 0; ch < kC0; ++ch)
+      for (int a = 0; a < 9; ++a) {
+        const double da = w->conv0[ch * 9 + a] - mean[a];
+        wc[ch * 9 + a] = (float)da;
+        for (int b2 = 0; b2 < 9; ++b2) cd[a * 9 + b2] += da * (w->conv0[ch * 9 + b2] - mean[b2]);
+      }
+    for (int i = 0; i < 81; ++i) cov[i] = (float)(cd[i] / kC0);
+    m->conv0c = up.f32(wc.data(), wc.size());
+    m->conv0cov = up.f32(cov.data(), cov.size());
+  }
+  m->ln0 = up.f32(w->ln0, kC0);
+  m->ln1 = up.f32(w->ln1, kC1);
+  {
+    std::vector<float> w1((size_t)kC1 * 9 * kC0);  // [c1][tap * c0 + ci]
+    for (int o = 0; o < kC1; ++o)
+      for (int ci = 0; ci < kC0; ++ci)
+        for (int tap = 0; tap < 9; ++tap) w1[(size_t)o * 9 * kC0 + tap * kC0 + ci] = w->conv1[((size_t)o * kC0 + ci) * 9 + tap];
+    m->conv1 = up.mat(w1);
+  }
+  m->in_proj = up.mat(w->in_proj, (size_t)H * kHidden);
+  m->out_proj = up.mat(w->out_proj, (size_t)c.out_dim * H);
+  m->out_bias = up.f32(w->out_bias, c.out_dim);
+  m->embed = up.mat(w->embed, (size_t)c.embed_dim * c.out_dim);
+  std::vector<float> R((size_t)kLeft * H), qs(kHeadDim);
+  for (int i = 0; i < c.n_layers && up.ok; ++i) {
+    const ae_host_layer &l = w->layers[i];
+    LayerDev L;
+    std::memset(&L, 0, sizeof(L));
+    L.ff1_pre = up.f32(l.ff1_pre, H);
+    L.ff1_post = up.f32(l.ff1_post, H);
+    L.ff2_pre = up.f32(l.ff2_pre, H);
+    L.ff2_post = up.f32(l.ff2_post, H);
+    L.norm_pre_attn = up.f32(l.norm_pre_attn, H);
+    L.norm_post_attn = up.f32(l.norm_post_attn, H);
+    L.norm_out = up.f32(l.norm_out, H);
+    L.lc_pre = up.f32(l.lc_pre, H);
+    L.lc_norm = up.f32(l.lc_norm, H);
+    {
+      std::vector<float> t((size_t)kKernel * H);  // tap-major
+      for (int ch = 0; ch < H; ++ch)
+        for (int k = 0; k < kKernel; ++k) t[(size_t)k * H + ch] = l.lc_dw[(size_t)ch * kKernel + k];
+      L.lc_dw = up.f32(t.data(), t.size());
+    }
+    float ks;
+    attention_tables_host(l.relative_k, l.per_dim_scale, H, c.heads, kLeft, R.data(), qs.data(), &ks);
+    m->k_scale = ks;
+    L.R = up.f32(R.data(), R.size());
+    L.qscale = up.f32(qs.data(), qs.size());
+    L.ff1_w1 = up.mat(l.ff1_w1, (size_t)c.ffn * H);
+    L.ff1_w2 = up.mat(l.ff1_w2, (size_t)H * c.ffn);
+    L.ff2_w1 = up.mat(l.ff2_w1, (size_t)c.ffn * H);
+    L.ff2_w2 = up.mat(l.ff2_w2, (size_t)H * c.ffn);
+    {
+      std::vector<float> qkv((size_t)3 * H * H);
+      std::memcpy(qkv.data(), l.q, (size_t)H * H * 4);
+      std::memcpy(qkv.data() + (size_t)H * H, l.k, (size_t)H * H * 4);
+      std::memcpy(qkv.data() + (size_t)2 * H * H, l.v, (size_t)H * H * 4);
+      L.qkv = up.mat(qkv);
+    }
+    L.post = up.mat(l.post, (size_t)H * H);
+    L.lc_end = up.mat(l.lc_end, (size_t)H * H);
+    {
+      std::vector<float> ls((size_t)2 * H * H);  // rows interleaved: (a_c, b_c) adjacent
+      for (int r = 0; r < H; ++r) {
+        std::memcpy(ls.data() + (size_t)(2 * r) * H, l.lc_start + (size_t)r * H, (size_t)H * 4);
+        std::memcpy(ls.data() + (size_t)(2 * r + 1) * H, l.lc_start + (size_t)(H + r) * H, (size_t)H * 4);
+      }
+      L.lc_start = up.mat(ls);
+    }
+    L.c_ff1_w1 = l.clip_ff1_w1; L.c_ff1_w2 = l.clip_ff1_w2; L.c_ff2_w1 = l.clip_ff2_w1; L.c_ff2_w2 = l.clip_ff2_w2;
+    L.c_q = l.clip_q; L.c_k = l.clip_k; L.c_v = l.clip_v; L.c_post = l.clip_post;
+    L.c_lc_start = l.clip_lc_start; L.c_lc_end = l.clip_lc_end;
+    m->layers.push_back(L);
+  }
+  if (c.n_layers == 0) m->k_scale = (float)(std::log(1.0 + std::exp(1.0)) / std::log(2.0));
+  if (!up.ok) {
+    ae_model_destroy(m);
+    return fail(AE_ENOMEM, "device allocation or copy failed while uploading the weights");
+  }
+  if (dtype == AE_BF16) {
+    bool ok = make_tmap_2d_bf16(&m->tm_conv1, m->conv1, 9 * kC0, kC1, 9 * kC0 * 2, 64, kC1) &&
+              make_tmap_2d_bf16(&m->tm_in_proj, m->in_proj, kHidden, H, kHidden * 2, 64, 256) &&
+              make_tmap_2d_bf16(&m->tm_out_proj, m->out_proj, H, c.out_dim, H * 2, 64, 256) &&
+              make_tmap_2d_bf16(&m->tm_embed, m->embed, c.out_dim, c.embed_dim, c.out_dim * 2, 64, 256);
+    for (auto &L : m->layers) {
+      ok = ok && make_tmap_2d_bf16(&L.tm_ff1_w1, L.ff1_w1, H, c.ffn, H * 2, 64, 256) &&
+           make_tmap_2d_bf16(&L.tm_ff1_w2, L.ff1_w2, c.ffn, H, (uint64_t)c.ffn * 2, 64, 256) &&
+           make_tmap_2d_bf16(&L.tm_ff2_w1, L.ff2_w1, H, c.ffn, H * 2, 64, 256) &&
+           make_tmap_2d_bf16(&L.tm_ff2_w2, L.ff2_w2, c.ffn, H, (uint64_t)c.ffn * 2, 64, 256) &&
+           make_tmap_2d_bf16(&L.tm_qkv, L.qkv, H, 3 * H, H * 2, 64, 256) &&
+           make_tmap_2d_bf16(&L.tm_post, L.post, H, H, H * 2, 64, 256) &&
+           make_tmap_2d_bf16(&L.tm_lc_start, L.lc_start, H, 2 * H, H * 2, 64, 256) &&
+           make_tmap_2d_bf16(&L.tm_lc_end, L.lc_end, H, H, H * 2, 64, 256);
+    }
+    if (!ok) {
+      ae_model_destroy(m);
+      return fail(AE_ECUDA, "tensor map encoding failed");
+    }
+  }
+  *out = m;
+  return AE_OK;
+}
+
+size_t ae_workspace_size(const ae_model *m, int64_t n_clips, int64_t total_frames, int64_t total_tokens) {
+  if (n_clips < 0 || total_frames < 0 || total_tokens < 0) return 0;
+  return ws_layout(m, n_clips, total_frames, total_tokens, m != nullptr).total;
+}
+
+ae_status ae_logmel(const float *d_wave, const int64_t *h_sample_off, int n_clips, float *d_mel, void *d_ws,
+                    size_t ws_bytes, ae_stream stream) {
+  ClipTables T;
+  ae_status st = build_tables(h_sample_off, n_clips, kSamples, T, "h_sample_off");
+  if (st) return st;
+  if (T.total_frames > 0 && (!d_wave || !d_mel)) return fail(AE_EINVAL, "d_wave or d_mel is null");
+  const WsLayout L = ws_layout(nullptr, T.n_clips, T.total_frames, 0, false);  // no token positions needed
+  if (n_clips == 0) return AE_OK;
+  if ((st = check_ws(d_ws, ws_bytes, L.total))) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  ClipTablesDev td;
+  cudaError_t e = tables_t(T, d_ws, L, &td, false, s);
+  if (e != cudaSuccess) return cuda_fail(e, "table upload");
+  if ((e = logmel_t(d_wave, d_mel, td, T, s)) != cudaSuccess) return cuda_fail(e, "logmel");
+  return AE_OK;
+}
+
+ae_status ae_subsample(const ae_model *m, const float *d_mel, const int64_t *h_frame_off, int n_clips, float *d_h,
+                       void *d_ws, size_t ws_bytes, ae_stream stream) {
+  ae_status st = check_model(m);
+  if (st) return st;
+  ClipTables T;
+  if ((st = build_tables(h_frame_off, n_clips, kFrames, T, "h_frame_off"))) return st;
+  if (T.total_tokens > 0 && (!d_mel || !d_h)) return fail(AE_EINVAL, "d_mel or d_h is null");
+  const WsLayout L = ws_layout(m, T.n_clips, T.total_frames, T.total_tokens, true);
+  if (n_clips == 0) return AE_OK;
+  if ((st = check_ws(d_ws, ws_bytes, L.total))) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  ClipTablesDev td;
+  cudaError_t e = tables_t(T, d_ws, L, &td, false, s);
+  if (e != cudaSuccess) return cuda_fail(e, "table upload");
+  if (T.total_tokens == 0) return AE_OK;
+  uint8_t *w = static_cast<uint8_t *>(d_ws);
+  if ((e = conv0_t(m, d_mel, w + L.y0, td, T, s)) != cudaSuccess) return cuda_fail(e, "conv0");
+  if ((e = conv1_t(m, w + L.y0, w + L.xs, td, T, s)) != cudaSuccess)
+    return cuda_fail(e, "conv1");
+  if ((e = gemm_t(m, w + L.xs, T.total_tokens, kHidden, m->in_proj, m->dtype == AE_BF16 ? &m->tm_in_proj : nullptr,
+                m->cfg.hidden, EPI_F32, ep_of(d_h, m->cfg.hidden, -INFINITY, INFINITY), s)) != cudaSuccess)
+    return cuda_fail(e, "in_proj");
+  return AE_OK;
+}
+
+ae_status ae_conformer_layer(const ae_model *m, int layer, float *d_h, const int64_t *h_tok_off, int n_clips,
+                             void *d_ws, size_t ws_bytes, ae_stream stream) {
+  ae_status st = check_model(m);
+  if (st) return st;
+  if (layer < 0 || layer >= m->cfg.n_layers) return fail(AE_EINVAL, "layer index out of range");
+  ClipTables T;
+  if ((st = build_tables(h_tok_off, n_clips, kTokens, T, "h_tok_off"))) return st;
+  if (T.total_tokens > 0 && !d_h) return fail(AE_EINVAL, "d_h is null");
+  const WsLayout L = ws_layout(m, T.n_clips, T.total_frames, T.total_tokens, true);
+  if (T.total_tokens == 0) return AE_OK;
+  if ((st = check_ws(d_ws, ws_bytes, L.total))) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  ClipTablesDev td;
+  cudaError_t e = tables_t(T, d_ws, L, &td, true, s);
+  if (e != cudaSuccess) return cuda_fail(e, "table upload");
+  Bufs b = bufs_of(d_ws, L, td);
+  b.h = d_h;
+  if ((e = run_layer(m, layer, b, T.total_tokens, false, kNextNone, s)) != cudaSuccess) return cuda_fail(e, "layer");
+  return AE_OK;
+}
+
+ae_status ae_encode(const ae_model *m, const float *d_wave, const int64_t *h_sample_off, int n_clips, float *d_out,
+                    void *d_ws, size_t ws_bytes, ae_stream stream) {
+  ae_status st = check_model(m);
+  if (st) return st;
+  ClipTables T;
+  if ((st = build_tables(h_sample_off, n_clips, kSamples, T, "h_sample_off"))) return st;
+  if (T.total_tokens > 0 && (!d_wave || !d_out)) return fail(AE_EINVAL, "d_wave or d_out is null");
+  const WsLayout L = ws_layout(m, T.n_clips, T.total_frames, T.total_tokens, true);
+  if (n_clips == 0) return AE_OK;
+  if ((st = check_ws(d_ws, ws_bytes, L.total))) return st;
+  return encode_dev(m, d_wave, T, d_out, d_ws, L, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t ae_encode_host_workspace_size(const ae_model *m, const int64_t *h_sample_off, int n_clips) {
+  ClipTables T;
+  if (!m || build_tables(h_sample_off, n_clips, kSamples, T, "h_sample_off") != AE_OK) return 0;
+  const WsLayout L = ws_layout(m, T.n_clips, T.total_frames, T.total_tokens, true);
+  return L.total + al256((size_t)T.total_samples * 4) + al256((size_t)T.total_tokens * m->cfg.embed_dim * 4);
+}
+
+ae_status ae_encode_host(const ae_model *m, const float *h_wave, const int64_t *h_sample_off, int n_clips,
+                         float *h_out, void *d_ws, size_t ws_bytes, ae_stream stream) {
+  ae_status st = check_model(m);
+  if (st) return st;
+  ClipTables T;
+  if ((st = build_tables(h_sample_off, n_clips, kSamples, T, "h_sample_off"))) return st;
+  if (T.total_samples > 0 && !h_wave) return fail(AE_EINVAL, "h_wave is null");
+  if (T.total_tokens > 0 && !h_out) return fail(AE_EINVAL, "h_out is null");
+  const WsLayout L = ws_layout(m, T.n_clips, T.total_frames, T.total_tokens, true);
+  const size_t wave_b = al256((size_t)T.total_samples * 4);
+  const size_t out_b = al256((size_t)T.total_tokens * m->cfg.embed_dim * 4);
+  if (n_clips == 0) return AE_OK;
+  if ((st = check_ws(d_ws, ws_bytes, L.total + wave_b + out_b))) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *w = static_cast<uint8_t *>(d_ws);
+  float *d_wave = reinterpret_cast<float *>(w + L.total);
+  float *d_out = reinterpret_cast<float *>(w + L.total + wave_b);
+  cudaError_t e;
+  if (T.total_samples > 0 &&
+      (e = cudaMemcpyAsync(d_wave, h_wave, (size_t)T.total_samples * 4, cudaMemcpyHostToDevice, s)) != cudaSuccess)
+    return cuda_fail(e, "copy in");
+  if ((st = encode_dev(m, d_wave, T, d_out, d_ws, L, s))) return st;
+  if (T.total_tokens > 0 &&
+      (e = cudaMemcpyAsync(h_out, d_out, (size_t)T.total_tokens * m->cfg.embed_dim * 4, cudaMemcpyDeviceToHost, s)) !=
+          cudaSuccess)
+    return cuda_fail(e, "copy out");
+  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_fail(e, "stream");
+  return AE_OK;
+}
+
+ae_status ae_local_attention(const void *d_q, const void *d_k, const void *d_v, int64_t ld_qkv, ae_dtype dtype,
+                             const float *d_R, const float *d_qscale, float k_scale, float softcap,
+                             const int64_t *h_tok_off, int n_clips, void *d_out, int64_t ld_out, void *d_ws,
+                             size_t ws_bytes, ae_stream stream) {
+  if (dtype != AE_F32 && dtype != AE_BF16) return fail(AE_EINVAL, "dtype");
+  ClipTables T;
+  ae_status st = build_tables(h_tok_off, n_clips, kTokens, T, "h_tok_off");
+  if (st) return st;
+  if (T.total_tokens > 0) {
+    if (!d_q || !d_k || !d_v || !d_out || !d_R || !d_qscale) return fail(AE_EINVAL, "a device pointer is null");
+    if (!aligned16(d_q) || !aligned16(d_k) || !aligned16(d_v) || !aligned16(d_out))
+      return fail(AE_EINVAL, "q, k, v and out must be 16-byte aligned");
+    const int64_t vec = dtype == AE_BF16 ? 8 : 4;
+    if (ld_qkv < kHidden || ld_out < kHidden || ld_qkv % vec || ld_out % vec)
+      return fail(AE_EINVAL, "row strides must be >= 1024 and a multiple of 16 bytes");
+    if (!(softcap > 0.f) || !std::isfinite(softcap) || !std::isfinite(k_scale))
+      return fail(AE_EINVAL, "softcap must be positive and finite");
+  }
+  const WsLayout L = ws_layout(nullptr, T.n_clips, 0, T.total_tokens, false);
+  if (T.total_tokens == 0) return AE_OK;
+  if ((st = check_ws(d_ws, ws_bytes, L.total))) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  ClipTablesDev td;
+  cudaError_t e = tables_t(T, d_ws, L, &td, true, s);
+  if (e != cudaSuccess) return cuda_fail(e, "table upload");
+  const double abytes = 4.0 * (dtype == AE_BF16 ? 2 : 4) * kHidden * (double)T.total_tokens;
+  if ((e = timed(AE_K_ATTENTION, 0.0, abytes, s, [&] {
+         return launch_attention(dtype == AE_BF16, d_q, d_k, d_v, ld_qkv, d_R, d_qscale, k_scale, softcap, td.pos,
+                                 T.total_tokens, d_out, ld_out, -INFINITY, INFINITY, s);
+       })) != cudaSuccess)
+    return cuda_fail(e, "attention");
+  return AE_OK;
+}
+
+ae_status ae_profile_enable(int on) {
+  Profiler &P = g_prof;
+  if (on && P.ev.empty()) {
+    const size_t cap = 16384;
+    P.ev.resize(2 * cap);
+    for (auto &e : P.ev)
+      if (cudaEventCreate(&e) != cudaSuccess) {
+        for (auto &x : P.ev)
+          if (x) cudaEventDestroy(x);
+        P.ev.clear();
+        return fail(AE_ECUDA, "could not create the timing events");
+      }
+    P.recs.resize(cap);
+    P.cap = cap;
+  }
+  P.on = on != 0;
+  return AE_OK;
+}
+
+ae_status ae_profile_read(double *ms, int64_t *launches, double *flops, double *bytes, int64_t *dropped) {
+  Profiler &P = g_prof;
+  double t[AE_K_COUNT] = {0}, f[AE_K_COUNT] = {0}, b[AE_K_COUNT] = {0};
+  int64_t n[AE_K_COUNT] = {0};
+  if (P.n > 0) {
+    cudaError_t e = cudaEventSynchronize(P.ev[2 * P.n - 1]);
+    if (e != cudaSuccess) return cuda_fail(e, "timing events");
+    for (size_t i = 0; i < P.n; ++i) {
+      float x = 0.f;
+      if ((e = cudaEventElapsedTime(&x, P.ev[2 * i], P.ev[2 * i + 1])) != cudaSuccess) return cuda_fail(e, "timing");
+      const int c = P.recs[i].cls;
+      t[c] += x;
+      n[c] += 1;
+      f[c] += P.recs[i].flops;
+      b[c] += P.recs[i].bytes;
+    }
+  }
+  for (int c = 0; c < AE_K_COUNT; ++c) {
+    if (ms) ms[c] = t[c];
+    if (launches) launches[c] = n[c];
+    if (flops) flops[c] = f[c];
+    if (bytes) bytes[c] = b[c];
+  }
+  if (dropped) *dropped = P.dropped;
+  P.n = 0;
+  P.dropped = 0;
+  return AE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,421 @@
+// Projections of the tower: y = epilogue(x W^T) with x [M][K] (packed token
+// rows, M ragged) and W [N][K] (the checkpoint's [out][in] layout).
+//
+// bf16 path: a persistent, warp-specialised tcgen05 kernel. Warp 0 streams
+// 128x64 tiles of x and 256x64 tiles of W into a 4-stage shared-memory ring
+// with TMA (128-byte swizzle, no multicast); warp 1 allocates 512 columns of
+// tensor memory and issues tcgen05.mma (M=128, N=256, K=16, bf16 in, f32
+// accumulate) into one of two 256-column accumulators; warps 2-5 read the
+// other accumulator with tcgen05.ld, apply the epilogue (ClipLin output
+// clamp, SiLU and the next projection's input clamp, GLU, or bias) and store.
+// Tiles are walked m-major so the CTAs in flight share rows of x in L2 while
+// W stays L2-resident.
+//
+// f32 path: a plain 64x64-tile FMA kernel with the same epilogues.
+#include <cudaTypedefs.h>
+
+#include "ae_internal.h"
+#include "common.cuh"
+
+namespace ae {
+
+__device__ unsigned g_status_word = 0;
+
+unsigned read_and_clear_status() {
+  unsigned v = 0, z = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status_word, sizeof(v)) != cudaSuccess) return ~0u;
+  cudaMemcpyToSymbol(g_status_word, &z, sizeof(z));
+  return v;
+}
+
+unsigned *device_status_word() {
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+  return static_cast<unsigned *>(p);
+}
+
+// ------------------------------------------------------------------ epilogue
+
+template <int MODE>
+__device__ __forceinline__ void epi_store_tc(const EpiArgs &ep, int row, int col, const uint32_t (&r)[32]) {
+  float lo = ep.lo, hi = ep.hi;
+  if (ep.seg_w > 0) {
+    const int sg = col / ep.seg_w;
+    lo = ep.seg_lo[sg];
+    hi = ep.seg_hi[sg];
+  }
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  if (MODE == EPI_F32) {
+    if (ep.bias) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] += __ldg(ep.bias + col + i);
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = clampf(v[i], lo, hi);
+    float *o = static_cast<float *>(ep.out) + (int64_t)row * ep.ld + col;
+#pragma unroll
+    for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4 *>(o + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+  } else if (MODE == EPI_GLU) {
+    uint32_t p[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float a0 = clampf(v[4 * j + 0], lo, hi), b0 = clampf(v[4 * j + 1], lo, hi);
+      float a1 = clampf(v[4 * j + 2], lo, hi), b1 = clampf(v[4 * j + 3], lo, hi);
+      p[j] = pack_bf16(a0 / (1.0f + __expf(-b0)), a1 / (1.0f + __expf(-b1)));
+    }
+    bf16 *o = static_cast<bf16 *>(ep.out) + (int64_t)row * ep.ld + col / 2;
+    reinterpret_cast<uint4 *>(o)[0] = make_uint4(p[0], p[1], p[2], p[3]);
+    reinterpret_cast<uint4 *>(o)[1] = make_uint4(p[4], p[5], p[6], p[7]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      float x = clampf(v[i], lo, hi);
+      if (MODE == EPI_SILU) x = clampf(x / (1.0f + __expf(-x)), ep.lo2, ep.hi2);
+      v[i] = x;
+    }
+    uint32_t p[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) p[j] = pack_bf16(v[2 * j], v[2 * j + 1]);
+    uint4 *o = reinterpret_cast<uint4 *>(static_cast<bf16 *>(ep.out) + (int64_t)row * ep.ld + col);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) o[j] = make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
+  }
+}
+
+// ------------------------------------------------------------------ tcgen05 kernel
+
+namespace {
+constexpr int BM = 128, BK = 64, BN = 256, STAGES = 4;
+constexpr uint32_t A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr size_t SMEM_TC = STAGES * STAGE_BYTES + 1024 + 256;
+}  // namespace
+
+template <int MODE>
+__global__ void __launch_bounds__(192, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const EpiArgs ep,
+              const int M, const int N, const int K, unsigned *status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+  uint64_t *empty = full + STAGES;
+  uint64_t *tfull = empty + STAGES;
+  uint64_t *tempty = tfull + 2;
+  uint64_t *done = tempty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m_blocks = (M + BM - 1) / BM, n_blocks = N / BN, kb_n = K / BK;
+  const int num_tiles = m_blocks * n_blocks;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 128);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    long issued = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const int mb = tile / n_blocks, nb = tile % n_blocks;
+      for (int kb = 0; kb < kb_n; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1) || *abort_flag) {
+          ok = false;
+          break;
+        }
+        uint8_t *sa = smem + stage * STAGE_BYTES;
+        mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+        tma_load_2d(sa, &tmA, kb * BK, mb * BM, &full[stage]);
+        tma_load_2d(sa + A_BYTES, &tmB, kb * BK, nb * BN, &full[stage]);
+        ++issued;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    if (!ok) {
+      atomicOr(status, kStatusWaitTimeout);
+      *abort_flag = 1;
+    }
+    // every load issued must land before the CTA may exit
+    for (int s = 0; s < STAGES; ++s) {
+      const long n = issued / STAGES + (s < issued % STAGES ? 1 : 0);
+      if (n > 0) mbar_wait(&full[s], (uint32_t)((n - 1) & 1));
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+    int stage = 0, acc = 0;
+    uint32_t phase = 0, acc_phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      if (!mbar_wait(&tempty[acc], acc_phase ^ 1) || *abort_flag) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * BN;
+      for (int kb = 0; kb < kb_n; ++kb) {
+        if (!mbar_wait(&full[stage], phase)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+        const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k)
+          tc_mma_bf16(d_tmem, sw128_desc(sa + k * 32), sw128_desc(sb + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
+        tc_commit(&empty[stage]);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) break;
+      tc_commit(&tfull[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+    if (!ok) {
+      atomicOr(status, kStatusWaitTimeout);
+      *abort_flag = 1;
+    }
+    tc_commit(done);  // arrives once every MMA issued above has completed
+    mbar_wait(done, 0);
+  } else if (warp >= 2) {
+    // ---------------- epilogue: warp w reads TMEM lanes 32*(w%4) .. +31
+    const int q = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const int mb = tile / n_blocks, nb = tile % n_blocks;
+      const bool got = mbar_wait(&tfull[acc], acc_phase);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int row = mb * BM + q * 32 + lane;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c * 32), r);
+        tmem_ld_wait();
+        if (row < M) epi_store_tc<MODE>(ep, row, nb * BN + c * 32, r);
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+    if (!ok && lane == 0) {
+      atomicOr(status, kStatusWaitTimeout);
+      *abort_flag = 1;
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ f32 FMA kernel
+
+template <int MODE>
+__global__ void __launch_bounds__(256) k_gemm_f32(const float *__restrict__ A, const float *__restrict__ B,
+                                                  const EpiArgs ep, int M, int N, int K) {
+  __shared__ float As[16][64 + 4];
+  __shared__ float Bs[16][64 + 4];
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  float acc[4][4] = {};
+  const int lr = threadIdx.x >> 2, lc = (threadIdx.x & 3) * 4;
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (m0 + lr < M) a = *reinterpret_cast<const float4 *>(A + (int64_t)(m0 + lr) * K + k0 + lc);
+    const float4 b = *reinterpret_cast<const float4 *>(B + (int64_t)(n0 + lr) * K + k0 + lc);
+    As[lc + 0][lr] = a.x; As[lc + 1][lr] = a.y; As[lc + 2][lr] = a.z; As[lc + 3][lr] = a.w;
+    Bs[lc + 0][lr] = b.x; Bs[lc + 1][lr] = b.y; Bs[lc + 2][lr] = b.z; Bs[lc + 3][lr] = b.w;
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float a4[4], b4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a4[i] = As[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b4[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a4[i], b4[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  const int col = n0 + tx * 4;
+  float lo = ep.lo, hi = ep.hi;
+  if (ep.seg_w > 0) {
+    const int sg = col / ep.seg_w;
+    lo = ep.seg_lo[sg];
+    hi = ep.seg_hi[sg];
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int row = m0 + ty * 4 + i;
+    if (row >= M) continue;
+    float v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float x = acc[i][j];
+      if (MODE == EPI_F32 && ep.bias) x += ep.bias[col + j];
+      x = clampf(x, lo, hi);
+      if (MODE == EPI_SILU) x = clampf(x / (1.0f + expf(-x)), ep.lo2, ep.hi2);
+      v[j] = x;
+    }
+    float *o = static_cast<float *>(ep.out) + (int64_t)row * ep.ld;
+    if (MODE == EPI_GLU) {
+      o[col / 2] = v[0] / (1.0f + expf(-v[1]));
+      o[col / 2 + 1] = v[2] / (1.0f + expf(-v[3]));
+    } else {
+      *reinterpret_cast<float4 *>(o + col) = make_float4(v[0], v[1], v[2], v[3]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+bool make_tmap_2d_bf16(CUtensorMap *tm, const void *base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                       uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Stem conv0 output viewed as 5-D for the implicit GEMM of conv1:
+// (c 128, fpar 2, fp 32, tpar 2, tp rows/2), boxes (64, 1, 32, 1, 4).
+bool make_tmap_stem_y0(CUtensorMap *tm, const void *y0, int64_t stem_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[5] = {(cuuint64_t)kC0, 2, (cuuint64_t)kF1 / 2, 2, (cuuint64_t)(stem_rows / 2)};
+  cuuint64_t strides[4] = {(cuuint64_t)kC0 * 2, (cuuint64_t)kC0 * 2 * 2, (cuuint64_t)kF1 * kC0 * 2,
+                           (cuuint64_t)kF1 * kC0 * 2 * 2};
+  cuuint32_t box[5] = {64, 1, 32, 1, (cuuint32_t)kConv1TileTok};
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(y0), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static int num_sms() {
+  static int n[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!n[dev]) cudaDeviceGetAttribute(&n[dev], cudaDevAttrMultiProcessorCount, dev);
+  return n[dev] > 0 ? n[dev] : 1;
+}
+
+template <int MODE>
+static cudaError_t launch_tc(const CUtensorMap &tA, const CUtensorMap &tB, const EpiArgs &ep, int M, int N, int K,
+                             cudaStream_t s) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_TC);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int tiles = ((M + BM - 1) / BM) * (N / BN);
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  k_gemm_tc<MODE><<<grid, 192, SMEM_TC, s>>>(tA, tB, ep, M, N, K, device_status_word());
+  return cudaGetLastError();
+}
+
+template <int MODE>
+static cudaError_t launch_f32(const float *x, const float *w, const EpiArgs &ep, int M, int N, int K,
+                              cudaStream_t s) {
+  dim3 grid(N / 64, (M + 63) / 64);
+  k_gemm_f32<MODE><<<grid, 256, 0, s>>>(x, w, ep, M, N, K);
+  return cudaGetLastError();
+}
+
+cudaError_t gemm(const ae_model *m, const void *x, int64_t M, int K, const void *w, const CUtensorMap *tmW, int N,
+                 int mode, const EpiArgs &ep, cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  if (m->dtype == AE_BF16) {
+    CUtensorMap tA, tB;
+    if (!make_tmap_2d_bf16(&tA, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK, BM)) return cudaErrorInvalidValue;
+    if (!tmW) {
+      if (!make_tmap_2d_bf16(&tB, w, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, BK, BN))
+        return cudaErrorInvalidValue;
+      tmW = &tB;
+    }
+    switch (mode) {
+      case EPI_F32: return launch_tc<EPI_F32>(tA, *tmW, ep, (int)M, N, K, s);
+      case EPI_BF16: return launch_tc<EPI_BF16>(tA, *tmW, ep, (int)M, N, K, s);
+      case EPI_SILU: return launch_tc<EPI_SILU>(tA, *tmW, ep, (int)M, N, K, s);
+      case EPI_GLU: return launch_tc<EPI_GLU>(tA, *tmW, ep, (int)M, N, K, s);
+    }
+    return cudaErrorInvalidValue;
+  }
+  const float *xf = static_cast<const float *>(x);
+  const float *wf = static_cast<const float *>(w);
+  switch (mode) {
+    case EPI_F32: return launch_f32<EPI_F32>(xf, wf, ep, (int)M, N, K, s);
+    case EPI_BF16: return launch_f32<EPI_BF16>(xf, wf, ep, (int)M, N, K, s);
+    case EPI_SILU: return launch_f32<EPI_SILU>(xf, wf, ep, (int)M, N, K, s);
+    case EPI_GLU: return launch_f32<EPI_GLU>(xf, wf, ep, (int)M, N, K, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace ae

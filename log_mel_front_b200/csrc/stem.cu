@@ -1,0 +1,317 @@
+// Subsampling stem (egemma2_audio.rs, AudioTower::subsample): two 3x3
+// stride-2 convolutions with zero padding 1 and no bias, each followed by a
+// bias-free LayerNorm over the channels (eps 1e-6) and ReLU.
+//
+// conv0 (1 -> 128 channels): the channel mean of the outputs is linear in
+// the 9-sample patch p and their variance is the quadratic form p^T C p of
+// the taps' channel covariance C, so one pass gives the normalised outputs:
+// y_c = relu(g_c (w'_c . p) / sqrt(p^T C p + eps)) with w'_c the taps minus
+// their channel mean (both precomputed in float64 at model creation). One
+// CTA writes one time row [64 freq][128 ch] of the channels-last output.
+//
+// The output rows of each clip are laid out with two zero rows in front and
+// zero rows after the last real one, up to 2 * tokens + 2 rows per clip, so
+// the second convolution's stride-2 windows never need a bounds test in
+// time and never read a neighbouring clip.
+//
+// conv1 (128 -> 32 channels) as an implicit GEMM on the tensor cores: the
+// output rows (token, freq) are GEMM rows, K = 9 taps x 128 channels. For
+// each tap the A tile (4 tokens x 32 freq x 64 channels) is one TMA box of a
+// 5-D view of conv0's output that splits time and frequency into (pair,
+// parity), so the stride-2 gather is a plain box; the frequency pad at -1 is
+// the TMA's out-of-range zero fill. tcgen05.mma (M=128, N=32) accumulates
+// in tensor memory; the epilogue thread of each row holds all 32 channels
+// and applies the LayerNorm, ReLU and the frequency-major flatten.
+#include "ae_internal.h"
+#include "common.cuh"
+
+namespace ae {
+
+// Clip of a packed row index, by binary search over a prefix array [B+1].
+__device__ __forceinline__ int clip_of(const int32_t *off, int n_clips, int64_t r) {
+  int lo = 0, hi = n_clips;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (off[mid] <= r) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+// ------------------------------------------------------------------ conv0 + LN + ReLU
+
+template <typename OutT>
+__global__ void __launch_bounds__(256) k_conv0(const float *__restrict__ mel, const float *__restrict__ wc,
+                                               const float *__restrict__ cov, const float *__restrict__ g0,
+                                               OutT *__restrict__ y0, const ClipTablesDev t) {
+  __shared__ float s_w[kC0 * 9];
+  __shared__ float s_g[kC0];
+  __shared__ float s_p[kF1][10];
+  __shared__ float s_r[kF1];
+  const int64_t row = blockIdx.x;
+  const int c = clip_of(t.stem_off, t.n_clips, row);
+  const int ti = (int)(row - t.stem_off[c]) - 2;
+  const int F = t.frame_off[c + 1] - t.frame_off[c];
+  const int t1 = (F + 1) / 2;
+  OutT *orow = y0 + row * (int64_t)(kF1 * kC0);
+  if (ti < 0 || ti >= t1) {
+    for (int i = threadIdx.x; i < kF1 * kC0; i += blockDim.x) orow[i] = Act<OutT>::zero();
+    return;
+  }
+  for (int i = threadIdx.x; i < kC0 * 9; i += blockDim.x) s_w[i] = wc[i];
+  for (int i = threadIdx.x; i < kC0; i += blockDim.x) s_g[i] = g0[i];
+  if (threadIdx.x < kF1) {
+    const int f = threadIdx.x;
+    const float *m = mel + (int64_t)t.frame_off[c] * kMels;
+    float p[9];
+#pragma unroll
+    for (int dt = 0; dt < 3; ++dt)
+#pragma unroll
+      for (int df = 0; df < 3; ++df) {
+        const int tr = 2 * ti + dt - 1, fr = 2 * f + df - 1;
+        p[dt * 3 + df] = (tr >= 0 && tr < F && fr >= 0 && fr < kMels) ? m[(int64_t)tr * kMels + fr] : 0.f;
+      }
+    float var = 0.f;
+#pragma unroll
+    for (int a = 0; a < 9; ++a) {
+      float s = 0.f;
+#pragma unroll
+      for (int b = 0; b < 9; ++b) s = fmaf(cov[a * 9 + b], p[b], s);
+      var = fmaf(p[a], s, var);
+    }
+#pragma unroll
+    for (int k = 0; k < 9; ++k) s_p[f][k] = p[k];
+    s_r[f] = rsqrtf(fmaxf(var, 0.f) + 1e-6f);
+  }
+  __syncthreads();
+  // thread -> (freq f, 32 consecutive channels)
+  const int f = threadIdx.x >> 2, c0 = (threadIdx.x & 3) * 32;
+  float p[9];
+#pragma unroll
+  for (int k = 0; k < 9; ++k) p[k] = s_p[f][k];
+  const float r = s_r[f];
+  OutT *o = orow + f * kC0 + c0;
+#pragma unroll
+  for (int q = 0; q < 32; q += 4) {
+    float v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float *w = s_w + (c0 + q + u) * 9;
+      float a = 0.f;
+#pragma unroll
+      for (int k = 0; k < 9; ++k) a = fmaf(w[k], p[k], a);
+      v[u] = fmaxf(a * r * s_g[c0 + q + u], 0.f);
+    }
+    store4(o + q, v);
+  }
+}
+
+// ------------------------------------------------------------------ conv1, tensor cores (bf16)
+
+namespace {
+constexpr int C1_STAGES = 4;
+constexpr uint32_t C1_A = 128 * 64 * 2, C1_B = kC1 * 64 * 2, C1_STAGE = C1_A + C1_B;
+constexpr size_t C1_SMEM = C1_STAGES * C1_STAGE + 1024 + 256;
+constexpr int C1_KB = 9 * kC0 / 64;  // 18 k-blocks of 64
+}  // namespace
+
+__global__ void __launch_bounds__(128, 1)
+    k_conv1_tc(const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmW,
+               const ClipTablesDev t, const float *__restrict__ g1, bf16 *__restrict__ xs, unsigned *status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + C1_STAGES * C1_STAGE);
+  uint64_t *empty = full + C1_STAGES;
+  uint64_t *accb = empty + C1_STAGES;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accb + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  __shared__ float s_g[kC1];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x;
+  const int c = clip_of(t.conv1_tile_off, t.n_clips, tile);
+  const int tok0 = (tile - t.conv1_tile_off[c]) * kConv1TileTok;
+  const int n_tok = t.tok_off[c + 1] - t.tok_off[c];
+  const int tp_base = t.stem_off[c] / 2 + tok0;
+
+  if (threadIdx.x < kC1) s_g[threadIdx.x] = g1[threadIdx.x];
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C1_STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(accb, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 32);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    int issued = 0;
+    bool ok = true;
+    for (int kb = 0; kb < C1_KB; ++kb) {
+      const int s = kb % C1_STAGES;
+      const uint32_t ph = (kb / C1_STAGES) & 1;
+      if (!mbar_wait(&empty[s], ph ^ 1) || *abort_flag) {
+        ok = false;
+        break;
+      }
+      const int tap = kb >> 1, half = kb & 1, dt = tap / 3, df = tap % 3;
+      // time row 2t + dt - 1 is stored row base + 2t + dt + 1 = 2 tp + tpar
+      const int tpar = (dt == 1) ? 0 : 1, tp = tp_base + (dt == 0 ? 0 : 1);
+      // frequency 2f + df - 1 = 2 fp + fpar
+      const int fpar = (df == 1) ? 0 : 1, fp = (df == 0) ? -1 : 0;
+      uint8_t *sa = smem + s * C1_STAGE;
+      mbar_arrive_expect_tx(&full[s], C1_STAGE);
+      tma_load_5d(sa, &tmY, half * 64, fpar, fp, tpar, tp, &full[s]);
+      tma_load_2d(sa + C1_A, &tmW, kb * 64, 0, &full[s]);
+      ++issued;
+    }
+    if (!ok) {
+      atomicOr(status, kStatusWaitTimeout);
+      *abort_flag = 1;
+    }
+    for (int s = 0; s < C1_STAGES; ++s) {
+      const int n = issued / C1_STAGES + (s < issued % C1_STAGES ? 1 : 0);
+      if (n > 0) mbar_wait(&full[s], (uint32_t)((n - 1) & 1));
+    }
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc = idesc_bf16_f32(128, kC1);
+    bool ok = true;
+    for (int kb = 0; kb < C1_KB; ++kb) {
+      const int s = kb % C1_STAGES;
+      const uint32_t ph = (kb / C1_STAGES) & 1;
+      if (!mbar_wait(&full[s], ph) || *abort_flag) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t sa = smem_u32(smem + s * C1_STAGE), sb = sa + C1_A;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        tc_mma_bf16(tmem, sw128_desc(sa + k * 32), sw128_desc(sb + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
+      tc_commit(&empty[s]);
+    }
+    if (!ok) {
+      atomicOr(status, kStatusWaitTimeout);
+      *abort_flag = 1;
+    }
+    tc_commit(accb);  // arrives when every MMA above has completed (or none was issued)
+  }
+  __syncwarp();
+  // ---- epilogue: row = warp * 32 + lane = (token tok0 + warp, freq lane)
+  const bool got = mbar_wait(accb, 0);
+  if (__all_sync(0xffffffffu, got)) {
+    tc_fence_after();
+    uint32_t r[32];
+    tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16), r);
+    tmem_ld_wait();
+    const int tok = tok0 + warp;
+    if (tok < n_tok && !*abort_flag) {
+      float v[32], mean = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        v[i] = __uint_as_float(r[i]);
+        mean += v[i];
+      }
+      mean *= (1.0f / 32);
+      float var = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) var = fmaf(v[i] - mean, v[i] - mean, var);
+      const float rs = rsqrtf(var * (1.0f / 32) + 1e-6f);
+      uint32_t p[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        p[i] = pack_bf16(fmaxf((v[2 * i] - mean) * rs * s_g[2 * i], 0.f),
+                         fmaxf((v[2 * i + 1] - mean) * rs * s_g[2 * i + 1], 0.f));
+      uint4 *o = reinterpret_cast<uint4 *>(xs + ((int64_t)t.tok_off[c] + tok) * kHidden + lane * kC1);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+    }
+  } else if (lane == 0) {
+    atomicOr(status, kStatusWaitTimeout);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 32);
+  }
+}
+
+// ------------------------------------------------------------------ conv1, float32 FMA
+
+// One warp per output row (token, freq): lane = output channel.
+__global__ void __launch_bounds__(256) k_conv1_f32(const float *__restrict__ y0, const float *__restrict__ w1,
+                                                   const float *__restrict__ g1, float *__restrict__ xs,
+                                                   const ClipTablesDev t, int64_t T) {
+  const int64_t gw = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (gw >= T * kF2) return;
+  const int64_t tokg = gw / kF2;
+  const int f = (int)(gw % kF2);
+  const int c = clip_of(t.tok_off, t.n_clips, tokg);
+  const int tok = (int)(tokg - t.tok_off[c]);
+  const float *w = w1 + (int64_t)lane * 9 * kC0;
+  float acc = 0.f;
+  for (int dt = 0; dt < 3; ++dt) {
+    const int64_t row = (int64_t)t.stem_off[c] + 2 * tok + dt + 1;  // time row 2 tok + dt - 1
+    for (int df = 0; df < 3; ++df) {
+      const int fr = 2 * f + df - 1;
+      if (fr < 0 || fr >= kF1) continue;
+      const float *src = y0 + (row * kF1 + fr) * kC0;
+      const float *wk = w + (dt * 3 + df) * kC0;
+      for (int ci = 0; ci < kC0; ++ci) acc = fmaf(src[ci], wk[ci], acc);
+    }
+  }
+  float s = acc;
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  const float mean = s * (1.0f / 32);
+  float d = (acc - mean) * (acc - mean);
+  for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+  const float rs = rsqrtf(d * (1.0f / 32) + 1e-6f);
+  xs[tokg * kHidden + f * kC1 + lane] = fmaxf((acc - mean) * rs * g1[lane], 0.f);
+}
+
+// ------------------------------------------------------------------ launchers
+
+cudaError_t launch_conv0(const ae_model *m, const float *mel, void *y0, const ClipTablesDev &t, int64_t stem_rows,
+                         cudaStream_t s) {
+  if (stem_rows <= 0) return cudaSuccess;
+  if (m->dtype == AE_BF16)
+    k_conv0<bf16><<<(unsigned)stem_rows, 256, 0, s>>>(mel, m->conv0c, m->conv0cov, m->ln0, static_cast<bf16 *>(y0), t);
+  else
+    k_conv0<float><<<(unsigned)stem_rows, 256, 0, s>>>(mel, m->conv0c, m->conv0cov, m->ln0, static_cast<float *>(y0), t);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_conv1(const ae_model *m, const void *y0, int64_t stem_rows, void *xs, const ClipTablesDev &t,
+                         int64_t conv1_tiles, int64_t tokens, cudaStream_t s) {
+  if (tokens <= 0) return cudaSuccess;
+  if (m->dtype == AE_BF16) {
+    static bool attr = false;
+    if (!attr) {
+      cudaError_t e = cudaFuncSetAttribute(k_conv1_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C1_SMEM);
+      if (e != cudaSuccess) return e;
+      attr = true;
+    }
+    CUtensorMap tmY;
+    if (!make_tmap_stem_y0(&tmY, y0, stem_rows)) return cudaErrorInvalidValue;
+    k_conv1_tc<<<(unsigned)conv1_tiles, 128, C1_SMEM, s>>>(tmY, m->tm_conv1, t, m->ln1, static_cast<bf16 *>(xs),
+                                                            device_status_word());
+  } else {
+    const int64_t warps = tokens * kF2;
+    k_conv1_f32<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(static_cast<const float *>(y0),
+                                                             static_cast<const float *>(m->conv1), m->ln1,
+                                                             static_cast<float *>(xs), t, tokens);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace ae
