@@ -656,18 +656,18 @@ ae_status ae_model_create(const ae_config *cfg, const ae_host_weights *w, ae_dty
   }
   if (dtype == AE_BF16) {
     bool ok = make_tmap_2d_bf16(&m->tm_conv1, m->conv1, 9 * kC0, kC1, 9 * kC0 * 2, 64, kC1) &&
-              make_tmap_2d_bf16(&m->tm_in_proj, m->in_proj, kHidden, H, kHidden * 2, 64, 256) &&
-              make_tmap_2d_bf16(&m->tm_out_proj, m->out_proj, H, c.out_dim, H * 2, 64, 256) &&
-              make_tmap_2d_bf16(&m->tm_embed, m->embed, c.out_dim, c.embed_dim, c.out_dim * 2, 64, 256);
+              make_tmap_2d_bf16(&m->tm_in_proj, m->in_proj, kHidden, H, kHidden * 2, 64, 128) &&
+              make_tmap_2d_bf16(&m->tm_out_proj, m->out_proj, H, c.out_dim, H * 2, 64, 128) &&
+              make_tmap_2d_bf16(&m->tm_embed, m->embed, c.out_dim, c.embed_dim, c.out_dim * 2, 64, 128);
     for (auto &L : m->layers) {
-      ok = ok && make_tmap_2d_bf16(&L.tm_ff1_w1, L.ff1_w1, H, c.ffn, H * 2, 64, 256) &&
-           make_tmap_2d_bf16(&L.tm_ff1_w2, L.ff1_w2, c.ffn, H, (uint64_t)c.ffn * 2, 64, 256) &&
-           make_tmap_2d_bf16(&L.tm_ff2_w1, L.ff2_w1, H, c.ffn, H * 2, 64, 256) &&
-           make_tmap_2d_bf16(&L.tm_ff2_w2, L.ff2_w2, c.ffn, H, (uint64_t)c.ffn * 2, 64, 256) &&
-           make_tmap_2d_bf16(&L.tm_qkv, L.qkv, H, 3 * H, H * 2, 64, 256) &&
-           make_tmap_2d_bf16(&L.tm_post, L.post, H, H, H * 2, 64, 256) &&
-           make_tmap_2d_bf16(&L.tm_lc_start, L.lc_start, H, 2 * H, H * 2, 64, 256) &&
-           make_tmap_2d_bf16(&L.tm_lc_end, L.lc_end, H, H, H * 2, 64, 256);
+      ok = ok && make_tmap_2d_bf16(&L.tm_ff1_w1, L.ff1_w1, H, c.ffn, H * 2, 64, 128) &&
+           make_tmap_2d_bf16(&L.tm_ff1_w2, L.ff1_w2, c.ffn, H, (uint64_t)c.ffn * 2, 64, 128) &&
+           make_tmap_2d_bf16(&L.tm_ff2_w1, L.ff2_w1, H, c.ffn, H * 2, 64, 128) &&
+           make_tmap_2d_bf16(&L.tm_ff2_w2, L.ff2_w2, c.ffn, H, (uint64_t)c.ffn * 2, 64, 128) &&
+           make_tmap_2d_bf16(&L.tm_qkv, L.qkv, H, 3 * H, H * 2, 64, 128) &&
+           make_tmap_2d_bf16(&L.tm_post, L.post, H, H, H * 2, 64, 128) &&
+           make_tmap_2d_bf16(&L.tm_lc_start, L.lc_start, H, 2 * H, H * 2, 64, 128) &&
+           make_tmap_2d_bf16(&L.tm_lc_end, L.lc_end, H, H, H * 2, 64, 128);
     }
     if (!ok) {
       ae_model_destroy(m);

@@ -5,124 +5,256 @@
 // cap * tanh(z / cap); natural-exp softmax over the distances; o_t =
 // sum_d p_d v_{t-d}.
 //
-// A CTA owns one head and 128 consecutive tokens. It stages that head's
-// k and v rows for the tokens and the 11-row halo before them in shared
-// memory (coalesced 16-byte loads; rows padded so lanes reading
-// consecutive rows hit distinct banks) plus the head's R[0..11] and the
-// per-dim scales. Each thread then owns one query: the 12 dot products run
-// over 16-dimension chunks held in registers, the softmax over the 12
-// logits is private to the thread, and the weighted sum of v is written
-// back chunk by chunk, clamped to the post projection's input bounds. No
-// cross-thread reduction is needed.
+// bf16 kernel: a CTA owns one head and 256 consecutive tokens; each of its
+// 128 threads owns two consecutive queries (t, t+1), which share 11 of the
+// 13 key/value rows they read. The CTA stages the head's k rows (and then,
+// in the same buffer, its v rows) for its tokens and the 11-row halo in
+// shared memory; rows are 256 bytes with their 16-byte chunks XOR-swizzled
+// by (row / 2) mod 8, so the eight lanes of a shared-memory phase, which read
+// rows two apart, hit distinct banks. R[0..11] is staged pre-divided by
+// k_scale, so q.k and q.R accumulate into one register per (query, distance)
+// and z = k_scale * acc. Dot products and the weighted sum of v use the
+// packed two-wide FMA (fma.rn.f32x2). The softmax over the 12 logits is
+// private to the thread; no cross-thread reduction is needed.
+//
+// float32 kernel (the float32 model): one query per thread, padded rows.
 #include "ae_internal.h"
 #include "common.cuh"
 
 namespace ae {
 
+// d += a * b on two lanes at once
+__device__ __forceinline__ void ffma2(float2 &d, float2 a, float2 b) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rd, {%0, %1};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rd;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(d.x), "+f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+}
+
+__device__ __forceinline__ float2 bf2(uint32_t w) { return make_float2(bf16lo(w), bf16hi(w)); }
+
+namespace {
+constexpr int A2_THREADS = 128;
+constexpr int A2_TOK = 2 * A2_THREADS;          // tokens per CTA
+constexpr int A2_ROWS = A2_TOK + kLeft - 1;     // staged rows
+constexpr size_t A2_SMEM = (size_t)A2_ROWS * kHeadDim * 2 + (kLeft * kHeadDim + kHeadDim) * 4;
+}  // namespace
+
+// 16-byte chunk c (0..15) of staged row r
+__device__ __forceinline__ const uint4 *a2_chunk(const bf16 *buf, int r, int c) {
+  return reinterpret_cast<const uint4 *>(buf + r * kHeadDim) + (c ^ ((r >> 1) & 7));
+}
+
+__device__ __forceinline__ void a2_stage(bf16 *buf, const bf16 *__restrict__ src, int64_t ld, int h, int64_t t0,
+                                         int64_t T) {
+  for (int idx = threadIdx.x; idx < A2_ROWS * 16; idx += A2_THREADS) {
+    const int r = idx >> 4, c = idx & 15;
+    const int64_t tok = t0 - (kLeft - 1) + r;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (tok >= 0 && tok < T) v = __ldg(reinterpret_cast<const uint4 *>(src + tok * ld + h * kHeadDim) + c);
+    reinterpret_cast<uint4 *>(buf + r * kHeadDim)[c ^ ((r >> 1) & 7)] = v;
+  }
+}
+
+__global__ void __launch_bounds__(A2_THREADS, 3)
+    k_attention_bf16(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const bf16 *__restrict__ v, int64_t ld,
+                     const float *__restrict__ R, const float *__restrict__ qscale, float k_scale, float cap,
+                     const int32_t *__restrict__ pos, int64_t T, bf16 *__restrict__ out, int64_t ld_out, float lo,
+                     float hi) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  bf16 *buf = reinterpret_cast<bf16 *>(smem_raw);
+  float *Rt = reinterpret_cast<float *>(buf + A2_ROWS * kHeadDim);  // R / k_scale, [12][128]
+  float *Qs = Rt + kLeft * kHeadDim;                                // [128]
+  const int h = blockIdx.y;
+  const int64_t t0 = (int64_t)blockIdx.x * A2_TOK;
+  const int i = threadIdx.x;
+  const float inv_ks = 1.0f / k_scale;
+  for (int x = i; x < kLeft * kHeadDim; x += A2_THREADS)
+    Rt[x] = R[(x / kHeadDim) * kHidden + h * kHeadDim + x % kHeadDim] * inv_ks;
+  Qs[i] = qscale[i];
+  a2_stage(buf, k, ld, h, t0, T);
+  __syncthreads();
+
+  const int64_t ta = t0 + 2 * i, tb = ta + 1;
+  const bool va = ta < T, vb = tb < T;
+  const int64_t tqa = va ? ta : T - 1, tqb = vb ? tb : T - 1;  // clamped row for loads
+  const int spa = va ? min(pos[ta] + 1, kLeft) : 1;
+  const int spb = vb ? min(pos[tb] + 1, kLeft) : 1;
+  const bf16 *qa_row = q + tqa * ld + h * kHeadDim;
+  const bf16 *qb_row = q + tqb * ld + h * kHeadDim;
+
+  float2 acc[2][kLeft];
+#pragma unroll
+  for (int d = 0; d < kLeft; ++d) acc[0][d] = acc[1][d] = make_float2(0.f, 0.f);
+#pragma unroll 1
+  for (int cc = 0; cc < kHeadDim / 16; ++cc) {
+    float2 qa[8], qb[8];
+    {
+      const uint4 a0 = __ldg(reinterpret_cast<const uint4 *>(qa_row + cc * 16));
+      const uint4 a1 = __ldg(reinterpret_cast<const uint4 *>(qa_row + cc * 16) + 1);
+      const uint4 b0 = __ldg(reinterpret_cast<const uint4 *>(qb_row + cc * 16));
+      const uint4 b1 = __ldg(reinterpret_cast<const uint4 *>(qb_row + cc * 16) + 1);
+      const uint32_t wa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const uint32_t wb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      const float4 *qs4 = reinterpret_cast<const float4 *>(Qs + cc * 16);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const float4 s = qs4[m];
+        const float2 a_lo = bf2(wa[2 * m]), a_hi = bf2(wa[2 * m + 1]);
+        const float2 b_lo = bf2(wb[2 * m]), b_hi = bf2(wb[2 * m + 1]);
+        qa[2 * m] = make_float2(a_lo.x * s.x, a_lo.y * s.y);
+        qa[2 * m + 1] = make_float2(a_hi.x * s.z, a_hi.y * s.w);
+        qb[2 * m] = make_float2(b_lo.x * s.x, b_lo.y * s.y);
+        qb[2 * m + 1] = make_float2(b_hi.x * s.z, b_hi.y * s.w);
+      }
+    }
+    // key rows 2i .. 2i+12 (local): distance 11-j for query a, 12-j for query b
+#pragma unroll
+    for (int j = 0; j <= kLeft; ++j) {
+      const uint4 c0 = *a2_chunk(buf, 2 * i + j, 2 * cc), c1 = *a2_chunk(buf, 2 * i + j, 2 * cc + 1);
+      const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const float2 kk = bf2(w[m]);
+        if (j <= kLeft - 1) ffma2(acc[0][kLeft - 1 - j], qa[m], kk);
+        if (j >= 1) ffma2(acc[1][kLeft - j], qb[m], kk);
+      }
+    }
+#pragma unroll
+    for (int d = 0; d < kLeft; ++d) {
+      const float4 *r4 = reinterpret_cast<const float4 *>(Rt + d * kHeadDim + cc * 16);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const float4 r = r4[m];
+        ffma2(acc[0][d], qa[2 * m], make_float2(r.x, r.y));
+        ffma2(acc[0][d], qa[2 * m + 1], make_float2(r.z, r.w));
+        ffma2(acc[1][d], qb[2 * m], make_float2(r.x, r.y));
+        ffma2(acc[1][d], qb[2 * m + 1], make_float2(r.z, r.w));
+      }
+    }
+  }
+  // ---- capped logits and softmax per query
+  float p[2][kLeft];
+#pragma unroll
+  for (int qq = 0; qq < 2; ++qq) {
+    const int span = qq == 0 ? spa : spb;
+    float mx = -INFINITY;
+#pragma unroll
+    for (int d = 0; d < kLeft; ++d) {
+      const float z = cap * tanhf(k_scale * (acc[qq][d].x + acc[qq][d].y) / cap);
+      p[qq][d] = d < span ? z : -INFINITY;
+      mx = fmaxf(mx, p[qq][d]);
+    }
+    float den = 0.f;
+#pragma unroll
+    for (int d = 0; d < kLeft; ++d) {
+      p[qq][d] = d < span ? __expf(p[qq][d] - mx) : 0.f;
+      den += p[qq][d];
+    }
+    const float rd = 1.0f / den;
+#pragma unroll
+    for (int d = 0; d < kLeft; ++d) p[qq][d] *= rd;
+  }
+  __syncthreads();  // everyone is done with the k rows
+  a2_stage(buf, v, ld, h, t0, T);
+  __syncthreads();
+  // ---- o = sum_d p_d v_{t-d}
+  bf16 *oa_row = out + tqa * ld_out + h * kHeadDim;
+  bf16 *ob_row = out + tqb * ld_out + h * kHeadDim;
+#pragma unroll 1
+  for (int cc = 0; cc < kHeadDim / 16; ++cc) {
+    float2 oa[8], ob[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) oa[m] = ob[m] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j <= kLeft; ++j) {
+      const uint4 c0 = *a2_chunk(buf, 2 * i + j, 2 * cc), c1 = *a2_chunk(buf, 2 * i + j, 2 * cc + 1);
+      const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+      const float pa = j <= kLeft - 1 ? p[0][kLeft - 1 - j] : 0.f;
+      const float pb = j >= 1 ? p[1][kLeft - j] : 0.f;
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const float2 vv = bf2(w[m]);
+        if (j <= kLeft - 1) ffma2(oa[m], make_float2(pa, pa), vv);
+        if (j >= 1) ffma2(ob[m], make_float2(pb, pb), vv);
+      }
+    }
+    uint32_t wa[8], wb[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      wa[m] = pack_bf16(clampf(oa[m].x, lo, hi), clampf(oa[m].y, lo, hi));
+      wb[m] = pack_bf16(clampf(ob[m].x, lo, hi), clampf(ob[m].y, lo, hi));
+    }
+    if (va) {
+      reinterpret_cast<uint4 *>(oa_row + cc * 16)[0] = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+      reinterpret_cast<uint4 *>(oa_row + cc * 16)[1] = make_uint4(wa[4], wa[5], wa[6], wa[7]);
+    }
+    if (vb) {
+      reinterpret_cast<uint4 *>(ob_row + cc * 16)[0] = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+      reinterpret_cast<uint4 *>(ob_row + cc * 16)[1] = make_uint4(wb[4], wb[5], wb[6], wb[7]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ float32 kernel
+
 namespace {
 constexpr int kTQ = 128;                 // queries per CTA
 constexpr int kRows = kTQ + kLeft - 1;   // staged k/v rows
+constexpr int kPitchF = kHeadDim + 4;    // floats per staged row (528 bytes)
 }  // namespace
 
-template <typename T> struct AttnIO;
-template <> struct AttnIO<bf16> {
-  static constexpr int kPitch = kHeadDim + 8;  // elements per staged row (272 bytes)
-  static constexpr int kChunks = kHeadDim * 2 / 16;
-  // 16 consecutive values at p (32-byte aligned) as float
-  static __device__ __forceinline__ void load16(const bf16 *p, float (&v)[16]) {
-    const uint4 a = reinterpret_cast<const uint4 *>(p)[0], b = reinterpret_cast<const uint4 *>(p)[1];
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      v[2 * i] = bf16lo(w[i]);
-      v[2 * i + 1] = bf16hi(w[i]);
-    }
-  }
-  static __device__ __forceinline__ void store16(bf16 *p, const float (&v)[16]) {
-    uint32_t w[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = pack_bf16(v[2 * i], v[2 * i + 1]);
-    reinterpret_cast<uint4 *>(p)[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    reinterpret_cast<uint4 *>(p)[1] = make_uint4(w[4], w[5], w[6], w[7]);
-  }
-};
-template <> struct AttnIO<float> {
-  static constexpr int kPitch = kHeadDim + 4;  // 528 bytes
-  static constexpr int kChunks = kHeadDim * 4 / 16;
-  static __device__ __forceinline__ void load16(const float *p, float (&v)[16]) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float4 x = reinterpret_cast<const float4 *>(p)[i];
-      v[4 * i] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z; v[4 * i + 3] = x.w;
-    }
-  }
-  static __device__ __forceinline__ void store16(float *p, const float (&v)[16]) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      reinterpret_cast<float4 *>(p)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-  }
-};
-
-template <typename T>
-__global__ void __launch_bounds__(kTQ) k_attention(const T *__restrict__ q, const T *__restrict__ k,
-                                                   const T *__restrict__ v, int64_t ld, const float *__restrict__ R,
-                                                   const float *__restrict__ qscale, float k_scale, float cap,
-                                                   const int32_t *__restrict__ pos, int64_t T_total,
-                                                   T *__restrict__ out, int64_t ld_out, float lo, float hi) {
-  using IO = AttnIO<T>;
-  extern __shared__ uint8_t smem_raw[];
-  T *Ks = reinterpret_cast<T *>(smem_raw);
-  T *Vs = Ks + kRows * IO::kPitch;
-  float *Rs = reinterpret_cast<float *>(Vs + kRows * IO::kPitch);  // [12][128]
-  float *Qs = Rs + kLeft * kHeadDim;                                // [128]
-
+__global__ void __launch_bounds__(kTQ) k_attention_f32(const float *__restrict__ q, const float *__restrict__ k,
+                                                       const float *__restrict__ v, int64_t ld,
+                                                       const float *__restrict__ R, const float *__restrict__ qscale,
+                                                       float k_scale, float cap, const int32_t *__restrict__ pos,
+                                                       int64_t T_total, float *__restrict__ out, int64_t ld_out,
+                                                       float lo, float hi) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  float *Ks = reinterpret_cast<float *>(smem_raw);
+  float *Vs = Ks + kRows * kPitchF;
+  float *Rs = Vs + kRows * kPitchF;  // [12][128]
+  float *Qs = Rs + kLeft * kHeadDim;  // [128]
   const int h = blockIdx.y;
   const int64_t t0 = (int64_t)blockIdx.x * kTQ;
   const int tid = threadIdx.x;
-
-  // ---- stage k, v rows t0-11 .. t0+127 of head h (zero outside [0, T))
-  for (int idx = tid; idx < kRows * IO::kChunks; idx += kTQ) {
-    const int r = idx / IO::kChunks, ch = idx % IO::kChunks;
+  for (int idx = tid; idx < kRows * (kHeadDim / 4); idx += kTQ) {
+    const int r = idx / (kHeadDim / 4), ch = idx % (kHeadDim / 4);
     const int64_t tok = t0 - (kLeft - 1) + r;
-    uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
+    float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), vv = kv;
     if (tok >= 0 && tok < T_total) {
-      kv = *reinterpret_cast<const uint4 *>(k + tok * ld + h * kHeadDim + ch * (16 / sizeof(T)));
-      vv = *reinterpret_cast<const uint4 *>(v + tok * ld + h * kHeadDim + ch * (16 / sizeof(T)));
+      kv = *reinterpret_cast<const float4 *>(k + tok * ld + h * kHeadDim + ch * 4);
+      vv = *reinterpret_cast<const float4 *>(v + tok * ld + h * kHeadDim + ch * 4);
     }
-    *reinterpret_cast<uint4 *>(Ks + r * IO::kPitch + ch * (16 / sizeof(T))) = kv;
-    *reinterpret_cast<uint4 *>(Vs + r * IO::kPitch + ch * (16 / sizeof(T))) = vv;
+    *reinterpret_cast<float4 *>(Ks + r * kPitchF + ch * 4) = kv;
+    *reinterpret_cast<float4 *>(Vs + r * kPitchF + ch * 4) = vv;
   }
-  for (int i = tid; i < kLeft * kHeadDim; i += kTQ) Rs[i] = R[(i / kHeadDim) * kHidden + h * kHeadDim + i % kHeadDim];
+  for (int x = tid; x < kLeft * kHeadDim; x += kTQ) Rs[x] = R[(x / kHeadDim) * kHidden + h * kHeadDim + x % kHeadDim];
   Qs[tid] = qscale[tid];
   __syncthreads();
-
   const int64_t t = t0 + tid;
   if (t >= T_total) return;
   const int span = min(pos[t] + 1, kLeft);
-  const T *qrow = q + t * ld + h * kHeadDim;
-
+  const float *qrow = q + t * ld + h * kHeadDim;
   float d1[kLeft], d2[kLeft];
 #pragma unroll
   for (int d = 0; d < kLeft; ++d) d1[d] = d2[d] = 0.f;
 #pragma unroll 1
-  for (int c = 0; c < kHeadDim / 16; ++c) {
-    float qv[16];
-    IO::load16(qrow + c * 16, qv);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) qv[i] *= Qs[c * 16 + i];
+  for (int c = 0; c < kHeadDim / 4; ++c) {
+    const float4 q4 = *reinterpret_cast<const float4 *>(qrow + c * 4);
+    const float qv[4] = {q4.x * Qs[c * 4], q4.y * Qs[c * 4 + 1], q4.z * Qs[c * 4 + 2], q4.w * Qs[c * 4 + 3]};
 #pragma unroll
     for (int d = 0; d < kLeft; ++d) {
-      float kk[16];
-      IO::load16(Ks + (tid + kLeft - 1 - d) * IO::kPitch + c * 16, kk);
-      const float *rr = Rs + d * kHeadDim + c * 16;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        d1[d] = fmaf(qv[i], kk[i], d1[d]);
-        d2[d] = fmaf(qv[i], rr[i], d2[d]);
-      }
+      const float4 kk = *reinterpret_cast<const float4 *>(Ks + (tid + kLeft - 1 - d) * kPitchF + c * 4);
+      const float4 rr = *reinterpret_cast<const float4 *>(Rs + d * kHeadDim + c * 4);
+      d1[d] = fmaf(qv[0], kk.x, fmaf(qv[1], kk.y, fmaf(qv[2], kk.z, fmaf(qv[3], kk.w, d1[d]))));
+      d2[d] = fmaf(qv[0], rr.x, fmaf(qv[1], rr.y, fmaf(qv[2], rr.z, fmaf(qv[3], rr.w, d2[d]))));
     }
   }
-  // ---- capped logits, softmax over the distances inside the clip
   float p[kLeft];
   float mx = -INFINITY;
 #pragma unroll
@@ -138,52 +270,53 @@ __global__ void __launch_bounds__(kTQ) k_attention(const T *__restrict__ q, cons
     den += p[d];
   }
   const float rden = 1.0f / den;
-#pragma unroll
-  for (int d = 0; d < kLeft; ++d) p[d] *= rden;
-  // ---- o = sum_d p_d v_{t-d}, clamped, chunk by chunk
-  T *orow = out + t * ld_out + h * kHeadDim;
+  float *orow = out + t * ld_out + h * kHeadDim;
 #pragma unroll 1
-  for (int c = 0; c < kHeadDim / 16; ++c) {
-    float o[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) o[i] = 0.f;
+  for (int c = 0; c < kHeadDim / 4; ++c) {
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int d = 0; d < kLeft; ++d) {
-      float vv[16];
-      IO::load16(Vs + (tid + kLeft - 1 - d) * IO::kPitch + c * 16, vv);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) o[i] = fmaf(p[d], vv[i], o[i]);
+      const float4 vv = *reinterpret_cast<const float4 *>(Vs + (tid + kLeft - 1 - d) * kPitchF + c * 4);
+      const float w = p[d] * rden;
+      o.x = fmaf(w, vv.x, o.x);
+      o.y = fmaf(w, vv.y, o.y);
+      o.z = fmaf(w, vv.z, o.z);
+      o.w = fmaf(w, vv.w, o.w);
     }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) o[i] = clampf(o[i], lo, hi);
-    IO::store16(orow + c * 16, o);
+    *reinterpret_cast<float4 *>(orow + c * 4) =
+        make_float4(clampf(o.x, lo, hi), clampf(o.y, lo, hi), clampf(o.z, lo, hi), clampf(o.w, lo, hi));
   }
-}
-
-template <typename T>
-static cudaError_t attn_launch(const void *q, const void *k, const void *v, int64_t ld, const float *R,
-                               const float *qscale, float k_scale, float cap, const int32_t *pos, int64_t n_tok,
-                               void *out, int64_t ld_out, float lo, float hi, cudaStream_t s) {
-  const size_t smem = 2 * kRows * AttnIO<T>::kPitch * sizeof(T) + (kLeft * kHeadDim + kHeadDim) * sizeof(float);
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_attention<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
-  dim3 grid((unsigned)((n_tok + kTQ - 1) / kTQ), kHeads);
-  k_attention<T><<<grid, kTQ, smem, s>>>(static_cast<const T *>(q), static_cast<const T *>(k),
-                                         static_cast<const T *>(v), ld, R, qscale, k_scale, cap, pos, n_tok,
-                                         static_cast<T *>(out), ld_out, lo, hi);
-  return cudaGetLastError();
 }
 
 cudaError_t launch_attention(bool is_bf16, const void *q, const void *k, const void *v, int64_t ld, const float *R,
                              const float *qscale, float k_scale, float cap, const int32_t *pos, int64_t T, void *out,
                              int64_t ld_out, float lo, float hi, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  if (is_bf16) return attn_launch<bf16>(q, k, v, ld, R, qscale, k_scale, cap, pos, T, out, ld_out, lo, hi, s);
-  return attn_launch<float>(q, k, v, ld, R, qscale, k_scale, cap, pos, T, out, ld_out, lo, hi, s);
+  if (is_bf16) {
+    static bool attr = false;
+    if (!attr) {
+      cudaError_t e = cudaFuncSetAttribute(k_attention_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)A2_SMEM);
+      if (e != cudaSuccess) return e;
+      attr = true;
+    }
+    dim3 grid((unsigned)((T + A2_TOK - 1) / A2_TOK), kHeads);
+    k_attention_bf16<<<grid, A2_THREADS, A2_SMEM, s>>>(static_cast<const bf16 *>(q), static_cast<const bf16 *>(k),
+                                                       static_cast<const bf16 *>(v), ld, R, qscale, k_scale, cap, pos,
+                                                       T, static_cast<bf16 *>(out), ld_out, lo, hi);
+    return cudaGetLastError();
+  }
+  const size_t smem = (2 * (size_t)kRows * kPitchF + kLeft * kHeadDim + kHeadDim) * sizeof(float);
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_attention_f32, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  dim3 grid((unsigned)((T + kTQ - 1) / kTQ), kHeads);
+  k_attention_f32<<<grid, kTQ, smem, s>>>(static_cast<const float *>(q), static_cast<const float *>(k),
+                                          static_cast<const float *>(v), ld, R, qscale, k_scale, cap, pos, T,
+                                          static_cast<float *>(out), ld_out, lo, hi);
+  return cudaGetLastError();
 }
 
 }  // namespace ae

@@ -1,15 +1,19 @@
 // Projections of the tower: y = epilogue(x W^T) with x [M][K] (packed token
 // rows, M ragged) and W [N][K] (the checkpoint's [out][in] layout).
 //
-// bf16 path: a persistent, warp-specialised tcgen05 kernel. Warp 0 streams
-// 128x64 tiles of x and 256x64 tiles of W into a 4-stage shared-memory ring
-// with TMA (128-byte swizzle, no multicast); warp 1 allocates 512 columns of
-// tensor memory and issues tcgen05.mma (M=128, N=256, K=16, bf16 in, f32
-// accumulate) into one of two 256-column accumulators; warps 2-5 read the
-// other accumulator with tcgen05.ld, apply the epilogue (ClipLin output
-// clamp, SiLU and the next projection's input clamp, GLU, or bias) and store.
-// Tiles are walked m-major so the CTAs in flight share rows of x in L2 while
-// W stays L2-resident.
+// bf16 path: a persistent tcgen05 kernel on CTA pairs (clusters of two SMs),
+// warp-specialised. Per 64-wide k-block, each CTA's warp 0 streams its half
+// of the pair tile (128 rows of x, 128 rows of W) into a 6-stage shared-memory
+// ring with TMA (128-byte swizzle, no multicast); the leader CTA's warp 1
+// issues tcgen05.mma.cta_group::2 (M=256, N=256, K=16, bf16 in, f32
+// accumulate), which reads the operand halves from both SMs, into one of two
+// 256-column accumulators in each CTA's tensor memory; warps 2-9 of each CTA
+// drain the other accumulator with tcgen05.ld and apply the epilogue
+// (ClipLin output clamp, SiLU and the next projection's input clamp, GLU, or
+// bias). Pairing halves the W bytes each SM stages per flop, which keeps the
+// shared-memory traffic (TMA writes plus tensor-core reads) under the SM's
+// bandwidth. Tiles are walked m-major so the pairs in flight share rows of x
+// in L2 while W stays L2-resident.
 //
 // f32 path: a plain 64x64-tile FMA kernel with the same epilogues.
 #include <cudaTypedefs.h>
@@ -40,9 +44,9 @@ template <int MODE>
 __device__ __forceinline__ void epi_store_tc(const EpiArgs &ep, int row, int col, const uint32_t (&r)[32]) {
   float lo = ep.lo, hi = ep.hi;
   if (ep.seg_w > 0) {
-    const int sg = col / ep.seg_w;
-    lo = ep.seg_lo[sg];
-    hi = ep.seg_hi[sg];
+    const int sg = col / ep.seg_w;  // selects, not a runtime index into the parameter array
+    lo = sg == 0 ? ep.seg_lo[0] : (sg == 1 ? ep.seg_lo[1] : ep.seg_lo[2]);
+    hi = sg == 0 ? ep.seg_hi[0] : (sg == 1 ? ep.seg_hi[1] : ep.seg_hi[2]);
   }
   float v[32];
 #pragma unroll
@@ -58,12 +62,14 @@ __device__ __forceinline__ void epi_store_tc(const EpiArgs &ep, int row, int col
 #pragma unroll
     for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4 *>(o + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
   } else if (MODE == EPI_GLU) {
+    // a * sigmoid(b) = a / (1 + e^-b): fast exp and reciprocal (2 ulp each; the
+    // bf16 rounding of the result is 2^-9), with the right limits at +-inf
     uint32_t p[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       float a0 = clampf(v[4 * j + 0], lo, hi), b0 = clampf(v[4 * j + 1], lo, hi);
       float a1 = clampf(v[4 * j + 2], lo, hi), b1 = clampf(v[4 * j + 3], lo, hi);
-      p[j] = pack_bf16(a0 / (1.0f + __expf(-b0)), a1 / (1.0f + __expf(-b1)));
+      p[j] = pack_bf16(__fdividef(a0, 1.0f + __expf(-b0)), __fdividef(a1, 1.0f + __expf(-b1)));
     }
     bf16 *o = static_cast<bf16 *>(ep.out) + (int64_t)row * ep.ld + col / 2;
     reinterpret_cast<uint4 *>(o)[0] = make_uint4(p[0], p[1], p[2], p[3]);
@@ -72,7 +78,7 @@ __device__ __forceinline__ void epi_store_tc(const EpiArgs &ep, int row, int col
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       float x = clampf(v[i], lo, hi);
-      if (MODE == EPI_SILU) x = clampf(x / (1.0f + __expf(-x)), ep.lo2, ep.hi2);
+      if (MODE == EPI_SILU) x = clampf(__fdividef(x, 1.0f + __expf(-x)), ep.lo2, ep.hi2);
       v[i] = x;
     }
     uint32_t p[16];
@@ -84,32 +90,46 @@ __device__ __forceinline__ void epi_store_tc(const EpiArgs &ep, int row, int col
   }
 }
 
-// ------------------------------------------------------------------ tcgen05 kernel
+// ------------------------------------------------------------------ tcgen05 pair kernel
 
 namespace {
-constexpr int BM = 128, BK = 64, BN = 256, STAGES = 4;
-constexpr uint32_t A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr int BM = 128;                 // rows of x per CTA (256 per pair)
+constexpr int BK = 64;                  // one 128-byte swizzle atom of bf16
+constexpr int BN = 256;                 // columns per pair tile (128 rows of W per CTA)
+constexpr int STAGES = 6;
+constexpr uint32_t A_BYTES = BM * BK * 2, B_BYTES = (BN / 2) * BK * 2, STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr uint32_t TMEM_COLS = 2 * BN;  // two 128 x 256 f32 accumulators per CTA
+constexpr int EPI_WARPS = 8;
+constexpr int GEMM_THREADS = 64 + 32 * EPI_WARPS;
 constexpr size_t SMEM_TC = STAGES * STAGE_BYTES + 1024 + 256;
 }  // namespace
 
+// Persistent pair kernel (cluster of 2 CTAs on 2 SMs). Pair tile 256 x 256:
+// CTA r of the pair loads rows [m0 + 128 r, +128) of x and rows
+// [n0 + 128 r, +128) of W for every 64-wide k-block; the leader (even) CTA
+// issues tcgen05.mma.cta_group::2 (M=256, N=256, K=16), which reads the A and
+// B halves from both CTAs' shared memory and accumulates rows 128 r .. +127
+// in CTA r's tensor memory. Each CTA's epilogue drains its own 128 rows.
 template <int MODE>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const EpiArgs ep,
               const int M, const int N, const int K, unsigned *status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
-  uint64_t *empty = full + STAGES;
-  uint64_t *tfull = empty + STAGES;
-  uint64_t *tempty = tfull + 2;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);  // used in the leader
+  uint64_t *empty = full + STAGES;                                              // per CTA
+  uint64_t *tfull = empty + STAGES;                                             // per CTA
+  uint64_t *tempty = tfull + 2;                                                 // used in the leader
   uint64_t *done = tempty + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m_blocks = (M + BM - 1) / BM, n_blocks = N / BN, kb_n = K / BK;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int m_blocks = (M + 2 * BM - 1) / (2 * BM), n_blocks = N / BN, kb_n = K / BK;
   const int num_tiles = m_blocks * n_blocks;
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -118,7 +138,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 128);
+      mbar_init(&tempty[i], 2 * EPI_WARPS);  // one arrival per epilogue warp of both CTAs
     }
     mbar_init(done, 1);
     *abort_flag = 0;
@@ -127,31 +147,32 @@ __global__ void __launch_bounds__(192, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // both CTAs' barriers are initialised before any cross-CTA arrival
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0 && lane == 0) {
-    // ---------------- TMA producer
+    // ---------------- TMA producer (both CTAs)
     int stage = 0;
     uint32_t phase = 0;
     long issued = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+    for (int tile = pair; tile < num_tiles && ok; tile += n_pairs) {
       const int mb = tile / n_blocks, nb = tile % n_blocks;
+      const int arow = mb * 2 * BM + (int)rank * BM, brow = nb * BN + (int)rank * (BN / 2);
       for (int kb = 0; kb < kb_n; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1) || *abort_flag) {
           ok = false;
           break;
         }
         uint8_t *sa = smem + stage * STAGE_BYTES;
-        mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-        tma_load_2d(sa, &tmA, kb * BK, mb * BM, &full[stage]);
-        tma_load_2d(sa + A_BYTES, &tmB, kb * BK, nb * BN, &full[stage]);
+        if (leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
+        tma_load_2d_pair(sa, &tmA, kb * BK, arow, &full[stage]);
+        tma_load_2d_pair(sa + A_BYTES, &tmB, kb * BK, brow, &full[stage]);
         ++issued;
         if (++stage == STAGES) {
           stage = 0;
@@ -163,18 +184,19 @@ __global__ void __launch_bounds__(192, 1)
       atomicOr(status, kStatusWaitTimeout);
       *abort_flag = 1;
     }
-    // every load issued must land before the CTA may exit
-    for (int s = 0; s < STAGES; ++s) {
-      const long n = issued / STAGES + (s < issued % STAGES ? 1 : 0);
-      if (n > 0) mbar_wait(&full[s], (uint32_t)((n - 1) & 1));
+    if (leader) {  // every load issued by the pair must land before the leader may exit
+      for (int s = 0; s < STAGES; ++s) {
+        const long n = issued / STAGES + (s < issued % STAGES ? 1 : 0);
+        if (n > 0) mbar_wait(&full[s], (uint32_t)((n - 1) & 1));
+      }
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer
-    constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+  } else if (warp == 1 && lane == 0 && leader) {
+    // ---------------- MMA issuer (leader CTA only)
+    constexpr uint32_t idesc = idesc_bf16_f32(2 * BM, BN);
     int stage = 0, acc = 0;
     uint32_t phase = 0, acc_phase = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+    for (int tile = pair; tile < num_tiles && ok; tile += n_pairs) {
       if (!mbar_wait(&tempty[acc], acc_phase ^ 1) || *abort_flag) {
         ok = false;
         break;
@@ -191,15 +213,15 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t sb = sa + A_BYTES;
 #pragma unroll
         for (int k = 0; k < BK / 16; ++k)
-          tc_mma_bf16(d_tmem, sw128_desc(sa + k * 32), sw128_desc(sb + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
-        tc_commit(&empty[stage]);
+          tc_mma_bf16_pair(d_tmem, sw128_desc(sa + k * 32), sw128_desc(sb + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
+        tc_commit_pair_both(&empty[stage]);  // frees the stage in both CTAs
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1;
         }
       }
       if (!ok) break;
-      tc_commit(&tfull[acc]);
+      tc_commit_pair_both(&tfull[acc]);  // accumulator ready in both CTAs
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
@@ -209,15 +231,18 @@ __global__ void __launch_bounds__(192, 1)
       atomicOr(status, kStatusWaitTimeout);
       *abort_flag = 1;
     }
-    tc_commit(done);  // arrives once every MMA issued above has completed
+    tc_commit_pair_local(done);  // arrives once every MMA issued above has completed
     mbar_wait(done, 0);
   } else if (warp >= 2) {
-    // ---------------- epilogue: warp w reads TMEM lanes 32*(w%4) .. +31
+    // ---------------- epilogue (both CTAs): warp w reads TMEM lanes 32*(w%4) .. +31;
+    // the two warps of a lane quarter split the tile's columns
     const int q = warp & 3;
+    const int c0 = ((warp - 2) >> 2) * (BN / 64);
+    const uint32_t tempty_leader = map_to_rank(&tempty[0], 0);
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    for (int tile = pair; tile < num_tiles; tile += n_pairs) {
       const int mb = tile / n_blocks, nb = tile % n_blocks;
       const bool got = mbar_wait(&tfull[acc], acc_phase);
       if (!__all_sync(0xffffffffu, got)) {
@@ -225,16 +250,24 @@ __global__ void __launch_bounds__(192, 1)
         break;
       }
       tc_fence_after();
-      const int row = mb * BM + q * 32 + lane;
+      const int row = mb * 2 * BM + (int)rank * BM + q * 32 + lane;
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      // two register buffers: the next chunk's tcgen05.ld is in flight during the math
+      uint32_t ra[32], rb[32];
+      tmem_ld32(tbase + c0 * 32, ra);
+      tmem_ld_wait();
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c * 32), r);
+      for (int c = 0; c < BN / 64; c += 2) {
+        tmem_ld32(tbase + (c0 + c + 1) * 32, rb);
+        if (row < M) epi_store_tc<MODE>(ep, row, nb * BN + (c0 + c) * 32, ra);
         tmem_ld_wait();
-        if (row < M) epi_store_tc<MODE>(ep, row, nb * BN + c * 32, r);
+        if (c + 2 < BN / 64) tmem_ld32(tbase + (c0 + c + 2) * 32, ra);
+        if (row < M) epi_store_tc<MODE>(ep, row, nb * BN + (c0 + c + 1) * 32, rb);
+        tmem_ld_wait();
       }
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader + (uint32_t)(acc * sizeof(uint64_t)));
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
@@ -245,10 +278,12 @@ __global__ void __launch_bounds__(192, 1)
       *abort_flag = 1;
     }
   }
+  tc_fence_before();
   __syncthreads();
+  cluster_sync();  // no CTA of the pair leaves while the other may still touch it
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 
@@ -287,9 +322,9 @@ __global__ void __launch_bounds__(256) k_gemm_f32(const float *__restrict__ A, c
   const int col = n0 + tx * 4;
   float lo = ep.lo, hi = ep.hi;
   if (ep.seg_w > 0) {
-    const int sg = col / ep.seg_w;
-    lo = ep.seg_lo[sg];
-    hi = ep.seg_hi[sg];
+    const int sg = col / ep.seg_w;  // selects, not a runtime index into the parameter array
+    lo = sg == 0 ? ep.seg_lo[0] : (sg == 1 ? ep.seg_lo[1] : ep.seg_lo[2]);
+    hi = sg == 0 ? ep.seg_hi[0] : (sg == 1 ? ep.seg_hi[1] : ep.seg_hi[2]);
   }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -374,9 +409,9 @@ static cudaError_t launch_tc(const CUtensorMap &tA, const CUtensorMap &tB, const
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  const int tiles = ((M + BM - 1) / BM) * (N / BN);
-  const int grid = tiles < num_sms() ? tiles : num_sms();
-  k_gemm_tc<MODE><<<grid, 192, SMEM_TC, s>>>(tA, tB, ep, M, N, K, device_status_word());
+  const int tiles = ((M + 2 * BM - 1) / (2 * BM)) * (N / BN);
+  const int pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;
+  k_gemm_tc<MODE><<<2 * pairs, GEMM_THREADS, SMEM_TC, s>>>(tA, tB, ep, M, N, K, device_status_word());
   return cudaGetLastError();
 }
 
@@ -395,7 +430,7 @@ cudaError_t gemm(const ae_model *m, const void *x, int64_t M, int K, const void 
     CUtensorMap tA, tB;
     if (!make_tmap_2d_bf16(&tA, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK, BM)) return cudaErrorInvalidValue;
     if (!tmW) {
-      if (!make_tmap_2d_bf16(&tB, w, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, BK, BN))
+      if (!make_tmap_2d_bf16(&tB, w, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, BK, BN / 2))
         return cudaErrorInvalidValue;
       tmW = &tB;
     }

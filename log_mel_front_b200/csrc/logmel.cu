@@ -27,17 +27,17 @@ namespace {
 constexpr int kGroups = 16;                        // frames in flight per CTA
 constexpr int kThreads = kGroups * 16;             // 256
 constexpr int kWaveSpan = kMelTile * kHop + kHop;  // samples staged per work item
-constexpr int kMaxBins = 16;                       // bins per band (11 suffice)
+constexpr int kMaxBins = 12;                       // bins per band (11 suffice), zero-padded
 constexpr int kPitch = 17;                         // padded row of the 16 x 16 transpose
 
 struct LogmelSmem {
   float2 tw[kFft];                         // W512^m = (cos, -sin)(2 pi m / 512)
   float win[kFrame];                       // Hann / 2 (the split's 1/2 folded in)
-  float wts[kMels][kMaxBins + 1];          // sparse mel bank (rows padded against bank conflicts)
-  int band_lo[kMels], band_n[kMels];
+  float wts[kMels][kMaxBins + 1];          // sparse mel bank, zero-padded (row pitch 13 against bank conflicts)
+  int band_lo[kMels];
   float wave[kWaveSpan];
   float2 xs[kGroups][kPitch * 16];         // per-group transpose / spectrum exchange
-  float mag[kGroups][kFft / 2 + 1];        // per-group magnitudes
+  float mag[kGroups][kFft / 2 + 16];       // per-group magnitudes (zero tail for the padded mel loop)
   int tile_clip, tile_f0, tile_nf;
 };
 }  // namespace
@@ -97,7 +97,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
   for (int j = tid; j < kFrame; j += kThreads) S.win[j] = (float)(0.25 - 0.25 * cospi((double)j / 160.0));
   if (tid < kMels) {
-    // HTK: 130 mel points over [mel(0), mel(8000)] (last point exact), bins at k * 31.25 Hz
+    // HTK: 130 mel points over [mel(0), mel(8000)] (last point exact), bins at k * 31.25 Hz;
+    // band b is the triangle over [f_b, f_b+2]; only the bins inside it are visited
     const double mel_hi = 2595.0 * log10(1.0 + 8000.0 / 700.0);
     const double step = mel_hi / 129.0;
     double f[3];
@@ -106,8 +107,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       const double mm = (p == 129) ? mel_hi : p * step;
       f[i] = 700.0 * (pow(10.0, mm / 2595.0) - 1.0);
     }
+    for (int q = 0; q < kMaxBins; ++q) S.wts[tid][q] = 0.f;
     int lo = -1, n = 0;
-    for (int k = 0; k <= kFft / 2; ++k) {
+    const int k0 = max(0, (int)floor(f[0] / 31.25)), k1 = min(kFft / 2, (int)ceil(f[2] / 31.25));
+    for (int k = k0; k <= k1; ++k) {
       const double fk = k * 31.25;
       const double down = (fk - f[0]) / (f[1] - f[0]);
       const double up = (f[2] - fk) / (f[2] - f[1]);
@@ -118,8 +121,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
     S.band_lo[tid] = lo < 0 ? 0 : lo;
-    S.band_n[tid] = n;
   }
+  for (int x = tid; x < kGroups * 16; x += kThreads) S.mag[x / 16][kFft / 2 + x % 16] = 0.f;
 
   __syncthreads();
   const int g = tid >> 4, j = tid & 15;
@@ -164,7 +167,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int n1 = 0; n1 < 16; ++n1) {
         if (n1 < 10) {
           const int m = 32 * n1 + 2 * j;
-          x[n1] = make_float2(wv[m] * S.win[m], wv[m + 1] * S.win[m + 1]);
+          const float2 a = *reinterpret_cast<const float2 *>(wv + m);
+          const float2 w = *reinterpret_cast<const float2 *>(S.win + m);
+          x[n1] = make_float2(a.x * w.x, a.y * w.y);
         } else {
           x[n1] = make_float2(0.f, 0.f);
         }
@@ -202,7 +207,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         const float wbr = fmaf(w.x, B.x, -w.y * B.y);
         const float wbi = fmaf(w.x, B.y, w.y * B.x);
         const float re = A.x + wbi, im = A.y - wbr;
-        mag[k] = sqrtf(fmaf(re, re, im * im));
+        const float m2 = fmaf(re, re, im * im);
+        mag[k] = m2 * rsqrtf(fmaxf(m2, 1e-37f));  // |X| (2 ulp), 0 for 0
         if (k == 0) mag[kFft / 2] = fabsf(2.0f * (a.x - a.y));  // Nyquist: Re Z0 - Im Z0 (Z halved)
       }
       __syncwarp(gmask);
@@ -211,9 +217,10 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
       for (int i = 0; i < kMels / 16; ++i) {
         const int b = j + 16 * i;
-        const int lo = S.band_lo[b], n = S.band_n[b];
+        const float *mg = mag + S.band_lo[b];
         float acc = 0.f;
-        for (int q = 0; q < n; ++q) acc = fmaf(S.wts[b][q], mag[lo + q], acc);
+#pragma unroll
+        for (int q = 0; q < kMaxBins; ++q) acc = fmaf(S.wts[b][q], mg[q], acc);
         orow[b] = logf(acc + 1e-3f);
       }
       __syncwarp(gmask);

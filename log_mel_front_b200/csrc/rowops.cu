@@ -122,19 +122,36 @@ cudaError_t launch_rowop(const ae_model *m, const RowArgs &r, cudaStream_t s) {
 
 // ------------------------------------------------------------------ light conv middle
 
-// w_dw is stored tap-major [kernel][hidden]. A warp walks kRowsPerWarp
-// consecutive rows; lane l owns channels (i * 32 + l) * 4 .. +3.
-constexpr int kRowsPerWarp = 4;
+// w_dw is stored tap-major [kernel][hidden] (20 KB, read through L1). A CTA
+// owns kLcRows consecutive rows: it stages those rows plus the 4 before them
+// in shared memory with coalesced 16-byte loads; each warp then computes
+// kLcRows / 8 rows, lane l owning channels (i * 32 + l) * 4 .. +3.
+constexpr int kLcRows = 16;
+constexpr int kLcHalo = kKernel - 1;
 
 template <typename ActT>
 __global__ void __launch_bounds__(256) k_lconv(const ActT *__restrict__ gl, const float *__restrict__ w_dw,
                                                const float *__restrict__ w_norm, float lo, float hi,
                                                ActT *__restrict__ out, const int32_t *__restrict__ pos, int64_t T) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const float *s_w = w_dw;
+  ActT *s_x = reinterpret_cast<ActT *>(smem_raw);                        // [kLcRows + halo][hidden]
   const int lane = threadIdx.x & 31;
-  const int64_t row0 = ((int64_t)blockIdx.x * 8 + (threadIdx.x >> 5)) * kRowsPerWarp;
+  const int64_t t0 = (int64_t)blockIdx.x * kLcRows;
+  constexpr int VEC = 16 / sizeof(ActT);                                 // elements per 16-byte load
+  constexpr int ROW_V = kHidden / VEC;
+  for (int i = threadIdx.x; i < (kLcRows + kLcHalo) * ROW_V; i += blockDim.x) {
+    const int r = i / ROW_V, cv = i % ROW_V;
+    const int64_t tok = t0 - kLcHalo + r;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (tok >= 0 && tok < T) v = __ldg(reinterpret_cast<const uint4 *>(gl + tok * kHidden) + cv);
+    reinterpret_cast<uint4 *>(s_x + (int64_t)r * kHidden)[cv] = v;
+  }
+  __syncthreads();
   constexpr int NV = kHidden / 128;
-  for (int rr = 0; rr < kRowsPerWarp; ++rr) {
-    const int64_t t = row0 + rr;
+  for (int rr = 0; rr < kLcRows / 8; ++rr) {
+    const int lr = (threadIdx.x >> 5) * (kLcRows / 8) + rr;  // local output row
+    const int64_t t = t0 + lr;
     if (t >= T) return;
     const int p = pos[t];
     float c[NV][4];
@@ -146,12 +163,12 @@ __global__ void __launch_bounds__(256) k_lconv(const ActT *__restrict__ gl, cons
     for (int k = 0; k < kKernel; ++k) {
       const int back = kKernel - 1 - k;
       if (back > p) continue;
-      const ActT *src = gl + (t - back) * kHidden;
+      const ActT *src = s_x + (int64_t)(lr + kLcHalo - back) * kHidden;
 #pragma unroll
       for (int i = 0; i < NV; ++i) {
         float x[4], w[4];
         load4(src + (i * 32 + lane) * 4, x);
-        load4(w_dw + k * kHidden + (i * 32 + lane) * 4, w);
+        load4(s_w + k * kHidden + (i * 32 + lane) * 4, w);
 #pragma unroll
         for (int u = 0; u < 4; ++u) c[i][u] = fmaf(w[u], x[u], c[i][u]);
       }
@@ -180,13 +197,29 @@ __global__ void __launch_bounds__(256) k_lconv(const ActT *__restrict__ gl, cons
 cudaError_t launch_lconv(const ae_model *m, const void *gl, const float *w_dw, const float *w_norm, float lo,
                          float hi, void *out, const int32_t *pos, int64_t T, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  const unsigned grid = (unsigned)((T + 8 * kRowsPerWarp - 1) / (8 * kRowsPerWarp));
-  if (m->dtype == AE_BF16)
-    k_lconv<bf16><<<grid, 256, 0, s>>>(static_cast<const bf16 *>(gl), w_dw, w_norm, lo, hi, static_cast<bf16 *>(out),
-                                       pos, T);
-  else
-    k_lconv<float><<<grid, 256, 0, s>>>(static_cast<const float *>(gl), w_dw, w_norm, lo, hi,
-                                        static_cast<float *>(out), pos, T);
+  const unsigned grid = (unsigned)((T + kLcRows - 1) / kLcRows);
+  const size_t base = (size_t)(kLcRows + kLcHalo) * kHidden;
+  if (m->dtype == AE_BF16) {
+    const size_t smem = base * 2;
+    static bool attr = false;
+    if (!attr) {
+      cudaError_t e = cudaFuncSetAttribute(k_lconv<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      attr = true;
+    }
+    k_lconv<bf16><<<grid, 256, smem, s>>>(static_cast<const bf16 *>(gl), w_dw, w_norm, lo, hi,
+                                          static_cast<bf16 *>(out), pos, T);
+  } else {
+    const size_t smem = base * 4;
+    static bool attr = false;
+    if (!attr) {
+      cudaError_t e = cudaFuncSetAttribute(k_lconv<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      attr = true;
+    }
+    k_lconv<float><<<grid, 256, smem, s>>>(static_cast<const float *>(gl), w_dw, w_norm, lo, hi,
+                                           static_cast<float *>(out), pos, T);
+  }
   return cudaGetLastError();
 }
 

@@ -39,69 +39,94 @@ __device__ __forceinline__ int clip_of(const int32_t *off, int n_clips, int64_t 
 
 // ------------------------------------------------------------------ conv0 + LN + ReLU
 
-template <typename OutT>
-__global__ void __launch_bounds__(256) k_conv0(const float *__restrict__ mel, const float *__restrict__ wc,
-                                               const float *__restrict__ cov, const float *__restrict__ g0,
-                                               OutT *__restrict__ y0, const ClipTablesDev t) {
-  __shared__ float s_w[kC0 * 9];
-  __shared__ float s_g[kC0];
-  __shared__ float s_p[kF1][10];
-  __shared__ float s_r[kF1];
-  const int64_t row = blockIdx.x;
-  const int c = clip_of(t.stem_off, t.n_clips, row);
-  const int ti = (int)(row - t.stem_off[c]) - 2;
-  const int F = t.frame_off[c + 1] - t.frame_off[c];
-  const int t1 = (F + 1) / 2;
-  OutT *orow = y0 + row * (int64_t)(kF1 * kC0);
-  if (ti < 0 || ti >= t1) {
-    for (int i = threadIdx.x; i < kF1 * kC0; i += blockDim.x) orow[i] = Act<OutT>::zero();
-    return;
+// A CTA writes kConv0Rows stem rows (64 positions each). Phase 1: each of the
+// 256 positions gets its 9-sample patch and 1/sqrt(p^T C p + eps) into shared
+// memory. Phase 2: thread (channel pair, position parity) holds its taps and
+// gains in registers and walks the positions, storing two channels at once:
+// consecutive threads write consecutive channels of one position, so every
+// row is written with full coalesced segments. Rows outside a clip's frames
+// (the zero padding) come out as zeros from all-zero patches.
+constexpr int kConv0Rows = 4;
+
+template <typename OutT> struct Pair;
+template <> struct Pair<bf16> {
+  static __device__ __forceinline__ void st(bf16 *p, float a, float b) {
+    *reinterpret_cast<uint32_t *>(p) = pack_bf16(a, b);
   }
-  for (int i = threadIdx.x; i < kC0 * 9; i += blockDim.x) s_w[i] = wc[i];
-  for (int i = threadIdx.x; i < kC0; i += blockDim.x) s_g[i] = g0[i];
-  if (threadIdx.x < kF1) {
-    const int f = threadIdx.x;
-    const float *m = mel + (int64_t)t.frame_off[c] * kMels;
+};
+template <> struct Pair<float> {
+  static __device__ __forceinline__ void st(float *p, float a, float b) {
+    *reinterpret_cast<float2 *>(p) = make_float2(a, b);
+  }
+};
+
+template <typename OutT>
+__global__ void __launch_bounds__(128) k_conv0(const float *__restrict__ mel, const float *__restrict__ wc,
+                                               const float *__restrict__ cov, const float *__restrict__ g0,
+                                               OutT *__restrict__ y0, const ClipTablesDev t, int64_t stem_rows) {
+  constexpr int P = kConv0Rows * kF1;  // positions per CTA
+  __shared__ __align__(16) float s_p[P][12];
+  __shared__ float s_r[P];
+  const int64_t row0 = (int64_t)blockIdx.x * kConv0Rows;
+  for (int i = threadIdx.x; i < P; i += blockDim.x) {
+    const int64_t row = row0 + i / kF1;
+    const int f = i % kF1;
     float p[9];
 #pragma unroll
-    for (int dt = 0; dt < 3; ++dt)
+    for (int k = 0; k < 9; ++k) p[k] = 0.f;
+    if (row < stem_rows) {
+      const int c = clip_of(t.stem_off, t.n_clips, row);
+      const int ti = (int)(row - t.stem_off[c]) - 2;
+      const int F = t.frame_off[c + 1] - t.frame_off[c];
+      if (ti >= 0 && ti < (F + 1) / 2) {
+        const float *m = mel + (int64_t)t.frame_off[c] * kMels;
 #pragma unroll
-      for (int df = 0; df < 3; ++df) {
-        const int tr = 2 * ti + dt - 1, fr = 2 * f + df - 1;
-        p[dt * 3 + df] = (tr >= 0 && tr < F && fr >= 0 && fr < kMels) ? m[(int64_t)tr * kMels + fr] : 0.f;
+        for (int dt = 0; dt < 3; ++dt)
+#pragma unroll
+          for (int df = 0; df < 3; ++df) {
+            const int tr = 2 * ti + dt - 1, fr = 2 * f + df - 1;
+            if (tr >= 0 && tr < F && fr >= 0 && fr < kMels) p[dt * 3 + df] = __ldg(m + (int64_t)tr * kMels + fr);
+          }
       }
+    }
     float var = 0.f;
 #pragma unroll
     for (int a = 0; a < 9; ++a) {
       float s = 0.f;
 #pragma unroll
-      for (int b = 0; b < 9; ++b) s = fmaf(cov[a * 9 + b], p[b], s);
+      for (int b = 0; b < 9; ++b) s = fmaf(__ldg(cov + a * 9 + b), p[b], s);
       var = fmaf(p[a], s, var);
     }
 #pragma unroll
-    for (int k = 0; k < 9; ++k) s_p[f][k] = p[k];
-    s_r[f] = rsqrtf(fmaxf(var, 0.f) + 1e-6f);
+    for (int k = 0; k < 9; ++k) s_p[i][k] = p[k];
+    s_r[i] = rsqrtf(fmaxf(var, 0.f) + 1e-6f);
   }
   __syncthreads();
-  // thread -> (freq f, 32 consecutive channels)
-  const int f = threadIdx.x >> 2, c0 = (threadIdx.x & 3) * 32;
-  float p[9];
+  const int cp = threadIdx.x & 63, par = threadIdx.x >> 6;  // channels 2cp, 2cp+1; positions of parity par
+  float w0[9], w1[9];
 #pragma unroll
-  for (int k = 0; k < 9; ++k) p[k] = s_p[f][k];
-  const float r = s_r[f];
-  OutT *o = orow + f * kC0 + c0;
+  for (int k = 0; k < 9; ++k) {
+    w0[k] = __ldg(wc + (2 * cp) * 9 + k);
+    w1[k] = __ldg(wc + (2 * cp + 1) * 9 + k);
+  }
+  const float g0a = __ldg(g0 + 2 * cp), g0b = __ldg(g0 + 2 * cp + 1);
+  const int64_t left_pos = (stem_rows - row0) * kF1;
+  const int n_pos = left_pos < P ? (int)left_pos : P;
+  OutT *out = y0 + row0 * (int64_t)(kF1 * kC0);
+#pragma unroll 4
+  for (int i = par; i < n_pos; i += 2) {
+    const float4 pa = *reinterpret_cast<const float4 *>(&s_p[i][0]);
+    const float4 pb = *reinterpret_cast<const float4 *>(&s_p[i][4]);
+    const float p8 = s_p[i][8];
+    const float r = s_r[i];
+    const float p[9] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w, p8};
+    float a = 0.f, b = 0.f;
 #pragma unroll
-  for (int q = 0; q < 32; q += 4) {
-    float v[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float *w = s_w + (c0 + q + u) * 9;
-      float a = 0.f;
-#pragma unroll
-      for (int k = 0; k < 9; ++k) a = fmaf(w[k], p[k], a);
-      v[u] = fmaxf(a * r * s_g[c0 + q + u], 0.f);
+    for (int k = 0; k < 9; ++k) {
+      a = fmaf(w0[k], p[k], a);
+      b = fmaf(w1[k], p[k], b);
     }
-    store4(o + q, v);
+    Pair<OutT>::st(out + (int64_t)i * kC0 + 2 * cp, fmaxf(a * r * g0a, 0.f), fmaxf(b * r * g0b, 0.f));
   }
 }
 
@@ -284,10 +309,11 @@ __global__ void __launch_bounds__(256) k_conv1_f32(const float *__restrict__ y0,
 cudaError_t launch_conv0(const ae_model *m, const float *mel, void *y0, const ClipTablesDev &t, int64_t stem_rows,
                          cudaStream_t s) {
   if (stem_rows <= 0) return cudaSuccess;
+  const unsigned grid = (unsigned)((stem_rows + kConv0Rows - 1) / kConv0Rows);
   if (m->dtype == AE_BF16)
-    k_conv0<bf16><<<(unsigned)stem_rows, 256, 0, s>>>(mel, m->conv0c, m->conv0cov, m->ln0, static_cast<bf16 *>(y0), t);
+    k_conv0<bf16><<<grid, 128, 0, s>>>(mel, m->conv0c, m->conv0cov, m->ln0, static_cast<bf16 *>(y0), t, stem_rows);
   else
-    k_conv0<float><<<(unsigned)stem_rows, 256, 0, s>>>(mel, m->conv0c, m->conv0cov, m->ln0, static_cast<float *>(y0), t);
+    k_conv0<float><<<grid, 128, 0, s>>>(mel, m->conv0c, m->conv0cov, m->ln0, static_cast<float *>(y0), t, stem_rows);
   return cudaGetLastError();
 }
 

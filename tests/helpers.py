@@ -27,14 +27,23 @@ def cosine(g, o) -> float:
 
 def assert_f32(g, o, what=""):
     e = rel_err(g, o)
+    print(f"[parity] {what}: rel err {e:.3e} (bound {F32_REL})")
     assert e <= F32_REL, f"{what}: rel err {e:.3e} > {F32_REL}"
     return e
 
 
 def assert_bf16(g, o, what=""):
     e, c = rel_err(g, o), cosine(g, o)
+    print(f"[parity] {what}: rel err {e:.3e} (bound {BF16_REL}), cosine {c:.7f} (bound {BF16_COS})")
     assert e <= BF16_REL and c >= BF16_COS, f"{what}: rel err {e:.3e} (<= {BF16_REL}), cosine {c:.6f} (>= {BF16_COS})"
     return e, c
+
+
+def assert_logmel(g, o, what=""):
+    e = float(np.max(np.abs(np.asarray(g, np.float64) - np.asarray(o, np.float64)))) if np.size(o) else 0.0
+    print(f"[parity] {what}: max abs err {e:.3e} (bound {LOGMEL_ABS})")
+    assert e <= LOGMEL_ABS, f"{what}: max abs err {e:.3e} > {LOGMEL_ABS}"
+    return e
 
 
 def offsets(lengths) -> np.ndarray:

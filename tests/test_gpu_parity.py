@@ -14,7 +14,8 @@ import pytest
 
 import synth
 from oracle import oracle as O
-from tests.helpers import (LOGMEL_ABS, assert_bf16, assert_f32, dev, offsets, rel_err, cosine, workspace)
+from tests.helpers import (LOGMEL_ABS, assert_bf16, assert_f32, assert_logmel, dev, offsets, rel_err, cosine,
+                           workspace)
 
 pytestmark = pytest.mark.gpu
 
@@ -85,7 +86,7 @@ def test_logmel_pr1_clip():
     g = gpu_logmel([wave])
     o = O.log_mel(wave)
     assert g.shape == (99, 128)
-    assert np.max(np.abs(g - o)) <= LOGMEL_ABS
+    assert_logmel(g, o, "log-mel pr1")
 
 
 def test_logmel_edge_lengths_packed():
@@ -102,7 +103,7 @@ def test_logmel_edge_lengths_packed():
         gi = g[off[i]:off[i + 1]]
         assert gi.shape == o.shape
         if len(o):
-            assert np.max(np.abs(gi - o)) <= LOGMEL_ABS, lens[i]
+            assert_logmel(gi, o, f"log-mel clip of {lens[i]} samples")
     sil = g[off[7]:off[8]]
     assert np.max(np.abs(sil - math.log(1e-3))) < 1e-6
 
@@ -122,8 +123,7 @@ def test_logmel_frontend_workload_full():
     assert g.shape == (64 * 2999, 128)
     for i, c in enumerate(clips):
         o = O.log_mel(c)
-        err = np.max(np.abs(g[i * 2999:(i + 1) * 2999] - o))
-        assert err <= LOGMEL_ABS, (i, err)
+        assert_logmel(g[i * 2999:(i + 1) * 2999], o, f"log-mel frontend clip {i}")
 
 
 # ------------------------------------------------------------------ stem
