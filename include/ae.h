@@ -214,6 +214,30 @@ ae_status ae_local_attention(const void *d_q, const void *d_k, const void *d_v, 
                              void *d_out, int64_t ld_out, void *d_ws, size_t ws_bytes,
                              ae_stream stream);
 
+/* --- log-mel without a caller workspace ---------------------------------------- */
+
+/* ae_logmel for callers that cannot allocate device memory at all: code that
+ * runs where the allocator must not be entered (a real-time audio callback,
+ * an inference host whose device memory belongs entirely to its own pool
+ * allocator, a plugin that is handed only its input and output buffers). It
+ * computes exactly what ae_logmel computes, but keeps its only scratch data,
+ * the per-call clip tables, in a fixed array inside the library (128 KiB in
+ * the device memory of every GPU that loads the library, held until the
+ * process exits) instead of a workspace. The pages have no counterpart: the
+ * reference front-end runs on the host.
+ *
+ * d_wave, h_sample_off, n_clips, d_mel and stream mean what they mean for
+ * ae_logmel. At most 4000 clips per call; more is refused with AE_EINVAL
+ * before anything is enqueued. The call calls no cudaMalloc or cudaFree.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture. Every call uses the same array and rewrites the
+ * part it reads, so calls that may overlap on the GPU (on different streams,
+ * or from several host threads) race with each other: order them on one
+ * stream. */
+ae_status ae_logmel_noalloc(const float *d_wave, const int64_t *h_sample_off, int n_clips, float *d_mel,
+                            ae_stream stream);
+
 /* --- kernel timing ------------------------------------------------------------ */
 
 /* Classes of the kernels the calls launch. */

@@ -84,6 +84,7 @@ _sig("ae_local_attention", _st, _vp, _vp, _vp, C.c_int64, _i32, _vp, _vp, C.c_fl
 _sig("ae_last_error", C.c_char_p)
 _sig("ae_device_status", _st)
 _sig("ae_version", C.c_char_p)
+_sig("ae_logmel_noalloc", _st, _vp, _i64p, _i32, _vp, _vp)
 _sig("ae_profile_enable", _st, _i32)
 _sig("ae_profile_read", _st, C.POINTER(C.c_double), _i64p, C.POINTER(C.c_double), C.POINTER(C.c_double), _i64p)
 
@@ -91,7 +92,7 @@ _sig("ae_profile_read", _st, C.POINTER(C.c_double), _i64p, C.POINTER(C.c_double)
 EXPORTS = ("ae_num_frames", "ae_num_tokens", "ae_model_create", "ae_model_destroy", "ae_workspace_size",
            "ae_logmel", "ae_subsample", "ae_conformer_layer", "ae_encode", "ae_encode_host_workspace_size",
            "ae_encode_host", "ae_attention_tables", "ae_local_attention", "ae_last_error", "ae_device_status",
-           "ae_version", "ae_profile_enable", "ae_profile_read")
+           "ae_version", "ae_profile_enable", "ae_profile_read", "ae_logmel_noalloc")
 
 KERNEL_CLASSES = ("tables", "logmel", "conv0", "conv1", "gemm", "attention", "lconv", "rowop")
 
@@ -157,6 +158,13 @@ def ae_logmel(d_wave, sample_off, d_mel, d_ws, ws_bytes: int, stream=None):
     a, p = _off(sample_off)
     _check(lib.ae_logmel(_ptr(d_wave), p, len(a) - 1, _ptr(d_mel), _ptr(d_ws), ws_bytes, _stream(stream)),
            "ae_logmel")
+
+
+def ae_logmel_noalloc(d_wave, sample_off, d_mel, stream=None):
+    """ae_logmel without a workspace: for callers that must not allocate device
+    memory (the clip tables live in a fixed array inside the library)."""
+    a, p = _off(sample_off)
+    _check(lib.ae_logmel_noalloc(_ptr(d_wave), p, len(a) - 1, _ptr(d_mel), _stream(stream)), "ae_logmel_noalloc")
 
 
 def ae_subsample(model, d_mel, frame_off, d_h, d_ws, ws_bytes: int, stream=None):

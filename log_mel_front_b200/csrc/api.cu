@@ -5,6 +5,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -481,6 +482,35 @@ static ae_status encode_dev(const ae_model *m, const float *d_wave, const ClipTa
   return AE_OK;
 }
 
+// ------------------------------------------------------------------ log-mel without a workspace
+
+// The clip tables of ae_logmel_noalloc live in this file-scope device array
+// (every GPU that loads the library holds it until the process exits). In
+// host code the name is only a stand-in: its device address is looked up
+// once per device with cudaGetSymbolAddress and passed to the kernels.
+constexpr int kNoAllocMaxClips = 4000;
+constexpr size_t kNoAllocScratchBytes = 131072;
+static __device__ __align__(256) unsigned char g_logmel_scratch[kNoAllocScratchBytes];
+
+static std::mutex g_noalloc_mu;
+static void *g_noalloc_ptr[64] = {nullptr};
+
+// Device address of the scratch array on the current device.
+static ae_status noalloc_scratch(void **out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return fail(AE_ECUDA, "no CUDA device");
+  if (dev >= 64) return fail(AE_EUNSUPPORTED, "device index above 63");
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_logmel_scratch);
+    if (e != cudaSuccess || !p) return cuda_fail(e, "cudaGetSymbolAddress of the log-mel scratch");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return AE_OK;
+}
+
 }  // namespace ae
 
 using namespace ae;
@@ -827,6 +857,30 @@ ae_status ae_local_attention(const void *d_q, const void *d_k, const void *d_v, 
                                  T.total_tokens, d_out, ld_out, -INFINITY, INFINITY, s);
        })) != cudaSuccess)
     return cuda_fail(e, "attention");
+  return AE_OK;
+}
+
+ae_status ae_logmel_noalloc(const float *d_wave, const int64_t *h_sample_off, int n_clips, float *d_mel,
+                            ae_stream stream) {
+  if (n_clips > kNoAllocMaxClips)
+    return fail(AE_EINVAL, "ae_logmel_noalloc takes at most " + std::to_string(kNoAllocMaxClips) +
+                               " clips per call (got " + std::to_string(n_clips) + "); split the batch");
+  ClipTables T;
+  ae_status st = build_tables(h_sample_off, n_clips, kSamples, T, "h_sample_off");
+  if (st) return st;
+  if (T.total_frames > 0 && (!d_wave || !d_mel)) return fail(AE_EINVAL, "d_wave or d_mel is null");
+  if (n_clips == 0) return AE_OK;
+  const WsLayout L = ws_layout(nullptr, T.n_clips, T.total_frames, 0, false);  // the tables alone
+  if (L.total > kNoAllocScratchBytes) return fail(AE_EINVAL, "clip tables exceed the fixed scratch array");
+  void *scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch))) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the upload rewrites every table word the front-end reads: nothing relies
+  // on the array's earlier contents
+  ClipTablesDev td;
+  cudaError_t e = tables_t(T, scratch, L, &td, false, s);
+  if (e != cudaSuccess) return cuda_fail(e, "table upload");
+  if ((e = logmel_t(d_wave, d_mel, td, T, s)) != cudaSuccess) return cuda_fail(e, "logmel");
   return AE_OK;
 }
 
