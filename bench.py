@@ -51,6 +51,46 @@ def peaks():
 
 # ------------------------------------------------------------------ clocks
 
+# DRAM traffic of the dominant kernel comes from a committed ncu summary
+# (dram__bytes_read.sum + dram__bytes_write.sum per launch over one step). The
+# summary records the sha256 of the kernel's sources at capture time; once they
+# differ the figure no longer describes the kernel and is reported as null.
+TRAFFIC_PROFILES = {
+    "gemm": ("profiles/gemm_tc_tower_dram.md",
+             ("log_mel_front_b200/csrc/gemm.cu", "log_mel_front_b200/csrc/common.cuh")),
+}
+
+
+def sources_sha256(paths) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def captured_traffic(kind: str):
+    """(bytes per launch, note) from the committed capture, or (None, why)."""
+    if kind not in TRAFFIC_PROFILES:
+        return None, "no capture for this kernel"
+    path, srcs = TRAFFIC_PROFILES[kind]
+    vals = {}
+    try:
+        with open(os.path.join(ROOT, path)) as f:
+            for line in f:
+                if ":" in line and line.split(":", 1)[0].strip() in ("traffic_bytes_per_launch", "source_sha256"):
+                    k, v = line.split(":", 1)
+                    vals[k.strip()] = v.strip().strip("`")
+    except OSError:
+        return None, "capture summary missing"
+    if "traffic_bytes_per_launch" not in vals or "source_sha256" not in vals:
+        return None, "capture summary incomplete"
+    if vals["source_sha256"] != sources_sha256(srcs):
+        return None, "kernel sources changed since the capture"
+    return float(vals["traffic_bytes_per_launch"]), path
+
+
 class Clocks:
     """nvidia-smi sampled every 200 ms during the timed region."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
@@ -314,10 +354,13 @@ def run_ours(args, rank, world, dist):
         achieved = dom["bytes"] / (dom["ms"] / 1e3) / 1e9
         peak = pk["hbm_gbs"]
         roof = {"bound": "hbm", "unit": "GB/s", "peak_kind": "HBM copy (" + pk["source"] + ")"}
+    traffic, traffic_src = captured_traffic(ours.dominant)
     roof.update({"kernel": {"gemm": "k_gemm_tc (all projections)", "logmel": "k_logmel",
                             "attention": "k_attention"}[ours.dominant],
                  "achieved": round(achieved, 2), "peak": peak, "frac": round(achieved / peak, 4),
-                 "traffic": None, "launches_per_step": dom["launches"] / args.steps,
+                 "traffic": None if traffic is None else round(traffic), "traffic_source": traffic_src,
+                 "algorithmic_bytes_per_launch": round(dom["bytes"] / max(dom["launches"], 1)),
+                 "launches_per_step": dom["launches"] / args.steps,
                  "share_of_step": round(dom["ms"] / max(ms_prof, 1e-9), 4)})
     classes = {k: {"ms_per_step": round(v["ms"] / args.steps, 4), "launches_per_step": v["launches"] / args.steps,
                    **({"tflops": round(v["flops"] / (v["ms"] / 1e3) / 1e12, 1)} if v["flops"] and v["ms"] else {}),

@@ -74,7 +74,7 @@ struct ae_model {
   int device;
   float k_scale;
   // stem
-  float *conv0c;    // [c0][9] taps minus their channel mean (the LayerNorm's mean is linear in the patch)
+  float *conv0c;    // [c0][9] (taps minus their channel mean) x LayerNorm gain: the norm's mean is linear in the patch
   float *conv0cov;  // [9][9] channel covariance of the taps: LayerNorm variance = p^T C p
   float *ln0, *ln1;
   void *conv1;      // [c1][9 * c0], k = (dt * 3 + df) * c0 + c
@@ -159,6 +159,23 @@ cudaError_t launch_attention(bool is_bf16, const void *q, const void *k, const v
 bool make_tmap_2d_bf16(CUtensorMap *tm, const void *base, uint64_t inner, uint64_t outer,
                        uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
 bool make_tmap_stem_y0(CUtensorMap *tm, const void *y0, int64_t stem_rows);
+
+// Launch with programmatic stream serialization (see pdl_wait/pdl_trigger).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                            Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
 
 unsigned *device_status_word();
 unsigned read_and_clear_status();

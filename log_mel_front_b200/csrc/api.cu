@@ -608,7 +608,7 @@ ae_status ae_model_create(const ae_config *cfg, const ae_host_weights *w, ae_dty
     for (int ch = 0; ch < kC0; ++ch)
       for (int a = 0; a < 9; ++a) {
         const double da = w->conv0[ch * 9 + a] - mean[a];
-        wc[ch * 9 + a] = (float)da;
+        wc[ch * 9 + a] = (float)(da * (double)w->ln0[ch]);  // LayerNorm gain folded into the centred taps
         for (int b2 = 0; b2 < 9; ++b2) cd[a * 9 + b2] += da * (w->conv0[ch * 9 + b2] - mean[b2]);
       }
     for (int i = 0; i < 81; ++i) cov[i] = (float)(cd[i] / kC0);

@@ -130,6 +130,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   const int m_blocks = (M + 2 * BM - 1) / (2 * BM), n_blocks = N / BN, kb_n = K / BK;
   const int num_tiles = m_blocks * n_blocks;
   const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  pdl_trigger();
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -154,6 +155,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   cluster_sync();  // both CTAs' barriers are initialised before any cross-CTA arrival
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // x (and the output buffer) belong to the previous kernels until here
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer (both CTAs)
@@ -290,10 +292,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
 // ------------------------------------------------------------------ f32 FMA kernel
 
 template <int MODE>
-__global__ void __launch_bounds__(256) k_gemm_f32(const float *__restrict__ A, const float *__restrict__ B,
+__global__ void __launch_bounds__(256) k_gemm_f32(const float *A, const float *__restrict__ B,
                                                   const EpiArgs ep, int M, int N, int K) {
   __shared__ float As[16][64 + 4];
   __shared__ float Bs[16][64 + 4];
+  pdl_trigger();
+  pdl_wait(A);
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
   float acc[4][4] = {};
@@ -411,16 +415,15 @@ static cudaError_t launch_tc(const CUtensorMap &tA, const CUtensorMap &tB, const
   }
   const int tiles = ((M + 2 * BM - 1) / (2 * BM)) * (N / BN);
   const int pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;
-  k_gemm_tc<MODE><<<2 * pairs, GEMM_THREADS, SMEM_TC, s>>>(tA, tB, ep, M, N, K, device_status_word());
-  return cudaGetLastError();
+  return launch_k(k_gemm_tc<MODE>, dim3(2 * pairs), dim3(GEMM_THREADS), SMEM_TC, s, tA, tB, ep, M, N, K,
+                  device_status_word());
 }
 
 template <int MODE>
 static cudaError_t launch_f32(const float *x, const float *w, const EpiArgs &ep, int M, int N, int K,
                               cudaStream_t s) {
   dim3 grid(N / 64, (M + 63) / 64);
-  k_gemm_f32<MODE><<<grid, 256, 0, s>>>(x, w, ep, M, N, K);
-  return cudaGetLastError();
+  return launch_k(k_gemm_f32<MODE>, grid, dim3(256), 0, s, x, w, ep, M, N, K);
 }
 
 cudaError_t gemm(const ae_model *m, const void *x, int64_t M, int K, const void *w, const CUtensorMap *tmW, int N,

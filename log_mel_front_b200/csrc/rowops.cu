@@ -27,34 +27,49 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 constexpr float kEps = 1e-6f;
 
-// NV = width / 128: lane l holds columns (i * 32 + l) * 4 .. +3, i < NV.
+// NV = width / 128: lane l holds columns (i * 32 + l) * 4 .. +3, i < NV. The
+// row's h and y are loaded first; the weight vectors are staged in shared
+// memory while those loads are in flight, so a row costs one memory round
+// trip.
 template <int NV, typename ActT>
-__global__ void __launch_bounds__(256) k_rowop(const RowArgs r) {
+__global__ void __launch_bounds__(256, NV <= 8 ? 3 : 2) k_rowop(const RowArgs r) {
+  constexpr int W = NV * 128;
+  __shared__ __align__(16) float s_wy[W], s_wo[W], s_wn[W];
   const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (row >= r.rows) return;
-  constexpr int W = NV * 128;
-  float *hrow = r.h + row * W;
-  float h[NV][4];
+  const bool live = row < r.rows;
+  pdl_trigger();
+  for (int i = threadIdx.x; i < W / 4; i += blockDim.x) {  // weights: independent of upstream kernels
+    if (r.wy) reinterpret_cast<float4 *>(s_wy)[i] = __ldg(reinterpret_cast<const float4 *>(r.wy) + i);
+    if (r.w_out) reinterpret_cast<float4 *>(s_wo)[i] = __ldg(reinterpret_cast<const float4 *>(r.w_out) + i);
+    if (r.w_next) reinterpret_cast<float4 *>(s_wn)[i] = __ldg(reinterpret_cast<const float4 *>(r.w_next) + i);
+  }
+  pdl_wait();
+  float *hrow = r.h + (live ? row : 0) * W;
+  float h[NV][4], y[NV][4];
+  if (live) {
 #pragma unroll
-  for (int i = 0; i < NV; ++i) load4(hrow + (i * 32 + lane) * 4, h[i]);
+    for (int i = 0; i < NV; ++i) load4(hrow + (i * 32 + lane) * 4, h[i]);
+    if (r.y) {
+#pragma unroll
+      for (int i = 0; i < NV; ++i) load4(r.y + row * W + (i * 32 + lane) * 4, y[i]);
+    }
+  }
+  __syncthreads();
+  if (!live) return;
   bool changed = false;
   if (r.y) {
-    const float *yrow = r.y + row * W;
-    float y[NV][4];
     float ss = 0.f;
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      load4(yrow + (i * 32 + lane) * 4, y[i]);
+    for (int i = 0; i < NV; ++i)
 #pragma unroll
       for (int u = 0; u < 4; ++u) ss = fmaf(y[i][u], y[i][u], ss);
-    }
     float sc = r.s;
     if (r.y_norm) sc *= rsqrtf(warp_sum(ss) * (1.0f / W) + kEps);
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
       float w[4] = {1.f, 1.f, 1.f, 1.f};
-      if (r.y_norm && r.wy) load4(r.wy + (i * 32 + lane) * 4, w);
+      if (r.y_norm && r.wy) load4(s_wy + (i * 32 + lane) * 4, w);
 #pragma unroll
       for (int u = 0; u < 4; ++u) h[i][u] = fmaf(sc * w[u], y[i][u], h[i][u]);
     }
@@ -70,7 +85,7 @@ __global__ void __launch_bounds__(256) k_rowop(const RowArgs r) {
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
       float w[4];
-      load4(r.w_out + (i * 32 + lane) * 4, w);
+      load4(s_wo + (i * 32 + lane) * 4, w);
 #pragma unroll
       for (int u = 0; u < 4; ++u) h[i][u] = h[i][u] * inv * w[u];
     }
@@ -94,7 +109,7 @@ __global__ void __launch_bounds__(256) k_rowop(const RowArgs r) {
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
       float w[4] = {1.f, 1.f, 1.f, 1.f};
-      if (r.w_next) load4(r.w_next + (i * 32 + lane) * 4, w);
+      if (r.w_next) load4(s_wn + (i * 32 + lane) * 4, w);
       float a[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) a[u] = clampf(h[i][u] * inv * w[u], r.lo, r.hi);
@@ -107,12 +122,11 @@ template <typename ActT>
 static cudaError_t rowop_width(const RowArgs &r, cudaStream_t s) {
   const unsigned grid = (unsigned)((r.rows + 7) / 8);
   switch (r.width) {
-    case 1024: k_rowop<8, ActT><<<grid, 256, 0, s>>>(r); break;
-    case 1536: k_rowop<12, ActT><<<grid, 256, 0, s>>>(r); break;
-    case 2048: k_rowop<16, ActT><<<grid, 256, 0, s>>>(r); break;
+    case 1024: return launch_k(k_rowop<8, ActT>, dim3(grid), dim3(256), 0, s, r);
+    case 1536: return launch_k(k_rowop<12, ActT>, dim3(grid), dim3(256), 0, s, r);
+    case 2048: return launch_k(k_rowop<16, ActT>, dim3(grid), dim3(256), 0, s, r);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_rowop(const ae_model *m, const RowArgs &r, cudaStream_t s) {
@@ -122,75 +136,81 @@ cudaError_t launch_rowop(const ae_model *m, const RowArgs &r, cudaStream_t s) {
 
 // ------------------------------------------------------------------ light conv middle
 
-// w_dw is stored tap-major [kernel][hidden] (20 KB, read through L1). A CTA
-// owns kLcRows consecutive rows: it stages those rows plus the 4 before them
-// in shared memory with coalesced 16-byte loads; each warp then computes
-// kLcRows / 8 rows, lane l owning channels (i * 32 + l) * 4 .. +3.
-constexpr int kLcRows = 16;
+// w_dw is stored tap-major [kernel][hidden]. Thread t of a 256-thread CTA
+// owns channels 4t .. 4t+3 for kLcRows consecutive rows: its 5 x 4 taps and
+// 4 norm weights stay in registers, and it walks the rows (plus the 4 before
+// them) with a sliding window, one coalesced 8-byte load per row. The conv
+// outputs of its rows stay in registers; the per-row sums of squares are
+// reduced across the CTA once for all its rows.
+constexpr int kLcRows = 8;
 constexpr int kLcHalo = kKernel - 1;
 
 template <typename ActT>
-__global__ void __launch_bounds__(256) k_lconv(const ActT *__restrict__ gl, const float *__restrict__ w_dw,
+__global__ void __launch_bounds__(256) k_lconv(const ActT *gl, const float *__restrict__ w_dw,
                                                const float *__restrict__ w_norm, float lo, float hi,
-                                               ActT *__restrict__ out, const int32_t *__restrict__ pos, int64_t T) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  const float *s_w = w_dw;
-  ActT *s_x = reinterpret_cast<ActT *>(smem_raw);                        // [kLcRows + halo][hidden]
-  const int lane = threadIdx.x & 31;
+                                               ActT *__restrict__ out, const int32_t *pos, int64_t T) {
+  __shared__ float s_ss[8][kLcRows];
+  __shared__ float s_inv[kLcRows];
+  const int ch = 4 * threadIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t t0 = (int64_t)blockIdx.x * kLcRows;
-  constexpr int VEC = 16 / sizeof(ActT);                                 // elements per 16-byte load
-  constexpr int ROW_V = kHidden / VEC;
-  for (int i = threadIdx.x; i < (kLcRows + kLcHalo) * ROW_V; i += blockDim.x) {
-    const int r = i / ROW_V, cv = i % ROW_V;
+  pdl_trigger();
+  float w[kKernel][4], wn[4];
+#pragma unroll
+  for (int k = 0; k < kKernel; ++k) load4(w_dw + k * kHidden + ch, w[k]);
+  load4(w_norm + ch, wn);
+  pdl_wait(gl, pos);
+  float x[kLcRows + kLcHalo][4];
+#pragma unroll
+  for (int r = 0; r < kLcRows + kLcHalo; ++r) {
     const int64_t tok = t0 - kLcHalo + r;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (tok >= 0 && tok < T) v = __ldg(reinterpret_cast<const uint4 *>(gl + tok * kHidden) + cv);
-    reinterpret_cast<uint4 *>(s_x + (int64_t)r * kHidden)[cv] = v;
+    if (tok >= 0 && tok < T) {
+      load4(gl + tok * kHidden + ch, x[r]);
+    } else {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) x[r][u] = 0.f;
+    }
   }
-  __syncthreads();
-  constexpr int NV = kHidden / 128;
-  for (int rr = 0; rr < kLcRows / 8; ++rr) {
-    const int lr = (threadIdx.x >> 5) * (kLcRows / 8) + rr;  // local output row
-    const int64_t t = t0 + lr;
-    if (t >= T) return;
-    const int p = pos[t];
-    float c[NV][4];
+  float c[kLcRows][4], ss[kLcRows];
 #pragma unroll
-    for (int i = 0; i < NV; ++i)
+  for (int r = 0; r < kLcRows; ++r) {
+    const int64_t tok = t0 + r;
+    const int p = tok < T ? pos[tok] : 0;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) c[i][u] = 0.f;
+    for (int u = 0; u < 4; ++u) c[r][u] = 0.f;
 #pragma unroll
     for (int k = 0; k < kKernel; ++k) {
       const int back = kKernel - 1 - k;
-      if (back > p) continue;
-      const ActT *src = s_x + (int64_t)(lr + kLcHalo - back) * kHidden;
+      if (back <= p) {
 #pragma unroll
-      for (int i = 0; i < NV; ++i) {
-        float x[4], w[4];
-        load4(src + (i * 32 + lane) * 4, x);
-        load4(s_w + k * kHidden + (i * 32 + lane) * 4, w);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) c[i][u] = fmaf(w[u], x[u], c[i][u]);
+        for (int u = 0; u < 4; ++u) c[r][u] = fmaf(w[k][u], x[r + kLcHalo - back][u], c[r][u]);
       }
     }
-    float ss = 0.f;
+    ss[r] = warp_sum(c[r][0] * c[r][0] + c[r][1] * c[r][1] + c[r][2] * c[r][2] + c[r][3] * c[r][3]);
+  }
+  if (lane == 0) {
 #pragma unroll
-    for (int i = 0; i < NV; ++i)
+    for (int r = 0; r < kLcRows; ++r) s_ss[warp][r] = ss[r];
+  }
+  __syncthreads();
+  if (threadIdx.x < kLcRows) {
+    float s = 0.f;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) ss = fmaf(c[i][u], c[i][u], ss);
-    const float inv = rsqrtf(warp_sum(ss) * (1.0f / kHidden) + kEps);
-    ActT *orow = out + t * kHidden;
+    for (int q = 0; q < 8; ++q) s += s_ss[q][threadIdx.x];
+    s_inv[threadIdx.x] = rsqrtf(s * (1.0f / kHidden) + kEps);
+  }
+  __syncthreads();
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      float w[4], v[4];
-      load4(w_norm + (i * 32 + lane) * 4, w);
+  for (int r = 0; r < kLcRows; ++r) {
+    const int64_t tok = t0 + r;
+    if (tok >= T) break;
+    const float inv = s_inv[r];
+    float v[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float y = c[i][u] * inv * w[u];
-        v[u] = clampf(y / (1.0f + __expf(-y)), lo, hi);
-      }
-      store4(orow + (i * 32 + lane) * 4, v);
+    for (int u = 0; u < 4; ++u) {
+      const float y = c[r][u] * inv * wn[u];
+      v[u] = clampf(__fdividef(y, 1.0f + __expf(-y)), lo, hi);
     }
+    store4(out + tok * kHidden + ch, v);
   }
 }
 
@@ -198,29 +218,11 @@ cudaError_t launch_lconv(const ae_model *m, const void *gl, const float *w_dw, c
                          float hi, void *out, const int32_t *pos, int64_t T, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
   const unsigned grid = (unsigned)((T + kLcRows - 1) / kLcRows);
-  const size_t base = (size_t)(kLcRows + kLcHalo) * kHidden;
-  if (m->dtype == AE_BF16) {
-    const size_t smem = base * 2;
-    static bool attr = false;
-    if (!attr) {
-      cudaError_t e = cudaFuncSetAttribute(k_lconv<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      attr = true;
-    }
-    k_lconv<bf16><<<grid, 256, smem, s>>>(static_cast<const bf16 *>(gl), w_dw, w_norm, lo, hi,
-                                          static_cast<bf16 *>(out), pos, T);
-  } else {
-    const size_t smem = base * 4;
-    static bool attr = false;
-    if (!attr) {
-      cudaError_t e = cudaFuncSetAttribute(k_lconv<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      attr = true;
-    }
-    k_lconv<float><<<grid, 256, smem, s>>>(static_cast<const float *>(gl), w_dw, w_norm, lo, hi,
-                                           static_cast<float *>(out), pos, T);
-  }
-  return cudaGetLastError();
+  if (m->dtype == AE_BF16)
+    return launch_k(k_lconv<bf16>, dim3(grid), dim3(256), 0, s, static_cast<const bf16 *>(gl), w_dw, w_norm, lo, hi,
+                    static_cast<bf16 *>(out), pos, T);
+  return launch_k(k_lconv<float>, dim3(grid), dim3(256), 0, s, static_cast<const float *>(gl), w_dw, w_norm, lo, hi,
+                  static_cast<float *>(out), pos, T);
 }
 
 // ------------------------------------------------------------------ tables
@@ -234,11 +236,15 @@ struct UploadChunk {
 };
 
 __global__ void k_upload(uint8_t *base, const UploadChunk ch) {
+  pdl_trigger();
+  pdl_wait();
   uint32_t *d = reinterpret_cast<uint32_t *>(base + ch.dst);
   for (int i = threadIdx.x; i < ch.n; i += blockDim.x) d[i] = ch.w[i];
 }
 
 __global__ void k_pos(int32_t *pos, const int32_t *tok_off) {
+  pdl_trigger();
+  pdl_wait();
   const int c = blockIdx.x;
   const int b = tok_off[c], n = tok_off[c + 1] - b;
   for (int i = threadIdx.x; i < n; i += blockDim.x) pos[b + i] = i;
@@ -246,8 +252,7 @@ __global__ void k_pos(int32_t *pos, const int32_t *tok_off) {
 
 cudaError_t launch_pos(int32_t *pos, const int32_t *tok_off, int n_clips, cudaStream_t s) {
   if (n_clips <= 0) return cudaSuccess;
-  k_pos<<<n_clips, 256, 0, s>>>(pos, tok_off);
-  return cudaGetLastError();
+  return launch_k(k_pos, dim3(n_clips), dim3(256), 0, s, pos, tok_off);
 }
 
 static size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -285,8 +290,7 @@ cudaError_t launch_upload_tables(const ClipTables &t, void *ws, const WsLayout &
     ch.dst = (int64_t)(w0 * 4);
     ch.n = (int)n;
     std::memcpy(ch.w, words.data() + w0, n * 4);
-    k_upload<<<1, 256, 0, s>>>(base, ch);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_k(k_upload, dim3(1), dim3(256), 0, s, base, ch);
     if (e != cudaSuccess) return e;
   }
   dev->n_clips = t.n_clips;

@@ -6,8 +6,9 @@
 // the 9-sample patch p and their variance is the quadratic form p^T C p of
 // the taps' channel covariance C, so one pass gives the normalised outputs:
 // y_c = relu(g_c (w'_c . p) / sqrt(p^T C p + eps)) with w'_c the taps minus
-// their channel mean (both precomputed in float64 at model creation). One
-// CTA writes one time row [64 freq][128 ch] of the channels-last output.
+// their channel mean (taps times gains, and C, precomputed in float64 at
+// model creation). A CTA writes four time rows [64 freq][128 ch] of the
+// channels-last output.
 //
 // The output rows of each clip are laid out with two zero rows in front and
 // zero rows after the last real one, up to 2 * tokens + 2 rows per clip, so
@@ -40,34 +41,26 @@ __device__ __forceinline__ int clip_of(const int32_t *off, int n_clips, int64_t 
 // ------------------------------------------------------------------ conv0 + LN + ReLU
 
 // A CTA writes kConv0Rows stem rows (64 positions each). Phase 1: each of the
-// 256 positions gets its 9-sample patch and 1/sqrt(p^T C p + eps) into shared
-// memory. Phase 2: thread (channel pair, position parity) holds its taps and
-// gains in registers and walks the positions, storing two channels at once:
-// consecutive threads write consecutive channels of one position, so every
-// row is written with full coalesced segments. Rows outside a clip's frames
-// (the zero padding) come out as zeros from all-zero patches.
+// 256 positions gets its 9-sample patch (stored duplicated as (p, p) pairs)
+// and 1/sqrt(p^T C p + eps) in shared memory. Phase 2: thread (channel quad,
+// position phase) holds its four channels' taps, pre-multiplied by the
+// LayerNorm gains at model creation, in registers and walks the positions:
+// two packed FMAs per tap cover the four channels; relu(r * (w'' . p)) is the
+// normalised output (r > 0). Consecutive threads write consecutive channels
+// of one position, so every row is written with full coalesced segments.
+// Rows outside a clip's frames (the zero padding) come out as zeros.
 constexpr int kConv0Rows = 4;
 
-template <typename OutT> struct Pair;
-template <> struct Pair<bf16> {
-  static __device__ __forceinline__ void st(bf16 *p, float a, float b) {
-    *reinterpret_cast<uint32_t *>(p) = pack_bf16(a, b);
-  }
-};
-template <> struct Pair<float> {
-  static __device__ __forceinline__ void st(float *p, float a, float b) {
-    *reinterpret_cast<float2 *>(p) = make_float2(a, b);
-  }
-};
-
 template <typename OutT>
-__global__ void __launch_bounds__(128) k_conv0(const float *__restrict__ mel, const float *__restrict__ wc,
-                                               const float *__restrict__ cov, const float *__restrict__ g0,
-                                               OutT *__restrict__ y0, const ClipTablesDev t, int64_t stem_rows) {
+__global__ void __launch_bounds__(128) k_conv0(const float *mel, const float *__restrict__ wg,
+                                               const float *__restrict__ cov, OutT *__restrict__ y0,
+                                               const ClipTablesDev t, int64_t stem_rows) {
   constexpr int P = kConv0Rows * kF1;  // positions per CTA
-  __shared__ __align__(16) float s_p[P][12];
+  __shared__ __align__(16) float2 s_pp[P][10];
   __shared__ float s_r[P];
   const int64_t row0 = (int64_t)blockIdx.x * kConv0Rows;
+  pdl_trigger();
+  pdl_wait(mel);
   for (int i = threadIdx.x; i < P; i += blockDim.x) {
     const int64_t row = row0 + i / kF1;
     const int f = i % kF1;
@@ -85,7 +78,7 @@ __global__ void __launch_bounds__(128) k_conv0(const float *__restrict__ mel, co
 #pragma unroll
           for (int df = 0; df < 3; ++df) {
             const int tr = 2 * ti + dt - 1, fr = 2 * f + df - 1;
-            if (tr >= 0 && tr < F && fr >= 0 && fr < kMels) p[dt * 3 + df] = __ldg(m + (int64_t)tr * kMels + fr);
+            if (tr >= 0 && tr < F && fr >= 0 && fr < kMels) p[dt * 3 + df] = ld_up(m + (int64_t)tr * kMels + fr);
           }
       }
     }
@@ -98,35 +91,37 @@ __global__ void __launch_bounds__(128) k_conv0(const float *__restrict__ mel, co
       var = fmaf(p[a], s, var);
     }
 #pragma unroll
-    for (int k = 0; k < 9; ++k) s_p[i][k] = p[k];
+    for (int k = 0; k < 9; ++k) s_pp[i][k] = make_float2(p[k], p[k]);
+    s_pp[i][9] = make_float2(0.f, 0.f);
     s_r[i] = rsqrtf(fmaxf(var, 0.f) + 1e-6f);
   }
   __syncthreads();
-  const int cp = threadIdx.x & 63, par = threadIdx.x >> 6;  // channels 2cp, 2cp+1; positions of parity par
-  float w0[9], w1[9];
+  const int cq = threadIdx.x & 31, ph = threadIdx.x >> 5;  // channels 4cq .. 4cq+3; positions ph, ph+4, ...
+  float2 w01[10], w23[10];
 #pragma unroll
   for (int k = 0; k < 9; ++k) {
-    w0[k] = __ldg(wc + (2 * cp) * 9 + k);
-    w1[k] = __ldg(wc + (2 * cp + 1) * 9 + k);
+    w01[k] = make_float2(__ldg(wg + (4 * cq) * 9 + k), __ldg(wg + (4 * cq + 1) * 9 + k));
+    w23[k] = make_float2(__ldg(wg + (4 * cq + 2) * 9 + k), __ldg(wg + (4 * cq + 3) * 9 + k));
   }
-  const float g0a = __ldg(g0 + 2 * cp), g0b = __ldg(g0 + 2 * cp + 1);
+  w01[9] = w23[9] = make_float2(0.f, 0.f);
   const int64_t left_pos = (stem_rows - row0) * kF1;
   const int n_pos = left_pos < P ? (int)left_pos : P;
-  OutT *out = y0 + row0 * (int64_t)(kF1 * kC0);
-#pragma unroll 4
-  for (int i = par; i < n_pos; i += 2) {
-    const float4 pa = *reinterpret_cast<const float4 *>(&s_p[i][0]);
-    const float4 pb = *reinterpret_cast<const float4 *>(&s_p[i][4]);
-    const float p8 = s_p[i][8];
-    const float r = s_r[i];
-    const float p[9] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w, p8};
-    float a = 0.f, b = 0.f;
+  OutT *out = y0 + row0 * (int64_t)(kF1 * kC0) + 4 * cq;
+#pragma unroll 2
+  for (int i = ph; i < n_pos; i += 4) {
+    float2 a = make_float2(0.f, 0.f), b = make_float2(0.f, 0.f);
+    const float4 *pp = reinterpret_cast<const float4 *>(&s_pp[i][0]);
 #pragma unroll
-    for (int k = 0; k < 9; ++k) {
-      a = fmaf(w0[k], p[k], a);
-      b = fmaf(w1[k], p[k], b);
+    for (int m = 0; m < 5; ++m) {
+      const float4 q = pp[m];
+      ffma2(a, w01[2 * m], make_float2(q.x, q.y));
+      ffma2(b, w23[2 * m], make_float2(q.x, q.y));
+      ffma2(a, w01[2 * m + 1], make_float2(q.z, q.w));
+      ffma2(b, w23[2 * m + 1], make_float2(q.z, q.w));
     }
-    Pair<OutT>::st(out + (int64_t)i * kC0 + 2 * cp, fmaxf(a * r * g0a, 0.f), fmaxf(b * r * g0b, 0.f));
+    const float r = s_r[i];
+    const float v[4] = {fmaxf(a.x * r, 0.f), fmaxf(a.y * r, 0.f), fmaxf(b.x * r, 0.f), fmaxf(b.y * r, 0.f)};
+    store4(out + (int64_t)i * kC0, v);
   }
 }
 
@@ -153,6 +148,8 @@ __global__ void __launch_bounds__(128, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile = blockIdx.x;
+  pdl_trigger();
+  pdl_wait();
   const int c = clip_of(t.conv1_tile_off, t.n_clips, tile);
   const int tok0 = (tile - t.conv1_tile_off[c]) * kConv1TileTok;
   const int n_tok = t.tok_off[c + 1] - t.tok_off[c];
@@ -273,11 +270,13 @@ __global__ void __launch_bounds__(128, 1)
 // ------------------------------------------------------------------ conv1, float32 FMA
 
 // One warp per output row (token, freq): lane = output channel.
-__global__ void __launch_bounds__(256) k_conv1_f32(const float *__restrict__ y0, const float *__restrict__ w1,
+__global__ void __launch_bounds__(256) k_conv1_f32(const float *y0, const float *__restrict__ w1,
                                                    const float *__restrict__ g1, float *__restrict__ xs,
                                                    const ClipTablesDev t, int64_t T) {
   const int64_t gw = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  pdl_trigger();
+  pdl_wait(y0);
   if (gw >= T * kF2) return;
   const int64_t tokg = gw / kF2;
   const int f = (int)(gw % kF2);
@@ -311,10 +310,10 @@ cudaError_t launch_conv0(const ae_model *m, const float *mel, void *y0, const Cl
   if (stem_rows <= 0) return cudaSuccess;
   const unsigned grid = (unsigned)((stem_rows + kConv0Rows - 1) / kConv0Rows);
   if (m->dtype == AE_BF16)
-    k_conv0<bf16><<<grid, 128, 0, s>>>(mel, m->conv0c, m->conv0cov, m->ln0, static_cast<bf16 *>(y0), t, stem_rows);
-  else
-    k_conv0<float><<<grid, 128, 0, s>>>(mel, m->conv0c, m->conv0cov, m->ln0, static_cast<float *>(y0), t, stem_rows);
-  return cudaGetLastError();
+    return launch_k(k_conv0<bf16>, dim3(grid), dim3(128), 0, s, mel, (const float *)m->conv0c,
+                    (const float *)m->conv0cov, static_cast<bf16 *>(y0), t, stem_rows);
+  return launch_k(k_conv0<float>, dim3(grid), dim3(128), 0, s, mel, (const float *)m->conv0c,
+                  (const float *)m->conv0cov, static_cast<float *>(y0), t, stem_rows);
 }
 
 cudaError_t launch_conv1(const ae_model *m, const void *y0, int64_t stem_rows, void *xs, const ClipTablesDev &t,
@@ -329,15 +328,12 @@ cudaError_t launch_conv1(const ae_model *m, const void *y0, int64_t stem_rows, v
     }
     CUtensorMap tmY;
     if (!make_tmap_stem_y0(&tmY, y0, stem_rows)) return cudaErrorInvalidValue;
-    k_conv1_tc<<<(unsigned)conv1_tiles, 128, C1_SMEM, s>>>(tmY, m->tm_conv1, t, m->ln1, static_cast<bf16 *>(xs),
-                                                            device_status_word());
-  } else {
-    const int64_t warps = tokens * kF2;
-    k_conv1_f32<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(static_cast<const float *>(y0),
-                                                             static_cast<const float *>(m->conv1), m->ln1,
-                                                             static_cast<float *>(xs), t, tokens);
+    return launch_k(k_conv1_tc, dim3((unsigned)conv1_tiles), dim3(128), C1_SMEM, s, tmY, m->tm_conv1, t,
+                    (const float *)m->ln1, static_cast<bf16 *>(xs), device_status_word());
   }
-  return cudaGetLastError();
+  const int64_t warps = tokens * kF2;
+  return launch_k(k_conv1_f32, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0, s, static_cast<const float *>(y0),
+                  static_cast<const float *>(m->conv1), (const float *)m->ln1, static_cast<float *>(xs), t, tokens);
 }
 
 }  // namespace ae
