@@ -160,7 +160,7 @@ bool make_tmap_2d_bf16(CUtensorMap *tm, const void *base, uint64_t inner, uint64
                        uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
 bool make_tmap_stem_y0(CUtensorMap *tm, const void *y0, int64_t stem_rows);
 
-// Launch with programmatic stream serialization (see pdl_wait/pdl_trigger).
+// Launch on stream s; the arguments are converted to the kernel's parameter types.
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                             Args &&...args) {
@@ -169,11 +169,6 @@ inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, siz
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
 }
 

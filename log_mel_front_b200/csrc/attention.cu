@@ -37,21 +37,21 @@ __device__ __forceinline__ const uint4 *a2_chunk(const bf16 *buf, int r, int c) 
   return reinterpret_cast<const uint4 *>(buf + r * kHeadDim) + (c ^ ((r >> 1) & 7));
 }
 
-__device__ __forceinline__ void a2_stage(bf16 *buf, const bf16 *src, int64_t ld, int h, int64_t t0,
+__device__ __forceinline__ void a2_stage(bf16 *buf, const bf16 *__restrict__ src, int64_t ld, int h, int64_t t0,
                                          int64_t T) {
   for (int idx = threadIdx.x; idx < A2_ROWS * 16; idx += A2_THREADS) {
     const int r = idx >> 4, c = idx & 15;
     const int64_t tok = t0 - (kLeft - 1) + r;
     uint4 v = make_uint4(0, 0, 0, 0);
-    if (tok >= 0 && tok < T) v = ld_up(reinterpret_cast<const uint4 *>(src + tok * ld + h * kHeadDim) + c);
+    if (tok >= 0 && tok < T) v = __ldg(reinterpret_cast<const uint4 *>(src + tok * ld + h * kHeadDim) + c);
     reinterpret_cast<uint4 *>(buf + r * kHeadDim)[c ^ ((r >> 1) & 7)] = v;
   }
 }
 
 __global__ void __launch_bounds__(A2_THREADS, 3)
-    k_attention_bf16(const bf16 *q, const bf16 *k, const bf16 *v, int64_t ld,
+    k_attention_bf16(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const bf16 *__restrict__ v, int64_t ld,
                      const float *__restrict__ R, const float *__restrict__ qscale, float k_scale, float cap,
-                     const int32_t *pos, int64_t T, bf16 *__restrict__ out, int64_t ld_out, float lo,
+                     const int32_t *__restrict__ pos, int64_t T, bf16 *__restrict__ out, int64_t ld_out, float lo,
                      float hi) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   bf16 *buf = reinterpret_cast<bf16 *>(smem_raw);
@@ -60,12 +60,10 @@ __global__ void __launch_bounds__(A2_THREADS, 3)
   const int h = blockIdx.y;
   const int64_t t0 = (int64_t)blockIdx.x * A2_TOK;
   const int i = threadIdx.x;
-  pdl_trigger();
   const float inv_ks = 1.0f / k_scale;
   for (int x = i; x < kLeft * kHeadDim; x += A2_THREADS)
     Rt[x] = R[(x / kHeadDim) * kHidden + h * kHeadDim + x % kHeadDim] * inv_ks;
   Qs[i] = qscale[i];
-  pdl_wait(q, k, v, pos);
   a2_stage(buf, k, ld, h, t0, T);
   __syncthreads();
 
@@ -81,18 +79,18 @@ __global__ void __launch_bounds__(A2_THREADS, 3)
 #pragma unroll
   for (int d = 0; d < kLeft; ++d) acc[0][d] = acc[1][d] = make_float2(0.f, 0.f);
   // q of the next chunk is loaded while the current one is used
-  uint4 na0 = ld_up(reinterpret_cast<const uint4 *>(qa_row)), na1 = ld_up(reinterpret_cast<const uint4 *>(qa_row) + 1);
-  uint4 nb0 = ld_up(reinterpret_cast<const uint4 *>(qb_row)), nb1 = ld_up(reinterpret_cast<const uint4 *>(qb_row) + 1);
+  uint4 na0 = __ldg(reinterpret_cast<const uint4 *>(qa_row)), na1 = __ldg(reinterpret_cast<const uint4 *>(qa_row) + 1);
+  uint4 nb0 = __ldg(reinterpret_cast<const uint4 *>(qb_row)), nb1 = __ldg(reinterpret_cast<const uint4 *>(qb_row) + 1);
 #pragma unroll 1
   for (int cc = 0; cc < kHeadDim / 16; ++cc) {
     float2 qa[8], qb[8];
     {
       const uint4 a0 = na0, a1 = na1, b0 = nb0, b1 = nb1;
       if (cc + 1 < kHeadDim / 16) {
-        na0 = ld_up(reinterpret_cast<const uint4 *>(qa_row + (cc + 1) * 16));
-        na1 = ld_up(reinterpret_cast<const uint4 *>(qa_row + (cc + 1) * 16) + 1);
-        nb0 = ld_up(reinterpret_cast<const uint4 *>(qb_row + (cc + 1) * 16));
-        nb1 = ld_up(reinterpret_cast<const uint4 *>(qb_row + (cc + 1) * 16) + 1);
+        na0 = __ldg(reinterpret_cast<const uint4 *>(qa_row + (cc + 1) * 16));
+        na1 = __ldg(reinterpret_cast<const uint4 *>(qa_row + (cc + 1) * 16) + 1);
+        nb0 = __ldg(reinterpret_cast<const uint4 *>(qb_row + (cc + 1) * 16));
+        nb1 = __ldg(reinterpret_cast<const uint4 *>(qb_row + (cc + 1) * 16) + 1);
       }
       const uint32_t wa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
       const uint32_t wb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
@@ -204,10 +202,10 @@ constexpr int kRows = kTQ + kLeft - 1;   // staged k/v rows
 constexpr int kPitchF = kHeadDim + 4;    // floats per staged row (528 bytes)
 }  // namespace
 
-__global__ void __launch_bounds__(kTQ) k_attention_f32(const float *q, const float *k,
-                                                       const float *v, int64_t ld,
+__global__ void __launch_bounds__(kTQ) k_attention_f32(const float *__restrict__ q, const float *__restrict__ k,
+                                                       const float *__restrict__ v, int64_t ld,
                                                        const float *__restrict__ R, const float *__restrict__ qscale,
-                                                       float k_scale, float cap, const int32_t *pos,
+                                                       float k_scale, float cap, const int32_t *__restrict__ pos,
                                                        int64_t T_total, float *__restrict__ out, int64_t ld_out,
                                                        float lo, float hi) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -218,8 +216,6 @@ __global__ void __launch_bounds__(kTQ) k_attention_f32(const float *q, const flo
   const int h = blockIdx.y;
   const int64_t t0 = (int64_t)blockIdx.x * kTQ;
   const int tid = threadIdx.x;
-  pdl_trigger();
-  pdl_wait(q, k, v, pos);
   for (int idx = tid; idx < kRows * (kHeadDim / 4); idx += kTQ) {
     const int r = idx / (kHeadDim / 4), ch = idx % (kHeadDim / 4);
     const int64_t tok = t0 - (kLeft - 1) + r;

@@ -29,36 +29,6 @@ __device__ __forceinline__ unsigned long long global_ns() {
   return t;
 }
 
-// ----------------------------------------------------------------- programmatic dependent launch
-// Every kernel of the library is launched with programmatic stream
-// serialization: it lets the next kernel in the stream start launching
-// (pdl_trigger, at the top of each kernel) and waits for the previous one to
-// complete and flush (pdl_wait) before its first access to data another
-// kernel writes or reads. Work before pdl_wait touches only the model's
-// weights and the kernel's own shared/tensor memory. Without the launch
-// attribute both are no-ops.
-//
-// The asm's memory clobber orders ordinary loads, but a load the compiler
-// deems invariant (read-only for the whole kernel, as through a
-// `const __restrict__` parameter or __ldg) may still be scheduled above it,
-// and would then read the previous kernel's output before it is complete.
-// So pointers to data that other kernels produce are passed to pdl_wait:
-// it routes each through an opaque asm after the wait, which makes every
-// address computed from them a value that only exists once the wait is over
-// and strips the read-only provenance. Those parameters carry no
-// __restrict__ and are not read with __ldg.
-template <typename T>
-__device__ __forceinline__ void opaque_ptr(T *&p) { asm volatile("" : "+l"(p)); }
-template <typename... P>
-__device__ __forceinline__ void pdl_wait(P *&...p) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  (opaque_ptr(p), ...);
-}
-// A load of data another kernel produced (an ordinary, coherent load).
-template <typename T>
-__device__ __forceinline__ T ld_up(const T *p) { return *p; }
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
 // ----------------------------------------------------------------- bf16 helpers
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }

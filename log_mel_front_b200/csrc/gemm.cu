@@ -130,7 +130,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   const int m_blocks = (M + 2 * BM - 1) / (2 * BM), n_blocks = N / BN, kb_n = K / BK;
   const int num_tiles = m_blocks * n_blocks;
   const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
-  pdl_trigger();
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -155,7 +154,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   cluster_sync();  // both CTAs' barriers are initialised before any cross-CTA arrival
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  pdl_wait();  // x (and the output buffer) belong to the previous kernels until here
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer (both CTAs)
@@ -292,12 +290,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
 // ------------------------------------------------------------------ f32 FMA kernel
 
 template <int MODE>
-__global__ void __launch_bounds__(256) k_gemm_f32(const float *A, const float *__restrict__ B,
+__global__ void __launch_bounds__(256) k_gemm_f32(const float *__restrict__ A, const float *__restrict__ B,
                                                   const EpiArgs ep, int M, int N, int K) {
   __shared__ float As[16][64 + 4];
   __shared__ float Bs[16][64 + 4];
-  pdl_trigger();
-  pdl_wait(A);
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
   float acc[4][4] = {};

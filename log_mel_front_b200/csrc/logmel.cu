@@ -84,11 +84,10 @@ __device__ __forceinline__ void dft16(float2 (&x)[16]) {
 }
 
 __global__ void __launch_bounds__(kThreads, 2)
-    k_logmel(const float *wave, float *__restrict__ mel, const ClipTablesDev t, int n_tiles) {
+    k_logmel(const float *__restrict__ wave, float *__restrict__ mel, const ClipTablesDev t, int n_tiles) {
   extern __shared__ uint8_t smem_raw[];
   LogmelSmem &S = *reinterpret_cast<LogmelSmem *>(smem_raw);
   const int tid = threadIdx.x;
-  pdl_trigger();
 
   // ---- tables, float64 from their definitions
   for (int m = tid; m < kFft; m += kThreads) {
@@ -133,7 +132,6 @@ __global__ void __launch_bounds__(kThreads, 2)
   for (int k1 = 0; k1 < 16; ++k1) tw1[k1] = S.tw[(2 * j * k1) & (kFft - 1)];
   float2 *xs = S.xs[g];
   float *mag = S.mag[g];
-  pdl_wait(wave);  // the tables above are built from constants; the clip tables and the wave come from upstream
 
   for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
     __syncthreads();  // previous work item done with the staged wave
@@ -157,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int span = nf * kHop + kHop;
     for (int i = tid; i < span; i += kThreads) {
       const int64_t sidx = first + i;
-      S.wave[i] = (sidx >= 0 && sidx < n_samp) ? ld_up(wave + s_begin + sidx) : 0.0f;
+      S.wave[i] = (sidx >= 0 && sidx < n_samp) ? __ldg(wave + s_begin + sidx) : 0.0f;
     }
     __syncthreads();
 

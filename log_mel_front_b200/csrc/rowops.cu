@@ -38,13 +38,11 @@ __global__ void __launch_bounds__(256, NV <= 8 ? 3 : 2) k_rowop(const RowArgs r)
   const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   const bool live = row < r.rows;
-  pdl_trigger();
-  for (int i = threadIdx.x; i < W / 4; i += blockDim.x) {  // weights: independent of upstream kernels
+  for (int i = threadIdx.x; i < W / 4; i += blockDim.x) {  // the norm weights this pass uses
     if (r.wy) reinterpret_cast<float4 *>(s_wy)[i] = __ldg(reinterpret_cast<const float4 *>(r.wy) + i);
     if (r.w_out) reinterpret_cast<float4 *>(s_wo)[i] = __ldg(reinterpret_cast<const float4 *>(r.w_out) + i);
     if (r.w_next) reinterpret_cast<float4 *>(s_wn)[i] = __ldg(reinterpret_cast<const float4 *>(r.w_next) + i);
   }
-  pdl_wait();
   float *hrow = r.h + (live ? row : 0) * W;
   float h[NV][4], y[NV][4];
   if (live) {
@@ -146,19 +144,17 @@ constexpr int kLcRows = 8;
 constexpr int kLcHalo = kKernel - 1;
 
 template <typename ActT>
-__global__ void __launch_bounds__(256) k_lconv(const ActT *gl, const float *__restrict__ w_dw,
+__global__ void __launch_bounds__(256) k_lconv(const ActT *__restrict__ gl, const float *__restrict__ w_dw,
                                                const float *__restrict__ w_norm, float lo, float hi,
-                                               ActT *__restrict__ out, const int32_t *pos, int64_t T) {
+                                               ActT *__restrict__ out, const int32_t *__restrict__ pos, int64_t T) {
   __shared__ float s_ss[8][kLcRows];
   __shared__ float s_inv[kLcRows];
   const int ch = 4 * threadIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t t0 = (int64_t)blockIdx.x * kLcRows;
-  pdl_trigger();
   float w[kKernel][4], wn[4];
 #pragma unroll
   for (int k = 0; k < kKernel; ++k) load4(w_dw + k * kHidden + ch, w[k]);
   load4(w_norm + ch, wn);
-  pdl_wait(gl, pos);
   float x[kLcRows + kLcHalo][4];
 #pragma unroll
   for (int r = 0; r < kLcRows + kLcHalo; ++r) {
@@ -236,15 +232,11 @@ struct UploadChunk {
 };
 
 __global__ void k_upload(uint8_t *base, const UploadChunk ch) {
-  pdl_trigger();
-  pdl_wait();
   uint32_t *d = reinterpret_cast<uint32_t *>(base + ch.dst);
   for (int i = threadIdx.x; i < ch.n; i += blockDim.x) d[i] = ch.w[i];
 }
 
 __global__ void k_pos(int32_t *pos, const int32_t *tok_off) {
-  pdl_trigger();
-  pdl_wait();
   const int c = blockIdx.x;
   const int b = tok_off[c], n = tok_off[c + 1] - b;
   for (int i = threadIdx.x; i < n; i += blockDim.x) pos[b + i] = i;

@@ -52,15 +52,13 @@ __device__ __forceinline__ int clip_of(const int32_t *off, int n_clips, int64_t 
 constexpr int kConv0Rows = 4;
 
 template <typename OutT>
-__global__ void __launch_bounds__(128) k_conv0(const float *mel, const float *__restrict__ wg,
+__global__ void __launch_bounds__(128) k_conv0(const float *__restrict__ mel, const float *__restrict__ wg,
                                                const float *__restrict__ cov, OutT *__restrict__ y0,
                                                const ClipTablesDev t, int64_t stem_rows) {
   constexpr int P = kConv0Rows * kF1;  // positions per CTA
   __shared__ __align__(16) float2 s_pp[P][10];
   __shared__ float s_r[P];
   const int64_t row0 = (int64_t)blockIdx.x * kConv0Rows;
-  pdl_trigger();
-  pdl_wait(mel);
   for (int i = threadIdx.x; i < P; i += blockDim.x) {
     const int64_t row = row0 + i / kF1;
     const int f = i % kF1;
@@ -78,7 +76,7 @@ __global__ void __launch_bounds__(128) k_conv0(const float *mel, const float *__
 #pragma unroll
           for (int df = 0; df < 3; ++df) {
             const int tr = 2 * ti + dt - 1, fr = 2 * f + df - 1;
-            if (tr >= 0 && tr < F && fr >= 0 && fr < kMels) p[dt * 3 + df] = ld_up(m + (int64_t)tr * kMels + fr);
+            if (tr >= 0 && tr < F && fr >= 0 && fr < kMels) p[dt * 3 + df] = __ldg(m + (int64_t)tr * kMels + fr);
           }
       }
     }
@@ -148,8 +146,6 @@ __global__ void __launch_bounds__(128, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile = blockIdx.x;
-  pdl_trigger();
-  pdl_wait();
   const int c = clip_of(t.conv1_tile_off, t.n_clips, tile);
   const int tok0 = (tile - t.conv1_tile_off[c]) * kConv1TileTok;
   const int n_tok = t.tok_off[c + 1] - t.tok_off[c];
@@ -270,13 +266,11 @@ __global__ void __launch_bounds__(128, 1)
 // ------------------------------------------------------------------ conv1, float32 FMA
 
 // One warp per output row (token, freq): lane = output channel.
-__global__ void __launch_bounds__(256) k_conv1_f32(const float *y0, const float *__restrict__ w1,
+__global__ void __launch_bounds__(256) k_conv1_f32(const float *__restrict__ y0, const float *__restrict__ w1,
                                                    const float *__restrict__ g1, float *__restrict__ xs,
                                                    const ClipTablesDev t, int64_t T) {
   const int64_t gw = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  pdl_trigger();
-  pdl_wait(y0);
   if (gw >= T * kF2) return;
   const int64_t tokg = gw / kF2;
   const int f = (int)(gw % kF2);
