@@ -224,6 +224,30 @@ class Ours:
             return self.h_wave.numel() * 4, self.h_mel.numel() * 4
         return 0, 0
 
+    def e2e_pipelined(self, k: int) -> float:
+        """k steps through ae_encode_host_async on two streams, each with its own
+        workspace and pinned output buffer, so one step's host copies overlap the
+        other's kernels; returns the device time of all k steps in ms (events on
+        the first stream, after it has joined the second)."""
+        ae, torch = self.ae, self.torch
+        if not hasattr(self, "ws2"):
+            self.ws2 = torch.empty_like(self.ws)
+            self.h_out2 = torch.empty_like(self.h_out).pin_memory()
+            self.stream2 = torch.cuda.Stream()
+        slots = [(self.stream, self.ws, self.h_out), (self.stream2, self.ws2, self.h_out2)]
+        torch.cuda.synchronize()
+        a, b, j = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        a.record(self.stream)
+        self.stream2.wait_event(a)
+        for i in range(k):
+            s, ws, out = slots[i % 2]
+            ae.ae_encode_host_async(self.model, self.h_wave, self.off, out, ws, ws.numel(), s)
+        j.record(self.stream2)
+        self.stream.wait_event(j)
+        b.record(self.stream)
+        b.synchronize()
+        return a.elapsed_time(b)
+
     def timed(self, k: int, fn):
         torch = self.torch
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k)]
@@ -319,13 +343,19 @@ def run_ours(args, rank, world, dist):
     # per-kernel-class timing over a replica of the timed region (events around every launch)
     ae.ae_profile_enable(True)
     ae.ae_profile_read()
-    ms_prof = ours.timed(args.steps, ours.step)
+    # at most 40 steps: the library keeps 16384 launch records
+    prof_steps = min(args.steps, 40)
+    ms_prof = ours.timed(prof_steps, ours.step)
     prof = ae.ae_profile_read()
     ae.ae_profile_enable(False)
     # end to end through the host-buffer entry point
     h2d = d2h = 0
     ms_e2e = None
-    if args.workload != "attention":
+    if args.workload in ("tower", "ragged"):
+        ours.e2e_pipelined(2)
+        ms_e2e = ours.e2e_pipelined(args.steps)
+        h2d, d2h = ours.h_wave.numel() * 4, ours.h_out.numel() * 4
+    elif args.workload != "attention":
         ours.step_e2e()
         torch.cuda.synchronize()
         sizes = []
@@ -333,11 +363,12 @@ def run_ours(args, rank, world, dist):
         def e2e():
             sizes.append(ours.step_e2e())
         ms_e2e = ours.timed(args.steps, e2e)
+        h2d, d2h = sizes[0]
+    if ms_e2e is not None:
         if dist:
             t = torch.tensor([ms_e2e], device="cuda")
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             ms_e2e = float(t.item())
-        h2d, d2h = sizes[0]
     if rank != 0:
         return None
     pk = peaks()
@@ -360,9 +391,9 @@ def run_ours(args, rank, world, dist):
                  "achieved": round(achieved, 2), "peak": peak, "frac": round(achieved / peak, 4),
                  "traffic": None if traffic is None else round(traffic), "traffic_source": traffic_src,
                  "algorithmic_bytes_per_launch": round(dom["bytes"] / max(dom["launches"], 1)),
-                 "launches_per_step": dom["launches"] / args.steps,
+                 "launches_per_step": dom["launches"] / prof_steps,
                  "share_of_step": round(dom["ms"] / max(ms_prof, 1e-9), 4)})
-    classes = {k: {"ms_per_step": round(v["ms"] / args.steps, 4), "launches_per_step": v["launches"] / args.steps,
+    classes = {k: {"ms_per_step": round(v["ms"] / prof_steps, 4), "launches_per_step": v["launches"] / prof_steps,
                    **({"tflops": round(v["flops"] / (v["ms"] / 1e3) / 1e12, 1)} if v["flops"] and v["ms"] else {}),
                    **({"gbs": round(v["bytes"] / (v["ms"] / 1e3) / 1e9, 1)} if v["bytes"] and v["ms"] else {})}
                for k, v in prof.items() if k != "dropped" and v["launches"]}
@@ -377,11 +408,12 @@ def run_ours(args, rank, world, dist):
         "e2e": None if ms_e2e is None else {
             "value": round(audio / (ms_e2e / args.steps / 1e3), 2), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "api": "ae_encode_host" if args.workload in ("tower", "ragged") else "ae_logmel + copies"},
-        "gpu_launches": int(launches),
+            "api": ("ae_encode_host_async, two streams (copies of one step overlap the kernels of the other)"
+                    if args.workload in ("tower", "ragged") else "ae_logmel + copies")},
+        "gpu_launches": int(round(launches / prof_steps * args.steps)),
         "roofline": roof,
         "kernel_classes": classes,
-        "profiled_ms_per_step": round(ms_prof / args.steps, 4),
+        "profiled_ms_per_step": round(ms_prof / prof_steps, 4),
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:

@@ -157,7 +157,9 @@ ae_status ae_logmel(const float *d_wave, const int64_t *h_sample_off, int n_clip
  * bias-free LayerNorm over channels (eps 1e-6), ReLU; 3x3 stride-2 conv
  * c0 -> c1, LayerNorm, ReLU; flatten frequency-major (f * c1 + c); times
  * in_proj^T (no bias, no clamp). d_mel: float32 [h_frame_off[n_clips]][128].
- * d_h: float32 [sum tokens][hidden], the residual stream entering layer 0. */
+ * d_h: float32 [sum tokens][hidden], the residual stream entering layer 0,
+ * 16-byte aligned (the projection writes it with TMA stores; AE_EINVAL
+ * otherwise). */
 ae_status ae_subsample(const ae_model *m, const float *d_mel, const int64_t *h_frame_off,
                        int n_clips, float *d_h, void *d_ws, size_t ws_bytes, ae_stream stream);
 
@@ -178,7 +180,8 @@ ae_status ae_conformer_layer(const ae_model *m, int layer, float *d_h, const int
 /* The whole forward (AudioTower::soft_tokens for one packed batch):
  * log-mel, stem, in_proj, every layer, then out_proj + bias, a weightless
  * RMS norm and embed. d_wave: float32 [h_sample_off[n_clips]]. d_out:
- * float32 [sum tokens][embed_dim], clip after clip. */
+ * float32 [sum tokens][embed_dim], clip after clip, 16-byte aligned (the
+ * projection writes it with TMA stores; AE_EINVAL otherwise). */
 ae_status ae_encode(const ae_model *m, const float *d_wave, const int64_t *h_sample_off,
                     int n_clips, float *d_out, void *d_ws, size_t ws_bytes, ae_stream stream);
 
@@ -190,6 +193,14 @@ ae_status ae_encode(const ae_model *m, const float *d_wave, const int64_t *h_sam
 size_t ae_encode_host_workspace_size(const ae_model *m, const int64_t *h_sample_off, int n_clips);
 ae_status ae_encode_host(const ae_model *m, const float *h_wave, const int64_t *h_sample_off,
                          int n_clips, float *h_out, void *d_ws, size_t ws_bytes, ae_stream stream);
+
+/* ae_encode_host without the final wait: the copies and kernels are only
+ * enqueued on `stream`. h_wave, h_out and d_ws belong to the call until the
+ * stream has reached this point (synchronize it, or wait on an event recorded
+ * after the call). Calls on different streams with their own workspaces and
+ * output buffers overlap one batch's copies with another's kernels. */
+ae_status ae_encode_host_async(const ae_model *m, const float *h_wave, const int64_t *h_sample_off,
+                               int n_clips, float *h_out, void *d_ws, size_t ws_bytes, ae_stream stream);
 
 /* --- the attention core alone ------------------------------------------------ */
 

@@ -78,6 +78,7 @@ _sig("ae_conformer_layer", _st, _vp, _i32, _vp, _i64p, _i32, _vp, _sz, _vp)
 _sig("ae_encode", _st, _vp, _vp, _i64p, _i32, _vp, _vp, _sz, _vp)
 _sig("ae_encode_host_workspace_size", _sz, _vp, _i64p, _i32)
 _sig("ae_encode_host", _st, _vp, _vp, _i64p, _i32, _vp, _vp, _sz, _vp)
+_sig("ae_encode_host_async", _st, _vp, _vp, _i64p, _i32, _vp, _vp, _sz, _vp)
 _sig("ae_attention_tables", _st, _fp, _fp, _i32, _i32, _i32, _fp, _fp, _fp)
 _sig("ae_local_attention", _st, _vp, _vp, _vp, C.c_int64, _i32, _vp, _vp, C.c_float, C.c_float, _i64p, _i32,
      _vp, C.c_int64, _vp, _sz, _vp)
@@ -91,7 +92,7 @@ _sig("ae_profile_read", _st, C.POINTER(C.c_double), _i64p, C.POINTER(C.c_double)
 # every symbol include/ae.h declares
 EXPORTS = ("ae_num_frames", "ae_num_tokens", "ae_model_create", "ae_model_destroy", "ae_workspace_size",
            "ae_logmel", "ae_subsample", "ae_conformer_layer", "ae_encode", "ae_encode_host_workspace_size",
-           "ae_encode_host", "ae_attention_tables", "ae_local_attention", "ae_last_error", "ae_device_status",
+           "ae_encode_host", "ae_encode_host_async", "ae_attention_tables", "ae_local_attention", "ae_last_error", "ae_device_status",
            "ae_version", "ae_profile_enable", "ae_profile_read", "ae_logmel_noalloc")
 
 KERNEL_CLASSES = ("tables", "logmel", "conv0", "conv1", "gemm", "attention", "lconv", "rowop")
@@ -194,6 +195,14 @@ def ae_encode_host(model, h_wave, sample_off, h_out, d_ws, ws_bytes: int, stream
     a, p = _off(sample_off)
     _check(lib.ae_encode_host(model.handle, _ptr(h_wave), p, len(a) - 1, _ptr(h_out), _ptr(d_ws), ws_bytes,
                               _stream(stream)), "ae_encode_host")
+
+
+def ae_encode_host_async(model, h_wave, sample_off, h_out, d_ws, ws_bytes: int, stream=None):
+    """Enqueues ae_encode_host on `stream` without waiting; the buffers belong
+    to the call until the stream has passed it."""
+    a, p = _off(sample_off)
+    _check(lib.ae_encode_host_async(model.handle, _ptr(h_wave), p, len(a) - 1, _ptr(h_out), _ptr(d_ws), ws_bytes,
+                                    _stream(stream)), "ae_encode_host_async")
 
 
 def ae_attention_tables(relative_k, per_dim_scale, hidden: int = 1024, heads: int = 8, left: int = 12):

@@ -134,12 +134,12 @@ cudaError_t gemm(const ae_model *m, const void *x, int64_t M, int K, const void 
                  int N, int mode, const EpiArgs &ep, cudaStream_t s);
 
 // Row update of the residual stream (one warp per row of `width` floats):
-//   if y:      h += s * (y_norm ? rms(y) * wy : y)
+//   if y:      h += s * (y_norm ? rms(y) * wy : y)   (y in the model's act type)
 //   if w_out:  h = rms(h) * w_out
 //   write h back if anything changed it
 //   if a_out:  a = clamp(rms(h) * w_next, lo, hi)  (act type of the model)
 struct RowArgs {
-  float *h; const float *y; const float *wy; float s; int y_norm;
+  float *h; const void *y; const float *wy; float s; int y_norm;
   const float *w_out;
   void *a_out; const float *w_next; int a_rms; float lo, hi;
   int width; int64_t rows;

@@ -120,7 +120,8 @@ static cudaError_t conv1_t(const ae_model *m, const void *y0, void *xs, const Cl
 static cudaError_t rowop_t(const ae_model *m, const RowArgs &r, cudaStream_t s) {
   const double W = r.width;
   const bool changed = r.y || r.w_out;
-  double per_row = 4.0 * W * (1.0 + (changed ? 1.0 : 0.0) + (r.y ? 1.0 : 0.0));
+  double per_row = 4.0 * W * (1.0 + (changed ? 1.0 : 0.0));  // h read, written back if changed
+  if (r.y) per_row += W * (double)act_bytes(m);
   if (r.a_out) per_row += W * (double)act_bytes(m);
   return timed(AE_K_ROWOP, 0.0, per_row * (double)r.rows, s, [&] { return launch_rowop(m, r, s); });
 }
@@ -327,6 +328,9 @@ static cudaError_t run_layer(const ae_model *m, int li, const Bufs &b, int64_t T
   const float rw = m->cfg.residual_weight;
   const size_t act = m->dtype == AE_BF16 ? 2 : 4;
   const bool tc = m->dtype == AE_BF16;
+  // the projections whose outputs feed a row pass write them in the act type
+  // (bf16 for the tensor-core model): the row pass is bound by its bytes
+  const int y_mode = tc ? EPI_BF16 : EPI_F32;
   if (!a_ready) {
     RowArgs r = row_of(b.h, H, T);
     r.a_out = b.a;
@@ -341,7 +345,7 @@ static cudaError_t run_layer(const ae_model *m, int li, const Bufs &b, int64_t T
     e1.lo2 = c2.lo_in;
     e1.hi2 = c2.hi_in;
     AE_TRY(gemm_t(m,b.a, T, H, w1, tc ? t1 : nullptr, F, EPI_SILU, e1, s));
-    return gemm_t(m, b.big, T, F, w2, tc ? t2 : nullptr, H, EPI_F32, ep_of(b.y, H, c2.lo_out, c2.hi_out), s);
+    return gemm_t(m, b.big, T, F, w2, tc ? t2 : nullptr, H, y_mode, ep_of(b.y, H, c2.lo_out, c2.hi_out), s);
   };
   // ---- FFN1
   AE_TRY(ffn(L.ff1_w1, &L.tm_ff1_w1, L.c_ff1_w1, L.ff1_w2, &L.tm_ff1_w2, L.c_ff1_w2));
@@ -364,8 +368,8 @@ static cudaError_t run_layer(const ae_model *m, int li, const Bufs &b, int64_t T
       return launch_attention(tc, qkv, qkv + act * H, qkv + 2 * act * H, 3 * H, L.R, L.qscale, m->k_scale,
                               m->cfg.softcap, b.pos, T, b.o, H, L.c_post.lo_in, L.c_post.hi_in, s);
     }));
-    AE_TRY(gemm_t(m,b.o, T, H, L.post, tc ? &L.tm_post : nullptr, H, EPI_F32,
-                ep_of(b.y, H, L.c_post.lo_out, L.c_post.hi_out), s));
+    AE_TRY(gemm_t(m, b.o, T, H, L.post, tc ? &L.tm_post : nullptr, H, y_mode,
+                  ep_of(b.y, H, L.c_post.lo_out, L.c_post.hi_out), s));
     RowArgs r = row_of(b.h, H, T);
     r.y = b.y; r.wy = L.norm_post_attn; r.s = 1.0f; r.y_norm = 1;
     r.a_out = b.a; r.w_next = L.lc_pre; r.lo = L.c_lc_start.lo_in; r.hi = L.c_lc_start.hi_in;
@@ -378,8 +382,8 @@ static cudaError_t run_layer(const ae_model *m, int li, const Bufs &b, int64_t T
     AE_TRY(timed(AE_K_LCONV, 0.0, (double)T * 2 * H * act, s, [&] {
       return launch_lconv(m, b.big, L.lc_dw, L.lc_norm, L.c_lc_end.lo_in, L.c_lc_end.hi_in, b.o, b.pos, T, s);
     }));
-    AE_TRY(gemm_t(m,b.o, T, H, L.lc_end, tc ? &L.tm_lc_end : nullptr, H, EPI_F32,
-                ep_of(b.y, H, L.c_lc_end.lo_out, L.c_lc_end.hi_out), s));
+    AE_TRY(gemm_t(m, b.o, T, H, L.lc_end, tc ? &L.tm_lc_end : nullptr, H, y_mode,
+                  ep_of(b.y, H, L.c_lc_end.lo_out, L.c_lc_end.hi_out), s));
     RowArgs r = row_of(b.h, H, T);
     r.y = b.y; r.s = 1.0f; r.y_norm = 0;
     r.a_out = b.a; r.w_next = L.ff2_pre; r.lo = L.c_ff2_w1.lo_in; r.hi = L.c_ff2_w1.hi_in;
@@ -737,6 +741,7 @@ ae_status ae_subsample(const ae_model *m, const float *d_mel, const int64_t *h_f
   ClipTables T;
   if ((st = build_tables(h_frame_off, n_clips, kFrames, T, "h_frame_off"))) return st;
   if (T.total_tokens > 0 && (!d_mel || !d_h)) return fail(AE_EINVAL, "d_mel or d_h is null");
+  if (!aligned16(d_h)) return fail(AE_EINVAL, "d_h is not 16-byte aligned");
   const WsLayout L = ws_layout(m, T.n_clips, T.total_frames, T.total_tokens, true);
   if (n_clips == 0) return AE_OK;
   if ((st = check_ws(d_ws, ws_bytes, L.total))) return st;
@@ -783,6 +788,7 @@ ae_status ae_encode(const ae_model *m, const float *d_wave, const int64_t *h_sam
   ClipTables T;
   if ((st = build_tables(h_sample_off, n_clips, kSamples, T, "h_sample_off"))) return st;
   if (T.total_tokens > 0 && (!d_wave || !d_out)) return fail(AE_EINVAL, "d_wave or d_out is null");
+  if (!aligned16(d_out)) return fail(AE_EINVAL, "d_out is not 16-byte aligned");
   const WsLayout L = ws_layout(m, T.n_clips, T.total_frames, T.total_tokens, true);
   if (n_clips == 0) return AE_OK;
   if ((st = check_ws(d_ws, ws_bytes, L.total))) return st;
@@ -796,8 +802,8 @@ size_t ae_encode_host_workspace_size(const ae_model *m, const int64_t *h_sample_
   return L.total + al256((size_t)T.total_samples * 4) + al256((size_t)T.total_tokens * m->cfg.embed_dim * 4);
 }
 
-ae_status ae_encode_host(const ae_model *m, const float *h_wave, const int64_t *h_sample_off, int n_clips,
-                         float *h_out, void *d_ws, size_t ws_bytes, ae_stream stream) {
+ae_status ae_encode_host_async(const ae_model *m, const float *h_wave, const int64_t *h_sample_off, int n_clips,
+                               float *h_out, void *d_ws, size_t ws_bytes, ae_stream stream) {
   ae_status st = check_model(m);
   if (st) return st;
   ClipTables T;
@@ -822,7 +828,15 @@ ae_status ae_encode_host(const ae_model *m, const float *h_wave, const int64_t *
       (e = cudaMemcpyAsync(h_out, d_out, (size_t)T.total_tokens * m->cfg.embed_dim * 4, cudaMemcpyDeviceToHost, s)) !=
           cudaSuccess)
     return cuda_fail(e, "copy out");
-  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_fail(e, "stream");
+  return AE_OK;
+}
+
+ae_status ae_encode_host(const ae_model *m, const float *h_wave, const int64_t *h_sample_off, int n_clips,
+                         float *h_out, void *d_ws, size_t ws_bytes, ae_stream stream) {
+  ae_status st = ae_encode_host_async(m, h_wave, h_sample_off, n_clips, h_out, d_ws, ws_bytes, stream);
+  if (st) return st;
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream");
   return AE_OK;
 }
 
@@ -836,8 +850,8 @@ ae_status ae_local_attention(const void *d_q, const void *d_k, const void *d_v, 
   if (st) return st;
   if (T.total_tokens > 0) {
     if (!d_q || !d_k || !d_v || !d_out || !d_R || !d_qscale) return fail(AE_EINVAL, "a device pointer is null");
-    if (!aligned16(d_q) || !aligned16(d_k) || !aligned16(d_v) || !aligned16(d_out))
-      return fail(AE_EINVAL, "q, k, v and out must be 16-byte aligned");
+    if (!aligned16(d_q) || !aligned16(d_k) || !aligned16(d_v) || !aligned16(d_out) || !aligned16(d_R))
+      return fail(AE_EINVAL, "q, k, v, out and R must be 16-byte aligned");
     const int64_t vec = dtype == AE_BF16 ? 8 : 4;
     if (ld_qkv < kHidden || ld_out < kHidden || ld_qkv % vec || ld_out % vec)
       return fail(AE_EINVAL, "row strides must be >= 1024 and a multiple of 16 bytes");

@@ -3,17 +3,18 @@
 //
 // bf16 path: a persistent tcgen05 kernel on CTA pairs (clusters of two SMs),
 // warp-specialised. Per 64-wide k-block, each CTA's warp 0 streams its half
-// of the pair tile (128 rows of x, 128 rows of W) into a 6-stage shared-memory
+// of the pair tile (128 rows of x, 128 rows of W) into a 4-stage shared-memory
 // ring with TMA (128-byte swizzle, no multicast); the leader CTA's warp 1
 // issues tcgen05.mma.cta_group::2 (M=256, N=256, K=16, bf16 in, f32
 // accumulate), which reads the operand halves from both SMs, into one of two
 // 256-column accumulators in each CTA's tensor memory; warps 2-9 of each CTA
 // drain the other accumulator with tcgen05.ld and apply the epilogue
 // (ClipLin output clamp, SiLU and the next projection's input clamp, GLU, or
-// bias). Pairing halves the W bytes each SM stages per flop, which keeps the
-// shared-memory traffic (TMA writes plus tensor-core reads) under the SM's
-// bandwidth. Tiles are walked m-major so the pairs in flight share rows of x
-// in L2 while W stays L2-resident.
+// bias) on the way to memory through a swizzled shared-memory box and
+// coalesced row stores. Pairing halves the W bytes each SM stages per flop,
+// which keeps the shared-memory traffic (TMA writes plus tensor-core reads)
+// under the SM's bandwidth. Tiles are walked m-major so the pairs in flight
+// share rows of x in L2 while W stays L2-resident.
 //
 // f32 path: a plain 64x64-tile FMA kernel with the same epilogues.
 #include <cudaTypedefs.h>
@@ -40,8 +41,20 @@ unsigned *device_status_word() {
 
 // ------------------------------------------------------------------ epilogue
 
+// 128-byte line of the staging buffer: the 16-byte granule g of row r sits at
+// granule g ^ (r & 7) (the TMA's 128-byte swizzle), so the 32 rows of a warp
+// write a granule column without bank conflicts.
+__device__ __forceinline__ void st_granule(uint8_t *line, int r7, int g, uint4 v) {
+  *reinterpret_cast<uint4 *>(line + ((g ^ r7) << 4)) = v;
+}
+
+// Epilogue of 32 accumulator columns [col, col + 32) of one row, written as
+// granules g0, g0 + 1, ... of the row's staging line: 8 granules of f32
+// (EPI_F32), 4 of bf16 (EPI_BF16, EPI_SILU), 2 of bf16 (EPI_GLU, which pairs
+// columns (2c, 2c + 1) into output column c).
 template <int MODE>
-__device__ __forceinline__ void epi_store_tc(const EpiArgs &ep, int row, int col, const uint32_t (&r)[32]) {
+__device__ __forceinline__ void epi_stage(const EpiArgs &ep, int col, const uint32_t (&r)[32], uint8_t *line, int r7,
+                                          int g0) {
   float lo = ep.lo, hi = ep.hi;
   if (ep.seg_w > 0) {
     const int sg = col / ep.seg_w;  // selects, not a runtime index into the parameter array
@@ -57,10 +70,11 @@ __device__ __forceinline__ void epi_store_tc(const EpiArgs &ep, int row, int col
       for (int i = 0; i < 32; ++i) v[i] += __ldg(ep.bias + col + i);
     }
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = clampf(v[i], lo, hi);
-    float *o = static_cast<float *>(ep.out) + (int64_t)row * ep.ld + col;
-#pragma unroll
-    for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4 *>(o + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+    for (int j = 0; j < 8; ++j)
+      st_granule(line, r7, g0 + j,
+                 make_uint4(__float_as_uint(clampf(v[4 * j], lo, hi)), __float_as_uint(clampf(v[4 * j + 1], lo, hi)),
+                            __float_as_uint(clampf(v[4 * j + 2], lo, hi)),
+                            __float_as_uint(clampf(v[4 * j + 3], lo, hi))));
   } else if (MODE == EPI_GLU) {
     // a * sigmoid(b) = a / (1 + e^-b): fast exp and reciprocal (2 ulp each; the
     // bf16 rounding of the result is 2^-9), with the right limits at +-inf
@@ -71,9 +85,8 @@ __device__ __forceinline__ void epi_store_tc(const EpiArgs &ep, int row, int col
       float a1 = clampf(v[4 * j + 2], lo, hi), b1 = clampf(v[4 * j + 3], lo, hi);
       p[j] = pack_bf16(__fdividef(a0, 1.0f + __expf(-b0)), __fdividef(a1, 1.0f + __expf(-b1)));
     }
-    bf16 *o = static_cast<bf16 *>(ep.out) + (int64_t)row * ep.ld + col / 2;
-    reinterpret_cast<uint4 *>(o)[0] = make_uint4(p[0], p[1], p[2], p[3]);
-    reinterpret_cast<uint4 *>(o)[1] = make_uint4(p[4], p[5], p[6], p[7]);
+    st_granule(line, r7, g0, make_uint4(p[0], p[1], p[2], p[3]));
+    st_granule(line, r7, g0 + 1, make_uint4(p[4], p[5], p[6], p[7]));
   } else {
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
@@ -84,9 +97,8 @@ __device__ __forceinline__ void epi_store_tc(const EpiArgs &ep, int row, int col
     uint32_t p[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) p[j] = pack_bf16(v[2 * j], v[2 * j + 1]);
-    uint4 *o = reinterpret_cast<uint4 *>(static_cast<bf16 *>(ep.out) + (int64_t)row * ep.ld + col);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) o[j] = make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
+    for (int j = 0; j < 4; ++j) st_granule(line, r7, g0 + j, make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]));
   }
 }
 
@@ -96,12 +108,14 @@ namespace {
 constexpr int BM = 128;                 // rows of x per CTA (256 per pair)
 constexpr int BK = 64;                  // one 128-byte swizzle atom of bf16
 constexpr int BN = 256;                 // columns per pair tile (128 rows of W per CTA)
-constexpr int STAGES = 6;
+constexpr int STAGES = 4;
 constexpr uint32_t A_BYTES = BM * BK * 2, B_BYTES = (BN / 2) * BK * 2, STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr uint32_t TMEM_COLS = 2 * BN;  // two 128 x 256 f32 accumulators per CTA
 constexpr int EPI_WARPS = 8;
+constexpr uint32_t LINE_BYTES = 32 * 128;  // one staging box: 32 rows x 128 bytes
+constexpr uint32_t EPI_BYTES = EPI_WARPS * LINE_BYTES;  // one box per epilogue warp
 constexpr int GEMM_THREADS = 64 + 32 * EPI_WARPS;
-constexpr size_t SMEM_TC = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr size_t SMEM_TC = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + 256;
 }  // namespace
 
 // Persistent pair kernel (cluster of 2 CTAs on 2 SMs). Pair tile 256 x 256:
@@ -112,11 +126,13 @@ constexpr size_t SMEM_TC = STAGES * STAGE_BYTES + 1024 + 256;
 // in CTA r's tensor memory. Each CTA's epilogue drains its own 128 rows.
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
-    k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const EpiArgs ep,
-              const int M, const int N, const int K, unsigned *status) {
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const EpiArgs ep, const int M, const int N, const int K,
+              unsigned *status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);  // used in the leader
+  uint8_t *epi_smem = smem + STAGES * STAGE_BYTES;                                 // store boxes
+  uint64_t *full = reinterpret_cast<uint64_t *>(epi_smem + EPI_BYTES);            // used in the leader
   uint64_t *empty = full + STAGES;                                              // per CTA
   uint64_t *tfull = empty + STAGES;                                             // per CTA
   uint64_t *tempty = tfull + 2;                                                 // used in the leader
@@ -234,10 +250,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     tc_commit_pair_local(done);  // arrives once every MMA issued above has completed
     mbar_wait(done, 0);
   } else if (warp >= 2) {
-    // ---------------- epilogue (both CTAs): warp w reads TMEM lanes 32*(w%4) .. +31;
-    // the two warps of a lane quarter split the tile's columns
-    const int q = warp & 3;
-    const int c0 = ((warp - 2) >> 2) * (BN / 64);
+    // ---------------- epilogue (both CTAs): warp w reads TMEM lanes 32*(w%4) .. +31
+    // (rows of the tile) and one half of the tile's 256 columns. Each lane
+    // writes its row's results into a 32-row x 128-byte box in shared memory
+    // (128-byte swizzle: conflict-free); the warp then reads the box back row
+    // by row and writes 4 full 128-byte row segments per store instruction.
+    constexpr int LOADS_PER_BOX = MODE == EPI_F32 ? 1 : (MODE == EPI_GLU ? 4 : 2);  // 32-column TMEM loads
+    constexpr int OUT_COLS_PER_BOX = MODE == EPI_F32 ? 32 : 64;                     // 128 bytes of output
+    constexpr int GRANULES_PER_LOAD = 8 / LOADS_PER_BOX;
+    constexpr int ES = MODE == EPI_F32 ? 4 : 2;
+    const int q = warp & 3, half = (warp - 2) >> 2;
+    uint8_t *box = epi_smem + (warp - 2) * LINE_BYTES;
     const uint32_t tempty_leader = map_to_rank(&tempty[0], 0);
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -250,19 +273,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         break;
       }
       tc_fence_after();
-      const int row = mb * 2 * BM + (int)rank * BM + q * 32 + lane;
-      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      const int row0 = mb * 2 * BM + (int)rank * BM + q * 32;
+      const int col0 = nb * BN + half * (BN / 2);
+      const int ocol0 = MODE == EPI_GLU ? col0 / 2 : col0;
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + half * (BN / 2));
+      auto stage = [&](int c, const uint32_t(&r)[32]) {
+        const int j = c % LOADS_PER_BOX;
+        epi_stage<MODE>(ep, col0 + c * 32, r, box + lane * 128, lane & 7, j * GRANULES_PER_LOAD);
+        if (j == LOADS_PER_BOX - 1) {
+          __syncwarp();
+          // lane l moves granule l % 8 of rows l / 8, l / 8 + 4, ...
+          const int g = lane & 7;
+          uint8_t *dst = static_cast<uint8_t *>(ep.out) +
+                         ((int64_t)ocol0 + (c / LOADS_PER_BOX) * OUT_COLS_PER_BOX) * ES + g * 16;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int rr = (lane >> 3) + 4 * i;
+            const uint4 v = *reinterpret_cast<const uint4 *>(box + rr * 128 + ((g ^ (rr & 7)) << 4));
+            if (row0 + rr < M) *reinterpret_cast<uint4 *>(dst + (int64_t)(row0 + rr) * ep.ld * ES) = v;
+          }
+          __syncwarp();
+        }
+      };
       // two register buffers: the next chunk's tcgen05.ld is in flight during the math
       uint32_t ra[32], rb[32];
-      tmem_ld32(tbase + c0 * 32, ra);
+      tmem_ld32(tbase, ra);
       tmem_ld_wait();
 #pragma unroll 1
       for (int c = 0; c < BN / 64; c += 2) {
-        tmem_ld32(tbase + (c0 + c + 1) * 32, rb);
-        if (row < M) epi_store_tc<MODE>(ep, row, nb * BN + (c0 + c) * 32, ra);
+        tmem_ld32(tbase + (c + 1) * 32, rb);
+        stage(c, ra);
         tmem_ld_wait();
-        if (c + 2 < BN / 64) tmem_ld32(tbase + (c0 + c + 2) * 32, ra);
-        if (row < M) epi_store_tc<MODE>(ep, row, nb * BN + (c0 + c + 1) * 32, rb);
+        if (c + 2 < BN / 64) tmem_ld32(tbase + (c + 2) * 32, ra);
+        stage(c + 1, rb);
         tmem_ld_wait();
       }
       tc_fence_before();
@@ -403,6 +446,7 @@ static int num_sms() {
 template <int MODE>
 static cudaError_t launch_tc(const CUtensorMap &tA, const CUtensorMap &tB, const EpiArgs &ep, int M, int N, int K,
                              cudaStream_t s) {
+
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_TC);

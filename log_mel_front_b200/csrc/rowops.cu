@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(256, NV <= 8 ? 3 : 2) k_rowop(const RowArgs r)
     for (int i = 0; i < NV; ++i) load4(hrow + (i * 32 + lane) * 4, h[i]);
     if (r.y) {
 #pragma unroll
-      for (int i = 0; i < NV; ++i) load4(r.y + row * W + (i * 32 + lane) * 4, y[i]);
+      for (int i = 0; i < NV; ++i) load4(static_cast<const ActT *>(r.y) + row * W + (i * 32 + lane) * 4, y[i]);
     }
   }
   __syncthreads();

@@ -236,6 +236,25 @@ def test_packing_is_bit_invariant_on_gpu(m_tower):
         assert np.array_equal(alone, g[off[i]:off[i + 1]]), i
 
 
+def test_encode_host_async_two_streams_match_device_path(m_tower):
+    """ae_encode_host_async on two streams with their own workspaces, four
+    calls in flight: each output equals ae_encode's, bit for bit."""
+    rng = np.random.default_rng(5)
+    clips = [(0.3 * rng.standard_normal(n)).astype(np.float32) for n in (16000, 48000, 3000)]
+    g, _ = gpu_encode(m_tower, clips)
+    flat, soff = synth.pack(clips)
+    h_wave = torch.from_numpy(flat).pin_memory()
+    nb = ae.ae_encode_host_workspace_size(m_tower, soff)
+    outs = [torch.full(g.shape, float("nan")).pin_memory() for _ in range(2)]
+    wss = [workspace(nb) for _ in range(2)]
+    streams = [torch.cuda.Stream() for _ in range(2)]
+    for i in range(4):
+        ae.ae_encode_host_async(m_tower, h_wave, soff, outs[i % 2], wss[i % 2], nb, streams[i % 2])
+    _sync()
+    for o in outs:
+        assert np.array_equal(o.numpy(), g)
+
+
 # ------------------------------------------------------------------ attention core
 
 def _attn_oracle(q, k, v, pos, R, qd, cap=50.0):
@@ -288,6 +307,28 @@ def test_attention_microbench_full_size_sampled():
         want = np.stack([_attn_oracle(qq[max(0, t - 11):t + 1], kk[max(0, t - 11):t + 1], vv[max(0, t - 11):t + 1],
                                       np.arange(max(0, t - 11), t + 1), Ro, qd)[-1] for t in idx])
         assert_bf16(got, want, f"attention seq {s}")
+
+
+@pytest.mark.parametrize("toks", [[2, 3], [1, 3, 12, 13, 127, 1, 128, 129]])
+def test_attention_bf16_edges_all_tokens(toks):
+    """Every token of short and ragged batches, q/k/v as strided views of one
+    [T][3072] buffer (the layout of the fused projection): clip starts inside a
+    128-token tile, sequences shorter than the window, T below, at and just
+    past a tile boundary."""
+    p = synth.attention_params()
+    rng = np.random.default_rng(len(toks))
+    T = sum(toks)
+    qkv = synth.round_to_bf16((2.0 * rng.standard_normal((T, 3072))).astype(np.float32))
+    d = dev(qkv).to(torch.bfloat16)
+    R, qs, ks = ae.ae_attention_tables(p["relk"], p["pds"])
+    out = torch.full((T, 1024), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ws = workspace(ae.ae_workspace_size(None, len(toks), 0, T))
+    ae.ae_local_attention(d[:, :1024], d[:, 1024:2048], d[:, 2048:], 3072, ae.AE_BF16, dev(R), dev(qs), ks, 50.0,
+                          offsets(toks), out, 1024, ws, ws.numel())
+    _sync()
+    Ro = O.relative_keys(p["relk"], 12, 1024)
+    o = _attn_oracle(qkv[:, :1024], qkv[:, 1024:2048], qkv[:, 2048:], O.positions(toks), Ro, O.softplus(p["pds"]))
+    assert_bf16(out.float().cpu().numpy(), o, f"attention bf16, {T} tokens in {len(toks)} clips")
 
 
 # ------------------------------------------------------------------ refusals (host checks, nothing enqueued)
