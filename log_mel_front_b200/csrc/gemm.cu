@@ -102,6 +102,64 @@ __device__ __forceinline__ void epi_stage(const EpiArgs &ep, int col, const uint
   }
 }
 
+__device__ __forceinline__ void st_global_32B(void *p, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t a4,
+                                              uint32_t a5, uint32_t a6, uint32_t a7) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a0), "r"(a1), "r"(a2),
+               "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7)
+               : "memory");
+}
+
+// Epilogue of 32 accumulator columns of one row, stored from registers as
+// whole 32-byte sectors (the bf16 outputs; f32 outputs go through epi_stage).
+template <int MODE>
+__device__ __forceinline__ void epi_store32(const EpiArgs &ep, int row, int col, const uint32_t (&r)[32]) {
+  float lo = ep.lo, hi = ep.hi;
+  if (ep.seg_w > 0) {
+    const int sg = col / ep.seg_w;
+    lo = sg == 0 ? ep.seg_lo[0] : (sg == 1 ? ep.seg_lo[1] : ep.seg_lo[2]);
+    hi = sg == 0 ? ep.seg_hi[0] : (sg == 1 ? ep.seg_hi[1] : ep.seg_hi[2]);
+  }
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  if (MODE == EPI_F32) {
+    if (ep.bias) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] += __ldg(ep.bias + col + i);
+    }
+    float *o = static_cast<float *>(ep.out) + (int64_t)row * ep.ld + col;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      st_global_32B(o + 8 * j, __float_as_uint(clampf(v[8 * j], lo, hi)), __float_as_uint(clampf(v[8 * j + 1], lo, hi)),
+                    __float_as_uint(clampf(v[8 * j + 2], lo, hi)), __float_as_uint(clampf(v[8 * j + 3], lo, hi)),
+                    __float_as_uint(clampf(v[8 * j + 4], lo, hi)), __float_as_uint(clampf(v[8 * j + 5], lo, hi)),
+                    __float_as_uint(clampf(v[8 * j + 6], lo, hi)), __float_as_uint(clampf(v[8 * j + 7], lo, hi)));
+  } else if (MODE == EPI_GLU) {
+    uint32_t p[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float a0 = clampf(v[4 * j + 0], lo, hi), b0 = clampf(v[4 * j + 1], lo, hi);
+      float a1 = clampf(v[4 * j + 2], lo, hi), b1 = clampf(v[4 * j + 3], lo, hi);
+      p[j] = pack_bf16(__fdividef(a0, 1.0f + __expf(-b0)), __fdividef(a1, 1.0f + __expf(-b1)));
+    }
+    bf16 *o = static_cast<bf16 *>(ep.out) + (int64_t)row * ep.ld + col / 2;
+    st_global_32B(o, p[0], p[1], p[2], p[3], p[4], p[5], p[6], p[7]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      float x = clampf(v[i], lo, hi);
+      if (MODE == EPI_SILU) x = clampf(__fdividef(x, 1.0f + __expf(-x)), ep.lo2, ep.hi2);
+      v[i] = x;
+    }
+    uint32_t p[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) p[j] = pack_bf16(v[2 * j], v[2 * j + 1]);
+    bf16 *o = static_cast<bf16 *>(ep.out) + (int64_t)row * ep.ld + col;
+    st_global_32B(o, p[0], p[1], p[2], p[3], p[4], p[5], p[6], p[7]);
+    st_global_32B(o + 16, p[8], p[9], p[10], p[11], p[12], p[13], p[14], p[15]);
+  }
+}
+
 // ------------------------------------------------------------------ tcgen05 pair kernel
 
 namespace {
@@ -251,10 +309,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     mbar_wait(done, 0);
   } else if (warp >= 2) {
     // ---------------- epilogue (both CTAs): warp w reads TMEM lanes 32*(w%4) .. +31
-    // (rows of the tile) and one half of the tile's 256 columns. Each lane
-    // writes its row's results into a 32-row x 128-byte box in shared memory
-    // (128-byte swizzle: conflict-free); the warp then reads the box back row
-    // by row and writes 4 full 128-byte row segments per store instruction.
+    // (rows of the tile) and one half of the tile's 256 columns. bf16 results
+    // leave each lane's row as whole 32-byte sectors. f32 results are written
+    // by each lane into a 32-row x 128-byte box in shared memory (128-byte
+    // swizzle: conflict-free), which the warp reads back row by row to write 4
+    // full 128-byte row segments per store instruction (measured faster for
+    // f32, slower for bf16, than the direct sector stores).
     constexpr int LOADS_PER_BOX = MODE == EPI_F32 ? 1 : (MODE == EPI_GLU ? 4 : 2);  // 32-column TMEM loads
     constexpr int OUT_COLS_PER_BOX = MODE == EPI_F32 ? 32 : 64;                     // 128 bytes of output
     constexpr int GRANULES_PER_LOAD = 8 / LOADS_PER_BOX;
@@ -278,6 +338,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       const int ocol0 = MODE == EPI_GLU ? col0 / 2 : col0;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + half * (BN / 2));
       auto stage = [&](int c, const uint32_t(&r)[32]) {
+        if (MODE != EPI_F32) {  // bf16 rows: 32-byte stores straight from registers
+          if (row0 + lane < M) epi_store32<MODE>(ep, row0 + lane, col0 + c * 32, r);
+          return;
+        }
         const int j = c % LOADS_PER_BOX;
         epi_stage<MODE>(ep, col0 + c * 32, r, box + lane * 128, lane & 7, j * GRANULES_PER_LOAD);
         if (j == LOADS_PER_BOX - 1) {
