@@ -15,6 +15,7 @@
 #include "ae_internal.h"
 #include "common.cuh"
 
+#include <algorithm>
 #include <cstring>
 
 namespace ae {
@@ -136,10 +137,12 @@ cudaError_t launch_rowop(const ae_model *m, const RowArgs &r, cudaStream_t s) {
 
 // w_dw is stored tap-major [kernel][hidden]. Thread t of a 256-thread CTA
 // owns channels 4t .. 4t+3 for kLcRows consecutive rows: its 5 x 4 taps and
-// 4 norm weights stay in registers, and it walks the rows (plus the 4 before
-// them) with a sliding window, one coalesced 8-byte load per row. The conv
-// outputs of its rows stay in registers; the per-row sums of squares are
-// reduced across the CTA once for all its rows.
+// 4 norm weights stay in registers, as channel pairs for the packed two-lane
+// FMA, and it loads its 8-byte slice of the rows (plus the 4 before them),
+// one coalesced load per row. The conv outputs of its rows stay in registers.
+// The per-row sums of squares are reduced across the warp with a butterfly
+// that halves the rows at every step (after it, lanes 4r .. 4r+3 hold row r),
+// then across the CTA's 8 warps once for all rows.
 constexpr int kLcRows = 8;
 constexpr int kLcHalo = kKernel - 1;
 
@@ -147,52 +150,79 @@ template <typename ActT>
 __global__ void __launch_bounds__(256) k_lconv(const ActT *__restrict__ gl, const float *__restrict__ w_dw,
                                                const float *__restrict__ w_norm, float lo, float hi,
                                                ActT *__restrict__ out, const int32_t *__restrict__ pos, int64_t T) {
+  static_assert(kLcRows == 8, "the butterfly below reduces 8 rows");
   __shared__ float s_ss[8][kLcRows];
   __shared__ float s_inv[kLcRows];
   const int ch = 4 * threadIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t t0 = (int64_t)blockIdx.x * kLcRows;
-  float w[kKernel][4], wn[4];
+  float2 w[kKernel][2], wn[2];
 #pragma unroll
-  for (int k = 0; k < kKernel; ++k) load4(w_dw + k * kHidden + ch, w[k]);
-  load4(w_norm + ch, wn);
-  float x[kLcRows + kLcHalo][4];
+  for (int k = 0; k < kKernel; ++k) {
+    float t[4];
+    load4(w_dw + k * kHidden + ch, t);
+    w[k][0] = make_float2(t[0], t[1]);
+    w[k][1] = make_float2(t[2], t[3]);
+  }
+  {
+    float t[4];
+    load4(w_norm + ch, t);
+    wn[0] = make_float2(t[0], t[1]);
+    wn[1] = make_float2(t[2], t[3]);
+  }
+  float2 x[kLcRows + kLcHalo][2];
 #pragma unroll
   for (int r = 0; r < kLcRows + kLcHalo; ++r) {
     const int64_t tok = t0 - kLcHalo + r;
-    if (tok >= 0 && tok < T) {
-      load4(gl + tok * kHidden + ch, x[r]);
-    } else {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) x[r][u] = 0.f;
-    }
+    float t[4] = {0.f, 0.f, 0.f, 0.f};
+    if (tok >= 0 && tok < T) load4(gl + tok * kHidden + ch, t);
+    x[r][0] = make_float2(t[0], t[1]);
+    x[r][1] = make_float2(t[2], t[3]);
   }
-  float c[kLcRows][4], ss[kLcRows];
+  float2 c[kLcRows][2];
+  float ss[kLcRows];
 #pragma unroll
   for (int r = 0; r < kLcRows; ++r) {
     const int64_t tok = t0 + r;
     const int p = tok < T ? pos[tok] : 0;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) c[r][u] = 0.f;
+    c[r][0] = c[r][1] = make_float2(0.f, 0.f);
 #pragma unroll
     for (int k = 0; k < kKernel; ++k) {
       const int back = kKernel - 1 - k;
       if (back <= p) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) c[r][u] = fmaf(w[k][u], x[r + kLcHalo - back][u], c[r][u]);
+        ffma2(c[r][0], w[k][0], x[r + kLcHalo - back][0]);
+        ffma2(c[r][1], w[k][1], x[r + kLcHalo - back][1]);
       }
     }
-    ss[r] = warp_sum(c[r][0] * c[r][0] + c[r][1] * c[r][1] + c[r][2] * c[r][2] + c[r][3] * c[r][3]);
+    float2 q = make_float2(0.f, 0.f);
+    ffma2(q, c[r][0], c[r][0]);
+    ffma2(q, c[r][1], c[r][1]);
+    ss[r] = q.x + q.y;
   }
-  if (lane == 0) {
+  // butterfly reduce-scatter: 8 rows -> 4 -> 2 -> 1 per lane, then a sum over the 4 lanes
+  {
+    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+    float v4[4], v2[2];
 #pragma unroll
-    for (int r = 0; r < kLcRows; ++r) s_ss[warp][r] = ss[r];
+    for (int i = 0; i < 4; ++i) {
+      const float mine = b4 ? ss[i + 4] : ss[i], other = b4 ? ss[i] : ss[i + 4];
+      v4[i] = mine + __shfl_xor_sync(0xffffffffu, other, 16);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const float mine = b3 ? v4[i + 2] : v4[i], other = b3 ? v4[i] : v4[i + 2];
+      v2[i] = mine + __shfl_xor_sync(0xffffffffu, other, 8);
+    }
+    float v = (b2 ? v2[1] : v2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? v2[0] : v2[1], 4);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    if ((lane & 3) == 0) s_ss[warp][lane >> 2] = v;  // row (lane >> 2): bits 4, 3, 2 of the lane
   }
   __syncthreads();
   if (threadIdx.x < kLcRows) {
-    float s = 0.f;
+    float sum = 0.f;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) s += s_ss[q][threadIdx.x];
-    s_inv[threadIdx.x] = rsqrtf(s * (1.0f / kHidden) + kEps);
+    for (int q = 0; q < 8; ++q) sum += s_ss[q][threadIdx.x];
+    s_inv[threadIdx.x] = rsqrtf(sum * (1.0f / kHidden) + kEps);
   }
   __syncthreads();
 #pragma unroll
@@ -200,12 +230,11 @@ __global__ void __launch_bounds__(256) k_lconv(const ActT *__restrict__ gl, cons
     const int64_t tok = t0 + r;
     if (tok >= T) break;
     const float inv = s_inv[r];
+    const float y[4] = {c[r][0].x * inv * wn[0].x, c[r][0].y * inv * wn[0].y, c[r][1].x * inv * wn[1].x,
+                        c[r][1].y * inv * wn[1].y};
     float v[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float y = c[r][u] * inv * wn[u];
-      v[u] = clampf(__fdividef(y, 1.0f + __expf(-y)), lo, hi);
-    }
+    for (int u = 0; u < 4; ++u) v[u] = clampf(__fdividef(y[u], 1.0f + __expf(-y[u])), lo, hi);
     store4(out + tok * kHidden + ch, v);
   }
 }
@@ -248,6 +277,23 @@ cudaError_t launch_pos(int32_t *pos, const int32_t *tok_off, int n_clips, cudaSt
 }
 
 static size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+
+cudaError_t launch_upload_bytes(const void *host, size_t bytes, void *dev, cudaStream_t s) {
+  static thread_local UploadChunk ch;
+  const size_t nw = (bytes + 3) / 4;
+  const uint8_t *src = static_cast<const uint8_t *>(host);
+  for (size_t w0 = 0; w0 < nw; w0 += 7936) {
+    const size_t n = nw - w0 < 7936 ? nw - w0 : 7936;
+    ch.dst = (int64_t)(w0 * 4);
+    ch.n = (int)n;
+    const size_t b = std::min(bytes - w0 * 4, n * 4);
+    std::memset(ch.w, 0, n * 4);
+    std::memcpy(ch.w, src + w0 * 4, b);
+    cudaError_t e = launch_k(k_upload, dim3(1), dim3(256), 0, s, static_cast<uint8_t *>(dev), ch);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
 
 size_t tables_bytes(int64_t n_clips) {
   const size_t B1 = (size_t)n_clips + 1;
