@@ -147,7 +147,8 @@ def workload_desc(name: str, info: dict) -> dict:
     base = {"tower": "16 clips x 30 s, 12 Conformer layers + embedding head, bf16 weights, f32 accumulation",
             "ragged": "256 clips of 1-30 s (uniform whole samples), packed, 12 layers + head, bf16",
             "frontend": "log-mel front-end only, 64 clips x 30 s, f32",
-            "attention": "local-attention core only, 32 x 8192 tokens, 8 heads x 128, bf16 q/k/v"}[name]
+            "attention": "local-attention core only, 32 x 8192 tokens, 8 heads x 128, bf16 q/k/v",
+            "resample": "mixdown + Kaiser-sinc resampling to 16 kHz, 64 stereo clips x 30 s at 44.1 kHz, f32"}[name]
     d = {"workload": f"{name}: {base}", "l2": "flushed between steps (256 MiB write)",
          "model": "gemma4_audio tower shape (random init)"}
     d.update(info)
@@ -183,6 +184,25 @@ class Ours:
             self.d_mel = torch.empty((self.frames, 128), device="cuda")
             self.h_mel = torch.empty((self.frames, 128)).pin_memory()
             self.dominant = "logmel"
+        elif name == "resample":
+            n = synth.RS_RATE * synth.RS_SECONDS
+            self.lens = [n] * synth.RS_CLIPS
+            self.off = np.arange(synth.RS_CLIPS + 1, dtype=np.int64) * n
+            planes = np.empty((2, synth.RS_CLIPS * n), np.float32)
+            for k in range(synth.RS_CLIPS):
+                ch = synth.resample_clip(k)
+                planes[0, k * n:(k + 1) * n] = ch[0]
+                planes[1, k * n:(k + 1) * n] = ch[1]
+            self.h_x = torch.from_numpy(planes).pin_memory()
+            self.d_x = self.h_x.cuda()
+            self.n_out = sum(ae.ae_resample_len(v, synth.RS_RATE) for v in self.lens)
+            self.d_y = torch.empty(self.n_out, device="cuda")
+            self.h_y = torch.empty(self.n_out).pin_memory()
+            self.ws_bytes = ae.ae_resample_workspace_size(self.off, synth.RS_RATE, 16000, 2)
+            self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
+            self.tokens = self.n_out
+            self.audio_s = synth.RS_CLIPS * float(synth.RS_SECONDS)
+            self.dominant = "resample"
         elif name == "attention":
             S, T = synth.ATT_SEQS, synth.ATT_T
             p = synth.attention_params()
@@ -206,6 +226,9 @@ class Ours:
             ae.ae_encode(self.model, self.d_wave, self.off, self.d_out, self.ws, self.ws_bytes, self.stream)
         elif self.name == "frontend":
             ae.ae_logmel(self.d_wave, self.off, self.d_mel, self.ws, self.ws_bytes, self.stream)
+        elif self.name == "resample":
+            ae.ae_resample(self.d_x, 2, self.d_x.shape[1], self.off, synth.RS_RATE, 16000, self.d_y, self.ws,
+                           self.ws_bytes, self.stream)
         else:
             ae.ae_local_attention(self.q, self.k, self.v, 1024, ae.AE_BF16, self.R, self.qs, self.ks, 50.0,
                                   self.tok_off, self.o, 1024, self.ws, self.ws_bytes, self.stream)
@@ -222,6 +245,12 @@ class Ours:
             self.h_mel.copy_(self.d_mel, non_blocking=True)
             self.stream.synchronize()
             return self.h_wave.numel() * 4, self.h_mel.numel() * 4
+        if self.name == "resample":
+            self.d_x.copy_(self.h_x, non_blocking=True)
+            self.step()
+            self.h_y.copy_(self.d_y, non_blocking=True)
+            self.stream.synchronize()
+            return self.h_x.numel() * 4, self.h_y.numel() * 4
         return 0, 0
 
     def e2e_pipelined(self, k: int) -> float:
@@ -276,6 +305,10 @@ class OracleRun:
             self.W = synth.model_weights(name)
             self.lens = synth.clip_lengths(name)
             self.next = 0
+        elif name == "resample":
+            from oracle import resample as RS
+            self.RS = RS
+            self.next = 0
         elif name == "attention":
             p = synth.attention_params()
             q, k, v = synth.attention_qkv(0, T=2048)
@@ -299,6 +332,13 @@ class OracleRun:
             t0 = time.perf_counter()
             O.log_mel(c)
             return time.perf_counter() - t0, 30.0, "clip 0 of the frontend workload (log-mel)"
+        if self.name == "resample":
+            i = self.next % synth.RS_CLIPS
+            self.next += 1
+            ch = synth.resample_clip(i)
+            t0 = time.perf_counter()
+            self.RS.to_mono_16k(ch, synth.RS_RATE)
+            return time.perf_counter() - t0, float(synth.RS_SECONDS), f"stereo clip {i} of the resample workload"
         t0 = time.perf_counter()
         O.local_attention_core(*self.qkv, np.arange(2048), self.R, self.qd, 8, 12, 50.0)
         return time.perf_counter() - t0, 2048 / 25.0, "2048 tokens of one attention sequence"
@@ -381,13 +421,21 @@ def run_ours(args, rank, world, dist):
         achieved = dom["flops"] / (dom["ms"] / 1e3) / 1e12
         peak = pk["bf16_tflops_sustained"]
         roof = {"bound": "tensor", "unit": "TFLOP/s", "peak_kind": "bf16 sustained (" + pk["source"] + ")"}
+    elif ours.dominant == "resample":
+        # the FIR is plain FP32 multiply-add: 148 SMs x 128 FP32 lanes x 2 flop at the max SM clock
+        sm_mhz = (clocks.get("sm_max_mhz") or 1965.0)
+        achieved = dom["flops"] / (dom["ms"] / 1e3) / 1e12
+        peak = round(148 * 128 * 2 * sm_mhz * 1e6 / 1e12, 2)
+        roof = {"bound": "alu", "unit": "TFLOP/s",
+                "peak_kind": f"FP32 FMA from unit counts: 148 SMs x 128 lanes x 2 flop x {sm_mhz:.0f} MHz"}
     else:
         achieved = dom["bytes"] / (dom["ms"] / 1e3) / 1e9
         peak = pk["hbm_gbs"]
         roof = {"bound": "hbm", "unit": "GB/s", "peak_kind": "HBM copy (" + pk["source"] + ")"}
     traffic, traffic_src = captured_traffic(ours.dominant)
     roof.update({"kernel": {"gemm": "k_gemm_tc (all projections)", "logmel": "k_logmel",
-                            "attention": "k_attention"}[ours.dominant],
+                            "attention": "k_attention_tc",
+                            "resample": "k_rs_fir (with its tap table and mixdown)"}[ours.dominant],
                  "achieved": round(achieved, 2), "peak": peak, "frac": round(achieved / peak, 4),
                  "traffic": None if traffic is None else round(traffic), "traffic_source": traffic_src,
                  "algorithmic_bytes_per_launch": round(dom["bytes"] / max(dom["launches"], 1)),
@@ -400,16 +448,20 @@ def run_ours(args, rank, world, dist):
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(per_step, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16" if args.workload != "frontend" else "f32", "data": "synthetic",
+        "vs_baseline": None, "dtype": "f32" if args.workload in ("frontend", "resample") else "bf16",
+        "data": "synthetic",
         "config": workload_desc(args.workload, {
-            "clips": len(getattr(ours, "lens", [])) or synth.ATT_SEQS, "tokens_per_replica": ours.tokens,
+            "clips": len(getattr(ours, "lens", [])) or synth.ATT_SEQS,
+            ("output_samples_per_replica" if args.workload == "resample" else "tokens_per_replica"): ours.tokens,
             "audio_seconds_per_replica": round(ours.audio_s, 3), "parallelism": f"replicas x{world}",
-            "soft_tokens_per_s": round(ours.tokens * world / (per_step / 1e3), 1)}),
+            ("output_samples_per_s" if args.workload == "resample" else "soft_tokens_per_s"):
+                round(ours.tokens * world / (per_step / 1e3), 1)}),
         "e2e": None if ms_e2e is None else {
             "value": round(audio / (ms_e2e / args.steps / 1e3), 2), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "api": ("ae_encode_host_async, two streams (copies of one step overlap the kernels of the other)"
-                    if args.workload in ("tower", "ragged") else "ae_logmel + copies")},
+            "api": {"tower": "ae_encode_host_async, two streams (copies of one step overlap the kernels of the other)",
+                    "ragged": "ae_encode_host_async, two streams (copies of one step overlap the kernels of the other)",
+                    "frontend": "ae_logmel + copies", "resample": "ae_resample + copies"}[args.workload]},
         "gpu_launches": int(round(launches / prof_steps * args.steps)),
         "roofline": roof,
         "kernel_classes": classes,
@@ -450,7 +502,7 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", choices=("tower", "ragged", "frontend", "attention"), default="tower")
+    ap.add_argument("--workload", choices=("tower", "ragged", "frontend", "attention", "resample"), default="tower")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)

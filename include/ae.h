@@ -249,6 +249,47 @@ ae_status ae_local_attention(const void *d_q, const void *d_k, const void *d_v, 
 ae_status ae_logmel_noalloc(const float *d_wave, const int64_t *h_sample_off, int n_clips, float *d_mel,
                             ae_stream stream);
 
+/* --- input conditioning: mixdown and resampling -------------------------------- */
+
+/* Output length of ae_resample for one clip of n_samples at rate_in:
+ * n_samples when the rates are equal or n_samples is 0, else
+ * ceil(p * n_samples / o) with o = rate_in / g, p = rate_out / g, g their
+ * gcd (egemma2_audio.rs, resample_hq: the length of its output). -1 for
+ * a negative count or a rate outside 1 .. 1000000. */
+int64_t ae_resample_len(int64_t n_samples, int32_t rate_in, int32_t rate_out);
+
+/* Workspace bytes ae_resample needs for these clips, rates and channel
+ * count (0 for invalid arguments): clip tables, the per-phase taps
+ * (rate_out / g rows) and, for more than one channel, the mixed-down input. */
+size_t ae_resample_workspace_size(const int64_t *h_sample_off, int n_clips, int32_t rate_in, int32_t rate_out,
+                                  int channels);
+
+/* Channel mixdown and band-limited resampling, per clip (egemma2_audio.rs,
+ * to_mono_16k and resample_hq):
+ *   mono[i] = (x_0[i] + x_1[i] + ... + x_{C-1}[i]) / C, float32 adds in
+ *   channel order and a float32 division (one channel passes unchanged);
+ *   y[n] = sum over inputs m with |t| < 64 of mono[m] c sinc(t)
+ *          I0(12.8 sqrt(1 - (t/64)^2)) / I0(12.8),
+ *   t = (m - n o / p) c, c = 0.958 min(o, p) / o, inputs outside the clip 0,
+ * for n < ae_resample_len(N, rate_in, rate_out). The taps are evaluated in
+ * float64 and applied in float32 with float32 accumulation in two
+ * interleaved partial sums over L = 2 ceil(64 / c) + 3 taps: against the
+ * float64 definition the error is below (L / 2 + 2) 2^-24 x 2.7 x max |mono|
+ * (2.7 bounds the taps' absolute sum), 3e-5 x max |mono| from 48 kHz and
+ * 6e-5 from 96 kHz. Equal rates copy mono.
+ * d_x: float32, channel ch of the packed clips at d_x + ch * ch_stride
+ * (ch_stride >= h_sample_off[n_clips] when channels > 1), clip k at
+ * [h_sample_off[k], h_sample_off[k+1]) in every channel. channels 1 .. 64.
+ * d_y: float32, clip k's outputs at the sum of the lengths of clips 0..k-1.
+ * Workspace: ae_resample_workspace_size(...), 256-byte aligned. Caller owns
+ * every buffer; nothing is allocated; the call is asynchronous on stream.
+ * Rates whose reduced output rate p makes the tap table exceed 2^26 entries
+ * are refused with AE_EUNSUPPORTED. Co-prime rates (large o) are computed
+ * from global memory, correctly but more slowly. */
+ae_status ae_resample(const float *d_x, int channels, int64_t ch_stride, const int64_t *h_sample_off, int n_clips,
+                      int32_t rate_in, int32_t rate_out, float *d_y, void *d_ws, size_t ws_bytes,
+                      ae_stream stream);
+
 /* --- kernel timing ------------------------------------------------------------ */
 
 /* Classes of the kernels the calls launch. */
@@ -261,7 +302,8 @@ typedef enum {
   AE_K_ATTENTION = 5,
   AE_K_LCONV = 6,    /* depthwise conv + RMS norm + SiLU */
   AE_K_ROWOP = 7,    /* residual / RMS-norm row passes */
-  AE_K_COUNT = 8
+  AE_K_RESAMPLE = 8, /* mixdown, resampler taps and FIR */
+  AE_K_COUNT = 9
 } ae_kernel_class;
 
 /* Kernel timing for measurement (the analogue of the page's

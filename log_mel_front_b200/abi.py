@@ -86,6 +86,9 @@ _sig("ae_last_error", C.c_char_p)
 _sig("ae_device_status", _st)
 _sig("ae_version", C.c_char_p)
 _sig("ae_logmel_noalloc", _st, _vp, _i64p, _i32, _vp, _vp)
+_sig("ae_resample_len", C.c_int64, C.c_int64, C.c_int32, C.c_int32)
+_sig("ae_resample_workspace_size", _sz, _i64p, _i32, C.c_int32, C.c_int32, _i32)
+_sig("ae_resample", _st, _vp, _i32, C.c_int64, _i64p, _i32, C.c_int32, C.c_int32, _vp, _vp, _sz, _vp)
 _sig("ae_profile_enable", _st, _i32)
 _sig("ae_profile_read", _st, C.POINTER(C.c_double), _i64p, C.POINTER(C.c_double), C.POINTER(C.c_double), _i64p)
 
@@ -93,9 +96,10 @@ _sig("ae_profile_read", _st, C.POINTER(C.c_double), _i64p, C.POINTER(C.c_double)
 EXPORTS = ("ae_num_frames", "ae_num_tokens", "ae_model_create", "ae_model_destroy", "ae_workspace_size",
            "ae_logmel", "ae_subsample", "ae_conformer_layer", "ae_encode", "ae_encode_host_workspace_size",
            "ae_encode_host", "ae_encode_host_async", "ae_attention_tables", "ae_local_attention", "ae_last_error", "ae_device_status",
-           "ae_version", "ae_profile_enable", "ae_profile_read", "ae_logmel_noalloc")
+           "ae_version", "ae_profile_enable", "ae_profile_read", "ae_logmel_noalloc", "ae_resample_len",
+           "ae_resample_workspace_size", "ae_resample")
 
-KERNEL_CLASSES = ("tables", "logmel", "conv0", "conv1", "gemm", "attention", "lconv", "rowop")
+KERNEL_CLASSES = ("tables", "logmel", "conv0", "conv1", "gemm", "attention", "lconv", "rowop", "resample")
 
 
 class AEError(RuntimeError):
@@ -234,6 +238,22 @@ def ae_version() -> str:
 
 def ae_profile_enable(on: bool = True):
     _check(lib.ae_profile_enable(1 if on else 0), "ae_profile_enable")
+
+
+def ae_resample_len(n_samples: int, rate_in: int, rate_out: int = 16000) -> int:
+    return lib.ae_resample_len(int(n_samples), int(rate_in), int(rate_out))
+
+
+def ae_resample_workspace_size(sample_off, rate_in: int, rate_out: int = 16000, channels: int = 1) -> int:
+    a, p = _off(sample_off)
+    return lib.ae_resample_workspace_size(p, len(a) - 1, int(rate_in), int(rate_out), int(channels))
+
+
+def ae_resample(d_x, channels: int, ch_stride: int, sample_off, rate_in: int, rate_out: int, d_y, d_ws,
+                ws_bytes: int, stream=None):
+    a, p = _off(sample_off)
+    _check(lib.ae_resample(_ptr(d_x), int(channels), int(ch_stride), p, len(a) - 1, int(rate_in), int(rate_out),
+                           _ptr(d_y), _ptr(d_ws), ws_bytes, _stream(stream)), "ae_resample")
 
 
 def ae_profile_read() -> dict:

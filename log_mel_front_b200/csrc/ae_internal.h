@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -85,6 +86,13 @@ struct ae_model {
   CUtensorMap tm_conv1, tm_in_proj, tm_out_proj, tm_embed;
   std::vector<ae::LayerDev> layers;
   std::vector<void *> allocs;
+  // ae_encode runs the two halves of a large batch on the caller's stream and
+  // on this side stream (fork and join through the two events), so that the
+  // tail waves of one half's kernels overlap the other's. The mutex keeps the
+  // fork/join sequence of concurrent calls on one model whole.
+  cudaStream_t side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  std::mutex split_mu;
 };
 
 namespace ae {
@@ -171,6 +179,31 @@ inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, siz
   cfg.stream = s;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
 }
+
+// Resampler (resample.cu): the rates reduced to o (in) and p (out), the cut-off
+// c in cycles per input sample, the window half-width 64 / c in input samples;
+// outputs in units of four: NT unit types, D input samples between units of a
+// type, W (padded W_pad) input offsets in a unit's window, the lowest offset
+// over all types; and the FIR's tiling (Q units of each of TG types per tile,
+// n_groups type groups, staged input span, tap rows staged or not, shared
+// memory).
+struct RsPlan {
+  int o = 1, p = 1;
+  double c = 0.0, half = 0.0;
+  int NT = 1, D = 1, W = 0, W_pad = 0, lo_min = 0, Q = 32, TG = 1, n_groups = 1, span = 0;
+  bool stage_coef = true;
+  size_t smem = 0;
+};
+int64_t rs_len(int64_t n, int rate_in, int rate_out);  // -1 for invalid arguments
+RsPlan rs_plan(int rate_in, int rate_out);
+cudaError_t launch_rs_table(const RsPlan &pl, float *coef, int32_t *lo, cudaStream_t s);
+cudaError_t launch_rs_mix(const float *x, int channels, int64_t ch_stride, int64_t n, float *mono, cudaStream_t s);
+cudaError_t launch_rs_fir(const RsPlan &pl, const float *mono, float *y, const float *coef, const int32_t *lo,
+                          const int64_t *in_off, const int64_t *out_off, const int32_t *tile_off, int n_clips,
+                          int n_tiles, cudaStream_t s);
+// Copies host words into device memory with kernel launches (the bytes travel
+// as kernel parameters), so the call stays asynchronous and capturable.
+cudaError_t launch_upload_bytes(const void *host, size_t bytes, void *dev, cudaStream_t s);
 
 unsigned *device_status_word();
 unsigned read_and_clear_status();

@@ -455,7 +455,7 @@ static ae_status check_ws(void *ws, size_t have, size_t need) {
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 // The encode sequence on device buffers (shared by ae_encode and ae_encode_host).
-static ae_status encode_dev(const ae_model *m, const float *d_wave, const ClipTables &T, float *d_out, void *d_ws,
+static ae_status encode_one(const ae_model *m, const float *d_wave, const ClipTables &T, float *d_out, void *d_ws,
                             const WsLayout &L, cudaStream_t s) {
   ClipTablesDev td;
   cudaError_t e = tables_t(T, d_ws, L, &td, true, s);
@@ -483,6 +483,61 @@ static ae_status encode_dev(const ae_model *m, const float *d_wave, const ClipTa
     if ((e = rowop_t(m, r, s)) != cudaSuccess) return cuda_fail(e, "head input");
   }
   if ((e = run_head(m, b, T.total_tokens, d_out, s)) != cudaSuccess) return cuda_fail(e, "head");
+  return AE_OK;
+}
+
+// Workspace of ae_encode: the layout of the whole batch plus room for the
+// rounding of two half-batch layouts (every region of a half is a prefix-sum
+// share of the whole, the stem regions dominate both halves' unions, and each
+// region rounds up to 256 bytes at most once more per half).
+constexpr size_t kSplitSlack = 64 * 1024;
+constexpr int64_t kSplitMinTokens = 4096;
+
+static size_t encode_ws_bytes(const ae_model *m, int64_t n_clips, int64_t frames, int64_t tokens) {
+  return ws_layout(m, n_clips, frames, tokens, true).total + kSplitSlack;
+}
+
+// Clips [a, b) of T as a table of their own (offsets rebased to clip a).
+static ClipTables sub_tables(const ClipTables &T, int a, int b) {
+  std::vector<int64_t> off(b - a + 1);
+  for (int i = a; i <= b; ++i) off[i - a] = T.sample_off[i] - T.sample_off[a];
+  ClipTables S;
+  build_tables(off.data(), b - a, kSamples, S, "h_sample_off");
+  return S;
+}
+
+// The whole forward. A batch of at least kSplitMinTokens tokens in two or
+// more clips runs as two halves of about equal token count, the first on s and
+// the second on the model's side stream, each with its own workspace layout;
+// the clips are independent, so the halves only share the weights. Outputs
+// land in the same rows as for one pass. Not while profiling (the per-kernel
+// event timing assumes one stream).
+static ae_status encode_dev(const ae_model *m, const float *d_wave, const ClipTables &T, float *d_out, void *d_ws,
+                            size_t ws_bytes, cudaStream_t s) {
+  const WsLayout L = ws_layout(m, T.n_clips, T.total_frames, T.total_tokens, true);
+  if (g_prof.on || T.n_clips < 2 || T.total_tokens < kSplitMinTokens || !m->side)
+    return encode_one(m, d_wave, T, d_out, d_ws, L, s);
+  int k = 1;  // first clip of the second half
+  while (k < T.n_clips - 1 && 2 * (int64_t)T.tok_off[k] < T.total_tokens) ++k;
+  const ClipTables A = sub_tables(T, 0, k), B = sub_tables(T, k, T.n_clips);
+  const WsLayout LA = ws_layout(m, A.n_clips, A.total_frames, A.total_tokens, true);
+  const WsLayout LB = ws_layout(m, B.n_clips, B.total_frames, B.total_tokens, true);
+  const size_t b_off = al256(LA.total);
+  if (b_off + LB.total > ws_bytes || A.total_tokens == 0 || B.total_tokens == 0)
+    return encode_one(m, d_wave, T, d_out, d_ws, L, s);
+  ae_model *mm = const_cast<ae_model *>(m);
+  std::lock_guard<std::mutex> guard(mm->split_mu);
+  cudaError_t e = cudaEventRecord(mm->fork, s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(mm->side, mm->fork, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "fork");
+  ae_status sa = encode_one(m, d_wave, A, d_out, d_ws, LA, s);
+  ae_status sb = sa ? sa
+                    : encode_one(m, d_wave + T.sample_off[k], B, d_out + (int64_t)T.tok_off[k] * m->cfg.embed_dim,
+                                 static_cast<uint8_t *>(d_ws) + b_off, LB, mm->side);
+  e = cudaEventRecord(mm->join, mm->side);  // joined whatever happened above
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, mm->join, 0);
+  if (sb) return sb;
+  if (e != cudaSuccess) return cuda_fail(e, "join");
   return AE_OK;
 }
 
@@ -549,6 +604,9 @@ ae_status ae_attention_tables(const float *relk, const float *pds, int hidden, i
 void ae_model_destroy(ae_model *m) {
   if (!m) return;
   for (void *p : m->allocs) cudaFree(p);
+  if (m->side) cudaStreamDestroy(m->side);
+  if (m->fork) cudaEventDestroy(m->fork);
+  if (m->join) cudaEventDestroy(m->join);
   delete m;
 }
 
@@ -599,6 +657,15 @@ ae_status ae_model_create(const ae_config *cfg, const ae_host_weights *w, ae_dty
   m->cfg = c;
   m->dtype = dtype;
   m->device = dev;
+  {
+    cudaError_t e = cudaStreamCreateWithFlags(&m->side, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&m->fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&m->join, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      ae_model_destroy(m);
+      return cuda_fail(e, "side stream");
+    }
+  }
   Uploader up{m};
   const int H = c.hidden;
   // conv0: taps minus their channel mean, and their channel covariance (float64)
@@ -714,7 +781,8 @@ ae_status ae_model_create(const ae_config *cfg, const ae_host_weights *w, ae_dty
 
 size_t ae_workspace_size(const ae_model *m, int64_t n_clips, int64_t total_frames, int64_t total_tokens) {
   if (n_clips < 0 || total_frames < 0 || total_tokens < 0) return 0;
-  return ws_layout(m, n_clips, total_frames, total_tokens, m != nullptr).total;
+  if (!m) return ws_layout(m, n_clips, total_frames, total_tokens, false).total;
+  return encode_ws_bytes(m, n_clips, total_frames, total_tokens);
 }
 
 ae_status ae_logmel(const float *d_wave, const int64_t *h_sample_off, int n_clips, float *d_mel, void *d_ws,
@@ -789,17 +857,17 @@ ae_status ae_encode(const ae_model *m, const float *d_wave, const int64_t *h_sam
   if ((st = build_tables(h_sample_off, n_clips, kSamples, T, "h_sample_off"))) return st;
   if (T.total_tokens > 0 && (!d_wave || !d_out)) return fail(AE_EINVAL, "d_wave or d_out is null");
   if (!aligned16(d_out)) return fail(AE_EINVAL, "d_out is not 16-byte aligned");
-  const WsLayout L = ws_layout(m, T.n_clips, T.total_frames, T.total_tokens, true);
+  const size_t need = encode_ws_bytes(m, T.n_clips, T.total_frames, T.total_tokens);
   if (n_clips == 0) return AE_OK;
-  if ((st = check_ws(d_ws, ws_bytes, L.total))) return st;
-  return encode_dev(m, d_wave, T, d_out, d_ws, L, reinterpret_cast<cudaStream_t>(stream));
+  if ((st = check_ws(d_ws, ws_bytes, need))) return st;
+  return encode_dev(m, d_wave, T, d_out, d_ws, need, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t ae_encode_host_workspace_size(const ae_model *m, const int64_t *h_sample_off, int n_clips) {
   ClipTables T;
   if (!m || build_tables(h_sample_off, n_clips, kSamples, T, "h_sample_off") != AE_OK) return 0;
-  const WsLayout L = ws_layout(m, T.n_clips, T.total_frames, T.total_tokens, true);
-  return L.total + al256((size_t)T.total_samples * 4) + al256((size_t)T.total_tokens * m->cfg.embed_dim * 4);
+  return encode_ws_bytes(m, T.n_clips, T.total_frames, T.total_tokens) + al256((size_t)T.total_samples * 4) +
+         al256((size_t)T.total_tokens * m->cfg.embed_dim * 4);
 }
 
 ae_status ae_encode_host_async(const ae_model *m, const float *h_wave, const int64_t *h_sample_off, int n_clips,
@@ -810,20 +878,20 @@ ae_status ae_encode_host_async(const ae_model *m, const float *h_wave, const int
   if ((st = build_tables(h_sample_off, n_clips, kSamples, T, "h_sample_off"))) return st;
   if (T.total_samples > 0 && !h_wave) return fail(AE_EINVAL, "h_wave is null");
   if (T.total_tokens > 0 && !h_out) return fail(AE_EINVAL, "h_out is null");
-  const WsLayout L = ws_layout(m, T.n_clips, T.total_frames, T.total_tokens, true);
+  const size_t enc = encode_ws_bytes(m, T.n_clips, T.total_frames, T.total_tokens);
   const size_t wave_b = al256((size_t)T.total_samples * 4);
   const size_t out_b = al256((size_t)T.total_tokens * m->cfg.embed_dim * 4);
   if (n_clips == 0) return AE_OK;
-  if ((st = check_ws(d_ws, ws_bytes, L.total + wave_b + out_b))) return st;
+  if ((st = check_ws(d_ws, ws_bytes, enc + wave_b + out_b))) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t *w = static_cast<uint8_t *>(d_ws);
-  float *d_wave = reinterpret_cast<float *>(w + L.total);
-  float *d_out = reinterpret_cast<float *>(w + L.total + wave_b);
+  float *d_wave = reinterpret_cast<float *>(w + enc);
+  float *d_out = reinterpret_cast<float *>(w + enc + wave_b);
   cudaError_t e;
   if (T.total_samples > 0 &&
       (e = cudaMemcpyAsync(d_wave, h_wave, (size_t)T.total_samples * 4, cudaMemcpyHostToDevice, s)) != cudaSuccess)
     return cuda_fail(e, "copy in");
-  if ((st = encode_dev(m, d_wave, T, d_out, d_ws, L, s))) return st;
+  if ((st = encode_dev(m, d_wave, T, d_out, d_ws, enc, s))) return st;
   if (T.total_tokens > 0 &&
       (e = cudaMemcpyAsync(h_out, d_out, (size_t)T.total_tokens * m->cfg.embed_dim * 4, cudaMemcpyDeviceToHost, s)) !=
           cudaSuccess)
@@ -871,6 +939,154 @@ ae_status ae_local_attention(const void *d_q, const void *d_k, const void *d_v, 
                                  T.total_tokens, d_out, ld_out, -INFINITY, INFINITY, s);
        })) != cudaSuccess)
     return cuda_fail(e, "attention");
+  return AE_OK;
+}
+
+// ------------------------------------------------------------------ mixdown and resampling
+
+namespace {
+constexpr int32_t kMaxRate = 1000000;
+constexpr int kMaxChannels = 64;
+constexpr int64_t kMaxRsTable = int64_t(1) << 26;  // taps in the per-call table
+constexpr int64_t kMaxRsSamples = int64_t(1) << 40;
+
+struct RsTables {
+  std::vector<int64_t> in_off, out_off;
+  std::vector<int32_t> tile_off;
+  int64_t total_in = 0, total_out = 0;
+  int64_t n_tiles = 0;
+};
+
+struct RsLayout {
+  size_t in_off = 0, out_off = 0, tile_off = 0, lo = 0, coef = 0, mono = 0, total = 0;
+};
+
+ae_status rs_check_rates(int32_t rate_in, int32_t rate_out) {
+  if (rate_in <= 0 || rate_out <= 0 || rate_in > kMaxRate || rate_out > kMaxRate)
+    return fail(AE_EINVAL, "rates must be in 1 .. 1000000");
+  return AE_OK;
+}
+
+ae_status rs_tables(const int64_t *off, int n, int32_t rate_in, int32_t rate_out, const RsPlan &pl, RsTables &t) {
+  if (n < 0) return fail(AE_EINVAL, "n_clips is negative");
+  if (n > kMaxClips) return fail(AE_EINVAL, "n_clips above 1048576");
+  if (!off) return fail(AE_EINVAL, "h_sample_off is null");
+  if (off[0] != 0) return fail(AE_EINVAL, "h_sample_off[0] must be 0");
+  t = RsTables();
+  t.in_off.assign(n + 1, 0);
+  t.out_off.assign(n + 1, 0);
+  t.tile_off.assign(n + 1, 0);
+  for (int i = 0; i < n; ++i) {
+    const int64_t len = off[i + 1] - off[i];
+    if (len < 0) return fail(AE_EINVAL, "h_sample_off is not non-decreasing at clip " + std::to_string(i));
+    t.in_off[i + 1] = off[i + 1];
+    const int64_t out = rs_len(len, rate_in, rate_out);
+    t.out_off[i + 1] = t.out_off[i] + out;
+    const int64_t units = (out + 3) / 4, per_type = (units + pl.NT - 1) / pl.NT;
+    const int64_t tiles = rate_in == rate_out ? 0 : (per_type + pl.Q - 1) / pl.Q;
+    if ((t.n_tiles + tiles) * pl.n_groups > INT32_MAX)
+      return fail(AE_EUNSUPPORTED, "too many resampler tiles in one call");
+    t.n_tiles += tiles;
+    t.tile_off[i + 1] = (int32_t)t.n_tiles;
+  }
+  t.total_in = off[n];
+  t.total_out = t.out_off[n];
+  if (t.total_in > kMaxRsSamples) return fail(AE_EINVAL, "more than 2^40 input samples");
+  return AE_OK;
+}
+
+RsLayout rs_layout(int n_clips, const RsPlan &pl, int64_t total_in, int channels, bool equal) {
+  RsLayout L;
+  size_t off = 0;
+  const size_t B1 = (size_t)n_clips + 1;
+  L.in_off = off;
+  off += al256(B1 * 8);
+  L.out_off = off;
+  off += al256(B1 * 8);
+  L.tile_off = off;
+  off += al256(B1 * 4);
+  L.lo = off;
+  off += equal ? 0 : al256((size_t)pl.NT * 4);
+  L.coef = off;
+  off += equal ? 0 : al256((size_t)pl.NT * pl.W_pad * 16);
+  L.mono = off;
+  off += (channels > 1 && !equal) ? al256((size_t)total_in * 4) : 0;
+  L.total = off;
+  return L;
+}
+}  // namespace
+
+int64_t ae_resample_len(int64_t n_samples, int32_t rate_in, int32_t rate_out) {
+  if (rate_in > kMaxRate || rate_out > kMaxRate) return -1;
+  return rs_len(n_samples, rate_in, rate_out);
+}
+
+size_t ae_resample_workspace_size(const int64_t *h_sample_off, int n_clips, int32_t rate_in, int32_t rate_out,
+                                  int channels) {
+  if (rs_check_rates(rate_in, rate_out) || channels < 1 || channels > kMaxChannels) return 0;
+  const RsPlan pl = rs_plan(rate_in, rate_out);
+  RsTables T;
+  if (rs_tables(h_sample_off, n_clips, rate_in, rate_out, pl, T) != AE_OK) return 0;
+  return rs_layout(n_clips, pl, T.total_in, channels, rate_in == rate_out).total;
+}
+
+ae_status ae_resample(const float *d_x, int channels, int64_t ch_stride, const int64_t *h_sample_off, int n_clips,
+                      int32_t rate_in, int32_t rate_out, float *d_y, void *d_ws, size_t ws_bytes,
+                      ae_stream stream) {
+  ae_status st = rs_check_rates(rate_in, rate_out);
+  if (st) return st;
+  if (channels < 1 || channels > kMaxChannels) return fail(AE_EINVAL, "channels must be in 1 .. 64");
+  const RsPlan pl = rs_plan(rate_in, rate_out);
+  const bool equal = rate_in == rate_out;
+  if (!equal && (int64_t)pl.NT * pl.W_pad * 4 > kMaxRsTable)
+    return fail(AE_EUNSUPPORTED, "the reduced output rate " + std::to_string(pl.p) + " needs a tap table above 2^26");
+  RsTables T;
+  if ((st = rs_tables(h_sample_off, n_clips, rate_in, rate_out, pl, T))) return st;
+  if (channels > 1 && ch_stride < T.total_in) return fail(AE_EINVAL, "ch_stride is below the packed sample count");
+  if (T.total_in > 0 && (!d_x || !d_y)) return fail(AE_EINVAL, "d_x or d_y is null");
+  const RsLayout L = rs_layout(n_clips, pl, T.total_in, channels, equal);
+  if (T.total_out == 0) return AE_OK;
+  if ((st = check_ws(d_ws, ws_bytes, L.total))) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *w = static_cast<uint8_t *>(d_ws);
+  cudaError_t e;
+  const double in_bytes = 4.0 * channels * (double)T.total_in, out_bytes = 4.0 * (double)T.total_out;
+  if (equal) {  // mono is the output
+    if ((e = timed(AE_K_RESAMPLE, 0.0, in_bytes + out_bytes, s, [&] {
+           return launch_rs_mix(d_x, channels, ch_stride, T.total_in, d_y, s);
+         })) != cudaSuccess)
+      return cuda_fail(e, "mixdown");
+    return AE_OK;
+  }
+  int64_t *in_off = reinterpret_cast<int64_t *>(w + L.in_off);
+  int64_t *out_off = reinterpret_cast<int64_t *>(w + L.out_off);
+  int32_t *tile_off = reinterpret_cast<int32_t *>(w + L.tile_off);
+  int32_t *lo = reinterpret_cast<int32_t *>(w + L.lo);
+  float *coef = reinterpret_cast<float *>(w + L.coef);
+  const float *mono = d_x;
+  if ((e = timed(AE_K_TABLES, 0.0, 0.0, s, [&] {
+         cudaError_t r = launch_upload_bytes(T.in_off.data(), T.in_off.size() * 8, in_off, s);
+         if (r == cudaSuccess) r = launch_upload_bytes(T.out_off.data(), T.out_off.size() * 8, out_off, s);
+         if (r == cudaSuccess) r = launch_upload_bytes(T.tile_off.data(), T.tile_off.size() * 4, tile_off, s);
+         return r;
+       })) != cudaSuccess)
+    return cuda_fail(e, "table upload");
+  if ((e = timed(AE_K_RESAMPLE, 0.0, 16.0 * pl.NT * pl.W_pad, s, [&] { return launch_rs_table(pl, coef, lo, s); })) !=
+      cudaSuccess)
+    return cuda_fail(e, "resampler taps");
+  if (channels > 1) {
+    float *m = reinterpret_cast<float *>(w + L.mono);
+    if ((e = timed(AE_K_RESAMPLE, 0.0, in_bytes + 4.0 * T.total_in, s, [&] {
+           return launch_rs_mix(d_x, channels, ch_stride, T.total_in, m, s);
+         })) != cudaSuccess)
+      return cuda_fail(e, "mixdown");
+    mono = m;
+  }
+  const double taps = (double)(2 * (int)std::ceil(pl.half) + 1);
+  if ((e = timed(AE_K_RESAMPLE, 2.0 * taps * (double)T.total_out, 4.0 * (double)T.total_in + out_bytes, s, [&] {
+         return launch_rs_fir(pl, mono, d_y, coef, lo, in_off, out_off, tile_off, n_clips, (int)T.n_tiles, s);
+       })) != cudaSuccess)
+    return cuda_fail(e, "resampler");
   return AE_OK;
 }
 

@@ -1,0 +1,284 @@
+// Channel mixdown and band-limited resampling (egemma2_audio.rs, to_mono_16k
+// and resample_hq): mono = float32 channel average; with the rates reduced by
+// their gcd to o (in) and p (out), output n sits at input position n o / p and
+//   y[n] = sum_m x[m] c sinc(t) I0(beta sqrt(1 - (t/64)^2)) / I0(beta),
+//   t = (m - n o / p) c,   c = 0.958 min(o, p) / o,   |t| < 64 zero crossings,
+// with ceil(p N / o) outputs and samples outside the clip taken as zero.
+//
+// Outputs are taken four at a time: unit u covers n = 4u .. 4u+3. Units of
+// the same type T = u mod NT (NT = p / gcd(p, 4)) have the same taps, and
+// consecutive units of one type sit D = 4 o / gcd(p, 4) input samples apart
+// (one frame of 441 samples for 44.1 kHz, 12 samples for 48 kHz). k_rs_table
+// evaluates, once per call and in float64, the taps of the four outputs of
+// every type at every input offset i of their common window (lo_T + i,
+// W_pad offsets), and stores them as one float4 per (T, i); zero outside each
+// output's 64 zero crossings.
+//
+// k_rs_fir: a CTA owns a tile of Q consecutive units of each of up to eight
+// types of one clip. It stages the input span the tile touches and the
+// types' tap rows in shared memory; a warp takes one (type, 32-unit group)
+// item at a time with lane = unit, so for every input offset the warp reads
+// one float4 of taps (the same shared-memory address for all lanes: a
+// broadcast) and each lane one input sample, and does four FMAs. Each lane
+// writes its unit's four outputs. When the span does not fit (large D, as for
+// co-prime rates) the FIR reads the input from global memory, and when the
+// tap rows do not fit it reads them from global memory too: correct, and
+// slower.
+#include <cmath>
+
+#include "ae_internal.h"
+#include "common.cuh"
+
+namespace ae {
+
+namespace {
+constexpr double kRsWidth = 64.0;
+constexpr double kRsRolloff = 0.958;
+constexpr double kRsBeta = 12.8;
+constexpr int kRsThreads = 256;
+constexpr int kRsWarps = kRsThreads / 32;
+constexpr size_t kRsSmemMax = 200 * 1024;  // staged input + staged output per CTA
+}  // namespace
+
+// I0(x) = sum_k ((x / 2)^2)^k / (k!)^2, summed while the terms still count.
+__device__ double rs_bessel_i0(double x) {
+  const double q = 0.25 * x * x;
+  double term = 1.0, sum = 1.0;
+  for (int k = 1; k < 400; ++k) {
+    term *= q / ((double)k * (double)k);
+    sum += term;
+    if (term < sum * 1e-17) break;
+  }
+  return sum;
+}
+
+// One thread per (type T, offset i): the taps of outputs 4T + r, r = 0..3,
+// at input lo_T + i (relative to the unit's base q D), lo_T = floor(4 T o / p
+// - 64 / c). Output 4T + r sits at input position 4 T o / p + r o / p.
+__global__ void k_rs_table(float4 *__restrict__ coef, int32_t *__restrict__ lo, int o, int p, int NT, int W_pad,
+                           double c, double half, double i0b) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)NT * W_pad) return;
+  const int T = (int)(idx / W_pad), i = (int)(idx % W_pad);
+  const double frac = 4.0 * (double)T * (double)o / (double)p;
+  const int l0 = (int)floor(frac - half);
+  if (i == 0) lo[T] = l0;
+  double v[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const double t = ((double)(l0 + i) - frac - (double)r * (double)o / (double)p) * c;
+    v[r] = 0.0;
+    if (fabs(t) < kRsWidth) {
+      const double q = t / kRsWidth;
+      const double win = rs_bessel_i0(kRsBeta * sqrt(1.0 - q * q)) / i0b;
+      const double pt = M_PI * t;
+      const double sinc = pt == 0.0 ? 1.0 : sin(pt) / pt;
+      v[r] = sinc * win * c;
+    }
+  }
+  coef[idx] = make_float4((float)v[0], (float)v[1], (float)v[2], (float)v[3]);
+}
+
+// mono[i] = (x_0[i] + ... + x_{C-1}[i]) / C in float32, channel order.
+__global__ void k_rs_mix(const float *__restrict__ x, int channels, int64_t ch_stride, int64_t n,
+                         float *__restrict__ mono) {
+  const float n_ch = (float)channels;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    float s = x[i];
+    for (int ch = 1; ch < channels; ++ch) s += x[ch * ch_stride + i];
+    mono[i] = s / n_ch;
+  }
+}
+
+struct RsArgs {
+  const float *x;           // mono input, packed clips
+  float *y;                 // packed outputs
+  const float4 *coef;       // [NT][W_pad]: taps of the unit's four outputs
+  const int32_t *lo;        // [NT]
+  const int64_t *in_off;    // [B + 1] input sample offsets
+  const int64_t *out_off;   // [B + 1] output sample offsets
+  const int32_t *tile_off;  // [B + 1] tile offsets
+  int n_clips, NT, D, W_pad, Q, TG, n_groups;
+  int lo_min, span;         // span: staged inputs per tile (0: read from global memory)
+  int stage_coef;           // the group's tap rows live in shared memory
+};
+
+__global__ void __launch_bounds__(kRsThreads) k_rs_fir(const RsArgs a) {
+  extern __shared__ __align__(16) float rs_smem[];
+  // tile = (clip, block of Q units of each type, group of TG types)
+  const int tile = blockIdx.x / a.n_groups, tg = blockIdx.x % a.n_groups;
+  int c = 0;
+  {
+    int l = 0, h = a.n_clips;  // last clip whose first tile is <= tile
+    while (h - l > 1) {
+      const int mid = (l + h) >> 1;
+      if (a.tile_off[mid] <= tile) l = mid; else h = mid;
+    }
+    c = l;
+  }
+  const int64_t in0 = a.in_off[c], n_in = a.in_off[c + 1] - in0;
+  const int64_t out0 = a.out_off[c], n_out = a.out_off[c + 1] - out0;
+  const int64_t q0 = (int64_t)(tile - a.tile_off[c]) * a.Q;
+  const int64_t base = q0 * a.D + a.lo_min;  // first input index the tile touches
+  const int T0 = tg * a.TG, n_types = min(a.TG, a.NT - T0);
+  const float *xin = a.x + in0;
+  float4 *cs = reinterpret_cast<float4 *>(rs_smem + a.span);  // [TG][W_pad] tap rows (stage_coef)
+  for (int i = threadIdx.x; i < a.span; i += kRsThreads) {
+    const int64_t m = base + i;
+    rs_smem[i] = (m >= 0 && m < n_in) ? __ldg(xin + m) : 0.f;
+  }
+  if (a.stage_coef) {
+    const float4 *src = a.coef + (int64_t)T0 * a.W_pad;
+    for (int i = threadIdx.x; i < n_types * a.W_pad; i += kRsThreads) cs[i] = __ldg(src + i);
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int groups = a.Q / 32, items = groups * n_types;
+  for (int item = warp; item < items; item += kRsWarps) {
+    const int tl = item % n_types, g = item / n_types, T = T0 + tl;
+    const int ql = g * 32 + lane;  // unit of type T within the tile
+    const float4 *cT = a.stage_coef ? cs + (int64_t)tl * a.W_pad : a.coef + (int64_t)T * a.W_pad;
+    const int64_t m0 = (q0 + ql) * a.D + a.lo[T];  // input index of offset 0
+    // two partial sums (even and odd offsets) per output
+    float4 e = make_float4(0.f, 0.f, 0.f, 0.f), d = e;
+    if (a.span > 0) {
+      const float *xr = rs_smem + (m0 - base);
+#pragma unroll 4
+      for (int i = 0; i < a.W_pad; i += 2) {
+        const float4 w0 = cT[i], w1 = cT[i + 1];
+        const float x0 = xr[i], x1 = xr[i + 1];
+        e.x = fmaf(w0.x, x0, e.x);
+        e.y = fmaf(w0.y, x0, e.y);
+        e.z = fmaf(w0.z, x0, e.z);
+        e.w = fmaf(w0.w, x0, e.w);
+        d.x = fmaf(w1.x, x1, d.x);
+        d.y = fmaf(w1.y, x1, d.y);
+        d.z = fmaf(w1.z, x1, d.z);
+        d.w = fmaf(w1.w, x1, d.w);
+      }
+    } else {
+      for (int i = 0; i < a.W_pad; i += 2) {
+        const float4 w0 = cT[i], w1 = cT[i + 1];
+        const int64_t m = m0 + i;
+        const float x0 = (m >= 0 && m < n_in) ? __ldg(xin + m) : 0.f;
+        const float x1 = (m + 1 >= 0 && m + 1 < n_in) ? __ldg(xin + m + 1) : 0.f;
+        e.x = fmaf(w0.x, x0, e.x);
+        e.y = fmaf(w0.y, x0, e.y);
+        e.z = fmaf(w0.z, x0, e.z);
+        e.w = fmaf(w0.w, x0, e.w);
+        d.x = fmaf(w1.x, x1, d.x);
+        d.y = fmaf(w1.y, x1, d.y);
+        d.z = fmaf(w1.z, x1, d.z);
+        d.w = fmaf(w1.w, x1, d.w);
+      }
+    }
+    const float r4[4] = {e.x + d.x, e.y + d.y, e.z + d.z, e.w + d.w};
+    const int64_t n0 = ((q0 + ql) * a.NT + T) * 4;  // first output of the unit
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+      if (n0 + r < n_out) a.y[out0 + n0 + r] = r4[r];
+  }
+}
+
+int64_t rs_len(int64_t n, int rate_in, int rate_out) {
+  if (n < 0 || rate_in <= 0 || rate_out <= 0) return -1;
+  if (rate_in == rate_out || n == 0) return n;
+  int64_t a = rate_in, b = rate_out;
+  while (b) {
+    const int64_t t = a % b;
+    a = b;
+    b = t;
+  }
+  const int64_t o = rate_in / a, p = rate_out / a;
+  return (p * n + o - 1) / o;
+}
+
+RsPlan rs_plan(int rate_in, int rate_out) {
+  RsPlan pl;
+  int64_t a = rate_in, b = rate_out;
+  while (b) {
+    const int64_t t = a % b;
+    a = b;
+    b = t;
+  }
+  pl.o = (int)(rate_in / a);
+  pl.p = (int)(rate_out / a);
+  pl.c = kRsRolloff * (double)std::min(pl.o, pl.p) / (double)pl.o;
+  pl.half = kRsWidth / pl.c;
+  const int g4 = pl.p % 4 == 0 ? 4 : (pl.p % 2 == 0 ? 2 : 1);  // gcd(p, 4)
+  pl.NT = pl.p / g4;
+  pl.D = (int)(4 * (int64_t)pl.o / g4);
+  // a unit's four outputs span 3 o / p input samples; each reaches half to either side
+  pl.W = (int)std::ceil(2.0 * pl.half + 3.0 * pl.o / pl.p) + 3;
+  pl.W_pad = (pl.W + 7) & ~7;
+  pl.lo_min = (int)std::floor(-pl.half) - 1;  // <= lo_T for every type
+  // a tile: Q units of each of (up to) TG types; enough (type, 32-unit group)
+  // items for the CTA's warps; the staged input span and the group's tap rows
+  // within the shared-memory budget
+  pl.TG = std::min(pl.NT, kRsWarps);
+  pl.n_groups = (pl.NT + pl.TG - 1) / pl.TG;
+  int groups = std::max(1, kRsWarps / pl.TG);
+  // lo_T < 4 T o / p <= D - 4 o / p, so offsets stay below Q D + W_pad - lo_min
+  auto span_of = [&](int q) -> int64_t { return (int64_t)q * pl.D + pl.W_pad - pl.lo_min + 2; };
+  const int64_t coef_bytes = 16 * (int64_t)pl.TG * pl.W_pad;
+  while (groups > 1 && 4 * span_of(32 * groups) + coef_bytes > (int64_t)kRsSmemMax) groups /= 2;
+  pl.Q = 32 * groups;
+  pl.stage_coef = coef_bytes <= (int64_t)kRsSmemMax / 2;
+  const int64_t span_b = 4 * span_of(pl.Q);
+  pl.span = span_b + (pl.stage_coef ? coef_bytes : 0) <= (int64_t)kRsSmemMax ? (int)span_of(pl.Q) : 0;
+  pl.span = (pl.span + 3) & ~3;  // the tap rows that follow stay 16-byte aligned
+  pl.smem = 4 * (size_t)pl.span + (pl.stage_coef ? (size_t)coef_bytes : 0);
+  return pl;
+}
+
+cudaError_t launch_rs_table(const RsPlan &pl, float *coef, int32_t *lo, cudaStream_t s) {
+  const int64_t n = (int64_t)pl.NT * pl.W_pad;
+  const double i0b = [] {
+    double q = 0.25 * kRsBeta * kRsBeta, term = 1.0, sum = 1.0;
+    for (int k = 1; k < 400; ++k) {
+      term *= q / ((double)k * (double)k);
+      sum += term;
+      if (term < sum * 1e-17) break;
+    }
+    return sum;
+  }();
+  return launch_k(k_rs_table, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, reinterpret_cast<float4 *>(coef),
+                  lo, pl.o, pl.p, pl.NT, pl.W_pad, pl.c, pl.half, i0b);
+}
+
+cudaError_t launch_rs_mix(const float *x, int channels, int64_t ch_stride, int64_t n, float *mono, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t blocks = std::min<int64_t>((n + 255) / 256, 148 * 16);
+  return launch_k(k_rs_mix, dim3((unsigned)blocks), dim3(256), 0, s, x, channels, ch_stride, n, mono);
+}
+
+cudaError_t launch_rs_fir(const RsPlan &pl, const float *mono, float *y, const float *coef, const int32_t *lo,
+                          const int64_t *in_off, const int64_t *out_off, const int32_t *tile_off, int n_clips,
+                          int n_tiles, cudaStream_t s) {
+  if (n_tiles <= 0) return cudaSuccess;
+  if (pl.smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(k_rs_fir, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRsSmemMax);
+    if (e != cudaSuccess) return e;
+  }
+  RsArgs a;
+  a.x = mono;
+  a.y = y;
+  a.coef = reinterpret_cast<const float4 *>(coef);
+  a.lo = lo;
+  a.in_off = in_off;
+  a.out_off = out_off;
+  a.tile_off = tile_off;
+  a.n_clips = n_clips;
+  a.NT = pl.NT;
+  a.D = pl.D;
+  a.W_pad = pl.W_pad;
+  a.Q = pl.Q;
+  a.TG = pl.TG;
+  a.n_groups = pl.n_groups;
+  a.lo_min = pl.lo_min;
+  a.span = pl.span;
+  a.stage_coef = pl.stage_coef ? 1 : 0;
+  return launch_k(k_rs_fir, dim3((unsigned)((int64_t)n_tiles * pl.n_groups)), dim3(kRsThreads), pl.smem, s, a);
+}
+
+}  // namespace ae

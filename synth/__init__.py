@@ -205,6 +205,29 @@ def model_weights(workload: str, n_layers: int | None = None, bf16: bool | None 
 
 # ----------------------------------------------------------------- attention microbench
 
+# Input conditioning (mixdown + resampling to 16 kHz): 64 stereo clips of 30 s
+# at 44.1 kHz, the common consumer source rate, each channel N(0, 0.2) noise
+# plus three sinusoids of 50-20000 Hz (some above the new Nyquist).
+RS_CLIPS = 64
+RS_RATE = 44100
+RS_SECONDS = 30
+
+
+def resample_clip(index: int, n: int | None = None, rate: int = RS_RATE, channels: int = 2) -> list[np.ndarray]:
+    """One clip of the resampling workload: a list of `channels` float32 arrays."""
+    n = rate * RS_SECONDS if n is None else n
+    rng = _rng(9, index)
+    t = np.arange(n, dtype=np.float64) / rate
+    out = []
+    for _ in range(channels):
+        x = 0.2 * rng.standard_normal(n)
+        for _ in range(3):
+            f = rng.uniform(50.0, 20000.0)
+            x = x + rng.uniform(0.05, 0.3) * np.sin(2 * np.pi * f * t + rng.uniform(0, 2 * np.pi))
+        out.append(x.astype(np.float32))
+    return out
+
+
 ATT_SEQS = 32
 ATT_T = 8192
 

@@ -236,6 +236,24 @@ def test_packing_is_bit_invariant_on_gpu(m_tower):
         assert np.array_equal(alone, g[off[i]:off[i + 1]]), i
 
 
+def test_two_half_batches_on_two_streams_are_bit_identical(m_tower):
+    """A batch of 4096+ tokens runs as two halves on two streams; with kernel
+    timing on, ae_encode takes a single pass on one stream. The two results
+    are bit for bit the same (every output row depends on its clip alone)."""
+    rng = np.random.default_rng(17)
+    lens = [480000] * 6 + [320000, 17, 240000, 1000]
+    clips = [(0.3 * rng.standard_normal(n)).astype(np.float32) for n in lens]
+    assert sum(O.num_tokens(len(c)) for c in clips) >= 4096
+    split, _ = gpu_encode(m_tower, clips)
+    ae.ae_profile_enable(True)
+    try:
+        single, _ = gpu_encode(m_tower, clips)
+    finally:
+        ae.ae_profile_enable(False)
+    assert np.all(np.isfinite(split))
+    assert np.array_equal(split, single)
+
+
 def test_encode_host_async_two_streams_match_device_path(m_tower):
     """ae_encode_host_async on two streams with their own workspaces, four
     calls in flight: each output equals ae_encode's, bit for bit."""
