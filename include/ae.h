@@ -198,7 +198,9 @@ ae_status ae_encode_host(const ae_model *m, const float *h_wave, const int64_t *
  * enqueued on `stream`. h_wave, h_out and d_ws belong to the call until the
  * stream has reached this point (synchronize it, or wait on an event recorded
  * after the call). Calls on different streams with their own workspaces and
- * output buffers overlap one batch's copies with another's kernels. */
+ * output buffers overlap one batch's copies with another's kernels; each call
+ * runs its batch as one pass on its stream (ae_encode and ae_encode_host split
+ * a large batch in two halves on two streams instead). */
 ae_status ae_encode_host_async(const ae_model *m, const float *h_wave, const int64_t *h_sample_off,
                                int n_clips, float *h_out, void *d_ws, size_t ws_bytes, ae_stream stream);
 

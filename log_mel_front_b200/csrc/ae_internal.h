@@ -39,6 +39,7 @@ enum EpiMode : int {
   EPI_BF16 = 1,       // v = clamp(acc) -> act
   EPI_SILU = 2,       // v = clamp2(silu(clamp(acc))) -> act
   EPI_GLU = 3,        // columns (2c, 2c+1) -> clamp, a * sigmoid(b) -> act column c
+  EPI_ADD_F32 = 4,    // out += clamp(acc): a float residual update, one add per element
 };
 
 struct EpiArgs {
@@ -87,11 +88,14 @@ struct ae_model {
   std::vector<ae::LayerDev> layers;
   std::vector<void *> allocs;
   // ae_encode runs the two halves of a large batch on the caller's stream and
-  // on this side stream (fork and join through the two events), so that the
-  // tail waves of one half's kernels overlap the other's. The mutex keeps the
-  // fork/join sequence of concurrent calls on one model whole.
-  cudaStream_t side = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
+  // on a side stream (fork and join through events), so that the tail waves
+  // of one half's kernels overlap the other's. Consecutive calls take the two
+  // side streams in turn, so that calls pipelined on two caller streams do
+  // not queue their second halves behind each other. The mutex keeps each
+  // call's fork/join sequence whole.
+  cudaStream_t side[2] = {nullptr, nullptr};
+  cudaEvent_t fork[2] = {nullptr, nullptr}, join[2] = {nullptr, nullptr};
+  int next_side = 0;
   std::mutex split_mu;
 };
 

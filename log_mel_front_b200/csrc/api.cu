@@ -75,7 +75,7 @@ static cudaError_t gemm_t(const ae_model *m, const void *x, int64_t M, int K, co
                           int N, int mode, const EpiArgs &ep, cudaStream_t s) {
   const double a = (double)act_bytes(m);
   const double out_cols = mode == EPI_GLU ? N / 2 : N;
-  const double out_b = mode == EPI_F32 ? 4.0 : a;
+  const double out_b = (mode == EPI_F32 || mode == EPI_ADD_F32) ? 4.0 : a;
   const double bytes = a * ((double)M * K + (double)N * K) + out_b * (double)M * out_cols;
   return timed(AE_K_GEMM, 2.0 * (double)M * N * K, bytes, s, [&] { return gemm(m, x, M, K, w, tmW, N, mode, ep, s); });
 }
@@ -382,10 +382,11 @@ static cudaError_t run_layer(const ae_model *m, int li, const Bufs &b, int64_t T
     AE_TRY(timed(AE_K_LCONV, 0.0, (double)T * 2 * H * act, s, [&] {
       return launch_lconv(m, b.big, L.lc_dw, L.lc_norm, L.c_lc_end.lo_in, L.c_lc_end.hi_in, b.o, b.pos, T, s);
     }));
-    AE_TRY(gemm_t(m, b.o, T, H, L.lc_end, tc ? &L.tm_lc_end : nullptr, H, y_mode,
-                  ep_of(b.y, H, L.c_lc_end.lo_out, L.c_lc_end.hi_out), s));
+    // this residual is a plain add (no norm), so the projection adds its clamped
+    // output into h itself; the row pass only forms the next operand
+    AE_TRY(gemm_t(m, b.o, T, H, L.lc_end, tc ? &L.tm_lc_end : nullptr, H, EPI_ADD_F32,
+                  ep_of(b.h, H, L.c_lc_end.lo_out, L.c_lc_end.hi_out), s));
     RowArgs r = row_of(b.h, H, T);
-    r.y = b.y; r.s = 1.0f; r.y_norm = 0;
     r.a_out = b.a; r.w_next = L.ff2_pre; r.lo = L.c_ff2_w1.lo_in; r.hi = L.c_ff2_w1.hi_in;
     AE_TRY(rowop_t(m, r, s));
   }
@@ -511,11 +512,13 @@ static ClipTables sub_tables(const ClipTables &T, int a, int b) {
 // the second on the model's side stream, each with its own workspace layout;
 // the clips are independent, so the halves only share the weights. Outputs
 // land in the same rows as for one pass. Not while profiling (the per-kernel
-// event timing assumes one stream).
+// event timing assumes one stream), and not when the caller asks for one pass
+// (the asynchronous host entry point, whose callers overlap whole calls on
+// their own streams: measured, a second split only adds contention there).
 static ae_status encode_dev(const ae_model *m, const float *d_wave, const ClipTables &T, float *d_out, void *d_ws,
-                            size_t ws_bytes, cudaStream_t s) {
+                            size_t ws_bytes, cudaStream_t s, bool may_split) {
   const WsLayout L = ws_layout(m, T.n_clips, T.total_frames, T.total_tokens, true);
-  if (g_prof.on || T.n_clips < 2 || T.total_tokens < kSplitMinTokens || !m->side)
+  if (!may_split || g_prof.on || T.n_clips < 2 || T.total_tokens < kSplitMinTokens || !m->side[0])
     return encode_one(m, d_wave, T, d_out, d_ws, L, s);
   int k = 1;  // first clip of the second half
   while (k < T.n_clips - 1 && 2 * (int64_t)T.tok_off[k] < T.total_tokens) ++k;
@@ -527,15 +530,18 @@ static ae_status encode_dev(const ae_model *m, const float *d_wave, const ClipTa
     return encode_one(m, d_wave, T, d_out, d_ws, L, s);
   ae_model *mm = const_cast<ae_model *>(m);
   std::lock_guard<std::mutex> guard(mm->split_mu);
-  cudaError_t e = cudaEventRecord(mm->fork, s);
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(mm->side, mm->fork, 0);
+  const int si = mm->next_side;
+  mm->next_side ^= 1;
+  cudaStream_t side = mm->side[si];
+  cudaError_t e = cudaEventRecord(mm->fork[si], s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(side, mm->fork[si], 0);
   if (e != cudaSuccess) return cuda_fail(e, "fork");
   ae_status sa = encode_one(m, d_wave, A, d_out, d_ws, LA, s);
   ae_status sb = sa ? sa
                     : encode_one(m, d_wave + T.sample_off[k], B, d_out + (int64_t)T.tok_off[k] * m->cfg.embed_dim,
-                                 static_cast<uint8_t *>(d_ws) + b_off, LB, mm->side);
-  e = cudaEventRecord(mm->join, mm->side);  // joined whatever happened above
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, mm->join, 0);
+                                 static_cast<uint8_t *>(d_ws) + b_off, LB, side);
+  e = cudaEventRecord(mm->join[si], side);  // joined whatever happened above
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, mm->join[si], 0);
   if (sb) return sb;
   if (e != cudaSuccess) return cuda_fail(e, "join");
   return AE_OK;
@@ -604,9 +610,11 @@ ae_status ae_attention_tables(const float *relk, const float *pds, int hidden, i
 void ae_model_destroy(ae_model *m) {
   if (!m) return;
   for (void *p : m->allocs) cudaFree(p);
-  if (m->side) cudaStreamDestroy(m->side);
-  if (m->fork) cudaEventDestroy(m->fork);
-  if (m->join) cudaEventDestroy(m->join);
+  for (int i = 0; i < 2; ++i) {
+    if (m->side[i]) cudaStreamDestroy(m->side[i]);
+    if (m->fork[i]) cudaEventDestroy(m->fork[i]);
+    if (m->join[i]) cudaEventDestroy(m->join[i]);
+  }
   delete m;
 }
 
@@ -658,9 +666,12 @@ ae_status ae_model_create(const ae_config *cfg, const ae_host_weights *w, ae_dty
   m->dtype = dtype;
   m->device = dev;
   {
-    cudaError_t e = cudaStreamCreateWithFlags(&m->side, cudaStreamNonBlocking);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&m->fork, cudaEventDisableTiming);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&m->join, cudaEventDisableTiming);
+    cudaError_t e = cudaSuccess;
+    for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
+      e = cudaStreamCreateWithFlags(&m->side[i], cudaStreamNonBlocking);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&m->fork[i], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&m->join[i], cudaEventDisableTiming);
+    }
     if (e != cudaSuccess) {
       ae_model_destroy(m);
       return cuda_fail(e, "side stream");
@@ -860,7 +871,7 @@ ae_status ae_encode(const ae_model *m, const float *d_wave, const int64_t *h_sam
   const size_t need = encode_ws_bytes(m, T.n_clips, T.total_frames, T.total_tokens);
   if (n_clips == 0) return AE_OK;
   if ((st = check_ws(d_ws, ws_bytes, need))) return st;
-  return encode_dev(m, d_wave, T, d_out, d_ws, need, reinterpret_cast<cudaStream_t>(stream));
+  return encode_dev(m, d_wave, T, d_out, d_ws, need, reinterpret_cast<cudaStream_t>(stream), true);
 }
 
 size_t ae_encode_host_workspace_size(const ae_model *m, const int64_t *h_sample_off, int n_clips) {
@@ -870,8 +881,8 @@ size_t ae_encode_host_workspace_size(const ae_model *m, const int64_t *h_sample_
          al256((size_t)T.total_tokens * m->cfg.embed_dim * 4);
 }
 
-ae_status ae_encode_host_async(const ae_model *m, const float *h_wave, const int64_t *h_sample_off, int n_clips,
-                               float *h_out, void *d_ws, size_t ws_bytes, ae_stream stream) {
+static ae_status encode_host(const ae_model *m, const float *h_wave, const int64_t *h_sample_off, int n_clips,
+                             float *h_out, void *d_ws, size_t ws_bytes, ae_stream stream, bool may_split) {
   ae_status st = check_model(m);
   if (st) return st;
   ClipTables T;
@@ -891,7 +902,7 @@ ae_status ae_encode_host_async(const ae_model *m, const float *h_wave, const int
   if (T.total_samples > 0 &&
       (e = cudaMemcpyAsync(d_wave, h_wave, (size_t)T.total_samples * 4, cudaMemcpyHostToDevice, s)) != cudaSuccess)
     return cuda_fail(e, "copy in");
-  if ((st = encode_dev(m, d_wave, T, d_out, d_ws, enc, s))) return st;
+  if ((st = encode_dev(m, d_wave, T, d_out, d_ws, enc, s, may_split))) return st;
   if (T.total_tokens > 0 &&
       (e = cudaMemcpyAsync(h_out, d_out, (size_t)T.total_tokens * m->cfg.embed_dim * 4, cudaMemcpyDeviceToHost, s)) !=
           cudaSuccess)
@@ -899,9 +910,14 @@ ae_status ae_encode_host_async(const ae_model *m, const float *h_wave, const int
   return AE_OK;
 }
 
+ae_status ae_encode_host_async(const ae_model *m, const float *h_wave, const int64_t *h_sample_off, int n_clips,
+                               float *h_out, void *d_ws, size_t ws_bytes, ae_stream stream) {
+  return encode_host(m, h_wave, h_sample_off, n_clips, h_out, d_ws, ws_bytes, stream, false);
+}
+
 ae_status ae_encode_host(const ae_model *m, const float *h_wave, const int64_t *h_sample_off, int n_clips,
                          float *h_out, void *d_ws, size_t ws_bytes, ae_stream stream) {
-  ae_status st = ae_encode_host_async(m, h_wave, h_sample_off, n_clips, h_out, d_ws, ws_bytes, stream);
+  ae_status st = encode_host(m, h_wave, h_sample_off, n_clips, h_out, d_ws, ws_bytes, stream, true);
   if (st) return st;
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "stream");

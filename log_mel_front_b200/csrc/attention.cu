@@ -62,7 +62,7 @@ constexpr uint32_t OFF_P = OFF_V + 2 * AT_V_REGION;
 constexpr uint32_t OFF_O = OFF_P + 3 * AT_P_REGION;
 constexpr uint32_t OFF_BAR = OFF_O + 4 * 2 * AT_O_BOX;
 constexpr size_t AT_SMEM = OFF_BAR + 1024 + 1024;          // barriers + q scales, alignment slack
-constexpr int AT_THREADS = 192;                           // producer warp, MMA warp, 4 softmax warps
+constexpr int AT_THREADS = 320;                           // producer warp, MMA warp, 8 softmax warps
 constexpr uint32_t AT_TMEM_COLS = 512;                    // S at column 0, O at column 256
 constexpr uint32_t AT_O_COL = 256;
 constexpr uint32_t AT_QK_BYTES = 2 * AT_Q_REGION + 2 * AT_KEYS * 128;
@@ -92,11 +92,11 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(qk_full, 1);
     mbar_init(v_full, 1);
-    mbar_init(q_ready, 128);
+    mbar_init(q_ready, 256);
     mbar_init(s_full, 1);
     mbar_init(p_full, 128);
     mbar_init(o_full, 1);
-    mbar_init(o_empty, 128);
+    mbar_init(o_empty, 256);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmO);
   }
-  if (threadIdx.x >= 64) s_qs[threadIdx.x - 64] = qscale[threadIdx.x - 64];
+  if (threadIdx.x >= 64 && threadIdx.x < 64 + kHeadDim) s_qs[threadIdx.x - 64] = qscale[threadIdx.x - 64];
   if (warp == 1) {
     tmem_alloc(tmem_slot, AT_TMEM_COLS);
     tmem_relinquish();
@@ -176,11 +176,13 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       *abort_flag = 1;
     }
   } else if (warp >= 2) {
-    // ---------------- softmax warps: thread of TMEM lane / tile row r
-    const int qw = warp & 3, r = 32 * qw + lane, r7 = r & 7, tid = threadIdx.x - 64;
-    uint8_t *box = sO + (warp - 2) * 2 * AT_O_BOX;
+    // ---------------- softmax warps: two per TMEM lane quarter, thread = tile row r;
+    // warp half hw takes head dims 64 hw .. +63 of q and of the output, and the
+    // hw = 0 warps the softmax of their rows
+    const int qw = warp & 3, hw = (warp - 2) >> 2, r = 32 * qw + lane, r7 = r & 7, tid = threadIdx.x - 64;
+    uint8_t *box = sO + (qw * 2 + hw) * AT_O_BOX;
     // P outside the band and the zero rows 156..159 of the B operand stay zero
-    for (int i = tid; i < (int)(3 * AT_P_REGION / 16); i += 128) reinterpret_cast<uint4 *>(sP)[i] = make_uint4(0, 0, 0, 0);
+    for (int i = tid; i < (int)(3 * AT_P_REGION / 16); i += 256) reinterpret_cast<uint4 *>(sP)[i] = make_uint4(0, 0, 0, 0);
     if (tid < 64) {
       const int rr = AT_KEYS + 12 + (tid >> 4), g = tid & 15;
       *reinterpret_cast<uint4 *>(sKR + (g >> 3) * AT_KR_REGION + rr * 128 + (((g & 7) ^ (rr & 7)) << 4)) =
@@ -194,7 +196,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       // ---- q s as hi + lo bf16 tiles, and R / k_scale under the k rows
       if (!__all_sync(0xffffffffu, mbar_wait(qk_full, it & 1))) { ok = false; break; }
 #pragma unroll 4
-      for (int j = 0; j < 16; ++j) {
+      for (int j = 8 * hw; j < 8 * hw + 8; ++j) {
         const uint32_t off = (j >> 3) * AT_Q_REGION + r * 128 + (((j & 7) ^ r7) << 4);
         const uint4 w = *reinterpret_cast<const uint4 *>(sQ + off);
         const float4 s0 = reinterpret_cast<const float4 *>(s_qs)[2 * j], s1 = reinterpret_cast<const float4 *>(s_qs)[2 * j + 1];
@@ -209,7 +211,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         *reinterpret_cast<uint4 *>(sQ + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
         *reinterpret_cast<uint4 *>(sQL + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
-      for (int rr = tid >> 4; rr < kLeft; rr += 8) {
+      for (int rr = tid >> 4; rr < kLeft; rr += 16) {
         const int g = tid & 15, row = AT_KEYS + rr;
         const float4 a = *reinterpret_cast<const float4 *>(R + (size_t)rr * kHidden + h * kHeadDim + g * 8);
         const float4 b = *reinterpret_cast<const float4 *>(R + (size_t)rr * kHidden + h * kHeadDim + g * 8 + 4);
@@ -219,7 +221,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       }
       fence_async_smem();
       mbar_arrive(q_ready);
-      // ---- scores -> probabilities -> banded P
+      // ---- scores -> probabilities -> banded P (warps of half 0)
+      if (hw == 0) {
       if (!__all_sync(0xffffffffu, mbar_wait(s_full, it & 1))) { ok = false; break; }
       tc_fence_after();
       uint32_t a32[32], a16[16], u16[16];
@@ -279,17 +282,18 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       tc_fence_before();
       fence_async_smem();
       mbar_arrive(p_full);
-      // ---- O rows out
+      }
+      // ---- O rows out: head dims 64 hw .. +63
       if (!__all_sync(0xffffffffu, mbar_wait(o_full, it & 1))) { ok = false; break; }
       tc_fence_after();
       if (lane == 0) bulk_wait_read<0>();  // the previous item's stores are done with the boxes
       __syncwarp();
 #pragma unroll 1
-      for (int c = 0; c < kHeadDim / 32; ++c) {
+      for (int c = 2 * hw; c < 2 * hw + 2; ++c) {
         uint32_t o[32];
         tmem_ld32(trow + AT_O_COL + 32 * c, o);
         tmem_ld_wait();
-        uint8_t *line = box + (c >> 1) * AT_O_BOX + lane * 128;
+        uint8_t *line = box + lane * 128;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int g = (c & 1) * 4 + j;
@@ -305,8 +309,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       fence_async_smem();
       __syncwarp();
       if (lane == 0 && t0 + 32 * qw < T) {
-        tma_store_2d(&tmO, box, h * kHeadDim, t0 + 32 * qw);
-        tma_store_2d(&tmO, box + AT_O_BOX, h * kHeadDim + 64, t0 + 32 * qw);
+        tma_store_2d(&tmO, box, h * kHeadDim + 64 * hw, t0 + 32 * qw);
         bulk_commit();
       }
     }

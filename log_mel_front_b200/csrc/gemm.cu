@@ -64,8 +64,8 @@ __device__ __forceinline__ void epi_stage(const EpiArgs &ep, int col, const uint
   float v[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-  if (MODE == EPI_F32) {
-    if (ep.bias) {
+  if (MODE == EPI_F32 || MODE == EPI_ADD_F32) {
+    if (MODE == EPI_F32 && ep.bias) {
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] += __ldg(ep.bias + col + i);
     }
@@ -315,10 +315,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     // swizzle: conflict-free), which the warp reads back row by row to write 4
     // full 128-byte row segments per store instruction (measured faster for
     // f32, slower for bf16, than the direct sector stores).
-    constexpr int LOADS_PER_BOX = MODE == EPI_F32 ? 1 : (MODE == EPI_GLU ? 4 : 2);  // 32-column TMEM loads
-    constexpr int OUT_COLS_PER_BOX = MODE == EPI_F32 ? 32 : 64;                     // 128 bytes of output
+    constexpr bool F32_OUT = MODE == EPI_F32 || MODE == EPI_ADD_F32;
+    constexpr int LOADS_PER_BOX = F32_OUT ? 1 : (MODE == EPI_GLU ? 4 : 2);  // 32-column TMEM loads
+    constexpr int OUT_COLS_PER_BOX = F32_OUT ? 32 : 64;                     // 128 bytes of output
     constexpr int GRANULES_PER_LOAD = 8 / LOADS_PER_BOX;
-    constexpr int ES = MODE == EPI_F32 ? 4 : 2;
+    constexpr int ES = F32_OUT ? 4 : 2;
     const int q = warp & 3, half = (warp - 2) >> 2;
     uint8_t *box = epi_smem + (warp - 2) * LINE_BYTES;
     const uint32_t tempty_leader = map_to_rank(&tempty[0], 0);
@@ -338,7 +339,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       const int ocol0 = MODE == EPI_GLU ? col0 / 2 : col0;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + half * (BN / 2));
       auto stage = [&](int c, const uint32_t(&r)[32]) {
-        if (MODE != EPI_F32) {  // bf16 rows: 32-byte stores straight from registers
+        if (!F32_OUT) {  // bf16 rows: 32-byte stores straight from registers
           if (row0 + lane < M) epi_store32<MODE>(ep, row0 + lane, col0 + c * 32, r);
           return;
         }
@@ -354,7 +355,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
           for (int i = 0; i < 8; ++i) {
             const int rr = (lane >> 3) + 4 * i;
             const uint4 v = *reinterpret_cast<const uint4 *>(box + rr * 128 + ((g ^ (rr & 7)) << 4));
-            if (row0 + rr < M) *reinterpret_cast<uint4 *>(dst + (int64_t)(row0 + rr) * ep.ld * ES) = v;
+            if (row0 + rr < M) {
+              uint8_t *p = dst + (int64_t)(row0 + rr) * ep.ld * ES;
+              if (MODE == EPI_ADD_F32)  // one vector add per 4 elements; no other thread touches them
+                asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(__uint_as_float(v.x)),
+                             "f"(__uint_as_float(v.y)), "f"(__uint_as_float(v.z)), "f"(__uint_as_float(v.w))
+                             : "memory");
+              else
+                *reinterpret_cast<uint4 *>(p) = v;
+            }
           }
           __syncwarp();
         }
@@ -450,6 +459,10 @@ __global__ void __launch_bounds__(256) k_gemm_f32(const float *__restrict__ A, c
     if (MODE == EPI_GLU) {
       o[col / 2] = v[0] / (1.0f + expf(-v[1]));
       o[col / 2 + 1] = v[2] / (1.0f + expf(-v[3]));
+    } else if (MODE == EPI_ADD_F32) {
+      float4 *p = reinterpret_cast<float4 *>(o + col);
+      const float4 h = *p;
+      *p = make_float4(h.x + v[0], h.y + v[1], h.z + v[2], h.w + v[3]);
     } else {
       *reinterpret_cast<float4 *>(o + col) = make_float4(v[0], v[1], v[2], v[3]);
     }
@@ -543,6 +556,7 @@ cudaError_t gemm(const ae_model *m, const void *x, int64_t M, int K, const void 
     }
     switch (mode) {
       case EPI_F32: return launch_tc<EPI_F32>(tA, *tmW, ep, (int)M, N, K, s);
+      case EPI_ADD_F32: return launch_tc<EPI_ADD_F32>(tA, *tmW, ep, (int)M, N, K, s);
       case EPI_BF16: return launch_tc<EPI_BF16>(tA, *tmW, ep, (int)M, N, K, s);
       case EPI_SILU: return launch_tc<EPI_SILU>(tA, *tmW, ep, (int)M, N, K, s);
       case EPI_GLU: return launch_tc<EPI_GLU>(tA, *tmW, ep, (int)M, N, K, s);
@@ -553,6 +567,7 @@ cudaError_t gemm(const ae_model *m, const void *x, int64_t M, int K, const void 
   const float *wf = static_cast<const float *>(w);
   switch (mode) {
     case EPI_F32: return launch_f32<EPI_F32>(xf, wf, ep, (int)M, N, K, s);
+    case EPI_ADD_F32: return launch_f32<EPI_ADD_F32>(xf, wf, ep, (int)M, N, K, s);
     case EPI_BF16: return launch_f32<EPI_BF16>(xf, wf, ep, (int)M, N, K, s);
     case EPI_SILU: return launch_f32<EPI_SILU>(xf, wf, ep, (int)M, N, K, s);
     case EPI_GLU: return launch_f32<EPI_GLU>(xf, wf, ep, (int)M, N, K, s);
