@@ -359,6 +359,23 @@ def oracle_baseline(name: str, budget_s: float = 20.0):
 
 # ------------------------------------------------------------------ arms
 
+def max_over_ranks(value: float, dist, device: str = "cuda") -> float:
+    """The largest value over all ranks (every rank gets it); the value itself
+    for a single process. The multi-GPU timings are reported this way."""
+    if not dist:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(audio_s_per_replica: float, world: int, ms_total: float, steps: int) -> float:
+    """Audio seconds per second of the whole job: every rank runs one replica of
+    the batch per step (weak scaling), timed as the slowest rank."""
+    return audio_s_per_replica * world / (ms_total / steps / 1e3)
+
+
 def run_ours(args, rank, world, dist):
     import torch
     ours = Ours(args.workload)
@@ -373,11 +390,8 @@ def run_ours(args, rank, world, dist):
         torch.cuda.synchronize()
         if dist:
             dist.barrier()
-        ms = ours.timed(args.steps, ours.step)
+        ms = max_over_ranks(ours.timed(args.steps, ours.step), dist)
         if dist:
-            t = torch.tensor([ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
             dist.barrier()
     clocks = clk.summary()
     # per-kernel-class timing over a replica of the timed region (events around every launch)
@@ -405,16 +419,13 @@ def run_ours(args, rank, world, dist):
         ms_e2e = ours.timed(args.steps, e2e)
         h2d, d2h = sizes[0]
     if ms_e2e is not None:
-        if dist:
-            t = torch.tensor([ms_e2e], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
+        ms_e2e = max_over_ranks(ms_e2e, dist)
     if rank != 0:
         return None
     pk = peaks()
     per_step = ms / args.steps
     audio = ours.audio_s * world
-    value = audio / (per_step / 1e3)
+    value = whole_job_value(ours.audio_s, world, ms, args.steps)
     launches = sum(v["launches"] for k, v in prof.items() if k != "dropped")
     dom = prof[ours.dominant]
     if ours.dominant in ("gemm",):
