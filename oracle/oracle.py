@@ -28,6 +28,12 @@ Readings of points the page leaves open (listed again in the design notes):
   float64 here (the page rounds some of them to float32; the difference is
   far below every tolerance).
 
+The e4m3 projections (``e4m3_round`` .. ``fp8_weights``) are the library's
+own low-precision variant, not the page's arithmetic: the page only keeps a
+quantized pack's kernels as an option. They are pinned by torch's
+``float8_e4m3fn`` conversion, the format's special values and invariants of
+the row quantisation.
+
 Parity status: every stage is pinned by the ``-m "not gpu"`` tests (page
 values, closed forms, invariants, brute force). The composition of a full
 layer and of the tower is pinned only by a tiny-size brute-force restatement
@@ -56,7 +62,8 @@ __all__ = [
     "silu", "sigmoid", "softplus", "sinusoids", "relative_keys", "q_scale_of",
     "k_scale_of", "ffn", "local_attention_core", "attention", "glu", "dwconv",
     "light_conv", "conformer_layer", "head", "positions", "encode",
-    "layer_tables",
+    "layer_tables", "e4m3_round", "e4m3_rows", "e4m3_dequant_rows", "input_scale", "quantize_input",
+    "fp8_weights", "FP8_MATRICES",
 ]
 
 
@@ -233,12 +240,88 @@ def rms(x: np.ndarray, w: np.ndarray | None = None) -> np.ndarray:
     return y if w is None else y * np.asarray(w, np.float64)
 
 
-def clip_lin(x: np.ndarray, W: np.ndarray, b=(-np.inf, np.inf, -np.inf, np.inf)) -> np.ndarray:
+def clip_lin(x: np.ndarray, W: np.ndarray, b=(-np.inf, np.inf, -np.inf, np.inf), fp8: bool = False) -> np.ndarray:
     """``ClipLin::apply`` (Gemma4ClippableLinear): clamp the input, x W^T
-    (no bias), clamp the output."""
+    (no bias), clamp the output. With ``fp8`` the clamped input is replaced by
+    its e4m3 value at the input scale (``quantize_input``) and W is expected
+    to hold the dequantised e4m3 rows (``e4m3_dequant_rows``)."""
     lo_in, hi_in, lo_out, hi_out = b
-    y = np.clip(x, lo_in, hi_in) @ np.asarray(W, np.float64).T
+    xc = np.clip(x, lo_in, hi_in)
+    if fp8:
+        xc = quantize_input(xc, input_scale(b))
+    y = xc @ np.asarray(W, np.float64).T
     return np.clip(y, lo_out, hi_out)
+
+
+# ------------------------------------------------------------------ e4m3 projections
+#
+# The low-precision variant of the projections (the page keeps a quantized
+# pack's kernels as an option, AudioTower::load with CMF_EGEMMA2_LOWMEM, but
+# gives no format): OCP 8-bit floating point E4M3, per-row weight scales and
+# an input scale fixed by the ClipLin input clamp. This arithmetic is the
+# library's own definition of its AE_FP8 model, written out here plainly.
+
+E4M3_MAX = 448.0
+
+
+def e4m3_round(x) -> np.ndarray:
+    """Nearest E4M3 value, ties to even, magnitudes beyond 448 saturated to
+    448. E4M3: sign, 4 exponent bits with bias 7, 3 mantissa bits; normal
+    values (1 + m/8) 2^(e-7) for e = 1..15 (the pattern e = 15, m = 7 is NaN,
+    so the largest finite value is 1.75 x 2^8 = 448); subnormals m 2^-9.
+    The grid spacing at |x| in [2^e, 2^(e+1)) is 2^(e-3) for e >= -6 and
+    2^-9 below 2^-6."""
+    x = np.asarray(x, np.float64)
+    a = np.abs(x)
+    _, ex = np.frexp(a)                       # a = f 2^ex, f in [0.5, 1)
+    e = np.maximum(ex - 1, -6)                # binade of a, subnormals share the lowest spacing
+    q = np.ldexp(1.0, e - 3)
+    r = np.minimum(np.round(a / q) * q, E4M3_MAX)   # np.round: half to even
+    return np.copysign(r, x)
+
+
+def e4m3_rows(W) -> tuple[np.ndarray, np.ndarray]:
+    """Per-row quantisation of a weight matrix [out, in]: s_n = max_k
+    |W[n, k]| / 448 (1 for an all-zero row), values e4m3_round(W[n, k] / s_n)
+    in float64. Returns (grid values, s)."""
+    W = np.asarray(W, np.float64)
+    amax = np.max(np.abs(W), axis=1) if W.size else np.zeros(W.shape[0])
+    s = np.where(amax > 0, amax / E4M3_MAX, 1.0)
+    return e4m3_round(W / s[:, None]), s
+
+
+def e4m3_dequant_rows(W) -> np.ndarray:
+    """The matrix the e4m3 model multiplies by: grid values times row scales."""
+    v, s = e4m3_rows(W)
+    return v * s[:, None]
+
+
+def input_scale(b) -> float:
+    """Scale of an e4m3 projection input clamped to [lo_in, hi_in]: 448 over
+    the larger bound (the clamp maps onto the format's finite range)."""
+    return E4M3_MAX / max(abs(float(b[0])), abs(float(b[1])))
+
+
+def quantize_input(x, q: float) -> np.ndarray:
+    """x replaced by e4m3_round(x q) / q."""
+    return e4m3_round(np.asarray(x, np.float64) * q) / q
+
+
+FP8_MATRICES = ("ff1.w1", "ff1.w2", "ff2.w1", "ff2.w2", "q", "k", "v", "lc_start")
+
+
+def fp8_weights(W: dict) -> dict:
+    """The e4m3 model's weights: a copy of W whose FP8_MATRICES are replaced
+    by their dequantised e4m3 rows (the other matrices stay as given)."""
+    out = dict(W)
+    out["layers"] = []
+    for ly in W["layers"]:
+        d = dict(ly)
+        for k in FP8_MATRICES:
+            d[k] = e4m3_dequant_rows(ly[k])
+        out["layers"].append(d)
+    out["fp8"] = True
+    return out
 
 
 def sigmoid(x):
@@ -291,11 +374,11 @@ def layer_tables(ly: dict, shape: dict) -> dict:
             "qd": softplus(ly["pds"])}
 
 
-def ffn(h: np.ndarray, ly: dict, f: str, bounds: dict, rw: float) -> np.ndarray:
+def ffn(h: np.ndarray, ly: dict, f: str, bounds: dict, rw: float, fp8: bool = False) -> np.ndarray:
     """``ffn``: h + rw * rms_post(W2 silu(W1 rms_pre(h))), W1/W2 clippable."""
     a = rms(h, ly[f + ".pre"])
-    u = silu(clip_lin(a, ly[f + ".w1"], bounds[f + ".w1"]))
-    y = clip_lin(u, ly[f + ".w2"], bounds[f + ".w2"])
+    u = silu(clip_lin(a, ly[f + ".w1"], bounds[f + ".w1"], fp8))
+    y = clip_lin(u, ly[f + ".w2"], bounds[f + ".w2"], fp8)
     return h + rw * rms(y, ly[f + ".post"])
 
 
@@ -336,12 +419,12 @@ def local_attention_core(q: np.ndarray, k: np.ndarray, v: np.ndarray, pos: np.nd
 
 
 def attention(h: np.ndarray, pos: np.ndarray, ly: dict, tb: dict, bounds: dict,
-              shape: dict) -> np.ndarray:
+              shape: dict, fp8: bool = False) -> np.ndarray:
     """Attention block: h + rms_post_attn(post(core(q, k, v of rms_pre_attn(h))))."""
     a = rms(h, ly["norm_pre_attn"])
-    q = clip_lin(a, ly["q"], bounds["q"])
-    k = clip_lin(a, ly["k"], bounds["k"])
-    v = clip_lin(a, ly["v"], bounds["v"])
+    q = clip_lin(a, ly["q"], bounds["q"], fp8)
+    k = clip_lin(a, ly["k"], bounds["k"], fp8)
+    v = clip_lin(a, ly["v"], bounds["v"], fp8)
     o = local_attention_core(q, k, v, pos, tb["R"], tb["qd"], shape["heads"], shape["left"],
                              shape["softcap"])
     y = clip_lin(o, ly["post"], bounds["post"])
@@ -369,26 +452,26 @@ def dwconv(x: np.ndarray, w: np.ndarray, pos: np.ndarray) -> np.ndarray:
     return out
 
 
-def light_conv(h: np.ndarray, pos: np.ndarray, ly: dict, bounds: dict) -> np.ndarray:
+def light_conv(h: np.ndarray, pos: np.ndarray, ly: dict, bounds: dict, fp8: bool = False) -> np.ndarray:
     """Light conv block: h + lc_end(silu(rms_conv_norm(dwconv(glu(lc_start(
     rms_lc_pre(h))))))) (no norm on this residual)."""
     a = rms(h, ly["lc_pre"])
-    g = clip_lin(a, ly["lc_start"], bounds["lc_start"])
+    g = clip_lin(a, ly["lc_start"], bounds["lc_start"], fp8)
     c = dwconv(glu(g), ly["lc_dw"], pos)
     c = silu(rms(c, ly["lc_norm"]))
     return h + clip_lin(c, ly["lc_end"], bounds["lc_end"])
 
 
 def conformer_layer(h: np.ndarray, pos: np.ndarray, ly: dict, bounds: dict, shape: dict,
-                    tb: dict | None = None) -> np.ndarray:
+                    tb: dict | None = None, fp8: bool = False) -> np.ndarray:
     """One layer of ``encode_locked``: FFN1, attention, light conv, FFN2,
-    RMS(norm_out)."""
+    RMS(norm_out). ``fp8``: the e4m3 model (ly from ``fp8_weights``)."""
     tb = layer_tables(ly, shape) if tb is None else tb
     rw = shape["residual_weight"]
-    h = ffn(h, ly, "ff1", bounds, rw)
-    h = attention(h, pos, ly, tb, bounds, shape)
-    h = light_conv(h, pos, ly, bounds)
-    h = ffn(h, ly, "ff2", bounds, rw)
+    h = ffn(h, ly, "ff1", bounds, rw, fp8)
+    h = attention(h, pos, ly, tb, bounds, shape, fp8)
+    h = light_conv(h, pos, ly, bounds, fp8)
+    h = ffn(h, ly, "ff2", bounds, rw, fp8)
     return rms(h, ly["norm_out"])
 
 
@@ -425,8 +508,9 @@ def encode(clips: list, weights: dict, trace: bool = False, mels: list | None = 
     pos = positions(lens)
     tr["subsample"] = h.copy()
     tr["layers"] = []
+    fp8 = bool(weights.get("fp8", False))
     for ly, bd in zip(weights["layers"], weights["bounds"]):
-        h = conformer_layer(h, pos, ly, bd, shape)
+        h = conformer_layer(h, pos, ly, bd, shape, fp8=fp8)
         if trace:
             tr["layers"].append(h.copy())
     e = head(h, weights["head"])
