@@ -62,7 +62,7 @@ __all__ = [
     "silu", "sigmoid", "softplus", "sinusoids", "relative_keys", "q_scale_of",
     "k_scale_of", "ffn", "local_attention_core", "attention", "glu", "dwconv",
     "light_conv", "conformer_layer", "head", "positions", "encode",
-    "layer_tables", "e4m3_round", "e4m3_rows", "e4m3_dequant_rows", "input_scale", "quantize_input",
+    "layer_tables", "e4m3_round", "e4m3_decode", "linear_e4m3", "e4m3_rows", "e4m3_dequant_rows", "input_scale", "quantize_input",
     "fp8_weights", "FP8_MATRICES",
 ]
 
@@ -278,6 +278,30 @@ def e4m3_round(x) -> np.ndarray:
     q = np.ldexp(1.0, e - 3)
     r = np.minimum(np.round(a / q) * q, E4M3_MAX)   # np.round: half to even
     return np.copysign(r, x)
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Values of E4M3 bit patterns (uint8): sign bit 7, exponent field e in
+    bits 3-6, mantissa m in bits 0-2; e = 0 gives m 2^-9, otherwise
+    (1 + m/8) 2^(e-7); e = 15 with m = 7 is NaN."""
+    c = np.asarray(codes, np.uint8).astype(np.int64)
+    e, m = (c >> 3) & 15, c & 7
+    v = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.ldexp(1.0, e - 7))
+    v = np.where((e == 15) & (m == 7), np.nan, v)
+    return np.where(c & 128, -v, v)
+
+
+def linear_e4m3(x_codes, w_codes, cs, lo: float, hi: float, silu_q: tuple | None = None) -> np.ndarray:
+    """One e4m3 projection by its definition: acc = x W^T over the decoded
+    codes (float64), times cs per output column, clamped to [lo, hi]; with
+    ``silu_q = (lo2, hi2, q)`` the output is e4m3_round(clamp(silu(v), lo2,
+    hi2) q) instead (grid values)."""
+    acc = e4m3_decode(x_codes) @ e4m3_decode(w_codes).T
+    v = np.clip(acc * np.asarray(cs, np.float64)[None, :], lo, hi)
+    if silu_q is None:
+        return v
+    lo2, hi2, q = silu_q
+    return e4m3_round(np.clip(silu(v), lo2, hi2) * q)
 
 
 def e4m3_rows(W) -> tuple[np.ndarray, np.ndarray]:

@@ -117,3 +117,33 @@ def test_fp8_weights_touch_only_the_e4m3_projections():
             assert not np.array_equal(F["layers"][0][k], v)
         else:
             assert F["layers"][0][k] is v
+
+
+def test_decode_matches_torch_bit_patterns():
+    codes = np.arange(256, dtype=np.uint8)
+    t = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    d = O.e4m3_decode(codes)
+    assert np.array_equal(np.isnan(d), np.isnan(t)) and np.isnan(d).sum() == 2
+    ok = ~np.isnan(t)
+    assert np.array_equal(d[ok], t[ok])
+    # encode . decode is the identity on the grid
+    assert np.array_equal(O.e4m3_round(d[ok]), d[ok])
+
+
+def test_linear_e4m3_against_integer_arithmetic():
+    """Codes scaled by 2^9 are integers: the accumulator is an exact integer
+    sum, checked with Python integers."""
+    r = np.random.default_rng(21)
+    finite = np.array([c for c in range(256) if c & 127 != 127], np.uint8)
+    x = r.choice(finite, size=(4, 256))
+    w = r.choice(finite, size=(3, 256))
+    cs = np.array([1.0, 0.5, 2.0 ** -10])
+    got = O.linear_e4m3(x, w, cs, -np.inf, np.inf)
+    xi = np.rint(O.e4m3_decode(x) * 512).astype(np.int64)
+    wi = np.rint(O.e4m3_decode(w) * 512).astype(np.int64)
+    for i in range(4):
+        for n in range(3):
+            acc = sum(int(a) * int(b) for a, b in zip(xi[i], wi[n]))
+            assert got[i, n] == float(Fraction(acc, 512 * 512) * Fraction(cs[n]))
+    s = O.linear_e4m3(x, w, cs, -8.0, 8.0, silu_q=(-8.0, 8.0, 56.0))
+    assert np.array_equal(O.e4m3_round(s), s) and np.max(np.abs(s)) <= 448.0
