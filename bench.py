@@ -1,7 +1,8 @@
 #!/usr/bin/env python
 """Throughput of the B200 audio-encoder forward.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload tower|ragged|frontend|attention]
+    python bench.py [--gpus N] [--steps K] [--warmup W]
+                    [--workload tower|tower_fp8|ragged|frontend|attention|resample]
     python bench.py --impl reference ...      # the CPU oracle on the same workload (bounded sample)
 
 A step is one ae_encode over one batch (default: 16 clips x 30 s, the
@@ -145,6 +146,9 @@ class Clocks:
 
 def workload_desc(name: str, info: dict) -> dict:
     base = {"tower": "16 clips x 30 s, 12 Conformer layers + embedding head, bf16 weights, f32 accumulation",
+            "tower_fp8": "16 clips x 30 s, 12 Conformer layers + embedding head; FFN W1/W2, q/k/v and lc_start "
+                         "on e4m3 operands (per-row weight scales, input scale from the ClipLin clamp), the other "
+                         "projections bf16; f32 accumulation",
             "ragged": "256 clips of 1-30 s (uniform whole samples), packed, 12 layers + head, bf16",
             "frontend": "log-mel front-end only, 64 clips x 30 s, f32",
             "attention": "local-attention core only, 32 x 8192 tokens, 8 heads x 128, bf16 q/k/v",
@@ -155,29 +159,37 @@ def workload_desc(name: str, info: dict) -> dict:
     return d
 
 
+ENCODE_WORKLOADS = ("tower", "tower_fp8", "ragged")
+
+
+def data_of(name: str) -> str:
+    """The synthetic batch a workload runs on (the e4m3 tower runs the tower's)."""
+    return "tower" if name == "tower_fp8" else name
+
+
 class Ours:
     def __init__(self, name: str):
         import torch
         import log_mel_front_b200 as ae
         self.ae, self.torch, self.name = ae, torch, name
         self.stream = torch.cuda.current_stream()
-        if name in ("tower", "ragged", "frontend"):
-            self.lens = synth.clip_lengths(name)
-            clips = synth.waves(name)
+        if name in ENCODE_WORKLOADS + ("frontend",):
+            self.lens = synth.clip_lengths(data_of(name))
+            clips = synth.waves(data_of(name))
             flat, self.off = synth.pack(clips)
             self.h_wave = torch.from_numpy(flat).pin_memory()
             self.d_wave = self.h_wave.cuda()
             self.frames = sum(ae.ae_num_frames(n) for n in self.lens)
             self.tokens = sum(ae.ae_num_tokens(n) for n in self.lens)
             self.audio_s = sum(min(n, synth.MAX_SAMPLES) for n in self.lens) / synth.SAMPLE_RATE
-        if name in ("tower", "ragged"):
-            self.model = ae.Model(synth.model_weights(name), ae.AE_BF16)
+        if name in ENCODE_WORKLOADS:
+            self.model = ae.Model(synth.model_weights(data_of(name)), ae.AE_FP8 if name == "tower_fp8" else ae.AE_BF16)
             self.ws_bytes = self.model.workspace_size(len(self.lens), self.frames, self.tokens)
             self.d_out = torch.empty((self.tokens, 512), device="cuda")
             self.h_out = torch.empty((self.tokens, 512)).pin_memory()
             self.ws_host_bytes = ae.ae_encode_host_workspace_size(self.model, self.off)
             self.ws = torch.empty(max(self.ws_bytes, self.ws_host_bytes), dtype=torch.uint8, device="cuda")
-            self.dominant = "gemm"
+            self.dominant = "gemm_fp8" if name == "tower_fp8" else "gemm"
         elif name == "frontend":
             self.ws_bytes = ae.ae_workspace_size(None, len(self.lens), self.frames, 0)
             self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
@@ -222,7 +234,7 @@ class Ours:
 
     def step(self):
         ae = self.ae
-        if self.name in ("tower", "ragged"):
+        if self.name in ENCODE_WORKLOADS:
             ae.ae_encode(self.model, self.d_wave, self.off, self.d_out, self.ws, self.ws_bytes, self.stream)
         elif self.name == "frontend":
             ae.ae_logmel(self.d_wave, self.off, self.d_mel, self.ws, self.ws_bytes, self.stream)
@@ -236,7 +248,7 @@ class Ours:
     def step_e2e(self):
         """One step through the host-buffer path; returns (h2d bytes, d2h bytes)."""
         ae, torch = self.ae, self.torch
-        if self.name in ("tower", "ragged"):
+        if self.name in ENCODE_WORKLOADS:
             ae.ae_encode_host(self.model, self.h_wave, self.off, self.h_out, self.ws, self.ws.numel(), self.stream)
             return self.h_wave.numel() * 4, self.h_out.numel() * 4
         if self.name == "frontend":
@@ -301,9 +313,11 @@ class OracleRun:
             self.threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
         except Exception:
             self.threads = os.cpu_count() or 1
-        if name in ("tower", "ragged"):
-            self.W = synth.model_weights(name)
-            self.lens = synth.clip_lengths(name)
+        if name in ENCODE_WORKLOADS:
+            self.W = synth.model_weights(data_of(name))
+            if name == "tower_fp8":
+                self.W = O.fp8_weights(self.W)
+            self.lens = synth.clip_lengths(data_of(name))
             self.next = 0
         elif name == "resample":
             from oracle import resample as RS
@@ -319,10 +333,10 @@ class OracleRun:
     def step(self):
         """One bounded unit of work; returns (seconds, audio seconds, description)."""
         O = self.O
-        if self.name in ("tower", "ragged"):
+        if self.name in ENCODE_WORKLOADS:
             i = self.next % len(self.lens)
             self.next += 1
-            c = synth.waves(self.name, [i])[0]
+            c = synth.waves(data_of(self.name), [i])[0]
             t0 = time.perf_counter()
             O.encode([c], self.W)
             dt = time.perf_counter() - t0
@@ -352,7 +366,7 @@ def oracle_baseline(name: str, budget_s: float = 20.0):
     while n == 0 or t < budget_s:
         dt, au, _ = r.step()
         t, a, n = t + dt, a + au, n + 1
-        if name == "tower" and n >= 16:
+        if data_of(name) == "tower" and n >= 16:
             break
     return a / t, f"{n} unit(s) of the {name} workload through the f64 oracle ({a:.1f} s of audio)", r.threads
 
@@ -405,7 +419,7 @@ def run_ours(args, rank, world, dist):
     # end to end through the host-buffer entry point
     h2d = d2h = 0
     ms_e2e = None
-    if args.workload in ("tower", "ragged"):
+    if args.workload in ENCODE_WORKLOADS:
         ours.e2e_pipelined(2)
         ms_e2e = ours.e2e_pipelined(args.steps)
         h2d, d2h = ours.h_wave.numel() * 4, ours.h_out.numel() * 4
@@ -428,10 +442,16 @@ def run_ours(args, rank, world, dist):
     value = whole_job_value(ours.audio_s, world, ms, args.steps)
     launches = sum(v["launches"] for k, v in prof.items() if k != "dropped")
     dom = prof[ours.dominant]
-    if ours.dominant in ("gemm",):
+    if ours.dominant == "gemm":
         achieved = dom["flops"] / (dom["ms"] / 1e3) / 1e12
         peak = pk["bf16_tflops_sustained"]
         roof = {"bound": "tensor", "unit": "TFLOP/s", "peak_kind": "bf16 sustained (" + pk["source"] + ")"}
+    elif ours.dominant == "gemm_fp8":
+        # e4m3 dense rate = the measured bf16 figure x the nominal ratio 4.5 / 2.25 PFLOP/s
+        achieved = dom["flops"] / (dom["ms"] / 1e3) / 1e12
+        peak = round(2.0 * pk["bf16_tflops_sustained"], 1)
+        roof = {"bound": "tensor", "unit": "TFLOP/s",
+                "peak_kind": "e4m3 = 2 x bf16 sustained (" + pk["source"] + "; nominal ratio 4.5 / 2.25 PFLOP/s)"}
     elif ours.dominant == "resample":
         # the FIR is plain FP32 multiply-add: 148 SMs x 128 FP32 lanes x 2 flop at the max SM clock
         sm_mhz = (clocks.get("sm_max_mhz") or 1965.0)
@@ -445,6 +465,7 @@ def run_ours(args, rank, world, dist):
         roof = {"bound": "hbm", "unit": "GB/s", "peak_kind": "HBM copy (" + pk["source"] + ")"}
     traffic, traffic_src = captured_traffic(ours.dominant)
     roof.update({"kernel": {"gemm": "k_gemm_tc (all projections)", "logmel": "k_logmel",
+                            "gemm_fp8": "k_gemm_tc<e4m3> (FFN W1/W2, q/k/v, lc_start)",
                             "attention": "k_attention_tc",
                             "resample": "k_rs_fir (with its tap table and mixdown)"}[ours.dominant],
                  "achieved": round(achieved, 2), "peak": peak, "frac": round(achieved / peak, 4),
@@ -459,7 +480,8 @@ def run_ours(args, rank, world, dist):
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(per_step, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32" if args.workload in ("frontend", "resample") else "bf16",
+        "vs_baseline": None,
+        "dtype": {"frontend": "f32", "resample": "f32", "tower_fp8": "e4m3+bf16"}.get(args.workload, "bf16"),
         "data": "synthetic",
         "config": workload_desc(args.workload, {
             "clips": len(getattr(ours, "lens", [])) or synth.ATT_SEQS,
@@ -471,6 +493,8 @@ def run_ours(args, rank, world, dist):
             "value": round(audio / (ms_e2e / args.steps / 1e3), 2), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "api": {"tower": "ae_encode_host_async, two streams (copies of one step overlap the kernels of the other)",
+                    "tower_fp8": "ae_encode_host_async, two streams (copies of one step overlap the kernels of the "
+                                 "other)",
                     "ragged": "ae_encode_host_async, two streams (copies of one step overlap the kernels of the other)",
                     "frontend": "ae_logmel + copies", "resample": "ae_resample + copies"}[args.workload]},
         "gpu_launches": int(round(launches / prof_steps * args.steps)),
@@ -513,7 +537,8 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", choices=("tower", "ragged", "frontend", "attention", "resample"), default="tower")
+    ap.add_argument("--workload", choices=("tower", "tower_fp8", "ragged", "frontend", "attention", "resample"),
+                    default="tower")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)

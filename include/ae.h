@@ -63,8 +63,24 @@ typedef enum {
  * products (CUDA-core FMA). AE_BF16: bf16 weights and bf16 operands of
  * every projection on the tcgen05 tensor cores with float32 accumulation;
  * the residual stream, norms, attention and convolution arithmetic stay
- * float32. The front-end is float32 in both. */
-typedef enum { AE_F32 = 0, AE_BF16 = 1 } ae_dtype;
+ * float32. The front-end is float32 in all three.
+ *
+ * AE_FP8: AE_BF16 with 8-bit projections where the model bounds the input.
+ * The page keeps a quantized pack's kernels as an option (egemma2_audio.rs,
+ * AudioTower::load, CMF_EGEMMA2_LOWMEM); here the low-precision format is
+ * OCP e4m3 on the tcgen05 kind::f8f6f4 path. The page gives no such format,
+ * so this arithmetic is this library's, not the page's. FFN W1 and W2, q/k/v and
+ * lc_start: each weight row n is stored as e4m3 codes of
+ * W[n][k] / s_n, s_n = max_k |W[n][k]| / 448 (1 for an all-zero row),
+ * rounded to nearest even from the float32 input in float64 arithmetic.
+ * Each input is stored as e4m3 codes of x * q, q = 448 / max(|lo_in|,
+ * |hi_in|) of the projection's input clamp, rounded to nearest even from
+ * float32. The producing kernel writes them: the row passes for W1,
+ * q/k/v and lc_start, and W1's SiLU epilogue for W2. The accumulator
+ * column n is multiplied by s_n / q before the epilogue. These projections
+ * need finite input bounds (AE_EUNSUPPORTED otherwise). post, lc_end,
+ * in_proj, out_proj, embed and conv1 stay bf16. */
+typedef enum { AE_F32 = 0, AE_BF16 = 1, AE_FP8 = 2 } ae_dtype;
 
 /* Hyper-parameters of the tower (egemma2_audio.rs, AudioTower::load reads
  * them from audio_config). The kernels are compiled for the release shape:
@@ -87,7 +103,9 @@ typedef struct { float lo_in, hi_in, lo_out, hi_out; } ae_clip;
 /* One Conformer layer's weights as host float32 arrays in the checkpoint's
  * layouts: matrices [out][in] row-major; norm weights [hidden];
  * per_dim_scale [head_dim]; lc_dw [hidden][kernel]. For AE_BF16 every
- * matrix is converted to bf16 by round-to-nearest-even at model creation.
+ * matrix is converted to bf16 by round-to-nearest-even at model creation;
+ * for AE_FP8 the e4m3 projections are quantised as described at ae_dtype
+ * and the other matrices converted to bf16.
  * q, k and v must share their input bounds (they read the same normalised
  * activations through one fused projection). */
 typedef struct {
@@ -227,6 +245,31 @@ ae_status ae_local_attention(const void *d_q, const void *d_k, const void *d_v, 
                              void *d_out, int64_t ld_out, void *d_ws, size_t ws_bytes,
                              ae_stream stream);
 
+/* --- one e4m3 projection alone ------------------------------------------------- */
+
+/* Output of ae_linear_e4m3. */
+typedef enum { AE_LIN_BF16 = 0, AE_LIN_SILU_E4M3 = 1 } ae_lin_out;
+
+/* The projection kernel of AE_FP8 models on its own (tcgen05 kind::f8f6f4,
+ * CTA pairs): acc[m][n] = sum_k x[m][k] w[n][k] in float32 over e4m3
+ * operands, then per output column n the factor cs[n] (the weight row's scale
+ * over the input's code scale), then:
+ *   AE_LIN_BF16:      y [M][N] bf16 = clamp(acc cs, lo, hi)
+ *   AE_LIN_SILU_E4M3: y [M][N] e4m3 codes of
+ *                     clamp(silu(clamp(acc cs, lo, hi)), lo2, hi2) * q_out
+ *                     (nearest even, magnitudes beyond 448 saturated)
+ * (the epilogues of q/k/v and FFN W2, and of FFN W1, which writes W2's input).
+ * d_x [M][K] and d_w [N][K]: e4m3 codes (OCP E4M3: sign, 4 exponent bits with
+ * bias 7, 3 mantissa bits; the patterns 0x7F and 0xFF are NaN), row-major,
+ * device memory, 16-byte aligned; d_cs [N] float32, 16-byte aligned; d_y
+ * 32-byte aligned. K a positive multiple of 128 up to 65536, N a positive
+ * multiple of 256 up to 65536, 0 <= M < 2^31. The caller owns every buffer;
+ * nothing is allocated. Arguments are checked before anything is enqueued
+ * (AE_EINVAL); launch errors give AE_ECUDA. Asynchronous on `stream`. */
+ae_status ae_linear_e4m3(const void *d_x, const void *d_w, const float *d_cs, int64_t M, int32_t N, int32_t K,
+                         float lo, float hi, ae_lin_out out, float lo2, float hi2, float q_out, void *d_y,
+                         ae_stream stream);
+
 /* --- log-mel without a caller workspace ---------------------------------------- */
 
 /* ae_logmel for callers that cannot allocate device memory at all: code that
@@ -300,12 +343,13 @@ typedef enum {
   AE_K_LOGMEL = 1,   /* fused log-mel front-end */
   AE_K_CONV0 = 2,    /* stem conv0 + LayerNorm + ReLU */
   AE_K_CONV1 = 3,    /* stem conv1 + LayerNorm + ReLU (implicit GEMM) */
-  AE_K_GEMM = 4,     /* every projection (tcgen05 for AE_BF16) */
+  AE_K_GEMM = 4,     /* the f32 and bf16 projections (tcgen05 for AE_BF16, AE_FP8) */
   AE_K_ATTENTION = 5,
   AE_K_LCONV = 6,    /* depthwise conv + RMS norm + SiLU */
   AE_K_ROWOP = 7,    /* residual / RMS-norm row passes */
   AE_K_RESAMPLE = 8, /* mixdown, resampler taps and FIR */
-  AE_K_COUNT = 9
+  AE_K_GEMM_FP8 = 9, /* the e4m3 projections of AE_FP8 (tcgen05 kind::f8f6f4) */
+  AE_K_COUNT = 10
 } ae_kernel_class;
 
 /* Kernel timing for measurement (the analogue of the page's

@@ -23,7 +23,8 @@ if not os.path.exists(LIB_PATH):
 lib = C.CDLL(LIB_PATH)
 
 AE_OK, AE_EINVAL, AE_EUNSUPPORTED, AE_EWORKSPACE, AE_ECUDA, AE_ENOMEM, AE_EDEVICE = range(7)
-AE_F32, AE_BF16 = 0, 1
+AE_F32, AE_BF16, AE_FP8 = 0, 1, 2
+AE_LIN_BF16, AE_LIN_SILU_E4M3 = 0, 1
 STATUS_NAMES = {0: "AE_OK", 1: "AE_EINVAL", 2: "AE_EUNSUPPORTED", 3: "AE_EWORKSPACE", 4: "AE_ECUDA",
                 5: "AE_ENOMEM", 6: "AE_EDEVICE"}
 
@@ -89,6 +90,8 @@ _sig("ae_logmel_noalloc", _st, _vp, _i64p, _i32, _vp, _vp)
 _sig("ae_resample_len", C.c_int64, C.c_int64, C.c_int32, C.c_int32)
 _sig("ae_resample_workspace_size", _sz, _i64p, _i32, C.c_int32, C.c_int32, _i32)
 _sig("ae_resample", _st, _vp, _i32, C.c_int64, _i64p, _i32, C.c_int32, C.c_int32, _vp, _vp, _sz, _vp)
+_sig("ae_linear_e4m3", _st, _vp, _vp, _vp, C.c_int64, C.c_int32, C.c_int32, C.c_float, C.c_float, _i32, C.c_float,
+     C.c_float, C.c_float, _vp, _vp)
 _sig("ae_profile_enable", _st, _i32)
 _sig("ae_profile_read", _st, C.POINTER(C.c_double), _i64p, C.POINTER(C.c_double), C.POINTER(C.c_double), _i64p)
 
@@ -97,9 +100,10 @@ EXPORTS = ("ae_num_frames", "ae_num_tokens", "ae_model_create", "ae_model_destro
            "ae_logmel", "ae_subsample", "ae_conformer_layer", "ae_encode", "ae_encode_host_workspace_size",
            "ae_encode_host", "ae_encode_host_async", "ae_attention_tables", "ae_local_attention", "ae_last_error", "ae_device_status",
            "ae_version", "ae_profile_enable", "ae_profile_read", "ae_logmel_noalloc", "ae_resample_len",
-           "ae_resample_workspace_size", "ae_resample")
+           "ae_resample_workspace_size", "ae_resample", "ae_linear_e4m3")
 
-KERNEL_CLASSES = ("tables", "logmel", "conv0", "conv1", "gemm", "attention", "lconv", "rowop", "resample")
+KERNEL_CLASSES = ("tables", "logmel", "conv0", "conv1", "gemm", "attention", "lconv", "rowop", "resample",
+                  "gemm_fp8")
 
 
 class AEError(RuntimeError):
@@ -226,6 +230,12 @@ def ae_local_attention(d_q, d_k, d_v, ld_qkv: int, dtype: int, d_R, d_qscale, k_
     _check(lib.ae_local_attention(_ptr(d_q), _ptr(d_k), _ptr(d_v), ld_qkv, dtype, _ptr(d_R), _ptr(d_qscale),
                                   k_scale, softcap, p, len(a) - 1, _ptr(d_out), ld_out, _ptr(d_ws), ws_bytes,
                                   _stream(stream)), "ae_local_attention")
+
+
+def ae_linear_e4m3(d_x, d_w, d_cs, M: int, N: int, K: int, lo: float, hi: float, d_y, out: int = AE_LIN_BF16,
+                   lo2: float = float("-inf"), hi2: float = float("inf"), q_out: float = 1.0, stream=None):
+    _check(lib.ae_linear_e4m3(_ptr(d_x), _ptr(d_w), _ptr(d_cs), M, N, K, lo, hi, out, lo2, hi2, q_out, _ptr(d_y),
+                              _stream(stream)), "ae_linear_e4m3")
 
 
 def ae_device_status() -> int:

@@ -40,6 +40,7 @@ enum EpiMode : int {
   EPI_SILU = 2,       // v = clamp2(silu(clamp(acc))) -> act
   EPI_GLU = 3,        // columns (2c, 2c+1) -> clamp, a * sigmoid(b) -> act column c
   EPI_ADD_F32 = 4,    // out += clamp(acc): a float residual update, one add per element
+  EPI_SILU_Q8 = 5,    // v = clamp2(silu(clamp(acc))) -> e4m3 code of v * q8 (the next projection's operand)
 };
 
 struct EpiArgs {
@@ -47,9 +48,12 @@ struct EpiArgs {
   int64_t ld;         // output row stride in elements
   const float *bias;  // [N] or null
   float lo, hi;       // first clamp
-  float lo2, hi2;     // clamp after the activation (EPI_SILU)
+  float lo2, hi2;     // clamp after the activation (EPI_SILU, EPI_SILU_Q8)
+  int clamp2;         // 0 when that clamp cannot bind (silu_clamp_binds)
   int seg_w;          // if > 0: columns [s*seg_w, (s+1)*seg_w) use seg_lo/hi[s] as the first clamp
   float seg_lo[3], seg_hi[3];
+  const float *cs;    // e4m3 projections: [N] factor of each accumulator column (weight row scale / q8 of x)
+  float q8;           // EPI_SILU_Q8: scale of the e4m3 output codes
 };
 
 // Device copy of one layer.
@@ -66,6 +70,11 @@ struct LayerDev {
   ae_clip c_ff1_w1, c_ff1_w2, c_ff2_w1, c_ff2_w2, c_q, c_k, c_v, c_post, c_lc_start, c_lc_end;
   // tensor maps of the weight operands (bf16 only)
   CUtensorMap tm_ff1_w1, tm_ff1_w2, tm_ff2_w1, tm_ff2_w2, tm_qkv, tm_post, tm_lc_start, tm_lc_end;
+  // AE_FP8: FFN W1/W2, q/k/v and lc_start hold e4m3 codes (the maps above are
+  // 8-bit maps then); cs_* are their accumulator column factors, q8_* the
+  // scales of their e4m3 inputs (448 over the input clamp's larger bound)
+  float *cs_ff1_w1, *cs_ff1_w2, *cs_ff2_w1, *cs_ff2_w2, *cs_qkv, *cs_lc_start;
+  float q8_ff1_w1, q8_ff1_w2, q8_ff2_w1, q8_ff2_w2, q8_qkv, q8_lc_start;
 };
 
 }  // namespace ae
@@ -144,16 +153,21 @@ cudaError_t launch_conv1(const ae_model *m, const void *y0, int64_t stem_rows, v
 // the weight's tensor map (or null to build one).
 cudaError_t gemm(const ae_model *m, const void *x, int64_t M, int K, const void *w, const CUtensorMap *tmW,
                  int N, int mode, const EpiArgs &ep, cudaStream_t s);
+// The same on e4m3 operands (tcgen05 kind::f8f6f4): x [M][K] codes, the
+// weight's 8-bit tensor map; ep.cs scales the accumulator columns.
+cudaError_t gemm_e4m3(const void *x, int64_t M, int K, const CUtensorMap &tmW, int N, int mode, const EpiArgs &ep,
+                      cudaStream_t s);
 
 // Row update of the residual stream (one warp per row of `width` floats):
 //   if y:      h += s * (y_norm ? rms(y) * wy : y)   (y in the model's act type)
 //   if w_out:  h = rms(h) * w_out
 //   write h back if anything changed it
-//   if a_out:  a = clamp(rms(h) * w_next, lo, hi)  (act type of the model)
+//   if a_out:  a = clamp(rms(h) * w_next, lo, hi)  (act type of the model;
+//              e4m3 codes of a * a_q8 when a_q8 > 0)
 struct RowArgs {
   float *h; const void *y; const float *wy; float s; int y_norm;
   const float *w_out;
-  void *a_out; const float *w_next; int a_rms; float lo, hi;
+  void *a_out; const float *w_next; int a_rms; float lo, hi; float a_q8;
   int width; int64_t rows;
 };
 cudaError_t launch_rowop(const ae_model *m, const RowArgs &r, cudaStream_t s);
@@ -170,6 +184,8 @@ cudaError_t launch_attention(bool is_bf16, const void *q, const void *k, const v
 // Tensor-map encoding (driver entry point looked up at run time).
 bool make_tmap_2d_bf16(CUtensorMap *tm, const void *base, uint64_t inner, uint64_t outer,
                        uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
+bool make_tmap_2d_u8(CUtensorMap *tm, const void *base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                     uint32_t box_inner, uint32_t box_outer);
 bool make_tmap_stem_y0(CUtensorMap *tm, const void *y0, int64_t stem_rows);
 
 // Launch on stream s; the arguments are converted to the kernel's parameter types.

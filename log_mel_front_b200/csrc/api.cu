@@ -68,16 +68,27 @@ static cudaError_t timed(int cls, double flops, double bytes, cudaStream_t s, F 
   return e;
 }
 
-static size_t act_bytes(const ae_model *m) { return m->dtype == AE_BF16 ? 2 : 4; }
+static size_t act_bytes(const ae_model *m) { return m->dtype == AE_F32 ? 4 : 2; }
 
 // A projection with its algorithmic flops (2 M N K) and bytes (x, W, y once).
 static cudaError_t gemm_t(const ae_model *m, const void *x, int64_t M, int K, const void *w, const CUtensorMap *tmW,
                           int N, int mode, const EpiArgs &ep, cudaStream_t s) {
   const double a = (double)act_bytes(m);
   const double out_cols = mode == EPI_GLU ? N / 2 : N;
-  const double out_b = (mode == EPI_F32 || mode == EPI_ADD_F32) ? 4.0 : a;
+  // EPI_ADD_F32 reads and writes the float32 residual
+  const double out_b = mode == EPI_ADD_F32 ? 8.0 : mode == EPI_F32 ? 4.0 : a;
   const double bytes = a * ((double)M * K + (double)N * K) + out_b * (double)M * out_cols;
   return timed(AE_K_GEMM, 2.0 * (double)M * N * K, bytes, s, [&] { return gemm(m, x, M, K, w, tmW, N, mode, ep, s); });
+}
+
+// An e4m3 projection: 1-byte x and W, y in bf16 (or e4m3 codes for EPI_SILU_Q8).
+static cudaError_t gemm8_t(const void *x, int64_t M, int K, const CUtensorMap &tmW, int N, int mode,
+                           const EpiArgs &ep, cudaStream_t s) {
+  const double out_cols = mode == EPI_GLU ? N / 2 : N;
+  const double out_b = mode == EPI_SILU_Q8 ? 1.0 : 2.0;
+  const double bytes = (double)M * K + (double)N * K + out_b * (double)M * out_cols;
+  return timed(AE_K_GEMM_FP8, 2.0 * (double)M * N * K, bytes, s,
+               [&] { return gemm_e4m3(x, M, K, tmW, N, mode, ep, s); });
 }
 
 static cudaError_t tables_t(const ClipTables &T, void *ws, const WsLayout &L, ClipTablesDev *td, bool pos,
@@ -122,7 +133,7 @@ static cudaError_t rowop_t(const ae_model *m, const RowArgs &r, cudaStream_t s) 
   const bool changed = r.y || r.w_out;
   double per_row = 4.0 * W * (1.0 + (changed ? 1.0 : 0.0));  // h read, written back if changed
   if (r.y) per_row += W * (double)act_bytes(m);
-  if (r.a_out) per_row += W * (double)act_bytes(m);
+  if (r.a_out) per_row += W * (r.a_q8 > 0.f ? 1.0 : (double)act_bytes(m));
   return timed(AE_K_ROWOP, 0.0, per_row * (double)r.rows, s, [&] { return launch_rowop(m, r, s); });
 }
 
@@ -182,7 +193,7 @@ WsLayout ws_layout(const ae_model *m, int64_t n_clips, int64_t frames, int64_t t
     L.total = off;
     return L;
   }
-  const size_t act = m->dtype == AE_BF16 ? 2 : 4;
+  const size_t act = m->dtype == AE_F32 ? 4 : 2;
   const int64_t H = m->cfg.hidden;
   L.h = off;
   off += al256((size_t)tokens * H * 4);
@@ -245,6 +256,29 @@ static uint16_t f2bf(float f) {
   return (uint16_t)(u >> 16);
 }
 
+// OCP e4m3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; largest
+// finite 448, subnormals k 2^-9) code of t, rounded to nearest even, with
+// magnitudes beyond 448 saturated to 448.
+static uint8_t e4m3_code(double t) {
+  const uint8_t sign = std::signbit(t) ? 0x80 : 0x00;
+  const double a = std::fabs(t);
+  if (!(a < 448.0)) return sign | 0x7E;  // also NaN: never produced from finite weights
+  if (a < 0.015625) {                    // below 2^-6: subnormal grid of 2^-9 (k = 8 is the smallest normal)
+    return sign | (uint8_t)std::nearbyint(std::ldexp(a, 9));
+  }
+  int ex;
+  std::frexp(a, &ex);  // a = f 2^ex, f in [0.5, 1)
+  const int e = ex - 1;  // a in [2^e, 2^(e+1))
+  int k = (int)std::nearbyint(std::ldexp(a, 3 - e));  // 8 .. 16 steps of 2^(e-3)
+  int be = e + 7;
+  if (k == 16) {
+    k = 8;
+    ++be;
+  }
+  if (be > 15 || (be == 15 && k > 14)) return sign | 0x7E;
+  return sign | (uint8_t)((be << 3) | (k - 8));
+}
+
 struct Uploader {
   ae_model *m;
   bool ok = true;
@@ -272,7 +306,35 @@ struct Uploader {
     return d;
   }
   void *mat(const float *h, size_t n) { return mat(std::vector<float>(h, h + n)); }
+  // e4m3 rows: row n as codes of W[n][k] / s_n, s_n = max_k |W[n][k]| / 448;
+  // *cs gets s_n / q8 per row (the accumulator column factor)
+  void *mat_e4m3(const std::vector<float> &h, size_t rows, size_t cols, float q8, float **cs) {
+    std::vector<uint8_t> codes(rows * cols);
+    std::vector<float> f(rows);
+    for (size_t r = 0; r < rows; ++r) {
+      const float *w = h.data() + r * cols;
+      double amax = 0.0;
+      for (size_t k = 0; k < cols; ++k) amax = std::max(amax, std::fabs((double)w[k]));
+      const double sn = amax > 0.0 ? amax / 448.0 : 1.0;
+      for (size_t k = 0; k < cols; ++k) codes[r * cols + k] = e4m3_code((double)w[k] / sn);
+      f[r] = (float)(sn / (double)q8);
+    }
+    *cs = f32(f.data(), f.size());
+    uint8_t *d = alloc<uint8_t>(codes.size());
+    if (d && cudaMemcpy(d, codes.data(), codes.size(), cudaMemcpyHostToDevice) != cudaSuccess) ok = false;
+    return d;
+  }
+  void *mat_e4m3(const float *h, size_t rows, size_t cols, float q8, float **cs) {
+    return mat_e4m3(std::vector<float>(h, h + rows * cols), rows, cols, q8, cs);
+  }
 };
+
+// Scale of an e4m3 input clamped to [lo, hi]: 448 over the larger bound.
+static float q8_of(const ae_clip &c) { return (float)(448.0 / std::max(std::fabs((double)c.lo_in), std::fabs((double)c.hi_in))); }
+static bool q8_ok(const ae_clip &c) {
+  const double b = std::max(std::fabs((double)c.lo_in), std::fabs((double)c.hi_in));
+  return std::isfinite(b) && b > 0.0;
+}
 
 static bool bad_clip(const ae_clip &c) {
   return std::isnan(c.lo_in) || std::isnan(c.hi_in) || std::isnan(c.lo_out) || std::isnan(c.hi_out) ||
@@ -297,7 +359,16 @@ static EpiArgs ep_of(void *out, int64_t ld, float lo, float hi) {
   e.hi = hi;
   e.lo2 = -INFINITY;
   e.hi2 = INFINITY;
+  e.clamp2 = 1;
   return e;
+}
+
+// Whether clamp(silu(c), lo2, hi2) can differ from silu(c) for c in [lo, hi]:
+// silu(c) = c sigmoid(c) is at least -0.2785 everywhere (its minimum, at
+// c = -1.2785) and below max(c, 0), so bounds of at most -0.5 and at least
+// max(hi, 0) cannot bind (the margin covers the kernels' approximations).
+static int silu_clamp_binds(float hi, float lo2, float hi2) {
+  return !(lo2 <= -0.5f && hi2 >= std::max(hi, 0.0f));
 }
 
 static RowArgs row_of(float *h, int width, int64_t rows) {
@@ -326,10 +397,11 @@ static cudaError_t run_layer(const ae_model *m, int li, const Bufs &b, int64_t T
   const LayerDev &L = m->layers[li];
   const int H = m->cfg.hidden, F = m->cfg.ffn;
   const float rw = m->cfg.residual_weight;
-  const size_t act = m->dtype == AE_BF16 ? 2 : 4;
-  const bool tc = m->dtype == AE_BF16;
+  const size_t act = act_bytes(m);
+  const bool tc = m->dtype != AE_F32;
+  const bool f8 = m->dtype == AE_FP8;  // FFN W1/W2, q/k/v and lc_start on e4m3 operands
   // the projections whose outputs feed a row pass write them in the act type
-  // (bf16 for the tensor-core model): the row pass is bound by its bytes
+  // (bf16 for the tensor-core models): the row pass is bound by its bytes
   const int y_mode = tc ? EPI_BF16 : EPI_F32;
   if (!a_ready) {
     RowArgs r = row_of(b.h, H, T);
@@ -337,22 +409,34 @@ static cudaError_t run_layer(const ae_model *m, int li, const Bufs &b, int64_t T
     r.w_next = L.ff1_pre;
     r.lo = L.c_ff1_w1.lo_in;
     r.hi = L.c_ff1_w1.hi_in;
+    r.a_q8 = f8 ? L.q8_ff1_w1 : 0.f;
     AE_TRY(rowop_t(m, r, s));
   }
   auto ffn = [&](void *w1, const CUtensorMap *t1, const ae_clip &c1, void *w2, const CUtensorMap *t2,
-                 const ae_clip &c2) -> cudaError_t {
+                 const ae_clip &c2, const float *cs1, const float *cs2, float q8_2) -> cudaError_t {
     EpiArgs e1 = ep_of(b.big, F, c1.lo_out, c1.hi_out);
     e1.lo2 = c2.lo_in;
     e1.hi2 = c2.hi_in;
-    AE_TRY(gemm_t(m,b.a, T, H, w1, tc ? t1 : nullptr, F, EPI_SILU, e1, s));
-    return gemm_t(m, b.big, T, F, w2, tc ? t2 : nullptr, H, y_mode, ep_of(b.y, H, c2.lo_out, c2.hi_out), s);
+    e1.clamp2 = silu_clamp_binds(c1.hi_out, c2.lo_in, c2.hi_in);
+    EpiArgs e2 = ep_of(b.y, H, c2.lo_out, c2.hi_out);
+    if (f8) {
+      e1.cs = cs1;
+      e1.q8 = q8_2;
+      e2.cs = cs2;
+      AE_TRY(gemm8_t(b.a, T, H, *t1, F, EPI_SILU_Q8, e1, s));
+      return gemm8_t(b.big, T, F, *t2, H, EPI_BF16, e2, s);
+    }
+    AE_TRY(gemm_t(m, b.a, T, H, w1, tc ? t1 : nullptr, F, EPI_SILU, e1, s));
+    return gemm_t(m, b.big, T, F, w2, tc ? t2 : nullptr, H, y_mode, e2, s);
   };
   // ---- FFN1
-  AE_TRY(ffn(L.ff1_w1, &L.tm_ff1_w1, L.c_ff1_w1, L.ff1_w2, &L.tm_ff1_w2, L.c_ff1_w2));
+  AE_TRY(ffn(L.ff1_w1, &L.tm_ff1_w1, L.c_ff1_w1, L.ff1_w2, &L.tm_ff1_w2, L.c_ff1_w2, L.cs_ff1_w1, L.cs_ff1_w2,
+             L.q8_ff1_w2));
   {
     RowArgs r = row_of(b.h, H, T);
     r.y = b.y; r.wy = L.ff1_post; r.s = rw; r.y_norm = 1;
     r.a_out = b.a; r.w_next = L.norm_pre_attn; r.lo = L.c_q.lo_in; r.hi = L.c_q.hi_in;
+    r.a_q8 = f8 ? L.q8_qkv : 0.f;
     AE_TRY(rowop_t(m, r, s));
   }
   // ---- attention: fused q/k/v projection, core, post
@@ -362,7 +446,12 @@ static cudaError_t run_layer(const ae_model *m, int li, const Bufs &b, int64_t T
     e.seg_lo[0] = L.c_q.lo_out; e.seg_hi[0] = L.c_q.hi_out;
     e.seg_lo[1] = L.c_k.lo_out; e.seg_hi[1] = L.c_k.hi_out;
     e.seg_lo[2] = L.c_v.lo_out; e.seg_hi[2] = L.c_v.hi_out;
-    AE_TRY(gemm_t(m,b.a, T, H, L.qkv, tc ? &L.tm_qkv : nullptr, 3 * H, EPI_BF16, e, s));
+    if (f8) {
+      e.cs = L.cs_qkv;
+      AE_TRY(gemm8_t(b.a, T, H, L.tm_qkv, 3 * H, EPI_BF16, e, s));
+    } else {
+      AE_TRY(gemm_t(m, b.a, T, H, L.qkv, tc ? &L.tm_qkv : nullptr, 3 * H, EPI_BF16, e, s));
+    }
     const uint8_t *qkv = static_cast<const uint8_t *>(b.big);
     AE_TRY(timed(AE_K_ATTENTION, 0.0, (double)T * 4 * H * act, s, [&] {
       return launch_attention(tc, qkv, qkv + act * H, qkv + 2 * act * H, 3 * H, L.R, L.qscale, m->k_scale,
@@ -373,12 +462,18 @@ static cudaError_t run_layer(const ae_model *m, int li, const Bufs &b, int64_t T
     RowArgs r = row_of(b.h, H, T);
     r.y = b.y; r.wy = L.norm_post_attn; r.s = 1.0f; r.y_norm = 1;
     r.a_out = b.a; r.w_next = L.lc_pre; r.lo = L.c_lc_start.lo_in; r.hi = L.c_lc_start.hi_in;
+    r.a_q8 = f8 ? L.q8_lc_start : 0.f;
     AE_TRY(rowop_t(m, r, s));
   }
   // ---- light conv
   {
-    AE_TRY(gemm_t(m,b.a, T, H, L.lc_start, tc ? &L.tm_lc_start : nullptr, 2 * H, EPI_GLU,
-                ep_of(b.big, H, L.c_lc_start.lo_out, L.c_lc_start.hi_out), s));
+    EpiArgs e = ep_of(b.big, H, L.c_lc_start.lo_out, L.c_lc_start.hi_out);
+    if (f8) {
+      e.cs = L.cs_lc_start;
+      AE_TRY(gemm8_t(b.a, T, H, L.tm_lc_start, 2 * H, EPI_GLU, e, s));
+    } else {
+      AE_TRY(gemm_t(m, b.a, T, H, L.lc_start, tc ? &L.tm_lc_start : nullptr, 2 * H, EPI_GLU, e, s));
+    }
     AE_TRY(timed(AE_K_LCONV, 0.0, (double)T * 2 * H * act, s, [&] {
       return launch_lconv(m, b.big, L.lc_dw, L.lc_norm, L.c_lc_end.lo_in, L.c_lc_end.hi_in, b.o, b.pos, T, s);
     }));
@@ -388,10 +483,12 @@ static cudaError_t run_layer(const ae_model *m, int li, const Bufs &b, int64_t T
                   ep_of(b.h, H, L.c_lc_end.lo_out, L.c_lc_end.hi_out), s));
     RowArgs r = row_of(b.h, H, T);
     r.a_out = b.a; r.w_next = L.ff2_pre; r.lo = L.c_ff2_w1.lo_in; r.hi = L.c_ff2_w1.hi_in;
+    r.a_q8 = f8 ? L.q8_ff2_w1 : 0.f;
     AE_TRY(rowop_t(m, r, s));
   }
   // ---- FFN2, norm_out, and the next consumer's input
-  AE_TRY(ffn(L.ff2_w1, &L.tm_ff2_w1, L.c_ff2_w1, L.ff2_w2, &L.tm_ff2_w2, L.c_ff2_w2));
+  AE_TRY(ffn(L.ff2_w1, &L.tm_ff2_w1, L.c_ff2_w1, L.ff2_w2, &L.tm_ff2_w2, L.c_ff2_w2, L.cs_ff2_w1, L.cs_ff2_w2,
+             L.q8_ff2_w2));
   {
     RowArgs r = row_of(b.h, H, T);
     r.y = b.y; r.wy = L.ff2_post; r.s = rw; r.y_norm = 1;
@@ -399,6 +496,7 @@ static cudaError_t run_layer(const ae_model *m, int li, const Bufs &b, int64_t T
     if (next == kNextLayer) {
       const LayerDev &N = m->layers[li + 1];
       r.a_out = b.a; r.w_next = N.ff1_pre; r.lo = N.c_ff1_w1.lo_in; r.hi = N.c_ff1_w1.hi_in;
+      r.a_q8 = f8 ? N.q8_ff1_w1 : 0.f;
     } else if (next == kNextPlain) {
       r.a_out = b.a; r.a_rms = 0;
     }
@@ -410,7 +508,7 @@ static cudaError_t run_layer(const ae_model *m, int li, const Bufs &b, int64_t T
 // Head: out_proj + bias, weightless RMS norm, embed. b.a holds h in the operand type.
 static cudaError_t run_head(const ae_model *m, const Bufs &b, int64_t T, float *out, cudaStream_t s) {
   const int H = m->cfg.hidden, OD = m->cfg.out_dim, ED = m->cfg.embed_dim;
-  const bool tc = m->dtype == AE_BF16;
+  const bool tc = m->dtype != AE_F32;
   EpiArgs e = ep_of(b.y, OD, -INFINITY, INFINITY);
   e.bias = m->out_bias;
   AE_TRY(gemm_t(m,b.a, T, H, m->out_proj, tc ? &m->tm_out_proj : nullptr, OD, EPI_F32, e, s));
@@ -469,7 +567,7 @@ static ae_status encode_one(const ae_model *m, const float *d_wave, const ClipTa
   if ((e = conv0_t(m, mel, w + L.y0, td, T, s)) != cudaSuccess) return cuda_fail(e, "conv0");
   if ((e = conv1_t(m, w + L.y0, w + L.xs, td, T, s)) != cudaSuccess)
     return cuda_fail(e, "conv1");
-  if ((e = gemm_t(m, w + L.xs, T.total_tokens, kHidden, m->in_proj, m->dtype == AE_BF16 ? &m->tm_in_proj : nullptr,
+  if ((e = gemm_t(m, w + L.xs, T.total_tokens, kHidden, m->in_proj, m->dtype != AE_F32 ? &m->tm_in_proj : nullptr,
                 m->cfg.hidden, EPI_F32, ep_of(b.h, m->cfg.hidden, -INFINITY, INFINITY), s)) != cudaSuccess)
     return cuda_fail(e, "in_proj");
   const int nl = m->cfg.n_layers;
@@ -634,7 +732,7 @@ ae_status ae_model_create(const ae_config *cfg, const ae_host_weights *w, ae_dty
   if (c.n_layers < 0 || c.n_layers > 4096) return fail(AE_EINVAL, "n_layers out of range");
   if (!(c.softcap > 0.f) || !std::isfinite(c.softcap) || !std::isfinite(c.residual_weight))
     return fail(AE_EINVAL, "softcap must be positive and finite, residual_weight finite");
-  if (dtype != AE_F32 && dtype != AE_BF16) return fail(AE_EINVAL, "dtype");
+  if (dtype != AE_F32 && dtype != AE_BF16 && dtype != AE_FP8) return fail(AE_EINVAL, "dtype");
   if (!w->conv0 || !w->ln0 || !w->conv1 || !w->ln1 || !w->in_proj || !w->out_proj || !w->out_bias || !w->embed ||
       (c.n_layers > 0 && !w->layers))
     return fail(AE_EINVAL, "a stem or head weight pointer is null");
@@ -652,6 +750,10 @@ ae_status ae_model_create(const ae_config *cfg, const ae_host_weights *w, ae_dty
     if (l.clip_q.lo_in != l.clip_k.lo_in || l.clip_q.lo_in != l.clip_v.lo_in || l.clip_q.hi_in != l.clip_k.hi_in ||
         l.clip_q.hi_in != l.clip_v.hi_in)
       return fail(AE_EUNSUPPORTED, "q, k and v input bounds differ in layer " + std::to_string(i));
+    if (dtype == AE_FP8 && !(q8_ok(l.clip_ff1_w1) && q8_ok(l.clip_ff1_w2) && q8_ok(l.clip_ff2_w1) &&
+                             q8_ok(l.clip_ff2_w2) && q8_ok(l.clip_q) && q8_ok(l.clip_lc_start)))
+      return fail(AE_EUNSUPPORTED, "AE_FP8 needs finite, nonzero input bounds on FFN W1/W2, q/k/v and lc_start "
+                                   "(layer " + std::to_string(i) + ")");
   }
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return fail(AE_ECUDA, "no CUDA device");
@@ -735,16 +837,30 @@ ae_status ae_model_create(const ae_config *cfg, const ae_host_weights *w, ae_dty
     m->k_scale = ks;
     L.R = up.f32(R.data(), R.size());
     L.qscale = up.f32(qs.data(), qs.size());
-    L.ff1_w1 = up.mat(l.ff1_w1, (size_t)c.ffn * H);
-    L.ff1_w2 = up.mat(l.ff1_w2, (size_t)H * c.ffn);
-    L.ff2_w1 = up.mat(l.ff2_w1, (size_t)c.ffn * H);
-    L.ff2_w2 = up.mat(l.ff2_w2, (size_t)H * c.ffn);
+    const bool f8 = dtype == AE_FP8;
+    if (f8) {
+      L.q8_ff1_w1 = q8_of(l.clip_ff1_w1);
+      L.q8_ff1_w2 = q8_of(l.clip_ff1_w2);
+      L.q8_ff2_w1 = q8_of(l.clip_ff2_w1);
+      L.q8_ff2_w2 = q8_of(l.clip_ff2_w2);
+      L.q8_qkv = q8_of(l.clip_q);
+      L.q8_lc_start = q8_of(l.clip_lc_start);
+      L.ff1_w1 = up.mat_e4m3(l.ff1_w1, c.ffn, H, L.q8_ff1_w1, &L.cs_ff1_w1);
+      L.ff1_w2 = up.mat_e4m3(l.ff1_w2, H, c.ffn, L.q8_ff1_w2, &L.cs_ff1_w2);
+      L.ff2_w1 = up.mat_e4m3(l.ff2_w1, c.ffn, H, L.q8_ff2_w1, &L.cs_ff2_w1);
+      L.ff2_w2 = up.mat_e4m3(l.ff2_w2, H, c.ffn, L.q8_ff2_w2, &L.cs_ff2_w2);
+    } else {
+      L.ff1_w1 = up.mat(l.ff1_w1, (size_t)c.ffn * H);
+      L.ff1_w2 = up.mat(l.ff1_w2, (size_t)H * c.ffn);
+      L.ff2_w1 = up.mat(l.ff2_w1, (size_t)c.ffn * H);
+      L.ff2_w2 = up.mat(l.ff2_w2, (size_t)H * c.ffn);
+    }
     {
       std::vector<float> qkv((size_t)3 * H * H);
       std::memcpy(qkv.data(), l.q, (size_t)H * H * 4);
       std::memcpy(qkv.data() + (size_t)H * H, l.k, (size_t)H * H * 4);
       std::memcpy(qkv.data() + (size_t)2 * H * H, l.v, (size_t)H * H * 4);
-      L.qkv = up.mat(qkv);
+      L.qkv = f8 ? up.mat_e4m3(qkv, 3 * H, H, L.q8_qkv, &L.cs_qkv) : up.mat(qkv);
     }
     L.post = up.mat(l.post, (size_t)H * H);
     L.lc_end = up.mat(l.lc_end, (size_t)H * H);
@@ -754,7 +870,7 @@ ae_status ae_model_create(const ae_config *cfg, const ae_host_weights *w, ae_dty
         std::memcpy(ls.data() + (size_t)(2 * r) * H, l.lc_start + (size_t)r * H, (size_t)H * 4);
         std::memcpy(ls.data() + (size_t)(2 * r + 1) * H, l.lc_start + (size_t)(H + r) * H, (size_t)H * 4);
       }
-      L.lc_start = up.mat(ls);
+      L.lc_start = f8 ? up.mat_e4m3(ls, 2 * H, H, L.q8_lc_start, &L.cs_lc_start) : up.mat(ls);
     }
     L.c_ff1_w1 = l.clip_ff1_w1; L.c_ff1_w2 = l.clip_ff1_w2; L.c_ff2_w1 = l.clip_ff2_w1; L.c_ff2_w2 = l.clip_ff2_w2;
     L.c_q = l.clip_q; L.c_k = l.clip_k; L.c_v = l.clip_v; L.c_post = l.clip_post;
@@ -766,12 +882,23 @@ ae_status ae_model_create(const ae_config *cfg, const ae_host_weights *w, ae_dty
     ae_model_destroy(m);
     return fail(AE_ENOMEM, "device allocation or copy failed while uploading the weights");
   }
-  if (dtype == AE_BF16) {
+  if (dtype != AE_F32) {
     bool ok = make_tmap_2d_bf16(&m->tm_conv1, m->conv1, 9 * kC0, kC1, 9 * kC0 * 2, 64, kC1) &&
               make_tmap_2d_bf16(&m->tm_in_proj, m->in_proj, kHidden, H, kHidden * 2, 64, 128) &&
               make_tmap_2d_bf16(&m->tm_out_proj, m->out_proj, H, c.out_dim, H * 2, 64, 128) &&
               make_tmap_2d_bf16(&m->tm_embed, m->embed, c.out_dim, c.embed_dim, c.out_dim * 2, 64, 128);
     for (auto &L : m->layers) {
+      if (dtype == AE_FP8) {  // 8-bit maps: one 128-byte row segment = 128 codes
+        ok = ok && make_tmap_2d_u8(&L.tm_ff1_w1, L.ff1_w1, H, c.ffn, H, 128, 128) &&
+             make_tmap_2d_u8(&L.tm_ff1_w2, L.ff1_w2, c.ffn, H, (uint64_t)c.ffn, 128, 128) &&
+             make_tmap_2d_u8(&L.tm_ff2_w1, L.ff2_w1, H, c.ffn, H, 128, 128) &&
+             make_tmap_2d_u8(&L.tm_ff2_w2, L.ff2_w2, c.ffn, H, (uint64_t)c.ffn, 128, 128) &&
+             make_tmap_2d_u8(&L.tm_qkv, L.qkv, H, 3 * H, H, 128, 128) &&
+             make_tmap_2d_bf16(&L.tm_post, L.post, H, H, H * 2, 64, 128) &&
+             make_tmap_2d_u8(&L.tm_lc_start, L.lc_start, H, 2 * H, H, 128, 128) &&
+             make_tmap_2d_bf16(&L.tm_lc_end, L.lc_end, H, H, H * 2, 64, 128);
+        continue;
+      }
       ok = ok && make_tmap_2d_bf16(&L.tm_ff1_w1, L.ff1_w1, H, c.ffn, H * 2, 64, 128) &&
            make_tmap_2d_bf16(&L.tm_ff1_w2, L.ff1_w2, c.ffn, H, (uint64_t)c.ffn * 2, 64, 128) &&
            make_tmap_2d_bf16(&L.tm_ff2_w1, L.ff2_w1, H, c.ffn, H * 2, 64, 128) &&
@@ -833,7 +960,7 @@ ae_status ae_subsample(const ae_model *m, const float *d_mel, const int64_t *h_f
   if ((e = conv0_t(m, d_mel, w + L.y0, td, T, s)) != cudaSuccess) return cuda_fail(e, "conv0");
   if ((e = conv1_t(m, w + L.y0, w + L.xs, td, T, s)) != cudaSuccess)
     return cuda_fail(e, "conv1");
-  if ((e = gemm_t(m, w + L.xs, T.total_tokens, kHidden, m->in_proj, m->dtype == AE_BF16 ? &m->tm_in_proj : nullptr,
+  if ((e = gemm_t(m, w + L.xs, T.total_tokens, kHidden, m->in_proj, m->dtype != AE_F32 ? &m->tm_in_proj : nullptr,
                 m->cfg.hidden, EPI_F32, ep_of(d_h, m->cfg.hidden, -INFINITY, INFINITY), s)) != cudaSuccess)
     return cuda_fail(e, "in_proj");
   return AE_OK;
@@ -955,6 +1082,38 @@ ae_status ae_local_attention(const void *d_q, const void *d_k, const void *d_v, 
                                  T.total_tokens, d_out, ld_out, -INFINITY, INFINITY, s);
        })) != cudaSuccess)
     return cuda_fail(e, "attention");
+  return AE_OK;
+}
+
+ae_status ae_linear_e4m3(const void *d_x, const void *d_w, const float *d_cs, int64_t M, int32_t N, int32_t K,
+                         float lo, float hi, ae_lin_out out, float lo2, float hi2, float q_out, void *d_y,
+                         ae_stream stream) {
+  if (out != AE_LIN_BF16 && out != AE_LIN_SILU_E4M3) return fail(AE_EINVAL, "out");
+  if (M < 0 || M > INT32_MAX) return fail(AE_EINVAL, "M must be in [0, 2^31)");
+  if (K <= 0 || K % 128 || K > 65536) return fail(AE_EINVAL, "K must be a positive multiple of 128 up to 65536");
+  if (N <= 0 || N % 256 || N > 65536) return fail(AE_EINVAL, "N must be a positive multiple of 256 up to 65536");
+  if (std::isnan(lo) || std::isnan(hi) || lo > hi) return fail(AE_EINVAL, "lo, hi");
+  if (out == AE_LIN_SILU_E4M3 && (std::isnan(lo2) || std::isnan(hi2) || lo2 > hi2 || !(q_out > 0.f) ||
+                                  !std::isfinite(q_out)))
+    return fail(AE_EINVAL, "lo2, hi2 or q_out");
+  if (M == 0) return AE_OK;
+  if (!d_x || !d_w || !d_cs || !d_y) return fail(AE_EINVAL, "a device pointer is null");
+  if (!aligned16(d_x) || !aligned16(d_w) || !aligned16(d_cs) || (reinterpret_cast<uintptr_t>(d_y) & 31))
+    return fail(AE_EINVAL, "x, w and cs must be 16-byte aligned, y 32-byte aligned");
+  CUtensorMap tW;
+  if (!make_tmap_2d_u8(&tW, d_w, (uint64_t)K, (uint64_t)N, (uint64_t)K, 128, 128))
+    return fail(AE_ECUDA, "tensor map encoding failed");
+  EpiArgs e = ep_of(d_y, N, lo, hi);
+  e.cs = d_cs;
+  if (out == AE_LIN_SILU_E4M3) {
+    e.lo2 = lo2;
+    e.hi2 = hi2;
+    e.clamp2 = silu_clamp_binds(hi, lo2, hi2);
+    e.q8 = q_out;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const cudaError_t err = gemm8_t(d_x, M, K, tW, N, out == AE_LIN_BF16 ? EPI_BF16 : EPI_SILU_Q8, e, s);
+  if (err != cudaSuccess) return cuda_fail(err, "e4m3 projection");
   return AE_OK;
 }
 

@@ -235,6 +235,13 @@ __device__ __forceinline__ uint32_t map_to_rank(const void *p, uint32_t rank) {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
+// The same arrive without release semantics: for a consumer that only signals
+// that data it has already waited for (tensor-memory loads completed by
+// tcgen05.wait::ld) may be overwritten, so none of its own memory writes need
+// to be visible first (a release would wait for its outstanding global stores).
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
 // TMA tile load of a CTA pair: lands in this CTA's shared memory, completes
 // bytes on the barrier at the same offset in the pair's even (leader) CTA.
 __device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *tm, int x, int y, uint64_t *bar) {
@@ -264,6 +271,17 @@ __device__ __forceinline__ void tc_mma_bf16_pair(uint32_t d_tmem, uint64_t adesc
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// The same pair MMA on 8-bit operands (kind::f8f6f4: K = 32 per instruction,
+// float32 accumulate); the operand formats are in the instruction descriptor.
+__device__ __forceinline__ void tc_mma_f8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -307,6 +325,23 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
 __device__ __forceinline__ uint64_t sw128_desc_mn(uint32_t saddr, uint32_t mn_stride) {
   return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)((mn_stride >> 4) & 0x3FFF) << 16) |
          ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor of kind::f8f6f4 with A and B e4m3 (format code 0 at
+// bits 7-9 and 10-12), D f32, both K-major.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Two floats to two e4m3 codes (round to nearest even, saturating to +-448):
+// a in the low byte, b in the high byte.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float a, float b) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(b), "f"(a));
+  return r;
+}
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  return pack_e4m3x2(a, b) | (pack_e4m3x2(c, d) << 16);
 }
 
 // The same instruction descriptor with B MN-major (bit 16).

@@ -48,11 +48,48 @@ __device__ __forceinline__ void st_granule(uint8_t *line, int r7, int g, uint4 v
   *reinterpret_cast<uint4 *>(line + ((g ^ r7) << 4)) = v;
 }
 
+// e4m3 projections: accumulator column j times cs[j] (the weight row's scale
+// over the input's code scale). Every lane reads the same 32 factors.
+__device__ __forceinline__ void scale_cols(const float *cs, float (&v)[32]) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float4 c = __ldg(reinterpret_cast<const float4 *>(cs) + j);
+    const float2 a = __fmul2_rn(make_float2(v[4 * j], v[4 * j + 1]), make_float2(c.x, c.y));
+    const float2 b = __fmul2_rn(make_float2(v[4 * j + 2], v[4 * j + 3]), make_float2(c.z, c.w));
+    v[4 * j] = a.x;
+    v[4 * j + 1] = a.y;
+    v[4 * j + 2] = b.x;
+    v[4 * j + 3] = b.y;
+  }
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// c * sigmoid(g) = c / (1 + 2^(-g log2 e)) for two lanes: the power of two and
+// the reciprocal from the special-function unit's approximations, the
+// multiplies and the add on the packed two-lane pipe. Limits: g -> -inf gives
+// 0 (the reciprocal of +inf), g -> +inf gives c.
+__device__ __forceinline__ float2 mul_sigmoid2(float2 c, float2 g) {
+  constexpr float kNegLog2e = -1.4426950408889634f;
+  const float2 t = __fmul2_rn(g, make_float2(kNegLog2e, kNegLog2e));
+  const float2 d = __fadd2_rn(make_float2(ex2_approx(t.x), ex2_approx(t.y)), make_float2(1.0f, 1.0f));
+  return __fmul2_rn(c, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
+}
+
 // Epilogue of 32 accumulator columns [col, col + 32) of one row, written as
 // granules g0, g0 + 1, ... of the row's staging line: 8 granules of f32
 // (EPI_F32), 4 of bf16 (EPI_BF16, EPI_SILU), 2 of bf16 (EPI_GLU, which pairs
 // columns (2c, 2c + 1) into output column c).
-template <int MODE>
+template <int MODE, bool SC>
 __device__ __forceinline__ void epi_stage(const EpiArgs &ep, int col, const uint32_t (&r)[32], uint8_t *line, int r7,
                                           int g0) {
   float lo = ep.lo, hi = ep.hi;
@@ -64,6 +101,7 @@ __device__ __forceinline__ void epi_stage(const EpiArgs &ep, int col, const uint
   float v[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  if (SC) scale_cols(ep.cs + col, v);
   if (MODE == EPI_F32 || MODE == EPI_ADD_F32) {
     if (MODE == EPI_F32 && ep.bias) {
 #pragma unroll
@@ -104,14 +142,15 @@ __device__ __forceinline__ void epi_stage(const EpiArgs &ep, int col, const uint
 
 __device__ __forceinline__ void st_global_32B(void *p, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t a4,
                                               uint32_t a5, uint32_t a6, uint32_t a7) {
+  // no memory clobber: nothing in the kernel reads the outputs, so the next
+  // chunk's loads may be scheduled ahead of these stores
   asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a0), "r"(a1), "r"(a2),
-               "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7)
-               : "memory");
+               "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7));
 }
 
 // Epilogue of 32 accumulator columns of one row, stored from registers as
 // whole 32-byte sectors (the bf16 outputs; f32 outputs go through epi_stage).
-template <int MODE>
+template <int MODE, bool SC>
 __device__ __forceinline__ void epi_store32(const EpiArgs &ep, int row, int col, const uint32_t (&r)[32]) {
   float lo = ep.lo, hi = ep.hi;
   if (ep.seg_w > 0) {
@@ -122,6 +161,7 @@ __device__ __forceinline__ void epi_store32(const EpiArgs &ep, int row, int col,
   float v[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  if (SC) scale_cols(ep.cs + col, v);
   if (MODE == EPI_F32) {
     if (ep.bias) {
 #pragma unroll
@@ -137,20 +177,46 @@ __device__ __forceinline__ void epi_store32(const EpiArgs &ep, int row, int col,
   } else if (MODE == EPI_GLU) {
     uint32_t p[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      float a0 = clampf(v[4 * j + 0], lo, hi), b0 = clampf(v[4 * j + 1], lo, hi);
-      float a1 = clampf(v[4 * j + 2], lo, hi), b1 = clampf(v[4 * j + 3], lo, hi);
-      p[j] = pack_bf16(__fdividef(a0, 1.0f + __expf(-b0)), __fdividef(a1, 1.0f + __expf(-b1)));
+    for (int j = 0; j < 8; ++j) {  // columns (4j, 4j+1, 4j+2, 4j+3) = (a, b, a, b)
+      const float2 a = make_float2(clampf(v[4 * j], lo, hi), clampf(v[4 * j + 2], lo, hi));
+      const float2 b = make_float2(clampf(v[4 * j + 1], lo, hi), clampf(v[4 * j + 3], lo, hi));
+      const float2 y = mul_sigmoid2(a, b);
+      p[j] = pack_bf16(y.x, y.y);
     }
     bf16 *o = static_cast<bf16 *>(ep.out) + (int64_t)row * ep.ld + col / 2;
     st_global_32B(o, p[0], p[1], p[2], p[3], p[4], p[5], p[6], p[7]);
-  } else {
+  } else if (MODE == EPI_SILU || MODE == EPI_SILU_Q8) {
+    float2 y[16];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      float x = clampf(v[i], lo, hi);
-      if (MODE == EPI_SILU) x = clampf(__fdividef(x, 1.0f + __expf(-x)), ep.lo2, ep.hi2);
-      v[i] = x;
+    for (int j = 0; j < 16; ++j) {
+      const float2 c = make_float2(clampf(v[2 * j], lo, hi), clampf(v[2 * j + 1], lo, hi));
+      y[j] = mul_sigmoid2(c, c);
     }
+    if (ep.clamp2) {  // the host clears it when the second clamp cannot bind
+#pragma unroll
+      for (int j = 0; j < 16; ++j) y[j] = make_float2(clampf(y[j].x, ep.lo2, ep.hi2), clampf(y[j].y, ep.lo2, ep.hi2));
+    }
+    if (MODE == EPI_SILU_Q8) {  // the next projection's e4m3 operand: 32 codes, one 32-byte sector
+      uint32_t p[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float2 a = __fmul2_rn(y[2 * j], make_float2(ep.q8, ep.q8));
+        const float2 b = __fmul2_rn(y[2 * j + 1], make_float2(ep.q8, ep.q8));
+        p[j] = pack_e4m3x4(a.x, a.y, b.x, b.y);
+      }
+      uint8_t *o = static_cast<uint8_t *>(ep.out) + (int64_t)row * ep.ld + col;
+      st_global_32B(o, p[0], p[1], p[2], p[3], p[4], p[5], p[6], p[7]);
+    } else {
+      uint32_t p[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) p[j] = pack_bf16(y[j].x, y[j].y);
+      bf16 *o = static_cast<bf16 *>(ep.out) + (int64_t)row * ep.ld + col;
+      st_global_32B(o, p[0], p[1], p[2], p[3], p[4], p[5], p[6], p[7]);
+      st_global_32B(o + 16, p[8], p[9], p[10], p[11], p[12], p[13], p[14], p[15]);
+    }
+  } else {  // EPI_BF16
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = clampf(v[i], lo, hi);
     uint32_t p[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) p[j] = pack_bf16(v[2 * j], v[2 * j + 1]);
@@ -166,14 +232,21 @@ namespace {
 constexpr int BM = 128;                 // rows of x per CTA (256 per pair)
 constexpr int BK = 64;                  // one 128-byte swizzle atom of bf16
 constexpr int BN = 256;                 // columns per pair tile (128 rows of W per CTA)
-constexpr int STAGES = 4;
 constexpr uint32_t A_BYTES = BM * BK * 2, B_BYTES = (BN / 2) * BK * 2, STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr uint32_t TMEM_COLS = 2 * BN;  // two 128 x 256 f32 accumulators per CTA
 constexpr int EPI_WARPS = 8;
 constexpr uint32_t LINE_BYTES = 32 * 128;  // one staging box: 32 rows x 128 bytes
 constexpr uint32_t EPI_BYTES = EPI_WARPS * LINE_BYTES;  // one box per epilogue warp
 constexpr int GEMM_THREADS = 64 + 32 * EPI_WARPS;
-constexpr size_t SMEM_TC = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + 256;
+// float32 outputs go through the staging boxes, which leave room for a
+// 4-stage ring; the other epilogues store from registers and take 6 stages,
+// which keeps more loads in flight (the e4m3 mainloop consumes a stage in half
+// the time of a bf16 one).
+__host__ __device__ constexpr bool f32_out(int mode) { return mode == EPI_F32 || mode == EPI_ADD_F32; }
+__host__ __device__ constexpr int stages_of(int mode) { return f32_out(mode) ? 4 : 6; }
+__host__ __device__ constexpr size_t smem_of(int mode) {
+  return stages_of(mode) * STAGE_BYTES + (f32_out(mode) ? EPI_BYTES : 0) + 1024 + 256;
+}
 }  // namespace
 
 // Persistent pair kernel (cluster of 2 CTAs on 2 SMs). Pair tile 256 x 256:
@@ -182,15 +255,16 @@ constexpr size_t SMEM_TC = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + 256;
 // issues tcgen05.mma.cta_group::2 (M=256, N=256, K=16), which reads the A and
 // B halves from both CTAs' shared memory and accumulates rows 128 r .. +127
 // in CTA r's tensor memory. Each CTA's epilogue drains its own 128 rows.
-template <int MODE>
+template <int MODE, bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const EpiArgs ep, const int M, const int N, const int K,
               unsigned *status) {
+  constexpr int STAGES = stages_of(MODE);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *epi_smem = smem + STAGES * STAGE_BYTES;                                 // store boxes
-  uint64_t *full = reinterpret_cast<uint64_t *>(epi_smem + EPI_BYTES);            // used in the leader
+  uint8_t *epi_smem = smem + STAGES * STAGE_BYTES;                                 // store boxes (f32 outputs)
+  uint64_t *full = reinterpret_cast<uint64_t *>(epi_smem + (f32_out(MODE) ? EPI_BYTES : 0));  // used in the leader
   uint64_t *empty = full + STAGES;                                              // per CTA
   uint64_t *tfull = empty + STAGES;                                             // per CTA
   uint64_t *tempty = tfull + 2;                                                 // used in the leader
@@ -201,7 +275,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
   const bool leader = rank == 0;
-  const int m_blocks = (M + 2 * BM - 1) / (2 * BM), n_blocks = N / BN, kb_n = K / BK;
+  // one k-block is a 128-byte swizzle atom per row: 64 bf16 or 128 e4m3 elements
+  constexpr int BKE = F8 ? 2 * BK : BK;
+  const int m_blocks = (M + 2 * BM - 1) / (2 * BM), n_blocks = N / BN, kb_n = K / BKE;
   const int num_tiles = m_blocks * n_blocks;
   const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
 
@@ -245,8 +321,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         }
         uint8_t *sa = smem + stage * STAGE_BYTES;
         if (leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
-        tma_load_2d_pair(sa, &tmA, kb * BK, arow, &full[stage]);
-        tma_load_2d_pair(sa + A_BYTES, &tmB, kb * BK, brow, &full[stage]);
+        tma_load_2d_pair(sa, &tmA, kb * BKE, arow, &full[stage]);
+        tma_load_2d_pair(sa + A_BYTES, &tmB, kb * BKE, brow, &full[stage]);
         ++issued;
         if (++stage == STAGES) {
           stage = 0;
@@ -266,7 +342,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     }
   } else if (warp == 1 && lane == 0 && leader) {
     // ---------------- MMA issuer (leader CTA only)
-    constexpr uint32_t idesc = idesc_bf16_f32(2 * BM, BN);
+    constexpr uint32_t idesc = F8 ? idesc_e4m3_f32(2 * BM, BN) : idesc_bf16_f32(2 * BM, BN);
     int stage = 0, acc = 0;
     uint32_t phase = 0, acc_phase = 0;
     bool ok = true;
@@ -286,8 +362,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
         const uint32_t sb = sa + A_BYTES;
 #pragma unroll
-        for (int k = 0; k < BK / 16; ++k)
-          tc_mma_bf16_pair(d_tmem, sw128_desc(sa + k * 32), sw128_desc(sb + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
+        for (int k = 0; k < 4; ++k) {  // 32 bytes of k per instruction: K = 16 bf16 or 32 e4m3
+          if (F8)
+            tc_mma_f8_pair(d_tmem, sw128_desc(sa + k * 32), sw128_desc(sb + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
+          else
+            tc_mma_bf16_pair(d_tmem, sw128_desc(sa + k * 32), sw128_desc(sb + k * 32), idesc,
+                             (kb | k) != 0 ? 1u : 0u);
+        }
         tc_commit_pair_both(&empty[stage]);  // frees the stage in both CTAs
         if (++stage == STAGES) {
           stage = 0;
@@ -340,11 +421,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + half * (BN / 2));
       auto stage = [&](int c, const uint32_t(&r)[32]) {
         if (!F32_OUT) {  // bf16 rows: 32-byte stores straight from registers
-          if (row0 + lane < M) epi_store32<MODE>(ep, row0 + lane, col0 + c * 32, r);
+          if (row0 + lane < M) epi_store32<MODE, F8>(ep, row0 + lane, col0 + c * 32, r);
           return;
         }
         const int j = c % LOADS_PER_BOX;
-        epi_stage<MODE>(ep, col0 + c * 32, r, box + lane * 128, lane & 7, j * GRANULES_PER_LOAD);
+        epi_stage<MODE, F8>(ep, col0 + c * 32, r, box + lane * 128, lane & 7, j * GRANULES_PER_LOAD);
         if (j == LOADS_PER_BOX - 1) {
           __syncwarp();
           // lane l moves granule l % 8 of rows l / 8, l / 8 + 4, ...
@@ -383,7 +464,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(tempty_leader + (uint32_t)(acc * sizeof(uint64_t)));
+      if (lane == 0) mbar_arrive_cluster_relaxed(tempty_leader + (uint32_t)(acc * sizeof(uint64_t)));
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
@@ -496,6 +577,19 @@ bool make_tmap_2d_bf16(CUtensorMap *tm, const void *base, uint64_t inner, uint64
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_tmap_2d_u8(CUtensorMap *tm, const void *base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                     uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Stem conv0 output viewed as 5-D for the implicit GEMM of conv1:
 // (c 128, fpar 2, fp 32, tpar 2, tp rows/2), boxes (64, 1, 32, 1, 4).
 bool make_tmap_stem_y0(CUtensorMap *tm, const void *y0, int64_t stem_rows) {
@@ -520,19 +614,19 @@ static int num_sms() {
   return n[dev] > 0 ? n[dev] : 1;
 }
 
-template <int MODE>
+template <int MODE, bool F8 = false>
 static cudaError_t launch_tc(const CUtensorMap &tA, const CUtensorMap &tB, const EpiArgs &ep, int M, int N, int K,
                              cudaStream_t s) {
-
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_TC);
+    cudaError_t e =
+        cudaFuncSetAttribute(k_gemm_tc<MODE, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_of(MODE));
     if (e != cudaSuccess) return e;
     attr = true;
   }
   const int tiles = ((M + 2 * BM - 1) / (2 * BM)) * (N / BN);
   const int pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;
-  return launch_k(k_gemm_tc<MODE>, dim3(2 * pairs), dim3(GEMM_THREADS), SMEM_TC, s, tA, tB, ep, M, N, K,
+  return launch_k(k_gemm_tc<MODE, F8>, dim3(2 * pairs), dim3(GEMM_THREADS), smem_of(MODE), s, tA, tB, ep, M, N, K,
                   device_status_word());
 }
 
@@ -546,7 +640,7 @@ static cudaError_t launch_f32(const float *x, const float *w, const EpiArgs &ep,
 cudaError_t gemm(const ae_model *m, const void *x, int64_t M, int K, const void *w, const CUtensorMap *tmW, int N,
                  int mode, const EpiArgs &ep, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
-  if (m->dtype == AE_BF16) {
+  if (m->dtype != AE_F32) {
     CUtensorMap tA, tB;
     if (!make_tmap_2d_bf16(&tA, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK, BM)) return cudaErrorInvalidValue;
     if (!tmW) {
@@ -571,6 +665,20 @@ cudaError_t gemm(const ae_model *m, const void *x, int64_t M, int K, const void 
     case EPI_BF16: return launch_f32<EPI_BF16>(xf, wf, ep, (int)M, N, K, s);
     case EPI_SILU: return launch_f32<EPI_SILU>(xf, wf, ep, (int)M, N, K, s);
     case EPI_GLU: return launch_f32<EPI_GLU>(xf, wf, ep, (int)M, N, K, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t gemm_e4m3(const void *x, int64_t M, int K, const CUtensorMap &tmW, int N, int mode, const EpiArgs &ep,
+                      cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  if (K % (2 * BK) || N % BN || !ep.cs) return cudaErrorInvalidValue;
+  CUtensorMap tA;
+  if (!make_tmap_2d_u8(&tA, x, (uint64_t)K, (uint64_t)M, (uint64_t)K, 2 * BK, BM)) return cudaErrorInvalidValue;
+  switch (mode) {
+    case EPI_BF16: return launch_tc<EPI_BF16, true>(tA, tmW, ep, (int)M, N, K, s);
+    case EPI_GLU: return launch_tc<EPI_GLU, true>(tA, tmW, ep, (int)M, N, K, s);
+    case EPI_SILU_Q8: return launch_tc<EPI_SILU_Q8, true>(tA, tmW, ep, (int)M, N, K, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(256, NV <= 8 ? 3 : 2) k_rowop(const RowArgs r)
       inv = rsqrtf(warp_sum(ss) * (1.0f / W) + kEps);
     }
     ActT *arow = static_cast<ActT *>(r.a_out) + row * W;
+    uint32_t *qrow = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(r.a_out) + row * W);
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
       float w[4] = {1.f, 1.f, 1.f, 1.f};
@@ -112,7 +113,10 @@ __global__ void __launch_bounds__(256, NV <= 8 ? 3 : 2) k_rowop(const RowArgs r)
       float a[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) a[u] = clampf(h[i][u] * inv * w[u], r.lo, r.hi);
-      store4(arow + (i * 32 + lane) * 4, a);
+      if (r.a_q8 > 0.f)  // e4m3 operand: 4 codes per lane, 128 contiguous bytes per warp
+        qrow[i * 32 + lane] = pack_e4m3x4(a[0] * r.a_q8, a[1] * r.a_q8, a[2] * r.a_q8, a[3] * r.a_q8);
+      else
+        store4(arow + (i * 32 + lane) * 4, a);
     }
   }
 }
@@ -130,7 +134,7 @@ static cudaError_t rowop_width(const RowArgs &r, cudaStream_t s) {
 
 cudaError_t launch_rowop(const ae_model *m, const RowArgs &r, cudaStream_t s) {
   if (r.rows <= 0) return cudaSuccess;
-  return m->dtype == AE_BF16 ? rowop_width<bf16>(r, s) : rowop_width<float>(r, s);
+  return m->dtype == AE_F32 ? rowop_width<float>(r, s) : rowop_width<bf16>(r, s);
 }
 
 // ------------------------------------------------------------------ light conv middle
@@ -243,7 +247,7 @@ cudaError_t launch_lconv(const ae_model *m, const void *gl, const float *w_dw, c
                          float hi, void *out, const int32_t *pos, int64_t T, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
   const unsigned grid = (unsigned)((T + kLcRows - 1) / kLcRows);
-  if (m->dtype == AE_BF16)
+  if (m->dtype != AE_F32)
     return launch_k(k_lconv<bf16>, dim3(grid), dim3(256), 0, s, static_cast<const bf16 *>(gl), w_dw, w_norm, lo, hi,
                     static_cast<bf16 *>(out), pos, T);
   return launch_k(k_lconv<float>, dim3(grid), dim3(256), 0, s, static_cast<const float *>(gl), w_dw, w_norm, lo, hi,

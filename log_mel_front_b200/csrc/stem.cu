@@ -303,7 +303,7 @@ cudaError_t launch_conv0(const ae_model *m, const float *mel, void *y0, const Cl
                          cudaStream_t s) {
   if (stem_rows <= 0) return cudaSuccess;
   const unsigned grid = (unsigned)((stem_rows + kConv0Rows - 1) / kConv0Rows);
-  if (m->dtype == AE_BF16)
+  if (m->dtype != AE_F32)
     return launch_k(k_conv0<bf16>, dim3(grid), dim3(128), 0, s, mel, (const float *)m->conv0c,
                     (const float *)m->conv0cov, static_cast<bf16 *>(y0), t, stem_rows);
   return launch_k(k_conv0<float>, dim3(grid), dim3(128), 0, s, mel, (const float *)m->conv0c,
@@ -313,7 +313,7 @@ cudaError_t launch_conv0(const ae_model *m, const float *mel, void *y0, const Cl
 cudaError_t launch_conv1(const ae_model *m, const void *y0, int64_t stem_rows, void *xs, const ClipTablesDev &t,
                          int64_t conv1_tiles, int64_t tokens, cudaStream_t s) {
   if (tokens <= 0) return cudaSuccess;
-  if (m->dtype == AE_BF16) {
+  if (m->dtype != AE_F32) {
     static bool attr = false;
     if (!attr) {
       cudaError_t e = cudaFuncSetAttribute(k_conv1_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C1_SMEM);
