@@ -59,6 +59,8 @@ def peaks():
 TRAFFIC_PROFILES = {
     "gemm": ("profiles/gemm_tc_tower_dram.md",
              ("log_mel_front_b200/csrc/gemm.cu", "log_mel_front_b200/csrc/common.cuh")),
+    "gemm_fp8": ("profiles/gemm_e4m3_tower_dram.md",
+                 ("log_mel_front_b200/csrc/gemm.cu", "log_mel_front_b200/csrc/common.cuh")),
 }
 
 
