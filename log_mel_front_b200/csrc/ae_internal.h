@@ -213,6 +213,8 @@ struct RsPlan {
   int NT = 1, D = 1, W = 0, W_pad = 0, lo_min = 0, Q = 32, TG = 1, n_groups = 1, span = 0;
   bool stage_coef = true;
   size_t smem = 0;
+  bool pipe = false;     // the persistent, double-buffered FIR applies
+  size_t smem_pipe = 0;  // its shared memory
 };
 int64_t rs_len(int64_t n, int rate_in, int rate_out);  // -1 for invalid arguments
 RsPlan rs_plan(int rate_in, int rate_out);

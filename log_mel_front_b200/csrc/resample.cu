@@ -14,16 +14,18 @@
 // W_pad offsets), and stores them as one float4 per (T, i); zero outside each
 // output's 64 zero crossings.
 //
-// k_rs_fir: a CTA owns a tile of Q consecutive units of each of up to eight
-// types of one clip. It stages the input span the tile touches and the
-// types' tap rows in shared memory; a warp takes one (type, 32-unit group)
-// item at a time with lane = unit, so for every input offset the warp reads
-// one float4 of taps (the same shared-memory address for all lanes: a
-// broadcast) and each lane one input sample, and does four FMAs. Each lane
-// writes its unit's four outputs. When the span does not fit (large D, as for
-// co-prime rates) the FIR reads the input from global memory, and when the
-// tap rows do not fit it reads them from global memory too: correct, and
-// slower.
+// The FIR works on tiles of Q consecutive units of each of up to eight types
+// of one clip: the input span the tile touches and the types' tap rows sit in
+// shared memory, and a warp takes a (type, 32-unit group) item with lane =
+// unit, so for every input offset the warp reads one float4 of taps (the same
+// shared-memory address for all lanes: a broadcast) and each lane one input
+// sample, and does four FMAs. k_rs_fir_pipe, the persistent form, keeps one
+// type group's tap rows for all its tiles, copies the next tile's span while
+// it computes the current one, and splits each item's offset window over two
+// warps. k_rs_fir, one CTA per tile, serves the plans whose tap rows and two
+// spans do not fit: when the span does not fit (large D, as for co-prime
+// rates) it reads the input from global memory, and when the tap rows do not
+// fit it reads them from global memory too: correct, and slower.
 #include <cmath>
 
 #include "ae_internal.h"
@@ -38,6 +40,7 @@ constexpr double kRsBeta = 12.8;
 constexpr int kRsThreads = 256;
 constexpr int kRsWarps = kRsThreads / 32;
 constexpr size_t kRsSmemMax = 200 * 1024;  // staged input + staged output per CTA
+constexpr size_t kRsPipeSmemMax = 220 * 1024;  // tap rows + two input spans (persistent form)
 }  // namespace
 
 // I0(x) = sum_k ((x / 2)^2)^k / (k!)^2, summed while the terms still count.
@@ -101,8 +104,132 @@ struct RsArgs {
   int n_clips, NT, D, W_pad, Q, TG, n_groups;
   int lo_min, span;         // span: staged inputs per tile (0: read from global memory)
   int stage_coef;           // the group's tap rows live in shared memory
+  int n_tiles;              // tiles of the call (each covers Q units of every type of one clip)
 };
 
+// Clip of a tile (the last clip whose first tile is <= tile; empty clips own
+// no tiles) and the tile's first unit and first input index within its clip.
+struct RsTile {
+  int64_t in0, n_in, out0, n_out, q0, base;
+};
+__device__ __forceinline__ RsTile rs_tile(const RsArgs &a, int tile) {
+  int l = 0, h = a.n_clips;
+  while (h - l > 1) {
+    const int mid = (l + h) >> 1;
+    if (a.tile_off[mid] <= tile) l = mid; else h = mid;
+  }
+  RsTile r;
+  r.in0 = a.in_off[l];
+  r.n_in = a.in_off[l + 1] - r.in0;
+  r.out0 = a.out_off[l];
+  r.n_out = a.out_off[l + 1] - r.out0;
+  r.q0 = (int64_t)(tile - a.tile_off[l]) * a.Q;
+  r.base = r.q0 * a.D + a.lo_min;
+  return r;
+}
+
+// 4-byte asynchronous copy global -> shared; with valid == false nothing is
+// read and the destination is zero-filled.
+__device__ __forceinline__ void cp_async4(float *dst, const float *src, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 4 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// Partial FIR of one warp item over input offsets [i0, i1) (even, i1 - i0 a
+// multiple of 2) from staged taps and a staged input span: lane = unit, four
+// outputs per lane, two partial sums (even and odd offsets).
+__device__ __forceinline__ float4 rs_partial(const RsArgs &a, const RsTile &r, const float *span, const float4 *cT,
+                                             int T, int ql, int i0, int i1) {
+  const int64_t m0 = (r.q0 + ql) * a.D + a.lo[T];
+  const float *xr = span + (m0 - r.base);
+  float4 e = make_float4(0.f, 0.f, 0.f, 0.f), d = e;
+#pragma unroll 4
+  for (int i = i0; i < i1; i += 2) {
+    const float4 w0 = cT[i], w1 = cT[i + 1];
+    const float x0 = xr[i], x1 = xr[i + 1];
+    e.x = fmaf(w0.x, x0, e.x);
+    e.y = fmaf(w0.y, x0, e.y);
+    e.z = fmaf(w0.z, x0, e.z);
+    e.w = fmaf(w0.w, x0, e.w);
+    d.x = fmaf(w1.x, x1, d.x);
+    d.y = fmaf(w1.y, x1, d.y);
+    d.z = fmaf(w1.z, x1, d.z);
+    d.w = fmaf(w1.w, x1, d.w);
+  }
+  return make_float4(e.x + d.x, e.y + d.y, e.z + d.z, e.w + d.w);
+}
+
+// Persistent form, for plans whose group tap rows and two input spans fit in
+// shared memory: CTA b serves type group b mod n_groups for the tiles
+// b / n_groups, + per, ... of the whole call. The group's tap rows are staged
+// once; the input span of the next tile is copied asynchronously (4 bytes a
+// lane, coalesced, zero-filled outside the clip) while the current tile is
+// computed, so the copies hide behind the multiply-adds. Each (type, 32-unit)
+// item is split over two warps, one per half of the offset window, so that
+// 16 warps keep the shared-memory loads' latency covered; the second half's
+// sums meet the first's in shared memory.
+constexpr int kRsPipeThreads = 512;
+constexpr int kRsPipeItems = kRsWarps;  // items per tile: (Q / 32) x types of the group <= 8
+
+__global__ void __launch_bounds__(kRsPipeThreads) k_rs_fir_pipe(const RsArgs a, int per) {
+  extern __shared__ __align__(16) float rs_smem[];
+  const int g = blockIdx.x % a.n_groups;
+  int t = blockIdx.x / a.n_groups;
+  if (t >= a.n_tiles) return;
+  const int T0 = g * a.TG, n_types = min(a.TG, a.NT - T0);
+  float4 *cs = reinterpret_cast<float4 *>(rs_smem);                  // [TG][W_pad]
+  float4 *red = cs + a.TG * a.W_pad;                                  // [items][32]: second halves
+  float *buf0 = reinterpret_cast<float *>(red + kRsPipeItems * 32);  // two input spans
+  auto stage = [&](int tile, float *dst) {
+    const RsTile r = rs_tile(a, tile);
+    const float *xin = a.x + r.in0;
+    for (int i = threadIdx.x; i < a.span; i += kRsPipeThreads) {
+      const int64_t m = r.base + i;
+      const bool ok = m >= 0 && m < r.n_in;
+      cp_async4(dst + i, ok ? xin + m : a.x, ok);
+    }
+  };
+  stage(t, buf0);
+  cp_async_commit();
+  {
+    const float4 *src = a.coef + (int64_t)T0 * a.W_pad;
+    for (int i = threadIdx.x; i < n_types * a.W_pad; i += kRsPipeThreads) cs[i] = __ldg(src + i);
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int items = (a.Q / 32) * n_types;
+  const int item = warp % kRsPipeItems, part = warp / kRsPipeItems;
+  const int hw = a.W_pad / 2;  // W_pad is a multiple of 8: both halves even
+  const int tl = item % n_types, ql = (item / n_types) * 32 + lane;
+  for (int k = 0; t < a.n_tiles; ++k, t += per) {
+    if (t + per < a.n_tiles) stage(t + per, buf0 + ((k + 1) & 1) * a.span);
+    cp_async_commit();  // possibly empty: keeps one group per iteration
+    cp_async_wait_1();  // this tile's span has landed (this thread's copies)
+    __syncthreads();    // ... and every thread's
+    const RsTile r = rs_tile(a, t);
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (item < items) {
+      v = rs_partial(a, r, buf0 + (k & 1) * a.span, cs + (int64_t)tl * a.W_pad, T0 + tl, ql, part * hw,
+                     (part + 1) * hw);
+      if (part == 1) red[item * 32 + lane] = v;
+    }
+    __syncthreads();
+    if (item < items && part == 0) {
+      const float4 u = red[item * 32 + lane];
+      const float r4[4] = {v.x + u.x, v.y + u.y, v.z + u.z, v.w + u.w};
+      const int T = T0 + tl;
+      const int64_t n0 = ((r.q0 + ql) * a.NT + T) * 4;  // first output of the unit
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (n0 + j < r.n_out) a.y[r.out0 + n0 + j] = r4[j];
+    }
+    __syncthreads();  // the span buffer is refilled and red rewritten on the next tiles
+  }
+}
+
+// Per-tile form (one CTA per tile and type group), for plans the persistent form
+// cannot hold: spans read from global memory, or tap rows too large to stage twice.
 __global__ void __launch_bounds__(kRsThreads) k_rs_fir(const RsArgs a) {
   extern __shared__ __align__(16) float rs_smem[];
   // tile = (clip, block of Q units of each type, group of TG types)
@@ -228,6 +355,9 @@ RsPlan rs_plan(int rate_in, int rate_out) {
   pl.span = span_b + (pl.stage_coef ? coef_bytes : 0) <= (int64_t)kRsSmemMax ? (int)span_of(pl.Q) : 0;
   pl.span = (pl.span + 3) & ~3;  // the tap rows that follow stay 16-byte aligned
   pl.smem = 4 * (size_t)pl.span + (pl.stage_coef ? (size_t)coef_bytes : 0);
+  // the persistent form keeps the tap rows, the second halves' sums and two input spans
+  pl.smem_pipe = 8 * (size_t)pl.span + (size_t)coef_bytes + 16 * 32 * (size_t)kRsWarps;
+  pl.pipe = pl.stage_coef && pl.span > 0 && pl.smem_pipe <= kRsPipeSmemMax;
   return pl;
 }
 
@@ -256,10 +386,6 @@ cudaError_t launch_rs_fir(const RsPlan &pl, const float *mono, float *y, const f
                           const int64_t *in_off, const int64_t *out_off, const int32_t *tile_off, int n_clips,
                           int n_tiles, cudaStream_t s) {
   if (n_tiles <= 0) return cudaSuccess;
-  if (pl.smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(k_rs_fir, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRsSmemMax);
-    if (e != cudaSuccess) return e;
-  }
   RsArgs a;
   a.x = mono;
   a.y = y;
@@ -278,6 +404,27 @@ cudaError_t launch_rs_fir(const RsPlan &pl, const float *mono, float *y, const f
   a.lo_min = pl.lo_min;
   a.span = pl.span;
   a.stage_coef = pl.stage_coef ? 1 : 0;
+  a.n_tiles = n_tiles;
+  if (pl.pipe) {
+    cudaError_t e = cudaFuncSetAttribute(k_rs_fir_pipe, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)pl.smem_pipe);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0, per_sm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_rs_fir_pipe, kRsPipeThreads,
+                                                           pl.smem_pipe)) != cudaSuccess)
+      return e;
+    // CTAs per type group: every resident slot busy, but no more than the tiles
+    const int per = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)sms * std::max(per_sm, 1) / pl.n_groups,
+                                                                 n_tiles));
+    return launch_k(k_rs_fir_pipe, dim3((unsigned)(per * pl.n_groups)), dim3(kRsPipeThreads), pl.smem_pipe, s, a,
+                    per);
+  }
+  if (pl.smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(k_rs_fir, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRsSmemMax);
+    if (e != cudaSuccess) return e;
+  }
   return launch_k(k_rs_fir, dim3((unsigned)((int64_t)n_tiles * pl.n_groups)), dim3(kRsThreads), pl.smem, s, a);
 }
 
