@@ -378,6 +378,15 @@ const char *ae_last_error(void);
  * device reported an error (AE_ECUDA); clears the library's flag. */
 ae_status ae_device_status(void);
 
+/* Exercises the failure path of the kernels' bounded waits without a fault:
+ * enqueues one CTA that waits, with the same bounded wait the kernels use,
+ * on a shared-memory barrier that completes only if `arrive` is nonzero. If
+ * it does not, the wait gives up after limit_us microseconds and records the
+ * timeout, so that the next ae_device_status returns AE_EDEVICE (and clears
+ * it) while the context stays usable. limit_us in [1, 1000000] (AE_EINVAL
+ * otherwise). Asynchronous on `stream`. */
+ae_status ae_selftest_bounded_wait(uint32_t limit_us, int arrive, ae_stream stream);
+
 /* Version of the library, "major.minor.patch". */
 const char *ae_version(void);
 

@@ -92,6 +92,7 @@ _sig("ae_resample_workspace_size", _sz, _i64p, _i32, C.c_int32, C.c_int32, _i32)
 _sig("ae_resample", _st, _vp, _i32, C.c_int64, _i64p, _i32, C.c_int32, C.c_int32, _vp, _vp, _sz, _vp)
 _sig("ae_linear_e4m3", _st, _vp, _vp, _vp, C.c_int64, C.c_int32, C.c_int32, C.c_float, C.c_float, _i32, C.c_float,
      C.c_float, C.c_float, _vp, _vp)
+_sig("ae_selftest_bounded_wait", _st, C.c_uint32, _i32, _vp)
 _sig("ae_profile_enable", _st, _i32)
 _sig("ae_profile_read", _st, C.POINTER(C.c_double), _i64p, C.POINTER(C.c_double), C.POINTER(C.c_double), _i64p)
 
@@ -100,7 +101,8 @@ EXPORTS = ("ae_num_frames", "ae_num_tokens", "ae_model_create", "ae_model_destro
            "ae_logmel", "ae_subsample", "ae_conformer_layer", "ae_encode", "ae_encode_host_workspace_size",
            "ae_encode_host", "ae_encode_host_async", "ae_attention_tables", "ae_local_attention", "ae_last_error", "ae_device_status",
            "ae_version", "ae_profile_enable", "ae_profile_read", "ae_logmel_noalloc", "ae_resample_len",
-           "ae_resample_workspace_size", "ae_resample", "ae_linear_e4m3")
+           "ae_resample_workspace_size", "ae_resample", "ae_linear_e4m3",
+           "ae_selftest_bounded_wait")
 
 KERNEL_CLASSES = ("tables", "logmel", "conv0", "conv1", "gemm", "attention", "lconv", "rowop", "resample",
                   "gemm_fp8")
@@ -240,6 +242,11 @@ def ae_linear_e4m3(d_x, d_w, d_cs, M: int, N: int, K: int, lo: float, hi: float,
 
 def ae_device_status() -> int:
     return lib.ae_device_status()
+
+
+def ae_selftest_bounded_wait(limit_us: int, arrive: bool = False, stream=None):
+    _check(lib.ae_selftest_bounded_wait(int(limit_us), 1 if arrive else 0, _stream(stream)),
+           "ae_selftest_bounded_wait")
 
 
 def ae_version() -> str:

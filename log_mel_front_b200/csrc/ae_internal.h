@@ -228,6 +228,7 @@ cudaError_t launch_rs_fir(const RsPlan &pl, const float *mono, float *y, const f
 cudaError_t launch_upload_bytes(const void *host, size_t bytes, void *dev, cudaStream_t s);
 
 unsigned *device_status_word();
+cudaError_t launch_wait_probe(unsigned long long limit_ns, int arrive, cudaStream_t s);
 unsigned read_and_clear_status();
 cudaError_t launch_pos(int32_t *pos, const int32_t *tok_off, int n_clips, cudaStream_t s);
 void set_error(const std::string &msg);

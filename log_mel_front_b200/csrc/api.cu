@@ -696,6 +696,14 @@ ae_status ae_device_status(void) {
   return AE_OK;
 }
 
+ae_status ae_selftest_bounded_wait(uint32_t limit_us, int arrive, ae_stream stream) {
+  if (limit_us < 1 || limit_us > 1000000) return fail(AE_EINVAL, "limit_us must be in [1, 1000000]");
+  const cudaError_t e =
+      launch_wait_probe(1000ull * limit_us, arrive ? 1 : 0, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "wait probe");
+  return AE_OK;
+}
+
 ae_status ae_attention_tables(const float *relk, const float *pds, int hidden, int heads, int left, float *R,
                               float *qscale, float *k_scale) {
   if (!relk || !pds || !R || !qscale || !k_scale) return fail(AE_EINVAL, "null pointer");

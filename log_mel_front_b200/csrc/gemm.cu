@@ -39,6 +39,23 @@ unsigned *device_status_word() {
   return static_cast<unsigned *>(p);
 }
 
+// The failure path of the bounded waits, exercised without a fault: thread 0
+// initialises an mbarrier of one arrival and waits on its first phase, which
+// completes only if `arrive` (then the wait succeeds at once); otherwise the
+// wait gives up after limit_ns and records the timeout as the kernels do.
+__global__ void k_wait_probe(unsigned long long limit_ns, int arrive, unsigned *status) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  if (arrive) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&bar)) : "memory");
+  if (!mbar_wait_for(&bar, 0, limit_ns)) atomicOr(status, kStatusWaitTimeout);
+}
+
+cudaError_t launch_wait_probe(unsigned long long limit_ns, int arrive, cudaStream_t s) {
+  return launch_k(k_wait_probe, dim3(1), dim3(32), 0, s, limit_ns, arrive, device_status_word());
+}
+
 // ------------------------------------------------------------------ epilogue
 
 // 128-byte line of the staging buffer: the 16-byte granule g of row r sits at

@@ -73,6 +73,16 @@ def test_refusals_before_any_device_work(ae):
     assert e.value.status == ae.AE_EINVAL
     # an empty batch is legal and does nothing
     ae.ae_logmel(0, [0], 0, 0, 0, stream=0)
+    # the bounded-wait self-test and the e4m3 projection check their arguments first
+    for limit in (0, 1000001):
+        with pytest.raises(ae.AEError) as e:
+            ae.ae_selftest_bounded_wait(limit, stream=0)
+        assert e.value.status == ae.AE_EINVAL
+    for M, N, K in ((4, 256, 100), (4, 200, 128), (-1, 256, 128), (4, 256, 131072)):
+        with pytest.raises(ae.AEError) as e:
+            ae.ae_linear_e4m3(0, 0, 0, M, N, K, -8.0, 8.0, 0, stream=0)
+        assert e.value.status == ae.AE_EINVAL
+    ae.ae_linear_e4m3(0, 0, 0, 0, 256, 128, -8.0, 8.0, 0, stream=0)  # M = 0: nothing to do
 
 
 def test_attention_tables_closed_form(ae):
