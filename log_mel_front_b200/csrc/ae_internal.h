@@ -202,12 +202,14 @@ inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, siz
 
 // Resampler (resample.cu): the rates reduced to o (in) and p (out), the cut-off
 // c in cycles per input sample, the window half-width 64 / c in input samples;
-// outputs in units of four: NT unit types, D input samples between units of a
+// outputs in units of U (4 or 8): NT unit types, D input samples between units of a
 // type, W (padded W_pad) input offsets in a unit's window, the lowest offset
 // over all types; and the FIR's tiling (Q units of each of TG types per tile,
 // n_groups type groups, staged input span, tap rows staged or not, shared
 // memory).
 struct RsPlan {
+  int U = 4;      // outputs per unit (4, or 8 in the persistent form when it fits)
+  int parts = 2;  // warps sharing one item's offset window (persistent form)
   int o = 1, p = 1;
   double c = 0.0, half = 0.0;
   int NT = 1, D = 1, W = 0, W_pad = 0, lo_min = 0, Q = 32, TG = 1, n_groups = 1, span = 0;

@@ -1165,7 +1165,7 @@ ae_status rs_tables(const int64_t *off, int n, int32_t rate_in, int32_t rate_out
     t.in_off[i + 1] = off[i + 1];
     const int64_t out = rs_len(len, rate_in, rate_out);
     t.out_off[i + 1] = t.out_off[i] + out;
-    const int64_t units = (out + 3) / 4, per_type = (units + pl.NT - 1) / pl.NT;
+    const int64_t units = (out + pl.U - 1) / pl.U, per_type = (units + pl.NT - 1) / pl.NT;
     const int64_t tiles = rate_in == rate_out ? 0 : (per_type + pl.Q - 1) / pl.Q;
     if ((t.n_tiles + tiles) * pl.n_groups > INT32_MAX)
       return fail(AE_EUNSUPPORTED, "too many resampler tiles in one call");
@@ -1191,7 +1191,7 @@ RsLayout rs_layout(int n_clips, const RsPlan &pl, int64_t total_in, int channels
   L.lo = off;
   off += equal ? 0 : al256((size_t)pl.NT * 4);
   L.coef = off;
-  off += equal ? 0 : al256((size_t)pl.NT * pl.W_pad * 16);
+  off += equal ? 0 : al256((size_t)pl.NT * pl.W_pad * pl.U * 4);
   L.mono = off;
   off += (channels > 1 && !equal) ? al256((size_t)total_in * 4) : 0;
   L.total = off;
@@ -1221,7 +1221,7 @@ ae_status ae_resample(const float *d_x, int channels, int64_t ch_stride, const i
   if (channels < 1 || channels > kMaxChannels) return fail(AE_EINVAL, "channels must be in 1 .. 64");
   const RsPlan pl = rs_plan(rate_in, rate_out);
   const bool equal = rate_in == rate_out;
-  if (!equal && (int64_t)pl.NT * pl.W_pad * 4 > kMaxRsTable)
+  if (!equal && (int64_t)pl.NT * pl.W_pad * pl.U > kMaxRsTable)
     return fail(AE_EUNSUPPORTED, "the reduced output rate " + std::to_string(pl.p) + " needs a tap table above 2^26");
   RsTables T;
   if ((st = rs_tables(h_sample_off, n_clips, rate_in, rate_out, pl, T))) return st;
@@ -1254,7 +1254,7 @@ ae_status ae_resample(const float *d_x, int channels, int64_t ch_stride, const i
          return r;
        })) != cudaSuccess)
     return cuda_fail(e, "table upload");
-  if ((e = timed(AE_K_RESAMPLE, 0.0, 16.0 * pl.NT * pl.W_pad, s, [&] { return launch_rs_table(pl, coef, lo, s); })) !=
+  if ((e = timed(AE_K_RESAMPLE, 0.0, 4.0 * pl.U * pl.NT * pl.W_pad, s, [&] { return launch_rs_table(pl, coef, lo, s); })) !=
       cudaSuccess)
     return cuda_fail(e, "resampler taps");
   if (channels > 1) {

@@ -55,31 +55,35 @@ __device__ double rs_bessel_i0(double x) {
   return sum;
 }
 
-// One thread per (type T, offset i): the taps of outputs 4T + r, r = 0..3,
-// at input lo_T + i (relative to the unit's base q D), lo_T = floor(4 T o / p
-// - 64 / c). Output 4T + r sits at input position 4 T o / p + r o / p.
-__global__ void k_rs_table(float4 *__restrict__ coef, int32_t *__restrict__ lo, int o, int p, int NT, int W_pad,
+// One thread per (type T, offset i): the taps of outputs U T + r, r < U, at
+// input lo_T + i (relative to the unit's base q D), lo_T = floor(U T o / p -
+// 64 / c), stored as U / 4 float4. Output U T + r sits at input position
+// U T o / p + r o / p.
+__global__ void k_rs_table(float4 *__restrict__ coef, int32_t *__restrict__ lo, int U, int o, int p, int NT, int W_pad,
                            double c, double half, double i0b) {
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (int64_t)NT * W_pad) return;
   const int T = (int)(idx / W_pad), i = (int)(idx % W_pad);
-  const double frac = 4.0 * (double)T * (double)o / (double)p;
+  const double frac = (double)U * (double)T * (double)o / (double)p;
   const int l0 = (int)floor(frac - half);
   if (i == 0) lo[T] = l0;
-  double v[4];
+  for (int j = 0; j < U / 4; ++j) {
+    double v[4];
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const double t = ((double)(l0 + i) - frac - (double)r * (double)o / (double)p) * c;
-    v[r] = 0.0;
-    if (fabs(t) < kRsWidth) {
-      const double q = t / kRsWidth;
-      const double win = rs_bessel_i0(kRsBeta * sqrt(1.0 - q * q)) / i0b;
-      const double pt = M_PI * t;
-      const double sinc = pt == 0.0 ? 1.0 : sin(pt) / pt;
-      v[r] = sinc * win * c;
+    for (int k = 0; k < 4; ++k) {
+      const int r = 4 * j + k;
+      const double t = ((double)(l0 + i) - frac - (double)r * (double)o / (double)p) * c;
+      v[k] = 0.0;
+      if (fabs(t) < kRsWidth) {
+        const double q = t / kRsWidth;
+        const double win = rs_bessel_i0(kRsBeta * sqrt(1.0 - q * q)) / i0b;
+        const double pt = M_PI * t;
+        const double sinc = pt == 0.0 ? 1.0 : sin(pt) / pt;
+        v[k] = sinc * win * c;
+      }
     }
+    coef[idx * (U / 4) + j] = make_float4((float)v[0], (float)v[1], (float)v[2], (float)v[3]);
   }
-  coef[idx] = make_float4((float)v[0], (float)v[1], (float)v[2], (float)v[3]);
 }
 
 // mono[i] = (x_0[i] + ... + x_{C-1}[i]) / C in float32, channel order.
@@ -137,28 +141,36 @@ __device__ __forceinline__ void cp_async4(float *dst, const float *src, bool val
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
-// Partial FIR of one warp item over input offsets [i0, i1) (even, i1 - i0 a
-// multiple of 2) from staged taps and a staged input span: lane = unit, four
-// outputs per lane, two partial sums (even and odd offsets).
-__device__ __forceinline__ float4 rs_partial(const RsArgs &a, const RsTile &r, const float *span, const float4 *cT,
-                                             int T, int ql, int i0, int i1) {
+// Partial FIR of one warp item over input offsets [i0, i1) (both even) from
+// staged taps ([offset][U / 4] float4) and a staged input span: lane = unit,
+// U outputs per lane, two partial sums each (even and odd offsets).
+template <int U>
+__device__ __forceinline__ void rs_partial(const RsArgs &a, const RsTile &r, const float *span, const float4 *cT,
+                                           int T, int ql, int i0, int i1, float (&acc)[U]) {
+  constexpr int V = U / 4;
   const int64_t m0 = (r.q0 + ql) * a.D + a.lo[T];
   const float *xr = span + (m0 - r.base);
-  float4 e = make_float4(0.f, 0.f, 0.f, 0.f), d = e;
+  float e[U], d[U];
+#pragma unroll
+  for (int k = 0; k < U; ++k) e[k] = d[k] = 0.f;
 #pragma unroll 4
   for (int i = i0; i < i1; i += 2) {
-    const float4 w0 = cT[i], w1 = cT[i + 1];
     const float x0 = xr[i], x1 = xr[i + 1];
-    e.x = fmaf(w0.x, x0, e.x);
-    e.y = fmaf(w0.y, x0, e.y);
-    e.z = fmaf(w0.z, x0, e.z);
-    e.w = fmaf(w0.w, x0, e.w);
-    d.x = fmaf(w1.x, x1, d.x);
-    d.y = fmaf(w1.y, x1, d.y);
-    d.z = fmaf(w1.z, x1, d.z);
-    d.w = fmaf(w1.w, x1, d.w);
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      const float4 w0 = cT[i * V + j], w1 = cT[(i + 1) * V + j];
+      e[4 * j] = fmaf(w0.x, x0, e[4 * j]);
+      e[4 * j + 1] = fmaf(w0.y, x0, e[4 * j + 1]);
+      e[4 * j + 2] = fmaf(w0.z, x0, e[4 * j + 2]);
+      e[4 * j + 3] = fmaf(w0.w, x0, e[4 * j + 3]);
+      d[4 * j] = fmaf(w1.x, x1, d[4 * j]);
+      d[4 * j + 1] = fmaf(w1.y, x1, d[4 * j + 1]);
+      d[4 * j + 2] = fmaf(w1.z, x1, d[4 * j + 2]);
+      d[4 * j + 3] = fmaf(w1.w, x1, d[4 * j + 3]);
+    }
   }
-  return make_float4(e.x + d.x, e.y + d.y, e.z + d.z, e.w + d.w);
+#pragma unroll
+  for (int k = 0; k < U; ++k) acc[k] = e[k] + d[k];
 }
 
 // Persistent form, for plans whose group tap rows and two input spans fit in
@@ -167,21 +179,24 @@ __device__ __forceinline__ float4 rs_partial(const RsArgs &a, const RsTile &r, c
 // once; the input span of the next tile is copied asynchronously (4 bytes a
 // lane, coalesced, zero-filled outside the clip) while the current tile is
 // computed, so the copies hide behind the multiply-adds. Each (type, 32-unit)
-// item is split over two warps, one per half of the offset window, so that
-// 16 warps keep the shared-memory loads' latency covered; the second half's
-// sums meet the first's in shared memory.
+// item is split over PARTS warps, one per slice of the offset window, so that
+// 16 warps keep the shared-memory loads' latency covered; the other slices'
+// sums meet the first's in shared memory. With U = 8 outputs per unit a warp
+// loads two broadcast float4 of taps and one input sample per offset for
+// eight multiply-adds (U = 4: one and one for four).
 constexpr int kRsPipeThreads = 512;
-constexpr int kRsPipeItems = kRsWarps;  // items per tile: (Q / 32) x types of the group <= 8
 
+template <int U, int PARTS>
 __global__ void __launch_bounds__(kRsPipeThreads) k_rs_fir_pipe(const RsArgs a, int per) {
+  constexpr int V = U / 4, ITEMS = kRsPipeThreads / 32 / PARTS;
   extern __shared__ __align__(16) float rs_smem[];
   const int g = blockIdx.x % a.n_groups;
   int t = blockIdx.x / a.n_groups;
   if (t >= a.n_tiles) return;
   const int T0 = g * a.TG, n_types = min(a.TG, a.NT - T0);
-  float4 *cs = reinterpret_cast<float4 *>(rs_smem);                  // [TG][W_pad]
-  float4 *red = cs + a.TG * a.W_pad;                                  // [items][32]: second halves
-  float *buf0 = reinterpret_cast<float *>(red + kRsPipeItems * 32);  // two input spans
+  float4 *cs = reinterpret_cast<float4 *>(rs_smem);                        // [TG][W_pad][V]
+  float4 *red = cs + (int64_t)a.TG * a.W_pad * V;                           // [PARTS - 1][ITEMS][32][V]
+  float *buf0 = reinterpret_cast<float *>(red + (PARTS - 1) * ITEMS * 32 * V);  // two input spans
   auto stage = [&](int tile, float *dst) {
     const RsTile r = rs_tile(a, tile);
     const float *xin = a.x + r.in0;
@@ -194,13 +209,13 @@ __global__ void __launch_bounds__(kRsPipeThreads) k_rs_fir_pipe(const RsArgs a, 
   stage(t, buf0);
   cp_async_commit();
   {
-    const float4 *src = a.coef + (int64_t)T0 * a.W_pad;
-    for (int i = threadIdx.x; i < n_types * a.W_pad; i += kRsPipeThreads) cs[i] = __ldg(src + i);
+    const float4 *src = a.coef + (int64_t)T0 * a.W_pad * V;
+    for (int i = threadIdx.x; i < n_types * a.W_pad * V; i += kRsPipeThreads) cs[i] = __ldg(src + i);
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int items = (a.Q / 32) * n_types;
-  const int item = warp % kRsPipeItems, part = warp / kRsPipeItems;
-  const int hw = a.W_pad / 2;  // W_pad is a multiple of 8: both halves even
+  const int item = warp % ITEMS, part = warp / ITEMS;
+  const int pw = a.W_pad / PARTS;  // W_pad is a multiple of 8: every slice is even
   const int tl = item % n_types, ql = (item / n_types) * 32 + lane;
   for (int k = 0; t < a.n_tiles; ++k, t += per) {
     if (t + per < a.n_tiles) stage(t + per, buf0 + ((k + 1) & 1) * a.span);
@@ -208,21 +223,34 @@ __global__ void __launch_bounds__(kRsPipeThreads) k_rs_fir_pipe(const RsArgs a, 
     cp_async_wait_1();  // this tile's span has landed (this thread's copies)
     __syncthreads();    // ... and every thread's
     const RsTile r = rs_tile(a, t);
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    float acc[U];
     if (item < items) {
-      v = rs_partial(a, r, buf0 + (k & 1) * a.span, cs + (int64_t)tl * a.W_pad, T0 + tl, ql, part * hw,
-                     (part + 1) * hw);
-      if (part == 1) red[item * 32 + lane] = v;
+      rs_partial<U>(a, r, buf0 + (k & 1) * a.span, cs + (int64_t)tl * a.W_pad * V, T0 + tl, ql, part * pw,
+                    (part + 1) * pw, acc);
+      if (part > 0) {
+        float4 *dst = red + (((part - 1) * ITEMS + item) * 32 + lane) * V;
+#pragma unroll
+        for (int j = 0; j < V; ++j) dst[j] = make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
+      }
     }
     __syncthreads();
     if (item < items && part == 0) {
-      const float4 u = red[item * 32 + lane];
-      const float r4[4] = {v.x + u.x, v.y + u.y, v.z + u.z, v.w + u.w};
-      const int T = T0 + tl;
-      const int64_t n0 = ((r.q0 + ql) * a.NT + T) * 4;  // first output of the unit
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (n0 + j < r.n_out) a.y[r.out0 + n0 + j] = r4[j];
+      for (int q = 1; q < PARTS; ++q) {
+        const float4 *src = red + (((q - 1) * ITEMS + item) * 32 + lane) * V;
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+          const float4 u = src[j];
+          acc[4 * j] += u.x;
+          acc[4 * j + 1] += u.y;
+          acc[4 * j + 2] += u.z;
+          acc[4 * j + 3] += u.w;
+        }
+      }
+      const int64_t n0 = ((r.q0 + ql) * a.NT + T0 + tl) * U;  // first output of the unit
+#pragma unroll
+      for (int j = 0; j < U; ++j)
+        if (n0 + j < r.n_out) a.y[r.out0 + n0 + j] = acc[j];
     }
     __syncthreads();  // the span buffer is refilled and red rewritten on the next tiles
   }
@@ -320,8 +348,13 @@ int64_t rs_len(int64_t n, int rate_in, int rate_out) {
   return (p * n + o - 1) / o;
 }
 
-RsPlan rs_plan(int rate_in, int rate_out) {
+// The plan for units of U outputs; `items` caps the (type, 32-unit) items of
+// a tile (the warps of the per-tile form, or 16 warps / parts in the
+// persistent form).
+static RsPlan rs_plan_u(int rate_in, int rate_out, int U, int items, int parts) {
   RsPlan pl;
+  pl.U = U;
+  pl.parts = parts;
   int64_t a = rate_in, b = rate_out;
   while (b) {
     const int64_t t = a % b;
@@ -332,22 +365,23 @@ RsPlan rs_plan(int rate_in, int rate_out) {
   pl.p = (int)(rate_out / a);
   pl.c = kRsRolloff * (double)std::min(pl.o, pl.p) / (double)pl.o;
   pl.half = kRsWidth / pl.c;
-  const int g4 = pl.p % 4 == 0 ? 4 : (pl.p % 2 == 0 ? 2 : 1);  // gcd(p, 4)
-  pl.NT = pl.p / g4;
-  pl.D = (int)(4 * (int64_t)pl.o / g4);
-  // a unit's four outputs span 3 o / p input samples; each reaches half to either side
-  pl.W = (int)std::ceil(2.0 * pl.half + 3.0 * pl.o / pl.p) + 3;
+  int gu = U;  // gcd(p, U), U a power of two
+  while (pl.p % gu) gu /= 2;
+  pl.NT = pl.p / gu;
+  pl.D = (int)((int64_t)U * pl.o / gu);
+  // a unit's U outputs span (U - 1) o / p input samples; each reaches half to either side
+  pl.W = (int)std::ceil(2.0 * pl.half + (double)(U - 1) * pl.o / pl.p) + 3;
   pl.W_pad = (pl.W + 7) & ~7;
   pl.lo_min = (int)std::floor(-pl.half) - 1;  // <= lo_T for every type
-  // a tile: Q units of each of (up to) TG types; enough (type, 32-unit group)
-  // items for the CTA's warps; the staged input span and the group's tap rows
+  // a tile: Q units of each of (up to) TG types, at most `items` (type,
+  // 32-unit group) items; the staged input span and the group's tap rows
   // within the shared-memory budget
-  pl.TG = std::min(pl.NT, kRsWarps);
+  pl.TG = std::min(pl.NT, items);
   pl.n_groups = (pl.NT + pl.TG - 1) / pl.TG;
-  int groups = std::max(1, kRsWarps / pl.TG);
-  // lo_T < 4 T o / p <= D - 4 o / p, so offsets stay below Q D + W_pad - lo_min
+  int groups = std::max(1, items / pl.TG);
+  // lo_T < U T o / p <= D - U o / p, so offsets stay below Q D + W_pad - lo_min
   auto span_of = [&](int q) -> int64_t { return (int64_t)q * pl.D + pl.W_pad - pl.lo_min + 2; };
-  const int64_t coef_bytes = 16 * (int64_t)pl.TG * pl.W_pad;
+  const int64_t coef_bytes = 4 * (int64_t)U * pl.TG * pl.W_pad;
   while (groups > 1 && 4 * span_of(32 * groups) + coef_bytes > (int64_t)kRsSmemMax) groups /= 2;
   pl.Q = 32 * groups;
   pl.stage_coef = coef_bytes <= (int64_t)kRsSmemMax / 2;
@@ -355,10 +389,19 @@ RsPlan rs_plan(int rate_in, int rate_out) {
   pl.span = span_b + (pl.stage_coef ? coef_bytes : 0) <= (int64_t)kRsSmemMax ? (int)span_of(pl.Q) : 0;
   pl.span = (pl.span + 3) & ~3;  // the tap rows that follow stay 16-byte aligned
   pl.smem = 4 * (size_t)pl.span + (pl.stage_coef ? (size_t)coef_bytes : 0);
-  // the persistent form keeps the tap rows, the second halves' sums and two input spans
-  pl.smem_pipe = 8 * (size_t)pl.span + (size_t)coef_bytes + 16 * 32 * (size_t)kRsWarps;
+  // the persistent form keeps the tap rows, the other slices' sums and two input spans
+  const size_t red_bytes = 4 * (size_t)U * 32 * (size_t)(kRsPipeThreads / 32 / parts) * (size_t)(parts - 1);
+  pl.smem_pipe = 8 * (size_t)pl.span + (size_t)coef_bytes + red_bytes;
   pl.pipe = pl.stage_coef && pl.span > 0 && pl.smem_pipe <= kRsPipeSmemMax;
   return pl;
+}
+
+RsPlan rs_plan(int rate_in, int rate_out) {
+  // eight outputs per unit in the persistent form when it fits (4 items of
+  // 4 warps each), else four (8 items of 2 warps, or the per-tile form)
+  const RsPlan p8 = rs_plan_u(rate_in, rate_out, 8, 4, 4);
+  if (p8.pipe) return p8;
+  return rs_plan_u(rate_in, rate_out, 4, kRsWarps, 2);
 }
 
 cudaError_t launch_rs_table(const RsPlan &pl, float *coef, int32_t *lo, cudaStream_t s) {
@@ -373,7 +416,7 @@ cudaError_t launch_rs_table(const RsPlan &pl, float *coef, int32_t *lo, cudaStre
     return sum;
   }();
   return launch_k(k_rs_table, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, reinterpret_cast<float4 *>(coef),
-                  lo, pl.o, pl.p, pl.NT, pl.W_pad, pl.c, pl.half, i0b);
+                  lo, pl.U, pl.o, pl.p, pl.NT, pl.W_pad, pl.c, pl.half, i0b);
 }
 
 cudaError_t launch_rs_mix(const float *x, int channels, int64_t ch_stride, int64_t n, float *mono, cudaStream_t s) {
@@ -406,20 +449,19 @@ cudaError_t launch_rs_fir(const RsPlan &pl, const float *mono, float *y, const f
   a.stage_coef = pl.stage_coef ? 1 : 0;
   a.n_tiles = n_tiles;
   if (pl.pipe) {
-    cudaError_t e = cudaFuncSetAttribute(k_rs_fir_pipe, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)pl.smem_pipe);
+    auto kern = pl.U == 8 ? k_rs_fir_pipe<8, 4> : k_rs_fir_pipe<4, 2>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem_pipe);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0, per_sm = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_rs_fir_pipe, kRsPipeThreads,
-                                                           pl.smem_pipe)) != cudaSuccess)
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kRsPipeThreads, pl.smem_pipe)) !=
+        cudaSuccess)
       return e;
     // CTAs per type group: every resident slot busy, but no more than the tiles
     const int per = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)sms * std::max(per_sm, 1) / pl.n_groups,
                                                                  n_tiles));
-    return launch_k(k_rs_fir_pipe, dim3((unsigned)(per * pl.n_groups)), dim3(kRsPipeThreads), pl.smem_pipe, s, a,
-                    per);
+    return launch_k(kern, dim3((unsigned)(per * pl.n_groups)), dim3(kRsPipeThreads), pl.smem_pipe, s, a, per);
   }
   if (pl.smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(k_rs_fir, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRsSmemMax);
