@@ -102,13 +102,12 @@ __device__ __forceinline__ float2 mul_sigmoid2(float2 c, float2 g) {
   return __fmul2_rn(c, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
 }
 
-// Epilogue of 32 accumulator columns [col, col + 32) of one row, written as
-// granules g0, g0 + 1, ... of the row's staging line: 8 granules of f32
-// (EPI_F32), 4 of bf16 (EPI_BF16, EPI_SILU), 2 of bf16 (EPI_GLU, which pairs
-// columns (2c, 2c + 1) into output column c).
-template <int MODE, bool SC>
-__device__ __forceinline__ void epi_stage(const EpiArgs &ep, int col, const uint32_t (&r)[32], uint8_t *line, int r7,
-                                          int g0) {
+// Float32 epilogue (EPI_F32, EPI_ADD_F32) of 32 accumulator columns [col,
+// col + 32) of one row: clamp (after the bias for EPI_F32), written as the 8
+// granules g0 .. g0 + 7 of the row's staging line.
+template <bool SC>
+__device__ __forceinline__ void epi_stage_f32(const EpiArgs &ep, bool bias, int col, const uint32_t (&r)[32],
+                                              uint8_t *line, int r7, int g0) {
   float lo = ep.lo, hi = ep.hi;
   if (ep.seg_w > 0) {
     const int sg = col / ep.seg_w;  // selects, not a runtime index into the parameter array
@@ -119,42 +118,16 @@ __device__ __forceinline__ void epi_stage(const EpiArgs &ep, int col, const uint
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
   if (SC) scale_cols(ep.cs + col, v);
-  if (MODE == EPI_F32 || MODE == EPI_ADD_F32) {
-    if (MODE == EPI_F32 && ep.bias) {
+  if (bias) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] += __ldg(ep.bias + col + i);
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      st_granule(line, r7, g0 + j,
-                 make_uint4(__float_as_uint(clampf(v[4 * j], lo, hi)), __float_as_uint(clampf(v[4 * j + 1], lo, hi)),
-                            __float_as_uint(clampf(v[4 * j + 2], lo, hi)),
-                            __float_as_uint(clampf(v[4 * j + 3], lo, hi))));
-  } else if (MODE == EPI_GLU) {
-    // a * sigmoid(b) = a / (1 + e^-b): fast exp and reciprocal (2 ulp each; the
-    // bf16 rounding of the result is 2^-9), with the right limits at +-inf
-    uint32_t p[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      float a0 = clampf(v[4 * j + 0], lo, hi), b0 = clampf(v[4 * j + 1], lo, hi);
-      float a1 = clampf(v[4 * j + 2], lo, hi), b1 = clampf(v[4 * j + 3], lo, hi);
-      p[j] = pack_bf16(__fdividef(a0, 1.0f + __expf(-b0)), __fdividef(a1, 1.0f + __expf(-b1)));
-    }
-    st_granule(line, r7, g0, make_uint4(p[0], p[1], p[2], p[3]));
-    st_granule(line, r7, g0 + 1, make_uint4(p[4], p[5], p[6], p[7]));
-  } else {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      float x = clampf(v[i], lo, hi);
-      if (MODE == EPI_SILU) x = clampf(__fdividef(x, 1.0f + __expf(-x)), ep.lo2, ep.hi2);
-      v[i] = x;
-    }
-    uint32_t p[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) p[j] = pack_bf16(v[2 * j], v[2 * j + 1]);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) st_granule(line, r7, g0 + j, make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]));
+    for (int i = 0; i < 32; ++i) v[i] += __ldg(ep.bias + col + i);
   }
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    st_granule(line, r7, g0 + j,
+               make_uint4(__float_as_uint(clampf(v[4 * j], lo, hi)), __float_as_uint(clampf(v[4 * j + 1], lo, hi)),
+                          __float_as_uint(clampf(v[4 * j + 2], lo, hi)),
+                          __float_as_uint(clampf(v[4 * j + 3], lo, hi))));
 }
 
 __device__ __forceinline__ void st_global_32B(void *p, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t a4,
@@ -166,7 +139,8 @@ __device__ __forceinline__ void st_global_32B(void *p, uint32_t a0, uint32_t a1,
 }
 
 // Epilogue of 32 accumulator columns of one row, stored from registers as
-// whole 32-byte sectors (the bf16 outputs; f32 outputs go through epi_stage).
+// whole 32-byte sectors (bf16 and e4m3 outputs; float32 outputs go through
+// epi_stage_f32).
 template <int MODE, bool SC>
 __device__ __forceinline__ void epi_store32(const EpiArgs &ep, int row, int col, const uint32_t (&r)[32]) {
   float lo = ep.lo, hi = ep.hi;
@@ -179,19 +153,8 @@ __device__ __forceinline__ void epi_store32(const EpiArgs &ep, int row, int col,
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
   if (SC) scale_cols(ep.cs + col, v);
-  if (MODE == EPI_F32) {
-    if (ep.bias) {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] += __ldg(ep.bias + col + i);
-    }
-    float *o = static_cast<float *>(ep.out) + (int64_t)row * ep.ld + col;
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      st_global_32B(o + 8 * j, __float_as_uint(clampf(v[8 * j], lo, hi)), __float_as_uint(clampf(v[8 * j + 1], lo, hi)),
-                    __float_as_uint(clampf(v[8 * j + 2], lo, hi)), __float_as_uint(clampf(v[8 * j + 3], lo, hi)),
-                    __float_as_uint(clampf(v[8 * j + 4], lo, hi)), __float_as_uint(clampf(v[8 * j + 5], lo, hi)),
-                    __float_as_uint(clampf(v[8 * j + 6], lo, hi)), __float_as_uint(clampf(v[8 * j + 7], lo, hi)));
-  } else if (MODE == EPI_GLU) {
+  static_assert(MODE != EPI_F32 && MODE != EPI_ADD_F32, "float32 outputs go through the staging boxes");
+  if (MODE == EPI_GLU) {
     uint32_t p[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {  // columns (4j, 4j+1, 4j+2, 4j+3) = (a, b, a, b)
@@ -414,10 +377,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     // full 128-byte row segments per store instruction (measured faster for
     // f32, slower for bf16, than the direct sector stores).
     constexpr bool F32_OUT = MODE == EPI_F32 || MODE == EPI_ADD_F32;
-    constexpr int LOADS_PER_BOX = F32_OUT ? 1 : (MODE == EPI_GLU ? 4 : 2);  // 32-column TMEM loads
-    constexpr int OUT_COLS_PER_BOX = F32_OUT ? 32 : 64;                     // 128 bytes of output
-    constexpr int GRANULES_PER_LOAD = 8 / LOADS_PER_BOX;
-    constexpr int ES = F32_OUT ? 4 : 2;
+    // float32 staging: one 32-column TMEM load fills a box row (128 bytes)
+    constexpr int LOADS_PER_BOX = 1, OUT_COLS_PER_BOX = 32, GRANULES_PER_LOAD = 8, ES = 4;
     const int q = warp & 3, half = (warp - 2) >> 2;
     uint8_t *box = epi_smem + (warp - 2) * LINE_BYTES;
     const uint32_t tempty_leader = map_to_rank(&tempty[0], 0);
@@ -437,33 +398,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       const int ocol0 = MODE == EPI_GLU ? col0 / 2 : col0;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + half * (BN / 2));
       auto stage = [&](int c, const uint32_t(&r)[32]) {
-        if (!F32_OUT) {  // bf16 rows: 32-byte stores straight from registers
+        if constexpr (!F32_OUT) {  // bf16 / e4m3 rows: 32-byte stores straight from registers
           if (row0 + lane < M) epi_store32<MODE, F8>(ep, row0 + lane, col0 + c * 32, r);
-          return;
-        }
-        const int j = c % LOADS_PER_BOX;
-        epi_stage<MODE, F8>(ep, col0 + c * 32, r, box + lane * 128, lane & 7, j * GRANULES_PER_LOAD);
-        if (j == LOADS_PER_BOX - 1) {
-          __syncwarp();
-          // lane l moves granule l % 8 of rows l / 8, l / 8 + 4, ...
-          const int g = lane & 7;
-          uint8_t *dst = static_cast<uint8_t *>(ep.out) +
-                         ((int64_t)ocol0 + (c / LOADS_PER_BOX) * OUT_COLS_PER_BOX) * ES + g * 16;
+        } else {
+          const int j = c % LOADS_PER_BOX;
+          epi_stage_f32<F8>(ep, MODE == EPI_F32 && ep.bias, col0 + c * 32, r, box + lane * 128, lane & 7,
+                            j * GRANULES_PER_LOAD);
+          if (j == LOADS_PER_BOX - 1) {
+            __syncwarp();
+            // lane l moves granule l % 8 of rows l / 8, l / 8 + 4, ...
+            const int g = lane & 7;
+            uint8_t *dst = static_cast<uint8_t *>(ep.out) +
+                           ((int64_t)ocol0 + (c / LOADS_PER_BOX) * OUT_COLS_PER_BOX) * ES + g * 16;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int rr = (lane >> 3) + 4 * i;
-            const uint4 v = *reinterpret_cast<const uint4 *>(box + rr * 128 + ((g ^ (rr & 7)) << 4));
-            if (row0 + rr < M) {
-              uint8_t *p = dst + (int64_t)(row0 + rr) * ep.ld * ES;
-              if (MODE == EPI_ADD_F32)  // one vector add per 4 elements; no other thread touches them
-                asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(__uint_as_float(v.x)),
-                             "f"(__uint_as_float(v.y)), "f"(__uint_as_float(v.z)), "f"(__uint_as_float(v.w))
-                             : "memory");
-              else
-                *reinterpret_cast<uint4 *>(p) = v;
+            for (int i = 0; i < 8; ++i) {
+              const int rr = (lane >> 3) + 4 * i;
+              const uint4 v = *reinterpret_cast<const uint4 *>(box + rr * 128 + ((g ^ (rr & 7)) << 4));
+              if (row0 + rr < M) {
+                uint8_t *p = dst + (int64_t)(row0 + rr) * ep.ld * ES;
+                if (MODE == EPI_ADD_F32)  // one vector add per 4 elements; no other thread touches them
+                  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(__uint_as_float(v.x)),
+                               "f"(__uint_as_float(v.y)), "f"(__uint_as_float(v.z)), "f"(__uint_as_float(v.w))
+                               : "memory");
+                else
+                  *reinterpret_cast<uint4 *>(p) = v;
+              }
             }
+            __syncwarp();
           }
-          __syncwarp();
         }
       };
       // two register buffers: the next chunk's tcgen05.ld is in flight during the math
