@@ -2,7 +2,7 @@
 """Throughput of the B200 audio-encoder forward.
 
     python bench.py [--gpus N] [--steps K] [--warmup W]
-                    [--workload tower|tower_fp8|ragged|frontend|attention|resample]
+                    [--workload tower|tower_fp8|ragged|frontend|lfm_frontend|attention|resample]
     python bench.py --impl reference ...      # the CPU oracle on the same workload (bounded sample)
 
 A step is one ae_encode over one batch (default: 16 clips x 30 s, the
@@ -153,6 +153,8 @@ def workload_desc(name: str, info: dict) -> dict:
                          "projections bf16; f32 accumulation",
             "ragged": "256 clips of 1-30 s (uniform whole samples), packed, 12 layers + head, bf16",
             "frontend": "log-mel front-end only, 64 clips x 30 s, f32",
+            "lfm_frontend": "second (LFM2A) log-mel front-end: pre-emphasis, centre padding, power spectrum, Slaney "
+                            "bank, per-band normalisation; 64 clips x 30 s, f32",
             "attention": "local-attention core only, 32 x 8192 tokens, 8 heads x 128, bf16 q/k/v",
             "resample": "mixdown + Kaiser-sinc resampling to 16 kHz, 64 stereo clips x 30 s at 44.1 kHz, f32"}[name]
     d = {"workload": f"{name}: {base}", "l2": "flushed between steps (256 MiB write)",
@@ -165,8 +167,9 @@ ENCODE_WORKLOADS = ("tower", "tower_fp8", "ragged")
 
 
 def data_of(name: str) -> str:
-    """The synthetic batch a workload runs on (the e4m3 tower runs the tower's)."""
-    return "tower" if name == "tower_fp8" else name
+    """The synthetic batch a workload runs on (the e4m3 tower runs the tower's,
+    the second front-end the first one's)."""
+    return {"tower_fp8": "tower", "lfm_frontend": "frontend"}.get(name, name)
 
 
 class Ours:
@@ -175,7 +178,7 @@ class Ours:
         import log_mel_front_b200 as ae
         self.ae, self.torch, self.name = ae, torch, name
         self.stream = torch.cuda.current_stream()
-        if name in ENCODE_WORKLOADS + ("frontend",):
+        if name in ENCODE_WORKLOADS + ("frontend", "lfm_frontend"):
             self.lens = synth.clip_lengths(data_of(name))
             clips = synth.waves(data_of(name))
             flat, self.off = synth.pack(clips)
@@ -192,6 +195,14 @@ class Ours:
             self.ws_host_bytes = ae.ae_encode_host_workspace_size(self.model, self.off)
             self.ws = torch.empty(max(self.ws_bytes, self.ws_host_bytes), dtype=torch.uint8, device="cuda")
             self.dominant = "gemm_fp8" if name == "tower_fp8" else "gemm"
+        elif name == "lfm_frontend":
+            self.cfg = ae.lfm_config()
+            self.frames = sum(ae.ae_lfm_num_frames(self.cfg, n) for n in self.lens)
+            self.ws_bytes = ae.ae_lfm_workspace_size(self.cfg, len(self.lens))
+            self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
+            self.d_mel = torch.empty((self.frames, self.cfg.n_mels), device="cuda")
+            self.h_mel = torch.empty((self.frames, self.cfg.n_mels)).pin_memory()
+            self.dominant = "lfm"
         elif name == "frontend":
             self.ws_bytes = ae.ae_workspace_size(None, len(self.lens), self.frames, 0)
             self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
@@ -240,6 +251,8 @@ class Ours:
             ae.ae_encode(self.model, self.d_wave, self.off, self.d_out, self.ws, self.ws_bytes, self.stream)
         elif self.name == "frontend":
             ae.ae_logmel(self.d_wave, self.off, self.d_mel, self.ws, self.ws_bytes, self.stream)
+        elif self.name == "lfm_frontend":
+            ae.ae_lfm_logmel(self.cfg, self.d_wave, self.off, self.d_mel, self.ws, self.ws_bytes, self.stream)
         elif self.name == "resample":
             ae.ae_resample(self.d_x, 2, self.d_x.shape[1], self.off, synth.RS_RATE, 16000, self.d_y, self.ws,
                            self.ws_bytes, self.stream)
@@ -253,7 +266,7 @@ class Ours:
         if self.name in ENCODE_WORKLOADS:
             ae.ae_encode_host(self.model, self.h_wave, self.off, self.h_out, self.ws, self.ws.numel(), self.stream)
             return self.h_wave.numel() * 4, self.h_out.numel() * 4
-        if self.name == "frontend":
+        if self.name in ("frontend", "lfm_frontend"):
             self.d_wave.copy_(self.h_wave, non_blocking=True)
             self.step()
             self.h_mel.copy_(self.d_mel, non_blocking=True)
@@ -348,6 +361,12 @@ class OracleRun:
             t0 = time.perf_counter()
             O.log_mel(c)
             return time.perf_counter() - t0, 30.0, "clip 0 of the frontend workload (log-mel)"
+        if self.name == "lfm_frontend":
+            from oracle import lfm as LF
+            c = synth.waves("frontend", [0])[0]
+            t0 = time.perf_counter()
+            LF.features(c)
+            return time.perf_counter() - t0, 30.0, "clip 0 of the frontend workload (second front-end)"
         if self.name == "resample":
             i = self.next % synth.RS_CLIPS
             self.next += 1
@@ -467,6 +486,7 @@ def run_ours(args, rank, world, dist):
         roof = {"bound": "hbm", "unit": "GB/s", "peak_kind": "HBM copy (" + pk["source"] + ")"}
     traffic, traffic_src = captured_traffic(ours.dominant)
     roof.update({"kernel": {"gemm": "k_gemm_tc (all projections)", "logmel": "k_logmel",
+                            "lfm": "k_lfm_spec + k_lfm_norm",
                             "gemm_fp8": "k_gemm_tc<e4m3> (FFN W1/W2, q/k/v, lc_start)",
                             "attention": "k_attention_tc",
                             "resample": "k_rs_fir (with its tap table and mixdown)"}[ours.dominant],
@@ -483,7 +503,8 @@ def run_ours(args, rank, world, dist):
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(per_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None,
-        "dtype": {"frontend": "f32", "resample": "f32", "tower_fp8": "e4m3+bf16"}.get(args.workload, "bf16"),
+        "dtype": {"frontend": "f32", "lfm_frontend": "f32", "resample": "f32",
+                  "tower_fp8": "e4m3+bf16"}.get(args.workload, "bf16"),
         "data": "synthetic",
         "config": workload_desc(args.workload, {
             "clips": len(getattr(ours, "lens", [])) or synth.ATT_SEQS,
@@ -498,7 +519,8 @@ def run_ours(args, rank, world, dist):
                     "tower_fp8": "ae_encode_host_async, two streams (copies of one step overlap the kernels of the "
                                  "other)",
                     "ragged": "ae_encode_host_async, two streams (copies of one step overlap the kernels of the other)",
-                    "frontend": "ae_logmel + copies", "resample": "ae_resample + copies"}[args.workload]},
+                    "frontend": "ae_logmel + copies", "lfm_frontend": "ae_lfm_logmel + copies",
+                    "resample": "ae_resample + copies"}[args.workload]},
         "gpu_launches": int(round(launches / prof_steps * args.steps)),
         "roofline": roof,
         "kernel_classes": classes,
@@ -539,7 +561,8 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", choices=("tower", "tower_fp8", "ragged", "frontend", "attention", "resample"),
+    ap.add_argument("--workload", choices=("tower", "tower_fp8", "ragged", "frontend", "lfm_frontend", "attention",
+                                           "resample"),
                     default="tower")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

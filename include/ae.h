@@ -294,6 +294,48 @@ ae_status ae_linear_e4m3(const void *d_x, const void *d_w, const float *d_cs, in
 ae_status ae_logmel_noalloc(const float *d_wave, const int64_t *h_sample_off, int n_clips, float *d_mel,
                             ae_stream stream);
 
+/* --- second log-mel front-end (LFM2A) ------------------------------------------- */
+
+/* The front-end of the LFM2A audio encoder as the page of its GPU port lays it
+ * out (log_mel_spectrogram_gpu: stft_frames, power_spec, mel_project,
+ * mel_norm): frames of n_fft samples every hop samples with n_fft / 2 samples
+ * of zero padding per side (1 + N / hop frames for N > 0 samples, none for
+ * N = 0); pre-emphasis y[n] = x[n] - preemph x[n-1] on the clip (x[-1] = 0);
+ * a periodic Hann window of win_length samples centred in the n_fft-wide
+ * frame; the power spectrum |X_k|^2, k = 0 .. n_fft / 2; a Slaney mel
+ * filterbank (librosa's default: Slaney scale, points evenly spaced from 0 to
+ * sample_rate / 2, triangles scaled by 2 / (f_{b+2} - f_b)); ln(max(mel,
+ * log_floor)); then per band (v - mean) / sqrt(var + var_eps) with the mean
+ * and biased variance of the first ceil(N / hop) frames (those whose centre
+ * lies in the clip) and zeros for the rest. The page names these constants
+ * but gives no values; ae_lfm_default_config fills in the ones this library
+ * takes (16 kHz, n_fft 512, window 400, hop 160, 128 bands, pre-emphasis
+ * 0.97, floor 2^-24, variance epsilon 1e-5). */
+typedef struct {
+  int32_t sample_rate, n_fft, win_length, hop, n_mels;
+  float preemph, log_floor, var_eps;
+} ae_lfm_config;
+
+void ae_lfm_default_config(ae_lfm_config *cfg);
+
+/* Frames of a clip of n samples: 1 + n / hop for n > 0, else 0 (-1 for an
+ * invalid cfg). */
+int64_t ae_lfm_num_frames(const ae_lfm_config *cfg, int64_t n_samples);
+
+/* Workspace bytes of ae_lfm_logmel for n_clips clips (0 for an invalid cfg). */
+size_t ae_lfm_workspace_size(const ae_lfm_config *cfg, int n_clips);
+
+/* d_wave: packed float32 clips (device), clip i = [h_sample_off[i],
+ * h_sample_off[i+1]); d_out: [total frames][n_mels] float32, time-major,
+ * clips back to back (16-byte aligned). Supported: n_fft 512; win_length and
+ * hop even, 2 <= win_length <= 512, 2 <= hop <= 320; 1 <= n_mels <= 128 with
+ * at most 32 nonzero bins per band; sample_rate in [1000, 1000000];
+ * log_floor > 0, var_eps >= 0, all finite (AE_EINVAL or AE_EUNSUPPORTED
+ * otherwise, before anything is enqueued). At most 2^31 - 1 frames in all.
+ * Asynchronous on `stream`; no allocation. */
+ae_status ae_lfm_logmel(const ae_lfm_config *cfg, const float *d_wave, const int64_t *h_sample_off, int n_clips,
+                        float *d_out, void *d_ws, size_t ws_bytes, ae_stream stream);
+
 /* --- input conditioning: mixdown and resampling -------------------------------- */
 
 /* Output length of ae_resample for one clip of n_samples at rate_in:
@@ -349,7 +391,8 @@ typedef enum {
   AE_K_ROWOP = 7,    /* residual / RMS-norm row passes */
   AE_K_RESAMPLE = 8, /* mixdown, resampler taps and FIR */
   AE_K_GEMM_FP8 = 9, /* the e4m3 projections of AE_FP8 (tcgen05 kind::f8f6f4) */
-  AE_K_COUNT = 10
+  AE_K_LFM = 10,     /* the second log-mel front-end (spectrum, bands, normalisation) */
+  AE_K_COUNT = 11
 } ae_kernel_class;
 
 /* Kernel timing for measurement (the analogue of the page's

@@ -32,6 +32,11 @@ _fp = C.POINTER(C.c_float)
 _i64p = C.POINTER(C.c_int64)
 
 
+class ae_lfm_config(C.Structure):
+    _fields_ = [("sample_rate", C.c_int32), ("n_fft", C.c_int32), ("win_length", C.c_int32), ("hop", C.c_int32),
+                ("n_mels", C.c_int32), ("preemph", C.c_float), ("log_floor", C.c_float), ("var_eps", C.c_float)]
+
+
 class ae_config(C.Structure):
     _fields_ = [(n, C.c_int32) for n in ("n_mels", "c0", "c1", "hidden", "heads", "ffn", "left", "kernel",
                                         "out_dim", "embed_dim", "n_layers")] + \
@@ -93,19 +98,24 @@ _sig("ae_resample", _st, _vp, _i32, C.c_int64, _i64p, _i32, C.c_int32, C.c_int32
 _sig("ae_linear_e4m3", _st, _vp, _vp, _vp, C.c_int64, C.c_int32, C.c_int32, C.c_float, C.c_float, _i32, C.c_float,
      C.c_float, C.c_float, _vp, _vp)
 _sig("ae_selftest_bounded_wait", _st, C.c_uint32, _i32, _vp)
+_sig("ae_lfm_default_config", None, C.POINTER(ae_lfm_config))
+_sig("ae_lfm_num_frames", C.c_int64, C.POINTER(ae_lfm_config), C.c_int64)
+_sig("ae_lfm_workspace_size", _sz, C.POINTER(ae_lfm_config), _i32)
+_sig("ae_lfm_logmel", _st, C.POINTER(ae_lfm_config), _vp, _i64p, _i32, _vp, _vp, _sz, _vp)
 _sig("ae_profile_enable", _st, _i32)
 _sig("ae_profile_read", _st, C.POINTER(C.c_double), _i64p, C.POINTER(C.c_double), C.POINTER(C.c_double), _i64p)
 
 # every symbol include/ae.h declares
 EXPORTS = ("ae_num_frames", "ae_num_tokens", "ae_model_create", "ae_model_destroy", "ae_workspace_size",
            "ae_logmel", "ae_subsample", "ae_conformer_layer", "ae_encode", "ae_encode_host_workspace_size",
-           "ae_encode_host", "ae_encode_host_async", "ae_attention_tables", "ae_local_attention", "ae_last_error", "ae_device_status",
-           "ae_version", "ae_profile_enable", "ae_profile_read", "ae_logmel_noalloc", "ae_resample_len",
-           "ae_resample_workspace_size", "ae_resample", "ae_linear_e4m3",
-           "ae_selftest_bounded_wait")
+           "ae_encode_host", "ae_encode_host_async", "ae_attention_tables", "ae_local_attention", "ae_last_error",
+           "ae_device_status", "ae_version", "ae_profile_enable", "ae_profile_read", "ae_logmel_noalloc",
+           "ae_resample_len", "ae_resample_workspace_size", "ae_resample", "ae_linear_e4m3",
+           "ae_selftest_bounded_wait", "ae_lfm_default_config", "ae_lfm_num_frames", "ae_lfm_workspace_size",
+           "ae_lfm_logmel")
 
 KERNEL_CLASSES = ("tables", "logmel", "conv0", "conv1", "gemm", "attention", "lconv", "rowop", "resample",
-                  "gemm_fp8")
+                  "gemm_fp8", "lfm")
 
 
 class AEError(RuntimeError):
@@ -242,6 +252,29 @@ def ae_linear_e4m3(d_x, d_w, d_cs, M: int, N: int, K: int, lo: float, hi: float,
 
 def ae_device_status() -> int:
     return lib.ae_device_status()
+
+
+def lfm_config(**kw) -> "ae_lfm_config":
+    """The library's defaults (ae_lfm_default_config) with the given fields replaced."""
+    c = ae_lfm_config()
+    lib.ae_lfm_default_config(C.byref(c))
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+def ae_lfm_num_frames(cfg, n_samples: int) -> int:
+    return lib.ae_lfm_num_frames(C.byref(cfg), int(n_samples))
+
+
+def ae_lfm_workspace_size(cfg, n_clips: int) -> int:
+    return lib.ae_lfm_workspace_size(C.byref(cfg), int(n_clips))
+
+
+def ae_lfm_logmel(cfg, d_wave, sample_off, d_out, d_ws, ws_bytes: int, stream=None):
+    a, p = _off(sample_off)
+    _check(lib.ae_lfm_logmel(C.byref(cfg), _ptr(d_wave), p, len(a) - 1, _ptr(d_out), _ptr(d_ws), ws_bytes,
+                             _stream(stream)), "ae_lfm_logmel")
 
 
 def ae_selftest_bounded_wait(limit_us: int, arrive: bool = False, stream=None):

@@ -16,8 +16,8 @@ CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libae.so")
 ROOT = os.path.dirname(HERE)
-SOURCES = ["api.cu", "gemm.cu", "logmel.cu", "stem.cu", "attention.cu", "rowops.cu", "resample.cu"]
-HEADERS = ["common.cuh", "ae_internal.h"]
+SOURCES = ["api.cu", "gemm.cu", "logmel.cu", "stem.cu", "attention.cu", "rowops.cu", "resample.cu", "lfm.cu"]
+HEADERS = ["common.cuh", "ae_internal.h", "fft16.cuh"]
 
 NVCC = os.environ.get("NVCC", "nvcc")
 FLAGS = [

@@ -229,6 +229,27 @@ cudaError_t launch_rs_fir(const RsPlan &pl, const float *mono, float *y, const f
 // as kernel parameters), so the call stays asynchronous and capturable.
 cudaError_t launch_upload_bytes(const void *host, size_t bytes, void *dev, cudaStream_t s);
 
+// Second log-mel front-end (lfm.cu): per-call tables in the workspace and the
+// parameters the kernels read.
+constexpr int kLfmMaxMels = 128;  // bands
+constexpr int kLfmMaxBins = 32;   // nonzero bins per band
+constexpr int kLfmTile = 32;      // frames per work item of the spectrum kernel
+struct LfmTablesDev {
+  int n_clips, n_tiles;              // tiles: kLfmTile frames of one clip
+  const int64_t *sample_off;         // [B + 1]
+  const int32_t *frame_off, *tile_off;  // [B + 1]
+  const int32_t *eff;                // [B]: frames whose statistics count
+  const int32_t *bank_lo;            // [n_mels]: first nonzero bin of each band
+  const float *bank_w;               // [n_mels][kLfmMaxBins]: its weights from there
+};
+struct LfmParams {
+  int n_mels, hop, win_length;
+  int bins;  // the widest band's nonzero bins, rounded up to 4 (<= kLfmMaxBins)
+  float preemph, log_floor, var_eps;
+};
+size_t lfm_smem_bytes(int hop);
+cudaError_t launch_lfm(const float *wave, float *out, const LfmTablesDev &t, const LfmParams &prm, cudaStream_t s);
+
 unsigned *device_status_word();
 cudaError_t launch_wait_probe(unsigned long long limit_ns, int arrive, cudaStream_t s);
 unsigned read_and_clear_status();

@@ -1125,6 +1125,164 @@ ae_status ae_linear_e4m3(const void *d_x, const void *d_w, const float *d_cs, in
   return AE_OK;
 }
 
+// ------------------------------------------------------------------ second log-mel front-end
+
+namespace {
+bool lfm_cfg_ok(const ae_lfm_config *c) {
+  return c && c->n_fft == 512 && c->win_length >= 2 && c->win_length <= 512 && c->win_length % 2 == 0 &&
+         c->hop >= 2 && c->hop <= 320 && c->hop % 2 == 0 && c->n_mels >= 1 && c->n_mels <= kLfmMaxMels &&
+         c->sample_rate >= 1000 && c->sample_rate <= 1000000 && std::isfinite(c->preemph) &&
+         std::isfinite(c->log_floor) && c->log_floor > 0.f && std::isfinite(c->var_eps) && c->var_eps >= 0.f;
+}
+
+// Slaney mel scale: 3 f / 200 below 1 kHz, 15 + 27 ln(f / 1000) / ln 6.4 above.
+double slaney_mel(double f) { return f < 1000.0 ? 3.0 * f / 200.0 : 15.0 + 27.0 * std::log(f / 1000.0) / std::log(6.4); }
+double slaney_hz(double m) { return m < 15.0 ? 200.0 * m / 3.0 : 1000.0 * std::exp((m - 15.0) * std::log(6.4) / 27.0); }
+
+// The bank as (first nonzero bin, kLfmMaxBins weights from there) per band,
+// float64 from the definition; false if a band has more nonzero bins.
+bool lfm_bank(const ae_lfm_config &c, std::vector<int32_t> &lo, std::vector<float> &w, int *widest) {
+  const int nb = c.n_fft / 2 + 1;
+  lo.assign(c.n_mels, 0);
+  w.assign((size_t)c.n_mels * kLfmMaxBins, 0.f);
+  *widest = 0;
+  const double m_hi = slaney_mel(c.sample_rate / 2.0);
+  std::vector<double> pts(c.n_mels + 2);
+  for (int i = 0; i < c.n_mels + 2; ++i) pts[i] = slaney_hz(m_hi * i / (c.n_mels + 1));
+  for (int b = 0; b < c.n_mels; ++b) {
+    const double enorm = 2.0 / (pts[b + 2] - pts[b]);
+    int first = -1, last = -1;
+    std::vector<double> v(nb, 0.0);
+    for (int k = 0; k < nb; ++k) {
+      const double fk = (double)k * c.sample_rate / c.n_fft;
+      const double down = (fk - pts[b]) / (pts[b + 1] - pts[b]);
+      const double up = (pts[b + 2] - fk) / (pts[b + 2] - pts[b + 1]);
+      v[k] = std::max(0.0, std::min(down, up)) * enorm;
+      if (v[k] > 0.0) {
+        if (first < 0) first = k;
+        last = k;
+      }
+    }
+    if (first < 0) continue;  // an empty band (narrower than a bin): all zero weights
+    if (last - first + 1 > kLfmMaxBins) return false;
+    *widest = std::max(*widest, last - first + 1);
+    lo[b] = first;
+    for (int q = 0; first + q <= last; ++q) w[(size_t)b * kLfmMaxBins + q] = (float)v[first + q];
+  }
+  return true;
+}
+
+struct LfmLayout {
+  size_t sample_off, frame_off, tile_off, eff, bank_lo, bank_w, total;
+};
+LfmLayout lfm_layout(int n_clips) {
+  LfmLayout L;
+  const size_t B1 = (size_t)n_clips + 1;
+  size_t off = 0;
+  L.sample_off = off; off += al256(B1 * 8);
+  L.frame_off = off; off += al256(B1 * 4);
+  L.tile_off = off; off += al256(B1 * 4);
+  L.eff = off; off += al256(std::max<size_t>(n_clips, 1) * 4);
+  L.bank_lo = off; off += al256((size_t)kLfmMaxMels * 4);
+  L.bank_w = off; off += al256((size_t)kLfmMaxMels * kLfmMaxBins * 4);
+  L.total = off;
+  return L;
+}
+}  // namespace
+
+void ae_lfm_default_config(ae_lfm_config *cfg) {
+  if (!cfg) return;
+  cfg->sample_rate = 16000;
+  cfg->n_fft = 512;
+  cfg->win_length = 400;
+  cfg->hop = 160;
+  cfg->n_mels = 128;
+  cfg->preemph = 0.97f;
+  cfg->log_floor = 5.9604644775390625e-08f;  // 2^-24
+  cfg->var_eps = 1e-5f;
+}
+
+int64_t ae_lfm_num_frames(const ae_lfm_config *cfg, int64_t n_samples) {
+  if (!lfm_cfg_ok(cfg)) return -1;
+  return n_samples > 0 ? 1 + n_samples / cfg->hop : 0;
+}
+
+size_t ae_lfm_workspace_size(const ae_lfm_config *cfg, int n_clips) {
+  if (!lfm_cfg_ok(cfg) || n_clips < 0) return 0;
+  return lfm_layout(n_clips).total;
+}
+
+ae_status ae_lfm_logmel(const ae_lfm_config *cfg, const float *d_wave, const int64_t *h_sample_off, int n_clips,
+                        float *d_out, void *d_ws, size_t ws_bytes, ae_stream stream) {
+  if (!cfg) return fail(AE_EINVAL, "cfg is null");
+  if (!lfm_cfg_ok(cfg))
+    return fail(AE_EUNSUPPORTED, "supported: n_fft 512, even win_length in [2, 512], even hop in [2, 320], n_mels "
+                                 "in [1, 128], sample_rate in [1000, 1e6], finite preemph, log_floor > 0, var_eps >= 0");
+  if (n_clips < 0 || n_clips > kMaxClips) return fail(AE_EINVAL, "n_clips out of range");
+  if (!h_sample_off) return fail(AE_EINVAL, "h_sample_off is null");
+  if (h_sample_off[0] != 0) return fail(AE_EINVAL, "h_sample_off[0] must be 0");
+  std::vector<int64_t> so(h_sample_off, h_sample_off + n_clips + 1);
+  std::vector<int32_t> fo(n_clips + 1, 0), to(n_clips + 1, 0), eff(std::max(n_clips, 1), 0);
+  int64_t frames = 0, tiles = 0;
+  for (int i = 0; i < n_clips; ++i) {
+    const int64_t n = so[i + 1] - so[i];
+    if (n < 0) return fail(AE_EINVAL, "h_sample_off is not non-decreasing at clip " + std::to_string(i));
+    const int64_t nf = n > 0 ? 1 + n / cfg->hop : 0;
+    frames += nf;
+    tiles += (nf + kLfmTile - 1) / kLfmTile;
+    if (frames > INT32_MAX) return fail(AE_EINVAL, "more than 2^31 - 1 frames in one call");
+    fo[i + 1] = (int32_t)frames;
+    to[i + 1] = (int32_t)tiles;
+    eff[i] = (int32_t)((n + cfg->hop - 1) / cfg->hop);
+  }
+  std::vector<int32_t> blo;
+  std::vector<float> bw;
+  int widest = 0;
+  if (!lfm_bank(*cfg, blo, bw, &widest)) return fail(AE_EUNSUPPORTED, "a mel band spans more than 32 FFT bins");
+  if (frames == 0) return AE_OK;
+  if (!d_wave || !d_out) return fail(AE_EINVAL, "d_wave or d_out is null");
+  if (!aligned16(d_out)) return fail(AE_EINVAL, "d_out must be 16-byte aligned");
+  const LfmLayout L = lfm_layout(n_clips);
+  ae_status st = check_ws(d_ws, ws_bytes, L.total);
+  if (st) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *w = static_cast<uint8_t *>(d_ws);
+  cudaError_t e = cudaSuccess;
+  auto up = [&](const void *h, size_t bytes, size_t off) {
+    if (e == cudaSuccess && bytes) e = launch_upload_bytes(h, bytes, w + off, s);
+  };
+  up(so.data(), so.size() * 8, L.sample_off);
+  up(fo.data(), fo.size() * 4, L.frame_off);
+  up(to.data(), to.size() * 4, L.tile_off);
+  up(eff.data(), eff.size() * 4, L.eff);
+  up(blo.data(), blo.size() * 4, L.bank_lo);
+  up(bw.data(), bw.size() * 4, L.bank_w);
+  if (e != cudaSuccess) return cuda_fail(e, "table upload");
+  LfmTablesDev t;
+  t.n_clips = n_clips;
+  t.n_tiles = (int)tiles;
+  t.sample_off = reinterpret_cast<const int64_t *>(w + L.sample_off);
+  t.frame_off = reinterpret_cast<const int32_t *>(w + L.frame_off);
+  t.tile_off = reinterpret_cast<const int32_t *>(w + L.tile_off);
+  t.eff = reinterpret_cast<const int32_t *>(w + L.eff);
+  t.bank_lo = reinterpret_cast<const int32_t *>(w + L.bank_lo);
+  t.bank_w = reinterpret_cast<const float *>(w + L.bank_w);
+  LfmParams prm;
+  prm.n_mels = cfg->n_mels;
+  prm.hop = cfg->hop;
+  prm.win_length = cfg->win_length;
+  prm.bins = (widest + 3) & ~3;
+  prm.preemph = cfg->preemph;
+  prm.log_floor = cfg->log_floor;
+  prm.var_eps = cfg->var_eps;
+  // bytes: every sample read once, every output row written by the spectrum
+  // pass and read and rewritten by the normalisation
+  const double bytes = 4.0 * (double)so[n_clips] + 12.0 * (double)frames * cfg->n_mels;
+  if ((e = timed(AE_K_LFM, 0.0, bytes, s, [&] { return launch_lfm(d_wave, d_out, t, prm, s); })) != cudaSuccess)
+    return cuda_fail(e, "lfm front-end");
+  return AE_OK;
+}
+
 // ------------------------------------------------------------------ mixdown and resampling
 
 namespace {

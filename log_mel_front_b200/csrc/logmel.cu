@@ -20,6 +20,7 @@
 // their definitions; CTAs are persistent, so this costs once per CTA.
 #include "ae_internal.h"
 #include "common.cuh"
+#include "fft16.cuh"
 
 namespace ae {
 
@@ -41,47 +42,6 @@ struct LogmelSmem {
   int tile_clip, tile_f0, tile_nf;
 };
 }  // namespace
-
-__device__ __forceinline__ float2 cadd(float2 a, float2 b) { return make_float2(a.x + b.x, a.y + b.y); }
-__device__ __forceinline__ float2 csub(float2 a, float2 b) { return make_float2(a.x - b.x, a.y - b.y); }
-__device__ __forceinline__ float2 cmul(float2 a, float2 w) {
-  return make_float2(fmaf(a.x, w.x, -a.y * w.y), fmaf(a.x, w.y, a.y * w.x));
-}
-
-// In-place 4-point DFT: y_k = sum_n a_n (-i)^(n k).
-__device__ __forceinline__ void dft4(float2 &a0, float2 &a1, float2 &a2, float2 &a3) {
-  const float2 s02 = cadd(a0, a2), d02 = csub(a0, a2), s13 = cadd(a1, a3), d13 = csub(a1, a3);
-  a0 = cadd(s02, s13);
-  a2 = csub(s02, s13);
-  a1 = make_float2(d02.x + d13.y, d02.y - d13.x);  // d02 - i d13
-  a3 = make_float2(d02.x - d13.y, d02.y + d13.x);  // d02 + i d13
-}
-
-// 16-point DFT in registers, natural order in and out: x[k] <- sum_n x[n] W16^(n k).
-// Four-step 4 x 4: n = 4 n1 + n2, k = k1 + 4 k2.
-__device__ __forceinline__ void dft16(float2 (&x)[16]) {
-  constexpr float C1 = 0.92387953251128674f, S1 = 0.38268343236508977f, R = 0.70710678118654752f;
-#pragma unroll
-  for (int n2 = 0; n2 < 4; ++n2) dft4(x[n2], x[4 + n2], x[8 + n2], x[12 + n2]);
-  // x[4 k1 + n2] *= W16^(n2 k1)
-  x[5] = cmul(x[5], make_float2(C1, -S1));    // W^1
-  x[6] = cmul(x[6], make_float2(R, -R));      // W^2
-  x[7] = cmul(x[7], make_float2(S1, -C1));    // W^3
-  x[9] = cmul(x[9], make_float2(R, -R));      // W^2
-  x[10] = make_float2(x[10].y, -x[10].x);     // W^4 = -i
-  x[11] = cmul(x[11], make_float2(-R, -R));   // W^6
-  x[13] = cmul(x[13], make_float2(S1, -C1));  // W^3
-  x[14] = cmul(x[14], make_float2(-R, -R));   // W^6
-  x[15] = cmul(x[15], make_float2(-C1, S1));  // W^9
-#pragma unroll
-  for (int k1 = 0; k1 < 4; ++k1) dft4(x[4 * k1], x[4 * k1 + 1], x[4 * k1 + 2], x[4 * k1 + 3]);
-  // X[k1 + 4 k2] sits at x[4 k1 + k2]: transpose the 4 x 4
-  float2 t[16];
-#pragma unroll
-  for (int k = 0; k < 16; ++k) t[k] = x[4 * (k & 3) + (k >> 2)];
-#pragma unroll
-  for (int k = 0; k < 16; ++k) x[k] = t[k];
-}
 
 __global__ void __launch_bounds__(kThreads, 2)
     k_logmel(const float *__restrict__ wave, float *__restrict__ mel, const ClipTablesDev t, int n_tiles) {

@@ -83,6 +83,19 @@ def test_refusals_before_any_device_work(ae):
             ae.ae_linear_e4m3(0, 0, 0, M, N, K, -8.0, 8.0, 0, stream=0)
         assert e.value.status == ae.AE_EINVAL
     ae.ae_linear_e4m3(0, 0, 0, 0, 256, 128, -8.0, 8.0, 0, stream=0)  # M = 0: nothing to do
+    # the second front-end: unsupported shapes, bad offsets, over-wide bands
+    for kw in (dict(n_fft=256), dict(hop=161), dict(win_length=600), dict(n_mels=129), dict(log_floor=0.0)):
+        with pytest.raises(ae.AEError) as e:
+            ae.ae_lfm_logmel(ae.lfm_config(**kw), 0, [0, 100], 0, 0, 1 << 20, stream=0)
+        assert e.value.status == ae.AE_EUNSUPPORTED
+    with pytest.raises(ae.AEError) as e:
+        ae.ae_lfm_logmel(ae.lfm_config(), 0, [0, 100, 50], 0, 0, 1 << 20, stream=0)
+    assert e.value.status == ae.AE_EINVAL
+    with pytest.raises(ae.AEError) as e:  # 8 bands over 257 bins: far more than 16 bins a band
+        ae.ae_lfm_logmel(ae.lfm_config(n_mels=8), 0, [0, 100], 0, 0, 1 << 20, stream=0)
+    assert e.value.status == ae.AE_EUNSUPPORTED
+    ae.ae_lfm_logmel(ae.lfm_config(), 0, [0, 0], 0, 0, 0, stream=0)  # no frames: nothing to do
+    assert [ae.ae_lfm_num_frames(ae.lfm_config(), n) for n in (0, 1, 160, 48123)] == [0, 1, 2, 301]
 
 
 def test_attention_tables_closed_form(ae):
