@@ -17,9 +17,9 @@
 // bins (at most 32, listed by the host). CTAs are persistent.
 //
 // k_lfm_norm: one CTA per (clip, 32 bands): lane = band, the eight warps
-// stride over frames; the mean and then the biased variance are accumulated
-// in float64 in a fixed order (deterministic), and the clip's rows are
-// rewritten in place.
+// stride over frames; the sum and the sum of squares are accumulated in
+// float64 in one pass and a fixed order (deterministic), giving the mean and
+// the biased variance, and the clip's rows are rewritten in place.
 #include <cstddef>
 
 #include "ae_internal.h"
@@ -101,6 +101,7 @@ __global__ void __launch_bounds__(kLfmThreads, 2)
     // local sample i is padded position f0 hop + i, clip sample f0 hop + i - 256
     const int64_t first = (int64_t)f0 * hop - kLfmFft / 2;
     const int span = (nf - 1) * hop + kLfmFft;
+#pragma unroll 4
     for (int i = tid; i < span; i += kLfmThreads) {
       const int64_t sidx = first + i;
       float v = 0.f;
@@ -168,38 +169,44 @@ __global__ void __launch_bounds__(kLfmThreads, 2)
 }
 
 __global__ void __launch_bounds__(256) k_lfm_norm(float *__restrict__ out, const LfmTablesDev t, const LfmParams prm) {
-  __shared__ double red[8][32];
+  __shared__ double red[2][8][32];
   const int c = blockIdx.x, bg = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = bg * 32 + lane;
   const bool live = b < prm.n_mels;
   const int nf = t.frame_off[c + 1] - t.frame_off[c], eff = t.eff[c];
   float *base = out + (int64_t)t.frame_off[c] * prm.n_mels + b;
-  auto reduce = [&](double v) -> double {  // sum over the 8 warps, fixed order
-    red[warp][lane] = v;
-    __syncthreads();
-    double s = 0.0;
-    for (int w = 0; w < 8; ++w) s += red[w][lane];
-    __syncthreads();
-    return s;
-  };
-  double s = 0.0;
-  if (live)
-    for (int f = warp; f < eff; f += 8) s += (double)base[(int64_t)f * prm.n_mels];
-  const double mean = reduce(s) / (eff > 0 ? eff : 1);
-  double q = 0.0;
-  if (live)
+  // one pass for the first two moments, in float64 (for a band whose values
+  // are all equal both sums are exact and the variance is exactly zero)
+  double s1 = 0.0, s2 = 0.0;
+  if (live) {
+#pragma unroll 8
     for (int f = warp; f < eff; f += 8) {
-      const double d = (double)base[(int64_t)f * prm.n_mels] - mean;
-      q += d * d;
+      const double v = (double)base[(int64_t)f * prm.n_mels];
+      s1 += v;
+      s2 = fma(v, v, s2);
     }
-  const double var = reduce(q) / (eff > 0 ? eff : 1);
+  }
+  red[0][warp][lane] = s1;
+  red[1][warp][lane] = s2;
+  __syncthreads();
+  s1 = 0.0;
+  s2 = 0.0;
+  for (int w = 0; w < 8; ++w) {  // fixed order: deterministic
+    s1 += red[0][w][lane];
+    s2 += red[1][w][lane];
+  }
+  const double n = eff > 0 ? (double)eff : 1.0;
+  const double mean = s1 / n;
+  const double var = fmax(0.0, s2 / n - mean * mean);
   const double inv = 1.0 / sqrt(var + (double)prm.var_eps);
-  if (live)
+  if (live) {
+#pragma unroll 8
     for (int f = warp; f < nf; f += 8) {
       float *p = base + (int64_t)f * prm.n_mels;
       *p = f < eff ? (float)(((double)*p - mean) * inv) : 0.f;
     }
+  }
 }
 
 cudaError_t launch_lfm(const float *wave, float *out, const LfmTablesDev &t, const LfmParams &prm, cudaStream_t s) {
