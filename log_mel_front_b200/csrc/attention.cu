@@ -25,7 +25,8 @@ namespace ae {
 // of any clips); a persistent CTA (one per SM) walks the items. Per item:
 //   * TMA loads the q tile [128 x 128], the 144 k rows t0-11 .. t0+132 and the
 //     144 v rows (the tensor maps zero-fill rows before 0 and past T);
-//   * the four softmax warps scale q by s and split the product into two bf16
+//   * the eight softmax warps (two per 32-row quarter of the tile, each on
+//     half of the 128 head dims) scale q by s and split the product into two bf16
 //     tiles, hi = bf16(q s) and lo = bf16(q s - hi), so the score MMA sees q s
 //     to about 16 bits (a single bf16 rounding of q s costs more accuracy
 //     than everything else in the kernel together); they also write the
@@ -34,15 +35,16 @@ namespace ae {
 //     the same accumulator) gives S = (q s) [k ; R/k_scale]^T in tensor
 //     memory: row r holds q_t.k_{t0-11+c} at column c and the position term
 //     q_t.R[d]/k_scale at column 144+d;
-//   * the thread of row r (t = t0 + r) reads columns 32w .. 32w+47 of its warp's
+//   * in the first warp of each pair, the thread of row r (t = t0 + r) reads
+//     columns 32w .. 32w+47 of its warp's
 //     32 rows and shifts them left by its lane (five select stages), so that
 //     column r + 11 - d, the key t - d, lands at index 11 - d; it caps and
 //     softmaxes the 12 logits (distances past the clip start masked by pos) and
 //     writes them as bf16 into its row of a banded P [128 x 144] whose other
 //     entries stay zero;
 //   * tcgen05.mma (M=128, N=128, K=144, v read MN-major) gives O = P V;
-//   * the thread drains its row of O, clamps it, and TMA stores leave through a
-//     shared-memory box per warp.
+//   * both warps of the pair drain their row's half of O (64 dims each), clamp
+//     it, and TMA stores leave through a shared-memory box per warp.
 // Buffers are single: the next item's q/k load starts when the score MMA has
 // read them, its v load when the PV MMA has, so loads overlap the softmax.
 namespace {
