@@ -1,20 +1,23 @@
 // Projections of the tower: y = epilogue(x W^T) with x [M][K] (packed token
 // rows, M ragged) and W [N][K] (the checkpoint's [out][in] layout).
 //
-// bf16 path: a persistent tcgen05 kernel on CTA pairs (clusters of two SMs),
-// warp-specialised. Per 64-wide k-block, each CTA's warp 0 streams its half
-// of the pair tile (128 rows of x, 128 rows of W) into a 4-stage shared-memory
-// ring with TMA (128-byte swizzle, no multicast); the leader CTA's warp 1
-// issues tcgen05.mma.cta_group::2 (M=256, N=256, K=16, bf16 in, f32
-// accumulate), which reads the operand halves from both SMs, into one of two
-// 256-column accumulators in each CTA's tensor memory; warps 2-9 of each CTA
-// drain the other accumulator with tcgen05.ld and apply the epilogue
-// (ClipLin output clamp, SiLU and the next projection's input clamp, GLU, or
-// bias) on the way to memory through a swizzled shared-memory box and
-// coalesced row stores. Pairing halves the W bytes each SM stages per flop,
-// which keeps the shared-memory traffic (TMA writes plus tensor-core reads)
-// under the SM's bandwidth. Tiles are walked m-major so the pairs in flight
-// share rows of x in L2 while W stays L2-resident.
+// Tensor-core path: a persistent tcgen05 kernel on CTA pairs (clusters of two
+// SMs), warp-specialised. Per k-block (one 128-byte swizzle atom per row: 64
+// bf16 or 128 e4m3 elements), each CTA's warp 0 streams its half of the pair
+// tile (128 rows of x, 128 rows of W) into a shared-memory ring with TMA (no
+// multicast): 6 stages for the epilogues that store from registers, 4 for the
+// float32 ones, which also need staging boxes. The leader CTA's warp 1 issues
+// tcgen05.mma.cta_group::2 (M=256, N=256; kind::f16 with K=16 for bf16,
+// kind::f8f6f4 with K=32 for e4m3, f32 accumulate), which reads the operand
+// halves from both SMs, into one of two 256-column accumulators in each CTA's
+// tensor memory. Warps 2-9 of each CTA drain the other accumulator with
+// tcgen05.ld and apply the epilogue: the e4m3 column factors, the ClipLin output
+// clamp, SiLU (and the next projection's input clamp, or its e4m3 codes), GLU,
+// bias or the residual add. bf16 and e4m3 results leave each lane's row as
+// 32-byte sectors from registers; float32 results go through a swizzled
+// shared-memory box and coalesced row stores. Pairing halves the W bytes each
+// SM stages per flop. Tiles are walked m-major, so the pairs in flight share
+// rows of x in L2 while W stays L2-resident.
 //
 // f32 path: a plain 64x64-tile FMA kernel with the same epilogues.
 #include <cudaTypedefs.h>
