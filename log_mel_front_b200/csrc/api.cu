@@ -1,7 +1,10 @@
 // C ABI of the audio-encoder library: argument checks, model creation (weight
-// conversion, load-time tables), workspace layout and the stream-ordered
-// call sequences of the hot path. Every computation of a call runs in the
-// kernels of this library; the host only validates, lays out and launches.
+// conversion or e4m3 quantisation, load-time tables), workspace layout and the
+// stream-ordered call sequences of the hot path and of the adjacent parts (the
+// resampler, the second log-mel front-end, the standalone e4m3 projection).
+// Every computation of a call runs in the kernels of this library; the host
+// only validates, builds the per-call and load-time tables, lays out and
+// launches.
 #include <algorithm>
 #include <cmath>
 #include <cstring>

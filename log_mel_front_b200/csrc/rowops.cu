@@ -4,9 +4,10 @@
 // k_rowop fuses, per row of the float32 residual stream, the page's
 // add_normed (h += s * rms_w(y)), the plain residual add of the light conv,
 // the layer's closing rms(norm_out), and the next projection's input:
-// a = clamp(rms(h) * w, lo, hi) in the GEMM operand type. One warp owns a
-// row; each lane holds width/32 values in registers, so h is read and
-// written once per call.
+// a = clamp(rms(h) * w, lo, hi) in the GEMM operand type, or as e4m3 codes of
+// a * q for the e4m3 projections (q = 448 over the clamp's larger bound). One
+// warp owns a row; each lane holds width/32 values in registers, so h is read
+// and written once per call.
 //
 // k_lconv is the light-conv middle (dwconv, glu already applied by the
 // lc_start epilogue): the causal depthwise conv over 5 rows that does not
