@@ -5,7 +5,11 @@
  *
  * The operations are those of the gemma4_audio tower as the docs.rs page of
  * cortiq-engine 0.8.49, egemma2_audio.rs, states them (module doc items 1-5,
- * and the functions named beside each call below).
+ * and the functions named beside each call below). Three adjacent parts sit
+ * beside it: the channel mixdown and resampling to 16 kHz that precede the
+ * front-end (ae_resample), an 8-bit (e4m3) variant of the tower's projections
+ * (AE_FP8, ae_linear_e4m3), and the LFM2A encoder's log-mel front-end
+ * (ae_lfm_logmel).
  *
  * Conventions shared by every call
  * --------------------------------
@@ -16,13 +20,16 @@
  * - Clips are packed back to back without padding. A batch of n_clips clips
  *   is described by host int64 offsets [n_clips + 1], non-decreasing,
  *   starting at 0 (samples, frames or tokens depending on the call).
- * - Clips longer than 480000 samples are cut to their first 480000 samples
- *   (the feature extractor's 30 s truncation). A clip of 160 samples or fewer
- *   has no frames and no tokens; it is legal and produces no rows.
+ * - In the tower's calls, clips longer than 480000 samples are cut to their
+ *   first 480000 samples (the feature extractor's 30 s truncation), and a
+ *   clip of 160 samples or fewer has no frames and no tokens; it is legal and
+ *   produces no rows. The resampler and the LFM2A front-end take clips of any
+ *   length.
  * - Calls are stream-ordered: they enqueue work on `stream` and return
  *   without waiting for it, except ae_encode_host, which waits. They never
  *   allocate device memory; all scratch space comes from the caller's
- *   workspace (d_ws, ws_bytes), whose size ae_workspace_size returns. Two
+ *   workspace (d_ws, ws_bytes), whose size ae_workspace_size (or the
+ *   resampler's and the LFM2A front-end's own *_workspace_size) returns. Two
  *   calls that share a workspace must be ordered on one stream.
  * - Every argument is checked on the host before anything is enqueued: null
  *   pointers, a workspace below the required size, offsets that are not
