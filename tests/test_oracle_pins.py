@@ -342,8 +342,8 @@ def test_attention_two_token_hand_computation():
     z1 = qs @ (ks * k[0]) + qs @ R[1]
     z0, z1 = 50 * math.tanh(z0 / 50), 50 * math.tanh(z1 / 50)
     p0 = 1 / (1 + math.exp(z1 - z0))
-    assert np.allclose(o[1], p0 * v[1] + (1 - p0) * v[0], atol=1e-12)
-    assert np.allclose(o[0], v[0], atol=1e-15)
+    assert np.allclose(o[1], p0 * v[1] + (1 - p0) * v[0], rtol=0, atol=1e-12)
+    assert np.allclose(o[0], v[0], rtol=0, atol=1e-15)
 
 
 def test_attention_softcap_bounds_logits():

@@ -101,8 +101,8 @@ def test_cutoff_and_transition_band_follow_the_kaiser_window(rate):
     side of it the gain is what the Kaiser window (beta 12.8, 64 zero
     crossings) predicts; a different beta, width or roll-off moves these by
     more than 1e-2."""
-    c = R.RS_ROLLOFF * 16000 / rate
-    fc = R.RS_ROLLOFF * 8000
+    c = 0.958 * 16000 / rate  # the page's RS_ROLLOFF, written out: the pin must not follow the oracle's constant
+    fc = 0.958 * 8000
     n = 2 * rate
     for f0 in (fc, 0.97 * fc, 1.03 * fc):
         y = R.resample(_tone(rate, f0, n), rate)
