@@ -106,3 +106,19 @@ def test_attention_tables_closed_form(ae):
     assert abs(ks - math.log2(1 + math.e)) < 1e-6
     assert np.allclose(qs, O.q_scale_of(128) * O.softplus(pds), rtol=1e-6)
     assert np.allclose(R, O.relative_keys(relk, 12, 1024), rtol=1e-5, atol=1e-6)
+
+
+def test_second_frontend_constants_in_sync_with_the_oracle(ae):
+    """The library's default configuration of the second front-end equals the
+    oracle's reading of the page's constants, field by field (the page names
+    them without values, so both sides must take the same reading), and the
+    two agree on frame counts."""
+    from oracle import lfm as L
+    c = ae.lfm_config()
+    d = L.DEFAULTS
+    assert (c.sample_rate, c.n_fft, c.win_length, c.hop, c.n_mels) == \
+        (d["sample_rate"], d["n_fft"], d["win_length"], d["hop"], d["n_mels"])
+    for f in ("preemph", "log_floor", "var_eps"):
+        assert getattr(c, f) == np.float32(d[f]), f
+    for n in (0, 1, 159, 160, 161, 16000, 480000, 480001):
+        assert ae.ae_lfm_num_frames(c, n) == L.num_frames(n, d["hop"]), n
