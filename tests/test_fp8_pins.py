@@ -147,3 +147,10 @@ def test_linear_e4m3_against_integer_arithmetic():
             assert got[i, n] == float(Fraction(acc, 512 * 512) * Fraction(cs[n]))
     s = O.linear_e4m3(x, w, cs, -8.0, 8.0, silu_q=(-8.0, 8.0, 56.0))
     assert np.array_equal(O.e4m3_round(s), s) and np.max(np.abs(s)) <= 448.0
+
+
+def test_rounding_is_odd_and_monotone():
+    x = np.sort(np.random.default_rng(4).uniform(-500, 500, 100_000))
+    r = O.e4m3_round(x)
+    assert np.all(np.diff(r) >= 0)
+    assert np.array_equal(O.e4m3_round(-x), -r)

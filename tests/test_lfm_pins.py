@@ -98,3 +98,16 @@ def test_tone_lands_in_its_band():
     pts = L.mel_to_hz_slaney(np.linspace(0.0, L.hz_to_mel_slaney(8000.0), 130))
     want = int(np.argmin(np.abs(pts[1:-1] - 1000.0)))
     assert abs(int(np.argmax(lm[50])) - want) <= 1
+
+
+def test_features_do_not_depend_on_the_input_scale():
+    """Above the log floor, scaling the clip by a adds 2 ln a to every log-mel
+    value, which the per-band normalisation removes. Scaling up keeps every band
+    above the floor (scaling down can push the weakest, pre-emphasised low bands
+    onto it, where the clamp breaks the identity)."""
+    x = (0.1 * np.random.default_rng(9).standard_normal(16000 * 2)).astype(np.float32)
+    F = L.features(x)
+    for a in (2.0, 4.0, 64.0):
+        G = L.features((a * x).astype(np.float32))
+        assert np.max(np.abs(G - F)) < 1e-6
+        assert np.allclose(L.log_mel((a * x).astype(np.float32)), L.log_mel(x) + 2 * math.log(a), atol=1e-5)

@@ -127,3 +127,22 @@ def test_coprime_rate_and_equal_rate():
     z = np.arange(10, dtype=np.float32)
     assert np.array_equal(R.resample(z, 16000), z)
     assert len(R.resample(np.zeros(0, np.float32), 48000)) == 0
+
+
+def test_linear_and_shift_equivariant():
+    """The definition is a linear, shift-invariant filter evaluated on a
+    lattice: resampling a x + b y gives a R(x) + b R(y), and delaying the input
+    by o samples (one lattice period) delays the output by p samples."""
+    rng = np.random.default_rng(12)
+    for rate in (48000, 44100):
+        o, p = R.reduced_rates(rate, 16000)
+        n = 3000 + 7 * o
+        x = rng.standard_normal(n).astype(np.float32)
+        y = rng.standard_normal(n).astype(np.float32)
+        lin = R.resample((2 * x - 3 * y).astype(np.float32), rate).astype(np.float64)
+        assert np.max(np.abs(lin - (2 * R.resample(x, rate).astype(np.float64)
+                                    - 3 * R.resample(y, rate).astype(np.float64)))) < 1e-5
+        xs = np.concatenate([np.zeros(o, np.float32), x])
+        a = R.resample(x, rate)
+        b = R.resample(xs, rate)
+        assert np.array_equal(b[p:p + len(a)], a) or np.max(np.abs(b[p:p + len(a)] - a)) < 1e-6
