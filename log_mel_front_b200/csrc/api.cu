@@ -13,6 +13,7 @@
 #include <vector>
 
 #include "ae_internal.h"
+#include "e4m3_host.h"
 
 namespace ae {
 
@@ -259,29 +260,6 @@ static uint16_t f2bf(float f) {
   return (uint16_t)(u >> 16);
 }
 
-// OCP e4m3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; largest
-// finite 448, subnormals k 2^-9) code of t, rounded to nearest even, with
-// magnitudes beyond 448 saturated to 448.
-static uint8_t e4m3_code(double t) {
-  const uint8_t sign = std::signbit(t) ? 0x80 : 0x00;
-  const double a = std::fabs(t);
-  if (!(a < 448.0)) return sign | 0x7E;  // also NaN: never produced from finite weights
-  if (a < 0.015625) {                    // below 2^-6: subnormal grid of 2^-9 (k = 8 is the smallest normal)
-    return sign | (uint8_t)std::nearbyint(std::ldexp(a, 9));
-  }
-  int ex;
-  std::frexp(a, &ex);  // a = f 2^ex, f in [0.5, 1)
-  const int e = ex - 1;  // a in [2^e, 2^(e+1))
-  int k = (int)std::nearbyint(std::ldexp(a, 3 - e));  // 8 .. 16 steps of 2^(e-3)
-  int be = e + 7;
-  if (k == 16) {
-    k = 8;
-    ++be;
-  }
-  if (be > 15 || (be == 15 && k > 14)) return sign | 0x7E;
-  return sign | (uint8_t)((be << 3) | (k - 8));
-}
-
 struct Uploader {
   ae_model *m;
   bool ok = true;
@@ -315,11 +293,8 @@ struct Uploader {
     std::vector<uint8_t> codes(rows * cols);
     std::vector<float> f(rows);
     for (size_t r = 0; r < rows; ++r) {
-      const float *w = h.data() + r * cols;
-      double amax = 0.0;
-      for (size_t k = 0; k < cols; ++k) amax = std::max(amax, std::fabs((double)w[k]));
-      const double sn = amax > 0.0 ? amax / 448.0 : 1.0;
-      for (size_t k = 0; k < cols; ++k) codes[r * cols + k] = e4m3_code((double)w[k] / sn);
+      double sn;
+      e4m3_quantise_row(h.data() + r * cols, cols, codes.data() + r * cols, &sn);
       f[r] = (float)(sn / (double)q8);
     }
     *cs = f32(f.data(), f.size());
