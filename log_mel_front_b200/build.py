@@ -17,7 +17,7 @@ OBJ = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libae.so")
 ROOT = os.path.dirname(HERE)
 SOURCES = ["api.cu", "gemm.cu", "logmel.cu", "stem.cu", "attention.cu", "rowops.cu", "resample.cu", "lfm.cu"]
-HEADERS = ["common.cuh", "ae_internal.h", "fft16.cuh", "e4m3_host.h"]
+HEADERS = ["common.cuh", "ae_internal.h", "fft16.cuh", "e4m3_host.h", "lfm_host.h"]
 
 NVCC = os.environ.get("NVCC", "nvcc")
 FLAGS = [
