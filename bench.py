@@ -405,6 +405,17 @@ def max_over_ranks(value: float, dist, device: str = "cuda") -> float:
     return float(t.item())
 
 
+def sum_over_ranks(value: int, dist, device: str = "cuda") -> int:
+    """The sum over all ranks (every rank gets it); the value itself for a
+    single process. The whole job's kernel launches are counted this way."""
+    if not dist:
+        return int(value)
+    import torch
+    t = torch.tensor([int(value)], dtype=torch.int64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return int(t.item())
+
+
 def whole_job_value(audio_s_per_replica: float, world: int, ms_total: float, steps: int) -> float:
     """Audio seconds per second of the whole job: every rank runs one replica of
     the batch per step (weak scaling), timed as the slowest rank."""
@@ -425,7 +436,11 @@ def run_ours(args, rank, world, dist):
         torch.cuda.synchronize()
         if dist:
             dist.barrier()
-        ms = max_over_ranks(ours.timed(args.steps, ours.step), dist)
+        n0 = ae.ae_launch_count()
+        ms_local = ours.timed(args.steps, ours.step)
+        launches_timed = ae.ae_launch_count() - n0  # this library's kernels inside the timed steps
+        ms = max_over_ranks(ms_local, dist)
+        launches_timed = sum_over_ranks(launches_timed, dist)
         if dist:
             dist.barrier()
     clocks = clk.summary()
@@ -461,7 +476,6 @@ def run_ours(args, rank, world, dist):
     per_step = ms / args.steps
     audio = ours.audio_s * world
     value = whole_job_value(ours.audio_s, world, ms, args.steps)
-    launches = sum(v["launches"] for k, v in prof.items() if k != "dropped")
     dom = prof[ours.dominant]
     if ours.dominant == "gemm":
         achieved = dom["flops"] / (dom["ms"] / 1e3) / 1e12
@@ -521,7 +535,7 @@ def run_ours(args, rank, world, dist):
                     "ragged": "ae_encode_host_async, two streams (copies of one step overlap the kernels of the other)",
                     "frontend": "ae_logmel + copies", "lfm_frontend": "ae_lfm_logmel + copies",
                     "resample": "ae_resample + copies"}[args.workload]},
-        "gpu_launches": int(round(launches / prof_steps * args.steps)),
+        "gpu_launches": int(launches_timed),
         "roofline": roof,
         "kernel_classes": classes,
         "profiled_ms_per_step": round(ms_prof / prof_steps, 4),

@@ -420,6 +420,12 @@ ae_status ae_profile_read(double *ms, int64_t *launches, double *flops, double *
 
 /* --- diagnostics ------------------------------------------------------------- */
 
+/* Number of kernels this library has launched since it was loaded (every call,
+ * thread and device; launches the CUDA runtime refused are not counted). Read
+ * it before and after a region to count the region's launches. */
+uint64_t ae_launch_count(void);
+
+
 /* Message of the last failed call on this thread ("" if none). */
 const char *ae_last_error(void);
 

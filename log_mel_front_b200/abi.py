@@ -98,6 +98,7 @@ _sig("ae_resample", _st, _vp, _i32, C.c_int64, _i64p, _i32, C.c_int32, C.c_int32
 _sig("ae_linear_e4m3", _st, _vp, _vp, _vp, C.c_int64, C.c_int32, C.c_int32, C.c_float, C.c_float, _i32, C.c_float,
      C.c_float, C.c_float, _vp, _vp)
 _sig("ae_selftest_bounded_wait", _st, C.c_uint32, _i32, _vp)
+_sig("ae_launch_count", C.c_uint64)
 _sig("ae_lfm_default_config", None, C.POINTER(ae_lfm_config))
 _sig("ae_lfm_num_frames", C.c_int64, C.POINTER(ae_lfm_config), C.c_int64)
 _sig("ae_lfm_workspace_size", _sz, C.POINTER(ae_lfm_config), _i32)
@@ -112,7 +113,7 @@ EXPORTS = ("ae_num_frames", "ae_num_tokens", "ae_model_create", "ae_model_destro
            "ae_device_status", "ae_version", "ae_profile_enable", "ae_profile_read", "ae_logmel_noalloc",
            "ae_resample_len", "ae_resample_workspace_size", "ae_resample", "ae_linear_e4m3",
            "ae_selftest_bounded_wait", "ae_lfm_default_config", "ae_lfm_num_frames", "ae_lfm_workspace_size",
-           "ae_lfm_logmel")
+           "ae_lfm_logmel", "ae_launch_count")
 
 KERNEL_CLASSES = ("tables", "logmel", "conv0", "conv1", "gemm", "attention", "lconv", "rowop", "resample",
                   "gemm_fp8", "lfm")
@@ -252,6 +253,11 @@ def ae_linear_e4m3(d_x, d_w, d_cs, M: int, N: int, K: int, lo: float, hi: float,
 
 def ae_device_status() -> int:
     return lib.ae_device_status()
+
+
+def ae_launch_count() -> int:
+    """Kernels the library has launched since it was loaded."""
+    return int(lib.ae_launch_count())
 
 
 def lfm_config(**kw) -> "ae_lfm_config":

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -188,6 +189,9 @@ bool make_tmap_2d_u8(CUtensorMap *tm, const void *base, uint64_t inner, uint64_t
                      uint32_t box_inner, uint32_t box_outer);
 bool make_tmap_stem_y0(CUtensorMap *tm, const void *y0, int64_t stem_rows);
 
+// Kernels this library has launched (ae_launch_count), all threads and devices.
+std::atomic<uint64_t> &launch_counter();
+
 // Launch on stream s; the arguments are converted to the kernel's parameter types.
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
@@ -197,7 +201,9 @@ inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, siz
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+  if (e == cudaSuccess) launch_counter().fetch_add(1, std::memory_order_relaxed);
+  return e;
 }
 
 // Resampler (resample.cu): the rates reduced to o (in) and p (out), the cut-off

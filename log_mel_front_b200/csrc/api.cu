@@ -21,6 +21,11 @@ namespace ae {
 static thread_local std::string g_last_error;
 void set_error(const std::string &msg) { g_last_error = msg; }
 
+std::atomic<uint64_t> &launch_counter() {
+  static std::atomic<uint64_t> n{0};
+  return n;
+}
+
 static size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 
 static int64_t frames_of_samples(int64_t n) {
@@ -674,6 +679,8 @@ ae_status ae_device_status(void) {
   if (v) return fail(AE_EDEVICE, "a kernel gave up a bounded wait");
   return AE_OK;
 }
+
+uint64_t ae_launch_count(void) { return launch_counter().load(std::memory_order_relaxed); }
 
 ae_status ae_selftest_bounded_wait(uint32_t limit_us, int arrive, ae_stream stream) {
   if (limit_us < 1 || limit_us > 1000000) return fail(AE_EINVAL, "limit_us must be in [1, 1000000]");

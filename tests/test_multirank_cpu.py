@@ -22,9 +22,10 @@ dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
 ms = 100.0 + 7.0 * rank          # the timed region of this rank
 dist.barrier()
 m = bench.max_over_ranks(ms, dist, device="cpu")
+n = bench.sum_over_ranks(100 + rank, dist, device="cpu")   # each rank's kernel launches
 dist.barrier()
 v = bench.whole_job_value(480.0, world, m, 10)
-print(json.dumps({"rank": rank, "max_ms": m, "value": v}), flush=True)
+print(json.dumps({"rank": rank, "max_ms": m, "value": v, "launches": n}), flush=True)
 dist.destroy_process_group()
 """
 
@@ -54,6 +55,7 @@ def test_two_ranks_agree_on_the_slowest_rank_and_the_whole_job_value():
     assert sorted(o["rank"] for o in outs) == [0, 1]
     for o in outs:
         assert o["max_ms"] == 107.0  # rank 1's time: the job is as slow as its slowest rank
+        assert o["launches"] == 201  # the whole job's launches: 100 + 101
         # two replicas of 480 audio seconds per 10.7 ms step
         assert abs(o["value"] - 2 * 480.0 / (107.0 / 10 / 1e3)) < 1e-6
 
@@ -62,6 +64,7 @@ def test_single_process_helpers():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.max_over_ranks(12.5, None) == 12.5
+    assert bench.sum_over_ranks(7, None) == 7
     assert abs(bench.whole_job_value(480.0, 1, 95.0, 10) - 480.0 / 9.5e-3) < 1e-6
 
 
