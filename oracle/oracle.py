@@ -35,9 +35,12 @@ quantized pack's kernels as an option. They are pinned by torch's
 the row quantisation.
 
 Parity status: every stage is pinned by the ``-m "not gpu"`` tests (page
-values, closed forms, invariants, brute force). The composition of a full
-layer and of the tower is pinned only by a tiny-size brute-force restatement
-and by packing invariance; no end-to-end value is printed on the pages.
+values, closed forms, invariants, brute force), the head and the input
+projection included (a hand-worked head example, the weightless norm's scale
+invariance, and a non-symmetric ``input_proj_linear`` that fixes which axis of
+the stored matrix is the output). The composition of a full layer and of the
+tower is pinned only by a tiny-size brute-force restatement and by packing
+invariance; no end-to-end value is printed on the pages.
 """
 from __future__ import annotations
 

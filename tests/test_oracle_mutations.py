@@ -78,6 +78,24 @@ MUTANTS = {
     "depthwise taps reversed": (
         O, "dwconv", lambda: _wrap("dwconv", lambda f, x, w, pos: f(x, np.asarray(w)[:, ::-1], pos)),
         [P.test_dwconv_impulse_response_and_clip_start]),
+    # stem projection and head (encode_locked)
+    "in_proj applied transposed": (
+        O, "subsample", lambda: (lambda mel, W: O.stem(mel, W) @ np.asarray(W["in_proj"], np.float64)),
+        [P.test_in_proj_rows_are_output_features]),
+    "head without out_bias": (
+        O, "head", lambda: (lambda h, W: O.rms(h @ np.asarray(W["out_proj"], np.float64).T)
+                            @ np.asarray(W["embed"], np.float64).T),
+        [P.test_head_hand_computation, P.test_head_norm_is_weightless_and_scale_invariant]),
+    "head without the weightless RMS norm": (
+        O, "head", lambda: (lambda h, W: (h @ np.asarray(W["out_proj"], np.float64).T
+                                          + np.asarray(W["out_bias"], np.float64))
+                            @ np.asarray(W["embed"], np.float64).T),
+        [P.test_head_hand_computation, P.test_head_norm_is_weightless_and_scale_invariant]),
+    "head RMS norm with 1e-3 instead of 1e-6": (
+        O, "head", lambda: (lambda h, W: ((lambda o: o / np.sqrt((o * o).mean(-1, keepdims=True) + 1e-3))(
+            h @ np.asarray(W["out_proj"], np.float64).T + np.asarray(W["out_bias"], np.float64)))
+                            @ np.asarray(W["embed"], np.float64).T),
+        [P.test_head_hand_computation]),
     # layer composition
     "FFN half-residual ignored": (
         O, "ffn", lambda: _wrap("ffn", lambda f, h, ly, name, bounds, rw, fp8=False: f(h, ly, name, bounds, 1.0, fp8)),

@@ -230,6 +230,68 @@ def test_stem_layer_norm_and_flatten():
     assert np.allclose(x[1, 7 * 4 + 2], ln[1, 7, 2])
 
 
+def _narrow_stem(seed):
+    rng = np.random.default_rng(seed)
+    return {"conv0": rng.standard_normal((8, 9)) * 0.3, "ln0": 1.0 + 0.1 * rng.standard_normal(8),
+            "conv1": rng.standard_normal((4, 8, 3, 3)) * 0.3, "ln1": 1.0 + 0.1 * rng.standard_normal(4)}
+
+
+def test_in_proj_rows_are_output_features():
+    """``input_proj_linear`` keeps the checkpoint layout [out][in] (the page
+    checks that its row count is the hidden width) and is applied as
+    ``gemm_nt``: output feature i = sum_j x_j W[i][j]. A square shift
+    permutation W[i][(i+1) mod n] = 1 makes output i read stem feature i+1; the
+    transposed product would read feature i-1. A wide-to-narrow projection
+    picks features by rows."""
+    W = _narrow_stem(21)
+    mel = np.random.default_rng(22).standard_normal((13, 128))
+    x = O.stem(mel, W)                        # [4, 4*32 = 128], frequency-major
+    n = x.shape[1]
+    shift = np.zeros((n, n))
+    shift[np.arange(n), (np.arange(n) + 1) % n] = 1.0
+    y = O.subsample(mel, dict(W, in_proj=shift))
+    assert np.array_equal(y, np.roll(x, -1, axis=1))
+    assert not np.array_equal(y, np.roll(x, 1, axis=1))
+    pick = np.zeros((3, n))
+    pick[[0, 1, 2], [5, 40, 127]] = [1.0, -2.0, 0.5]
+    y = O.subsample(mel, dict(W, in_proj=pick))
+    assert y.shape == (x.shape[0], 3)
+    assert np.array_equal(y, np.stack([x[:, 5], -2.0 * x[:, 40], 0.5 * x[:, 127]], axis=1))
+
+
+def test_head_hand_computation():
+    """``encode_locked`` tail: o = out_proj h + out_bias, a weightless RMS norm,
+    then embed_audio, on a 2 -> 3 -> 2 example worked by hand:
+    h = (1, 2); out_proj rows (1, 0), (0, 1), (1, 1) give (1, 2, 3); the bias
+    (0.5, -1, 1) gives o = (1.5, 1, 4); mean(o^2) = (2.25 + 1 + 16) / 3 = 19.25 / 3;
+    embed rows (1, 0, 0), (0, 1, -1) give (1.5, 1 - 4) / sqrt(19.25 / 3 + 1e-6)."""
+    W = {"out_proj": np.array([[1.0, 0.0], [0.0, 1.0], [1.0, 1.0]]),
+         "out_bias": np.array([0.5, -1.0, 1.0]),
+         "embed": np.array([[1.0, 0.0, 0.0], [0.0, 1.0, -1.0]])}
+    got = O.head(np.array([[1.0, 2.0]]), W)
+    s = math.sqrt(19.25 / 3.0 + 1e-6)
+    assert got.shape == (1, 2)
+    assert np.allclose(got, [[1.5 / s, -3.0 / s]], rtol=0, atol=1e-14)
+
+
+def test_head_norm_is_weightless_and_scale_invariant():
+    """With a zero bias the weightless RMS norm makes the head invariant to the
+    scale of h (once eps is negligible), and every row entering embed has unit
+    root mean square: with embed = identity the output rows are exactly that."""
+    rng = np.random.default_rng(23)
+    h = rng.standard_normal((5, 6))
+    W = {"out_proj": rng.standard_normal((9, 6)), "out_bias": np.zeros(9), "embed": np.eye(9)}
+    e = O.head(h, W)
+    assert np.allclose(np.sqrt((e ** 2).mean(1)), 1.0, rtol=0, atol=1e-5)
+    big = O.head(1e4 * h, W)
+    o = h @ W["out_proj"].T
+    assert np.allclose(big, o / np.sqrt((o ** 2).mean(1, keepdims=True)), rtol=0, atol=1e-12)
+    assert np.allclose(big, e, rtol=0, atol=1e-6)             # eps / mean(o^2) ~ 1e-7 here
+    # a bias breaks the invariance (it is added before the norm)
+    Wb = dict(W, out_bias=rng.standard_normal(9))
+    assert not np.allclose(O.head(1e4 * h, Wb), O.head(h, Wb), atol=1e-3)
+
+
 # ------------------------------------------------------------------ projections and norms
 
 def test_matrix_product_matches_triple_loop_and_clamps():
