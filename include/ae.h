@@ -294,7 +294,9 @@ ae_status ae_linear_e4m3(const void *d_x, const void *d_w, const float *d_cs, in
  * before anything is enqueued. The call calls no cudaMalloc or cudaFree.
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture. Every call uses the same array and rewrites the
+ * before any stream capture. The address is kept per device with the CUDA
+ * context it belongs to: after cudaDeviceReset (a new context) the next call
+ * looks it up again, and that call, too, must come before any capture. Every call uses the same array and rewrites the
  * part it reads, so calls that may overlap on the GPU (on different streams,
  * or from several host threads) race with each other: order them on one
  * stream. */
@@ -337,7 +339,7 @@ size_t ae_lfm_workspace_size(const ae_lfm_config *cfg, int n_clips);
  * clips back to back (16-byte aligned). Supported: n_fft 512; win_length and
  * hop even, 2 <= win_length <= 512, 2 <= hop <= 320; 1 <= n_mels <= 128 with
  * at most 32 nonzero bins per band; sample_rate in [1000, 1000000];
- * log_floor > 0, var_eps >= 0, all finite (AE_EINVAL or AE_EUNSUPPORTED
+ * log_floor > 0, var_eps > 0 (a silent band would divide 0 by 0), all finite (AE_EINVAL or AE_EUNSUPPORTED
  * otherwise, before anything is enqueued). At most 2^31 - 1 frames in all.
  * Asynchronous on `stream`; no allocation. */
 ae_status ae_lfm_logmel(const ae_lfm_config *cfg, const float *d_wave, const int64_t *h_sample_off, int n_clips,

@@ -192,6 +192,23 @@ bool make_tmap_stem_y0(CUtensorMap *tm, const void *y0, int64_t stem_rows);
 // Kernels this library has launched (ae_launch_count), all threads and devices.
 std::atomic<uint64_t> &launch_counter();
 
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current
+// device. The attribute belongs to the device, so `done` keeps one bit per
+// device index (0..63) whose attribute is already set; the call is
+// thread-safe (setting it twice is harmless). Devices above 63 set it on
+// every call.
+template <typename... KArgs>
+inline cudaError_t smem_attr(void (*kernel)(KArgs...), size_t bytes, std::atomic<uint64_t> &done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
 // Launch on stream s; the arguments are converted to the kernel's parameter types.
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,

@@ -634,13 +634,34 @@ static ae_status encode_dev(const ae_model *m, const float *d_wave, const ClipTa
 // The clip tables of ae_logmel_noalloc live in this file-scope device array
 // (every GPU that loads the library holds it until the process exits). In
 // host code the name is only a stand-in: its device address is looked up
-// once per device with cudaGetSymbolAddress and passed to the kernels.
+// with cudaGetSymbolAddress, with the device current, and passed to the
+// kernels. The address is cached per device together with the CUDA context
+// it was taken in; a different current context (after cudaDeviceReset, say)
+// makes the next call look it up again.
 constexpr int kNoAllocMaxClips = 4000;
 constexpr size_t kNoAllocScratchBytes = 131072;
 static __device__ __align__(256) unsigned char g_logmel_scratch[kNoAllocScratchBytes];
 
 static std::mutex g_noalloc_mu;
 static void *g_noalloc_ptr[64] = {nullptr};
+static void *g_noalloc_ctx[64] = {nullptr};
+
+// The current CUDA context (driver cuCtxGetCurrent, looked up at run time), or
+// nullptr if the entry point is unavailable.
+static void *current_context() {
+  using Fn = int (*)(void **);
+  static Fn fn = [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<Fn>(p);
+    return static_cast<Fn>(nullptr);
+  }();
+  void *ctx = nullptr;
+  if (!fn || fn(&ctx) != 0) return nullptr;
+  return ctx;
+}
 
 // Device address of the scratch array on the current device.
 static ae_status noalloc_scratch(void **out) {
@@ -648,11 +669,13 @@ static ae_status noalloc_scratch(void **out) {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return fail(AE_ECUDA, "no CUDA device");
   if (dev >= 64) return fail(AE_EUNSUPPORTED, "device index above 63");
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  void *ctx = current_context();
+  if (!g_noalloc_ptr[dev] || !ctx || ctx != g_noalloc_ctx[dev]) {
     void *p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_logmel_scratch);
     if (e != cudaSuccess || !p) return cuda_fail(e, "cudaGetSymbolAddress of the log-mel scratch");
     g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = current_context();  // the lookup may have created the primary context
   }
   *out = g_noalloc_ptr[dev];
   return AE_OK;
@@ -1118,7 +1141,7 @@ bool lfm_cfg_ok(const ae_lfm_config *c) {
   return c && c->n_fft == 512 && c->win_length >= 2 && c->win_length <= 512 && c->win_length % 2 == 0 &&
          c->hop >= 2 && c->hop <= 320 && c->hop % 2 == 0 && c->n_mels >= 1 && c->n_mels <= kLfmMaxMels &&
          c->sample_rate >= 1000 && c->sample_rate <= 1000000 && std::isfinite(c->preemph) &&
-         std::isfinite(c->log_floor) && c->log_floor > 0.f && std::isfinite(c->var_eps) && c->var_eps >= 0.f;
+         std::isfinite(c->log_floor) && c->log_floor > 0.f && std::isfinite(c->var_eps) && c->var_eps > 0.f;
 }
 
 struct LfmLayout {

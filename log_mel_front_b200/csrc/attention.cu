@@ -422,12 +422,8 @@ cudaError_t launch_attention(bool is_bf16, const void *q, const void *k, const v
                              int64_t ld_out, float lo, float hi, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
   if (is_bf16) {
-    static bool attr = false;
-    if (!attr) {
-      cudaError_t e = cudaFuncSetAttribute(k_attention_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AT_SMEM);
-      if (e != cudaSuccess) return e;
-      attr = true;
-    }
+    static std::atomic<uint64_t> attr{0};
+    if (const cudaError_t e = smem_attr(k_attention_tc, AT_SMEM, attr)) return e;
     CUtensorMap tq, tk, tv, to;
     const uint64_t rb = (uint64_t)ld * 2, ob = (uint64_t)ld_out * 2;
     if (!make_tmap_2d_bf16(&tq, q, kHidden, (uint64_t)T, rb, 64, AT_Q) ||
@@ -444,12 +440,8 @@ cudaError_t launch_attention(bool is_bf16, const void *q, const void *k, const v
                     cap, pos, (int)T, lo, hi, device_status_word());
   }
   const size_t smem = (2 * (size_t)kRows * kPitchF + kLeft * kHeadDim + kHeadDim) * sizeof(float);
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_attention_f32, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static std::atomic<uint64_t> attr{0};
+  if (const cudaError_t e = smem_attr(k_attention_f32, smem, attr)) return e;
   dim3 grid((unsigned)((T + kTQ - 1) / kTQ), kHeads);
   return launch_k(k_attention_f32, grid, dim3(kTQ), smem, s, static_cast<const float *>(q),
                   static_cast<const float *>(k), static_cast<const float *>(v), ld, R, qscale, k_scale, cap, pos, T,

@@ -588,24 +588,23 @@ bool make_tmap_stem_y0(CUtensorMap *tm, const void *y0, int64_t stem_rows) {
 }
 
 static int num_sms() {
-  static int n[64] = {0};
+  static std::atomic<int> n[64];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) dev = 0;
-  if (!n[dev]) cudaDeviceGetAttribute(&n[dev], cudaDevAttrMultiProcessorCount, dev);
-  return n[dev] > 0 ? n[dev] : 1;
+  int v = 0;
+  if (dev >= 0 && dev < 64) v = n[dev].load(std::memory_order_relaxed);
+  if (!v) {
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    if (dev >= 0 && dev < 64 && v > 0) n[dev].store(v, std::memory_order_relaxed);
+  }
+  return v > 0 ? v : 1;
 }
 
 template <int MODE, bool F8 = false>
 static cudaError_t launch_tc(const CUtensorMap &tA, const CUtensorMap &tB, const EpiArgs &ep, int M, int N, int K,
                              cudaStream_t s) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e =
-        cudaFuncSetAttribute(k_gemm_tc<MODE, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_of(MODE));
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static std::atomic<uint64_t> attr{0};
+  if (const cudaError_t e = smem_attr(k_gemm_tc<MODE, F8>, smem_of(MODE), attr)) return e;
   const int tiles = ((M + 2 * BM - 1) / (2 * BM)) * (N / BN);
   const int pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;
   return launch_k(k_gemm_tc<MODE, F8>, dim3(2 * pairs), dim3(GEMM_THREADS), smem_of(MODE), s, tA, tB, ep, M, N, K,

@@ -176,8 +176,10 @@ __global__ void __launch_bounds__(256) k_lfm_norm(float *__restrict__ out, const
   const bool live = b < prm.n_mels;
   const int nf = t.frame_off[c + 1] - t.frame_off[c], eff = t.eff[c];
   float *base = out + (int64_t)t.frame_off[c] * prm.n_mels + b;
-  // one pass for the first two moments, in float64 (for a band whose values
-  // are all equal both sums are exact and the variance is exactly zero)
+  // one pass for the first two moments, in float64. Only the first moment is
+  // exact for a band whose values are all equal; s2 / n - mean^2 can round to
+  // a tiny value of either sign, which the clamp at zero and var_eps (> 0,
+  // checked on the host) absorb
   double s1 = 0.0, s2 = 0.0;
   if (live) {
 #pragma unroll 8

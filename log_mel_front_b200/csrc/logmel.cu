@@ -192,12 +192,8 @@ cudaError_t launch_logmel(const float *wave, float *mel, const ClipTablesDev &t,
                           cudaStream_t s) {
   if (mel_tiles <= 0) return cudaSuccess;
   const size_t smem = sizeof(LogmelSmem);
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_logmel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static std::atomic<uint64_t> attr{0};
+  if (const cudaError_t e = smem_attr(k_logmel, smem, attr)) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -314,12 +314,8 @@ cudaError_t launch_conv1(const ae_model *m, const void *y0, int64_t stem_rows, v
                          int64_t conv1_tiles, int64_t tokens, cudaStream_t s) {
   if (tokens <= 0) return cudaSuccess;
   if (m->dtype != AE_F32) {
-    static bool attr = false;
-    if (!attr) {
-      cudaError_t e = cudaFuncSetAttribute(k_conv1_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C1_SMEM);
-      if (e != cudaSuccess) return e;
-      attr = true;
-    }
+    static std::atomic<uint64_t> attr{0};
+    if (const cudaError_t e = smem_attr(k_conv1_tc, C1_SMEM, attr)) return e;
     CUtensorMap tmY;
     if (!make_tmap_stem_y0(&tmY, y0, stem_rows)) return cudaErrorInvalidValue;
     return launch_k(k_conv1_tc, dim3((unsigned)conv1_tiles), dim3(128), C1_SMEM, s, tmY, m->tm_conv1, t,

@@ -122,3 +122,14 @@ def test_second_frontend_constants_in_sync_with_the_oracle(ae):
         assert getattr(c, f) == np.float32(d[f]), f
     for n in (0, 1, 159, 160, 161, 16000, 480000, 480001):
         assert ae.ae_lfm_num_frames(c, n) == L.num_frames(n, d["hop"]), n
+
+
+def test_second_frontend_refuses_a_zero_variance_epsilon(ae):
+    """var_eps must be positive: with 0, a band whose frames are all equal (a
+    silent clip) would be normalised by 0 / 0. The refusal is a host check
+    (no GPU needed): the size helpers report the configuration invalid."""
+    c = ae.lfm_config()
+    assert ae.ae_lfm_num_frames(c, 16000) > 0
+    c.var_eps = 0.0
+    assert ae.ae_lfm_num_frames(c, 16000) == -1
+    assert ae.ae_lfm_workspace_size(c, 4) == 0

@@ -64,3 +64,19 @@ def test_noalloc_refuses_too_many_clips():
     with pytest.raises(ae.AEError) as e:
         ae.ae_logmel_noalloc(0, off, 0)
     assert e.value.status == ae.AE_EINVAL and "at most 4000 clips" in str(e.value)
+
+
+def test_noalloc_at_the_clip_limit():
+    """4000 clips, the most one call takes: the clip tables come closest to
+    filling the fixed array here. Short clips of 161 to 400 samples (one or two
+    frames each) keep the call small; its rows must equal ae_logmel's."""
+    rng = np.random.default_rng(4000)
+    lens = rng.integers(161, 401, size=4000)
+    clips = [(0.3 * rng.standard_normal(int(n))).astype(np.float32) for n in lens]
+    want = _with_workspace(clips)
+    got = _without_workspace(clips)
+    assert got.shape == want.shape == (_frames(clips), 128)
+    assert np.all(np.isfinite(got))
+    err = float(np.max(np.abs(got - want)))
+    print(f"[parity] ae_logmel_noalloc at 4000 clips vs ae_logmel: max abs diff {err:.3e} (bound {LOGMEL_ABS})")
+    assert err <= LOGMEL_ABS
