@@ -147,6 +147,28 @@ int64_t ae_num_frames(int64_t n_samples);
 /* Soft tokens of a clip of n samples: ceil(ceil(frames / 2) / 2). */
 int64_t ae_num_tokens(int64_t n_samples);
 
+/* --- data-parallel partition of a batch ------------------------------------ */
+
+/* Assigns the clips of a batch to n_parts devices (or streams) for
+ * data-parallel encoding. Every clip's output rows depend on that clip alone
+ * (egemma2_audio.rs, encode_locked: the stem runs per clip, attention spans
+ * min(pos + 1, 12) rows of the clip and the depthwise conv stops at its
+ * start), so the parts need no exchange, only the model on every device.
+ * Greedy token balance: clips in decreasing order of soft tokens
+ * (ae_num_tokens of their length; equal counts by lower clip index) each go
+ * to the part holding the fewest tokens so far (equal totals by lower part
+ * index). The largest part's total then exceeds the smallest one's by at
+ * most one clip's tokens (750 at most). Deterministic: every caller that
+ * passes the same lengths gets the same assignment, so ranks can compute it
+ * independently.
+ * h_sample_off: host int64 [n_clips + 1] sample offsets, as for ae_encode.
+ * h_part: host int32 [n_clips], receives each clip's part in [0, n_parts).
+ * h_tokens: host int64 [n_parts] or NULL, receives each part's token total.
+ * n_parts in [1, 65536]. Host only: no device is touched and nothing is
+ * enqueued; AE_EINVAL for bad offsets, counts or null pointers. */
+ae_status ae_partition_clips(const int64_t *h_sample_off, int n_clips, int n_parts, int32_t *h_part,
+                             int64_t *h_tokens);
+
 /* --- model ----------------------------------------------------------------- */
 
 /* Validates cfg and the weight pointers, converts and uploads the weights

@@ -75,6 +75,7 @@ def _sig(name, res, *args):
 
 _sig("ae_num_frames", C.c_int64, C.c_int64)
 _sig("ae_num_tokens", C.c_int64, C.c_int64)
+_sig("ae_partition_clips", _st, _i64p, _i32, _i32, C.POINTER(C.c_int32), _i64p)
 _sig("ae_model_create", _st, C.POINTER(ae_config), C.POINTER(ae_host_weights), _i32, C.POINTER(_vp))
 _sig("ae_model_destroy", None, _vp)
 _sig("ae_workspace_size", _sz, _vp, C.c_int64, C.c_int64, C.c_int64)
@@ -113,7 +114,7 @@ EXPORTS = ("ae_num_frames", "ae_num_tokens", "ae_model_create", "ae_model_destro
            "ae_device_status", "ae_version", "ae_profile_enable", "ae_profile_read", "ae_logmel_noalloc",
            "ae_resample_len", "ae_resample_workspace_size", "ae_resample", "ae_linear_e4m3",
            "ae_selftest_bounded_wait", "ae_lfm_default_config", "ae_lfm_num_frames", "ae_lfm_workspace_size",
-           "ae_lfm_logmel", "ae_launch_count")
+           "ae_lfm_logmel", "ae_launch_count", "ae_partition_clips")
 
 KERNEL_CLASSES = ("tables", "logmel", "conv0", "conv1", "gemm", "attention", "lconv", "rowop", "resample",
                   "gemm_fp8", "lfm")
@@ -170,6 +171,17 @@ def ae_num_frames(n: int) -> int:
 
 def ae_num_tokens(n: int) -> int:
     return lib.ae_num_tokens(int(n))
+
+
+def ae_partition_clips(sample_off, n_parts: int) -> tuple[np.ndarray, np.ndarray]:
+    """(part of each clip int32 [n_clips], tokens of each part int64 [n_parts])."""
+    a, p = _off(sample_off)
+    n = len(a) - 1
+    part = np.zeros(max(n, 0), np.int32)
+    tok = np.zeros(max(int(n_parts), 1), np.int64)
+    _check(lib.ae_partition_clips(p, n, int(n_parts), part.ctypes.data_as(C.POINTER(C.c_int32)),
+                                  tok.ctypes.data_as(_i64p)), "ae_partition_clips")
+    return part, tok[:int(n_parts)]
 
 
 def ae_workspace_size(model, n_clips: int, total_frames: int, total_tokens: int) -> int:

@@ -1344,6 +1344,40 @@ size_t ae_resample_workspace_size(const int64_t *h_sample_off, int n_clips, int3
   return rs_layout(n_clips, pl, T.total_in, channels, rate_in == rate_out).total;
 }
 
+ae_status ae_partition_clips(const int64_t *h_sample_off, int n_clips, int n_parts, int32_t *h_part,
+                             int64_t *h_tokens) {
+  if (n_parts < 1 || n_parts > 65536) return fail(AE_EINVAL, "n_parts must lie in [1, 65536]");
+  if (n_clips < 0) return fail(AE_EINVAL, "n_clips is negative");
+  if (!h_sample_off) return fail(AE_EINVAL, "h_sample_off is null");
+  if (n_clips > 0 && !h_part) return fail(AE_EINVAL, "h_part is null");
+  if (h_sample_off[0] != 0) return fail(AE_EINVAL, "h_sample_off[0] must be 0");
+  std::vector<int64_t> tok((size_t)n_clips);
+  for (int i = 0; i < n_clips; ++i) {
+    const int64_t n = h_sample_off[i + 1] - h_sample_off[i];
+    if (n < 0) return fail(AE_EINVAL, "h_sample_off is not non-decreasing at clip " + std::to_string(i));
+    tok[(size_t)i] = tokens_of_frames(frames_of_samples(n));
+  }
+  std::vector<int> order((size_t)n_clips);
+  for (int i = 0; i < n_clips; ++i) order[(size_t)i] = i;
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return tok[(size_t)a] > tok[(size_t)b]; });
+  // min-heap of (tokens so far, part index): the lightest part, lowest index first
+  using Load = std::pair<int64_t, int>;
+  std::vector<Load> heap((size_t)n_parts);
+  for (int p = 0; p < n_parts; ++p) heap[(size_t)p] = Load(0, p);
+  auto heavier = [](const Load &a, const Load &b) { return a > b; };
+  std::make_heap(heap.begin(), heap.end(), heavier);
+  for (int i : order) {
+    std::pop_heap(heap.begin(), heap.end(), heavier);
+    Load &l = heap.back();
+    h_part[i] = l.second;
+    l.first += tok[(size_t)i];
+    std::push_heap(heap.begin(), heap.end(), heavier);
+  }
+  if (h_tokens)
+    for (const Load &l : heap) h_tokens[l.second] = l.first;
+  return AE_OK;
+}
+
 ae_status ae_resample(const float *d_x, int channels, int64_t ch_stride, const int64_t *h_sample_off, int n_clips,
                       int32_t rate_in, int32_t rate_out, float *d_y, void *d_ws, size_t ws_bytes,
                       ae_stream stream) {

@@ -116,6 +116,27 @@ def clip_lengths(workload: str) -> list[int]:
     raise ValueError(workload)
 
 
+def global_lengths(workload: str, n_batches: int) -> list[int]:
+    """Clip lengths of a global batch of n_batches times the workload's batch
+    (the data-parallel runs split it over devices): batch 0 is the workload's
+    own clips, batch b > 0 draws the same way with its own seed."""
+    lens = list(clip_lengths(workload))
+    for b in range(1, n_batches):
+        if workload == "ragged":
+            rng = _rng(WORKLOADS["ragged"]["config_index"], 999_999, b)
+            lens += [int(v) for v in rng.integers(16000, 480000, size=256, endpoint=True)]
+        else:
+            lens += list(clip_lengths(workload))
+    return lens
+
+
+def global_waves(workload: str, lengths: list[int], clips: list[int]) -> list[np.ndarray]:
+    """Clips (by global index) of a global batch with these lengths; for the
+    indices of batch 0 these are exactly ``waves(workload)``'s clips."""
+    seed = WORKLOADS[workload]["config_index"]
+    return [noise_tones_clip(lengths[i], seed, i) for i in clips]
+
+
 def waves(workload: str, clips: list[int] | None = None) -> list[np.ndarray]:
     """The workload's clips (or the listed subset of them), float32 each."""
     if workload == "pr1":

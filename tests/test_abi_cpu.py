@@ -133,3 +133,11 @@ def test_second_frontend_refuses_a_zero_variance_epsilon(ae):
     c.var_eps = 0.0
     assert ae.ae_lfm_num_frames(c, 16000) == -1
     assert ae.ae_lfm_workspace_size(c, 4) == 0
+
+
+def test_partition_refusals(ae):
+    import numpy as np
+    for off, parts in (([0, 100, 50], 2), ([0, 10], 0), ([0, 10], 70000), ([5, 10], 2)):
+        with pytest.raises(ae.AEError) as e:
+            ae.ae_partition_clips(np.array(off, np.int64), parts)
+        assert e.value.status == ae.AE_EINVAL

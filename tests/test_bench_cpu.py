@@ -13,14 +13,22 @@ import bench  # noqa: E402
 
 
 def test_traffic_captures_describe_the_committed_kernel():
-    for kind in ("gemm", "gemm_fp8"):
-        value, src = bench.captured_traffic(kind)
-        assert value is not None and value > 0, (kind, src)
-        assert os.path.exists(os.path.join(ROOT, src))
+    for (kind, workload), (path, _) in bench.TRAFFIC_PROFILES.items():
+        if not os.path.exists(os.path.join(ROOT, path)):
+            continue   # a capture not taken yet reports null
+        value, src = bench.captured_traffic(kind, workload)
+        assert value is not None and value > 0, (kind, workload, src)
 
 
 def test_no_capture_means_null():
-    assert bench.captured_traffic("attention")[0] is None
+    assert bench.captured_traffic("attention", "attention")[0] is None
+    assert bench.captured_traffic("gemm", "attention")[0] is None
+
+
+def test_tensor_peak_follows_the_clock():
+    assert bench.tensor_peak_kind({"sm_mhz": 1940.0, "sm_max_mhz": 1965.0}) == (True, "burst")
+    assert bench.tensor_peak_kind({"sm_mhz": 1350.0, "sm_max_mhz": 1965.0}) == (False, "sustained")
+    assert bench.tensor_peak_kind({"sm_mhz": None, "sm_max_mhz": None}) == (False, "sustained")
 
 
 def test_workload_tables():

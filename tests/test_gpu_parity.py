@@ -71,12 +71,14 @@ def gpu_encode(model, clips, embed_dim=512):
     frames = sum(O.num_frames(len(c)) for c in clips)
     toks = sum(O.num_tokens(len(c)) for c in clips)
     d_wave = dev(flat)
-    d_out = torch.full((max(toks, 1), embed_dim), float("nan"), device="cuda")
+    d_out = torch.full((toks + 1, embed_dim), float("nan"), device="cuda")   # one sentinel row
     nb = model.workspace_size(len(clips), frames, toks)
     ws = workspace(nb)
     ae.ae_encode(model, d_wave, off, d_out, ws, ws.numel())
     _sync()
-    return d_out[:toks].cpu().numpy(), offsets([O.num_tokens(len(c)) for c in clips])
+    g = d_out.cpu().numpy()
+    assert np.all(np.isnan(g[toks])), "rows written beyond the batch's token count"
+    return g[:toks], offsets([O.num_tokens(len(c)) for c in clips])
 
 
 # ------------------------------------------------------------------ log-mel
@@ -209,7 +211,8 @@ def test_encode_tower_full_batch_sampled_clips(m_tower, w_tower):
     g, off = gpu_encode(m_tower, clips)
     assert g.shape == (16 * 750, 512)
     assert np.all(np.isfinite(g))
-    for i in (0, 9):
+    # every clip (about 3 s of oracle time each)
+    for i in range(16):
         o = O.encode([clips[i]], w_tower)[0]
         assert_bf16(g[off[i]:off[i + 1]], o, f"tower clip {i}")
 
@@ -218,10 +221,20 @@ def test_encode_ragged_full_batch_sampled_clips(m_tower, w_tower):
     lens = synth.clip_lengths("ragged")
     clips = synth.waves("ragged")
     g, off = gpu_encode(m_tower, clips)
+    # every clip's row count is ae_num_tokens of its length (the library's own
+    # count), equal to the page's formula, and the rows fill the output exactly
+    assert [ae.ae_num_tokens(n) for n in lens] == [O.num_tokens(n) for n in lens]
     assert g.shape[0] == sum(O.num_tokens(n) for n in lens)
     assert np.all(np.isfinite(g))
+    # 16 clips: the shortest, the longest and 14 more drawn with a fixed seed
+    # (spread over the batch, so that a row count wrong anywhere before a
+    # sampled clip would shift its rows and fail its comparison), the last one
+    # of the batch among them
     order = np.argsort(lens)
-    picks = [int(order[0]), int(order[-1]), 17]
+    rng = np.random.default_rng(404)
+    rest = [i for i in range(len(lens)) if i not in (int(order[0]), int(order[-1]), len(lens) - 1)]
+    picks = [int(order[0]), int(order[-1]), len(lens) - 1] + sorted(rng.choice(rest, 13, replace=False).tolist())
+    assert len(set(picks)) == 16
     for i in picks:
         o = O.encode([clips[i]], w_tower)[0]
         assert_bf16(g[off[i]:off[i + 1]], o, f"ragged clip {i} ({lens[i]} samples)")
