@@ -9,9 +9,11 @@ import numpy as np
 import pytest
 
 from oracle import lfm as LF
+from oracle import lfm_encoder as LE
 from oracle import oracle as O
 from oracle import resample as RS
 from tests import test_fp8_pins as P8
+from tests import test_lfm_encoder_pins as PE
 from tests import test_lfm_pins as PL
 from tests import test_oracle_pins as P
 from tests import test_resample_pins as PR
@@ -117,7 +119,50 @@ MODULE_MUTANTS = {
         [PL.test_slaney_scale_closed_forms]),
     "second front-end without pre-emphasis": (
         LF, "DEFAULTS", lambda: dict(LF.DEFAULTS, preemph=0.0), [lambda: PL.test_frame_count_and_power_match_torch_stft(400)]),
+    # LFM2A encoder body
+    "XL relative shift reversed (p row t-1+i-j)": (
+        LE, "xl_attention", lambda: (lambda q, k, v, p, bu, bv, heads:
+                                     LE_ORIG["xl_attention"](q, k, v, p[::-1].copy(), bu, bv, heads)),
+        [lambda: PE.test_relative_shift_direction(1)]),
+    "macaron FFN at full weight": (
+        LE, "macaron_ffn", lambda: (lambda x, ly, f, eps: 2.0 * LE_ORIG["macaron_ffn"](x, ly, f, eps) - x),
+        [PE.test_macaron_ffn_half_weight]),
+    "GELU in its tanh form": (
+        LE, "gelu_erf", lambda: (lambda x: 0.5 * np.asarray(x) * (1 + np.tanh(math.sqrt(2 / math.pi) *
+                                                                             (np.asarray(x) + 0.044715 * np.asarray(x) ** 3)))),
+        [PE.test_gelu_is_the_erf_form]),
+    "stem flattened frequency-major": (
+        LE, "stem", lambda: (lambda mel, W: _stem_freq_major(mel, W)), [PE.test_stem_geometry_and_flatten]),
+    "depthwise conv made causal": (
+        LE, "depthwise_conv1d", lambda: (lambda x, w, b: _causal_dw(x, w, b)),
+        [lambda: PE.test_depthwise_conv_impulse_response(9)]),
 }
+
+
+LE_ORIG = {"xl_attention": LE.xl_attention, "macaron_ffn": LE.macaron_ffn}
+
+
+def _stem_freq_major(mel, W):
+    x = np.asarray(mel, np.float64)[None]
+    for i, (dw, stride, pad, k) in enumerate(LE.STEM_MODES):
+        x = LE.conv2d(x, W[f"stem{i}.w"], W[f"stem{i}.b"], stride, pad, x.shape[0] if dw else 1)
+        if LE.STEM_RELU[i]:
+            x = np.maximum(x, 0.0)
+    c, t, f = x.shape
+    flat = x.transpose(1, 2, 0).reshape(t, f * c)
+    return flat @ np.asarray(W["pre_w"], np.float64).T + np.asarray(W["pre_b"], np.float64)
+
+
+def _causal_dw(x, w, b):
+    x, w = np.asarray(x, np.float64), np.asarray(w, np.float64)
+    t, C = x.shape
+    k = w.shape[0]
+    xp = np.zeros((t + k - 1, C))
+    xp[k - 1:] = x
+    y = np.zeros((t, C))
+    for m in range(k):
+        y += w[m][None, :] * xp[m:m + t]
+    return y + np.asarray(b, np.float64)[None, :]
 
 
 def _e4m3_half_up(x):
