@@ -2,7 +2,7 @@
 """Throughput of the B200 audio-encoder forward.
 
     python bench.py [--gpus N] [--steps K] [--warmup W]
-                    [--workload ragged|tower|tower_fp8|frontend|lfm_frontend|attention|resample]
+                    [--workload ragged|tower|tower_fp8|frontend|lfm_frontend|lfm_encoder|attention|resample]
     python bench.py --impl reference ...      # the CPU oracle on the same workload (bounded sample)
 
 A step is one ae_encode over one batch (default: the ragged batch, 256 clips
@@ -173,6 +173,9 @@ def workload_desc(name: str, info: dict) -> dict:
             "frontend": "log-mel front-end only, 64 clips x 30 s, f32",
             "lfm_frontend": "second (LFM2A) log-mel front-end: pre-emphasis, centre padding, power spectrum, Slaney "
                             "bank, per-band normalisation; 64 clips x 30 s, f32",
+            "lfm_encoder": "LFM2A encoder from PCM: the second log-mel front-end, the 5-layer conv stem, 17 "
+                           "Conformer blocks with Transformer-XL attention and the erf-GELU adapter to 2048; 16 "
+                           "clips x 30 s (376 tokens each), bf16 weights, f32 accumulation",
             "attention": "local-attention core only, 32 x 8192 tokens, 8 heads x 128, bf16 q/k/v",
             "resample": "mixdown + Kaiser-sinc resampling to 16 kHz, 64 stereo clips x 30 s at 44.1 kHz, f32"}[name]
     d = {"workload": f"{name}: {base}", "l2": "flushed between steps (256 MiB write)",
@@ -182,7 +185,7 @@ def workload_desc(name: str, info: dict) -> dict:
 
 
 ENCODE_WORKLOADS = ("tower", "tower_fp8", "ragged")
-CLIP_WORKLOADS = ENCODE_WORKLOADS + ("frontend", "lfm_frontend")
+CLIP_WORKLOADS = ENCODE_WORKLOADS + ("frontend", "lfm_frontend", "lfm_encoder")
 
 
 def rank_clips(lengths, world: int, rank: int, partition) -> list[int]:
@@ -203,7 +206,7 @@ def audio_seconds(lengths) -> float:
 def data_of(name: str) -> str:
     """The synthetic batch a workload runs on (the e4m3 tower runs the tower's,
     the second front-end the first one's)."""
-    return {"tower_fp8": "tower", "lfm_frontend": "frontend"}.get(name, name)
+    return {"tower_fp8": "tower", "lfm_frontend": "frontend", "lfm_encoder": "tower"}.get(name, name)
 
 
 class Ours:
@@ -234,6 +237,21 @@ class Ours:
             self.ws_host_bytes = ae.ae_encode_host_workspace_size(self.model, self.off)
             self.ws = torch.empty(max(self.ws_bytes, self.ws_host_bytes), dtype=torch.uint8, device="cuda")
             self.dominant = "gemm_fp8" if name == "tower_fp8" else "gemm"
+        elif name == "lfm_encoder":
+            self.cfg = ae.lfm_config()
+            self.lfm_frames = [ae.ae_lfm_num_frames(self.cfg, n) for n in self.lens]
+            self.frames = sum(self.lfm_frames)
+            self.lfm_ws_bytes = ae.ae_lfm_workspace_size(self.cfg, len(self.lens))
+            self.lfm_ws = torch.empty(self.lfm_ws_bytes, dtype=torch.uint8, device="cuda")
+            self.d_mel = torch.empty((self.frames, 128), device="cuda")
+            self.enc = ae.LencModel(synth.lfm_encoder_weights())
+            self.frame_off = np.concatenate([[0], np.cumsum(self.lfm_frames)]).astype(np.int64)
+            self.tokens = sum(ae.ae_lenc_num_tokens(f) for f in self.lfm_frames)
+            self.ws_bytes = self.enc.workspace_size(self.frame_off)
+            self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device="cuda")
+            self.d_out = torch.empty((self.tokens, 2048), device="cuda")
+            self.h_out = torch.empty((self.tokens, 2048)).pin_memory()
+            self.dominant = "lenc_gemm"
         elif name == "lfm_frontend":
             self.cfg = ae.lfm_config()
             self.frames = sum(ae.ae_lfm_num_frames(self.cfg, n) for n in self.lens)
@@ -292,6 +310,9 @@ class Ours:
             ae.ae_logmel(self.d_wave, self.off, self.d_mel, self.ws, self.ws_bytes, self.stream)
         elif self.name == "lfm_frontend":
             ae.ae_lfm_logmel(self.cfg, self.d_wave, self.off, self.d_mel, self.ws, self.ws_bytes, self.stream)
+        elif self.name == "lfm_encoder":
+            ae.ae_lfm_logmel(self.cfg, self.d_wave, self.off, self.d_mel, self.lfm_ws, self.lfm_ws_bytes, self.stream)
+            ae.ae_lenc_encode(self.enc, self.d_mel, self.frame_off, self.d_out, self.ws, self.ws_bytes, self.stream)
         elif self.name == "resample":
             ae.ae_resample(self.d_x, 2, self.d_x.shape[1], self.off, synth.RS_RATE, 16000, self.d_y, self.ws,
                            self.ws_bytes, self.stream)
@@ -311,6 +332,12 @@ class Ours:
             self.h_mel.copy_(self.d_mel, non_blocking=True)
             self.stream.synchronize()
             return self.h_wave.numel() * 4, self.h_mel.numel() * 4
+        if self.name == "lfm_encoder":
+            self.d_wave.copy_(self.h_wave, non_blocking=True)
+            self.step()
+            self.h_out.copy_(self.d_out, non_blocking=True)
+            self.stream.synchronize()
+            return self.h_wave.numel() * 4, self.h_out.numel() * 4
         if self.name == "resample":
             self.d_x.copy_(self.h_x, non_blocking=True)
             self.step()
@@ -406,6 +433,15 @@ class OracleRun:
             t0 = time.perf_counter()
             LF.features(c)
             return time.perf_counter() - t0, 30.0, "clip 0 of the frontend workload (second front-end)"
+        if self.name == "lfm_encoder":
+            from oracle import lfm as LF
+            from oracle import lfm_encoder as LE
+            if not hasattr(self, "lenc_w"):
+                self.lenc_w = synth.lfm_encoder_weights()
+            c = synth.waves("tower", [0])[0]
+            t0 = time.perf_counter()
+            LE.encode(LF.features(c), self.lenc_w)
+            return time.perf_counter() - t0, 30.0, "clip 0 of the tower workload through the LFM2A front-end and encoder"
         if self.name == "resample":
             i = self.next % synth.RS_CLIPS
             self.next += 1
@@ -524,7 +560,7 @@ def run_ours(args, rank, world, dist):
         job_tokens = ours.tokens * world
     dom = prof[ours.dominant]
     burst, kind = tensor_peak_kind(clocks)
-    if ours.dominant in ("gemm", "gemm_fp8"):
+    if ours.dominant in ("gemm", "gemm_fp8", "lenc_gemm"):
         # e4m3 dense rate = the measured bf16 figure x the nominal ratio 4.5 / 2.25 PFLOP/s
         mult = 2.0 if ours.dominant == "gemm_fp8" else 1.0
         achieved = dom["flops"] / (dom["ms"] / 1e3) / 1e12
@@ -548,6 +584,7 @@ def run_ours(args, rank, world, dist):
     traffic, traffic_src = captured_traffic(ours.dominant, args.workload)
     roof.update({"kernel": {"gemm": "k_gemm_tc (all projections)", "logmel": "k_logmel",
                             "lfm": "k_lfm_spec + k_lfm_norm",
+                            "lenc_gemm": "k_gemm_tc (the LFM2A encoder's projections)",
                             "gemm_fp8": "k_gemm_tc<e4m3> (FFN W1/W2, q/k/v, lc_start)",
                             "attention": "k_attention_tc",
                             "resample": "k_rs_fir (with its tap table and mixdown)"}[ours.dominant],
@@ -564,7 +601,7 @@ def run_ours(args, rank, world, dist):
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(per_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None,
-        "dtype": {"frontend": "f32", "lfm_frontend": "f32", "resample": "f32",
+        "dtype": {"frontend": "f32", "lfm_frontend": "f32", "resample": "f32", "lfm_encoder": "bf16",
                   "tower_fp8": "e4m3+bf16"}.get(args.workload, "bf16"),
         "data": "synthetic",
         "config": workload_desc(args.workload, (({
@@ -586,6 +623,7 @@ def run_ours(args, rank, world, dist):
                                  "other)",
                     "ragged": "ae_encode_host_async, two streams (copies of one step overlap the kernels of the other)",
                     "frontend": "ae_logmel + copies", "lfm_frontend": "ae_lfm_logmel + copies",
+                    "lfm_encoder": "ae_lfm_logmel + ae_lenc_encode + copies",
                     "resample": "ae_resample + copies"}[args.workload]},
         "gpu_launches": int(launches_timed),
         "roofline": roof,
@@ -627,8 +665,8 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", choices=("tower", "tower_fp8", "ragged", "frontend", "lfm_frontend", "attention",
-                                           "resample"),
+    ap.add_argument("--workload", choices=("tower", "tower_fp8", "ragged", "frontend", "lfm_frontend", "lfm_encoder",
+                                           "attention", "resample"),
                     default="ragged")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

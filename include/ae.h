@@ -367,6 +367,109 @@ size_t ae_lfm_workspace_size(const ae_lfm_config *cfg, int n_clips);
 ae_status ae_lfm_logmel(const ae_lfm_config *cfg, const float *d_wave, const int64_t *h_sample_off, int n_clips,
                         float *d_out, void *d_ws, size_t ws_bytes, ae_stream stream);
 
+/* --- LFM2A Conformer encoder ---------------------------------------------------- */
+
+/* The Conformer body of the LFM2A audio encoder as the page of its GPU port
+ * runs it (cera 0.5.3, audio_encoder_gpu.rs: encode_audio_gpu, macaron_ffn,
+ * conv_stem_gpu with STEM_LAYER_MODES / STEM_RELU_AFTER, and the ops of the
+ * AudioEncoderGpuOps trait), from a log-mel spectrogram such as
+ * ae_lfm_logmel's:
+ *   stem: 3x3 stride-2 conv 1 -> C (+bias, ReLU), depthwise 3x3 stride 2
+ *   (+bias), pointwise C -> C (+bias, ReLU), depthwise 3x3 stride 2 (+bias),
+ *   pointwise C -> C (+bias, ReLU), all with zero padding 1 per side; the
+ *   (channel, time, freq) result flattened to (time, channel * freq) and
+ *   pre_encode_out (+bias) to n_embd;
+ *   n_layers blocks, each: x += 0.5 FFN(LN(x)) with FFN = down(silu(up(.)
+ *   + b) ) + b; a = LN(x); q, k, v = linear + bias; p = pos_emb W_pos^T (no
+ *   bias); x += o(attn) + b_o, where attn is Transformer-XL attention,
+ *   softmax_j(((q_i + u) . k_j + (q_i + v) . p_{i-j}) / sqrt(head_dim)) v_j
+ *   over the keys of the clip; conv module: g = GLU(pw1(LN(x)) + b) (first
+ *   half times sigmoid of the second), a depthwise conv over time of k taps
+ *   (pad (k - 1) / 2 left, the rest right, within the clip) + bias, a
+ *   per-channel affine, SiLU, x += pw2(.) + b; x += 0.5 FFN2(LN(x)); x =
+ *   LN(x);
+ *   adapter: out = down(gelu_erf(up(LN(x)) + b)) + b (erf-form GELU).
+ * LayerNorms use the biased variance and their weight and bias. pos_emb has
+ * 2 t - 1 rows for relative positions t - 1 .. -(t - 1), row p holding
+ * sin(p w_i), cos(p w_i) in columns 2i, 2i + 1, w_i = 10000^(-2i / n_embd);
+ * the page shows neither this table nor the attention's relative shift, so
+ * both are this library's reading of them. Projections run as bf16 tcgen05
+ * GEMMs with float32 accumulation; the residual stream, norms and softmax are
+ * float32. The kernels are compiled for n_mels 128, n_embd 512, n_head 8
+ * (head_dim 64), stem channels 256; n_ff, adapter_ff and llm_hidden multiples
+ * of 256; 1 <= conv_k <= 33; n_layers >= 0; at most 4096 rows after the stem
+ * per clip (AE_EUNSUPPORTED otherwise). */
+typedef struct {
+  int32_t n_mels, n_embd, n_head, n_layers, n_ff, conv_k, stem_ch, adapter_ff, llm_hidden;
+  float eps;  /* LayerNorm epsilon */
+} ae_lenc_config;
+
+/* One block's weights, host float32, matrices [out][in] row-major: the FFN's
+ * up [n_ff][n_embd] and down [n_embd][n_ff], q/k/v/o and pw2 [n_embd][n_embd],
+ * linear_pos [n_embd][n_embd], pw1 [2 n_embd][n_embd], dw [conv_k][n_embd]
+ * (taps first); every vector [n_embd] except up_b [n_ff] and pw1_b
+ * [2 n_embd]. norm_conv_* is the conv module's LayerNorm, conv_norm_* its
+ * per-channel affine. */
+typedef struct {
+  const float *ffn1_norm_w, *ffn1_norm_b, *ffn1_up_w, *ffn1_up_b, *ffn1_down_w, *ffn1_down_b;
+  const float *ln1_w, *ln1_b;
+  const float *q_w, *q_b, *k_w, *k_b, *v_w, *v_b, *o_w, *o_b;
+  const float *linear_pos_w, *pos_bias_u, *pos_bias_v;
+  const float *norm_conv_w, *norm_conv_b, *pw1_w, *pw1_b, *dw_w, *dw_b, *conv_norm_w, *conv_norm_b, *pw2_w, *pw2_b;
+  const float *ffn2_norm_w, *ffn2_norm_b, *ffn2_up_w, *ffn2_up_b, *ffn2_down_w, *ffn2_down_b;
+  const float *ln2_w, *ln2_b;
+} ae_lenc_host_block;
+
+/* Stem weights [C][1][3][3] (layers 0, 1, 3) and [C][C] (layers 2, 4) with
+ * biases [C]; pre_encode_out [n_embd][C * n_mels / 8] with columns in the
+ * page's (channel, freq) order, bias [n_embd]; blocks [n_layers]; adapter
+ * LayerNorm [n_embd], up [adapter_ff][n_embd] + [adapter_ff], down
+ * [llm_hidden][adapter_ff] + [llm_hidden]. */
+typedef struct {
+  const float *stem_w[5], *stem_b[5];
+  const float *pre_w, *pre_b;
+  const ae_lenc_host_block *blocks;
+  const float *ad_norm_w, *ad_norm_b, *ad_up_w, *ad_up_b, *ad_down_w, *ad_down_b;
+} ae_lenc_host_weights;
+
+typedef struct ae_lenc ae_lenc;
+
+/* The sizes the page names without values, as this library reads them: 128
+ * mels, n_embd 512, 8 heads, 17 layers, n_ff 2048, conv_k 9, 256 stem
+ * channels, adapter_ff 2048, llm_hidden 2048, eps 1e-5. */
+void ae_lenc_default_config(ae_lenc_config *cfg);
+
+/* Rows after the stem for a clip of n_frames mel frames: three times
+ * ceil(n / 2) (0 for n_frames <= 0). */
+int64_t ae_lenc_num_tokens(int64_t n_frames);
+
+/* Validates cfg and the pointers, converts the matrices to bf16 and uploads
+ * everything to the current device. Synchronous; *out is NULL on failure. */
+ae_status ae_lenc_create(const ae_lenc_config *cfg, const ae_lenc_host_weights *w, ae_lenc **out);
+void ae_lenc_destroy(ae_lenc *m);
+
+/* Workspace bytes of ae_lenc_stem / ae_lenc_encode for clips with these mel
+ * frame offsets, and of ae_lenc_block for these token offsets (0 for invalid
+ * offsets). */
+size_t ae_lenc_workspace_size(const ae_lenc *m, const int64_t *h_frame_off, int n_clips);
+size_t ae_lenc_block_workspace_size(const ae_lenc *m, const int64_t *h_tok_off, int n_clips);
+
+/* The stem and pre_encode_out per clip: d_mel float32 [h_frame_off[n]][128]
+ * -> d_x float32 [sum tokens][n_embd] (16-byte aligned). */
+ae_status ae_lenc_stem(const ae_lenc *m, const float *d_mel, const int64_t *h_frame_off, int n_clips, float *d_x,
+                       void *d_ws, size_t ws_bytes, ae_stream stream);
+
+/* Block `layer` in place on d_x float32 [h_tok_off[n]][n_embd] (16-byte
+ * aligned); attention within each clip. */
+ae_status ae_lenc_block(const ae_lenc *m, int layer, float *d_x, const int64_t *h_tok_off, int n_clips,
+                        void *d_ws, size_t ws_bytes, ae_stream stream);
+
+/* The whole body: stem, every block, adapter. d_out float32 [sum tokens]
+ * [llm_hidden], clip after clip (16-byte aligned). A clip with no tokens gives
+ * no rows. Asynchronous on `stream`; nothing is allocated. */
+ae_status ae_lenc_encode(const ae_lenc *m, const float *d_mel, const int64_t *h_frame_off, int n_clips,
+                         float *d_out, void *d_ws, size_t ws_bytes, ae_stream stream);
+
 /* --- input conditioning: mixdown and resampling -------------------------------- */
 
 /* Output length of ae_resample for one clip of n_samples at rate_in:
@@ -423,7 +526,10 @@ typedef enum {
   AE_K_RESAMPLE = 8, /* mixdown, resampler taps and FIR */
   AE_K_GEMM_FP8 = 9, /* the e4m3 projections of AE_FP8 (tcgen05 kind::f8f6f4) */
   AE_K_LFM = 10,     /* the second log-mel front-end (spectrum, bands, normalisation) */
-  AE_K_COUNT = 11
+  AE_K_LENC_GEMM = 11,      /* the LFM2A encoder's projections (tcgen05, bf16) */
+  AE_K_LENC_ATTENTION = 12, /* its Transformer-XL attention */
+  AE_K_LENC_ROW = 13,       /* its stem convolutions, LayerNorms, conv-module middle, position table */
+  AE_K_COUNT = 14
 } ae_kernel_class;
 
 /* Kernel timing for measurement (the analogue of the page's

@@ -14,7 +14,7 @@ __version__ = "0.1.0"
 def __getattr__(name):
     if name.startswith("__"):
         raise AttributeError(name)
-    if name in ("abi", "build"):
+    if name in ("abi", "build", "gen_htk_bank"):
         return importlib.import_module(f"{__name__}.{name}")
     abi = importlib.import_module(f"{__name__}.abi")  # loads libae.so; ImportError if it is missing
     return getattr(abi, name)

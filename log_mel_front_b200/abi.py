@@ -114,10 +114,12 @@ EXPORTS = ("ae_num_frames", "ae_num_tokens", "ae_model_create", "ae_model_destro
            "ae_device_status", "ae_version", "ae_profile_enable", "ae_profile_read", "ae_logmel_noalloc",
            "ae_resample_len", "ae_resample_workspace_size", "ae_resample", "ae_linear_e4m3",
            "ae_selftest_bounded_wait", "ae_lfm_default_config", "ae_lfm_num_frames", "ae_lfm_workspace_size",
-           "ae_lfm_logmel", "ae_launch_count", "ae_partition_clips")
+           "ae_lfm_logmel", "ae_launch_count", "ae_partition_clips", "ae_lenc_default_config", "ae_lenc_num_tokens",
+           "ae_lenc_create", "ae_lenc_destroy", "ae_lenc_workspace_size", "ae_lenc_block_workspace_size",
+           "ae_lenc_stem", "ae_lenc_block", "ae_lenc_encode")
 
 KERNEL_CLASSES = ("tables", "logmel", "conv0", "conv1", "gemm", "attention", "lconv", "rowop", "resample",
-                  "gemm_fp8", "lfm")
+                  "gemm_fp8", "lfm", "lenc_gemm", "lenc_attention", "lenc_row")
 
 
 class AEError(RuntimeError):
@@ -390,3 +392,136 @@ class Model:
             self.close()
         except Exception:
             pass
+
+
+# ------------------------------------------------------------------ LFM2A Conformer encoder
+
+class ae_lenc_config(C.Structure):
+    _fields_ = [(n, C.c_int32) for n in ("n_mels", "n_embd", "n_head", "n_layers", "n_ff", "conv_k", "stem_ch",
+                                        "adapter_ff", "llm_hidden")] + [("eps", C.c_float)]
+
+
+LENC_BLOCK_FIELDS = ("ffn1_norm_w", "ffn1_norm_b", "ffn1_up_w", "ffn1_up_b", "ffn1_down_w", "ffn1_down_b",
+                     "ln1_w", "ln1_b", "q_w", "q_b", "k_w", "k_b", "v_w", "v_b", "o_w", "o_b",
+                     "linear_pos_w", "pos_bias_u", "pos_bias_v",
+                     "norm_conv_w", "norm_conv_b", "pw1_w", "pw1_b", "dw_w", "dw_b", "conv_norm_w", "conv_norm_b",
+                     "pw2_w", "pw2_b",
+                     "ffn2_norm_w", "ffn2_norm_b", "ffn2_up_w", "ffn2_up_b", "ffn2_down_w", "ffn2_down_b",
+                     "ln2_w", "ln2_b")
+
+
+def _lenc_key(field: str) -> str:
+    """The weight-dict key (synth.lfm_encoder_weights) of a block field."""
+    if field.startswith(("ffn1_", "ffn2_")):
+        return field[:4] + "." + field[5:]
+    if field[:2] in ("q_", "k_", "v_", "o_") and len(field) == 3:
+        return "attn_" + field
+    if field in ("pw1_w", "pw1_b", "dw_w", "dw_b", "pw2_w", "pw2_b"):
+        return "conv_" + field
+    return field
+
+
+class ae_lenc_host_block(C.Structure):
+    _fields_ = [(n, _fp) for n in LENC_BLOCK_FIELDS]
+
+
+class ae_lenc_host_weights(C.Structure):
+    _fields_ = [("stem_w", _fp * 5), ("stem_b", _fp * 5), ("pre_w", _fp), ("pre_b", _fp),
+                ("blocks", C.POINTER(ae_lenc_host_block)),
+                ("ad_norm_w", _fp), ("ad_norm_b", _fp), ("ad_up_w", _fp), ("ad_up_b", _fp),
+                ("ad_down_w", _fp), ("ad_down_b", _fp)]
+
+
+_sig("ae_lenc_default_config", None, C.POINTER(ae_lenc_config))
+_sig("ae_lenc_num_tokens", C.c_int64, C.c_int64)
+_sig("ae_lenc_create", _st, C.POINTER(ae_lenc_config), C.POINTER(ae_lenc_host_weights), C.POINTER(_vp))
+_sig("ae_lenc_destroy", None, _vp)
+_sig("ae_lenc_workspace_size", _sz, _vp, _i64p, _i32)
+_sig("ae_lenc_block_workspace_size", _sz, _vp, _i64p, _i32)
+_sig("ae_lenc_stem", _st, _vp, _vp, _i64p, _i32, _vp, _vp, _sz, _vp)
+_sig("ae_lenc_block", _st, _vp, _i32, _vp, _i64p, _i32, _vp, _sz, _vp)
+_sig("ae_lenc_encode", _st, _vp, _vp, _i64p, _i32, _vp, _vp, _sz, _vp)
+
+
+def lenc_config(**kw) -> "ae_lenc_config":
+    """The library's defaults (ae_lenc_default_config) with the given fields replaced."""
+    c = ae_lenc_config()
+    lib.ae_lenc_default_config(C.byref(c))
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+def ae_lenc_num_tokens(n_frames: int) -> int:
+    return lib.ae_lenc_num_tokens(int(n_frames))
+
+
+class LencModel:
+    """An ae_lenc built from a weight dict in the page's layouts
+    (``synth.lfm_encoder_weights`` produces one)."""
+
+    def __init__(self, W: dict):
+        s = W["cfg"]
+        cfg = lenc_config(**{k: s[k] for k in ("n_mels", "n_embd", "n_head", "n_layers", "n_ff", "conv_k", "stem_ch",
+                                               "adapter_ff", "llm_hidden", "eps")})
+        keep = []
+
+        def fp(a):
+            a = _f32(a)
+            keep.append(a)
+            return a.ctypes.data_as(_fp)
+
+        L = len(W["layers"])
+        blocks = (ae_lenc_host_block * max(L, 1))()
+        for i, ly in enumerate(W["layers"]):
+            for f in LENC_BLOCK_FIELDS:
+                setattr(blocks[i], f, fp(ly[_lenc_key(f)]))
+        w = ae_lenc_host_weights()
+        for i in range(5):
+            w.stem_w[i] = fp(W[f"stem{i}.w"])
+            w.stem_b[i] = fp(W[f"stem{i}.b"])
+        w.pre_w, w.pre_b = fp(W["pre_w"]), fp(W["pre_b"])
+        w.blocks = blocks
+        for k in ("ad_norm_w", "ad_norm_b", "ad_up_w", "ad_up_b", "ad_down_w", "ad_down_b"):
+            setattr(w, k, fp(W[k]))
+        h = C.c_void_p()
+        _check(lib.ae_lenc_create(C.byref(cfg), C.byref(w), C.byref(h)), "ae_lenc_create")
+        self.handle = h.value
+        self.cfg = dict(s)
+
+    def workspace_size(self, frame_off) -> int:
+        a, p = _off(frame_off)
+        return lib.ae_lenc_workspace_size(self.handle, p, len(a) - 1)
+
+    def block_workspace_size(self, tok_off) -> int:
+        a, p = _off(tok_off)
+        return lib.ae_lenc_block_workspace_size(self.handle, p, len(a) - 1)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lib.ae_lenc_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def ae_lenc_stem(model, d_mel, frame_off, d_x, d_ws, ws_bytes: int, stream=None):
+    a, p = _off(frame_off)
+    _check(lib.ae_lenc_stem(model.handle, _ptr(d_mel), p, len(a) - 1, _ptr(d_x), _ptr(d_ws), ws_bytes,
+                            _stream(stream)), "ae_lenc_stem")
+
+
+def ae_lenc_block(model, layer: int, d_x, tok_off, d_ws, ws_bytes: int, stream=None):
+    a, p = _off(tok_off)
+    _check(lib.ae_lenc_block(model.handle, int(layer), _ptr(d_x), p, len(a) - 1, _ptr(d_ws), ws_bytes,
+                             _stream(stream)), "ae_lenc_block")
+
+
+def ae_lenc_encode(model, d_mel, frame_off, d_out, d_ws, ws_bytes: int, stream=None):
+    a, p = _off(frame_off)
+    _check(lib.ae_lenc_encode(model.handle, _ptr(d_mel), p, len(a) - 1, _ptr(d_out), _ptr(d_ws), ws_bytes,
+                              _stream(stream)), "ae_lenc_encode")

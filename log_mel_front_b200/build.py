@@ -16,8 +16,9 @@ CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libae.so")
 ROOT = os.path.dirname(HERE)
-SOURCES = ["api.cu", "gemm.cu", "logmel.cu", "stem.cu", "attention.cu", "rowops.cu", "resample.cu", "lfm.cu"]
-HEADERS = ["common.cuh", "ae_internal.h", "fft16.cuh", "e4m3_host.h", "lfm_host.h"]
+SOURCES = ["api.cu", "gemm.cu", "logmel.cu", "stem.cu", "attention.cu", "rowops.cu", "resample.cu", "lfm.cu",
+           "lenc.cu", "lenc_attention.cu", "lenc_api.cu"]
+HEADERS = ["common.cuh", "ae_internal.h", "fft16.cuh", "e4m3_host.h", "lfm_host.h", "htk_bank.h"]
 
 NVCC = os.environ.get("NVCC", "nvcc")
 FLAGS = [

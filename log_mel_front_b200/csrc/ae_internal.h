@@ -9,6 +9,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <type_traits>
 #include <string>
 #include <vector>
 
@@ -42,6 +43,11 @@ enum EpiMode : int {
   EPI_GLU = 3,        // columns (2c, 2c+1) -> clamp, a * sigmoid(b) -> act column c
   EPI_ADD_F32 = 4,    // out += clamp(acc): a float residual update, one add per element
   EPI_SILU_Q8 = 5,    // v = clamp2(silu(clamp(acc))) -> e4m3 code of v * q8 (the next projection's operand)
+  EPI_BIAS_BF16 = 6,     // v = clamp(acc + bias) -> bf16
+  EPI_BIAS_SILU = 7,     // v = silu(acc + bias) -> bf16
+  EPI_BIAS_GLU = 8,      // columns (2c, 2c+1) + bias -> a * sigmoid(b) -> bf16 column c
+  EPI_BIAS_GELU = 9,     // v = gelu_erf(acc + bias) -> bf16
+  EPI_BIAS_ADD_F32 = 10, // out += alpha * (acc + bias): a float residual update
 };
 
 struct EpiArgs {
@@ -55,6 +61,7 @@ struct EpiArgs {
   float seg_lo[3], seg_hi[3];
   const float *cs;    // e4m3 projections: [N] factor of each accumulator column (weight row scale / q8 of x)
   float q8;           // EPI_SILU_Q8: scale of the e4m3 output codes
+  float alpha;        // EPI_BIAS_ADD_F32: weight of the update
 };
 
 // Device copy of one layer.
@@ -134,7 +141,7 @@ struct WsLayout {
   size_t total = 0;
 };
 
-constexpr int kMelTile = 64;       // frames per log-mel work item
+constexpr int kMelTile = 32;       // frames per log-mel work item
 constexpr int kConv1TileTok = 4;   // tokens per conv1 tile (4 x 32 frequency rows = 128 GEMM rows)
 
 WsLayout ws_layout(const ae_model *m, int64_t n_clips, int64_t frames, int64_t tokens, bool with_model);
@@ -272,6 +279,54 @@ struct LfmParams {
 };
 size_t lfm_smem_bytes(int hop);
 cudaError_t launch_lfm(const float *wave, float *out, const LfmTablesDev &t, const LfmParams &prm, cudaStream_t s);
+
+// LFM2A Conformer encoder (lenc.cu, lenc_attention.cu): the shape the kernels
+// are compiled for, per-call clip tables in the workspace and the arguments
+// of the LayerNorm pass.
+constexpr int kLencMels = 128;    // mel bands in
+constexpr int kLencEmbd = 512;    // model width
+constexpr int kLencHeads = 8;     // heads of 64
+constexpr int kLencStemCh = 256;  // stem channels
+constexpr int kLencMaxTok = 4096; // rows after the stem per clip
+constexpr int kLencMaxConvK = 33; // depthwise conv taps
+struct LencTablesDev {
+  int n_clips;
+  const int32_t *frame_off;  // [B + 1] mel frames
+  const int32_t *s2_off;     // [B + 1] rows after the first two stem convolutions
+  const int32_t *tok_off;    // [B + 1] rows after the stem (tokens)
+  const int32_t *qblk_off;   // [B + 1] 128-token query blocks
+};
+struct LencLnArgs {
+  float *x; int64_t rows; float eps;
+  const float *w1, *b1; int write_x;
+  const float *w2, *b2;  // optional second LayerNorm for the operand
+  bf16 *a;               // optional bf16 operand out
+};
+cudaError_t launch_lenc_stem01(const float *mel, const float *w0, const float *b0, const float *w1, const float *b1,
+                               void *y2, const LencTablesDev &t, int64_t s2_rows, cudaStream_t s);
+cudaError_t launch_lenc_dw2(const void *y, const float *w, const float *b, void *out, const LencTablesDev &t,
+                            int64_t tokens, cudaStream_t s);
+cudaError_t launch_lenc_ln(const LencLnArgs &r, cudaStream_t s);
+cudaError_t launch_lenc_dwconv(const void *g, const float *w, const float *db, const float *aw, const float *ab, int k,
+                               void *out, const int32_t *tok_off, int n_clips, int64_t T, cudaStream_t s);
+cudaError_t launch_lenc_relpos(void *pe, int t_max, cudaStream_t s);
+cudaError_t launch_lenc_xlattn(const void *qkv, int64_t T, const void *ptab, int64_t p_rows, int64_t p_cols, int p_col,
+                               const float *bias_u, const float *bias_v, const int32_t *tok_off,
+                               const int32_t *qblk_off, int n_clips, int n_qblk, int t_max, void *out,
+                               cudaStream_t s);
+// bf16 GEMM for callers without an ae_model: y = epilogue(x W^T), x [M][K]
+// bf16, W given by its tensor map ([N][K] bf16).
+cudaError_t gemm_bf16(const void *x, int64_t M, int K, const CUtensorMap &tmW, int N, int mode, const EpiArgs &ep,
+                      cudaStream_t s);
+
+// Runs fn(ctx), which enqueues kernels on s, inside a kernel-timing record of
+// class cls with its algorithmic flops and bytes (ae_profile_enable).
+cudaError_t profiled(int cls, double flops, double bytes, cudaStream_t s, cudaError_t (*fn)(void *), void *ctx);
+template <class F>
+inline cudaError_t profiled_f(int cls, double flops, double bytes, cudaStream_t s, F &&f) {
+  return profiled(cls, flops, bytes, s, [](void *c) { return (*static_cast<std::remove_reference_t<F> *>(c))(); },
+                  &f);
+}
 
 unsigned *device_status_word();
 cudaError_t launch_wait_probe(unsigned long long limit_ns, int arrive, cudaStream_t s);

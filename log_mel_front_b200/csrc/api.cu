@@ -78,6 +78,11 @@ static cudaError_t timed(int cls, double flops, double bytes, cudaStream_t s, F 
   return e;
 }
 
+// The timing record for callers outside this file (the LFM2A encoder).
+cudaError_t profiled(int cls, double flops, double bytes, cudaStream_t s, cudaError_t (*fn)(void *), void *ctx) {
+  return timed(cls, flops, bytes, s, [&] { return fn(ctx); });
+}
+
 static size_t act_bytes(const ae_model *m) { return m->dtype == AE_F32 ? 4 : 2; }
 
 // A projection with its algorithmic flops (2 M N K) and bytes (x, W, y once).

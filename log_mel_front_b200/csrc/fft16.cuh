@@ -6,8 +6,10 @@
 
 namespace ae {
 
-__device__ __forceinline__ float2 cadd(float2 a, float2 b) { return make_float2(a.x + b.x, a.y + b.y); }
-__device__ __forceinline__ float2 csub(float2 a, float2 b) { return make_float2(a.x - b.x, a.y - b.y); }
+// complex add and subtract on the packed two-lane float32 pipe (one
+// instruction each; the subtraction as a fused multiply-add by -1, exact)
+__device__ __forceinline__ float2 cadd(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 csub(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.f, -1.f), a); }
 __device__ __forceinline__ float2 cmul(float2 a, float2 w) {
   return make_float2(fmaf(a.x, w.x, -a.y * w.y), fmaf(a.x, w.y, a.y * w.x));
 }
@@ -17,8 +19,9 @@ __device__ __forceinline__ void dft4(float2 &a0, float2 &a1, float2 &a2, float2 
   const float2 s02 = cadd(a0, a2), d02 = csub(a0, a2), s13 = cadd(a1, a3), d13 = csub(a1, a3);
   a0 = cadd(s02, s13);
   a2 = csub(s02, s13);
-  a1 = make_float2(d02.x + d13.y, d02.y - d13.x);  // d02 - i d13
-  a3 = make_float2(d02.x - d13.y, d02.y + d13.x);  // d02 + i d13
+  const float2 q = make_float2(d13.y, -d13.x);    // -i d13
+  a1 = cadd(d02, q);                               // d02 - i d13
+  a3 = csub(d02, q);                               // d02 + i d13
 }
 
 // 16-point DFT in registers, natural order in and out: x[k] <- sum_n x[n] W16^(n k).

@@ -109,8 +109,8 @@ __device__ __forceinline__ float2 mul_sigmoid2(float2 c, float2 g) {
 // col + 32) of one row: clamp (after the bias for EPI_F32), written as the 8
 // granules g0 .. g0 + 7 of the row's staging line.
 template <bool SC>
-__device__ __forceinline__ void epi_stage_f32(const EpiArgs &ep, bool bias, int col, const uint32_t (&r)[32],
-                                              uint8_t *line, int r7, int g0) {
+__device__ __forceinline__ void epi_stage_f32(const EpiArgs &ep, bool bias, float alpha, int col,
+                                              const uint32_t (&r)[32], uint8_t *line, int r7, int g0) {
   float lo = ep.lo, hi = ep.hi;
   if (ep.seg_w > 0) {
     const int sg = col / ep.seg_w;  // selects, not a runtime index into the parameter array
@@ -124,6 +124,10 @@ __device__ __forceinline__ void epi_stage_f32(const EpiArgs &ep, bool bias, int 
   if (bias) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] += __ldg(ep.bias + col + i);
+  }
+  if (alpha != 1.0f) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] *= alpha;
   }
 #pragma unroll
   for (int j = 0; j < 8; ++j)
@@ -156,8 +160,37 @@ __device__ __forceinline__ void epi_store32(const EpiArgs &ep, int row, int col,
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
   if (SC) scale_cols(ep.cs + col, v);
-  static_assert(MODE != EPI_F32 && MODE != EPI_ADD_F32, "float32 outputs go through the staging boxes");
-  if (MODE == EPI_GLU) {
+  static_assert(MODE != EPI_F32 && MODE != EPI_ADD_F32 && MODE != EPI_BIAS_ADD_F32,
+                "float32 outputs go through the staging boxes");
+  // the bias modes add the column bias, then take the path of their plain mode
+  // (GELU has its own)
+  constexpr bool BIAS = MODE == EPI_BIAS_BF16 || MODE == EPI_BIAS_SILU || MODE == EPI_BIAS_GLU || MODE == EPI_BIAS_GELU;
+  constexpr int BASE = MODE == EPI_BIAS_BF16 ? EPI_BF16
+                       : MODE == EPI_BIAS_SILU ? EPI_SILU
+                       : MODE == EPI_BIAS_GLU  ? EPI_GLU
+                                               : MODE;
+  if (BIAS) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float4 b = __ldg(reinterpret_cast<const float4 *>(ep.bias + col) + j);
+      v[4 * j] += b.x;
+      v[4 * j + 1] += b.y;
+      v[4 * j + 2] += b.z;
+      v[4 * j + 3] += b.w;
+    }
+  }
+  if (BASE == EPI_BIAS_GELU) {  // x (1 + erf(x / sqrt 2)) / 2
+    uint32_t p[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float a = v[2 * j], b = v[2 * j + 1];
+      p[j] = pack_bf16(0.5f * a * (1.0f + erff(a * 0.70710678118654752f)),
+                       0.5f * b * (1.0f + erff(b * 0.70710678118654752f)));
+    }
+    bf16 *o = static_cast<bf16 *>(ep.out) + (int64_t)row * ep.ld + col;
+    st_global_32B(o, p[0], p[1], p[2], p[3], p[4], p[5], p[6], p[7]);
+    st_global_32B(o + 16, p[8], p[9], p[10], p[11], p[12], p[13], p[14], p[15]);
+  } else if (BASE == EPI_GLU) {
     uint32_t p[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {  // columns (4j, 4j+1, 4j+2, 4j+3) = (a, b, a, b)
@@ -168,7 +201,7 @@ __device__ __forceinline__ void epi_store32(const EpiArgs &ep, int row, int col,
     }
     bf16 *o = static_cast<bf16 *>(ep.out) + (int64_t)row * ep.ld + col / 2;
     st_global_32B(o, p[0], p[1], p[2], p[3], p[4], p[5], p[6], p[7]);
-  } else if (MODE == EPI_SILU || MODE == EPI_SILU_Q8) {
+  } else if (BASE == EPI_SILU || BASE == EPI_SILU_Q8) {
     float2 y[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
@@ -225,7 +258,9 @@ constexpr int GEMM_THREADS = 64 + 32 * EPI_WARPS;
 // 4-stage ring; the other epilogues store from registers and take 6 stages,
 // which keeps more loads in flight (the e4m3 mainloop consumes a stage in half
 // the time of a bf16 one).
-__host__ __device__ constexpr bool f32_out(int mode) { return mode == EPI_F32 || mode == EPI_ADD_F32; }
+__host__ __device__ constexpr bool f32_out(int mode) {
+  return mode == EPI_F32 || mode == EPI_ADD_F32 || mode == EPI_BIAS_ADD_F32;
+}
 __host__ __device__ constexpr int stages_of(int mode) { return f32_out(mode) ? 4 : 6; }
 __host__ __device__ constexpr size_t smem_of(int mode) {
   return stages_of(mode) * STAGE_BYTES + (f32_out(mode) ? EPI_BYTES : 0) + 1024 + 256;
@@ -379,7 +414,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     // swizzle: conflict-free), which the warp reads back row by row to write 4
     // full 128-byte row segments per store instruction (measured faster for
     // f32, slower for bf16, than the direct sector stores).
-    constexpr bool F32_OUT = MODE == EPI_F32 || MODE == EPI_ADD_F32;
+    constexpr bool F32_OUT = f32_out(MODE);
     // float32 staging: one 32-column TMEM load fills a box row (128 bytes)
     constexpr int LOADS_PER_BOX = 1, OUT_COLS_PER_BOX = 32, GRANULES_PER_LOAD = 8, ES = 4;
     const int q = warp & 3, half = (warp - 2) >> 2;
@@ -398,14 +433,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       tc_fence_after();
       const int row0 = mb * 2 * BM + (int)rank * BM + q * 32;
       const int col0 = nb * BN + half * (BN / 2);
-      const int ocol0 = MODE == EPI_GLU ? col0 / 2 : col0;
+      const int ocol0 = (MODE == EPI_GLU || MODE == EPI_BIAS_GLU) ? col0 / 2 : col0;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + half * (BN / 2));
       auto stage = [&](int c, const uint32_t(&r)[32]) {
         if constexpr (!F32_OUT) {  // bf16 / e4m3 rows: 32-byte stores straight from registers
           if (row0 + lane < M) epi_store32<MODE, F8>(ep, row0 + lane, col0 + c * 32, r);
         } else {
           const int j = c % LOADS_PER_BOX;
-          epi_stage_f32<F8>(ep, MODE == EPI_F32 && ep.bias, col0 + c * 32, r, box + lane * 128, lane & 7,
+          epi_stage_f32<F8>(ep, (MODE == EPI_F32 || MODE == EPI_BIAS_ADD_F32) && ep.bias,
+                            MODE == EPI_BIAS_ADD_F32 ? ep.alpha : 1.0f, col0 + c * 32, r, box + lane * 128, lane & 7,
                             j * GRANULES_PER_LOAD);
           if (j == LOADS_PER_BOX - 1) {
             __syncwarp();
@@ -419,7 +455,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
               const uint4 v = *reinterpret_cast<const uint4 *>(box + rr * 128 + ((g ^ (rr & 7)) << 4));
               if (row0 + rr < M) {
                 uint8_t *p = dst + (int64_t)(row0 + rr) * ep.ld * ES;
-                if (MODE == EPI_ADD_F32)  // one vector add per 4 elements; no other thread touches them
+                if (MODE == EPI_ADD_F32 || MODE == EPI_BIAS_ADD_F32)  // one vector add per 4 elements; no other thread touches them
                   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(__uint_as_float(v.x)),
                                "f"(__uint_as_float(v.y)), "f"(__uint_as_float(v.z)), "f"(__uint_as_float(v.w))
                                : "memory");
@@ -646,6 +682,24 @@ cudaError_t gemm(const ae_model *m, const void *x, int64_t M, int K, const void 
     case EPI_BF16: return launch_f32<EPI_BF16>(xf, wf, ep, (int)M, N, K, s);
     case EPI_SILU: return launch_f32<EPI_SILU>(xf, wf, ep, (int)M, N, K, s);
     case EPI_GLU: return launch_f32<EPI_GLU>(xf, wf, ep, (int)M, N, K, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t gemm_bf16(const void *x, int64_t M, int K, const CUtensorMap &tmW, int N, int mode, const EpiArgs &ep,
+                      cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  if (K % BK || N % BN || M > INT32_MAX) return cudaErrorInvalidValue;
+  CUtensorMap tA;
+  if (!make_tmap_2d_bf16(&tA, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK, BM)) return cudaErrorInvalidValue;
+  switch (mode) {
+    case EPI_F32: return launch_tc<EPI_F32>(tA, tmW, ep, (int)M, N, K, s);
+    case EPI_BF16: return launch_tc<EPI_BF16>(tA, tmW, ep, (int)M, N, K, s);
+    case EPI_BIAS_BF16: return launch_tc<EPI_BIAS_BF16>(tA, tmW, ep, (int)M, N, K, s);
+    case EPI_BIAS_SILU: return launch_tc<EPI_BIAS_SILU>(tA, tmW, ep, (int)M, N, K, s);
+    case EPI_BIAS_GLU: return launch_tc<EPI_BIAS_GLU>(tA, tmW, ep, (int)M, N, K, s);
+    case EPI_BIAS_GELU: return launch_tc<EPI_BIAS_GELU>(tA, tmW, ep, (int)M, N, K, s);
+    case EPI_BIAS_ADD_F32: return launch_tc<EPI_BIAS_ADD_F32>(tA, tmW, ep, (int)M, N, K, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -1,0 +1,326 @@
+// Self-attention with a Transformer-XL relative-position bias, over whole
+// clips (cera 0.5.3, audio_encoder_gpu.rs: the `xl_attention` op of the LFM2A
+// Conformer): per head, score(i, j) = ((q_i + u) . k_j + (q_i + v) .
+// p_{i - j}) / sqrt(64), softmax over the keys j of the clip, out_i =
+// sum_j softmax * v_j. p_r is the projected position row of relative
+// distance r; the table holds r = t_max - 1 .. -(t_max - 1) top to bottom,
+// so row (t_max - 1 - r) is distance r.
+//
+// One CTA per (clip, 128-query block, head); warp 0 loads tiles with TMA,
+// warp 1 issues tcgen05.mma, warps 2-5 own one query row per thread. Per
+// 128-key block:
+//   * TMA: the 128 key rows and value rows of the block, and the 256 position
+//     rows of the distances the block spans (r = i - j from i0 - j0 - 127 to
+//     i0 - j0 + 127; rows outside the table are zero-filled);
+//   * S = (q + u) K^T (M=128, N=128) and T = (q + v) Pband^T (M=128, N=256)
+//     into tensor memory; (q + u) and (q + v) are written once, as bf16, by
+//     the row threads;
+//   * the row thread of query li needs T[li][127 - li + lj] for key lj: a
+//     window that starts one column earlier per row. It loads the two 32-column
+//     chunks of T that cover its window for 32 keys, writes them into its row
+//     of a per-warp scratch (row pitch 66 floats) and reads them back from
+//     offset 31 - lane (conflict-free: 65 lane + const); then adds S, scales
+//     and masks keys past the clip end, 32 keys at a time;
+//   * two passes over the key blocks: the first keeps each row's running
+//     maximum and sum of exponentials (rescaled as the maximum grows); the
+//     second recomputes the logits, writes the normalised probabilities as
+//     bf16 (K-major, 128-byte swizzle) and tcgen05.mma accumulates P V
+//     (M=128, N=64, V read MN-major) in tensor memory over the blocks, which
+//     the row thread reads once at the end. The second pass costs one more
+//     score MMA and skew per block, and keeps the row threads' registers to the
+//     96 of one chunk (no output accumulator, no rescale of it).
+// Every wait is bounded and reports through the library's status word.
+#include "ae_internal.h"
+#include "common.cuh"
+
+namespace ae {
+
+namespace {
+constexpr int XA_Q = 128, XA_K = 128, XA_HD = 64;
+constexpr uint32_t XA_TILE = 128 * 128;               // 128 rows x 64 bf16
+constexpr uint32_t OFF_QU = 0, OFF_QV = OFF_QU + XA_TILE, OFF_K = OFF_QV + XA_TILE, OFF_V = OFF_K + XA_TILE;
+constexpr uint32_t OFF_PB = OFF_V + XA_TILE;             // 256 position rows
+constexpr uint32_t OFF_S = OFF_PB + 2 * XA_TILE;         // probabilities: two 64-key regions
+constexpr uint32_t OFF_SCR = OFF_S + 2 * XA_TILE;        // skew scratch, 4 warps x 32 rows x 66 floats
+constexpr int SCR_PITCH = 66;
+constexpr uint32_t OFF_BAR = OFF_SCR + 4 * 32 * SCR_PITCH * 4;
+constexpr size_t XA_SMEM = OFF_BAR + 256 + 1024;
+constexpr int XA_THREADS = 192;
+constexpr uint32_t XA_TMEM_COLS = 512, COL_S = 0, COL_T = 128, COL_O = 384;
+constexpr uint32_t XA_KV_BYTES = 4 * XA_TILE;            // K, V and two position boxes
+static_assert(XA_SMEM <= 227 * 1024, "shared memory");
+static_assert(OFF_PB % 1024 == 0 && OFF_S % 1024 == 0 && OFF_SCR % 16 == 0, "swizzle atoms");
+}  // namespace
+
+__global__ void __launch_bounds__(XA_THREADS, 1)
+    k_lenc_xlattn(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmP,
+                  const float *__restrict__ bias_u, const float *__restrict__ bias_v,
+                  const int32_t *__restrict__ tok_off, const int32_t *__restrict__ qblk_off, int n_clips,
+                  int t_max, int p_col, bf16 *__restrict__ out, int ld_out, unsigned *status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sQu = smem + OFF_QU, *sQv = smem + OFF_QV, *sK = smem + OFF_K, *sV = smem + OFF_V, *sPb = smem + OFF_PB,
+          *sS = smem + OFF_S;
+  float *scr = reinterpret_cast<float *>(smem + OFF_SCR);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+  uint64_t *q_full = bars, *q_ready = bars + 1, *kv_full = bars + 2, *s_full = bars + 3, *s_free = bars + 4,
+           *p_full = bars + 5, *o_full = bars + 6;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 7);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // item -> (clip, query block, head)
+  const int head = blockIdx.x % kLencHeads, qitem = blockIdx.x / kLencHeads;
+  int c = 0;
+  {
+    int lo = 0, hi = n_clips;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (qblk_off[mid] <= qitem) lo = mid; else hi = mid;
+    }
+    c = lo;
+  }
+  const int tok0 = tok_off[c], t_c = tok_off[c + 1] - tok0;
+  const int i0 = (qitem - qblk_off[c]) * XA_Q;
+  const int n_kb = (t_c + XA_K - 1) / XA_K;
+
+  // rounds: n_kb of the first pass (K and position rows), then n_kb of the
+  // second (K, position rows and V)
+  const int n_rounds = 2 * n_kb;
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_ready, 128);
+    mbar_init(kv_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 128);
+    mbar_init(p_full, 128);
+    mbar_init(o_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmQKV);
+    tma_prefetch_desc(&tmP);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, XA_TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    bool ok = true;
+    mbar_arrive_expect_tx(q_full, XA_TILE);
+    tma_load_2d(sQu, &tmQKV, head * XA_HD, tok0 + i0, q_full);
+    int issued = 0;
+    for (int rd = 0; rd < n_rounds; ++rd) {
+      const bool second = rd >= n_kb;
+      const int kb = second ? rd - n_kb : rd;
+      // K and the position rows are free once the previous round's score MMAs
+      // have completed; V once the previous block's P V has
+      if (rd > 0 && !mbar_wait(s_full, (rd - 1) & 1)) { ok = false; break; }
+      if (second && kb > 0 && !mbar_wait(o_full, (kb - 1) & 1)) { ok = false; break; }
+      if (*abort_flag) break;
+      const int j0 = kb * XA_K;
+      const int prow = t_max - 128 - i0 + j0;  // table row of distance i0 - j0 + 127
+      mbar_arrive_expect_tx(kv_full, second ? XA_KV_BYTES : XA_KV_BYTES - XA_TILE);
+      tma_load_2d(sK, &tmQKV, kLencEmbd + head * XA_HD, tok0 + j0, kv_full);
+      tma_load_2d(sPb, &tmP, p_col + head * XA_HD, prow, kv_full);
+      tma_load_2d(sPb + XA_TILE, &tmP, p_col + head * XA_HD, prow + 128, kv_full);
+      if (second) tma_load_2d(sV, &tmQKV, 2 * kLencEmbd + head * XA_HD, tok0 + j0, kv_full);
+      ++issued;
+    }
+    if (!ok) {
+      atomicOr(status, kStatusWaitTimeout);
+      *abort_flag = 1;
+    }
+    mbar_wait(q_full, 0);
+    if (issued > 0) mbar_wait(kv_full, (issued - 1) & 1);  // every load lands before the CTA ends
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    constexpr uint32_t idesc_s = idesc_bf16_f32(XA_Q, XA_K);
+    constexpr uint32_t idesc_t = idesc_bf16_f32(XA_Q, 2 * XA_K);
+    constexpr uint32_t idesc_o = idesc_bf16_f32_bmn(XA_Q, XA_HD);
+    const uint32_t aqu = smem_u32(sQu), aqv = smem_u32(sQv), ak = smem_u32(sK), av = smem_u32(sV),
+                   apb = smem_u32(sPb), as = smem_u32(sS);
+    bool ok = mbar_wait(q_ready, 0);
+    for (int rd = 0; rd < n_rounds && ok; ++rd) {
+      const bool second = rd >= n_kb;
+      const int kb = second ? rd - n_kb : rd;
+      if (!mbar_wait(kv_full, rd & 1) || (rd > 0 && !mbar_wait(s_free, (rd - 1) & 1)) || *abort_flag) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int k = 0; k < XA_HD / 16; ++k)
+        tc_mma_bf16(tmem + COL_S, sw128_desc(aqu + k * 32), sw128_desc(ak + k * 32), idesc_s, k > 0 ? 1u : 0u);
+#pragma unroll
+      for (int k = 0; k < XA_HD / 16; ++k)
+        tc_mma_bf16(tmem + COL_T, sw128_desc(aqv + k * 32), sw128_desc(apb + k * 32), idesc_t, k > 0 ? 1u : 0u);
+      tc_commit(s_full);
+      if (!second) continue;
+      if (!mbar_wait(p_full, kb & 1) || *abort_flag) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int ks = 0; ks < XA_K / 16; ++ks)
+        tc_mma_bf16(tmem + COL_O, sw128_desc(as + (ks >> 2) * XA_TILE + (ks & 3) * 32),
+                    sw128_desc_mn(av + ks * 2048, XA_TILE), idesc_o, (kb | ks) != 0 ? 1u : 0u);
+      tc_commit(o_full);
+    }
+    if (!ok) {
+      atomicOr(status, kStatusWaitTimeout);
+      *abort_flag = 1;
+    }
+  } else if (warp >= 2) {
+    // ---------------- row threads: TMEM lane quarter qw, query row li = 32 qw + lane
+    const int qw = warp & 3, li = 32 * qw + lane, r7 = li & 7;
+    const uint32_t trow = tmem + ((uint32_t)(32 * qw) << 16);
+    float *my = scr + (size_t)(qw * 32 + lane) * SCR_PITCH;
+    bool ok = true;
+    // ---- q + u and q + v as bf16 operand tiles
+    if (!__all_sync(0xffffffffu, mbar_wait(q_full, 0))) ok = false;
+    if (ok) {
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        const uint32_t off = li * 128 + ((g ^ r7) << 4);
+        const uint4 w = *reinterpret_cast<const uint4 *>(sQu + off);
+        const float q[8] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y),
+                            bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w)};
+        const float4 u0 = *reinterpret_cast<const float4 *>(bias_u + head * XA_HD + 8 * g);
+        const float4 u1 = *reinterpret_cast<const float4 *>(bias_u + head * XA_HD + 8 * g + 4);
+        const float4 v0 = *reinterpret_cast<const float4 *>(bias_v + head * XA_HD + 8 * g);
+        const float4 v1 = *reinterpret_cast<const float4 *>(bias_v + head * XA_HD + 8 * g + 4);
+        *reinterpret_cast<uint4 *>(sQu + off) =
+            make_uint4(pack_bf16(q[0] + u0.x, q[1] + u0.y), pack_bf16(q[2] + u0.z, q[3] + u0.w),
+                       pack_bf16(q[4] + u1.x, q[5] + u1.y), pack_bf16(q[6] + u1.z, q[7] + u1.w));
+        *reinterpret_cast<uint4 *>(sQv + off) =
+            make_uint4(pack_bf16(q[0] + v0.x, q[1] + v0.y), pack_bf16(q[2] + v0.z, q[3] + v0.w),
+                       pack_bf16(q[4] + v1.x, q[5] + v1.y), pack_bf16(q[6] + v1.z, q[7] + v1.w));
+      }
+      fence_async_smem();
+    }
+    mbar_arrive(q_ready);
+    constexpr float kScale = 0.125f * 1.4426950408889634f;  // 1/sqrt(64), in base 2
+    float m_run = -INFINITY, l_run = 0.f, inv_l = 0.f;
+    for (int rd = 0; rd < n_rounds && ok; ++rd) {
+      const bool second = rd >= n_kb;
+      const int kb = second ? rd - n_kb : rd;
+      const int j0 = kb * XA_K;
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full, rd & 1))) { ok = false; break; }
+      // the previous block's P V has read the probabilities' buffer
+      if (second && kb > 0 && !__all_sync(0xffffffffu, mbar_wait(o_full, (kb - 1) & 1))) { ok = false; break; }
+      tc_fence_after();
+      if (second && kb == 0) inv_l = 1.0f / l_run;
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        uint32_t a[32], b[32], ac[32];
+        const int ca = 3 - qw + q;  // chunk of T holding column 127 - li + 32 q (or the next one)
+        tmem_ld32(trow + COL_T + 32 * ca, a);
+        tmem_ld32(trow + COL_T + 32 * (ca + 1), b);
+        tmem_ld32(trow + COL_S + 32 * q, ac);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          *reinterpret_cast<float2 *>(my + 2 * e) = make_float2(__uint_as_float(a[2 * e]), __uint_as_float(a[2 * e + 1]));
+          *reinterpret_cast<float2 *>(my + 32 + 2 * e) =
+              make_float2(__uint_as_float(b[2 * e]), __uint_as_float(b[2 * e + 1]));
+        }
+        __syncwarp();
+        float z[32];
+        float cm = -INFINITY;
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          const int j = j0 + 32 * q + x;
+          z[x] = j < t_c ? (__uint_as_float(ac[x]) + my[31 - lane + x]) * kScale : -INFINITY;
+          cm = fmaxf(cm, z[x]);
+        }
+        __syncwarp();
+        if (!second) {
+          const float m_new = fmaxf(m_run, cm);
+          float ls = 0.f;
+#pragma unroll
+          for (int x = 0; x < 32; ++x) ls += exp2f(z[x] - m_new);  // exp2(-inf) = 0
+          if (m_new != -INFINITY) {
+            l_run = l_run * exp2f(m_run - m_new) + ls;
+            m_run = m_new;
+          }
+        } else {
+          // probabilities of keys 32 q .. 32 q + 31: granules 4 q .. 4 q + 3 of the row
+#pragma unroll
+          for (int gg = 0; gg < 4; ++gg) {
+            const int g = 4 * q + gg;
+            float p[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) p[e] = exp2f(z[8 * gg + e] - m_run) * inv_l;
+            *reinterpret_cast<uint4 *>(sS + (g >> 3) * XA_TILE + li * 128 + (((g & 7) ^ r7) << 4)) = make_uint4(
+                pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]), pack_bf16(p[4], p[5]), pack_bf16(p[6], p[7]));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(s_free);  // this round's scores are read
+      if (second) {
+        fence_async_smem();
+        mbar_arrive(p_full);
+      }
+    }
+    if (ok && !__all_sync(0xffffffffu, mbar_wait(o_full, (n_kb - 1) & 1))) ok = false;
+    if (ok) {
+      tc_fence_after();
+      uint32_t o0[32], o1[32];
+      tmem_ld32(trow + COL_O, o0);
+      tmem_ld32(trow + COL_O + 32, o1);
+      tmem_ld_wait();
+      if (i0 + li < t_c) {
+        bf16 *orow = out + (int64_t)(tok0 + i0 + li) * ld_out + head * XA_HD;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          *reinterpret_cast<uint4 *>(orow + 8 * g) = make_uint4(
+              pack_bf16(__uint_as_float(o0[8 * g]), __uint_as_float(o0[8 * g + 1])),
+              pack_bf16(__uint_as_float(o0[8 * g + 2]), __uint_as_float(o0[8 * g + 3])),
+              pack_bf16(__uint_as_float(o0[8 * g + 4]), __uint_as_float(o0[8 * g + 5])),
+              pack_bf16(__uint_as_float(o0[8 * g + 6]), __uint_as_float(o0[8 * g + 7])));
+          *reinterpret_cast<uint4 *>(orow + 32 + 8 * g) = make_uint4(
+              pack_bf16(__uint_as_float(o1[8 * g]), __uint_as_float(o1[8 * g + 1])),
+              pack_bf16(__uint_as_float(o1[8 * g + 2]), __uint_as_float(o1[8 * g + 3])),
+              pack_bf16(__uint_as_float(o1[8 * g + 4]), __uint_as_float(o1[8 * g + 5])),
+              pack_bf16(__uint_as_float(o1[8 * g + 6]), __uint_as_float(o1[8 * g + 7])));
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      atomicOr(status, kStatusWaitTimeout);
+      *abort_flag = 1;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, XA_TMEM_COLS);
+  }
+}
+
+cudaError_t launch_lenc_xlattn(const void *qkv, int64_t T, const void *ptab, int64_t p_rows, int64_t p_cols, int p_col,
+                               const float *bias_u, const float *bias_v, const int32_t *tok_off,
+                               const int32_t *qblk_off, int n_clips, int n_qblk, int t_max, void *out,
+                               cudaStream_t s) {
+  if (n_qblk <= 0 || T <= 0) return cudaSuccess;
+  static std::atomic<uint64_t> attr{0};
+  if (const cudaError_t e = smem_attr(k_lenc_xlattn, XA_SMEM, attr)) return e;
+  CUtensorMap tq, tp;
+  if (!make_tmap_2d_bf16(&tq, qkv, 3 * kLencEmbd, (uint64_t)T, 3 * kLencEmbd * 2, 64, 128) ||
+      !make_tmap_2d_bf16(&tp, ptab, (uint64_t)p_cols, (uint64_t)p_rows, (uint64_t)p_cols * 2, 64, 128))
+    return cudaErrorInvalidValue;
+  return launch_k(k_lenc_xlattn, dim3((unsigned)(n_qblk * kLencHeads)), dim3(XA_THREADS), XA_SMEM, s, tq, tp, bias_u,
+                  bias_v, tok_off, qblk_off, n_clips, t_max, p_col, static_cast<bf16 *>(out), kLencEmbd,
+                  device_status_word());
+}
+
+}  // namespace ae

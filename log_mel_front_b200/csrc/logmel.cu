@@ -1,190 +1,253 @@
 // Log-mel front-end (egemma2_audio.rs, MelFrontend::log_mel), fused in one
 // kernel: framing with the 160-sample semicausal pad, periodic Hann window,
-// 512-point real FFT, magnitude, sparse 128-band HTK mel projection and
+// 512-point real FFT, magnitude, 128-band HTK mel projection and
 // ln(mel + 0.001).
 //
-// Work item: 64 consecutive frames of one clip. The CTA stages the
-// contiguous waveform span those frames cover (64*160 + 160 samples) in
-// shared memory with coalesced loads; 16 groups of 16 threads then take one
-// frame each. Per frame the 320 windowed samples are packed as 160 complex
-// values z[n] = x[2n] + i x[2n+1] (the other 96 are zero) and transformed
-// by a 256-point complex FFT in the four-step form 16 x 16: each thread does
-// a 16-point DFT in registers, multiplies by the W256 twiddles, the group
-// transposes through padded shared memory, and each thread does the second
-// 16-point DFT. The real spectrum follows from the usual split
-// X[k] = E[k] - i W512^k O[k] with E, O from Z[k] and conj(Z[256-k]). The
-// mel projection walks only each band's nonzero bins (at most 11, 506 in
-// all) instead of the dense 257 x 128 product.
+// Work item: 32 consecutive frames of one clip; one CTA of 256 threads per
+// item at a time, two CTAs per SM, persistent over the items. Per item:
 //
-// Tables (twiddles, window, mel bank) are built per CTA in float64 from
-// their definitions; CTAs are persistent, so this costs once per CTA.
+//  1. Staging. The contiguous waveform span of the 32 frames (33 x 160
+//     samples) is copied into shared memory with 4-byte cp.async (zero fill
+//     outside the clip, which is the semicausal pad and the clip end).
+//  2. Spectra: 16 groups of 16 threads, two frames per group. A frame's 320
+//     windowed samples are packed as 160 complex values z[n] = x[2n] +
+//     i x[2n+1] and transformed by a 256-point complex FFT in the four-step
+//     form 16 x 16: thread j does the DFT-16 over n1 of z[16 n1 + j] in
+//     registers (10 of its 16 inputs are nonzero), multiplies by W256^(j k1),
+//     the group transposes through a padded shared-memory tile, and thread j
+//     does the DFT-16 that yields Z[j + 16 k2]. The real spectrum follows from
+//     X[k] = A - i W512^k B and X[256 - k] = conj(A + i W512^k B), with
+//     A = Z[k] + conj Z[256 - k], B = Z[k] - conj Z[256 - k]: thread j takes
+//     the pairs of its k2 < 8, Z[256 - k] coming from thread 16 - j by one
+//     shuffle per pair (threads 0 and 8 hold both members). The window carries
+//     the split's factor 1/2. The 257 magnitudes go to a [frame][bin] tile.
+//  3. Bands: one frame per lane. Warp w computes the bands [kWarpBand[w],
+//     kWarpBand[w+1]) of the 32 frames as straight-line code with the HTK
+//     weights as literals (htk_bank.h, 506 multiply-adds per frame, split
+//     evenly over the warps), reading the magnitudes from the tile (odd row
+//     pitch: lane f reads row f without bank conflicts), then the log.
+//  4. Store: the [32][128] result leaves as whole contiguous rows.
+//
+// Per-thread constants (the window values and FFT twiddles it uses) are
+// computed once at kernel start in float32 (sincospif / cospif, within an
+// ulp or so of the float64 values). The log is ln(2) (e + log2(m)) for
+// x = m 2^e, m in [1, 2), with the hardware's lg2 on m, whose absolute error
+// there is about 2^-22: the result is within 1e-6 of ln(x) for the values
+// that occur (x >= 0.001).
 #include "ae_internal.h"
 #include "common.cuh"
 #include "fft16.cuh"
 
 namespace ae {
 
+// ln(acc + 0.001) for acc >= 0.
+__device__ __forceinline__ float log_floor_sum(float acc) {
+  const float x = acc + 1e-3f;
+  const int bits = __float_as_int(x);
+  const float e = (float)((bits >> 23) - 127);
+  const float m = __int_as_float((bits & 0x007FFFFF) | 0x3F800000);
+  float l2;
+  asm("lg2.approx.f32 %0, %1;" : "=f"(l2) : "f"(m));
+  return (e + l2) * 0.69314718055994531f;
+}
+
+}  // namespace ae
+
+#include "htk_bank.h"
+
+namespace ae {
+
 namespace {
-constexpr int kGroups = 16;                        // frames in flight per CTA
-constexpr int kThreads = kGroups * 16;             // 256
-constexpr int kWaveSpan = kMelTile * kHop + kHop;  // samples staged per work item
-constexpr int kMaxBins = 12;                       // bins per band (11 suffice), zero-padded
-constexpr int kPitch = 17;                         // padded row of the 16 x 16 transpose
+constexpr int kItem = kMelTile;                // frames per work item (32)
+constexpr int kThreads = 256;
+constexpr int kGroups = kThreads / 16;         // 16-thread FFT groups
+constexpr int kSpan = kItem * kHop + kHop;     // staged samples per item
+constexpr int kPitch = 17;                     // padded row of the 16 x 16 transpose (float2)
+constexpr int kMagPitch = 273;                 // odd: the band phase reads column k of 32 rows conflict-free
+constexpr int kOutPitch = 129;
+constexpr int kBins = kFft / 2 + 1;
+
+static_assert(kItem == 32 && kGroups * 2 == kItem, "one frame per lane in the band phase, two per FFT group");
 
 struct LogmelSmem {
-  float2 tw[kFft];                         // W512^m = (cos, -sin)(2 pi m / 512)
-  float win[kFrame];                       // Hann / 2 (the split's 1/2 folded in)
-  float wts[kMels][kMaxBins + 1];          // sparse mel bank, zero-padded (row pitch 13 against bank conflicts)
-  int band_lo[kMels];
-  float wave[kWaveSpan];
-  float2 xs[kGroups][kPitch * 16];         // per-group transpose / spectrum exchange
-  float mag[kGroups][kFft / 2 + 16];       // per-group magnitudes (zero tail for the padded mel loop)
-  int tile_clip, tile_f0, tile_nf;
+  float wave[kSpan];
+  union {
+    float2 xs[kGroups][16 * kPitch];           // per-group transpose tiles (spectra phase)
+    float out[kItem][kOutPitch];               // log-mel rows (band and store phases)
+  } u;
+  float mag[kItem][kMagPitch];
 };
+
+__device__ __forceinline__ void cp_async4(float *dst, const float *src, bool valid) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  const int n = valid ? 4 : 0;  // src-size 0: 4 zero bytes
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(d), "l"(src), "r"(n) : "memory");
+}
+
+struct Item {
+  int clip, f0, nf;
+};
+
+__device__ __forceinline__ Item item_of(const ClipTablesDev &t, int tile) {
+  int lo = 0, hi = t.n_clips;  // last clip c with mel_tile_off[c] <= tile
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (t.mel_tile_off[mid] <= tile) lo = mid; else hi = mid;
+  }
+  Item it;
+  it.clip = lo;
+  it.f0 = (tile - t.mel_tile_off[lo]) * kItem;
+  it.nf = min(kItem, t.frame_off[lo + 1] - t.frame_off[lo] - it.f0);
+  return it;
+}
+
+// W32^k2 = (cos, -sin)(2 pi k2 / 32), k2 < 8
+__device__ __forceinline__ float2 w32(int k2) {
+  constexpr float c[8] = {1.0f, 0.98078528040323043f, 0.92387953251128674f, 0.83146961230254524f,
+                          0.70710678118654752f, 0.55557023301960218f, 0.38268343236508977f,
+                          0.19509032201612825f};
+  return make_float2(c[k2], -c[(8 - k2) & 7] * (k2 != 0));
+}
+
+template <int W>
+__device__ __forceinline__ void band_phase(const LogmelSmem &S, LogmelSmem &D, int f) {
+  htk::bands<W>(S.mag[f], D.u.out[f]);
+}
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads, 2)
     k_logmel(const float *__restrict__ wave, float *__restrict__ mel, const ClipTablesDev t, int n_tiles) {
-  extern __shared__ uint8_t smem_raw[];
+  extern __shared__ __align__(16) uint8_t smem_raw[];
   LogmelSmem &S = *reinterpret_cast<LogmelSmem *>(smem_raw);
-  const int tid = threadIdx.x;
-
-  // ---- tables, float64 from their definitions
-  for (int m = tid; m < kFft; m += kThreads) {
-    double s, c;
-    sincospi((double)m / 256.0, &s, &c);  // angle 2 pi m / 512
-    S.tw[m] = make_float2((float)c, (float)-s);
-  }
-  for (int j = tid; j < kFrame; j += kThreads) S.win[j] = (float)(0.25 - 0.25 * cospi((double)j / 160.0));
-  if (tid < kMels) {
-    // HTK: 130 mel points over [mel(0), mel(8000)] (last point exact), bins at k * 31.25 Hz;
-    // band b is the triangle over [f_b, f_b+2]; only the bins inside it are visited
-    const double mel_hi = 2595.0 * log10(1.0 + 8000.0 / 700.0);
-    const double step = mel_hi / 129.0;
-    double f[3];
-    for (int i = 0; i < 3; ++i) {
-      const int p = tid + i;
-      const double mm = (p == 129) ? mel_hi : p * step;
-      f[i] = 700.0 * (pow(10.0, mm / 2595.0) - 1.0);
-    }
-    for (int q = 0; q < kMaxBins; ++q) S.wts[tid][q] = 0.f;
-    int lo = -1, n = 0;
-    const int k0 = max(0, (int)floor(f[0] / 31.25)), k1 = min(kFft / 2, (int)ceil(f[2] / 31.25));
-    for (int k = k0; k <= k1; ++k) {
-      const double fk = k * 31.25;
-      const double down = (fk - f[0]) / (f[1] - f[0]);
-      const double up = (f[2] - fk) / (f[2] - f[1]);
-      const double w = fmax(0.0, fmin(down, up));
-      if (w > 0.0 && n < kMaxBins) {
-        if (lo < 0) lo = k;
-        S.wts[tid][n++] = (float)w;
-      }
-    }
-    S.band_lo[tid] = lo < 0 ? 0 : lo;
-  }
-  for (int x = tid; x < kGroups * 16; x += kThreads) S.mag[x / 16][kFft / 2 + x % 16] = 0.f;
-
-  __syncthreads();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = tid >> 4, j = tid & 15;
   const unsigned gmask = 0xFFFFu << (16 * (g & 1));
-  float2 tw1[16];  // W256^(j k1): depends only on the thread
+
+  // ---- per-thread constants
+  float2 win[10];  // Hann / 2 at samples 32 n1 + 2 j and + 1 (the split's 1/2 folded in)
 #pragma unroll
-  for (int k1 = 0; k1 < 16; ++k1) tw1[k1] = S.tw[(2 * j * k1) & (kFft - 1)];
-  float2 *xs = S.xs[g];
-  float *mag = S.mag[g];
+  for (int n1 = 0; n1 < 10; ++n1) {
+    const int m = 32 * n1 + 2 * j;
+    win[n1] = make_float2(0.25f - 0.25f * cospif((float)m / 160.0f), 0.25f - 0.25f * cospif((float)(m + 1) / 160.0f));
+  }
+  float2 tw1[16];  // W256^(j k1) = W512^(2 j k1)
+#pragma unroll
+  for (int k1 = 0; k1 < 16; ++k1) {
+    float s, c;
+    sincospif((float)((2 * j * k1) & (kFft - 1)) / 256.0f, &s, &c);
+    tw1[k1] = make_float2(c, -s);
+  }
+  float2 wj;  // W512^j
+  {
+    float s, c;
+    sincospif((float)j / 256.0f, &s, &c);
+    wj = make_float2(c, -s);
+  }
 
-  for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-    __syncthreads();  // previous work item done with the staged wave
-    if (tid == 0) {
-      int lo = 0, hi = t.n_clips;  // last clip c with mel_tile_off[c] <= tile
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (t.mel_tile_off[mid] <= tile) lo = mid; else hi = mid;
-      }
-      const int nfr = t.frame_off[lo + 1] - t.frame_off[lo];
-      S.tile_clip = lo;
-      S.tile_f0 = (tile - t.mel_tile_off[lo]) * kMelTile;
-      S.tile_nf = min(kMelTile, nfr - S.tile_f0);
-    }
-    __syncthreads();
-    const int c = S.tile_clip, f0 = S.tile_f0, nf = S.tile_nf;
-    const int64_t s_begin = t.sample_off[c];
-    const int64_t n_samp = min(t.sample_off[c + 1] - s_begin, (int64_t)kMaxSamples);
-    // local sample i is clip sample (f0 - 1) * 160 + i
-    const int64_t first = (int64_t)(f0 - 1) * kHop;
-    const int span = nf * kHop + kHop;
+  int tile = blockIdx.x;
+  Item it = tile < n_tiles ? item_of(t, tile) : Item{0, 0, 0};
+  // ---- stage the first item
+  auto stage = [&](const Item &x) {
+    const int64_t s_begin = t.sample_off[x.clip];
+    const int64_t n_samp = min(t.sample_off[x.clip + 1] - s_begin, (int64_t)kMaxSamples);
+    const int64_t first = (int64_t)(x.f0 - 1) * kHop;  // local sample i is clip sample first + i
+    const int span = x.nf * kHop + kHop;
+    // local indices inside the clip: [lo, hi)
+    const int lo = (int)max((int64_t)0, -first), hi = (int)min((int64_t)span, n_samp - first);
+    const float *src = wave + s_begin + first;
     for (int i = tid; i < span; i += kThreads) {
-      const int64_t sidx = first + i;
-      S.wave[i] = (sidx >= 0 && sidx < n_samp) ? __ldg(wave + s_begin + sidx) : 0.0f;
+      const bool ok = i >= lo && i < hi;
+      cp_async4(S.wave + i, ok ? src + i : wave, ok);
     }
-    __syncthreads();
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  if (tile < n_tiles) stage(it);
 
-    for (int fi = g; fi < nf; fi += kGroups) {
+  for (; tile < n_tiles; tile += gridDim.x) {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();  // staged wave visible; the previous item's output rows are stored
+
+    // ---- spectra: frames g and g + 16 of the item
+    float2 *xs = S.u.xs[g];
+#pragma unroll 1
+    for (int fi = g; fi < it.nf; fi += kGroups) {
       const float *wv = S.wave + fi * kHop;
-      // ---- stage 1: z[16 n1 + j], n1 < 10 nonzero; DFT over n1
       float2 x[16];
 #pragma unroll
       for (int n1 = 0; n1 < 16; ++n1) {
         if (n1 < 10) {
-          const int m = 32 * n1 + 2 * j;
-          const float2 a = *reinterpret_cast<const float2 *>(wv + m);
-          const float2 w = *reinterpret_cast<const float2 *>(S.win + m);
-          x[n1] = make_float2(a.x * w.x, a.y * w.y);
+          const float2 a = *reinterpret_cast<const float2 *>(wv + 32 * n1 + 2 * j);
+          x[n1] = make_float2(a.x * win[n1].x, a.y * win[n1].y);
         } else {
           x[n1] = make_float2(0.f, 0.f);
         }
       }
       dft16(x);
 #pragma unroll
-      for (int k1 = 1; k1 < 16; ++k1) x[k1] = cmul(x[k1], tw1[k1]);  // W256^(j k1)
+      for (int k1 = 1; k1 < 16; ++k1) x[k1] = cmul(x[k1], tw1[k1]);
 #pragma unroll
       for (int k1 = 0; k1 < 16; ++k1) xs[k1 * kPitch + j] = x[k1];
       __syncwarp(gmask);
-      // ---- stage 2: thread j = k1 gathers over n2 and finishes
 #pragma unroll
       for (int n2 = 0; n2 < 16; ++n2) x[n2] = xs[j * kPitch + n2];
       dft16(x);  // x[k2] = Z[j + 16 k2]
-      __syncwarp(gmask);
+      // ---- real split: pairs (k, 256 - k), k = j + 16 k2, k2 < 8
+      float *mg = S.mag[fi];
+      const int partner = (lane & 16) | ((16 - j) & 15);
 #pragma unroll
-      for (int k2 = 0; k2 < 16; ++k2) xs[k2 * kPitch + j] = x[k2];
-      __syncwarp(gmask);
-      // ---- real split and magnitude: X[k] = (Z_k + conj Z_k') - i W512^k (Z_k - conj Z_k'), k' = 256 - k
-#pragma unroll
-      for (int k2 = 0; k2 < 16; ++k2) {
+      for (int k2 = 0; k2 < 8; ++k2) {
+        const float2 o = x[k2];
+        float2 mr;
+        mr.x = __shfl_sync(gmask, x[15 - k2].x, partner);
+        mr.y = __shfl_sync(gmask, x[15 - k2].y, partner);
+        if (j == 0) mr = x[(16 - k2) & 15];  // thread 0 pairs 16 k2 with 16 (16 - k2), k2 = 0 with itself
+        const float2 mc = make_float2(mr.x, -mr.y);  // conj Z[256 - k]
+        const float2 A = cadd(o, mc), B = csub(o, mc);
+        const float2 w = cmul(wj, w32(k2));  // W512^(j + 16 k2)
+        const float2 wb = cmul(B, w);
+        // P = i W B = (-Im, Re)
+        const float2 P = make_float2(-wb.y, wb.x);
+        const float2 x1 = csub(A, P), x2 = cadd(A, P);  // X[k], conj X[256 - k]
+        const float2 q1 = __fmul2_rn(x1, x1), q2 = __fmul2_rn(x2, x2);
+        const float m1 = q1.x + q1.y, m2 = q2.x + q2.y;
         const int k = j + 16 * k2;
-        float2 b;
-        if (j == 0) {
-          const int kk = (16 - k2) & 15;  // k' = 16 (16 - k2) mod 256
-          b = xs[kk * kPitch];
-        } else {
-          b = xs[(15 - k2) * kPitch + (16 - j)];
-        }
-        const float2 a = x[k2];
-        const float2 A = make_float2(a.x + b.x, a.y - b.y);
-        const float2 B = make_float2(a.x - b.x, a.y + b.y);
-        const float2 w = S.tw[k];  // (cos, -sin)
-        // -i (w B) = (Im(wB), -Re(wB))
-        const float wbr = fmaf(w.x, B.x, -w.y * B.y);
-        const float wbi = fmaf(w.x, B.y, w.y * B.x);
-        const float re = A.x + wbi, im = A.y - wbr;
-        const float m2 = fmaf(re, re, im * im);
-        mag[k] = m2 * rsqrtf(fmaxf(m2, 1e-37f));  // |X| (2 ulp), 0 for 0
-        if (k == 0) mag[kFft / 2] = fabsf(2.0f * (a.x - a.y));  // Nyquist: Re Z0 - Im Z0 (Z halved)
+        mg[k] = m1 * rsqrtf(fmaxf(m1, 1e-37f));  // |X| to about 2 ulp, 0 for 0
+        mg[kFft / 2 - k] = m2 * rsqrtf(fmaxf(m2, 1e-37f));
       }
-      __syncwarp(gmask);
-      // ---- mel bands j, j+16, ...: sparse dot, log, store
-      float *orow = mel + ((int64_t)t.frame_off[c] + f0 + fi) * kMels;
-#pragma unroll
-      for (int i = 0; i < kMels / 16; ++i) {
-        const int b = j + 16 * i;
-        const float *mg = mag + S.band_lo[b];
-        float acc = 0.f;
-#pragma unroll
-        for (int q = 0; q < kMaxBins; ++q) acc = fmaf(S.wts[b][q], mg[q], acc);
-        orow[b] = logf(acc + 1e-3f);
+      if (j == 0) {
+        // k = 128 is its own partner: |X[128]| = 2 |Z[128]|
+        const float m8 = fmaf(x[8].x, x[8].x, x[8].y * x[8].y);
+        mg[kFft / 4] = 2.0f * m8 * rsqrtf(fmaxf(m8, 1e-37f));
       }
-      __syncwarp(gmask);
+      __syncwarp(gmask);  // the tile is free for the next frame
     }
+    __syncthreads();  // magnitudes complete
+
+    // ---- bands: lane = frame
+    if (lane < it.nf) {
+      switch (warp) {
+        case 0: band_phase<0>(S, S, lane); break;
+        case 1: band_phase<1>(S, S, lane); break;
+        case 2: band_phase<2>(S, S, lane); break;
+        case 3: band_phase<3>(S, S, lane); break;
+        case 4: band_phase<4>(S, S, lane); break;
+        case 5: band_phase<5>(S, S, lane); break;
+        case 6: band_phase<6>(S, S, lane); break;
+        default: band_phase<7>(S, S, lane); break;
+      }
+    }
+    __syncthreads();  // rows complete; the staged wave is free
+
+    // ---- next item's staging overlaps this item's store
+    const Item cur = it;
+    const int next = tile + gridDim.x;
+    if (next < n_tiles) {
+      it = item_of(t, next);
+      stage(it);
+    }
+    float *orow = mel + ((int64_t)t.frame_off[cur.clip] + cur.f0) * kMels;
+    const int n = cur.nf * kMels;
+    for (int i = tid; i < n; i += kThreads) orow[i] = S.u.out[i >> 7][i & (kMels - 1)];
   }
 }
 

@@ -29,6 +29,17 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 constexpr float kEps = 1e-6f;
 
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // NV = width / 128: lane l holds columns (i * 32 + l) * 4 .. +3, i < NV. The
 // row's h and y are loaded first; the weight vectors are staged in shared
 // memory while those loads are in flight, so a row costs one memory round
@@ -144,7 +155,8 @@ cudaError_t launch_rowop(const ae_model *m, const RowArgs &r, cudaStream_t s) {
 // owns channels 4t .. 4t+3 for kLcRows consecutive rows: its 5 x 4 taps and
 // 4 norm weights stay in registers, as channel pairs for the packed two-lane
 // FMA, and it loads its 8-byte slice of the rows (plus the 4 before them),
-// one coalesced load per row. The conv outputs of its rows stay in registers.
+// one coalesced load per row. The conv outputs of its rows stay in registers;
+// SiLU runs on the packed two-lane pipe.
 // The per-row sums of squares are reduced across the warp with a butterfly
 // that halves the rows at every step (after it, lanes 4r .. 4r+3 hold row r),
 // then across the CTA's 8 warps once for all rows.
@@ -234,12 +246,17 @@ __global__ void __launch_bounds__(256) k_lconv(const ActT *__restrict__ gl, cons
   for (int r = 0; r < kLcRows; ++r) {
     const int64_t tok = t0 + r;
     if (tok >= T) break;
-    const float inv = s_inv[r];
-    const float y[4] = {c[r][0].x * inv * wn[0].x, c[r][0].y * inv * wn[0].y, c[r][1].x * inv * wn[1].x,
-                        c[r][1].y * inv * wn[1].y};
+    const float2 inv = make_float2(s_inv[r], s_inv[r]);
     float v[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) v[u] = clampf(__fdividef(y[u], 1.0f + __expf(-y[u])), lo, hi);
+    for (int h = 0; h < 2; ++h) {  // silu(y) = y / (1 + 2^(-y log2 e)), two channels per packed op
+      const float2 y = __fmul2_rn(c[r][h], __fmul2_rn(inv, wn[h]));
+      const float2 e = __fmul2_rn(y, make_float2(-1.4426950408889634f, -1.4426950408889634f));
+      const float2 d = __fadd2_rn(make_float2(ex2_approx(e.x), ex2_approx(e.y)), make_float2(1.0f, 1.0f));
+      const float2 sl = __fmul2_rn(y, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
+      v[2 * h] = clampf(sl.x, lo, hi);
+      v[2 * h + 1] = clampf(sl.y, lo, hi);
+    }
     store4(out + tok * kHidden + ch, v);
   }
 }

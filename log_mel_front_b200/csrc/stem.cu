@@ -40,15 +40,19 @@ __device__ __forceinline__ int clip_of(const int32_t *off, int n_clips, int64_t 
 
 // ------------------------------------------------------------------ conv0 + LN + ReLU
 
-// A CTA writes kConv0Rows stem rows (64 positions each). Phase 1: each of the
-// 256 positions gets its 9-sample patch (stored duplicated as (p, p) pairs)
-// and 1/sqrt(p^T C p + eps) in shared memory. Phase 2: thread (channel quad,
-// position phase) holds its four channels' taps, pre-multiplied by the
-// LayerNorm gains at model creation, in registers and walks the positions:
-// two packed FMAs per tap cover the four channels; relu(r * (w'' . p)) is the
-// normalised output (r > 0). Consecutive threads write consecutive channels
-// of one position, so every row is written with full coalesced segments.
-// Rows outside a clip's frames (the zero padding) come out as zeros.
+// A CTA writes kConv0Rows stem rows (64 positions each). Phase 1: four
+// threads locate the rows' clips; the three mel rows each stem row reads are
+// staged in shared memory (coalesced, with a zero band on either side); the
+// 45 distinct entries of the symmetric 9x9 covariance C sit in registers;
+// each of the 256 positions then gets its 9-sample patch (stored duplicated
+// as (p, p) pairs) and 1/sqrt(p^T C p + eps) in shared memory. Phase 2:
+// thread (channel quad, position phase) holds its four channels' taps,
+// pre-multiplied by the LayerNorm gains at model creation, in registers and
+// walks the positions: two packed FMAs per tap cover the four channels;
+// relu(r * (w'' . p)) is the normalised output (r > 0). Consecutive threads
+// write consecutive channels of one position, so every row is written with
+// full coalesced segments. Rows outside a clip's frames (the zero padding)
+// come out as zeros.
 constexpr int kConv0Rows = 4;
 
 template <typename OutT>
@@ -56,36 +60,60 @@ __global__ void __launch_bounds__(128) k_conv0(const float *__restrict__ mel, co
                                                const float *__restrict__ cov, OutT *__restrict__ y0,
                                                const ClipTablesDev t, int64_t stem_rows) {
   constexpr int P = kConv0Rows * kF1;  // positions per CTA
+  constexpr int MP = kMels + 2;        // staged mel row with a zero band on either side
   __shared__ __align__(16) float2 s_pp[P][10];
   __shared__ float s_r[P];
+  __shared__ float s_mel[kConv0Rows][3][MP];
+  __shared__ int64_t s_base[kConv0Rows];
+  __shared__ int s_ti[kConv0Rows], s_F[kConv0Rows];
   const int64_t row0 = (int64_t)blockIdx.x * kConv0Rows;
-  for (int i = threadIdx.x; i < P; i += blockDim.x) {
-    const int64_t row = row0 + i / kF1;
-    const int f = i % kF1;
-    float p[9];
-#pragma unroll
-    for (int k = 0; k < 9; ++k) p[k] = 0.f;
+  if (threadIdx.x < kConv0Rows) {
+    const int64_t row = row0 + threadIdx.x;
+    int ti = -1, F = 0;
+    int64_t base = 0;
     if (row < stem_rows) {
       const int c = clip_of(t.stem_off, t.n_clips, row);
-      const int ti = (int)(row - t.stem_off[c]) - 2;
-      const int F = t.frame_off[c + 1] - t.frame_off[c];
-      if (ti >= 0 && ti < (F + 1) / 2) {
-        const float *m = mel + (int64_t)t.frame_off[c] * kMels;
-#pragma unroll
-        for (int dt = 0; dt < 3; ++dt)
-#pragma unroll
-          for (int df = 0; df < 3; ++df) {
-            const int tr = 2 * ti + dt - 1, fr = 2 * f + df - 1;
-            if (tr >= 0 && tr < F && fr >= 0 && fr < kMels) p[dt * 3 + df] = __ldg(m + (int64_t)tr * kMels + fr);
-          }
-      }
+      F = t.frame_off[c + 1] - t.frame_off[c];
+      ti = (int)(row - t.stem_off[c]) - 2;
+      if (ti >= (F + 1) / 2) ti = -1;
+      base = (int64_t)t.frame_off[c] * kMels;
     }
+    s_ti[threadIdx.x] = ti;
+    s_F[threadIdx.x] = F;
+    s_base[threadIdx.x] = base;
+  }
+  // C_aa and 2 C_ab (b > a): p^T C p = sum_a p_a (C_aa p_a + sum_{b>a} 2 C_ab p_b)
+  float cv[45];
+  {
+    int n = 0;
+#pragma unroll
+    for (int a = 0; a < 9; ++a)
+#pragma unroll
+      for (int b = a; b < 9; ++b) cv[n++] = (b == a ? 1.0f : 2.0f) * __ldg(cov + a * 9 + b);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kConv0Rows * 3 * MP; i += blockDim.x) {
+    const int rr = i / (3 * MP), dt = (i / MP) % 3, cc = i % MP;
+    const int ti = s_ti[rr], tr = 2 * ti + dt - 1, fr = cc - 1;
+    float v = 0.f;
+    if (ti >= 0 && tr >= 0 && tr < s_F[rr] && fr >= 0 && fr < kMels) v = __ldg(mel + s_base[rr] + (int64_t)tr * kMels + fr);
+    s_mel[rr][dt][cc] = v;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < P; i += blockDim.x) {
+    const int rr = i / kF1, f = i % kF1;
+    float p[9];
+#pragma unroll
+    for (int dt = 0; dt < 3; ++dt)
+#pragma unroll
+      for (int df = 0; df < 3; ++df) p[dt * 3 + df] = s_mel[rr][dt][2 * f + df];  // column 2f + df - 1, shifted by the band
     float var = 0.f;
+    int n = 0;
 #pragma unroll
     for (int a = 0; a < 9; ++a) {
       float s = 0.f;
 #pragma unroll
-      for (int b = 0; b < 9; ++b) s = fmaf(__ldg(cov + a * 9 + b), p[b], s);
+      for (int b = a; b < 9; ++b) s = fmaf(cv[n++], p[b], s);
       var = fmaf(p[a], s, var);
     }
 #pragma unroll

@@ -264,3 +264,79 @@ def attention_qkv(seq: int, T: int = ATT_T, hidden: int = 1024) -> tuple[np.ndar
     """q, k, v of one sequence: [T, hidden] float32 holding bf16 values of N(0,1)."""
     r = _rng(WORKLOADS["attention"]["config_index"], 1 + seq)
     return tuple(round_to_bf16(r.standard_normal((T, hidden), dtype=np.float32)) for _ in range(3))
+
+
+# ----------------------------------------------------------------- LFM2A encoder body
+
+# The LFM2A Conformer encoder's shape as the library reads it (17 blocks of
+# width 512 with 8 heads; the other sizes are readings, the page names them
+# without values).
+LENC_SHAPE = dict(n_mels=128, n_embd=512, n_head=8, n_layers=17, n_ff=2048, conv_k=9, stem_ch=256,
+                  adapter_ff=2048, llm_hidden=2048, eps=1e-5)
+
+LENC_BLOCK_VECTORS = ("ffn1.norm_b", "ffn1.down_b", "ln1_b", "attn_q_b", "attn_k_b", "attn_v_b", "attn_o_b",
+                      "pos_bias_u", "pos_bias_v", "norm_conv_b", "conv_dw_b", "conv_norm_b", "conv_pw2_b",
+                      "ffn2.norm_b", "ffn2.down_b", "ln2_b")
+
+
+def lfm_encoder_weights(n_layers: int | None = None, shape: dict | None = None, seed: int = 5000) -> dict:
+    """Random-init weights of the LFM2A encoder body in the page's tensor
+    layouts (matrices [out, in], stem convolutions [C_out][C_in/groups][kh][kw],
+    the depthwise conv1d taps [k][C]). Stem convolutions and pre_encode_out
+    N(0, 1 / fan_in), so the activations keep their scale through the ReLUs;
+    block and adapter matrices N(0, 0.02); LayerNorm gains and the conv
+    module's channel scale 1 + N(0, 0.02); biases and the depthwise taps
+    N(0, 0.02) and N(0, 1 / k). Every matrix the tensor cores multiply (the
+    pointwise stem convolutions, pre_encode_out, the block and adapter
+    matrices, linear_pos) is rounded to bf16 here, so the bf16 values are the
+    model; vectors and the 3x3 stem taps stay float32."""
+    s = dict(LENC_SHAPE if shape is None else shape)
+    L = s["n_layers"] if n_layers is None else n_layers
+    s["n_layers"] = L
+    D, F, C, K = s["n_embd"], s["n_ff"], s["stem_ch"], s["conv_k"]
+    r = _rng(seed, 0)
+    W = {"cfg": s, "layers": []}
+    for i, (dw, k, cin) in enumerate(((False, 3, 1), (True, 3, C), (False, 1, C), (True, 3, C), (False, 1, C))):
+        fan = (1 if dw else cin) * k * k
+        w = _normal(r, (C, 1 if dw else cin, k, k), fan ** -0.5)
+        W[f"stem{i}.w"] = w if k == 3 else round_to_bf16(w)
+        W[f"stem{i}.b"] = _normal(r, (C,), 0.02)
+    fq = s["n_mels"] // 8
+    W["pre_w"] = round_to_bf16(_normal(r, (D, C * fq), (C * fq) ** -0.5))
+    W["pre_b"] = _normal(r, (D,), 0.02)
+    for l in range(L):
+        r = _rng(seed, 1 + l)
+        ly = {}
+        for f in ("ffn1", "ffn2"):
+            ly[f + ".norm_w"] = _normal(r, (D,), 0.02, 1.0)
+            ly[f + ".norm_b"] = _normal(r, (D,), 0.02)
+            ly[f + ".up_w"] = round_to_bf16(_normal(r, (F, D), 0.02))
+            ly[f + ".up_b"] = _normal(r, (F,), 0.02)
+            ly[f + ".down_w"] = round_to_bf16(_normal(r, (D, F), 0.02))
+            ly[f + ".down_b"] = _normal(r, (D,), 0.02)
+        for n in ("ln1", "ln2", "norm_conv"):
+            ly[n + "_w"] = _normal(r, (D,), 0.02, 1.0)
+            ly[n + "_b"] = _normal(r, (D,), 0.02)
+        for c in "qkvo":
+            ly[f"attn_{c}_w"] = round_to_bf16(_normal(r, (D, D), 0.02))
+            ly[f"attn_{c}_b"] = _normal(r, (D,), 0.02)
+        ly["linear_pos_w"] = round_to_bf16(_normal(r, (D, D), 0.02))
+        ly["pos_bias_u"] = _normal(r, (D,), 0.02)
+        ly["pos_bias_v"] = _normal(r, (D,), 0.02)
+        ly["conv_pw1_w"] = round_to_bf16(_normal(r, (2 * D, D), 0.02))
+        ly["conv_pw1_b"] = _normal(r, (2 * D,), 0.02)
+        ly["conv_dw_w"] = _normal(r, (K, D), K ** -0.5)
+        ly["conv_dw_b"] = _normal(r, (D,), 0.02)
+        ly["conv_norm_w"] = _normal(r, (D,), 0.02, 1.0)
+        ly["conv_norm_b"] = _normal(r, (D,), 0.02)
+        ly["conv_pw2_w"] = round_to_bf16(_normal(r, (D, D), 0.02))
+        ly["conv_pw2_b"] = _normal(r, (D,), 0.02)
+        W["layers"].append(ly)
+    r = _rng(seed, 100_000)
+    W["ad_norm_w"] = _normal(r, (D,), 0.02, 1.0)
+    W["ad_norm_b"] = _normal(r, (D,), 0.02)
+    W["ad_up_w"] = round_to_bf16(_normal(r, (s["adapter_ff"], D), 0.02))
+    W["ad_up_b"] = _normal(r, (s["adapter_ff"],), 0.02)
+    W["ad_down_w"] = round_to_bf16(_normal(r, (s["llm_hidden"], s["adapter_ff"]), 0.02))
+    W["ad_down_b"] = _normal(r, (s["llm_hidden"],), 0.02)
+    return W
