@@ -208,11 +208,15 @@ __global__ void __launch_bounds__(256) k_lenc_ln(const LencLnArgs r) {
 // memory (bf16) and each thread computes two channels of every row.
 constexpr int kDwRows = 32;
 
+// KT > 0: the tap count known at compile time (the taps of the thread's two
+// channels in registers); KT = 0: any k <= 33, taps read per use.
+template <int KT>
 __global__ void __launch_bounds__(256) k_lenc_dwconv(const bf16 *__restrict__ g, const float *__restrict__ w,
                                                      const float *__restrict__ db, const float *__restrict__ aw,
-                                                     const float *__restrict__ ab, int k, bf16 *__restrict__ out,
+                                                     const float *__restrict__ ab, int k_rt, bf16 *__restrict__ out,
                                                      const int32_t *__restrict__ tok_off, int n_clips, int64_t T) {
   extern __shared__ __align__(16) uint32_t s_g[];  // [kDwRows + k - 1][256] bf16 pairs
+  const int k = KT > 0 ? KT : k_rt;
   const int lo = (k - 1) / 2;
   const int64_t t0 = (int64_t)blockIdx.x * kDwRows;
   const int nrows = kDwRows + k - 1;
@@ -221,8 +225,13 @@ __global__ void __launch_bounds__(256) k_lenc_dwconv(const bf16 *__restrict__ g,
     const int64_t tr = t0 - lo + rr;
     s_g[i] = (tr >= 0 && tr < T) ? *reinterpret_cast<const uint32_t *>(g + tr * kLencEmbd + 2 * cp) : 0u;
   }
-  __syncthreads();
   const int ch = 2 * threadIdx.x;
+  float2 wr[KT > 0 ? KT : 1];
+  if (KT > 0) {
+#pragma unroll
+    for (int m = 0; m < (KT > 0 ? KT : 1); ++m) wr[m] = make_float2(__ldg(w + m * kLencEmbd + ch), __ldg(w + m * kLencEmbd + ch + 1));
+  }
+  __syncthreads();
   const float2 bias = make_float2(db[ch], db[ch + 1]), sc = make_float2(aw[ch], aw[ch + 1]),
                sh = make_float2(ab[ch], ab[ch + 1]);
   int c = lenc_clip_of(tok_off, n_clips, t0 < T ? t0 : T - 1);
@@ -231,13 +240,22 @@ __global__ void __launch_bounds__(256) k_lenc_dwconv(const bf16 *__restrict__ g,
     const int64_t tt = t0 + r;
     if (tt >= T) break;
     while (tok_off[c + 1] <= tt) ++c;  // rows are in order; clips may be empty
-    const int64_t s = tok_off[c], e = tok_off[c + 1];
-    const int m0 = (int)max((int64_t)0, s - (tt - lo)), m1 = (int)min((int64_t)k, e - (tt - lo));
+    const int64_t s0 = tok_off[c], e = tok_off[c + 1];
+    const int m0 = (int)max((int64_t)0, s0 - (tt - lo)), m1 = (int)min((int64_t)k, e - (tt - lo));
     float2 a = bias;
-    for (int m = m0; m < m1; ++m) {
-      const uint32_t v = s_g[(r + m) * 256 + threadIdx.x];
-      ffma2(a, make_float2(__ldg(w + m * kLencEmbd + ch), __ldg(w + m * kLencEmbd + ch + 1)),
-            make_float2(bf16lo(v), bf16hi(v)));
+    if (KT > 0) {
+#pragma unroll
+      for (int m = 0; m < (KT > 0 ? KT : 1); ++m)
+        if (m >= m0 && m < m1) {
+          const uint32_t v = s_g[(r + m) * 256 + threadIdx.x];
+          ffma2(a, wr[m], make_float2(bf16lo(v), bf16hi(v)));
+        }
+    } else {
+      for (int m = m0; m < m1; ++m) {
+        const uint32_t v = s_g[(r + m) * 256 + threadIdx.x];
+        ffma2(a, make_float2(__ldg(w + m * kLencEmbd + ch), __ldg(w + m * kLencEmbd + ch + 1)),
+              make_float2(bf16lo(v), bf16hi(v)));
+      }
     }
     const float2 y = __ffma2_rn(a, sc, sh);
     const float2 z = make_float2(y.x / (1.0f + __expf(-y.x)), y.y / (1.0f + __expf(-y.y)));
@@ -287,9 +305,10 @@ cudaError_t launch_lenc_dwconv(const void *g, const float *w, const float *db, c
                                void *out, const int32_t *tok_off, int n_clips, int64_t T, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
   const size_t smem = (size_t)(kDwRows + k - 1) * 256 * 4;
-  static std::atomic<uint64_t> attr{0};
-  if (const cudaError_t e = smem_attr(k_lenc_dwconv, smem, attr)) return e;
-  return launch_k(k_lenc_dwconv, dim3((unsigned)((T + kDwRows - 1) / kDwRows)), dim3(256), smem, s,
+  static std::atomic<uint64_t> attr9{0}, attr0{0};
+  auto kern = k == 9 ? k_lenc_dwconv<9> : k_lenc_dwconv<0>;
+  if (const cudaError_t e = smem_attr(kern, smem, k == 9 ? attr9 : attr0)) return e;
+  return launch_k(kern, dim3((unsigned)((T + kDwRows - 1) / kDwRows)), dim3(256), smem, s,
                   static_cast<const bf16 *>(g), w, db, aw, ab, k, static_cast<bf16 *>(out), tok_off, n_clips, T);
 }
 

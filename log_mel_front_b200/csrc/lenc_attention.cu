@@ -21,14 +21,13 @@
 //     of a per-warp scratch (row pitch 66 floats) and reads them back from
 //     offset 31 - lane (conflict-free: 65 lane + const); then adds S, scales
 //     and masks keys past the clip end, 32 keys at a time;
-//   * two passes over the key blocks: the first keeps each row's running
-//     maximum and sum of exponentials (rescaled as the maximum grows); the
-//     second recomputes the logits, writes the normalised probabilities as
-//     bf16 (K-major, 128-byte swizzle) and tcgen05.mma accumulates P V
-//     (M=128, N=64, V read MN-major) in tensor memory over the blocks, which
-//     the row thread reads once at the end. The second pass costs one more
-//     score MMA and skew per block, and keeps the row threads' registers to the
-//     96 of one chunk (no output accumulator, no rescale of it).
+//   * online softmax over the key blocks: the row thread keeps its row's
+//     running maximum and sum, writes the block's probabilities (relative to
+//     the new maximum) as bf16 (K-major, 128-byte swizzle), and, when the
+//     maximum grew, first rescales its own row of the P V accumulator in tensor
+//     memory (one tcgen05.ld and one tcgen05.st of 64 columns); tcgen05.mma
+//     then accumulates P V (M=128, N=64, V read MN-major) into it. The row
+//     thread reads the accumulator once at the end and divides by the sum.
 // Every wait is bounded and reports through the library's status word.
 #include "ae_internal.h"
 #include "common.cuh"
@@ -51,6 +50,21 @@ constexpr uint32_t XA_KV_BYTES = 4 * XA_TILE;            // K, V and two positio
 static_assert(XA_SMEM <= 227 * 1024, "shared memory");
 static_assert(OFF_PB % 1024 == 0 && OFF_S % 1024 == 0 && OFF_SCR % 16 == 0, "swizzle atoms");
 }  // namespace
+
+// 32 lanes x 32 consecutive 32-bit columns from registers into tensor memory
+// (thread i of the warp writes row lane-base + i), and the wait for them.
+__device__ __forceinline__ void xa_tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void xa_tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __global__ void __launch_bounds__(XA_THREADS, 1)
     k_lenc_xlattn(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmP,
@@ -84,9 +98,6 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
   const int i0 = (qitem - qblk_off[c]) * XA_Q;
   const int n_kb = (t_c + XA_K - 1) / XA_K;
 
-  // rounds: n_kb of the first pass (K and position rows), then n_kb of the
-  // second (K, position rows and V)
-  const int n_rounds = 2 * n_kb;
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_ready, 128);
@@ -115,21 +126,18 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
     mbar_arrive_expect_tx(q_full, XA_TILE);
     tma_load_2d(sQu, &tmQKV, head * XA_HD, tok0 + i0, q_full);
     int issued = 0;
-    for (int rd = 0; rd < n_rounds; ++rd) {
-      const bool second = rd >= n_kb;
-      const int kb = second ? rd - n_kb : rd;
-      // K and the position rows are free once the previous round's score MMAs
-      // have completed; V once the previous block's P V has
-      if (rd > 0 && !mbar_wait(s_full, (rd - 1) & 1)) { ok = false; break; }
-      if (second && kb > 0 && !mbar_wait(o_full, (kb - 1) & 1)) { ok = false; break; }
+    for (int kb = 0; kb < n_kb; ++kb) {
+      // K and the position rows are free once the previous block's score MMAs
+      // have completed; V once its P V has
+      if (kb > 0 && (!mbar_wait(s_full, (kb - 1) & 1) || !mbar_wait(o_full, (kb - 1) & 1))) { ok = false; break; }
       if (*abort_flag) break;
       const int j0 = kb * XA_K;
       const int prow = t_max - 128 - i0 + j0;  // table row of distance i0 - j0 + 127
-      mbar_arrive_expect_tx(kv_full, second ? XA_KV_BYTES : XA_KV_BYTES - XA_TILE);
+      mbar_arrive_expect_tx(kv_full, XA_KV_BYTES);
       tma_load_2d(sK, &tmQKV, kLencEmbd + head * XA_HD, tok0 + j0, kv_full);
       tma_load_2d(sPb, &tmP, p_col + head * XA_HD, prow, kv_full);
       tma_load_2d(sPb + XA_TILE, &tmP, p_col + head * XA_HD, prow + 128, kv_full);
-      if (second) tma_load_2d(sV, &tmQKV, 2 * kLencEmbd + head * XA_HD, tok0 + j0, kv_full);
+      tma_load_2d(sV, &tmQKV, 2 * kLencEmbd + head * XA_HD, tok0 + j0, kv_full);
       ++issued;
     }
     if (!ok) {
@@ -146,10 +154,8 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
     const uint32_t aqu = smem_u32(sQu), aqv = smem_u32(sQv), ak = smem_u32(sK), av = smem_u32(sV),
                    apb = smem_u32(sPb), as = smem_u32(sS);
     bool ok = mbar_wait(q_ready, 0);
-    for (int rd = 0; rd < n_rounds && ok; ++rd) {
-      const bool second = rd >= n_kb;
-      const int kb = second ? rd - n_kb : rd;
-      if (!mbar_wait(kv_full, rd & 1) || (rd > 0 && !mbar_wait(s_free, (rd - 1) & 1)) || *abort_flag) {
+    for (int kb = 0; kb < n_kb && ok; ++kb) {
+      if (!mbar_wait(kv_full, kb & 1) || (kb > 0 && !mbar_wait(s_free, (kb - 1) & 1)) || *abort_flag) {
         ok = false;
         break;
       }
@@ -161,7 +167,6 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
       for (int k = 0; k < XA_HD / 16; ++k)
         tc_mma_bf16(tmem + COL_T, sw128_desc(aqv + k * 32), sw128_desc(apb + k * 32), idesc_t, k > 0 ? 1u : 0u);
       tc_commit(s_full);
-      if (!second) continue;
       if (!mbar_wait(p_full, kb & 1) || *abort_flag) {
         ok = false;
         break;
@@ -207,23 +212,19 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
     }
     mbar_arrive(q_ready);
     constexpr float kScale = 0.125f * 1.4426950408889634f;  // 1/sqrt(64), in base 2
-    float m_run = -INFINITY, l_run = 0.f, inv_l = 0.f;
-    for (int rd = 0; rd < n_rounds && ok; ++rd) {
-      const bool second = rd >= n_kb;
-      const int kb = second ? rd - n_kb : rd;
+    float m_run = -INFINITY, l_run = 0.f;
+    for (int kb = 0; kb < n_kb && ok; ++kb) {
       const int j0 = kb * XA_K;
-      if (!__all_sync(0xffffffffu, mbar_wait(s_full, rd & 1))) { ok = false; break; }
-      // the previous block's P V has read the probabilities' buffer
-      if (second && kb > 0 && !__all_sync(0xffffffffu, mbar_wait(o_full, (kb - 1) & 1))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full, kb & 1))) { ok = false; break; }
       tc_fence_after();
-      if (second && kb == 0) inv_l = 1.0f / l_run;
-#pragma unroll 1
+      // ---- the block's 128 logits: S plus the skewed window of T
+      float z[XA_K];
+#pragma unroll
       for (int q = 0; q < 4; ++q) {
-        uint32_t a[32], b[32], ac[32];
+        uint32_t a[32], b[32];
         const int ca = 3 - qw + q;  // chunk of T holding column 127 - li + 32 q (or the next one)
         tmem_ld32(trow + COL_T + 32 * ca, a);
         tmem_ld32(trow + COL_T + 32 * (ca + 1), b);
-        tmem_ld32(trow + COL_S + 32 * q, ac);
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -231,48 +232,62 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
           *reinterpret_cast<float2 *>(my + 32 + 2 * e) =
               make_float2(__uint_as_float(b[2 * e]), __uint_as_float(b[2 * e + 1]));
         }
+        tmem_ld32(trow + COL_S + 32 * q, a);
+        tmem_ld_wait();
         __syncwarp();
-        float z[32];
-        float cm = -INFINITY;
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
           const int j = j0 + 32 * q + x;
-          z[x] = j < t_c ? (__uint_as_float(ac[x]) + my[31 - lane + x]) * kScale : -INFINITY;
-          cm = fmaxf(cm, z[x]);
+          z[32 * q + x] = j < t_c ? (__uint_as_float(a[x]) + my[31 - lane + x]) * kScale : -INFINITY;
         }
         __syncwarp();
-        if (!second) {
-          const float m_new = fmaxf(m_run, cm);
-          float ls = 0.f;
-#pragma unroll
-          for (int x = 0; x < 32; ++x) ls += exp2f(z[x] - m_new);  // exp2(-inf) = 0
-          if (m_new != -INFINITY) {
-            l_run = l_run * exp2f(m_run - m_new) + ls;
-            m_run = m_new;
-          }
-        } else {
-          // probabilities of keys 32 q .. 32 q + 31: granules 4 q .. 4 q + 3 of the row
-#pragma unroll
-          for (int gg = 0; gg < 4; ++gg) {
-            const int g = 4 * q + gg;
-            float p[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) p[e] = exp2f(z[8 * gg + e] - m_run) * inv_l;
-            *reinterpret_cast<uint4 *>(sS + (g >> 3) * XA_TILE + li * 128 + (((g & 7) ^ r7) << 4)) = make_uint4(
-                pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]), pack_bf16(p[4], p[5]), pack_bf16(p[6], p[7]));
-          }
-        }
       }
       tc_fence_before();
-      mbar_arrive(s_free);  // this round's scores are read
-      if (second) {
-        fence_async_smem();
-        mbar_arrive(p_full);
+      mbar_arrive(s_free);  // this block's scores are read
+      float bm = -INFINITY;
+#pragma unroll
+      for (int x = 0; x < XA_K; ++x) bm = fmaxf(bm, z[x]);
+      const float m_new = fmaxf(m_run, bm);   // finite: every block holds a key of the clip
+      const float alpha = exp2f(m_run - m_new);  // 0 on the first block
+      // the previous block's P V is done: the probabilities' buffer is free and
+      // the accumulator holds every earlier block
+      if (kb > 0 && !__all_sync(0xffffffffu, mbar_wait(o_full, (kb - 1) & 1))) { ok = false; break; }
+      tc_fence_after();
+      float ls = 0.f;
+#pragma unroll
+      for (int g = 0; g < 16; ++g) {
+        float p[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          p[e] = exp2f(z[8 * g + e] - m_new);
+          ls += p[e];
+        }
+        *reinterpret_cast<uint4 *>(sS + (g >> 3) * XA_TILE + li * 128 + (((g & 7) ^ r7) << 4)) =
+            make_uint4(pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]), pack_bf16(p[4], p[5]), pack_bf16(p[6], p[7]));
       }
+      l_run = l_run * alpha + ls;
+      m_run = m_new;
+      if (kb > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+        // rescale this row of the accumulator to the new maximum
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t o[32];
+          tmem_ld32(trow + COL_O + 32 * h2, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int d = 0; d < 32; ++d) o[d] = __float_as_uint(__uint_as_float(o[d]) * alpha);
+          xa_tmem_st32(trow + COL_O + 32 * h2, o);
+        }
+        xa_tmem_st_wait();
+      }
+      tc_fence_before();
+      fence_async_smem();
+      mbar_arrive(p_full);
     }
     if (ok && !__all_sync(0xffffffffu, mbar_wait(o_full, (n_kb - 1) & 1))) ok = false;
     if (ok) {
       tc_fence_after();
+      const float inv = 1.0f / l_run;
       uint32_t o0[32], o1[32];
       tmem_ld32(trow + COL_O, o0);
       tmem_ld32(trow + COL_O + 32, o1);
@@ -282,15 +297,15 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           *reinterpret_cast<uint4 *>(orow + 8 * g) = make_uint4(
-              pack_bf16(__uint_as_float(o0[8 * g]), __uint_as_float(o0[8 * g + 1])),
-              pack_bf16(__uint_as_float(o0[8 * g + 2]), __uint_as_float(o0[8 * g + 3])),
-              pack_bf16(__uint_as_float(o0[8 * g + 4]), __uint_as_float(o0[8 * g + 5])),
-              pack_bf16(__uint_as_float(o0[8 * g + 6]), __uint_as_float(o0[8 * g + 7])));
+              pack_bf16(__uint_as_float(o0[8 * g]) * inv, __uint_as_float(o0[8 * g + 1]) * inv),
+              pack_bf16(__uint_as_float(o0[8 * g + 2]) * inv, __uint_as_float(o0[8 * g + 3]) * inv),
+              pack_bf16(__uint_as_float(o0[8 * g + 4]) * inv, __uint_as_float(o0[8 * g + 5]) * inv),
+              pack_bf16(__uint_as_float(o0[8 * g + 6]) * inv, __uint_as_float(o0[8 * g + 7]) * inv));
           *reinterpret_cast<uint4 *>(orow + 32 + 8 * g) = make_uint4(
-              pack_bf16(__uint_as_float(o1[8 * g]), __uint_as_float(o1[8 * g + 1])),
-              pack_bf16(__uint_as_float(o1[8 * g + 2]), __uint_as_float(o1[8 * g + 3])),
-              pack_bf16(__uint_as_float(o1[8 * g + 4]), __uint_as_float(o1[8 * g + 5])),
-              pack_bf16(__uint_as_float(o1[8 * g + 6]), __uint_as_float(o1[8 * g + 7])));
+              pack_bf16(__uint_as_float(o1[8 * g]) * inv, __uint_as_float(o1[8 * g + 1]) * inv),
+              pack_bf16(__uint_as_float(o1[8 * g + 2]) * inv, __uint_as_float(o1[8 * g + 3]) * inv),
+              pack_bf16(__uint_as_float(o1[8 * g + 4]) * inv, __uint_as_float(o1[8 * g + 5]) * inv),
+              pack_bf16(__uint_as_float(o1[8 * g + 6]) * inv, __uint_as_float(o1[8 * g + 7]) * inv));
         }
       }
     }
