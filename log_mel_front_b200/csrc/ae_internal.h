@@ -95,6 +95,7 @@ struct ae_model {
   // stem
   float *conv0c;    // [c0][9] (taps minus their channel mean) x LayerNorm gain: the norm's mean is linear in the patch
   float *conv0cov;  // [9][9] channel covariance of the taps: LayerNorm variance = p^T C p
+  void *conv0b;     // [c0][64] bf16: conv0c split as (hi, lo, hi, 0...) per row, the B operand of k_conv0_tc
   float *ln0, *ln1;
   void *conv1;      // [c1][9 * c0], k = (dt * 3 + df) * c0 + c
   void *in_proj;    // [hidden][1024]

@@ -820,6 +820,26 @@ ae_status ae_model_create(const ae_config *cfg, const ae_host_weights *w, ae_dty
     for (int i = 0; i < 81; ++i) cov[i] = (float)(cd[i] / kC0);
     m->conv0c = up.f32(wc.data(), wc.size());
     m->conv0cov = up.f32(cov.data(), cov.size());
+    if (dtype != AE_F32) {
+      // the tensor-core conv0's B rows: k = 0..8 hi parts, 9..17 lo parts, 18..26 hi parts
+      // again, against A = (p_hi, p_hi, p_lo): p_hi w_hi + p_hi w_lo + p_lo w_hi
+      std::vector<uint16_t> b((size_t)kC0 * 64, 0);
+      for (int ch = 0; ch < kC0; ++ch)
+        for (int k = 0; k < 9; ++k) {
+          const float v = wc[ch * 9 + k];
+          const uint16_t hi = f2bf(v);
+          float hf;
+          const uint32_t hu = (uint32_t)hi << 16;
+          std::memcpy(&hf, &hu, 4);
+          const uint16_t lo = f2bf(v - hf);
+          b[(size_t)ch * 64 + k] = hi;
+          b[(size_t)ch * 64 + 9 + k] = lo;
+          b[(size_t)ch * 64 + 18 + k] = hi;
+        }
+      uint16_t *d = up.alloc<uint16_t>(b.size());
+      if (d && cudaMemcpy(d, b.data(), b.size() * 2, cudaMemcpyHostToDevice) != cudaSuccess) up.ok = false;
+      m->conv0b = d;
+    }
   }
   m->ln0 = up.f32(w->ln0, kC0);
   m->ln1 = up.f32(w->ln1, kC1);

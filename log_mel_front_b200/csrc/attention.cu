@@ -24,87 +24,148 @@ namespace ae {
 // Work item = one head x 128 consecutive tokens t0 .. t0+127 (the packed rows
 // of any clips); a persistent CTA (one per SM) walks the items. Per item:
 //   * TMA loads the q tile [128 x 128], the 144 k rows t0-11 .. t0+132 and the
-//     144 v rows (the tensor maps zero-fill rows before 0 and past T);
-//   * the eight softmax warps (two per 32-row quarter of the tile, each on
-//     half of the 128 head dims) scale q by s and split the product into two bf16
-//     tiles, hi = bf16(q s) and lo = bf16(q s - hi), so the score MMA sees q s
-//     to about 16 bits (a single bf16 rounding of q s costs more accuracy
-//     than everything else in the kernel together); they also write the
-//     head's R[d] / k_scale as rows 144..155 under the k rows;
-//   * tcgen05.mma (M=128, N=160, K=128, issued for hi and then for lo into
-//     the same accumulator) gives S = (q s) [k ; R/k_scale]^T in tensor
-//     memory: row r holds q_t.k_{t0-11+c} at column c and the position term
-//     q_t.R[d]/k_scale at column 144+d;
-//   * in the first warp of each pair, the thread of row r (t = t0 + r) reads
-//     columns 32w .. 32w+47 of its warp's
-//     32 rows and shifts them left by its lane (five select stages), so that
-//     column r + 11 - d, the key t - d, lands at index 11 - d; it caps and
+//     144 v rows (the tensor maps zero-fill rows before 0 and past T) into one
+//     of two shared-memory stages;
+//   * four q warps (one per 32-row quarter) scale q by s and split the product
+//     into two bf16 parts, hi = bf16(q s) and lo = bf16(q s - hi), which they
+//     store into tensor memory as the A operand of the score MMA, so that it
+//     sees q s to about 16 bits (a single bf16 rounding of q s costs more
+//     accuracy than everything else in the kernel together); they also write
+//     the head's R[d] / k_scale as rows 144..155 under the k rows;
+//   * tcgen05.mma (A from tensor memory, M=128, N=160, K=128 for hi and again
+//     for lo into the same accumulator) gives S = (q s) [k ; R/k_scale]^T in
+//     tensor memory: row r holds q_t.k_{t0-11+c} at column c and the position
+//     term q_t.R[d]/k_scale at column 144+d;
+//   * four softmax warps: the thread of row r (t = t0 + r) reads columns
+//     32w .. 32w+47 of its warp's 32 rows and shifts them left by its lane
+//     (five select stages), so that column r + 11 - d, the key t - d, lands at
+//     index 11 - d; it caps (cap tanh(z / cap), tanh from the exponential) and
 //     softmaxes the 12 logits (distances past the clip start masked by pos) and
-//     writes them as bf16 into its row of a banded P [128 x 144] whose other
-//     entries stay zero;
-//   * tcgen05.mma (M=128, N=128, K=144, v read MN-major) gives O = P V;
-//   * both warps of the pair drain their row's half of O (64 dims each), clamp
-//     it, and TMA stores leave through a shared-memory box per warp.
-// Buffers are single: the next item's q/k load starts when the score MMA has
-// read them, its v load when the PV MMA has, so loads overlap the softmax.
+//     writes its row of the banded P [128 x 160] (bf16) into tensor memory: the
+//     64-key window of its warp, the band shifted right by its lane, zeros
+//     around it (the columns outside every warp's window stay zero from the
+//     start);
+//   * tcgen05.mma (A = P from tensor memory, M=128, N=128, K=144, v read
+//     MN-major) gives O = P V;
+//   * the q warps drain O, clamp it and store it from registers, whole 32-byte
+//     sectors per row where the output's alignment allows.
+// The stages overlap across items: the q warps split item i+1 as soon as the
+// score MMA of item i has read the previous split, while the softmax warps
+// work on item i; the MMA warp issues the score MMA of item i+1 before the
+// P V MMA of item i; the q warps drain item i after splitting item i+1. A
+// stage's q/k are reloaded once the score MMA that read them completes, its v
+// once the P V MMA has.
 namespace {
-constexpr int AT_Q = 128;                                 // queries per item
-constexpr int AT_KEYS = 144;                              // key rows per item (139 used)
-constexpr int AT_BROWS = AT_KEYS + 16;                    // score MMA B rows: keys, R rows, zero rows
-constexpr uint32_t AT_Q_REGION = AT_Q * 128;              // 64 head dims of q: 16 KB
-constexpr uint32_t AT_KR_REGION = AT_BROWS * 128;         // 20 KB
-constexpr uint32_t AT_V_REGION = AT_KEYS * 128;           // 18 KB
-constexpr uint32_t AT_P_REGION = AT_Q * 128;              // 64 keys of P: 16 KB
-constexpr uint32_t AT_O_BOX = 32 * 128;                   // store box: 32 rows x 64 dims
-constexpr uint32_t OFF_Q = 0;                             // hi part of q s (the TMA lands q here)
-constexpr uint32_t OFF_QL = OFF_Q + 2 * AT_Q_REGION;      // lo part of q s
-constexpr uint32_t OFF_KR = OFF_QL + 2 * AT_Q_REGION;
+constexpr int AT_Q = 128;                                  // queries per item
+constexpr int AT_KEYS = 144;                               // key rows per item (139 used)
+constexpr int AT_BROWS = AT_KEYS + 16;                     // score MMA B rows: keys, R rows, zero rows
+constexpr uint32_t AT_Q_REGION = AT_Q * 128;               // 64 head dims of q: 16 KB
+constexpr uint32_t AT_KR_REGION = AT_BROWS * 128;          // 20 KB
+constexpr uint32_t AT_V_REGION = AT_KEYS * 128;            // 18 KB
+constexpr uint32_t OFF_Q = 0;                              // offsets within a stage
+constexpr uint32_t OFF_KR = OFF_Q + 2 * AT_Q_REGION;
 constexpr uint32_t OFF_V = OFF_KR + 2 * AT_KR_REGION;
-constexpr uint32_t OFF_P = OFF_V + 2 * AT_V_REGION;
-constexpr uint32_t OFF_O = OFF_P + 3 * AT_P_REGION;
-constexpr uint32_t OFF_BAR = OFF_O + 4 * 2 * AT_O_BOX;
+constexpr uint32_t AT_STAGE = OFF_V + 2 * AT_V_REGION;     // 108 KB
+constexpr uint32_t OFF_BAR = 2 * AT_STAGE;
 constexpr size_t AT_SMEM = OFF_BAR + 1024 + 1024;          // barriers + q scales, alignment slack
-constexpr int AT_THREADS = 320;                           // producer warp, MMA warp, 8 softmax warps
-constexpr uint32_t AT_TMEM_COLS = 512;                    // S at column 0, O at column 256
-constexpr uint32_t AT_O_COL = 256;
+constexpr int AT_THREADS = 320;                            // producer, MMA, 4 softmax warps, 4 q warps
+constexpr uint32_t AT_TMEM_COLS = 512;
+constexpr uint32_t COL_S = 0;                              // scores, 160 f32 columns
+constexpr uint32_t COL_P = 160;                            // banded P, 160 bf16 = 80 columns
+constexpr uint32_t COL_QH = 256;                           // q s hi part, 128 bf16 = 64 columns
+constexpr uint32_t COL_QL = 320;                           // q s lo part (directly after hi: one K = 256 operand)
+constexpr uint32_t COL_O = 384;                            // P V, 128 f32 columns
 constexpr uint32_t AT_QK_BYTES = 2 * AT_Q_REGION + 2 * AT_KEYS * 128;
 constexpr uint32_t AT_V_BYTES = 2 * AT_V_REGION;
 static_assert(AT_SMEM <= 227 * 1024, "shared memory");
-static_assert(OFF_KR % 1024 == 0 && OFF_V % 1024 == 0 && OFF_P % 1024 == 0 && OFF_O % 1024 == 0, "swizzle atoms");
+static_assert(AT_STAGE % 1024 == 0 && OFF_KR % 1024 == 0 && OFF_V % 1024 == 0, "swizzle atoms");
 static_assert(AT_KR_REGION % 1024 == 0 && AT_V_REGION % 1024 == 0, "swizzle atoms");
+static_assert(COL_QL == COL_QH + 64 && COL_O + 128 <= AT_TMEM_COLS && COL_P + 80 <= COL_QH, "tensor-memory map");
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, bf16 inputs, f32 accumulate: A's row m is
+// tensor-memory lane m, two bf16 per 32-bit column (the lower k in the low
+// half), K = 16 per instruction over 8 columns. One thread issues.
+__device__ __forceinline__ void at_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 32 lanes x 32 (16) consecutive 32-bit columns from registers into tensor
+// memory (thread i of the warp writes row lane-base + i), and the wait for them.
+__device__ __forceinline__ void at_tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void at_tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void at_tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void at_st32B(void *p, uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t e,
+                                         uint32_t f, uint32_t g, uint32_t h) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d),
+               "r"(e), "r"(f), "r"(g), "r"(h)
+               : "memory");
+}
+__device__ __forceinline__ float at_ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float at_rcp(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 }  // namespace
 
 __global__ void __launch_bounds__(AT_THREADS, 1)
     k_attention_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                   const __grid_constant__ CUtensorMap tmV, bf16 *__restrict__ out, int64_t ld_out, bool out_v8,
                    const float *__restrict__ R, const float *__restrict__ qscale, float k_scale, float cap,
                    const int32_t *__restrict__ pos, int T, float lo, float hi, unsigned *status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sQ = smem + OFF_Q, *sQL = smem + OFF_QL, *sKR = smem + OFF_KR, *sV = smem + OFF_V, *sP = smem + OFF_P, *sO = smem + OFF_O;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-  uint64_t *qk_full = bars, *v_full = bars + 1, *q_ready = bars + 2, *s_full = bars + 3, *p_full = bars + 4,
-           *o_full = bars + 5, *o_empty = bars + 6;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 7);
+  uint64_t *qk_full = bars, *v_full = bars + 2, *qk_free = bars + 4, *v_free = bars + 6;  // per stage
+  uint64_t *q_ready = bars + 8, *s_full = bars + 9, *s_free = bars + 10, *p_full = bars + 11, *o_full = bars + 12,
+           *o_empty = bars + 13;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 14);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   float *s_qs = reinterpret_cast<float *>(smem + OFF_BAR + 128);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = ((T + AT_Q - 1) / AT_Q) * kHeads;
   if (threadIdx.x == 0) {
-    mbar_init(qk_full, 1);
-    mbar_init(v_full, 1);
-    mbar_init(q_ready, 256);
+    for (int i = 0; i < 8; ++i) mbar_init(bars + i, 1);
+    mbar_init(q_ready, 128);
     mbar_init(s_full, 1);
+    mbar_init(s_free, 128);
     mbar_init(p_full, 128);
     mbar_init(o_full, 1);
-    mbar_init(o_empty, 256);
+    mbar_init(o_empty, 128);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
-    tma_prefetch_desc(&tmO);
   }
   if (threadIdx.x >= 64 && threadIdx.x < 64 + kHeadDim) s_qs[threadIdx.x - 64] = qscale[threadIdx.x - 64];
   if (warp == 1) {
@@ -118,23 +179,25 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer
-    int n_qk = 0, n_v = 0;
+    int n_qk = 0, n_v = 0;  // items whose q/k (v) loads were issued; item i uses stage i & 1
     bool ok = true;
     for (int item = blockIdx.x, it = 0; item < n_items; item += gridDim.x, ++it) {
+      const int st = it & 1, u = it >> 1;
+      uint8_t *stage = smem + st * AT_STAGE;
       const int t0 = (item >> 3) * AT_Q, x = (item & 7) * kHeadDim;
-      if (it > 0 && !mbar_wait(s_full, (it - 1) & 1)) { ok = false; break; }  // q/k buffers read
+      if (u > 0 && !mbar_wait(&qk_free[st], (u - 1) & 1)) { ok = false; break; }  // score MMA read q, k
       if (*abort_flag) break;
-      mbar_arrive_expect_tx(qk_full, AT_QK_BYTES);
-      tma_load_2d(sQ, &tmQ, x, t0, qk_full);
-      tma_load_2d(sQ + AT_Q_REGION, &tmQ, x + 64, t0, qk_full);
-      tma_load_2d(sKR, &tmK, x, t0 - (kLeft - 1), qk_full);
-      tma_load_2d(sKR + AT_KR_REGION, &tmK, x + 64, t0 - (kLeft - 1), qk_full);
+      mbar_arrive_expect_tx(&qk_full[st], AT_QK_BYTES);
+      tma_load_2d(stage + OFF_Q, &tmQ, x, t0, &qk_full[st]);
+      tma_load_2d(stage + OFF_Q + AT_Q_REGION, &tmQ, x + 64, t0, &qk_full[st]);
+      tma_load_2d(stage + OFF_KR, &tmK, x, t0 - (kLeft - 1), &qk_full[st]);
+      tma_load_2d(stage + OFF_KR + AT_KR_REGION, &tmK, x + 64, t0 - (kLeft - 1), &qk_full[st]);
       ++n_qk;
-      if (it > 0 && !mbar_wait(o_full, (it - 1) & 1)) { ok = false; break; }  // v buffer read
+      if (u > 0 && !mbar_wait(&v_free[st], (u - 1) & 1)) { ok = false; break; }  // P V MMA read v
       if (*abort_flag) break;
-      mbar_arrive_expect_tx(v_full, AT_V_BYTES);
-      tma_load_2d(sV, &tmV, x, t0 - (kLeft - 1), v_full);
-      tma_load_2d(sV + AT_V_REGION, &tmV, x + 64, t0 - (kLeft - 1), v_full);
+      mbar_arrive_expect_tx(&v_full[st], AT_V_BYTES);
+      tma_load_2d(stage + OFF_V, &tmV, x, t0 - (kLeft - 1), &v_full[st]);
+      tma_load_2d(stage + OFF_V + AT_V_REGION, &tmV, x + 64, t0 - (kLeft - 1), &v_full[st]);
       ++n_v;
     }
     if (!ok) {
@@ -142,96 +205,89 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       *abort_flag = 1;
     }
     // every load issued must land before the CTA may end
-    if (n_qk > 0) mbar_wait(qk_full, (n_qk - 1) & 1);
-    if (n_v > 0) mbar_wait(v_full, (n_v - 1) & 1);
+#pragma unroll
+    for (int st = 0; st < 2; ++st) {
+      const int uq = (n_qk + 1 - st) / 2, uv = (n_v + 1 - st) / 2;  // uses of stage st
+      if (uq > 0) mbar_wait(&qk_full[st], (uq - 1) & 1);
+      if (uv > 0) mbar_wait(&v_full[st], (uv - 1) & 1);
+    }
   } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer
+    // ---------------- MMA issuer: the score MMA of item i, then the P V MMA of item i - 1
     constexpr uint32_t idesc_s = idesc_bf16_f32(AT_Q, AT_BROWS);
     constexpr uint32_t idesc_o = idesc_bf16_f32_bmn(AT_Q, kHeadDim);
-    const uint32_t aq = smem_u32(sQ), aql = smem_u32(sQL), akr = smem_u32(sKR), ap = smem_u32(sP),
-                   av = smem_u32(sV);
     bool ok = true;
-    for (int item = blockIdx.x, it = 0; item < n_items; item += gridDim.x, ++it) {
-      if (!mbar_wait(q_ready, it & 1) || *abort_flag) { ok = false; break; }
+    auto pv = [&](int j) -> bool {  // O = P V of item j
+      const int st = j & 1;
+      if (!mbar_wait(p_full, j & 1) || !mbar_wait(&v_full[st], (j >> 1) & 1) ||
+          (j > 0 && !mbar_wait(o_empty, (j - 1) & 1)) || *abort_flag)
+        return false;
       tc_fence_after();
+      const uint32_t av = smem_u32(smem + st * AT_STAGE + OFF_V);
 #pragma unroll
-      for (int ks = 0; ks < 2 * kHeadDim / 16; ++ks) {
-        const int kk = ks & 7;
-        tc_mma_bf16(tmem, sw128_desc((ks < 8 ? aq : aql) + (kk >> 2) * AT_Q_REGION + (kk & 3) * 32),
-                    sw128_desc(akr + (kk >> 2) * AT_KR_REGION + (kk & 3) * 32), idesc_s, ks > 0 ? 1u : 0u);
-      }
-      tc_commit(s_full);
-      if (!mbar_wait(p_full, it & 1) || !mbar_wait(v_full, it & 1) ||
-          (it > 0 && !mbar_wait(o_empty, (it - 1) & 1)) || *abort_flag) {
+      for (int ks = 0; ks < AT_KEYS / 16; ++ks)
+        at_mma_ts(tmem + COL_O, tmem + COL_P + 8 * ks, sw128_desc_mn(av + ks * 2048, AT_V_REGION), idesc_o,
+                  ks > 0 ? 1u : 0u);
+      tc_commit(&v_free[st]);
+      tc_commit(o_full);
+      return true;
+    };
+    int it = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it) {
+      const int st = it & 1;
+      const uint32_t akr = smem_u32(smem + st * AT_STAGE + OFF_KR);
+      // q s of this item is in tensor memory, and the softmax has read the previous scores
+      if (!mbar_wait(q_ready, it & 1) || (it > 0 && !mbar_wait(s_free, (it - 1) & 1)) || *abort_flag) {
         ok = false;
         break;
       }
       tc_fence_after();
 #pragma unroll
-      for (int ks = 0; ks < AT_KEYS / 16; ++ks)
-        tc_mma_bf16(tmem + AT_O_COL, sw128_desc(ap + (ks >> 2) * AT_P_REGION + (ks & 3) * 32),
-                    sw128_desc_mn(av + ks * 2048, AT_V_REGION), idesc_o, ks > 0 ? 1u : 0u);
-      tc_commit(o_full);
+      for (int ks = 0; ks < 2 * kHeadDim / 16; ++ks) {
+        const int kk = ks & 7;  // hi part for ks < 8, lo part after: the same k rows
+        at_mma_ts(tmem + COL_S, tmem + COL_QH + 8 * ks,
+                  sw128_desc(akr + (kk >> 2) * AT_KR_REGION + (kk & 3) * 32), idesc_s, ks > 0 ? 1u : 0u);
+      }
+      tc_commit(&qk_free[st]);
+      tc_commit(s_full);
+      if (it > 0 && !pv(it - 1)) { ok = false; break; }
     }
+    if (ok && it > 0 && !pv(it - 1)) ok = false;
     if (!ok) {
       atomicOr(status, kStatusWaitTimeout);
       *abort_flag = 1;
     }
-  } else if (warp >= 2) {
-    // ---------------- softmax warps: two per TMEM lane quarter, thread = tile row r;
-    // warp half hw takes head dims 64 hw .. +63 of q and of the output, and the
-    // hw = 0 warps the softmax of their rows
-    const int qw = warp & 3, hw = (warp - 2) >> 2, r = 32 * qw + lane, r7 = r & 7, tid = threadIdx.x - 64;
-    uint8_t *box = sO + (qw * 2 + hw) * AT_O_BOX;
-    // P outside the band and the zero rows 156..159 of the B operand stay zero
-    for (int i = tid; i < (int)(3 * AT_P_REGION / 16); i += 256) reinterpret_cast<uint4 *>(sP)[i] = make_uint4(0, 0, 0, 0);
-    if (tid < 64) {
-      const int rr = AT_KEYS + 12 + (tid >> 4), g = tid & 15;
-      *reinterpret_cast<uint4 *>(sKR + (g >> 3) * AT_KR_REGION + rr * 128 + (((g & 7) ^ (rr & 7)) << 4)) =
-          make_uint4(0, 0, 0, 0);
-    }
-    const float zs = k_scale / cap, inv_ks = 1.0f / k_scale;
+  } else if (warp >= 2 && warp < 6) {
+    // ---------------- softmax warps: TMEM lane quarter qw, thread = tile row r
+    const int qw = warp & 3, r = 32 * qw + lane;
     const uint32_t trow = tmem + ((uint32_t)(32 * qw) << 16);
+    {  // P's columns outside the warps' windows stay zero
+      uint32_t z[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) z[i] = 0u;
+      at_tmem_st32(trow + COL_P, z);
+      at_tmem_st32(trow + COL_P + 32, z);
+      uint32_t z16[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) z16[i] = 0u;
+      at_tmem_st16(trow + COL_P + 64, z16);
+      at_tmem_st_wait();
+    }
+    // z = cap tanh(zs x) = cap (1 - 2 / (1 + 2^(e2 x))), e2 = 2 log2(e) zs: the
+    // exponential and reciprocal to about 2^-22 give z to about 1e-6 cap
+    const float zs = k_scale / cap, e2 = 2.0f * 1.4426950408889634f * zs;
     bool ok = true;
     for (int item = blockIdx.x, it = 0; item < n_items; item += gridDim.x, ++it) {
-      const int t0 = (item >> 3) * AT_Q, h = item & 7, t = t0 + r;
-      // ---- q s as hi + lo bf16 tiles, and R / k_scale under the k rows
-      if (!__all_sync(0xffffffffu, mbar_wait(qk_full, it & 1))) { ok = false; break; }
-#pragma unroll 4
-      for (int j = 8 * hw; j < 8 * hw + 8; ++j) {
-        const uint32_t off = (j >> 3) * AT_Q_REGION + r * 128 + (((j & 7) ^ r7) << 4);
-        const uint4 w = *reinterpret_cast<const uint4 *>(sQ + off);
-        const float4 s0 = reinterpret_cast<const float4 *>(s_qs)[2 * j], s1 = reinterpret_cast<const float4 *>(s_qs)[2 * j + 1];
-        const float f[8] = {bf16lo(w.x) * s0.x, bf16hi(w.x) * s0.y, bf16lo(w.y) * s0.z, bf16hi(w.y) * s0.w,
-                            bf16lo(w.z) * s1.x, bf16hi(w.z) * s1.y, bf16lo(w.w) * s1.z, bf16hi(w.w) * s1.w};
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          hi[e] = pack_bf16(f[2 * e], f[2 * e + 1]);
-          lo[e] = pack_bf16(f[2 * e] - bf16lo(hi[e]), f[2 * e + 1] - bf16hi(hi[e]));
-        }
-        *reinterpret_cast<uint4 *>(sQ + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4 *>(sQL + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      }
-      for (int rr = tid >> 4; rr < kLeft; rr += 16) {
-        const int g = tid & 15, row = AT_KEYS + rr;
-        const float4 a = *reinterpret_cast<const float4 *>(R + (size_t)rr * kHidden + h * kHeadDim + g * 8);
-        const float4 b = *reinterpret_cast<const float4 *>(R + (size_t)rr * kHidden + h * kHeadDim + g * 8 + 4);
-        *reinterpret_cast<uint4 *>(sKR + (g >> 3) * AT_KR_REGION + row * 128 + (((g & 7) ^ (row & 7)) << 4)) =
-            make_uint4(pack_bf16(a.x * inv_ks, a.y * inv_ks), pack_bf16(a.z * inv_ks, a.w * inv_ks),
-                       pack_bf16(b.x * inv_ks, b.y * inv_ks), pack_bf16(b.z * inv_ks, b.w * inv_ks));
-      }
-      fence_async_smem();
-      mbar_arrive(q_ready);
-      // ---- scores -> probabilities -> banded P (warps of half 0)
-      if (hw == 0) {
+      const int t = (item >> 3) * AT_Q + r;
+      const int pos_t = t < T ? pos[t] : -1;  // issued before the wait, used after it
       if (!__all_sync(0xffffffffu, mbar_wait(s_full, it & 1))) { ok = false; break; }
       tc_fence_after();
       uint32_t a32[32], a16[16], u16[16];
-      tmem_ld32(trow + 32 * qw, a32);
-      tmem_ld16(trow + 32 * qw + 32, a16);
-      tmem_ld16(trow + AT_KEYS, u16);
+      tmem_ld32(trow + COL_S + 32 * qw, a32);
+      tmem_ld16(trow + COL_S + 32 * qw + 32, a16);
+      tmem_ld16(trow + COL_S + AT_KEYS, u16);
       tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(s_free);  // the scores are in registers
       float sc[48];
 #pragma unroll
       for (int i = 0; i < 32; ++i) sc[i] = __uint_as_float(a32[i]);
@@ -248,11 +304,12 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       for (int i = 0; i < 28; ++i) sc[i] = (lane & 8) ? sc[i + 8] : sc[i];
 #pragma unroll
       for (int i = 0; i < 12; ++i) sc[i] = (lane & 16) ? sc[i + 16] : sc[i];
-      const int span = t < T ? min(pos[t] + 1, kLeft) : 0;
+      const int span = min(pos_t + 1, kLeft);
       float pr[kLeft], mx = -INFINITY;
 #pragma unroll
       for (int d = 0; d < kLeft; ++d) {
-        const float z = cap * tanhf(zs * (sc[kLeft - 1 - d] + __uint_as_float(u16[d])));
+        const float x = sc[kLeft - 1 - d] + __uint_as_float(u16[d]);
+        const float z = cap * fmaf(-2.0f, at_rcp(1.0f + at_ex2(e2 * x)), 1.0f);
         pr[d] = d < span ? z : -INFINITY;
         mx = fmaxf(mx, pr[d]);
       }
@@ -263,59 +320,139 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         den += pr[d];
       }
       const float rd = span > 0 ? 1.0f / den : 0.f;
-      // band of row r: column r + i holds p_{11-i}; written as the three
-      // granules (8 columns each) from column r & ~7, zeros around the band
-      float a[24];
+      // the warp's window holds keys 32 qw .. 32 qw + 63 (32 columns of bf16
+      // pairs); row r's band, key r + i = p_{11-i}, sits at window index
+      // lane + i: shift by the lane's low bit in floats, pair up, then shift
+      // the pairs by lane >> 1
+      float c[14];
 #pragma unroll
-      for (int j = 0; j < 24; ++j) a[j] = j < kLeft ? pr[kLeft - 1 - j] * rd : 0.f;
-#pragma unroll
-      for (int j = 23; j >= 0; --j) a[j] = (r7 & 4) ? (j >= 4 ? a[j - 4] : 0.f) : a[j];
-#pragma unroll
-      for (int j = 23; j >= 0; --j) a[j] = (r7 & 2) ? (j >= 2 ? a[j - 2] : 0.f) : a[j];
-#pragma unroll
-      for (int j = 23; j >= 0; --j) a[j] = (r7 & 1) ? (j >= 1 ? a[j - 1] : 0.f) : a[j];
-#pragma unroll
-      for (int gg = 0; gg < 3; ++gg) {
-        const int G = (r >> 3) + gg;
-        *reinterpret_cast<uint4 *>(sP + (G >> 3) * AT_P_REGION + r * 128 + (((G & 7) ^ r7) << 4)) =
-            make_uint4(pack_bf16(a[8 * gg], a[8 * gg + 1]), pack_bf16(a[8 * gg + 2], a[8 * gg + 3]),
-                       pack_bf16(a[8 * gg + 4], a[8 * gg + 5]), pack_bf16(a[8 * gg + 6], a[8 * gg + 7]));
+      for (int j = 0; j < 14; ++j) {
+        const float cur = j < kLeft ? pr[kLeft - 1 - j] * rd : 0.f;
+        const float prev = (j >= 1 && j - 1 < kLeft) ? pr[kLeft - j] * rd : 0.f;
+        c[j] = (lane & 1) ? prev : cur;
       }
-      tc_fence_before();
-      fence_async_smem();
-      mbar_arrive(p_full);
-      }
-      // ---- O rows out: head dims 64 hw .. +63
-      if (!__all_sync(0xffffffffu, mbar_wait(o_full, it & 1))) { ok = false; break; }
+      uint32_t w[22];
+#pragma unroll
+      for (int k = 0; k < 22; ++k) w[k] = k < 7 ? pack_bf16(c[2 * k], c[2 * k + 1]) : 0u;
+      const int hs = lane >> 1;
+#pragma unroll
+      for (int k = 21; k >= 0; --k) w[k] = (hs & 8) ? (k >= 8 ? w[k - 8] : 0u) : w[k];
+#pragma unroll
+      for (int k = 21; k >= 0; --k) w[k] = (hs & 4) ? (k >= 4 ? w[k - 4] : 0u) : w[k];
+#pragma unroll
+      for (int k = 21; k >= 0; --k) w[k] = (hs & 2) ? (k >= 2 ? w[k - 2] : 0u) : w[k];
+#pragma unroll
+      for (int k = 21; k >= 0; --k) w[k] = (hs & 1) ? (k >= 1 ? w[k - 1] : 0u) : w[k];
+      uint32_t pw[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) pw[k] = k < 22 ? w[k] : 0u;
+      // the previous item's P V has read P
+      if (it > 0 && !__all_sync(0xffffffffu, mbar_wait(o_full, (it - 1) & 1))) { ok = false; break; }
       tc_fence_after();
-      if (lane == 0) bulk_wait_read<0>();  // the previous item's stores are done with the boxes
-      __syncwarp();
+      at_tmem_st32(trow + COL_P + 16 * qw, pw);
+      at_tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    if (!ok && lane == 0) {
+      atomicOr(status, kStatusWaitTimeout);
+      *abort_flag = 1;
+    }
+  } else if (warp >= 6) {
+    // ---------------- q warps: split item i's q s into tensor memory, then drain item i - 1
+    const int qw = warp & 3, r = 32 * qw + lane, r7 = r & 7, tid = threadIdx.x - 192;
+    const uint32_t trow = tmem + ((uint32_t)(32 * qw) << 16);
+    // rows 156..159 of both stages' B operand stay zero
+    {
+      const int s = tid >> 6, rr = AT_KEYS + 12 + ((tid >> 4) & 3), g = tid & 15;
+      *reinterpret_cast<uint4 *>(smem + s * AT_STAGE + OFF_KR + (g >> 3) * AT_KR_REGION + rr * 128 +
+                                 (((g & 7) ^ (rr & 7)) << 4)) = make_uint4(0, 0, 0, 0);
+    }
+    const float inv_ks = 1.0f / k_scale;
+    bool ok = true;
+    auto drain = [&](int j, int jitem) -> bool {  // O rows of item j out
+      if (!__all_sync(0xffffffffu, mbar_wait(o_full, j & 1))) return false;
+      tc_fence_after();
+      const int t = (jitem >> 3) * AT_Q + r, h = jitem & 7;
+      bf16 *orow = out + (int64_t)t * ld_out + h * kHeadDim;
 #pragma unroll 1
-      for (int c = 2 * hw; c < 2 * hw + 2; ++c) {
+      for (int c = 0; c < 4; ++c) {
         uint32_t o[32];
-        tmem_ld32(trow + AT_O_COL + 32 * c, o);
+        tmem_ld32(trow + COL_O + 32 * c, o);
         tmem_ld_wait();
-        uint8_t *line = box + lane * 128;
+        uint32_t w[16];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int g = (c & 1) * 4 + j;
-          *reinterpret_cast<uint4 *>(line + ((g ^ (lane & 7)) << 4)) = make_uint4(
-              pack_bf16(clampf(__uint_as_float(o[8 * j]), lo, hi), clampf(__uint_as_float(o[8 * j + 1]), lo, hi)),
-              pack_bf16(clampf(__uint_as_float(o[8 * j + 2]), lo, hi), clampf(__uint_as_float(o[8 * j + 3]), lo, hi)),
-              pack_bf16(clampf(__uint_as_float(o[8 * j + 4]), lo, hi), clampf(__uint_as_float(o[8 * j + 5]), lo, hi)),
-              pack_bf16(clampf(__uint_as_float(o[8 * j + 6]), lo, hi), clampf(__uint_as_float(o[8 * j + 7]), lo, hi)));
+        for (int j2 = 0; j2 < 16; ++j2)
+          w[j2] = pack_bf16(clampf(__uint_as_float(o[2 * j2]), lo, hi), clampf(__uint_as_float(o[2 * j2 + 1]), lo, hi));
+        if (t < T) {
+          if (out_v8) {
+            at_st32B(orow + 32 * c, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+            at_st32B(orow + 32 * c + 16, w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]);
+          } else {
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+              *reinterpret_cast<uint4 *>(orow + 32 * c + 8 * g) =
+                  make_uint4(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
+          }
         }
       }
       tc_fence_before();
       mbar_arrive(o_empty);
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0 && t0 + 32 * qw < T) {
-        tma_store_2d(&tmO, box, h * kHeadDim + 64 * hw, t0 + 32 * qw);
-        bulk_commit();
+      return true;
+    };
+    int it = 0, prev_item = -1;
+    int r_head0 = -1, r_head1 = -1;  // the head whose R rows each stage holds (one head per stage
+                                     // when the grid is a multiple of 4, as on 148 SMs)
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it) {
+      const int st = it & 1, u = it >> 1;
+      uint8_t *sQ = smem + st * AT_STAGE + OFF_Q, *sKR = smem + st * AT_STAGE + OFF_KR;
+      const int h = item & 7;
+      // this item's q and k have landed, and the previous score MMA has read the previous split
+      if (!__all_sync(0xffffffffu, mbar_wait(&qk_full[st], u & 1)) ||
+          (it > 0 && !__all_sync(0xffffffffu, mbar_wait(s_full, (it - 1) & 1)))) {
+        ok = false;
+        break;
       }
+      tc_fence_after();
+#pragma unroll 1
+      for (int hw = 0; hw < 2; ++hw) {  // head dims 64 hw .. 64 hw + 63
+        uint32_t qh[32], ql[32];
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const uint4 wv = *reinterpret_cast<const uint4 *>(sQ + hw * AT_Q_REGION + r * 128 + ((jj ^ r7) << 4));
+          const int j = 8 * hw + jj;
+          const float4 s0 = reinterpret_cast<const float4 *>(s_qs)[2 * j], s1 = reinterpret_cast<const float4 *>(s_qs)[2 * j + 1];
+          const float f[8] = {bf16lo(wv.x) * s0.x, bf16hi(wv.x) * s0.y, bf16lo(wv.y) * s0.z, bf16hi(wv.y) * s0.w,
+                              bf16lo(wv.z) * s1.x, bf16hi(wv.z) * s1.y, bf16lo(wv.w) * s1.z, bf16hi(wv.w) * s1.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t hv = pack_bf16(f[2 * e], f[2 * e + 1]);
+            qh[4 * jj + e] = hv;
+            ql[4 * jj + e] = pack_bf16(f[2 * e] - bf16lo(hv), f[2 * e + 1] - bf16hi(hv));
+          }
+        }
+        at_tmem_st32(trow + COL_QH + 32 * hw, qh);
+        at_tmem_st32(trow + COL_QL + 32 * hw, ql);
+      }
+      if ((st ? r_head1 : r_head0) != h) {  // the TMA never writes rows 144.., so they keep the stage's last head
+        if (st) r_head1 = h; else r_head0 = h;
+        for (int rr = tid >> 4; rr < kLeft; rr += 8) {
+          const int g = tid & 15, row = AT_KEYS + rr;
+          const float4 a = *reinterpret_cast<const float4 *>(R + (size_t)rr * kHidden + h * kHeadDim + g * 8);
+          const float4 b = *reinterpret_cast<const float4 *>(R + (size_t)rr * kHidden + h * kHeadDim + g * 8 + 4);
+          *reinterpret_cast<uint4 *>(sKR + (g >> 3) * AT_KR_REGION + row * 128 + (((g & 7) ^ (row & 7)) << 4)) =
+              make_uint4(pack_bf16(a.x * inv_ks, a.y * inv_ks), pack_bf16(a.z * inv_ks, a.w * inv_ks),
+                         pack_bf16(b.x * inv_ks, b.y * inv_ks), pack_bf16(b.z * inv_ks, b.w * inv_ks));
+        }
+      }
+      at_tmem_st_wait();
+      tc_fence_before();
+      fence_async_smem();
+      mbar_arrive(q_ready);
+      if (it > 0 && !drain(it - 1, prev_item)) { ok = false; break; }
+      prev_item = item;
     }
-    if (lane == 0) bulk_wait_all();
+    if (ok && it > 0 && !drain(it - 1, prev_item)) ok = false;
     if (!ok && lane == 0) {
       atomicOr(status, kStatusWaitTimeout);
       *abort_flag = 1;
@@ -424,20 +561,21 @@ cudaError_t launch_attention(bool is_bf16, const void *q, const void *k, const v
   if (is_bf16) {
     static std::atomic<uint64_t> attr{0};
     if (const cudaError_t e = smem_attr(k_attention_tc, AT_SMEM, attr)) return e;
-    CUtensorMap tq, tk, tv, to;
-    const uint64_t rb = (uint64_t)ld * 2, ob = (uint64_t)ld_out * 2;
+    CUtensorMap tq, tk, tv;
+    const uint64_t rb = (uint64_t)ld * 2;
     if (!make_tmap_2d_bf16(&tq, q, kHidden, (uint64_t)T, rb, 64, AT_Q) ||
         !make_tmap_2d_bf16(&tk, k, kHidden, (uint64_t)T, rb, 64, AT_KEYS) ||
-        !make_tmap_2d_bf16(&tv, v, kHidden, (uint64_t)T, rb, 64, AT_KEYS) ||
-        !make_tmap_2d_bf16(&to, out, kHidden, (uint64_t)T, ob, 64, 32))
+        !make_tmap_2d_bf16(&tv, v, kHidden, (uint64_t)T, rb, 64, AT_KEYS))
       return cudaErrorInvalidValue;
+    // rows leave as 32-byte sectors when the output and its stride allow it, else as 16-byte pieces
+    const bool v8 = (reinterpret_cast<uintptr_t>(out) % 32) == 0 && (ld_out % 16) == 0;
     int dev = 0, sms = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t items = (T + AT_Q - 1) / AT_Q * kHeads;
     const unsigned grid = (unsigned)(items < sms ? items : (sms > 0 ? sms : 1));
-    return launch_k(k_attention_tc, dim3(grid), dim3(AT_THREADS), AT_SMEM, s, tq, tk, tv, to, R, qscale, k_scale,
-                    cap, pos, (int)T, lo, hi, device_status_word());
+    return launch_k(k_attention_tc, dim3(grid), dim3(AT_THREADS), AT_SMEM, s, tq, tk, tv, static_cast<bf16 *>(out),
+                    ld_out, v8, R, qscale, k_scale, cap, pos, (int)T, lo, hi, device_status_word());
   }
   const size_t smem = (2 * (size_t)kRows * kPitchF + kLeft * kHeadDim + kHeadDim) * sizeof(float);
   static std::atomic<uint64_t> attr{0};

@@ -151,6 +151,213 @@ __global__ void __launch_bounds__(128) k_conv0(const float *__restrict__ mel, co
   }
 }
 
+// ------------------------------------------------------------------ conv0 + LN + ReLU, tensor cores
+
+// The same normalised conv0 as a tcgen05 product, for the bf16 and e4m3
+// models: a work item is two stem rows, 128 positions (M = 128), against the
+// 128 channels (N = 128). Position r's A row is its 9-sample patch split into
+// bf16 parts, (p_hi, p_hi, p_lo) in k = 0..26, and channel c's B row is
+// (w_hi, w_lo, w_hi) of its centred, gain-folded taps (built at model
+// creation), so the product is p_hi w_hi + p_hi w_lo + p_lo w_hi: the taps
+// and the patch to about 16 bits, accumulated in float32 (K = 64, zero beyond
+// 27). Thread r builds row r, computes its LayerNorm factor 1/sqrt(p^T C p +
+// eps) from the covariance in registers, and after the MMA drains its own
+// tensor-memory lane (the 128 channels of its position), scales, applies
+// ReLU and stages its 256-byte row in shared memory (128-byte swizzle, as two
+// 64-channel halves); two TMA tensor stores write the item's output, one
+// contiguous 32 KB block of whole lines. Persistent CTAs, at most four per SM
+// (128 tensor-memory columns each); the six mel rows an item reads are copied
+// into one of two shared-memory buffers with cp.async while the item before
+// it is computed.
+namespace {
+constexpr uint32_t C0T_TILE = 128 * 128;  // 128 rows x 64 bf16, 128-byte swizzle
+constexpr int C0T_MP = 136;               // staged mel row: zero at 3, mel columns 0..127 at 4..131
+constexpr size_t C0T_SMEM = 56 * 1024;    // four CTAs per SM at most (4 x 57 KB with the runtime's reserve)
+// size bytes from global to shared memory, asynchronously; zeros where !valid
+__device__ __forceinline__ void c0_cp_async(void *dst, const void *src, bool valid, int size) {
+  const uint32_t d = smem_u32(dst);
+  if (size == 16)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(valid ? 16 : 0) : "memory");
+  else
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(d), "l"(src), "r"(valid ? 4 : 0) : "memory");
+}
+__device__ __forceinline__ void c0_cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void c0_cp_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+struct C0Row {  // where a stem row's three mel rows come from
+  int64_t base;
+  int ti, F;
+};
+__device__ __forceinline__ C0Row c0_row(const ClipTablesDev &t, int64_t row, int64_t stem_rows) {
+  C0Row r{0, -1, 0};
+  if (row < stem_rows) {
+    const int c = clip_of(t.stem_off, t.n_clips, row);
+    r.F = t.frame_off[c + 1] - t.frame_off[c];
+    r.ti = (int)(row - t.stem_off[c]) - 2;
+    if (r.ti >= (r.F + 1) / 2) r.ti = -1;
+    r.base = (int64_t)t.frame_off[c] * kMels;
+  }
+  return r;
+}
+}  // namespace
+
+__global__ void __launch_bounds__(128, 4) k_conv0_tc(const __grid_constant__ CUtensorMap tmY, const float *__restrict__ mel,
+                                                      bool mel16, const bf16 *__restrict__ bw,
+                                                      const float *__restrict__ cov, const ClipTablesDev t,
+                                                      int64_t stem_rows, int n_items, unsigned *status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // A, then (once the MMA has read it) the staged channels 0..63; B; the staged channels 64..127
+  uint8_t *sA = smem, *sB = smem + C0T_TILE, *sO = smem + 2 * C0T_TILE;
+  float *s_mel = reinterpret_cast<float *>(smem + 3 * C0T_TILE);  // [2 buffers][2 stem rows x 3][C0T_MP]
+  C0Row *s_row = reinterpret_cast<C0Row *>(s_mel + 2 * 6 * C0T_MP);  // [2 buffers][2]
+  uint64_t *bar = reinterpret_cast<uint64_t *>(s_row + 4);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, r7 = tid & 7;
+  // the mel rows of one item into buffer b: 16-byte pieces where the mel
+  // array allows (rows are 512 bytes), else 4-byte ones
+  auto stage = [&](int b) {
+    float *dst = s_mel + b * 6 * C0T_MP;
+    const int per_row = mel16 ? 32 : 128, w = mel16 ? 4 : 1;
+    for (int i = tid; i < 6 * per_row; i += 128) {
+      const int q = i / (3 * per_row), dt = (i / per_row) % 3, sg = i % per_row;
+      const C0Row R = s_row[2 * b + q];
+      const int tr = 2 * R.ti + dt - 1;
+      const bool valid = R.ti >= 0 && tr >= 0 && tr < R.F;
+      c0_cp_async(dst + (q * 3 + dt) * C0T_MP + 4 + sg * w, valid ? mel + R.base + (int64_t)tr * kMels + sg * w : mel,
+                  valid, 4 * w);
+    }
+    c0_cp_commit();
+  };
+  // B (the taps) into shared memory once, swizzled; A's granules 4..7 stay zero
+  for (int i = tid; i < 128 * 8; i += 128) {
+    const int n = i >> 3, g = i & 7;
+    *reinterpret_cast<uint4 *>(sB + n * 128 + ((g ^ (n & 7)) << 4)) = __ldg(reinterpret_cast<const uint4 *>(bw) + i);
+  }
+#pragma unroll
+  for (int g = 4; g < 8; ++g) *reinterpret_cast<uint4 *>(sA + tid * 128 + ((g ^ r7) << 4)) = make_uint4(0, 0, 0, 0);
+  for (int i = tid; i < 12; i += 128) s_mel[i * C0T_MP + 3] = 0.f;  // column -1 of every staged row
+  float cv[45];  // C_aa and 2 C_ab (b > a)
+  {
+    int n = 0;
+#pragma unroll
+    for (int a = 0; a < 9; ++a)
+#pragma unroll
+      for (int b = a; b < 9; ++b) cv[n++] = (b == a ? 1.0f : 2.0f) * __ldg(cov + a * 9 + b);
+  }
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tmY);
+  }
+  if (tid < 2) s_row[tid] = c0_row(t, (int64_t)blockIdx.x * 2 + tid, stem_rows);
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t trow = tmem + ((uint32_t)(32 * warp) << 16);
+  const int rr = tid >> 6, f = tid & 63;  // this thread's position: stem row rr of the item, frequency f
+  if (blockIdx.x < n_items) stage(0);
+  uint32_t phase = 0;
+  for (int item = blockIdx.x, it = 0; item < n_items; item += gridDim.x, ++it) {
+    const int b = it & 1;
+    const int next = item + gridDim.x;
+    if (tid < 2 && next < n_items) s_row[2 * (b ^ 1) + tid] = c0_row(t, (int64_t)next * 2 + tid, stem_rows);
+    c0_cp_wait_all();
+    if (tid == 0) bulk_wait_read<0>();  // the previous item's stores have read A's and sO's staged rows
+    __syncthreads();  // this item's rows have landed; the next item's sources are known
+    if (next < n_items) stage(b ^ 1);
+    const float *m = s_mel + b * 6 * C0T_MP + rr * 3 * C0T_MP + 3 + 2 * f;  // column 2f - 1 of the first row
+    float p[9];
+#pragma unroll
+    for (int dt = 0; dt < 3; ++dt)
+#pragma unroll
+      for (int df = 0; df < 3; ++df) p[dt * 3 + df] = m[dt * C0T_MP + df];
+    float var = 0.f;
+    {
+      int n = 0;
+#pragma unroll
+      for (int a = 0; a < 9; ++a) {
+        float sa = 0.f;
+#pragma unroll
+        for (int c = a; c < 9; ++c) sa = fmaf(cv[n++], p[c], sa);
+        var = fmaf(p[a], sa, var);
+      }
+    }
+    const float rinv = rsqrtf(fmaxf(var, 0.f) + 1e-6f);
+    {
+      float kv[32];
+#pragma unroll
+      for (int k = 0; k < 9; ++k) {
+        const float hi = __bfloat162float(__float2bfloat16_rn(p[k]));
+        kv[k] = hi;
+        kv[9 + k] = hi;
+        kv[18 + k] = p[k] - hi;
+      }
+#pragma unroll
+      for (int k = 27; k < 32; ++k) kv[k] = 0.f;
+#pragma unroll
+      for (int g = 0; g < 4; ++g)
+        *reinterpret_cast<uint4 *>(sA + tid * 128 + ((g ^ r7) << 4)) =
+            make_uint4(pack_bf16(kv[8 * g], kv[8 * g + 1]), pack_bf16(kv[8 * g + 2], kv[8 * g + 3]),
+                       pack_bf16(kv[8 * g + 4], kv[8 * g + 5]), pack_bf16(kv[8 * g + 6], kv[8 * g + 7]));
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t aa = smem_u32(sA), ab = smem_u32(sB);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        tc_mma_bf16(tmem, sw128_desc(aa + k * 32), sw128_desc(ab + k * 32), idesc_bf16_f32(128, 128), k > 0 ? 1u : 0u);
+      tc_commit(bar);
+    }
+    if (!__syncthreads_and(mbar_wait(bar, phase))) {
+      if (tid == 0) atomicOr(status, kStatusWaitTimeout);
+      break;
+    }
+    phase ^= 1;
+    tc_fence_after();
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {  // channels 32 c .. 32 c + 31: granules 4 (c & 1) .. +3 of a staged half
+      uint32_t v[32];
+      tmem_ld32(trow + 32 * c, v);
+      tmem_ld_wait();
+      uint8_t *line = (c < 2 ? sA : sO) + tid * 128;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int g = 4 * (c & 1) + j;
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          w[e] = pack_bf16(fmaxf(__uint_as_float(v[8 * j + 2 * e]) * rinv, 0.f),
+                           fmaxf(__uint_as_float(v[8 * j + 2 * e + 1]) * rinv, 0.f));
+        *reinterpret_cast<uint4 *>(line + ((g ^ r7) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+    tc_fence_before();
+    fence_async_smem();
+    __syncthreads();  // rows staged; tensor memory is free for the next item
+    if (tid == 0) {  // positions beyond the last stem row fall outside the map and are not written
+      tma_store_2d(&tmY, sA, 0, item * 128);
+      tma_store_2d(&tmY, sO, 64, item * 128);
+      bulk_commit();
+    }
+  }
+  if (tid == 0) bulk_wait_all();
+  c0_cp_wait_all();  // no copy may still be in flight when the CTA ends
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
 // ------------------------------------------------------------------ conv1, tensor cores (bf16)
 
 namespace {
@@ -331,9 +538,20 @@ cudaError_t launch_conv0(const ae_model *m, const float *mel, void *y0, const Cl
                          cudaStream_t s) {
   if (stem_rows <= 0) return cudaSuccess;
   const unsigned grid = (unsigned)((stem_rows + kConv0Rows - 1) / kConv0Rows);
-  if (m->dtype != AE_F32)
-    return launch_k(k_conv0<bf16>, dim3(grid), dim3(128), 0, s, mel, (const float *)m->conv0c,
-                    (const float *)m->conv0cov, static_cast<bf16 *>(y0), t, stem_rows);
+  if (m->dtype != AE_F32) {
+    static std::atomic<uint64_t> attr{0};
+    if (const cudaError_t e = smem_attr(k_conv0_tc, C0T_SMEM, attr)) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t items = (stem_rows + 1) / 2;
+    const unsigned g = (unsigned)std::min<int64_t>(items, 4 * (int64_t)(sms > 0 ? sms : 148));
+    const bool mel16 = (reinterpret_cast<uintptr_t>(mel) & 15) == 0;
+    CUtensorMap tm;  // y0 as [stem rows x 64 positions][128 channels], boxes of 128 positions x 64 channels
+    if (!make_tmap_2d_bf16(&tm, y0, kC0, (uint64_t)stem_rows * kF1, kC0 * 2, 64, 128)) return cudaErrorInvalidValue;
+    return launch_k(k_conv0_tc, dim3(g), dim3(128), C0T_SMEM, s, tm, mel, mel16, static_cast<const bf16 *>(m->conv0b),
+                    (const float *)m->conv0cov, t, stem_rows, (int)items, device_status_word());
+  }
   return launch_k(k_conv0<float>, dim3(grid), dim3(128), 0, s, mel, (const float *)m->conv0c,
                   (const float *)m->conv0cov, static_cast<float *>(y0), t, stem_rows);
 }

@@ -139,6 +139,23 @@ def test_encode_edges_and_packing(m2, w2):
             assert np.array_equal(alone, g[off[i]:off[i + 1]])
 
 
+def test_packed_batch_matches_single_clips(m2, w2):
+    """Eight clips of 10-30 s packed into one call (2,376 tokens): every clip's
+    rows equal the clip encoded alone, bit for bit, and two of them match the
+    oracle."""
+    lens = [480000] * 3 + [320000, 160000, 240000, 400000, 480000]
+    mels = _mels(lens, seed=41)
+    g, toks = _gpu_encode(m2, mels)
+    assert sum(toks) >= 2048 and len(toks) >= 2
+    off = offsets(toks)
+    for i, x in enumerate(mels):
+        alone, _ = _gpu_encode(m2, [x])
+        assert np.array_equal(alone, g[off[i]:off[i + 1]]), f"clip {i} differs from the clip alone"
+    for i in (3, 4):
+        o = E.encode(mels[i].astype(np.float64), w2)
+        assert_bf16(g[off[i]:off[i + 1]], o, f"LFM2A encode in a split batch, clip {i} ({toks[i]} tokens)")
+
+
 def test_refusals(m2):
     off = offsets([16])
     with pytest.raises(ae.AEError) as e:
