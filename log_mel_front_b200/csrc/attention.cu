@@ -47,14 +47,15 @@ namespace ae {
 //     start);
 //   * tcgen05.mma (A = P from tensor memory, M=128, N=128, K=144, v read
 //     MN-major) gives O = P V;
-//   * the q warps drain O, clamp it and store it from registers, whole 32-byte
-//     sectors per row where the output's alignment allows.
+//   * the softmax warps (head dims 64..127) and the q warps (0..63) drain O,
+//     clamp it and store it from registers, whole 32-byte sectors per row
+//     where the output's alignment allows.
 // The stages overlap across items: the q warps split item i+1 as soon as the
 // score MMA of item i has read the previous split, while the softmax warps
-// work on item i; the MMA warp issues the score MMA of item i+1 before the
-// P V MMA of item i; the q warps drain item i after splitting item i+1. A
-// stage's q/k are reloaded once the score MMA that read them completes, its v
-// once the P V MMA has.
+// work on item i; the MMA warp issues item i's P V as soon as its P is
+// written, then item i+1's score MMA; both warp groups drain item i while the
+// score MMA of item i+1 runs. A stage's q/k are reloaded once the score MMA
+// that read them completes, its v once the P V MMA has.
 namespace {
 constexpr int AT_Q = 128;                                  // queries per item
 constexpr int AT_KEYS = 144;                               // key rows per item (139 used)
@@ -69,6 +70,7 @@ constexpr uint32_t AT_STAGE = OFF_V + 2 * AT_V_REGION;     // 108 KB
 constexpr uint32_t OFF_BAR = 2 * AT_STAGE;
 constexpr size_t AT_SMEM = OFF_BAR + 1024 + 1024;          // barriers + q scales, alignment slack
 constexpr int AT_THREADS = 320;                            // producer, MMA, 4 softmax warps, 4 q warps
+constexpr int AT_DRAIN_THREADS = 256;                      // both warp groups drain half of O
 constexpr uint32_t AT_TMEM_COLS = 512;
 constexpr uint32_t COL_S = 0;                              // scores, 160 f32 columns
 constexpr uint32_t COL_P = 160;                            // banded P, 160 bf16 = 80 columns
@@ -160,7 +162,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     mbar_init(s_free, 128);
     mbar_init(p_full, 128);
     mbar_init(o_full, 1);
-    mbar_init(o_empty, 128);
+    mbar_init(o_empty, AT_DRAIN_THREADS);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
@@ -176,6 +178,38 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // O rows of item j, head dims 64 hw .. 64 hw + 63, out by the warp of lane quarter warp & 3
+  auto drain_half = [&](int j, int jitem, int hw) -> bool {
+    if (!__all_sync(0xffffffffu, mbar_wait(o_full, j & 1))) return false;
+    tc_fence_after();
+    const int qw = warp & 3, r = 32 * qw + lane;
+    const uint32_t trow = tmem + ((uint32_t)(32 * qw) << 16);
+    const int t = (jitem >> 3) * AT_Q + r, h = jitem & 7;
+    bf16 *orow = out + (int64_t)t * ld_out + h * kHeadDim + 64 * hw;
+#pragma unroll 1
+    for (int c = 0; c < 2; ++c) {
+      uint32_t o[32];
+      tmem_ld32(trow + COL_O + 64 * hw + 32 * c, o);
+      tmem_ld_wait();
+      uint32_t w[16];
+#pragma unroll
+      for (int j2 = 0; j2 < 16; ++j2)
+        w[j2] = pack_bf16(clampf(__uint_as_float(o[2 * j2]), lo, hi), clampf(__uint_as_float(o[2 * j2 + 1]), lo, hi));
+      if (t < T) {
+        if (out_v8) {
+          at_st32B(orow + 32 * c, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+          at_st32B(orow + 32 * c + 16, w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]);
+        } else {
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            *reinterpret_cast<uint4 *>(orow + 32 * c + 8 * g) = make_uint4(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
+        }
+      }
+    }
+    tc_fence_before();
+    mbar_arrive(o_empty);
+    return true;
+  };
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer
@@ -212,7 +246,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       if (uv > 0) mbar_wait(&v_full[st], (uv - 1) & 1);
     }
   } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer: the score MMA of item i, then the P V MMA of item i - 1
+    // ---------------- MMA issuer: the score MMA of item i, then (once P is written) its P V MMA
     constexpr uint32_t idesc_s = idesc_bf16_f32(AT_Q, AT_BROWS);
     constexpr uint32_t idesc_o = idesc_bf16_f32_bmn(AT_Q, kHeadDim);
     bool ok = true;
@@ -249,9 +283,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       }
       tc_commit(&qk_free[st]);
       tc_commit(s_full);
-      if (it > 0 && !pv(it - 1)) { ok = false; break; }
+      if (!pv(it)) { ok = false; break; }
     }
-    if (ok && it > 0 && !pv(it - 1)) ok = false;
     if (!ok) {
       atomicOr(status, kStatusWaitTimeout);
       *abort_flag = 1;
@@ -346,13 +379,12 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       uint32_t pw[32];
 #pragma unroll
       for (int k = 0; k < 32; ++k) pw[k] = k < 22 ? w[k] : 0u;
-      // the previous item's P V has read P
-      if (it > 0 && !__all_sync(0xffffffffu, mbar_wait(o_full, (it - 1) & 1))) { ok = false; break; }
-      tc_fence_after();
+      // the previous item's P V has read P: these warps waited for it before draining it
       at_tmem_st32(trow + COL_P + 16 * qw, pw);
       at_tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full);
+      if (!drain_half(it, item, 1)) { ok = false; break; }
     }
     if (!ok && lane == 0) {
       atomicOr(status, kStatusWaitTimeout);
@@ -370,36 +402,6 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     }
     const float inv_ks = 1.0f / k_scale;
     bool ok = true;
-    auto drain = [&](int j, int jitem) -> bool {  // O rows of item j out
-      if (!__all_sync(0xffffffffu, mbar_wait(o_full, j & 1))) return false;
-      tc_fence_after();
-      const int t = (jitem >> 3) * AT_Q + r, h = jitem & 7;
-      bf16 *orow = out + (int64_t)t * ld_out + h * kHeadDim;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t o[32];
-        tmem_ld32(trow + COL_O + 32 * c, o);
-        tmem_ld_wait();
-        uint32_t w[16];
-#pragma unroll
-        for (int j2 = 0; j2 < 16; ++j2)
-          w[j2] = pack_bf16(clampf(__uint_as_float(o[2 * j2]), lo, hi), clampf(__uint_as_float(o[2 * j2 + 1]), lo, hi));
-        if (t < T) {
-          if (out_v8) {
-            at_st32B(orow + 32 * c, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
-            at_st32B(orow + 32 * c + 16, w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]);
-          } else {
-#pragma unroll
-            for (int g = 0; g < 4; ++g)
-              *reinterpret_cast<uint4 *>(orow + 32 * c + 8 * g) =
-                  make_uint4(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(o_empty);
-      return true;
-    };
     int it = 0, prev_item = -1;
     int r_head0 = -1, r_head1 = -1;  // the head whose R rows each stage holds (one head per stage
                                      // when the grid is a multiple of 4, as on 148 SMs)
@@ -449,10 +451,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       tc_fence_before();
       fence_async_smem();
       mbar_arrive(q_ready);
-      if (it > 0 && !drain(it - 1, prev_item)) { ok = false; break; }
+      if (it > 0 && !drain_half(it - 1, prev_item, 0)) { ok = false; break; }
       prev_item = item;
     }
-    if (ok && it > 0 && !drain(it - 1, prev_item)) ok = false;
+    if (ok && it > 0 && !drain_half(it - 1, prev_item, 0)) ok = false;
     if (!ok && lane == 0) {
       atomicOr(status, kStatusWaitTimeout);
       *abort_flag = 1;
