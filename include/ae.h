@@ -232,6 +232,18 @@ ae_status ae_conformer_layer(const ae_model *m, int layer, float *d_h, const int
 ae_status ae_encode(const ae_model *m, const float *d_wave, const int64_t *h_sample_off,
                     int n_clips, float *d_out, void *d_ws, size_t ws_bytes, ae_stream stream);
 
+/* ae_encode with per-stage copies, the `trace` of AudioTower::encode_mels
+ * (egemma2_audio.rs: the subsampling output, every layer's output and the
+ * tower output, all packed), for stage-by-stage comparison. One pass on
+ * `stream` (no half-batch split). d_mel (nullable): float32 [sum frames][128],
+ * the log-mel rows. d_trace (nullable): float32 [n_layers + 1][sum tokens]
+ * [hidden]: slot 0 the residual stream after in_proj, slot l + 1 after layer
+ * l. d_out, the workspace and the errors are those of ae_encode; the copies
+ * are device-to-device, asynchronous on `stream`. */
+ae_status ae_encode_trace(const ae_model *m, const float *d_wave, const int64_t *h_sample_off, int n_clips,
+                          float *d_out, float *d_mel, float *d_trace, void *d_ws, size_t ws_bytes,
+                          ae_stream stream);
+
 /* ae_encode from host memory to host memory: copies h_wave into the
  * workspace, runs ae_encode, copies the rows back to h_out and waits for
  * the stream. Pinned host buffers make the copies asynchronous DMA. The

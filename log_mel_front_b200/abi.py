@@ -83,6 +83,7 @@ _sig("ae_logmel", _st, _vp, _i64p, _i32, _vp, _vp, _sz, _vp)
 _sig("ae_subsample", _st, _vp, _vp, _i64p, _i32, _vp, _vp, _sz, _vp)
 _sig("ae_conformer_layer", _st, _vp, _i32, _vp, _i64p, _i32, _vp, _sz, _vp)
 _sig("ae_encode", _st, _vp, _vp, _i64p, _i32, _vp, _vp, _sz, _vp)
+_sig("ae_encode_trace", _st, _vp, _vp, _i64p, _i32, _vp, _vp, _vp, _vp, _sz, _vp)
 _sig("ae_encode_host_workspace_size", _sz, _vp, _i64p, _i32)
 _sig("ae_encode_host", _st, _vp, _vp, _i64p, _i32, _vp, _vp, _sz, _vp)
 _sig("ae_encode_host_async", _st, _vp, _vp, _i64p, _i32, _vp, _vp, _sz, _vp)
@@ -109,7 +110,8 @@ _sig("ae_profile_read", _st, C.POINTER(C.c_double), _i64p, C.POINTER(C.c_double)
 
 # every symbol include/ae.h declares
 EXPORTS = ("ae_num_frames", "ae_num_tokens", "ae_model_create", "ae_model_destroy", "ae_workspace_size",
-           "ae_logmel", "ae_subsample", "ae_conformer_layer", "ae_encode", "ae_encode_host_workspace_size",
+           "ae_logmel", "ae_subsample", "ae_conformer_layer", "ae_encode", "ae_encode_trace",
+           "ae_encode_host_workspace_size",
            "ae_encode_host", "ae_encode_host_async", "ae_attention_tables", "ae_local_attention", "ae_last_error",
            "ae_device_status", "ae_version", "ae_profile_enable", "ae_profile_read", "ae_logmel_noalloc",
            "ae_resample_len", "ae_resample_workspace_size", "ae_resample", "ae_linear_e4m3",
@@ -219,6 +221,12 @@ def ae_encode(model, d_wave, sample_off, d_out, d_ws, ws_bytes: int, stream=None
     a, p = _off(sample_off)
     _check(lib.ae_encode(model.handle, _ptr(d_wave), p, len(a) - 1, _ptr(d_out), _ptr(d_ws), ws_bytes,
                          _stream(stream)), "ae_encode")
+
+
+def ae_encode_trace(model, d_wave, sample_off, d_out, d_mel, d_trace, d_ws, ws_bytes: int, stream=None):
+    a, p = _off(sample_off)
+    _check(lib.ae_encode_trace(model.handle, _ptr(d_wave), p, len(a) - 1, _ptr(d_out), _ptr(d_mel), _ptr(d_trace),
+                               _ptr(d_ws), ws_bytes, _stream(stream)), "ae_encode_trace")
 
 
 def ae_encode_host_workspace_size(model, sample_off) -> int:

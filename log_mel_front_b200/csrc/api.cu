@@ -543,8 +543,15 @@ static ae_status check_ws(void *ws, size_t have, size_t need) {
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 // The encode sequence on device buffers (shared by ae_encode and ae_encode_host).
+// Optional per-stage copies of one pass (the page's `trace` of encode_mels):
+// the log-mel rows and the residual stream after in_proj and after each layer.
+struct TraceOut {
+  float *mel = nullptr;     // [sum frames][128]
+  float *layers = nullptr;  // [n_layers + 1][sum tokens][hidden]
+};
+
 static ae_status encode_one(const ae_model *m, const float *d_wave, const ClipTables &T, float *d_out, void *d_ws,
-                            const WsLayout &L, cudaStream_t s) {
+                            const WsLayout &L, cudaStream_t s, const TraceOut *tr = nullptr) {
   ClipTablesDev td;
   cudaError_t e = tables_t(T, d_ws, L, &td, true, s);
   if (e != cudaSuccess) return cuda_fail(e, "table upload");
@@ -553,16 +560,28 @@ static ae_status encode_one(const ae_model *m, const float *d_wave, const ClipTa
   float *mel = reinterpret_cast<float *>(w + L.mel);
   Bufs b = bufs_of(d_ws, L, td);
   if ((e = logmel_t(d_wave, mel, td, T, s)) != cudaSuccess) return cuda_fail(e, "logmel");
+  const size_t h_bytes = (size_t)T.total_tokens * m->cfg.hidden * 4;
+  auto trace_h = [&](int slot) -> cudaError_t {  // the residual stream into trace slot `slot`
+    if (!tr || !tr->layers) return cudaSuccess;
+    return cudaMemcpyAsync(reinterpret_cast<uint8_t *>(tr->layers) + (size_t)slot * h_bytes, b.h, h_bytes,
+                           cudaMemcpyDeviceToDevice, s);
+  };
+  if (tr && tr->mel &&
+      (e = cudaMemcpyAsync(tr->mel, mel, (size_t)T.total_frames * kMels * 4, cudaMemcpyDeviceToDevice, s)) !=
+          cudaSuccess)
+    return cuda_fail(e, "trace copy");
   if ((e = conv0_t(m, mel, w + L.y0, td, T, s)) != cudaSuccess) return cuda_fail(e, "conv0");
   if ((e = conv1_t(m, w + L.y0, w + L.xs, td, T, s)) != cudaSuccess)
     return cuda_fail(e, "conv1");
   if ((e = gemm_t(m, w + L.xs, T.total_tokens, kHidden, m->in_proj, m->dtype != AE_F32 ? &m->tm_in_proj : nullptr,
                 m->cfg.hidden, EPI_F32, ep_of(b.h, m->cfg.hidden, -INFINITY, INFINITY), s)) != cudaSuccess)
     return cuda_fail(e, "in_proj");
+  if ((e = trace_h(0)) != cudaSuccess) return cuda_fail(e, "trace copy");
   const int nl = m->cfg.n_layers;
   for (int li = 0; li < nl; ++li) {
     e = run_layer(m, li, b, T.total_tokens, li > 0, li + 1 < nl ? kNextLayer : kNextPlain, s);
     if (e != cudaSuccess) return cuda_fail(e, "layer");
+    if ((e = trace_h(li + 1)) != cudaSuccess) return cuda_fail(e, "trace copy");
   }
   if (nl == 0) {
     RowArgs r = row_of(b.h, m->cfg.hidden, T.total_tokens);
@@ -1041,6 +1060,24 @@ ae_status ae_encode(const ae_model *m, const float *d_wave, const int64_t *h_sam
   if (n_clips == 0) return AE_OK;
   if ((st = check_ws(d_ws, ws_bytes, need))) return st;
   return encode_dev(m, d_wave, T, d_out, d_ws, need, reinterpret_cast<cudaStream_t>(stream), true);
+}
+
+ae_status ae_encode_trace(const ae_model *m, const float *d_wave, const int64_t *h_sample_off, int n_clips,
+                          float *d_out, float *d_mel, float *d_trace, void *d_ws, size_t ws_bytes, ae_stream stream) {
+  ae_status st = check_model(m);
+  if (st) return st;
+  ClipTables T;
+  if ((st = build_tables(h_sample_off, n_clips, kSamples, T, "h_sample_off"))) return st;
+  if (T.total_tokens > 0 && (!d_wave || !d_out)) return fail(AE_EINVAL, "d_wave or d_out is null");
+  if (!aligned16(d_out)) return fail(AE_EINVAL, "d_out is not 16-byte aligned");
+  const size_t need = encode_ws_bytes(m, T.n_clips, T.total_frames, T.total_tokens);
+  if (n_clips == 0) return AE_OK;
+  if ((st = check_ws(d_ws, ws_bytes, need))) return st;
+  TraceOut tr;
+  tr.mel = d_mel;
+  tr.layers = d_trace;
+  const WsLayout L = ws_layout(m, T.n_clips, T.total_frames, T.total_tokens, true);
+  return encode_one(m, d_wave, T, d_out, d_ws, L, reinterpret_cast<cudaStream_t>(stream), &tr);
 }
 
 size_t ae_encode_host_workspace_size(const ae_model *m, const int64_t *h_sample_off, int n_clips) {

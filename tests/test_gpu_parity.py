@@ -206,6 +206,54 @@ def test_encode_pr1_f32(m_pr1, w_pr1):
     assert_f32(g, o, "encode pr1")
 
 
+def _trace_case(model, W, clips):
+    """ae_encode_trace on clips; returns the GPU stages and the oracle's trace."""
+    flat, off = synth.pack(clips)
+    frames = sum(O.num_frames(len(c)) for c in clips)
+    toks = sum(O.num_tokens(len(c)) for c in clips)
+    H, nl = W["shape"]["hidden"], len(W["layers"])
+    d_wave = dev(flat)
+    d_out = torch.full((toks, W["shape"]["embed_dim"]), float("nan"), device="cuda")
+    d_mel = torch.full((frames, 128), float("nan"), device="cuda")
+    d_tr = torch.full((nl + 1, toks, H), float("nan"), device="cuda")
+    ws = workspace(model.workspace_size(len(clips), frames, toks))
+    ae.ae_encode_trace(model, d_wave, off, d_out, d_mel, d_tr, ws, ws.numel())
+    _sync()
+    g = (d_mel.cpu().numpy(), d_tr.cpu().numpy(), d_out.cpu().numpy())
+    # without trace buffers the call is ae_encode: the same rows, bit for bit
+    d_out2 = torch.full_like(d_out, float("nan"))
+    ae.ae_encode_trace(model, d_wave, off, d_out2, None, None, ws, ws.numel())
+    _sync()
+    assert np.array_equal(d_out2.cpu().numpy(), g[2])
+    o, tr = O.encode(clips, W, trace=True)
+    return g, (np.concatenate(tr["mels"]), tr["subsample"], tr["layers"], np.concatenate(o))
+
+
+def test_encode_trace_stages_f32(m_pr1, w_pr1):
+    """The per-stage dump (encode_mels' trace): log-mel rows, the residual
+    stream after in_proj and after the layer, and the output of two packed
+    clips, each against the oracle's trace of the same call."""
+    wave = synth.pr1_wave()
+    (mel, tr, out), (o_mel, o_sub, o_layers, o_out) = _trace_case(m_pr1, w_pr1, [wave, wave[:9000]])
+    assert_logmel(mel, o_mel, "trace: log-mel")
+    assert_f32(tr[0], o_sub, "trace: after in_proj")
+    for li, ol in enumerate(o_layers):
+        assert_f32(tr[li + 1], ol, f"trace: after layer {li}")
+    assert_f32(out, o_out, "trace: output")
+
+
+def test_encode_trace_stages_bf16_tower(m_tower, w_tower):
+    """The same dump through all 12 bf16 layers of the tower model, two clips."""
+    clips = [c[:24000] for c in synth.waves("tower")[:2]]
+    (mel, tr, out), (o_mel, o_sub, o_layers, o_out) = _trace_case(m_tower, w_tower, clips)
+    assert len(o_layers) == 12 and tr.shape[0] == 13
+    assert_logmel(mel, o_mel, "trace: log-mel")
+    assert_bf16(tr[0], o_sub, "trace: after in_proj")
+    for li, ol in enumerate(o_layers):
+        assert_bf16(tr[li + 1], ol, f"trace: after layer {li}")
+    assert_bf16(out, o_out, "trace: output")
+
+
 def test_encode_tower_full_batch_sampled_clips(m_tower, w_tower):
     clips = synth.waves("tower")
     g, off = gpu_encode(m_tower, clips)
