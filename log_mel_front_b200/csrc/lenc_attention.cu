@@ -7,7 +7,10 @@
 // so row (t_max - 1 - r) is distance r.
 //
 // One CTA per (clip, 128-query block, head); warp 0 loads tiles with TMA,
-// warp 1 issues tcgen05.mma, warps 2-5 own one query row per thread. Per
+// warp 1 issues tcgen05.mma, and two row warps per 32-row quarter of the tile
+// own a query row per thread, each warp half of the keys (64 of a block's 128)
+// and half of the output dims; the two exchange their rows' block maxima and
+// final sums through shared memory (64-arrival mbarriers per quarter). Per
 // 128-key block:
 //   * TMA: the 128 key rows and value rows of the block, and the 256 position
 //     rows of the distances the block spans (r = i - j from i0 - j0 - 127 to
@@ -20,7 +23,8 @@
 //     chunks of T that cover its window for 32 keys, writes them into its row
 //     of a per-warp scratch (row pitch 66 floats) and reads them back from
 //     offset 31 - lane (conflict-free: 65 lane + const); then adds S, scales
-//     and masks keys past the clip end, 32 keys at a time;
+//     and masks keys past the clip end, 32 keys at a time (two such chunks per
+//     warp and block);
 //   * online softmax over the key blocks: the row thread keeps its row's
 //     running maximum and sum, writes the block's probabilities (relative to
 //     the new maximum) as bf16 (K-major, 128-byte swizzle), and, when the
@@ -40,11 +44,13 @@ constexpr uint32_t XA_TILE = 128 * 128;               // 128 rows x 64 bf16
 constexpr uint32_t OFF_QU = 0, OFF_QV = OFF_QU + XA_TILE, OFF_K = OFF_QV + XA_TILE, OFF_V = OFF_K + XA_TILE;
 constexpr uint32_t OFF_PB = OFF_V + XA_TILE;             // 256 position rows
 constexpr uint32_t OFF_S = OFF_PB + 2 * XA_TILE;         // probabilities: two 64-key regions
-constexpr uint32_t OFF_SCR = OFF_S + 2 * XA_TILE;        // skew scratch, 4 warps x 32 rows x 66 floats
+constexpr uint32_t OFF_SCR = OFF_S + 2 * XA_TILE;        // skew scratch, 8 warps x 32 rows x 66 floats
 constexpr int SCR_PITCH = 66;
-constexpr uint32_t OFF_BAR = OFF_SCR + 4 * 32 * SCR_PITCH * 4;
+constexpr uint32_t OFF_X = OFF_SCR + 8 * 32 * SCR_PITCH * 4;  // [2 block parities][2 key halves][128] maxima, [2][128] sums
+constexpr uint32_t OFF_BAR = OFF_X + (2 * 2 * 128 + 2 * 128) * 4;
 constexpr size_t XA_SMEM = OFF_BAR + 256 + 1024;
-constexpr int XA_THREADS = 192;
+constexpr int XA_THREADS = 320;
+constexpr int XA_ROW_THREADS = 256;
 constexpr uint32_t XA_TMEM_COLS = 512, COL_S = 0, COL_T = 128, COL_O = 384;
 constexpr uint32_t XA_KV_BYTES = 4 * XA_TILE;            // K, V and two position boxes
 static_assert(XA_SMEM <= 227 * 1024, "shared memory");
@@ -80,6 +86,8 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
   uint64_t *q_full = bars, *q_ready = bars + 1, *kv_full = bars + 2, *s_full = bars + 3, *s_free = bars + 4,
            *p_full = bars + 5, *o_full = bars + 6;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 7);
+  // per lane quarter: the two row warps' exchanges (q tiles read, block maxima, final sums)
+  uint64_t *xq = bars + 8, *xm = bars + 12, *xs = bars + 16;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -100,12 +108,17 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    mbar_init(q_ready, 128);
+    mbar_init(q_ready, XA_ROW_THREADS);
     mbar_init(kv_full, 1);
     mbar_init(s_full, 1);
-    mbar_init(s_free, 128);
-    mbar_init(p_full, 128);
+    mbar_init(s_free, XA_ROW_THREADS);
+    mbar_init(p_full, XA_ROW_THREADS);
     mbar_init(o_full, 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&xq[i], 64);
+      mbar_init(&xm[i], 64);
+      mbar_init(&xs[i], 64);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQKV);
@@ -183,44 +196,54 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
       *abort_flag = 1;
     }
   } else if (warp >= 2) {
-    // ---------------- row threads: TMEM lane quarter qw, query row li = 32 qw + lane
-    const int qw = warp & 3, li = 32 * qw + lane, r7 = li & 7;
+    // ---------------- row threads: TMEM lane quarter qw, query row li = 32 qw + lane;
+    // warp half kh: keys 64 kh .. 64 kh + 63 of each block, output dims 32 kh .. 32 kh + 31
+    const int qw = warp & 3, kh = (warp - 2) >> 2, li = 32 * qw + lane, r7 = li & 7;
     const uint32_t trow = tmem + ((uint32_t)(32 * qw) << 16);
-    float *my = scr + (size_t)(qw * 32 + lane) * SCR_PITCH;
+    float *my = scr + (size_t)((kh * 4 + qw) * 32 + lane) * SCR_PITCH;
+    float *xmax = reinterpret_cast<float *>(smem + OFF_X), *xsum = xmax + 2 * 2 * 128;
+    // the two warps of a quarter meet at an mbarrier of 64 arrivals (bounded wait)
+    auto pair_sync = [&](uint64_t *b, uint32_t parity) -> bool {
+      mbar_arrive(b);
+      return __all_sync(0xffffffffu, mbar_wait(b, parity));
+    };
     bool ok = true;
-    // ---- q + u and q + v as bf16 operand tiles
+    // ---- q + u (warp half 0) and q + v (half 1) as bf16 operand tiles, in place
+    // of / beside the raw q rows, once both halves have read them
     if (!__all_sync(0xffffffffu, mbar_wait(q_full, 0))) ok = false;
-    if (ok) {
+    {
+      uint4 w[8];
 #pragma unroll
-      for (int g = 0; g < 8; ++g) {
-        const uint32_t off = li * 128 + ((g ^ r7) << 4);
-        const uint4 w = *reinterpret_cast<const uint4 *>(sQu + off);
-        const float q[8] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y),
-                            bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w)};
-        const float4 u0 = *reinterpret_cast<const float4 *>(bias_u + head * XA_HD + 8 * g);
-        const float4 u1 = *reinterpret_cast<const float4 *>(bias_u + head * XA_HD + 8 * g + 4);
-        const float4 v0 = *reinterpret_cast<const float4 *>(bias_v + head * XA_HD + 8 * g);
-        const float4 v1 = *reinterpret_cast<const float4 *>(bias_v + head * XA_HD + 8 * g + 4);
-        *reinterpret_cast<uint4 *>(sQu + off) =
-            make_uint4(pack_bf16(q[0] + u0.x, q[1] + u0.y), pack_bf16(q[2] + u0.z, q[3] + u0.w),
-                       pack_bf16(q[4] + u1.x, q[5] + u1.y), pack_bf16(q[6] + u1.z, q[7] + u1.w));
-        *reinterpret_cast<uint4 *>(sQv + off) =
-            make_uint4(pack_bf16(q[0] + v0.x, q[1] + v0.y), pack_bf16(q[2] + v0.z, q[3] + v0.w),
-                       pack_bf16(q[4] + v1.x, q[5] + v1.y), pack_bf16(q[6] + v1.z, q[7] + v1.w));
+      for (int g = 0; g < 8; ++g) w[g] = *reinterpret_cast<const uint4 *>(sQu + li * 128 + ((g ^ r7) << 4));
+      if (!pair_sync(&xq[qw], 0)) ok = false;
+      if (ok) {
+        const float *bias = (kh == 0 ? bias_u : bias_v) + head * XA_HD;
+        uint8_t *dst = kh == 0 ? sQu : sQv;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          const float q[8] = {bf16lo(w[g].x), bf16hi(w[g].x), bf16lo(w[g].y), bf16hi(w[g].y),
+                              bf16lo(w[g].z), bf16hi(w[g].z), bf16lo(w[g].w), bf16hi(w[g].w)};
+          const float4 b0 = *reinterpret_cast<const float4 *>(bias + 8 * g);
+          const float4 b1 = *reinterpret_cast<const float4 *>(bias + 8 * g + 4);
+          *reinterpret_cast<uint4 *>(dst + li * 128 + ((g ^ r7) << 4)) =
+              make_uint4(pack_bf16(q[0] + b0.x, q[1] + b0.y), pack_bf16(q[2] + b0.z, q[3] + b0.w),
+                         pack_bf16(q[4] + b1.x, q[5] + b1.y), pack_bf16(q[6] + b1.z, q[7] + b1.w));
+        }
+        fence_async_smem();
       }
-      fence_async_smem();
     }
     mbar_arrive(q_ready);
     constexpr float kScale = 0.125f * 1.4426950408889634f;  // 1/sqrt(64), in base 2
-    float m_run = -INFINITY, l_run = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;  // l_run: this warp half's keys only
     for (int kb = 0; kb < n_kb && ok; ++kb) {
-      const int j0 = kb * XA_K;
+      const int j0 = kb * XA_K + 64 * kh;
       if (!__all_sync(0xffffffffu, mbar_wait(s_full, kb & 1))) { ok = false; break; }
       tc_fence_after();
-      // ---- the block's 128 logits: S plus the skewed window of T
-      float z[XA_K];
+      // ---- this half's 64 logits: S plus the skewed window of T
+      float z[64];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int qq = 0; qq < 2; ++qq) {
+        const int q = 2 * kh + qq;  // 32-key chunk of the block
         uint32_t a[32], b[32];
         const int ca = 3 - qw + q;  // chunk of T holding column 127 - li + 32 q (or the next one)
         tmem_ld32(trow + COL_T + 32 * ca, a);
@@ -237,8 +260,8 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
         __syncwarp();
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
-          const int j = j0 + 32 * q + x;
-          z[32 * q + x] = j < t_c ? (__uint_as_float(a[x]) + my[31 - lane + x]) * kScale : -INFINITY;
+          const int j = j0 + 32 * qq + x;
+          z[32 * qq + x] = j < t_c ? (__uint_as_float(a[x]) + my[31 - lane + x]) * kScale : -INFINITY;
         }
         __syncwarp();
       }
@@ -246,8 +269,11 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
       mbar_arrive(s_free);  // this block's scores are read
       float bm = -INFINITY;
 #pragma unroll
-      for (int x = 0; x < XA_K; ++x) bm = fmaxf(bm, z[x]);
-      const float m_new = fmaxf(m_run, bm);   // finite: every block holds a key of the clip
+      for (int x = 0; x < 64; ++x) bm = fmaxf(bm, z[x]);
+      xmax[((kb & 1) * 2 + kh) * 128 + li] = bm;
+      if (!pair_sync(&xm[qw], kb & 1)) { ok = false; break; }
+      // finite: every block holds a key of the clip, in one half or the other
+      const float m_new = fmaxf(m_run, fmaxf(bm, xmax[((kb & 1) * 2 + (kh ^ 1)) * 128 + li]));
       const float alpha = exp2f(m_run - m_new);  // 0 on the first block
       // the previous block's P V is done: the probabilities' buffer is free and
       // the accumulator holds every earlier block
@@ -255,29 +281,26 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
       tc_fence_after();
       float ls = 0.f;
 #pragma unroll
-      for (int g = 0; g < 16; ++g) {
+      for (int g = 0; g < 8; ++g) {  // granules 0..7 of region kh: keys 64 kh + 8 g ..
         float p[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           p[e] = exp2f(z[8 * g + e] - m_new);
           ls += p[e];
         }
-        *reinterpret_cast<uint4 *>(sS + (g >> 3) * XA_TILE + li * 128 + (((g & 7) ^ r7) << 4)) =
+        *reinterpret_cast<uint4 *>(sS + kh * XA_TILE + li * 128 + ((g ^ r7) << 4)) =
             make_uint4(pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]), pack_bf16(p[4], p[5]), pack_bf16(p[6], p[7]));
       }
       l_run = l_run * alpha + ls;
       m_run = m_new;
       if (kb > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
-        // rescale this row of the accumulator to the new maximum
+        // rescale this warp's 32 columns of the row's accumulator to the new maximum
+        uint32_t o[32];
+        tmem_ld32(trow + COL_O + 32 * kh, o);
+        tmem_ld_wait();
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          uint32_t o[32];
-          tmem_ld32(trow + COL_O + 32 * h2, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int d = 0; d < 32; ++d) o[d] = __float_as_uint(__uint_as_float(o[d]) * alpha);
-          xa_tmem_st32(trow + COL_O + 32 * h2, o);
-        }
+        for (int d = 0; d < 32; ++d) o[d] = __float_as_uint(__uint_as_float(o[d]) * alpha);
+        xa_tmem_st32(trow + COL_O + 32 * kh, o);
         xa_tmem_st_wait();
       }
       tc_fence_before();
@@ -285,28 +308,24 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
       mbar_arrive(p_full);
     }
     if (ok && !__all_sync(0xffffffffu, mbar_wait(o_full, (n_kb - 1) & 1))) ok = false;
+    // both halves' sums (also after a failure; the wait is bounded either way)
+    xsum[kh * 128 + li] = l_run;
+    if (!pair_sync(&xs[qw], 0)) ok = false;
     if (ok) {
       tc_fence_after();
-      const float inv = 1.0f / l_run;
-      uint32_t o0[32], o1[32];
-      tmem_ld32(trow + COL_O, o0);
-      tmem_ld32(trow + COL_O + 32, o1);
+      const float inv = 1.0f / (l_run + xsum[(kh ^ 1) * 128 + li]);
+      uint32_t o0[32];
+      tmem_ld32(trow + COL_O + 32 * kh, o0);
       tmem_ld_wait();
       if (i0 + li < t_c) {
-        bf16 *orow = out + (int64_t)(tok0 + i0 + li) * ld_out + head * XA_HD;
+        bf16 *orow = out + (int64_t)(tok0 + i0 + li) * ld_out + head * XA_HD + 32 * kh;
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
+        for (int g = 0; g < 4; ++g)
           *reinterpret_cast<uint4 *>(orow + 8 * g) = make_uint4(
               pack_bf16(__uint_as_float(o0[8 * g]) * inv, __uint_as_float(o0[8 * g + 1]) * inv),
               pack_bf16(__uint_as_float(o0[8 * g + 2]) * inv, __uint_as_float(o0[8 * g + 3]) * inv),
               pack_bf16(__uint_as_float(o0[8 * g + 4]) * inv, __uint_as_float(o0[8 * g + 5]) * inv),
               pack_bf16(__uint_as_float(o0[8 * g + 6]) * inv, __uint_as_float(o0[8 * g + 7]) * inv));
-          *reinterpret_cast<uint4 *>(orow + 32 + 8 * g) = make_uint4(
-              pack_bf16(__uint_as_float(o1[8 * g]) * inv, __uint_as_float(o1[8 * g + 1]) * inv),
-              pack_bf16(__uint_as_float(o1[8 * g + 2]) * inv, __uint_as_float(o1[8 * g + 3]) * inv),
-              pack_bf16(__uint_as_float(o1[8 * g + 4]) * inv, __uint_as_float(o1[8 * g + 5]) * inv),
-              pack_bf16(__uint_as_float(o1[8 * g + 6]) * inv, __uint_as_float(o1[8 * g + 7]) * inv));
-        }
       }
     }
     if (!ok && lane == 0) {
