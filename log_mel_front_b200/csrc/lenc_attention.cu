@@ -12,9 +12,11 @@
 // and half of the output dims; the two exchange their rows' block maxima and
 // final sums through shared memory (64-arrival mbarriers per quarter). Per
 // 128-key block:
-//   * TMA: the 128 key rows and value rows of the block, and the 256 position
-//     rows of the distances the block spans (r = i - j from i0 - j0 - 127 to
-//     i0 - j0 + 127; rows outside the table are zero-filled);
+//   * TMA: the 128 key rows and the 256 position rows of the distances the
+//     block spans (r = i - j from i0 - j0 - 127 to i0 - j0 + 127; rows outside
+//     the table are zero-filled) into one of two stages, loaded while the
+//     block before is processed, and the 128 value rows (one buffer, loaded
+//     once the previous block's P V has read it);
 //   * S = (q + u) K^T (M=128, N=128) and T = (q + v) Pband^T (M=128, N=256)
 //     into tensor memory; (q + u) and (q + v) are written once, as bf16, by
 //     the row threads;
@@ -27,11 +29,11 @@
 //     warp and block);
 //   * online softmax over the key blocks: the row thread keeps its row's
 //     running maximum and sum, writes the block's probabilities (relative to
-//     the new maximum) as bf16 (K-major, 128-byte swizzle), and, when the
-//     maximum grew, first rescales its own row of the P V accumulator in tensor
-//     memory (one tcgen05.ld and one tcgen05.st of 64 columns); tcgen05.mma
-//     then accumulates P V (M=128, N=64, V read MN-major) into it. The row
-//     thread reads the accumulator once at the end and divides by the sum.
+//     the new maximum) as bf16 into tensor memory, and, when the maximum grew,
+//     first rescales its part of the row's P V accumulator there (one
+//     tcgen05.ld and one tcgen05.st); tcgen05.mma then accumulates P V (A = P
+//     from tensor memory, M=128, N=64, K=128, V read MN-major) into it. The
+//     row thread reads the accumulator once at the end and divides by the sum.
 // Every wait is bounded and reports through the library's status word.
 #include "ae_internal.h"
 #include "common.cuh"
@@ -41,20 +43,33 @@ namespace ae {
 namespace {
 constexpr int XA_Q = 128, XA_K = 128, XA_HD = 64;
 constexpr uint32_t XA_TILE = 128 * 128;               // 128 rows x 64 bf16
-constexpr uint32_t OFF_QU = 0, OFF_QV = OFF_QU + XA_TILE, OFF_K = OFF_QV + XA_TILE, OFF_V = OFF_K + XA_TILE;
-constexpr uint32_t OFF_PB = OFF_V + XA_TILE;             // 256 position rows
-constexpr uint32_t OFF_S = OFF_PB + 2 * XA_TILE;         // probabilities: two 64-key regions
-constexpr uint32_t OFF_SCR = OFF_S + 2 * XA_TILE;        // skew scratch, 8 warps x 32 rows x 66 floats
+constexpr uint32_t OFF_QU = 0, OFF_QV = OFF_QU + XA_TILE, OFF_V = OFF_QV + XA_TILE;
+constexpr uint32_t OFF_K = OFF_V + XA_TILE;              // [2 stages] 128 key rows
+constexpr uint32_t OFF_PB = OFF_K + 2 * XA_TILE;         // [2 stages] 256 position rows
+constexpr uint32_t OFF_SCR = OFF_PB + 4 * XA_TILE;       // skew scratch, 8 warps x 32 rows x 66 floats
 constexpr int SCR_PITCH = 66;
 constexpr uint32_t OFF_X = OFF_SCR + 8 * 32 * SCR_PITCH * 4;  // [2 block parities][2 key halves][128] maxima, [2][128] sums
 constexpr uint32_t OFF_BAR = OFF_X + (2 * 2 * 128 + 2 * 128) * 4;
 constexpr size_t XA_SMEM = OFF_BAR + 256 + 1024;
 constexpr int XA_THREADS = 320;
 constexpr int XA_ROW_THREADS = 256;
-constexpr uint32_t XA_TMEM_COLS = 512, COL_S = 0, COL_T = 128, COL_O = 384;
-constexpr uint32_t XA_KV_BYTES = 4 * XA_TILE;            // K, V and two position boxes
+constexpr uint32_t XA_TMEM_COLS = 512, COL_S = 0, COL_T = 128, COL_O = 384, COL_P = 448;  // P: 128 bf16 keys
+constexpr uint32_t XA_KP_BYTES = 3 * XA_TILE;            // K and two position boxes
 static_assert(XA_SMEM <= 227 * 1024, "shared memory");
-static_assert(OFF_PB % 1024 == 0 && OFF_S % 1024 == 0 && OFF_SCR % 16 == 0, "swizzle atoms");
+static_assert(OFF_K % 1024 == 0 && OFF_PB % 1024 == 0 && OFF_SCR % 16 == 0, "swizzle atoms");
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, bf16, f32 accumulate: A's row m is lane m,
+// two bf16 per 32-bit column (the lower k in the low half), K = 16 per
+// instruction over 8 columns. One thread issues.
+__device__ __forceinline__ void xa_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 }  // namespace
 
 // 32 lanes x 32 consecutive 32-bit columns from registers into tensor memory
@@ -79,12 +94,12 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
                   int t_max, int p_col, bf16 *__restrict__ out, int ld_out, unsigned *status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sQu = smem + OFF_QU, *sQv = smem + OFF_QV, *sK = smem + OFF_K, *sV = smem + OFF_V, *sPb = smem + OFF_PB,
-          *sS = smem + OFF_S;
+  uint8_t *sQu = smem + OFF_QU, *sQv = smem + OFF_QV, *sV = smem + OFF_V;
   float *scr = reinterpret_cast<float *>(smem + OFF_SCR);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-  uint64_t *q_full = bars, *q_ready = bars + 1, *kv_full = bars + 2, *s_full = bars + 3, *s_free = bars + 4,
+  uint64_t *q_full = bars, *q_ready = bars + 1, *v_full = bars + 2, *s_full = bars + 3, *s_free = bars + 4,
            *p_full = bars + 5, *o_full = bars + 6;
+  uint64_t *kp_full = bars + 20, *kp_free = bars + 22;  // per stage: K and position rows landed / read
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 7);
   // per lane quarter: the two row warps' exchanges (q tiles read, block maxima, final sums)
   uint64_t *xq = bars + 8, *xm = bars + 12, *xs = bars + 16;
@@ -109,7 +124,11 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_ready, XA_ROW_THREADS);
-    mbar_init(kv_full, 1);
+    mbar_init(v_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kp_full[i], 1);
+      mbar_init(&kp_free[i], 1);
+    }
     mbar_init(s_full, 1);
     mbar_init(s_free, XA_ROW_THREADS);
     mbar_init(p_full, XA_ROW_THREADS);
@@ -134,41 +153,58 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0 && lane == 0) {
-    // ---------------- TMA producer
+    // ---------------- TMA producer: K and position rows of block kb into stage kb & 1
+    // (once the score MMAs of block kb - 2 have read it), V of block kb into its
+    // buffer (once the P V of block kb - 1 has read it)
     bool ok = true;
     mbar_arrive_expect_tx(q_full, XA_TILE);
     tma_load_2d(sQu, &tmQKV, head * XA_HD, tok0 + i0, q_full);
-    int issued = 0;
-    for (int kb = 0; kb < n_kb; ++kb) {
-      // K and the position rows are free once the previous block's score MMAs
-      // have completed; V once its P V has
-      if (kb > 0 && (!mbar_wait(s_full, (kb - 1) & 1) || !mbar_wait(o_full, (kb - 1) & 1))) { ok = false; break; }
-      if (*abort_flag) break;
+    int n_kp = 0, n_v = 0;
+    auto load_kp = [&](int kb) -> bool {
+      const int st = kb & 1;
+      if (kb >= 2 && !mbar_wait(&kp_free[st], ((kb >> 1) - 1) & 1)) return false;
+      if (*abort_flag) return false;
       const int j0 = kb * XA_K;
       const int prow = t_max - 128 - i0 + j0;  // table row of distance i0 - j0 + 127
-      mbar_arrive_expect_tx(kv_full, XA_KV_BYTES);
-      tma_load_2d(sK, &tmQKV, kLencEmbd + head * XA_HD, tok0 + j0, kv_full);
-      tma_load_2d(sPb, &tmP, p_col + head * XA_HD, prow, kv_full);
-      tma_load_2d(sPb + XA_TILE, &tmP, p_col + head * XA_HD, prow + 128, kv_full);
-      tma_load_2d(sV, &tmQKV, 2 * kLencEmbd + head * XA_HD, tok0 + j0, kv_full);
-      ++issued;
-    }
+      mbar_arrive_expect_tx(&kp_full[st], XA_KP_BYTES);
+      tma_load_2d(smem + OFF_K + st * XA_TILE, &tmQKV, kLencEmbd + head * XA_HD, tok0 + j0, &kp_full[st]);
+      tma_load_2d(smem + OFF_PB + st * 2 * XA_TILE, &tmP, p_col + head * XA_HD, prow, &kp_full[st]);
+      tma_load_2d(smem + OFF_PB + st * 2 * XA_TILE + XA_TILE, &tmP, p_col + head * XA_HD, prow + 128, &kp_full[st]);
+      ++n_kp;
+      return true;
+    };
+    auto load_v = [&](int kb) -> bool {
+      if (kb >= 1 && !mbar_wait(o_full, (kb - 1) & 1)) return false;
+      if (*abort_flag) return false;
+      mbar_arrive_expect_tx(v_full, XA_TILE);
+      tma_load_2d(sV, &tmQKV, 2 * kLencEmbd + head * XA_HD, tok0 + kb * XA_K, v_full);
+      ++n_v;
+      return true;
+    };
+    if (n_kb > 0) ok = load_kp(0) && load_v(0);
+    for (int kb = 1; kb < n_kb && ok; ++kb) ok = load_kp(kb) && load_v(kb);
     if (!ok) {
       atomicOr(status, kStatusWaitTimeout);
       *abort_flag = 1;
     }
-    mbar_wait(q_full, 0);
-    if (issued > 0) mbar_wait(kv_full, (issued - 1) & 1);  // every load lands before the CTA ends
+    mbar_wait(q_full, 0);  // every load lands before the CTA ends
+#pragma unroll
+    for (int st = 0; st < 2; ++st) {
+      const int u = (n_kp + 1 - st) / 2;  // uses of stage st
+      if (u > 0) mbar_wait(&kp_full[st], (u - 1) & 1);
+    }
+    if (n_v > 0) mbar_wait(v_full, (n_v - 1) & 1);
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
     constexpr uint32_t idesc_s = idesc_bf16_f32(XA_Q, XA_K);
     constexpr uint32_t idesc_t = idesc_bf16_f32(XA_Q, 2 * XA_K);
     constexpr uint32_t idesc_o = idesc_bf16_f32_bmn(XA_Q, XA_HD);
-    const uint32_t aqu = smem_u32(sQu), aqv = smem_u32(sQv), ak = smem_u32(sK), av = smem_u32(sV),
-                   apb = smem_u32(sPb), as = smem_u32(sS);
+    const uint32_t aqu = smem_u32(sQu), aqv = smem_u32(sQv), av = smem_u32(sV);
     bool ok = mbar_wait(q_ready, 0);
     for (int kb = 0; kb < n_kb && ok; ++kb) {
-      if (!mbar_wait(kv_full, kb & 1) || (kb > 0 && !mbar_wait(s_free, (kb - 1) & 1)) || *abort_flag) {
+      const int st = kb & 1;
+      const uint32_t ak = smem_u32(smem + OFF_K + st * XA_TILE), apb = smem_u32(smem + OFF_PB + st * 2 * XA_TILE);
+      if (!mbar_wait(&kp_full[st], (kb >> 1) & 1) || (kb > 0 && !mbar_wait(s_free, (kb - 1) & 1)) || *abort_flag) {
         ok = false;
         break;
       }
@@ -179,16 +215,17 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
 #pragma unroll
       for (int k = 0; k < XA_HD / 16; ++k)
         tc_mma_bf16(tmem + COL_T, sw128_desc(aqv + k * 32), sw128_desc(apb + k * 32), idesc_t, k > 0 ? 1u : 0u);
+      tc_commit(&kp_free[st]);
       tc_commit(s_full);
-      if (!mbar_wait(p_full, kb & 1) || *abort_flag) {
+      if (!mbar_wait(p_full, kb & 1) || !mbar_wait(v_full, kb & 1) || *abort_flag) {
         ok = false;
         break;
       }
       tc_fence_after();
 #pragma unroll
       for (int ks = 0; ks < XA_K / 16; ++ks)
-        tc_mma_bf16(tmem + COL_O, sw128_desc(as + (ks >> 2) * XA_TILE + (ks & 3) * 32),
-                    sw128_desc_mn(av + ks * 2048, XA_TILE), idesc_o, (kb | ks) != 0 ? 1u : 0u);
+        xa_mma_ts(tmem + COL_O, tmem + COL_P + 8 * ks, sw128_desc_mn(av + ks * 2048, XA_TILE), idesc_o,
+                  (kb | ks) != 0 ? 1u : 0u);
       tc_commit(o_full);
     }
     if (!ok) {
@@ -280,17 +317,14 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
       if (kb > 0 && !__all_sync(0xffffffffu, mbar_wait(o_full, (kb - 1) & 1))) { ok = false; break; }
       tc_fence_after();
       float ls = 0.f;
+      uint32_t pw[32];  // keys 64 kh .. 64 kh + 63 as bf16 pairs: tensor-memory columns COL_P + 32 kh ..
 #pragma unroll
-      for (int g = 0; g < 8; ++g) {  // granules 0..7 of region kh: keys 64 kh + 8 g ..
-        float p[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          p[e] = exp2f(z[8 * g + e] - m_new);
-          ls += p[e];
-        }
-        *reinterpret_cast<uint4 *>(sS + kh * XA_TILE + li * 128 + ((g ^ r7) << 4)) =
-            make_uint4(pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]), pack_bf16(p[4], p[5]), pack_bf16(p[6], p[7]));
+      for (int x = 0; x < 32; ++x) {
+        const float p0 = exp2f(z[2 * x] - m_new), p1 = exp2f(z[2 * x + 1] - m_new);
+        ls += p0 + p1;
+        pw[x] = pack_bf16(p0, p1);
       }
+      xa_tmem_st32(trow + COL_P + 32 * kh, pw);
       l_run = l_run * alpha + ls;
       m_run = m_new;
       if (kb > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
@@ -301,10 +335,9 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
 #pragma unroll
         for (int d = 0; d < 32; ++d) o[d] = __float_as_uint(__uint_as_float(o[d]) * alpha);
         xa_tmem_st32(trow + COL_O + 32 * kh, o);
-        xa_tmem_st_wait();
       }
+      xa_tmem_st_wait();  // P (and the rescaled accumulator) are in tensor memory
       tc_fence_before();
-      fence_async_smem();
       mbar_arrive(p_full);
     }
     if (ok && !__all_sync(0xffffffffu, mbar_wait(o_full, (n_kb - 1) & 1))) ok = false;
