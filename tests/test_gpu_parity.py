@@ -159,6 +159,32 @@ def test_subsample_bf16_ragged(m_tower, w_tower):
     assert_bf16(g, o, "subsample bf16")
 
 
+def test_subsample_bf16_mel_not_16_byte_aligned(m_tower, w_tower):
+    """d_mel 4 bytes past a 16-byte boundary (allowed by ae_subsample): the
+    tensor-core conv0 stages its mel rows with 4-byte copies instead of
+    16-byte ones; same rows as the aligned call, bit for bit, and the oracle's."""
+    rng = np.random.default_rng(5)
+    clips = [(0.3 * rng.standard_normal(n)).astype(np.float32) for n in (16000, 7000, 48000)]
+    mels = [O.log_mel(c) for c in clips]
+    frames = [m.shape[0] for m in mels]
+    T = sum(O.num_tokens(len(c)) for c in clips)
+    flat = np.concatenate(mels).astype(np.float32)
+    base = torch.zeros(flat.size + 4, device="cuda")
+    base[1:1 + flat.size] = torch.from_numpy(flat.ravel()).cuda()
+    d_mis = base[1:1 + flat.size]
+    assert d_mis.data_ptr() % 16 == 4
+    ws = workspace(m_tower.workspace_size(len(clips), sum(frames), T))
+    outs = []
+    for d_mel in (dev(flat), d_mis):
+        d_h = torch.full((T, 1024), float("nan"), device="cuda")
+        ae.ae_subsample(m_tower, d_mel, offsets(frames), d_h, ws, ws.numel())
+        _sync()
+        outs.append(d_h.cpu().numpy())
+    assert np.array_equal(outs[0], outs[1])
+    o = np.concatenate([O.subsample(m.astype(np.float32).astype(np.float64), w_tower["stem"]) for m in mels])
+    assert_bf16(outs[1], o, "subsample bf16, unaligned mel")
+
+
 # ------------------------------------------------------------------ one layer
 
 def _layer_case(model, W, layer, h, toks):
@@ -408,6 +434,34 @@ def test_attention_bf16_edges_all_tokens(toks):
     Ro = O.relative_keys(p["relk"], 12, 1024)
     o = _attn_oracle(qkv[:, :1024], qkv[:, 1024:2048], qkv[:, 2048:], O.positions(toks), Ro, O.softplus(p["pds"]))
     assert_bf16(out.float().cpu().numpy(), o, f"attention bf16, {T} tokens in {len(toks)} clips")
+
+
+def test_attention_bf16_output_stride_not_32_byte_aligned():
+    """An output row stride of 1032 elements (16-byte but not 32-byte multiples):
+    rows leave as 16-byte pieces instead of 32-byte sectors; the same values as
+    the dense output, bit for bit, and the oracle's."""
+    p = synth.attention_params()
+    rng = np.random.default_rng(77)
+    toks = [300, 5, 200]
+    T = sum(toks)
+    qkv = synth.round_to_bf16((2.0 * rng.standard_normal((T, 3072))).astype(np.float32))
+    d = dev(qkv).to(torch.bfloat16)
+    R, qs, ks = ae.ae_attention_tables(p["relk"], p["pds"])
+    ws = workspace(ae.ae_workspace_size(None, len(toks), 0, T))
+    outs = []
+    for ld in (1024, 1032):
+        buf = torch.full((T, ld), float("nan"), dtype=torch.bfloat16, device="cuda")
+        ae.ae_local_attention(d[:, :1024], d[:, 1024:2048], d[:, 2048:], 3072, ae.AE_BF16, dev(R), dev(qs), ks, 50.0,
+                              offsets(toks), buf, ld, ws, ws.numel())
+        _sync()
+        g = buf.float().cpu().numpy()
+        if ld > 1024:
+            assert np.all(np.isnan(g[:, 1024:])), "columns past the row written"
+        outs.append(g[:, :1024])
+    assert np.array_equal(outs[0], outs[1])
+    Ro = O.relative_keys(p["relk"], 12, 1024)
+    o = _attn_oracle(qkv[:, :1024], qkv[:, 1024:2048], qkv[:, 2048:], O.positions(toks), Ro, O.softplus(p["pds"]))
+    assert_bf16(outs[1], o, "attention bf16, output stride 1032")
 
 
 # ------------------------------------------------------------------ refusals (host checks, nothing enqueued)
