@@ -23,19 +23,19 @@ namespace ae {
 //
 // Work item = one head x 128 consecutive tokens t0 .. t0+127 (the packed rows
 // of any clips); a persistent CTA (one per SM) walks the items. Per item:
-//   * TMA loads the q tile [128 x 128], the 144 k rows t0-11 .. t0+132 and the
-//     144 v rows (the tensor maps zero-fill rows before 0 and past T) into one
-//     of two shared-memory stages;
+//   * TMA loads the q tile [128 x 128] and the 144 k rows t0-11 .. t0+132 into
+//     one of two shared-memory stages, and the 144 v rows into one buffer (the
+//     tensor maps zero-fill rows before 0 and past T);
 //   * four q warps (one per 32-row quarter) scale q by s and split the product
-//     into two bf16 parts, hi = bf16(q s) and lo = bf16(q s - hi), which they
-//     store into tensor memory as the A operand of the score MMA, so that it
-//     sees q s to about 16 bits (a single bf16 rounding of q s costs more
-//     accuracy than everything else in the kernel together); they also write
-//     the head's R[d] / k_scale as rows 144..155 under the k rows;
-//   * tcgen05.mma (A from tensor memory, M=128, N=160, K=128 for hi and again
-//     for lo into the same accumulator) gives S = (q s) [k ; R/k_scale]^T in
-//     tensor memory: row r holds q_t.k_{t0-11+c} at column c and the position
-//     term q_t.R[d]/k_scale at column 144+d;
+//     into two bf16 parts, hi = bf16(q s), written over the q tile, and lo =
+//     bf16(q s - hi), written to a tile of its own, so the score MMA sees q s
+//     to about 16 bits (a single bf16 rounding of q s costs more accuracy than
+//     everything else in the kernel together); they also write the head's
+//     R[d] / k_scale as rows 144..155 under the k rows;
+//   * tcgen05.mma (M=128, N=160, K=128 for hi and again for lo into the same
+//     accumulator, both operands in shared memory) gives S = (q s)
+//     [k ; R/k_scale]^T in tensor memory: row r holds q_t.k_{t0-11+c} at
+//     column c and the position term q_t.R[d]/k_scale at column 144+d;
 //   * four softmax warps: the thread of row r (t = t0 + r) reads columns
 //     32w .. 32w+47 of its warp's 32 rows and shifts them left by its lane
 //     (five select stages), so that column r + 11 - d, the key t - d, lands at
@@ -46,16 +46,16 @@ namespace ae {
 //     around it (the columns outside every warp's window stay zero from the
 //     start);
 //   * tcgen05.mma (A = P from tensor memory, M=128, N=128, K=144, v read
-//     MN-major) gives O = P V;
+//     MN-major) gives O = P V in one of two tensor-memory accumulators;
 //   * the softmax warps (head dims 64..127) and the q warps (0..63) drain O,
 //     clamp it and store it from registers, whole 32-byte sectors per row
 //     where the output's alignment allows.
 // The stages overlap across items: the q warps split item i+1 as soon as the
 // score MMA of item i has read the previous split, while the softmax warps
 // work on item i; the MMA warp issues item i's P V as soon as its P is
-// written, then item i+1's score MMA; both warp groups drain item i while the
-// score MMA of item i+1 runs. A stage's q/k are reloaded once the score MMA
-// that read them completes, its v once the P V MMA has.
+// written, then item i+1's score MMA; item i's O is drained while item i+1
+// runs. A stage's q/k are reloaded once the score MMA that read them
+// completes, v once the P V MMA has.
 namespace {
 constexpr int AT_Q = 128;                                  // queries per item
 constexpr int AT_KEYS = 144;                               // key rows per item (139 used)
@@ -63,26 +63,25 @@ constexpr int AT_BROWS = AT_KEYS + 16;                     // score MMA B rows: 
 constexpr uint32_t AT_Q_REGION = AT_Q * 128;               // 64 head dims of q: 16 KB
 constexpr uint32_t AT_KR_REGION = AT_BROWS * 128;          // 20 KB
 constexpr uint32_t AT_V_REGION = AT_KEYS * 128;            // 18 KB
-constexpr uint32_t OFF_Q = 0;                              // offsets within a stage
+constexpr uint32_t OFF_Q = 0;                              // offsets within a stage: q (then hi), k rows
 constexpr uint32_t OFF_KR = OFF_Q + 2 * AT_Q_REGION;
-constexpr uint32_t OFF_V = OFF_KR + 2 * AT_KR_REGION;
-constexpr uint32_t AT_STAGE = OFF_V + 2 * AT_V_REGION;     // 108 KB
-constexpr uint32_t OFF_BAR = 2 * AT_STAGE;
+constexpr uint32_t AT_STAGE = OFF_KR + 2 * AT_KR_REGION;   // 72 KB
+constexpr uint32_t OFF_QL = 2 * AT_STAGE;                  // lo part of q s
+constexpr uint32_t OFF_V = OFF_QL + 2 * AT_Q_REGION;
+constexpr uint32_t OFF_BAR = OFF_V + 2 * AT_V_REGION;
 constexpr size_t AT_SMEM = OFF_BAR + 1024 + 1024;          // barriers + q scales, alignment slack
 constexpr int AT_THREADS = 320;                            // producer, MMA, 4 softmax warps, 4 q warps
 constexpr int AT_DRAIN_THREADS = 256;                      // both warp groups drain half of O
 constexpr uint32_t AT_TMEM_COLS = 512;
 constexpr uint32_t COL_S = 0;                              // scores, 160 f32 columns
 constexpr uint32_t COL_P = 160;                            // banded P, 160 bf16 = 80 columns
-constexpr uint32_t COL_QH = 256;                           // q s hi part, 128 bf16 = 64 columns
-constexpr uint32_t COL_QL = 320;                           // q s lo part (directly after hi: one K = 256 operand)
-constexpr uint32_t COL_O = 384;                            // P V, 128 f32 columns
+constexpr uint32_t COL_O = 256;                            // two P V accumulators, 128 f32 columns each
 constexpr uint32_t AT_QK_BYTES = 2 * AT_Q_REGION + 2 * AT_KEYS * 128;
 constexpr uint32_t AT_V_BYTES = 2 * AT_V_REGION;
 static_assert(AT_SMEM <= 227 * 1024, "shared memory");
-static_assert(AT_STAGE % 1024 == 0 && OFF_KR % 1024 == 0 && OFF_V % 1024 == 0, "swizzle atoms");
+static_assert(AT_STAGE % 1024 == 0 && OFF_KR % 1024 == 0 && OFF_QL % 1024 == 0 && OFF_V % 1024 == 0, "swizzle atoms");
 static_assert(AT_KR_REGION % 1024 == 0 && AT_V_REGION % 1024 == 0, "swizzle atoms");
-static_assert(COL_QL == COL_QH + 64 && COL_O + 128 <= AT_TMEM_COLS && COL_P + 80 <= COL_QH, "tensor-memory map");
+static_assert(COL_P + 80 <= COL_O && COL_O + 256 <= AT_TMEM_COLS, "tensor-memory map");
 
 // D[tmem] (+)= A[tmem] * B[smem]^T, bf16 inputs, f32 accumulate: A's row m is
 // tensor-memory lane m, two bf16 per 32-bit column (the lower k in the low
@@ -146,9 +145,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-  uint64_t *qk_full = bars, *v_full = bars + 2, *qk_free = bars + 4, *v_free = bars + 6;  // per stage
-  uint64_t *q_ready = bars + 8, *s_full = bars + 9, *s_free = bars + 10, *p_full = bars + 11, *o_full = bars + 12,
-           *o_empty = bars + 13;
+  uint64_t *qk_full = bars, *qk_free = bars + 2;                      // per stage
+  uint64_t *o_full = bars + 4, *o_empty = bars + 6;                   // per accumulator
+  uint64_t *v_full = bars + 8, *v_free = bars + 9, *q_ready = bars + 10, *s_full = bars + 11, *s_free = bars + 12,
+           *p_full = bars + 13;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 14);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   float *s_qs = reinterpret_cast<float *>(smem + OFF_BAR + 128);
@@ -156,13 +156,17 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = ((T + AT_Q - 1) / AT_Q) * kHeads;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 8; ++i) mbar_init(bars + i, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);   // qk_full, qk_free
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&o_full[i], 1);
+      mbar_init(&o_empty[i], AT_DRAIN_THREADS);
+    }
+    mbar_init(v_full, 1);
+    mbar_init(v_free, 1);
     mbar_init(q_ready, 128);
     mbar_init(s_full, 1);
     mbar_init(s_free, 128);
     mbar_init(p_full, 128);
-    mbar_init(o_full, 1);
-    mbar_init(o_empty, AT_DRAIN_THREADS);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
@@ -178,9 +182,11 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // O rows of item j, head dims 64 hw .. 64 hw + 63, out by the warp of lane quarter warp & 3
+  // O rows of item j (the j-th of this CTA), head dims 64 hw .. 64 hw + 63, out by
+  // the warp of lane quarter warp & 3
   auto drain_half = [&](int j, int jitem, int hw) -> bool {
-    if (!__all_sync(0xffffffffu, mbar_wait(o_full, j & 1))) return false;
+    const int b = j & 1;
+    if (!__all_sync(0xffffffffu, mbar_wait(&o_full[b], (j >> 1) & 1))) return false;
     tc_fence_after();
     const int qw = warp & 3, r = 32 * qw + lane;
     const uint32_t trow = tmem + ((uint32_t)(32 * qw) << 16);
@@ -189,7 +195,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
 #pragma unroll 1
     for (int c = 0; c < 2; ++c) {
       uint32_t o[32];
-      tmem_ld32(trow + COL_O + 64 * hw + 32 * c, o);
+      tmem_ld32(trow + COL_O + 128 * b + 64 * hw + 32 * c, o);
       tmem_ld_wait();
       uint32_t w[16];
 #pragma unroll
@@ -207,19 +213,20 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       }
     }
     tc_fence_before();
-    mbar_arrive(o_empty);
+    mbar_arrive(&o_empty[b]);
     return true;
   };
 
   if (warp == 0 && lane == 0) {
-    // ---------------- TMA producer
-    int n_qk = 0, n_v = 0;  // items whose q/k (v) loads were issued; item i uses stage i & 1
+    // ---------------- TMA producer: q, k of item i into stage i & 1 once the
+    // score MMA of item i - 2 has read it; v of item i once the P V of item i - 1 has
+    int n_qk = 0, n_v = 0;
     bool ok = true;
     for (int item = blockIdx.x, it = 0; item < n_items; item += gridDim.x, ++it) {
       const int st = it & 1, u = it >> 1;
       uint8_t *stage = smem + st * AT_STAGE;
       const int t0 = (item >> 3) * AT_Q, x = (item & 7) * kHeadDim;
-      if (u > 0 && !mbar_wait(&qk_free[st], (u - 1) & 1)) { ok = false; break; }  // score MMA read q, k
+      if (u > 0 && !mbar_wait(&qk_free[st], (u - 1) & 1)) { ok = false; break; }
       if (*abort_flag) break;
       mbar_arrive_expect_tx(&qk_full[st], AT_QK_BYTES);
       tma_load_2d(stage + OFF_Q, &tmQ, x, t0, &qk_full[st]);
@@ -227,11 +234,11 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       tma_load_2d(stage + OFF_KR, &tmK, x, t0 - (kLeft - 1), &qk_full[st]);
       tma_load_2d(stage + OFF_KR + AT_KR_REGION, &tmK, x + 64, t0 - (kLeft - 1), &qk_full[st]);
       ++n_qk;
-      if (u > 0 && !mbar_wait(&v_free[st], (u - 1) & 1)) { ok = false; break; }  // P V MMA read v
+      if (it > 0 && !mbar_wait(v_free, (it - 1) & 1)) { ok = false; break; }
       if (*abort_flag) break;
-      mbar_arrive_expect_tx(&v_full[st], AT_V_BYTES);
-      tma_load_2d(stage + OFF_V, &tmV, x, t0 - (kLeft - 1), &v_full[st]);
-      tma_load_2d(stage + OFF_V + AT_V_REGION, &tmV, x + 64, t0 - (kLeft - 1), &v_full[st]);
+      mbar_arrive_expect_tx(v_full, AT_V_BYTES);
+      tma_load_2d(smem + OFF_V, &tmV, x, t0 - (kLeft - 1), v_full);
+      tma_load_2d(smem + OFF_V + AT_V_REGION, &tmV, x + 64, t0 - (kLeft - 1), v_full);
       ++n_v;
     }
     if (!ok) {
@@ -241,35 +248,20 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     // every load issued must land before the CTA may end
 #pragma unroll
     for (int st = 0; st < 2; ++st) {
-      const int uq = (n_qk + 1 - st) / 2, uv = (n_v + 1 - st) / 2;  // uses of stage st
+      const int uq = (n_qk + 1 - st) / 2;  // uses of stage st
       if (uq > 0) mbar_wait(&qk_full[st], (uq - 1) & 1);
-      if (uv > 0) mbar_wait(&v_full[st], (uv - 1) & 1);
     }
+    if (n_v > 0) mbar_wait(v_full, (n_v - 1) & 1);
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer: the score MMA of item i, then (once P is written) its P V MMA
     constexpr uint32_t idesc_s = idesc_bf16_f32(AT_Q, AT_BROWS);
     constexpr uint32_t idesc_o = idesc_bf16_f32_bmn(AT_Q, kHeadDim);
+    const uint32_t aql = smem_u32(smem + OFF_QL), av = smem_u32(smem + OFF_V);
     bool ok = true;
-    auto pv = [&](int j) -> bool {  // O = P V of item j
-      const int st = j & 1;
-      if (!mbar_wait(p_full, j & 1) || !mbar_wait(&v_full[st], (j >> 1) & 1) ||
-          (j > 0 && !mbar_wait(o_empty, (j - 1) & 1)) || *abort_flag)
-        return false;
-      tc_fence_after();
-      const uint32_t av = smem_u32(smem + st * AT_STAGE + OFF_V);
-#pragma unroll
-      for (int ks = 0; ks < AT_KEYS / 16; ++ks)
-        at_mma_ts(tmem + COL_O, tmem + COL_P + 8 * ks, sw128_desc_mn(av + ks * 2048, AT_V_REGION), idesc_o,
-                  ks > 0 ? 1u : 0u);
-      tc_commit(&v_free[st]);
-      tc_commit(o_full);
-      return true;
-    };
-    int it = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it) {
-      const int st = it & 1;
-      const uint32_t akr = smem_u32(smem + st * AT_STAGE + OFF_KR);
-      // q s of this item is in tensor memory, and the softmax has read the previous scores
+    for (int item = blockIdx.x, it = 0; item < n_items; item += gridDim.x, ++it) {
+      const int st = it & 1, b = it & 1;
+      const uint32_t aq = smem_u32(smem + st * AT_STAGE + OFF_Q), akr = smem_u32(smem + st * AT_STAGE + OFF_KR);
+      // q s of this item is split, and the softmax has read the previous scores
       if (!mbar_wait(q_ready, it & 1) || (it > 0 && !mbar_wait(s_free, (it - 1) & 1)) || *abort_flag) {
         ok = false;
         break;
@@ -278,12 +270,24 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
 #pragma unroll
       for (int ks = 0; ks < 2 * kHeadDim / 16; ++ks) {
         const int kk = ks & 7;  // hi part for ks < 8, lo part after: the same k rows
-        at_mma_ts(tmem + COL_S, tmem + COL_QH + 8 * ks,
-                  sw128_desc(akr + (kk >> 2) * AT_KR_REGION + (kk & 3) * 32), idesc_s, ks > 0 ? 1u : 0u);
+        tc_mma_bf16(tmem + COL_S, sw128_desc((ks < 8 ? aq : aql) + (kk >> 2) * AT_Q_REGION + (kk & 3) * 32),
+                    sw128_desc(akr + (kk >> 2) * AT_KR_REGION + (kk & 3) * 32), idesc_s, ks > 0 ? 1u : 0u);
       }
       tc_commit(&qk_free[st]);
       tc_commit(s_full);
-      if (!pv(it)) { ok = false; break; }
+      // P is written, v has landed, and this accumulator's previous item is drained
+      if (!mbar_wait(p_full, it & 1) || !mbar_wait(v_full, it & 1) ||
+          (it >= 2 && !mbar_wait(&o_empty[b], ((it >> 1) - 1) & 1)) || *abort_flag) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int ks = 0; ks < AT_KEYS / 16; ++ks)
+        at_mma_ts(tmem + COL_O + 128 * b, tmem + COL_P + 8 * ks, sw128_desc_mn(av + ks * 2048, AT_V_REGION),
+                  idesc_o, ks > 0 ? 1u : 0u);
+      tc_commit(v_free);
+      tc_commit(&o_full[b]);
     }
     if (!ok) {
       atomicOr(status, kStatusWaitTimeout);
@@ -391,15 +395,15 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       *abort_flag = 1;
     }
   } else if (warp >= 6) {
-    // ---------------- q warps: split item i's q s into tensor memory, then drain item i - 1
+    // ---------------- q warps: split item i's q s (hi over q, lo into its tile), then drain item i - 1
     const int qw = warp & 3, r = 32 * qw + lane, r7 = r & 7, tid = threadIdx.x - 192;
-    const uint32_t trow = tmem + ((uint32_t)(32 * qw) << 16);
     // rows 156..159 of both stages' B operand stay zero
     {
       const int s = tid >> 6, rr = AT_KEYS + 12 + ((tid >> 4) & 3), g = tid & 15;
       *reinterpret_cast<uint4 *>(smem + s * AT_STAGE + OFF_KR + (g >> 3) * AT_KR_REGION + rr * 128 +
                                  (((g & 7) ^ (rr & 7)) << 4)) = make_uint4(0, 0, 0, 0);
     }
+    uint8_t *sQL = smem + OFF_QL;
     const float inv_ks = 1.0f / k_scale;
     bool ok = true;
     int it = 0, prev_item = -1;
@@ -409,32 +413,27 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       const int st = it & 1, u = it >> 1;
       uint8_t *sQ = smem + st * AT_STAGE + OFF_Q, *sKR = smem + st * AT_STAGE + OFF_KR;
       const int h = item & 7;
-      // this item's q and k have landed, and the previous score MMA has read the previous split
+      // this item's q and k have landed, and the previous score MMA has read the lo tile
       if (!__all_sync(0xffffffffu, mbar_wait(&qk_full[st], u & 1)) ||
           (it > 0 && !__all_sync(0xffffffffu, mbar_wait(s_full, (it - 1) & 1)))) {
         ok = false;
         break;
       }
-      tc_fence_after();
-#pragma unroll 1
-      for (int hw = 0; hw < 2; ++hw) {  // head dims 64 hw .. 64 hw + 63
-        uint32_t qh[32], ql[32];
+#pragma unroll 4
+      for (int j = 0; j < 16; ++j) {  // head dims 8 j .. 8 j + 7 of row r
+        const uint32_t off = (j >> 3) * AT_Q_REGION + r * 128 + (((j & 7) ^ r7) << 4);
+        const uint4 wv = *reinterpret_cast<const uint4 *>(sQ + off);
+        const float4 s0 = reinterpret_cast<const float4 *>(s_qs)[2 * j], s1 = reinterpret_cast<const float4 *>(s_qs)[2 * j + 1];
+        const float f[8] = {bf16lo(wv.x) * s0.x, bf16hi(wv.x) * s0.y, bf16lo(wv.y) * s0.z, bf16hi(wv.y) * s0.w,
+                            bf16lo(wv.z) * s1.x, bf16hi(wv.z) * s1.y, bf16lo(wv.w) * s1.z, bf16hi(wv.w) * s1.w};
+        uint32_t hv[4], lv[4];
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          const uint4 wv = *reinterpret_cast<const uint4 *>(sQ + hw * AT_Q_REGION + r * 128 + ((jj ^ r7) << 4));
-          const int j = 8 * hw + jj;
-          const float4 s0 = reinterpret_cast<const float4 *>(s_qs)[2 * j], s1 = reinterpret_cast<const float4 *>(s_qs)[2 * j + 1];
-          const float f[8] = {bf16lo(wv.x) * s0.x, bf16hi(wv.x) * s0.y, bf16lo(wv.y) * s0.z, bf16hi(wv.y) * s0.w,
-                              bf16lo(wv.z) * s1.x, bf16hi(wv.z) * s1.y, bf16lo(wv.w) * s1.z, bf16hi(wv.w) * s1.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint32_t hv = pack_bf16(f[2 * e], f[2 * e + 1]);
-            qh[4 * jj + e] = hv;
-            ql[4 * jj + e] = pack_bf16(f[2 * e] - bf16lo(hv), f[2 * e + 1] - bf16hi(hv));
-          }
+        for (int e = 0; e < 4; ++e) {
+          hv[e] = pack_bf16(f[2 * e], f[2 * e + 1]);
+          lv[e] = pack_bf16(f[2 * e] - bf16lo(hv[e]), f[2 * e + 1] - bf16hi(hv[e]));
         }
-        at_tmem_st32(trow + COL_QH + 32 * hw, qh);
-        at_tmem_st32(trow + COL_QL + 32 * hw, ql);
+        *reinterpret_cast<uint4 *>(sQ + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+        *reinterpret_cast<uint4 *>(sQL + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
       }
       if ((st ? r_head1 : r_head0) != h) {  // the TMA never writes rows 144.., so they keep the stage's last head
         if (st) r_head1 = h; else r_head0 = h;
@@ -447,8 +446,6 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                          pack_bf16(b.x * inv_ks, b.y * inv_ks), pack_bf16(b.z * inv_ks, b.w * inv_ks));
         }
       }
-      at_tmem_st_wait();
-      tc_fence_before();
       fence_async_smem();
       mbar_arrive(q_ready);
       if (it > 0 && !drain_half(it - 1, prev_item, 0)) { ok = false; break; }
