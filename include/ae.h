@@ -228,7 +228,10 @@ ae_status ae_conformer_layer(const ae_model *m, int layer, float *d_h, const int
  * log-mel, stem, in_proj, every layer, then out_proj + bias, a weightless
  * RMS norm and embed. d_wave: float32 [h_sample_off[n_clips]]. d_out:
  * float32 [sum tokens][embed_dim], clip after clip, 16-byte aligned (the
- * projection writes it with TMA stores; AE_EINVAL otherwise). */
+ * projection writes it with TMA stores; AE_EINVAL otherwise). A batch of 4096
+ * to 32768 tokens in two or more clips runs as two half-batches, the second on
+ * a stream the model owns, forked from and joined back into `stream` (the
+ * rows are those of one pass; larger batches fill the GPU in one pass). */
 ae_status ae_encode(const ae_model *m, const float *d_wave, const int64_t *h_sample_off,
                     int n_clips, float *d_out, void *d_ws, size_t ws_bytes, ae_stream stream);
 
@@ -259,7 +262,7 @@ ae_status ae_encode_host(const ae_model *m, const float *h_wave, const int64_t *
  * after the call). Calls on different streams with their own workspaces and
  * output buffers overlap one batch's copies with another's kernels; each call
  * runs its batch as one pass on its stream (ae_encode and ae_encode_host split
- * a large batch in two halves on two streams instead). */
+ * a batch of 4096 to 32768 tokens in two halves on two streams instead). */
 ae_status ae_encode_host_async(const ae_model *m, const float *h_wave, const int64_t *h_sample_off,
                                int n_clips, float *h_out, void *d_ws, size_t ws_bytes, ae_stream stream);
 

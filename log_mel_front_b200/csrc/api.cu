@@ -599,6 +599,10 @@ static ae_status encode_one(const ae_model *m, const float *d_wave, const ClipTa
 // region rounds up to 256 bytes at most once more per half).
 constexpr size_t kSplitSlack = 64 * 1024;
 constexpr int64_t kSplitMinTokens = 4096;
+// Above this the halves' kernels fill the GPU on their own and the second
+// stream only adds contention (measured on the 96k-token ragged batch: one
+// pass 62.5-62.8 ms per step, two halves 63.5-63.9 ms, same box, interleaved).
+constexpr int64_t kSplitMaxTokens = 32768;
 
 static size_t encode_ws_bytes(const ae_model *m, int64_t n_clips, int64_t frames, int64_t tokens) {
   return ws_layout(m, n_clips, frames, tokens, true).total + kSplitSlack;
@@ -613,7 +617,7 @@ static ClipTables sub_tables(const ClipTables &T, int a, int b) {
   return S;
 }
 
-// The whole forward. A batch of at least kSplitMinTokens tokens in two or
+// The whole forward. A batch of kSplitMinTokens to kSplitMaxTokens tokens in two or
 // more clips runs as two halves of about equal token count, the first on s and
 // the second on the model's side stream, each with its own workspace layout;
 // the clips are independent, so the halves only share the weights. Outputs
@@ -624,7 +628,8 @@ static ClipTables sub_tables(const ClipTables &T, int a, int b) {
 static ae_status encode_dev(const ae_model *m, const float *d_wave, const ClipTables &T, float *d_out, void *d_ws,
                             size_t ws_bytes, cudaStream_t s, bool may_split) {
   const WsLayout L = ws_layout(m, T.n_clips, T.total_frames, T.total_tokens, true);
-  if (!may_split || g_prof.on || T.n_clips < 2 || T.total_tokens < kSplitMinTokens || !m->side[0])
+  if (!may_split || g_prof.on || T.n_clips < 2 || T.total_tokens < kSplitMinTokens ||
+      T.total_tokens > kSplitMaxTokens || !m->side[0])
     return encode_one(m, d_wave, T, d_out, d_ws, L, s);
   int k = 1;  // first clip of the second half
   while (k < T.n_clips - 1 && 2 * (int64_t)T.tok_off[k] < T.total_tokens) ++k;
