@@ -2,7 +2,7 @@
 """Throughput of the B200 audio-encoder forward.
 
     python bench.py [--gpus N] [--steps K] [--warmup W]
-                    [--workload ragged|tower|tower_fp8|frontend|lfm_frontend|lfm_encoder|attention|resample]
+                    [--workload ragged|tower|tower_fp8|frontend|lfm_frontend|lfm_encoder|lfm_ragged|attention|resample]
     python bench.py --impl reference ...      # the CPU oracle on the same workload (bounded sample)
 
 A step is one ae_encode over one batch (default: the ragged batch, 256 clips
@@ -176,6 +176,8 @@ def workload_desc(name: str, info: dict) -> dict:
             "lfm_encoder": "LFM2A encoder from PCM: the second log-mel front-end, the 5-layer conv stem, 17 "
                            "Conformer blocks with Transformer-XL attention and the erf-GELU adapter to 2048; 16 "
                            "clips x 30 s (376 tokens each), bf16 weights, f32 accumulation",
+            "lfm_ragged": "LFM2A encoder from PCM (second log-mel front-end, stem, 17 blocks, adapter) on the "
+                          "ragged batch: 256 clips of 1-30 s, packed, bf16 weights, f32 accumulation",
             "attention": "local-attention core only, 32 x 8192 tokens, 8 heads x 128, bf16 q/k/v",
             "resample": "mixdown + Kaiser-sinc resampling to 16 kHz, 64 stereo clips x 30 s at 44.1 kHz, f32"}[name]
     d = {"workload": f"{name}: {base}", "l2": "flushed between steps (256 MiB write)",
@@ -185,7 +187,8 @@ def workload_desc(name: str, info: dict) -> dict:
 
 
 ENCODE_WORKLOADS = ("tower", "tower_fp8", "ragged")
-CLIP_WORKLOADS = ENCODE_WORKLOADS + ("frontend", "lfm_frontend", "lfm_encoder")
+LFM_ENCODER_WORKLOADS = ("lfm_encoder", "lfm_ragged")
+CLIP_WORKLOADS = ENCODE_WORKLOADS + ("frontend", "lfm_frontend") + LFM_ENCODER_WORKLOADS
 
 
 def rank_clips(lengths, world: int, rank: int, partition) -> list[int]:
@@ -206,7 +209,8 @@ def audio_seconds(lengths) -> float:
 def data_of(name: str) -> str:
     """The synthetic batch a workload runs on (the e4m3 tower runs the tower's,
     the second front-end the first one's)."""
-    return {"tower_fp8": "tower", "lfm_frontend": "frontend", "lfm_encoder": "tower"}.get(name, name)
+    return {"tower_fp8": "tower", "lfm_frontend": "frontend", "lfm_encoder": "tower", "lfm_ragged": "ragged"}.get(
+        name, name)
 
 
 class Ours:
@@ -222,6 +226,9 @@ class Ours:
             self.lens = [lens_all[i] for i in self.mine]
             self.job_clips, self.job_audio_s = len(lens_all), audio_seconds(lens_all)
             self.job_tokens = sum(ae.ae_num_tokens(n) for n in lens_all)
+            if name in LFM_ENCODER_WORKLOADS:  # the LFM2A encoder's own rows: its stem leaves 12.5 per second
+                cfg = ae.lfm_config()
+                self.job_tokens = sum(ae.ae_lenc_num_tokens(ae.ae_lfm_num_frames(cfg, n)) for n in lens_all)
             clips = synth.global_waves(data_of(name), lens_all, self.mine)
             flat, self.off = synth.pack(clips)
             self.h_wave = torch.from_numpy(flat).pin_memory()
@@ -237,7 +244,7 @@ class Ours:
             self.ws_host_bytes = ae.ae_encode_host_workspace_size(self.model, self.off)
             self.ws = torch.empty(max(self.ws_bytes, self.ws_host_bytes), dtype=torch.uint8, device="cuda")
             self.dominant = "gemm_fp8" if name == "tower_fp8" else "gemm"
-        elif name == "lfm_encoder":
+        elif name in LFM_ENCODER_WORKLOADS:
             self.cfg = ae.lfm_config()
             self.lfm_frames = [ae.ae_lfm_num_frames(self.cfg, n) for n in self.lens]
             self.frames = sum(self.lfm_frames)
@@ -310,7 +317,7 @@ class Ours:
             ae.ae_logmel(self.d_wave, self.off, self.d_mel, self.ws, self.ws_bytes, self.stream)
         elif self.name == "lfm_frontend":
             ae.ae_lfm_logmel(self.cfg, self.d_wave, self.off, self.d_mel, self.ws, self.ws_bytes, self.stream)
-        elif self.name == "lfm_encoder":
+        elif self.name in LFM_ENCODER_WORKLOADS:
             ae.ae_lfm_logmel(self.cfg, self.d_wave, self.off, self.d_mel, self.lfm_ws, self.lfm_ws_bytes, self.stream)
             ae.ae_lenc_encode(self.enc, self.d_mel, self.frame_off, self.d_out, self.ws, self.ws_bytes, self.stream)
         elif self.name == "resample":
@@ -332,7 +339,7 @@ class Ours:
             self.h_mel.copy_(self.d_mel, non_blocking=True)
             self.stream.synchronize()
             return self.h_wave.numel() * 4, self.h_mel.numel() * 4
-        if self.name == "lfm_encoder":
+        if self.name in LFM_ENCODER_WORKLOADS:
             self.d_wave.copy_(self.h_wave, non_blocking=True)
             self.step()
             self.h_out.copy_(self.d_out, non_blocking=True)
@@ -404,6 +411,8 @@ class OracleRun:
             from oracle import resample as RS
             self.RS = RS
             self.next = 0
+        elif name in LFM_ENCODER_WORKLOADS:
+            self.next = 0
         elif name == "attention":
             p = synth.attention_params()
             q, k, v = synth.attention_qkv(0, T=2048)
@@ -433,15 +442,19 @@ class OracleRun:
             t0 = time.perf_counter()
             LF.features(c)
             return time.perf_counter() - t0, 30.0, "clip 0 of the frontend workload (second front-end)"
-        if self.name == "lfm_encoder":
+        if self.name in LFM_ENCODER_WORKLOADS:
             from oracle import lfm as LF
             from oracle import lfm_encoder as LE
             if not hasattr(self, "lenc_w"):
                 self.lenc_w = synth.lfm_encoder_weights()
-            c = synth.waves("tower", [0])[0]
+            data = data_of(self.name)
+            i = self.next % len(synth.clip_lengths(data))
+            self.next += 1
+            c = synth.waves(data, [i])[0]
             t0 = time.perf_counter()
             LE.encode(LF.features(c), self.lenc_w)
-            return time.perf_counter() - t0, 30.0, "clip 0 of the tower workload through the LFM2A front-end and encoder"
+            return (time.perf_counter() - t0, min(len(c), synth.MAX_SAMPLES) / synth.SAMPLE_RATE,
+                    f"clip {i} of the {data} workload through the LFM2A front-end and encoder")
         if self.name == "resample":
             i = self.next % synth.RS_CLIPS
             self.next += 1
@@ -601,7 +614,7 @@ def run_ours(args, rank, world, dist):
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(per_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None,
-        "dtype": {"frontend": "f32", "lfm_frontend": "f32", "resample": "f32", "lfm_encoder": "bf16",
+        "dtype": {"frontend": "f32", "lfm_frontend": "f32", "resample": "f32", "lfm_encoder": "bf16", "lfm_ragged": "bf16",
                   "tower_fp8": "e4m3+bf16"}.get(args.workload, "bf16"),
         "data": "synthetic",
         "config": workload_desc(args.workload, (({
@@ -624,6 +637,7 @@ def run_ours(args, rank, world, dist):
                     "ragged": "ae_encode_host_async, two streams (copies of one step overlap the kernels of the other)",
                     "frontend": "ae_logmel + copies", "lfm_frontend": "ae_lfm_logmel + copies",
                     "lfm_encoder": "ae_lfm_logmel + ae_lenc_encode + copies",
+                    "lfm_ragged": "ae_lfm_logmel + ae_lenc_encode + copies",
                     "resample": "ae_resample + copies"}[args.workload]},
         "gpu_launches": int(launches_timed),
         "roofline": roof,
@@ -666,6 +680,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", choices=("tower", "tower_fp8", "ragged", "frontend", "lfm_frontend", "lfm_encoder",
+                                           "lfm_ragged",
                                            "attention", "resample"),
                     default="ragged")
     ap.add_argument("--no-cpu-baseline", action="store_true")

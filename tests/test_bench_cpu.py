@@ -34,7 +34,9 @@ def test_tensor_peak_follows_the_clock():
 def test_workload_tables():
     assert bench.data_of("tower_fp8") == "tower" and bench.data_of("lfm_frontend") == "frontend"
     assert bench.data_of("ragged") == "ragged"
-    for w in ("tower", "tower_fp8", "ragged", "frontend", "lfm_frontend", "lfm_encoder", "attention", "resample"):
+    assert bench.data_of("lfm_encoder") == "tower" and bench.data_of("lfm_ragged") == "ragged"
+    for w in ("tower", "tower_fp8", "ragged", "frontend", "lfm_frontend", "lfm_encoder", "lfm_ragged", "attention",
+              "resample"):
         d = bench.workload_desc(w, {"parallelism": "replicas x1"})
         assert d["workload"].startswith(w + ":") and "l2" in d
 
