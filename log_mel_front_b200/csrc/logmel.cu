@@ -8,7 +8,9 @@
 //
 //  1. Staging. The contiguous waveform span of the 32 frames (33 x 160
 //     samples) is copied into shared memory with 4-byte cp.async (zero fill
-//     outside the clip, which is the semicausal pad and the clip end).
+//     outside the clip, which is the semicausal pad and the clip end), into
+//     one of two buffers: the next item's copy is issued when an item starts,
+//     so it is in flight during the whole item.
 //  2. Spectra: 16 groups of 16 threads, two frames per group. A frame's 320
 //     windowed samples are packed as 160 complex values z[n] = x[2n] +
 //     i x[2n+1] and transformed by a 256-point complex FFT in the four-step
@@ -30,25 +32,21 @@
 //
 // Per-thread constants (the window values and FFT twiddles it uses) are
 // computed once at kernel start in float32 (sincospif / cospif, within an
-// ulp or so of the float64 values). The log is ln(2) (e + log2(m)) for
-// x = m 2^e, m in [1, 2), with the hardware's lg2 on m, whose absolute error
-// there is about 2^-22: the result is within 1e-6 of ln(x) for the values
-// that occur (x >= 0.001).
+// ulp or so of the float64 values). The log is ln(2) log2(x) with the
+// hardware's base-2 logarithm, within 1e-5 of ln(x) for the values that
+// occur (x >= 0.001).
 #include "ae_internal.h"
 #include "common.cuh"
 #include "fft16.cuh"
 
 namespace ae {
 
-// ln(acc + 0.001) for acc >= 0.
+// ln(acc + 0.001) for acc >= 0: the hardware's base-2 logarithm (within a few
+// ulp of the result for the arguments that occur, x >= 0.001), times ln 2.
 __device__ __forceinline__ float log_floor_sum(float acc) {
-  const float x = acc + 1e-3f;
-  const int bits = __float_as_int(x);
-  const float e = (float)((bits >> 23) - 127);
-  const float m = __int_as_float((bits & 0x007FFFFF) | 0x3F800000);
   float l2;
-  asm("lg2.approx.f32 %0, %1;" : "=f"(l2) : "f"(m));
-  return (e + l2) * 0.69314718055994531f;
+  asm("lg2.approx.f32 %0, %1;" : "=f"(l2) : "f"(acc + 1e-3f));
+  return l2 * 0.69314718055994531f;
 }
 
 }  // namespace ae
@@ -70,7 +68,7 @@ constexpr int kBins = kFft / 2 + 1;
 static_assert(kItem == 32 && kGroups * 2 == kItem, "one frame per lane in the band phase, two per FFT group");
 
 struct LogmelSmem {
-  float wave[kSpan];
+  float wave[2][kSpan];                        // this item's samples and the next one's (in flight)
   union {
     float2 xs[kGroups][16 * kPitch];           // per-group transpose tiles (spectra phase)
     float out[kItem][kOutPitch];               // log-mel rows (band and store phases)
@@ -147,7 +145,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   int tile = blockIdx.x;
   Item it = tile < n_tiles ? item_of(t, tile) : Item{0, 0, 0};
   // ---- stage the first item
-  auto stage = [&](const Item &x) {
+  auto stage = [&](const Item &x, int buf) {
     const int64_t s_begin = t.sample_off[x.clip];
     const int64_t n_samp = min(t.sample_off[x.clip + 1] - s_begin, (int64_t)kMaxSamples);
     const int64_t first = (int64_t)(x.f0 - 1) * kHop;  // local sample i is clip sample first + i
@@ -157,21 +155,28 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float *src = wave + s_begin + first;
     for (int i = tid; i < span; i += kThreads) {
       const bool ok = i >= lo && i < hi;
-      cp_async4(S.wave + i, ok ? src + i : wave, ok);
+      cp_async4(S.wave[buf] + i, ok ? src + i : wave, ok);
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
-  if (tile < n_tiles) stage(it);
+  if (tile < n_tiles) stage(it, 0);
 
-  for (; tile < n_tiles; tile += gridDim.x) {
+  for (int buf = 0; tile < n_tiles; tile += gridDim.x, buf ^= 1) {
     asm volatile("cp.async.wait_all;" ::: "memory");
-    __syncthreads();  // staged wave visible; the previous item's output rows are stored
+    __syncthreads();  // this item's wave visible; the previous item's output rows are stored
+    // ---- the next item's samples load during this whole item
+    const Item cur = it;
+    const int next = tile + gridDim.x;
+    if (next < n_tiles) {
+      it = item_of(t, next);
+      stage(it, buf ^ 1);
+    }
 
     // ---- spectra: frames g and g + 16 of the item
     float2 *xs = S.u.xs[g];
 #pragma unroll 1
-    for (int fi = g; fi < it.nf; fi += kGroups) {
-      const float *wv = S.wave + fi * kHop;
+    for (int fi = g; fi < cur.nf; fi += kGroups) {
+      const float *wv = S.wave[buf] + fi * kHop;
       float2 x[16];
 #pragma unroll
       for (int n1 = 0; n1 < 16; ++n1) {
@@ -224,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();  // magnitudes complete
 
     // ---- bands: lane = frame
-    if (lane < it.nf) {
+    if (lane < cur.nf) {
       switch (warp) {
         case 0: band_phase<0>(S, S, lane); break;
         case 1: band_phase<1>(S, S, lane); break;
@@ -236,15 +241,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         default: band_phase<7>(S, S, lane); break;
       }
     }
-    __syncthreads();  // rows complete; the staged wave is free
-
-    // ---- next item's staging overlaps this item's store
-    const Item cur = it;
-    const int next = tile + gridDim.x;
-    if (next < n_tiles) {
-      it = item_of(t, next);
-      stage(it);
-    }
+    __syncthreads();  // rows complete
     float *orow = mel + ((int64_t)t.frame_off[cur.clip] + cur.f0) * kMels;
     const int n = cur.nf * kMels;
     for (int i = tid; i < n; i += kThreads) orow[i] = S.u.out[i >> 7][i & (kMels - 1)];
