@@ -67,6 +67,18 @@ constexpr int kBins = kFft / 2 + 1;
 
 static_assert(kItem == 32 && kGroups * 2 == kItem, "one frame per lane in the band phase, two per FFT group");
 
+// Where an item's samples come from and its rows go: resolved for a run of the
+// CTA's items at once (one clip search per thread, in parallel), so that no
+// item waits on a chain of dependent table loads.
+struct TileRec {
+  long long first;    // index in the wave array of the item's local sample 0 (before the clip for frame 0)
+  int out_row;        // output row of the item's first frame
+  unsigned short hi;  // local samples [lo, hi) lie inside the clip
+  unsigned char pad;  // 1: the item starts at frame 0, lo = kHop (the semicausal pad); 0: lo = 0
+  unsigned char nf;   // frames in the item
+};
+constexpr int kRecs = 192;
+
 struct LogmelSmem {
   float wave[2][kSpan];                        // this item's samples and the next one's (in flight)
   union {
@@ -74,7 +86,10 @@ struct LogmelSmem {
     float out[kItem][kOutPitch];               // log-mel rows (band and store phases)
   } u;
   float mag[kItem][kMagPitch];
+  TileRec rec[kRecs];                          // the CTA's items kRecs at a time
 };
+static_assert(sizeof(TileRec) == 16, "tile record");
+static_assert(2 * (sizeof(LogmelSmem) + 1024) <= 228 * 1024, "two CTAs per SM");
 
 __device__ __forceinline__ void cp_async4(float *dst, const float *src, bool valid) {
   const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
@@ -142,40 +157,57 @@ __global__ void __launch_bounds__(kThreads, 2)
     wj = make_float2(c, -s);
   }
 
-  int tile = blockIdx.x;
-  Item it = tile < n_tiles ? item_of(t, tile) : Item{0, 0, 0};
-  // ---- stage the first item
-  auto stage = [&](const Item &x, int buf) {
-    const int64_t s_begin = t.sample_off[x.clip];
-    const int64_t n_samp = min(t.sample_off[x.clip + 1] - s_begin, (int64_t)kMaxSamples);
-    const int64_t first = (int64_t)(x.f0 - 1) * kHop;  // local sample i is clip sample first + i
-    const int span = x.nf * kHop + kHop;
-    // local indices inside the clip: [lo, hi)
-    const int lo = (int)max((int64_t)0, -first), hi = (int)min((int64_t)span, n_samp - first);
-    const float *src = wave + s_begin + first;
+  // this CTA's items are tiles blockIdx.x + k gridDim.x, k < my_tiles
+  const int my_tiles = (int)blockIdx.x < n_tiles ? (n_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  auto fill = [&](int base) {  // records of items base .. base + kRecs - 1
+    for (int k = tid; k < kRecs && base + k < my_tiles; k += kThreads) {
+      const Item x = item_of(t, (int)blockIdx.x + (base + k) * (int)gridDim.x);
+      const int64_t s_begin = t.sample_off[x.clip];
+      const int64_t n_samp = min(t.sample_off[x.clip + 1] - s_begin, (int64_t)kMaxSamples);
+      const int64_t first = (int64_t)(x.f0 - 1) * kHop;  // local sample i is clip sample first + i
+      const int64_t span = x.nf * kHop + kHop;
+      TileRec r;
+      r.first = s_begin + first;
+      r.out_row = t.frame_off[x.clip] + x.f0;
+      r.hi = (unsigned short)max((int64_t)0, min(span, n_samp - first));
+      r.pad = first < 0 ? 1 : 0;
+      r.nf = (unsigned char)x.nf;
+      S.rec[k] = r;
+    }
+  };
+  // ---- stage an item: its waveform span, zero outside the clip
+  auto stage = [&](const TileRec &r, int buf) {
+    const int span = r.nf * kHop + kHop, lo = r.pad ? kHop : 0, hi = r.hi;
+    const float *src = wave + r.first;
     for (int i = tid; i < span; i += kThreads) {
       const bool ok = i >= lo && i < hi;
       cp_async4(S.wave[buf] + i, ok ? src + i : wave, ok);
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
-  if (tile < n_tiles) stage(it, 0);
+  fill(0);
+  __syncthreads();
+  if (my_tiles > 0) stage(S.rec[0], 0);
 
-  for (int buf = 0; tile < n_tiles; tile += gridDim.x, buf ^= 1) {
+  for (int k = 0; k < my_tiles; ++k) {
+    const int buf = k & 1;
     asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();  // this item's wave visible; the previous item's output rows are stored
+    const int cur_nf = S.rec[k % kRecs].nf, cur_row = S.rec[k % kRecs].out_row;
     // ---- the next item's samples load during this whole item
-    const Item cur = it;
-    const int next = tile + gridDim.x;
-    if (next < n_tiles) {
-      it = item_of(t, next);
-      stage(it, buf ^ 1);
+    if (k + 1 < my_tiles) {
+      if ((k + 1) % kRecs == 0) {  // the next run of records (uniform across the CTA)
+        __syncthreads();
+        fill(k + 1);
+        __syncthreads();
+      }
+      stage(S.rec[(k + 1) % kRecs], buf ^ 1);
     }
 
     // ---- spectra: frames g and g + 16 of the item
     float2 *xs = S.u.xs[g];
 #pragma unroll 1
-    for (int fi = g; fi < cur.nf; fi += kGroups) {
+    for (int fi = g; fi < cur_nf; fi += kGroups) {
       const float *wv = S.wave[buf] + fi * kHop;
       float2 x[16];
 #pragma unroll
@@ -229,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();  // magnitudes complete
 
     // ---- bands: lane = frame
-    if (lane < cur.nf) {
+    if (lane < cur_nf) {
       switch (warp) {
         case 0: band_phase<0>(S, S, lane); break;
         case 1: band_phase<1>(S, S, lane); break;
@@ -242,8 +274,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
     __syncthreads();  // rows complete
-    float *orow = mel + ((int64_t)t.frame_off[cur.clip] + cur.f0) * kMels;
-    const int n = cur.nf * kMels;
+    float *orow = mel + (int64_t)cur_row * kMels;
+    const int n = cur_nf * kMels;
     for (int i = tid; i < n; i += kThreads) orow[i] = S.u.out[i >> 7][i & (kMels - 1)];
   }
 }
