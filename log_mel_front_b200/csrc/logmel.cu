@@ -7,10 +7,12 @@
 // item at a time, two CTAs per SM, persistent over the items. Per item:
 //
 //  1. Staging. The contiguous waveform span of the 32 frames (33 x 160
-//     samples) is copied into shared memory with 4-byte cp.async (zero fill
-//     outside the clip, which is the semicausal pad and the clip end), into
-//     one of two buffers: the next item's copy is issued when an item starts,
-//     so it is in flight during the whole item.
+//     samples) is copied into shared memory with cp.async, zero fill outside
+//     the clip (the semicausal pad and the clip end), into one of two buffers:
+//     the next item's copy is issued when an item starts, so it is in flight
+//     during the whole item. The copies are 16 bytes wide where the span
+//     starts on a 16-byte boundary (every item of a clip whose first sample
+//     does), else 4 bytes wide.
 //  2. Spectra: 16 groups of 16 threads, two frames per group. A frame's 320
 //     windowed samples are packed as 160 complex values z[n] = x[2n] +
 //     i x[2n+1] and transformed by a 256-point complex FFT in the four-step
@@ -21,14 +23,16 @@
 //     X[k] = A - i W512^k B and X[256 - k] = conj(A + i W512^k B), with
 //     A = Z[k] + conj Z[256 - k], B = Z[k] - conj Z[256 - k]: thread j takes
 //     the pairs of its k2 < 8, Z[256 - k] coming from thread 16 - j by one
-//     shuffle per pair (threads 0 and 8 hold both members). The window carries
-//     the split's factor 1/2. The 257 magnitudes go to a [frame][bin] tile.
+//     shuffle per pair (threads 0 and 8 hold both members); the W512^k come
+//     from a per-CTA table. The window carries the split's factor 1/2. The 257
+//     magnitudes (the hardware square root of |X|^2) go to a [frame][bin] tile.
 //  3. Bands: one frame per lane. Warp w computes the bands [kWarpBand[w],
 //     kWarpBand[w+1]) of the 32 frames as straight-line code with the HTK
 //     weights as literals (htk_bank.h, 506 multiply-adds per frame, split
 //     evenly over the warps), reading the magnitudes from the tile (odd row
 //     pitch: lane f reads row f without bank conflicts), then the log.
-//  4. Store: the [32][128] result leaves as whole contiguous rows.
+//  4. Store: the [32][128] result leaves as whole contiguous rows, thread t
+//     storing column t mod 128 of every other row.
 //
 // Per-thread constants (the window values and FFT twiddles it uses) are
 // computed once at kernel start in float32 (sincospif / cospif, within an
@@ -77,7 +81,7 @@ struct TileRec {
   unsigned char pad;  // 1: the item starts at frame 0, lo = kHop (the semicausal pad); 0: lo = 0
   unsigned char nf;   // frames in the item
 };
-constexpr int kRecs = 192;
+constexpr int kRecs = 128;
 
 struct LogmelSmem {
   float wave[2][kSpan];                        // this item's samples and the next one's (in flight)
@@ -86,6 +90,7 @@ struct LogmelSmem {
     float out[kItem][kOutPitch];               // log-mel rows (band and store phases)
   } u;
   float mag[kItem][kMagPitch];
+  float2 wk[8][16];                            // W512^(j + 16 k2) at [k2][j]: the split's twiddles
   TileRec rec[kRecs];                          // the CTA's items kRecs at a time
 };
 static_assert(sizeof(TileRec) == 16, "tile record");
@@ -95,6 +100,19 @@ __device__ __forceinline__ void cp_async4(float *dst, const float *src, bool val
   const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
   const int n = valid ? 4 : 0;  // src-size 0: 4 zero bytes
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(d), "l"(src), "r"(n) : "memory");
+}
+
+// 16-byte copy of which the first nbytes come from src and the rest are zero
+__device__ __forceinline__ void cp_async16(float *dst, const float *src, int nbytes) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(nbytes) : "memory");
+}
+
+// |X| from |X|^2 >= 0: the hardware square root (0 for 0)
+__device__ __forceinline__ float magnitude(float sq) {
+  float r;
+  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(sq));
+  return r;
 }
 
 struct Item {
@@ -112,14 +130,6 @@ __device__ __forceinline__ Item item_of(const ClipTablesDev &t, int tile) {
   it.f0 = (tile - t.mel_tile_off[lo]) * kItem;
   it.nf = min(kItem, t.frame_off[lo + 1] - t.frame_off[lo] - it.f0);
   return it;
-}
-
-// W32^k2 = (cos, -sin)(2 pi k2 / 32), k2 < 8
-__device__ __forceinline__ float2 w32(int k2) {
-  constexpr float c[8] = {1.0f, 0.98078528040323043f, 0.92387953251128674f, 0.83146961230254524f,
-                          0.70710678118654752f, 0.55557023301960218f, 0.38268343236508977f,
-                          0.19509032201612825f};
-  return make_float2(c[k2], -c[(8 - k2) & 7] * (k2 != 0));
 }
 
 template <int W>
@@ -150,11 +160,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     sincospif((float)((2 * j * k1) & (kFft - 1)) / 256.0f, &s, &c);
     tw1[k1] = make_float2(c, -s);
   }
-  float2 wj;  // W512^j
-  {
+  for (int e = tid; e < 8 * 16; e += kThreads) {  // W512^(j + 16 k2), e = 16 k2 + j
     float s, c;
-    sincospif((float)j / 256.0f, &s, &c);
-    wj = make_float2(c, -s);
+    sincospif((float)((e & 15) + 16 * (e >> 4)) / 256.0f, &s, &c);
+    S.wk[e >> 4][e & 15] = make_float2(c, -s);
   }
 
   // this CTA's items are tiles blockIdx.x + k gridDim.x, k < my_tiles
@@ -179,9 +188,20 @@ __global__ void __launch_bounds__(kThreads, 2)
   auto stage = [&](const TileRec &r, int buf) {
     const int span = r.nf * kHop + kHop, lo = r.pad ? kHop : 0, hi = r.hi;
     const float *src = wave + r.first;
-    for (int i = tid; i < span; i += kThreads) {
-      const bool ok = i >= lo && i < hi;
-      cp_async4(S.wave[buf] + i, ok ? src + i : wave, ok);
+    float *dst = S.wave[buf];
+    if ((reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+      // span and lo are multiples of 4: a chunk is outside [lo, hi), inside, or cut by hi
+      const float *any = src + lo;  // an aligned address for the chunks that read nothing
+#pragma unroll 2
+      for (int i = 4 * tid; i < span; i += 4 * kThreads) {
+        const int nb = i < lo ? 0 : 4 * max(0, min(4, hi - i));
+        cp_async16(dst + i, nb ? src + i : any, nb);
+      }
+    } else {
+      for (int i = tid; i < span; i += kThreads) {
+        const bool ok = i >= lo && i < hi;
+        cp_async4(dst + i, ok ? src + i : wave, ok);
+      }
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
@@ -214,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int n1 = 0; n1 < 16; ++n1) {
         if (n1 < 10) {
           const float2 a = *reinterpret_cast<const float2 *>(wv + 32 * n1 + 2 * j);
-          x[n1] = make_float2(a.x * win[n1].x, a.y * win[n1].y);
+          x[n1] = __fmul2_rn(a, win[n1]);
         } else {
           x[n1] = make_float2(0.f, 0.f);
         }
@@ -240,21 +260,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (j == 0) mr = x[(16 - k2) & 15];  // thread 0 pairs 16 k2 with 16 (16 - k2), k2 = 0 with itself
         const float2 mc = make_float2(mr.x, -mr.y);  // conj Z[256 - k]
         const float2 A = cadd(o, mc), B = csub(o, mc);
-        const float2 w = cmul(wj, w32(k2));  // W512^(j + 16 k2)
-        const float2 wb = cmul(B, w);
+        const float2 wb = cmul(B, S.wk[k2][j]);  // W512^(j + 16 k2) B
         // P = i W B = (-Im, Re)
         const float2 P = make_float2(-wb.y, wb.x);
         const float2 x1 = csub(A, P), x2 = cadd(A, P);  // X[k], conj X[256 - k]
         const float2 q1 = __fmul2_rn(x1, x1), q2 = __fmul2_rn(x2, x2);
         const float m1 = q1.x + q1.y, m2 = q2.x + q2.y;
         const int k = j + 16 * k2;
-        mg[k] = m1 * rsqrtf(fmaxf(m1, 1e-37f));  // |X| to about 2 ulp, 0 for 0
-        mg[kFft / 2 - k] = m2 * rsqrtf(fmaxf(m2, 1e-37f));
+        mg[k] = magnitude(m1);
+        mg[kFft / 2 - k] = magnitude(m2);
       }
       if (j == 0) {
         // k = 128 is its own partner: |X[128]| = 2 |Z[128]|
-        const float m8 = fmaf(x[8].x, x[8].x, x[8].y * x[8].y);
-        mg[kFft / 4] = 2.0f * m8 * rsqrtf(fmaxf(m8, 1e-37f));
+        mg[kFft / 4] = 2.0f * magnitude(fmaf(x[8].x, x[8].x, x[8].y * x[8].y));
       }
       __syncwarp(gmask);  // the tile is free for the next frame
     }
@@ -274,9 +292,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
     __syncthreads();  // rows complete
-    float *orow = mel + (int64_t)cur_row * kMels;
-    const int n = cur_nf * kMels;
-    for (int i = tid; i < n; i += kThreads) orow[i] = S.u.out[i >> 7][i & (kMels - 1)];
+    float *orow = mel + (int64_t)cur_row * kMels + (tid & (kMels - 1));
+    const int r0 = tid >> 7;
+#pragma unroll
+    for (int q = 0; q < kItem; q += kThreads / kMels)
+      if (r0 + q < cur_nf) orow[(r0 + q) * kMels] = S.u.out[r0 + q][tid & (kMels - 1)];
   }
 }
 

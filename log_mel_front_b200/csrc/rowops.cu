@@ -279,15 +279,40 @@ cudaError_t launch_lconv(const ae_model *m, const void *gl, const float *w_dw, c
 
 // The per-call tables travel as kernel parameters (copied at launch, so the
 // call never waits on the host and stays capturable).
+template <int W>
 struct UploadChunk {
   int64_t dst;  // byte offset in the workspace
   int n;        // 32-bit words
-  uint32_t w[7936];
+  uint32_t w[W];
 };
 
-__global__ void k_upload(uint8_t *base, const UploadChunk ch) {
+template <int W>
+__global__ void k_upload(uint8_t *base, const UploadChunk<W> ch) {
   uint32_t *d = reinterpret_cast<uint32_t *>(base + ch.dst);
   for (int i = threadIdx.x; i < ch.n; i += blockDim.x) d[i] = ch.w[i];
+}
+
+// Copies nw words from the host to dev in chunks of at most 7936 words, each in
+// the smallest parameter block that holds it (a launch copies its whole
+// parameter block, so a few tables do not pay for 31 KB).
+template <int W>
+static cudaError_t upload_chunk(const uint32_t *src, size_t n, uint8_t *dst, cudaStream_t s) {
+  static thread_local UploadChunk<W> ch;
+  ch.dst = 0;
+  ch.n = (int)n;
+  std::memcpy(ch.w, src, n * 4);
+  return launch_k(k_upload<W>, dim3(1), dim3(256), 0, s, dst, ch);
+}
+
+static cudaError_t upload_words(const uint32_t *src, size_t nw, uint8_t *dst, cudaStream_t s) {
+  for (size_t w0 = 0; w0 < nw; w0 += 7936) {
+    const size_t n = nw - w0 < 7936 ? nw - w0 : 7936;
+    const cudaError_t e = n <= 512    ? upload_chunk<512>(src + w0, n, dst + 4 * w0, s)
+                          : n <= 2048 ? upload_chunk<2048>(src + w0, n, dst + 4 * w0, s)
+                                      : upload_chunk<7936>(src + w0, n, dst + 4 * w0, s);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 __global__ void k_pos(int32_t *pos, const int32_t *tok_off) {
@@ -304,20 +329,9 @@ cudaError_t launch_pos(int32_t *pos, const int32_t *tok_off, int n_clips, cudaSt
 static size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 
 cudaError_t launch_upload_bytes(const void *host, size_t bytes, void *dev, cudaStream_t s) {
-  static thread_local UploadChunk ch;
-  const size_t nw = (bytes + 3) / 4;
-  const uint8_t *src = static_cast<const uint8_t *>(host);
-  for (size_t w0 = 0; w0 < nw; w0 += 7936) {
-    const size_t n = nw - w0 < 7936 ? nw - w0 : 7936;
-    ch.dst = (int64_t)(w0 * 4);
-    ch.n = (int)n;
-    const size_t b = std::min(bytes - w0 * 4, n * 4);
-    std::memset(ch.w, 0, n * 4);
-    std::memcpy(ch.w, src + w0 * 4, b);
-    cudaError_t e = launch_k(k_upload, dim3(1), dim3(256), 0, s, static_cast<uint8_t *>(dev), ch);
-    if (e != cudaSuccess) return e;
-  }
-  return cudaSuccess;
+  std::vector<uint32_t> words((bytes + 3) / 4, 0u);
+  std::memcpy(words.data(), host, bytes);
+  return upload_words(words.data(), words.size(), static_cast<uint8_t *>(dev), s);
 }
 
 size_t tables_bytes(int64_t n_clips) {
@@ -346,16 +360,7 @@ cudaError_t launch_upload_tables(const ClipTables &t, void *ws, const WsLayout &
   const size_t o_mt = put(t.mel_tile_off.data(), B1 * 4);
   const size_t o_ct = put(t.conv1_tile_off.data(), B1 * 4);
   uint8_t *base = static_cast<uint8_t *>(ws) + L.tables;
-  const size_t nw = off / 4;
-  static thread_local UploadChunk ch;
-  for (size_t w0 = 0; w0 < nw; w0 += 7936) {
-    const size_t n = nw - w0 < 7936 ? nw - w0 : 7936;
-    ch.dst = (int64_t)(w0 * 4);
-    ch.n = (int)n;
-    std::memcpy(ch.w, words.data() + w0, n * 4);
-    cudaError_t e = launch_k(k_upload, dim3(1), dim3(256), 0, s, base, ch);
-    if (e != cudaSuccess) return e;
-  }
+  if (const cudaError_t e = upload_words(words.data(), off / 4, base, s)) return e;
   dev->n_clips = t.n_clips;
   dev->sample_off = reinterpret_cast<const int64_t *>(base + o_s);
   dev->frame_off = reinterpret_cast<const int32_t *>(base + o_f);

@@ -110,6 +110,21 @@ def test_logmel_edge_lengths_packed():
     assert np.max(np.abs(sil - math.log(1e-3))) < 1e-6
 
 
+def test_logmel_same_clip_at_every_sample_alignment():
+    # the staging copies 16 bytes at a time where a clip starts on a 16-byte
+    # boundary and 4 bytes at a time elsewhere: the same clip placed at the four
+    # offsets mod 4 (one-sample spacer clips between) gives the same rows
+    rng = np.random.default_rng(11)
+    c = (0.3 * rng.standard_normal(7776)).astype(np.float32)
+    one = np.array([0.25], np.float32)
+    g = gpu_logmel([c, one, c, one, c, one, c])
+    n, n1 = O.num_frames(len(c)), O.num_frames(1)
+    starts = [k * (n + n1) for k in range(4)]
+    for s0 in starts[1:]:
+        assert np.array_equal(g[s0:s0 + n], g[:n])
+    assert_logmel(g[:n], O.log_mel(c), "log-mel 7776-sample clip")
+
+
 def test_logmel_tone_band():
     t = np.arange(16000) / 16000
     wave = (0.5 * np.sin(2 * np.pi * 1000.0 * t)).astype(np.float32)
