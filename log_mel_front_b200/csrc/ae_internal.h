@@ -265,20 +265,25 @@ cudaError_t launch_upload_bytes(const void *host, size_t bytes, void *dev, cudaS
 constexpr int kLfmMaxMels = 128;  // bands
 constexpr int kLfmMaxBins = 32;   // nonzero bins per band
 constexpr int kLfmTile = 32;      // frames per work item of the spectrum kernel
+constexpr int kLfmWarps = 8;      // warps of the spectrum kernel's band phase
 struct LfmTablesDev {
   int n_clips, n_tiles;              // tiles: kLfmTile frames of one clip
   const int64_t *sample_off;         // [B + 1]
   const int32_t *frame_off, *tile_off;  // [B + 1]
   const int32_t *eff;                // [B]: frames whose statistics count
-  const int32_t *bank_lo;            // [n_mels]: first nonzero bin of each band
-  const float *bank_w;               // [n_mels][kLfmMaxBins]: its weights from there
+  const int32_t *bank_lo, *bank_cnt, *bank_off;  // [n_mels]: first bin, bins, offset in bank_w
+  const float *bank_w;               // [nnz]: the bands' weights, packed
+  unsigned long long *moments;       // [B][kLfmMaxMels][2]: sum v, sum v^2 in 2^-24 units (zeroed per call)
 };
 struct LfmParams {
   int n_mels, hop, win_length;
-  int bins;  // the widest band's nonzero bins, rounded up to 4 (<= kLfmMaxBins)
+  int nnz;          // packed weights
+  int wave_floats;  // staged-sample buffer of the spectrum kernel (a multiple of 4)
+  int vec16;        // 1: the waveform base is 16-byte aligned (16-byte staging copies)
   float preemph, log_floor, var_eps;
+  int wband[kLfmWarps + 1];  // bands of each warp in the band phase
 };
-size_t lfm_smem_bytes(int hop);
+size_t lfm_smem_bytes(const LfmParams &prm);
 cudaError_t launch_lfm(const float *wave, float *out, const LfmTablesDev &t, const LfmParams &prm, cudaStream_t s);
 
 // LFM2A Conformer encoder (lenc.cu, lenc_attention.cu): the shape the kernels

@@ -1212,7 +1212,7 @@ bool lfm_cfg_ok(const ae_lfm_config *c) {
 }
 
 struct LfmLayout {
-  size_t sample_off, frame_off, tile_off, eff, bank_lo, bank_w, total;
+  size_t sample_off, frame_off, tile_off, eff, bank_lo, bank_cnt, bank_off, bank_w, moments, total;
 };
 LfmLayout lfm_layout(int n_clips) {
   LfmLayout L;
@@ -1223,7 +1223,10 @@ LfmLayout lfm_layout(int n_clips) {
   L.tile_off = off; off += al256(B1 * 4);
   L.eff = off; off += al256(std::max<size_t>(n_clips, 1) * 4);
   L.bank_lo = off; off += al256((size_t)kLfmMaxMels * 4);
+  L.bank_cnt = off; off += al256((size_t)kLfmMaxMels * 4);
+  L.bank_off = off; off += al256((size_t)kLfmMaxMels * 4);
   L.bank_w = off; off += al256((size_t)kLfmMaxMels * kLfmMaxBins * 4);
+  L.moments = off; off += al256(std::max<size_t>(n_clips, 1) * kLfmMaxMels * 2 * 8);
   L.total = off;
   return L;
 }
@@ -1274,11 +1277,25 @@ ae_status ae_lfm_logmel(const ae_lfm_config *cfg, const float *d_wave, const int
     to[i + 1] = (int32_t)tiles;
     eff[i] = (int32_t)((n + cfg->hop - 1) / cfg->hop);
   }
-  std::vector<int32_t> blo;
-  std::vector<float> bw;
-  int widest = 0;
-  if (!lfm_bank(*cfg, blo, bw, &widest, kLfmMaxBins))
-    return fail(AE_EUNSUPPORTED, "a mel band spans more than 32 FFT bins");
+  // the packed bank of the last configuration this thread used (built in
+  // float64 on the host; the sample rate, n_fft and n_mels decide it)
+  thread_local struct {
+    int32_t sr = 0, n_fft = 0, n_mels = 0;
+    bool ok = false;
+    LfmPackedBank P;
+  } bank;
+  if (bank.sr != cfg->sample_rate || bank.n_fft != cfg->n_fft || bank.n_mels != cfg->n_mels) {
+    std::vector<int32_t> blo;
+    std::vector<float> bw;
+    int widest = 0;
+    bank.ok = lfm_bank(*cfg, blo, bw, &widest, kLfmMaxBins);
+    bank.P = bank.ok ? lfm_bank_pack(blo, bw, cfg->n_mels, kLfmMaxBins, kLfmWarps) : LfmPackedBank{};
+    bank.sr = cfg->sample_rate;
+    bank.n_fft = cfg->n_fft;
+    bank.n_mels = cfg->n_mels;
+  }
+  if (!bank.ok) return fail(AE_EUNSUPPORTED, "a mel band spans more than 32 FFT bins");
+  const LfmPackedBank &P = bank.P;
   if (frames == 0) return AE_OK;
   if (!d_wave || !d_out) return fail(AE_EINVAL, "d_wave or d_out is null");
   if (!aligned16(d_out)) return fail(AE_EINVAL, "d_out must be 16-byte aligned");
@@ -1287,16 +1304,17 @@ ae_status ae_lfm_logmel(const ae_lfm_config *cfg, const float *d_wave, const int
   if (st) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t *w = static_cast<uint8_t *>(d_ws);
-  cudaError_t e = cudaSuccess;
-  auto up = [&](const void *h, size_t bytes, size_t off) {
-    if (e == cudaSuccess && bytes) e = launch_upload_bytes(h, bytes, w + off, s);
-  };
-  up(so.data(), so.size() * 8, L.sample_off);
-  up(fo.data(), fo.size() * 4, L.frame_off);
-  up(to.data(), to.size() * 4, L.tile_off);
-  up(eff.data(), eff.size() * 4, L.eff);
-  up(blo.data(), blo.size() * 4, L.bank_lo);
-  up(bw.data(), bw.size() * 4, L.bank_w);
+  std::vector<uint8_t> h(L.bank_w + P.w.size() * 4, 0);  // the tables up to the packed weights in use
+  auto put = [&](const void *src, size_t bytes, size_t off) { if (bytes) std::memcpy(h.data() + off, src, bytes); };
+  put(so.data(), so.size() * 8, L.sample_off);
+  put(fo.data(), fo.size() * 4, L.frame_off);
+  put(to.data(), to.size() * 4, L.tile_off);
+  put(eff.data(), eff.size() * 4, L.eff);
+  put(P.lo.data(), P.lo.size() * 4, L.bank_lo);
+  put(P.cnt.data(), P.cnt.size() * 4, L.bank_cnt);
+  put(P.off.data(), P.off.size() * 4, L.bank_off);
+  put(P.w.data(), P.w.size() * 4, L.bank_w);
+  cudaError_t e = launch_upload_bytes(h.data(), h.size(), w, s);
   if (e != cudaSuccess) return cuda_fail(e, "table upload");
   LfmTablesDev t;
   t.n_clips = n_clips;
@@ -1306,17 +1324,21 @@ ae_status ae_lfm_logmel(const ae_lfm_config *cfg, const float *d_wave, const int
   t.tile_off = reinterpret_cast<const int32_t *>(w + L.tile_off);
   t.eff = reinterpret_cast<const int32_t *>(w + L.eff);
   t.bank_lo = reinterpret_cast<const int32_t *>(w + L.bank_lo);
+  t.bank_cnt = reinterpret_cast<const int32_t *>(w + L.bank_cnt);
+  t.bank_off = reinterpret_cast<const int32_t *>(w + L.bank_off);
   t.bank_w = reinterpret_cast<const float *>(w + L.bank_w);
+  t.moments = reinterpret_cast<unsigned long long *>(w + L.moments);
   LfmParams prm;
   prm.n_mels = cfg->n_mels;
   prm.hop = cfg->hop;
   prm.win_length = cfg->win_length;
-  prm.bins = (widest + 3) & ~3;
+  prm.nnz = (int)P.w.size();
+  prm.wave_floats = ((kLfmTile - 1) * cfg->hop + 516 + 3) / 4 * 4;  // span + the predecessor + alignment shift
+  prm.vec16 = aligned16(d_wave) ? 1 : 0;
   prm.preemph = cfg->preemph;
   prm.log_floor = cfg->log_floor;
   prm.var_eps = cfg->var_eps;
-  // bytes: every sample read once, every output row written by the spectrum
-  // pass and read and rewritten by the normalisation
+  for (int i = 0; i <= kLfmWarps; ++i) prm.wband[i] = P.wband[i];
   const double bytes = 4.0 * (double)so[n_clips] + 12.0 * (double)frames * cfg->n_mels;
   if ((e = timed(AE_K_LFM, 0.0, bytes, s, [&] { return launch_lfm(d_wave, d_out, t, prm, s); })) != cudaSuccess)
     return cuda_fail(e, "lfm front-end");

@@ -50,4 +50,43 @@ inline bool lfm_bank(const ae_lfm_config &c, std::vector<int32_t> &lo, std::vect
   return true;
 }
 
+// The bank as the spectrum kernel reads it: per band its first bin, its number
+// of bins up to the last nonzero weight and the offset of those weights in one
+// packed array; and the bands of each of the `warps` warps of the band phase,
+// contiguous and balanced by work (one multiply-add per weight and
+// kLfmBandCost more per band: the log, the floor and the store).
+constexpr int kLfmBandCost = 8;
+struct LfmPackedBank {
+  std::vector<int32_t> lo, cnt, off;
+  std::vector<float> w;
+  std::vector<int32_t> wband;  // warps + 1 boundaries, 0 .. n_mels
+};
+
+inline LfmPackedBank lfm_bank_pack(const std::vector<int32_t> &lo, const std::vector<float> &w, int n_mels,
+                                   int max_bins, int warps) {
+  LfmPackedBank P;
+  P.lo.assign(lo.begin(), lo.begin() + n_mels);
+  P.cnt.assign(n_mels, 0);
+  P.off.assign(n_mels, 0);
+  int64_t total = 0;
+  for (int b = 0; b < n_mels; ++b) {
+    int n = 0;
+    for (int q = 0; q < max_bins; ++q)
+      if (w[(size_t)b * max_bins + q] != 0.f) n = q + 1;
+    P.cnt[b] = n;
+    P.off[b] = (int32_t)P.w.size();
+    for (int q = 0; q < n; ++q) P.w.push_back(w[(size_t)b * max_bins + q]);
+    total += n + kLfmBandCost;
+  }
+  P.wband.assign(1, 0);
+  int64_t acc = 0;
+  for (int b = 0; b < n_mels; ++b) {
+    acc += P.cnt[b] + kLfmBandCost;
+    if ((int)P.wband.size() < warps && acc * warps >= total * (int64_t)P.wband.size()) P.wband.push_back(b + 1);
+  }
+  while ((int)P.wband.size() <= warps) P.wband.push_back(n_mels);
+  P.wband[warps] = n_mels;
+  return P;
+}
+
 }  // namespace ae
