@@ -151,30 +151,59 @@ cudaError_t launch_rowop(const ae_model *m, const RowArgs &r, cudaStream_t s) {
 
 // ------------------------------------------------------------------ light conv middle
 
-// w_dw is stored tap-major [kernel][hidden]. Thread t of a 256-thread CTA
-// owns channels 4t .. 4t+3 for kLcRows consecutive rows: its 5 x 4 taps and
-// 4 norm weights stay in registers, as channel pairs for the packed two-lane
-// FMA, and it loads its 8-byte slice of the rows (plus the 4 before them),
-// one coalesced load per row. The conv outputs of its rows stay in registers;
-// SiLU runs on the packed two-lane pipe.
-// The per-row sums of squares are reduced across the warp with a butterfly
-// that halves the rows at every step (after it, lanes 4r .. 4r+3 hold row r),
-// then across the CTA's 8 warps once for all rows.
+// w_dw is stored tap-major [kernel][hidden]. Persistent CTAs of 256 threads;
+// the work item is a tile of kLcRows consecutive rows. The rows a tile reads
+// (its own and the kKernel - 1 before them) are contiguous in memory, so one
+// bulk copy brings them into shared memory; each CTA keeps two tiles in
+// flight (double buffer, one mbarrier per buffer) and issues the copy of the
+// tile after next as soon as every thread has read the current buffer.
+// Thread t owns channels 4t .. 4t+3: its 5 x 4 taps and 4 norm weights stay
+// in registers as channel pairs for the packed two-lane FMA, and it adds each
+// buffered row into the (up to five) outputs that use it as the row arrives,
+// so no window of rows is held in registers. The per-row sums of squares are
+// reduced across the warp with a butterfly that halves the rows at every step
+// (after it, lanes 4r .. 4r+3 hold row r), then across the CTA's 8 warps once
+// for all rows; SiLU runs on the packed two-lane pipe.
 constexpr int kLcRows = 8;
 constexpr int kLcHalo = kKernel - 1;
 
-// Four CTAs per SM (64 registers): on the ragged batch 1.49 ms per step against about
-// 1.60 ms at three (a few bytes of spill in the bf16 form); the tower's short launches
-// lose about 4 %.
 template <typename ActT>
-__global__ void __launch_bounds__(256, 4) k_lconv(const ActT *__restrict__ gl, const float *__restrict__ w_dw,
+__host__ __device__ constexpr int lc_buf_bytes() {
+  return (kLcRows + kLcHalo) * kHidden * (int)sizeof(ActT);
+}
+
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void lds4(const float *p, float2 (&v)[2]) {
+  const float4 t = *reinterpret_cast<const float4 *>(p);
+  v[0] = make_float2(t.x, t.y);
+  v[1] = make_float2(t.z, t.w);
+}
+__device__ __forceinline__ void lds4(const bf16 *p, float2 (&v)[2]) {
+  const uint2 t = *reinterpret_cast<const uint2 *>(p);
+  v[0] = make_float2(bf16lo(t.x), bf16hi(t.x));
+  v[1] = make_float2(bf16lo(t.y), bf16hi(t.y));
+}
+
+template <typename ActT>
+__global__ void __launch_bounds__(256, 3) k_lconv(const ActT *__restrict__ gl, const float *__restrict__ w_dw,
                                                const float *__restrict__ w_norm, float lo, float hi,
-                                               ActT *__restrict__ out, const int32_t *__restrict__ pos, int64_t T) {
+                                               ActT *__restrict__ out, const int32_t *__restrict__ pos, int64_t T,
+                                               int64_t n_tiles, unsigned *status) {
   static_assert(kLcRows == 8, "the butterfly below reduces 8 rows");
+  constexpr int kBuf = lc_buf_bytes<ActT>();
+  constexpr int kRowBytes = kHidden * (int)sizeof(ActT);
+  extern __shared__ __align__(128) uint8_t lc_smem[];
+  __shared__ uint64_t bar[2];
   __shared__ float s_ss[8][kLcRows];
   __shared__ float s_inv[kLcRows];
+  __shared__ int s_pos[2][kLcRows];  // positions of the buffered tiles' rows in their clips
   const int ch = 4 * threadIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t t0 = (int64_t)blockIdx.x * kLcRows;
   float2 w[kKernel][2], wn[2];
 #pragma unroll
   for (int k = 0; k < kKernel; ++k) {
@@ -189,90 +218,141 @@ __global__ void __launch_bounds__(256, 4) k_lconv(const ActT *__restrict__ gl, c
     wn[0] = make_float2(t[0], t[1]);
     wn[1] = make_float2(t[2], t[3]);
   }
-  float2 x[kLcRows + kLcHalo][2];
-#pragma unroll
-  for (int r = 0; r < kLcRows + kLcHalo; ++r) {
-    const int64_t tok = t0 - kLcHalo + r;
-    float t[4] = {0.f, 0.f, 0.f, 0.f};
-    if (tok >= 0 && tok < T) load4(gl + tok * kHidden + ch, t);
-    x[r][0] = make_float2(t[0], t[1]);
-    x[r][1] = make_float2(t[2], t[3]);
+  if (threadIdx.x == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    fence_mbar_init();
   }
-  float2 c[kLcRows][2];
-  float ss[kLcRows];
+  const int64_t my = (int64_t)blockIdx.x < n_tiles ? (n_tiles - 1 - (int64_t)blockIdx.x) / gridDim.x + 1 : 0;
+  // row r of item k: its position, read by thread r two items ahead so that
+  // no item waits on a global load
+  auto pos_of = [&](int64_t k, int r) {
+    const int64_t tok = ((int64_t)blockIdx.x + k * gridDim.x) * kLcRows + r;
+    return k < my && tok < T ? pos[tok] : 0;
+  };
+  if (threadIdx.x < kLcRows) {
+    s_pos[0][threadIdx.x] = pos_of(0, threadIdx.x);
+    s_pos[1][threadIdx.x] = pos_of(1, threadIdx.x);
+  }
+  __syncthreads();
+  // buffer row i of item k holds token t0 - kLcHalo + i; tokens before 0 or from T on are not copied
+  auto issue = [&](int64_t k) {
+    const int64_t t0 = ((int64_t)blockIdx.x + k * gridDim.x) * kLcRows;
+    const int64_t a = t0 - kLcHalo > 0 ? t0 - kLcHalo : 0, b = t0 + kLcRows < T ? t0 + kLcRows : T;
+    const uint32_t bytes = (uint32_t)((b - a) * kRowBytes);
+    mbar_arrive_expect_tx(&bar[k & 1], bytes);
+    bulk_load(lc_smem + (k & 1) * kBuf + (a - (t0 - kLcHalo)) * kRowBytes, gl + a * kHidden, bytes, &bar[k & 1]);
+  };
+  if (threadIdx.x == 0) {
+    if (my > 0) issue(0);
+    if (my > 1) issue(1);
+  }
+  for (int64_t k = 0; k < my; ++k) {
+    const int64_t t0 = ((int64_t)blockIdx.x + k * gridDim.x) * kLcRows;
+    const int pn = threadIdx.x < kLcRows ? pos_of(k + 2, threadIdx.x) : 0;  // stored at the end of this item
+    if (!__syncthreads_and(mbar_wait(&bar[k & 1], (uint32_t)((k >> 1) & 1)))) {
+      if (threadIdx.x == 0) atomicOr(status, kStatusWaitTimeout);
+      break;
+    }
+    int p[kLcRows];  // position of each row in its clip (taps never reach before the clip start)
 #pragma unroll
-  for (int r = 0; r < kLcRows; ++r) {
-    const int64_t tok = t0 + r;
-    const int p = tok < T ? pos[tok] : 0;
-    c[r][0] = c[r][1] = make_float2(0.f, 0.f);
+    for (int r = 0; r < kLcRows; ++r) p[r] = s_pos[k & 1][r];
+    const ActT *sx = reinterpret_cast<const ActT *>(lc_smem + (k & 1) * kBuf) + ch;
+    float2 c[kLcRows][2];
 #pragma unroll
-    for (int k = 0; k < kKernel; ++k) {
-      const int back = kKernel - 1 - k;
-      if (back <= p) {
-        ffma2(c[r][0], w[k][0], x[r + kLcHalo - back][0]);
-        ffma2(c[r][1], w[k][1], x[r + kLcHalo - back][1]);
+    for (int r = 0; r < kLcRows; ++r) c[r][0] = c[r][1] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < kLcRows + kLcHalo; ++i) {  // buffer row i feeds outputs r = i - 4 .. i with tap i - r
+      float2 x[2];
+      lds4(sx + i * kHidden, x);
+#pragma unroll
+      for (int r = (i - kLcHalo > 0 ? i - kLcHalo : 0); r <= (i < kLcRows - 1 ? i : kLcRows - 1); ++r) {
+        if (r + kLcHalo - i <= p[r]) {
+          ffma2(c[r][0], w[i - r][0], x[0]);
+          ffma2(c[r][1], w[i - r][1], x[1]);
+        }
       }
     }
-    float2 q = make_float2(0.f, 0.f);
-    ffma2(q, c[r][0], c[r][0]);
-    ffma2(q, c[r][1], c[r][1]);
-    ss[r] = q.x + q.y;
-  }
-  // butterfly reduce-scatter: 8 rows -> 4 -> 2 -> 1 per lane, then a sum over the 4 lanes
-  {
-    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
-    float v4[4], v2[2];
+    float ss[kLcRows];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float mine = b4 ? ss[i + 4] : ss[i], other = b4 ? ss[i] : ss[i + 4];
-      v4[i] = mine + __shfl_xor_sync(0xffffffffu, other, 16);
+    for (int r = 0; r < kLcRows; ++r) {
+      float2 q = make_float2(0.f, 0.f);
+      ffma2(q, c[r][0], c[r][0]);
+      ffma2(q, c[r][1], c[r][1]);
+      ss[r] = q.x + q.y;
     }
+    // butterfly reduce-scatter: 8 rows -> 4 -> 2 -> 1 per lane, then a sum over the 4 lanes
+    {
+      const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+      float v4[4], v2[2];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const float mine = b3 ? v4[i + 2] : v4[i], other = b3 ? v4[i] : v4[i + 2];
-      v2[i] = mine + __shfl_xor_sync(0xffffffffu, other, 8);
+      for (int i = 0; i < 4; ++i) {
+        const float mine = b4 ? ss[i + 4] : ss[i], other = b4 ? ss[i] : ss[i + 4];
+        v4[i] = mine + __shfl_xor_sync(0xffffffffu, other, 16);
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const float mine = b3 ? v4[i + 2] : v4[i], other = b3 ? v4[i] : v4[i + 2];
+        v2[i] = mine + __shfl_xor_sync(0xffffffffu, other, 8);
+      }
+      float v = (b2 ? v2[1] : v2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? v2[0] : v2[1], 4);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      if ((lane & 3) == 0) s_ss[warp][lane >> 2] = v;  // row (lane >> 2): bits 4, 3, 2 of the lane
     }
-    float v = (b2 ? v2[1] : v2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? v2[0] : v2[1], 4);
-    v += __shfl_xor_sync(0xffffffffu, v, 2);
-    v += __shfl_xor_sync(0xffffffffu, v, 1);
-    if ((lane & 3) == 0) s_ss[warp][lane >> 2] = v;  // row (lane >> 2): bits 4, 3, 2 of the lane
-  }
-  __syncthreads();
-  if (threadIdx.x < kLcRows) {
-    float sum = 0.f;
+    __syncthreads();  // sums in; every thread is done with this buffer
+    if (threadIdx.x == 0 && k + 2 < my) issue(k + 2);
+    if (threadIdx.x < kLcRows) {
+      float sum = 0.f;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) sum += s_ss[q][threadIdx.x];
-    s_inv[threadIdx.x] = rsqrtf(sum * (1.0f / kHidden) + kEps);
-  }
-  __syncthreads();
-#pragma unroll
-  for (int r = 0; r < kLcRows; ++r) {
-    const int64_t tok = t0 + r;
-    if (tok >= T) break;
-    const float2 inv = make_float2(s_inv[r], s_inv[r]);
-    float v[4];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {  // silu(y) = y / (1 + 2^(-y log2 e)), two channels per packed op
-      const float2 y = __fmul2_rn(c[r][h], __fmul2_rn(inv, wn[h]));
-      const float2 e = __fmul2_rn(y, make_float2(-1.4426950408889634f, -1.4426950408889634f));
-      const float2 d = __fadd2_rn(make_float2(ex2_approx(e.x), ex2_approx(e.y)), make_float2(1.0f, 1.0f));
-      const float2 sl = __fmul2_rn(y, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
-      v[2 * h] = clampf(sl.x, lo, hi);
-      v[2 * h + 1] = clampf(sl.y, lo, hi);
+      for (int q = 0; q < 8; ++q) sum += s_ss[q][threadIdx.x];
+      s_inv[threadIdx.x] = rsqrtf(sum * (1.0f / kHidden) + kEps);
     }
-    store4(out + tok * kHidden + ch, v);
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < kLcRows; ++r) {
+      const int64_t tok = t0 + r;
+      if (tok >= T) break;
+      const float2 inv = make_float2(s_inv[r], s_inv[r]);
+      float v[4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {  // silu(y) = y / (1 + 2^(-y log2 e)), two channels per packed op
+        const float2 y = __fmul2_rn(c[r][h], __fmul2_rn(inv, wn[h]));
+        const float2 e = __fmul2_rn(y, make_float2(-1.4426950408889634f, -1.4426950408889634f));
+        const float2 d = __fadd2_rn(make_float2(ex2_approx(e.x), ex2_approx(e.y)), make_float2(1.0f, 1.0f));
+        const float2 sl = __fmul2_rn(y, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
+        v[2 * h] = clampf(sl.x, lo, hi);
+        v[2 * h + 1] = clampf(sl.y, lo, hi);
+      }
+      store4(out + tok * kHidden + ch, v);
+    }
+    if (threadIdx.x < kLcRows) s_pos[k & 1][threadIdx.x] = pn;  // every thread read this item's after two barriers
   }
 }
 
 cudaError_t launch_lconv(const ae_model *m, const void *gl, const float *w_dw, const float *w_norm, float lo,
                          float hi, void *out, const int32_t *pos, int64_t T, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  const unsigned grid = (unsigned)((T + kLcRows - 1) / kLcRows);
-  if (m->dtype != AE_F32)
-    return launch_k(k_lconv<bf16>, dim3(grid), dim3(256), 0, s, static_cast<const bf16 *>(gl), w_dw, w_norm, lo, hi,
-                    static_cast<bf16 *>(out), pos, T);
-  return launch_k(k_lconv<float>, dim3(grid), dim3(256), 0, s, static_cast<const float *>(gl), w_dw, w_norm, lo, hi,
-                  static_cast<float *>(out), pos, T);
+  if ((reinterpret_cast<uintptr_t>(gl) & 15) != 0) return cudaErrorMisalignedAddress;  // bulk copies
+  const int64_t tiles = (T + kLcRows - 1) / kLcRows;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // resident CTAs per SM: three by registers; the float32 form's buffers allow two
+  const int64_t slots = (m->dtype != AE_F32 ? 3 : 2) * (int64_t)sms;
+  const unsigned grid = (unsigned)(tiles < slots ? tiles : slots);
+  if (m->dtype != AE_F32) {
+    static std::atomic<uint64_t> attr{0};
+    constexpr size_t smem = 2 * lc_buf_bytes<bf16>();
+    if (const cudaError_t e = smem_attr(k_lconv<bf16>, smem, attr)) return e;
+    return launch_k(k_lconv<bf16>, dim3(grid), dim3(256), smem, s, static_cast<const bf16 *>(gl), w_dw, w_norm, lo,
+                    hi, static_cast<bf16 *>(out), pos, T, tiles, device_status_word());
+  }
+  static std::atomic<uint64_t> attr{0};
+  constexpr size_t smem = 2 * lc_buf_bytes<float>();
+  if (const cudaError_t e = smem_attr(k_lconv<float>, smem, attr)) return e;
+  return launch_k(k_lconv<float>, dim3(grid), dim3(256), smem, s, static_cast<const float *>(gl), w_dw, w_norm, lo,
+                  hi, static_cast<float *>(out), pos, T, tiles, device_status_word());
 }
 
 // ------------------------------------------------------------------ tables
