@@ -295,12 +295,14 @@ constexpr int kLencHeads = 8;     // heads of 64
 constexpr int kLencStemCh = 256;  // stem channels
 constexpr int kLencMaxTok = 4096; // rows after the stem per clip
 constexpr int kLencMaxConvK = 33; // depthwise conv taps
+constexpr int kLencStemRun = 16;  // rows after the first two stem convolutions per work item
 struct LencTablesDev {
   int n_clips;
   const int32_t *frame_off;  // [B + 1] mel frames
   const int32_t *s2_off;     // [B + 1] rows after the first two stem convolutions
   const int32_t *tok_off;    // [B + 1] rows after the stem (tokens)
   const int32_t *qblk_off;   // [B + 1] 128-token query blocks
+  const int32_t *s2item_off; // [B + 1] work items of kLencStemRun such rows (the first stem kernel)
 };
 struct LencLnArgs {
   float *x; int64_t rows; float eps;
@@ -308,8 +310,8 @@ struct LencLnArgs {
   const float *w2, *b2;  // optional second LayerNorm for the operand
   bf16 *a;               // optional bf16 operand out
 };
-cudaError_t launch_lenc_stem01(const float *mel, const float *w0, const float *b0, const float *w1, const float *b1,
-                               void *y2, const LencTablesDev &t, int64_t s2_rows, cudaStream_t s);
+cudaError_t launch_lenc_stem01(const float *mel, const void *w0b, const float *b0, const float *w1, const float *b1,
+                               void *y2, const LencTablesDev &t, int64_t s2_items, cudaStream_t s);
 cudaError_t launch_lenc_dw2(const void *y, const float *w, const float *b, void *out, const LencTablesDev &t,
                             int64_t tokens, cudaStream_t s);
 cudaError_t launch_lenc_ln(const LencLnArgs &r, cudaStream_t s);

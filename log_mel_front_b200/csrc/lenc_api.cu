@@ -22,7 +22,8 @@
 struct ae_lenc {
   ae_lenc_config cfg;
   std::vector<void *> allocs;
-  float *w0, *b0, *w1, *b1, *b2, *w3, *b3, *b4, *pre_b;
+  float *b0, *w1, *b1, *b2, *w3, *b3, *b4, *pre_b;
+  void *w0b;  // the first stem convolution's taps as the tensor-core B operand (split in bf16 parts)
   void *w2, *w4, *pre_w;
   CUtensorMap tm_w2, tm_w4, tm_pre;
   struct Block {
@@ -57,6 +58,13 @@ uint16_t to_bf16(float f) {
   if ((u & 0x7fffffffu) > 0x7f800000u) return 0x7fc0;
   u += 0x7fffu + ((u >> 16) & 1u);
   return (uint16_t)(u >> 16);
+}
+
+float from_bf16(uint16_t b) {
+  const uint32_t u = (uint32_t)b << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
 }
 
 size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -119,9 +127,9 @@ bool cfg_ok(const ae_lenc_config *c, std::string *why) {
 // Per-call tables: frame, stem-row, token and query-block offsets.
 struct LencTables {
   int n_clips = 0;
-  int64_t frames = 0, s2_rows = 0, tokens = 0, qblk = 0;
+  int64_t frames = 0, s2_rows = 0, tokens = 0, qblk = 0, s2_items = 0;
   int t_max = 0;
-  std::vector<int32_t> frame_off, s2_off, tok_off, qblk_off;
+  std::vector<int32_t> frame_off, s2_off, tok_off, qblk_off, s2item_off;
 };
 
 // kind 0: frame offsets; kind 1: token offsets (the block call)
@@ -135,6 +143,7 @@ ae_status lenc_tables(const int64_t *off, int n, int kind, LencTables &T) {
   T.s2_off.assign(n + 1, 0);
   T.tok_off.assign(n + 1, 0);
   T.qblk_off.assign(n + 1, 0);
+  T.s2item_off.assign(n + 1, 0);
   for (int c = 0; c < n; ++c) {
     const int64_t len = off[c + 1] - off[c];
     if (len < 0) return lfail(AE_EINVAL, "offsets are not non-decreasing at clip " + std::to_string(c));
@@ -144,6 +153,7 @@ ae_status lenc_tables(const int64_t *off, int n, int kind, LencTables &T) {
       return lfail(AE_EUNSUPPORTED, "clip " + std::to_string(c) + " has more than 4096 rows after the stem");
     T.frames += F;
     T.s2_rows += half_up(half_up(F));
+    T.s2_items += (half_up(half_up(F)) + kLencStemRun - 1) / kLencStemRun;
     T.tokens += t;
     T.qblk += (t + 127) / 128;
     if (T.frames > 64000000 || T.s2_rows > 4000000 || T.tokens > 2000000)
@@ -153,6 +163,7 @@ ae_status lenc_tables(const int64_t *off, int n, int kind, LencTables &T) {
     T.s2_off[c + 1] = (int32_t)T.s2_rows;
     T.tok_off[c + 1] = (int32_t)T.tokens;
     T.qblk_off[c + 1] = (int32_t)T.qblk;
+    T.s2item_off[c + 1] = (int32_t)T.s2_items;
   }
   return AE_OK;
 }
@@ -170,7 +181,7 @@ LencLayout lenc_layout(const ae_lenc_config &c, const LencTables &T) {
     return o;
   };
   const size_t B1 = (size_t)T.n_clips + 1;
-  L.tables = put(4 * B1 * 4);
+  L.tables = put(5 * B1 * 4);
   L.x = put((size_t)T.tokens * kLencEmbd * 4);
   const size_t u0 = off;  // the stem's buffers and the blocks' share this region
   L.y2 = put((size_t)T.s2_rows * 32 * kLencStemCh * 2);
@@ -194,11 +205,12 @@ LencLayout lenc_layout(const ae_lenc_config &c, const LencTables &T) {
 
 ae_status upload_tables(const LencTables &T, void *ws, const LencLayout &L, LencTablesDev *td, cudaStream_t s) {
   const size_t B1 = (size_t)T.n_clips + 1;
-  std::vector<int32_t> h(4 * B1);
+  std::vector<int32_t> h(5 * B1);
   std::copy(T.frame_off.begin(), T.frame_off.end(), h.begin());
   std::copy(T.s2_off.begin(), T.s2_off.end(), h.begin() + B1);
   std::copy(T.tok_off.begin(), T.tok_off.end(), h.begin() + 2 * B1);
   std::copy(T.qblk_off.begin(), T.qblk_off.end(), h.begin() + 3 * B1);
+  std::copy(T.s2item_off.begin(), T.s2item_off.end(), h.begin() + 4 * B1);
   int32_t *d = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + L.tables);
   const cudaError_t e = profiled_f(AE_K_TABLES, 0.0, 0.0, s, [&] { return launch_upload_bytes(h.data(), h.size() * 4, d, s); });
   if (e != cudaSuccess) return lcuda(e, "clip tables");
@@ -207,6 +219,7 @@ ae_status upload_tables(const LencTables &T, void *ws, const LencLayout &L, Lenc
   td->s2_off = d + B1;
   td->tok_off = d + 2 * B1;
   td->qblk_off = d + 3 * B1;
+  td->s2item_off = d + 4 * B1;
   return AE_OK;
 }
 
@@ -268,7 +281,7 @@ cudaError_t run_stem(const ae_lenc *m, const float *mel, const Bufs &b, cudaStre
   const int C = kLencStemCh;
   LE_TRY(profiled_f(AE_K_LENC_ROW, 2.0 * 9 * 10 * C * 32.0 * T.s2_rows,
                     4.0 * T.frames * kLencMels + 2.0 * T.s2_rows * 32 * C, s,
-                    [&] { return launch_lenc_stem01(mel, m->w0, m->b0, m->w1, m->b1, y2, b.td, T.s2_rows, s); }));
+                    [&] { return launch_lenc_stem01(mel, m->w0b, m->b0, m->w1, m->b1, y2, b.td, T.s2_items, s); }));
   EpiArgs e = epi(y2b, C, m->b2);
   e.lo = 0.f;  // ReLU
   LE_TRY(proj(y2, T.s2_rows * 32, C, m->tm_w2, C, EPI_BIAS_BF16, e, s));
@@ -415,7 +428,22 @@ ae_status ae_lenc_create(const ae_lenc_config *cfg, const ae_lenc_host_weights *
   ae_lenc *m = new ae_lenc();
   m->cfg = *cfg;
   Up up{m};
-  m->w0 = up.f32(w->stem_w[0], (size_t)C * 9);
+  {
+    // channel c's row of 64 bf16: (w_hi, w_lo, w_hi) of its 9 taps, zeros after, against
+    // the patch row (p_hi, p_hi, p_lo): p_hi w_hi + p_hi w_lo + p_lo w_hi, about 16 bits
+    std::vector<uint16_t> wb((size_t)C * 64, 0);
+    for (int c = 0; c < C; ++c)
+      for (int k = 0; k < 9; ++k) {
+        const float v = w->stem_w[0][(size_t)c * 9 + k];
+        const uint16_t hi = to_bf16(v);
+        wb[(size_t)c * 64 + k] = hi;
+        wb[(size_t)c * 64 + 9 + k] = to_bf16(v - from_bf16(hi));
+        wb[(size_t)c * 64 + 18 + k] = hi;
+      }
+    uint16_t *d = up.alloc<uint16_t>(wb.size());
+    if (d && cudaMemcpy(d, wb.data(), wb.size() * 2, cudaMemcpyHostToDevice) != cudaSuccess) up.ok = false;
+    m->w0b = d;
+  }
   m->b0 = up.f32(w->stem_b[0], C);
   m->w1 = up.f32(w->stem_w[1], (size_t)C * 9);
   m->b1 = up.f32(w->stem_b[1], C);

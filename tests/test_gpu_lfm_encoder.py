@@ -87,6 +87,19 @@ def test_stem_matches_oracle(m2, w2):
     assert_bf16(g, o, "LFM2A stem")
 
 
+def test_stem_work_item_edges(m2, w2):
+    """The first stem kernel takes runs of 16 rows of its output per work item:
+    clips of 1, 2, 63, 64, 65, 128 and 129 frames put the last run's edge on,
+    before and after a multiple of 16 rows (and one clip is a single run)."""
+    lens = [100, 160, 9920, 10080, 10240, 20320, 20480]
+    mels = _mels(lens, seed=43)
+    assert [x.shape[0] for x in mels] == [1, 2, 63, 64, 65, 128, 129]
+    g, toks = _gpu_stem(m2, mels)
+    o = np.concatenate([E.stem(x.astype(np.float64), w2) for x in mels])
+    assert g.shape == o.shape == (sum(toks), 512)
+    assert_bf16(g, o, "LFM2A stem at work-item edges")
+
+
 @pytest.mark.parametrize("toks", [[1], [5, 128, 129, 3], [300, 7, 256]])
 def test_block_matches_oracle(m2, w2, toks):
     """One block from the same float32 input: the attention runs over whole clips
