@@ -85,6 +85,13 @@ __device__ __forceinline__ void xa_tmem_st32(uint32_t taddr, const uint32_t (&r)
       "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
+// 2^x with the hardware's base-2 exponential (0 for x = -inf); the
+// probabilities it gives are rounded to bf16 for the P V product
+__device__ __forceinline__ float xa_ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ void xa_tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __global__ void __launch_bounds__(XA_THREADS, 1)
@@ -295,10 +302,15 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
         tmem_ld32(trow + COL_S + 32 * q, a);
         tmem_ld_wait();
         __syncwarp();
+        if (j0 + 32 * qq + 32 <= t_c) {  // every key of the chunk lies in the clip
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const int j = j0 + 32 * qq + x;
-          z[32 * qq + x] = j < t_c ? (__uint_as_float(a[x]) + my[31 - lane + x]) * kScale : -INFINITY;
+          for (int x = 0; x < 32; ++x) z[32 * qq + x] = (__uint_as_float(a[x]) + my[31 - lane + x]) * kScale;
+        } else {
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            const int j = j0 + 32 * qq + x;
+            z[32 * qq + x] = j < t_c ? (__uint_as_float(a[x]) + my[31 - lane + x]) * kScale : -INFINITY;
+          }
         }
         __syncwarp();
       }
@@ -311,7 +323,7 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
       if (!pair_sync(&xm[qw], kb & 1)) { ok = false; break; }
       // finite: every block holds a key of the clip, in one half or the other
       const float m_new = fmaxf(m_run, fmaxf(bm, xmax[((kb & 1) * 2 + (kh ^ 1)) * 128 + li]));
-      const float alpha = exp2f(m_run - m_new);  // 0 on the first block
+      const float alpha = xa_ex2(m_run - m_new);  // 0 on the first block
       // the previous block's P V is done: the probabilities' buffer is free and
       // the accumulator holds every earlier block
       if (kb > 0 && !__all_sync(0xffffffffu, mbar_wait(o_full, (kb - 1) & 1))) { ok = false; break; }
@@ -320,7 +332,7 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
       uint32_t pw[32];  // keys 64 kh .. 64 kh + 63 as bf16 pairs: tensor-memory columns COL_P + 32 kh ..
 #pragma unroll
       for (int x = 0; x < 32; ++x) {
-        const float p0 = exp2f(z[2 * x] - m_new), p1 = exp2f(z[2 * x + 1] - m_new);
+        const float p0 = xa_ex2(z[2 * x] - m_new), p1 = xa_ex2(z[2 * x + 1] - m_new);
         ls += p0 + p1;
         pw[x] = pack_bf16(p0, p1);
       }
