@@ -207,14 +207,14 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
     constexpr uint32_t idesc_t = idesc_bf16_f32(XA_Q, 2 * XA_K);
     constexpr uint32_t idesc_o = idesc_bf16_f32_bmn(XA_Q, XA_HD);
     const uint32_t aqu = smem_u32(sQu), aqv = smem_u32(sQv), av = smem_u32(sV);
-    bool ok = mbar_wait(q_ready, 0);
-    for (int kb = 0; kb < n_kb && ok; ++kb) {
+    // the score products of block kb + 1 go out as soon as the row threads have
+    // read block kb's, so they run during block kb's softmax; P V of block kb
+    // follows once its probabilities are in tensor memory
+    auto scores = [&](int kb) -> bool {
       const int st = kb & 1;
       const uint32_t ak = smem_u32(smem + OFF_K + st * XA_TILE), apb = smem_u32(smem + OFF_PB + st * 2 * XA_TILE);
-      if (!mbar_wait(&kp_full[st], (kb >> 1) & 1) || (kb > 0 && !mbar_wait(s_free, (kb - 1) & 1)) || *abort_flag) {
-        ok = false;
-        break;
-      }
+      if (!mbar_wait(&kp_full[st], (kb >> 1) & 1) || (kb > 0 && !mbar_wait(s_free, (kb - 1) & 1)) || *abort_flag)
+        return false;
       tc_fence_after();
 #pragma unroll
       for (int k = 0; k < XA_HD / 16; ++k)
@@ -224,6 +224,14 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
         tc_mma_bf16(tmem + COL_T, sw128_desc(aqv + k * 32), sw128_desc(apb + k * 32), idesc_t, k > 0 ? 1u : 0u);
       tc_commit(&kp_free[st]);
       tc_commit(s_full);
+      return true;
+    };
+    bool ok = mbar_wait(q_ready, 0) && (n_kb == 0 || scores(0));
+    for (int kb = 0; kb < n_kb && ok; ++kb) {
+      if (kb + 1 < n_kb && !scores(kb + 1)) {
+        ok = false;
+        break;
+      }
       if (!mbar_wait(p_full, kb & 1) || !mbar_wait(v_full, kb & 1) || *abort_flag) {
         ok = false;
         break;
