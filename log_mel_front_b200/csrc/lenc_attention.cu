@@ -115,8 +115,17 @@ __global__ void __launch_bounds__(XA_THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // item -> (clip, query block, head)
   const int head = blockIdx.x % kLencHeads, qitem = blockIdx.x / kLencHeads;
+  // the last clip whose first query block is <= qitem: for up to 1024 clips each
+  // warp counts the offsets <= qitem with independent loads (one round trip;
+  // the offsets are non-decreasing), else a binary search
   int c = 0;
-  {
+  if (n_clips <= 1024) {
+    int cnt = 0;
+    for (int i = lane; i < n_clips; i += 32) cnt += qblk_off[i] <= qitem ? 1 : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    c = cnt - 1;
+  } else {
     int lo = 0, hi = n_clips;
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
