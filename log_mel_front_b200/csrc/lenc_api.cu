@@ -252,8 +252,10 @@ cudaError_t proj(const void *x, int64_t M, int K, const CUtensorMap &tm, int N, 
   return profiled_f(AE_K_LENC_GEMM, fl, by, s, [&] { return gemm_bf16(x, M, K, tm, N, mode, ep, s); });
 }
 
+// x's rows through LayerNorm(w1, b1), written back to x if write_x; then the
+// bf16 operand a of those rows, or of LayerNorm(w2, b2) of them when w2 is given
 cudaError_t ln(float *x, int64_t rows, float eps, const float *w1, const float *b1, bool write_x, bf16 *a,
-               cudaStream_t s) {
+               cudaStream_t s, const float *w2 = nullptr, const float *b2 = nullptr) {
   LencLnArgs r;
   std::memset(&r, 0, sizeof(r));
   r.x = x;
@@ -263,6 +265,8 @@ cudaError_t ln(float *x, int64_t rows, float eps, const float *w1, const float *
   r.b1 = b1;
   r.write_x = write_x ? 1 : 0;
   r.a = a;
+  r.w2 = w2;
+  r.b2 = b2;
   const double by = (double)rows * kLencEmbd * (4.0 + (write_x ? 4.0 : 0.0) + (a ? 2.0 : 0.0));
   return profiled_f(AE_K_LENC_ROW, 0.0, by, s, [&] { return launch_lenc_ln(r, s); });
 }
@@ -305,7 +309,12 @@ cudaError_t run_positions(const ae_lenc *m, const Bufs &b, cudaStream_t s) {
               epi(b.ws + b.L.P, (int64_t)m->cfg.n_layers * kLencEmbd, nullptr), s);
 }
 
-cudaError_t run_block(const ae_lenc *m, int li, const Bufs &b, cudaStream_t s) {
+// One block. With `first_ready` the operand of the first FFN's LayerNorm is
+// already in a (the previous block's closing pass made it); with next_w the
+// closing LayerNorm also makes the operand of the LayerNorm that follows (the
+// next block's first, or the adapter's), in the same pass over the rows.
+cudaError_t run_block(const ae_lenc *m, int li, const Bufs &b, cudaStream_t s, bool first_ready = false,
+                      const float *next_w = nullptr, const float *next_b = nullptr) {
   const ae_lenc::Block &B = m->blocks[li];
   const LencTables &T = *b.T;
   const int64_t n = T.tokens;
@@ -314,14 +323,14 @@ cudaError_t run_block(const ae_lenc *m, int li, const Bufs &b, cudaStream_t s) {
   bf16 *a = reinterpret_cast<bf16 *>(b.ws + b.L.a);
   void *big = b.ws + b.L.big, *qkv = b.ws + b.L.qkv, *o = b.ws + b.L.o, *cb = b.ws + b.L.cbuf;
   auto ffn = [&](const float *nw, const float *nb, const CUtensorMap &up, const float *ub, const CUtensorMap &down,
-                 const float *db) -> cudaError_t {
-    LE_TRY(ln(b.x, n, eps, nw, nb, false, a, s));
+                 const float *db, bool ready) -> cudaError_t {
+    if (!ready) LE_TRY(ln(b.x, n, eps, nw, nb, false, a, s));
     LE_TRY(proj(a, n, D, up, F, EPI_BIAS_SILU, epi(big, F, ub), s));
     EpiArgs e = epi(b.x, D, db);
     e.alpha = 0.5f;  // macaron half weight
     return proj(big, n, F, down, D, EPI_BIAS_ADD_F32, e, s);
   };
-  LE_TRY(ffn(B.f1_nw, B.f1_nb, B.tm_f1_up, B.f1_ub, B.tm_f1_down, B.f1_db));
+  LE_TRY(ffn(B.f1_nw, B.f1_nb, B.tm_f1_up, B.f1_ub, B.tm_f1_down, B.f1_db, first_ready));
   // attention
   LE_TRY(ln(b.x, n, eps, B.ln1_w, B.ln1_b, false, a, s));
   LE_TRY(proj(a, n, D, B.tm_qkv, 3 * D, EPI_BIAS_BF16, epi(qkv, 3 * D, B.qkv_b), s));
@@ -345,15 +354,15 @@ cudaError_t run_block(const ae_lenc *m, int li, const Bufs &b, cudaStream_t s) {
     return launch_lenc_dwconv(big, B.dw_w, B.dw_b, B.cn_w, B.cn_b, m->cfg.conv_k, cb, b.td.tok_off, T.n_clips, n, s);
   }));
   LE_TRY(proj(cb, n, D, B.tm_pw2, D, EPI_BIAS_ADD_F32, epi(b.x, D, B.pw2_b), s));
-  LE_TRY(ffn(B.f2_nw, B.f2_nb, B.tm_f2_up, B.f2_ub, B.tm_f2_down, B.f2_db));
-  return ln(b.x, n, eps, B.ln2_w, B.ln2_b, true, nullptr, s);
+  LE_TRY(ffn(B.f2_nw, B.f2_nb, B.tm_f2_up, B.f2_ub, B.tm_f2_down, B.f2_db, false));
+  return ln(b.x, n, eps, B.ln2_w, B.ln2_b, true, next_w ? a : nullptr, s, next_w, next_b);
 }
 
-cudaError_t run_adapter(const ae_lenc *m, const Bufs &b, float *out, cudaStream_t s) {
+cudaError_t run_adapter(const ae_lenc *m, const Bufs &b, float *out, cudaStream_t s, bool norm_ready = false) {
   const int64_t n = b.T->tokens;
   bf16 *a = reinterpret_cast<bf16 *>(b.ws + b.L.a);
   void *big = b.ws + b.L.big;
-  LE_TRY(ln(b.x, n, m->cfg.eps, m->ad_nw, m->ad_nb, false, a, s));
+  if (!norm_ready) LE_TRY(ln(b.x, n, m->cfg.eps, m->ad_nw, m->ad_nb, false, a, s));
   LE_TRY(proj(a, n, kLencEmbd, m->tm_ad_up, m->cfg.adapter_ff, EPI_BIAS_GELU, epi(big, m->cfg.adapter_ff, m->ad_ub),
               s));
   return proj(big, n, m->cfg.adapter_ff, m->tm_ad_down, m->cfg.llm_hidden, EPI_F32,
@@ -588,8 +597,13 @@ ae_status ae_lenc_encode(const ae_lenc *m, const float *d_mel, const int64_t *h_
   const cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = run_stem(m, d_mel, b, s);
   if (e == cudaSuccess) e = run_positions(m, b, s);
-  for (int l = 0; l < m->cfg.n_layers && e == cudaSuccess; ++l) e = run_block(m, l, b, s);
-  if (e == cudaSuccess) e = run_adapter(m, b, d_out, s);
+  const int L = m->cfg.n_layers;
+  for (int l = 0; l < L && e == cudaSuccess; ++l) {
+    const bool last = l + 1 == L;
+    e = run_block(m, l, b, s, l > 0, last ? m->ad_nw : m->blocks[l + 1].f1_nw,
+                  last ? m->ad_nb : m->blocks[l + 1].f1_nb);
+  }
+  if (e == cudaSuccess) e = run_adapter(m, b, d_out, s, L > 0);
   return e == cudaSuccess ? AE_OK : lcuda(e, "ae_lenc_encode");
 }
 
