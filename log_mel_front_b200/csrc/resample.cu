@@ -150,27 +150,29 @@ __device__ __forceinline__ void rs_partial(const RsArgs &a, const RsTile &r, con
   constexpr int V = U / 4;
   const int64_t m0 = (r.q0 + ql) * a.D + a.lo[T];
   const float *xr = span + (m0 - r.base);
-  float e[U], d[U];
+  // two outputs' taps against the same input sample per packed two-lane FMA
+  // (each lane a fused multiply-add, as fmaf)
+  float2 e[U / 2], d[U / 2];
 #pragma unroll
-  for (int k = 0; k < U; ++k) e[k] = d[k] = 0.f;
+  for (int k = 0; k < U / 2; ++k) e[k] = d[k] = make_float2(0.f, 0.f);
 #pragma unroll 4
   for (int i = i0; i < i1; i += 2) {
     const float x0 = xr[i], x1 = xr[i + 1];
+    const float2 xx0 = make_float2(x0, x0), xx1 = make_float2(x1, x1);
 #pragma unroll
     for (int j = 0; j < V; ++j) {
       const float4 w0 = cT[i * V + j], w1 = cT[(i + 1) * V + j];
-      e[4 * j] = fmaf(w0.x, x0, e[4 * j]);
-      e[4 * j + 1] = fmaf(w0.y, x0, e[4 * j + 1]);
-      e[4 * j + 2] = fmaf(w0.z, x0, e[4 * j + 2]);
-      e[4 * j + 3] = fmaf(w0.w, x0, e[4 * j + 3]);
-      d[4 * j] = fmaf(w1.x, x1, d[4 * j]);
-      d[4 * j + 1] = fmaf(w1.y, x1, d[4 * j + 1]);
-      d[4 * j + 2] = fmaf(w1.z, x1, d[4 * j + 2]);
-      d[4 * j + 3] = fmaf(w1.w, x1, d[4 * j + 3]);
+      e[2 * j] = __ffma2_rn(make_float2(w0.x, w0.y), xx0, e[2 * j]);
+      e[2 * j + 1] = __ffma2_rn(make_float2(w0.z, w0.w), xx0, e[2 * j + 1]);
+      d[2 * j] = __ffma2_rn(make_float2(w1.x, w1.y), xx1, d[2 * j]);
+      d[2 * j + 1] = __ffma2_rn(make_float2(w1.z, w1.w), xx1, d[2 * j + 1]);
     }
   }
 #pragma unroll
-  for (int k = 0; k < U; ++k) acc[k] = e[k] + d[k];
+  for (int k = 0; k < U / 2; ++k) {
+    acc[2 * k] = e[k].x + d[k].x;
+    acc[2 * k + 1] = e[k].y + d[k].y;
+  }
 }
 
 // Persistent form, for plans whose group tap rows and two input spans fit in
