@@ -248,8 +248,17 @@ struct RsPlan {
   size_t smem = 0;
   bool pipe = false;     // the persistent, double-buffered FIR applies
   size_t smem_pipe = 0;  // its shared memory
+  // tensor-core form: rows of tcN outputs (a multiple of p and of 16, at most
+  // 160) sit tcD = tcN o / p inputs apart; a row reads the tcK inputs from
+  // tcLo on (relative to its first output's position), tcK a multiple of 64
+  bool tc = false;
+  int tcN = 0, tcD = 0, tcLo = 0, tcK = 0;
 };
 int64_t rs_len(int64_t n, int rate_in, int rate_out);  // -1 for invalid arguments
+cudaError_t launch_rs_btc(const RsPlan &pl, void *bmat, cudaStream_t s);
+cudaError_t launch_rs_fir_tc(const RsPlan &pl, const float *mono, float *y, void *bmat, const int64_t *in_off,
+                             const int64_t *out_off, const int32_t *tile_off, int n_clips, int n_tiles,
+                             cudaStream_t s);
 RsPlan rs_plan(int rate_in, int rate_out);
 cudaError_t launch_rs_table(const RsPlan &pl, float *coef, int32_t *lo, cudaStream_t s);
 cudaError_t launch_rs_mix(const float *x, int channels, int64_t ch_stride, int64_t n, float *mono, cudaStream_t s);

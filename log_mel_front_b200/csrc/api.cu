@@ -1361,7 +1361,7 @@ struct RsTables {
 };
 
 struct RsLayout {
-  size_t in_off = 0, out_off = 0, tile_off = 0, lo = 0, coef = 0, mono = 0, total = 0;
+  size_t in_off = 0, out_off = 0, tile_off = 0, lo = 0, coef = 0, bmat = 0, mono = 0, total = 0;
 };
 
 ae_status rs_check_rates(int32_t rate_in, int32_t rate_out) {
@@ -1386,7 +1386,10 @@ ae_status rs_tables(const int64_t *off, int n, int32_t rate_in, int32_t rate_out
     const int64_t out = rs_len(len, rate_in, rate_out);
     t.out_off[i + 1] = t.out_off[i] + out;
     const int64_t units = (out + pl.U - 1) / pl.U, per_type = (units + pl.NT - 1) / pl.NT;
-    const int64_t tiles = rate_in == rate_out ? 0 : (per_type + pl.Q - 1) / pl.Q;
+    // tensor-core form: tiles of 128 rows of tcN outputs
+    const int64_t tiles = rate_in == rate_out ? 0
+                          : pl.tc         ? ((out + pl.tcN - 1) / pl.tcN + 127) / 128
+                                          : (per_type + pl.Q - 1) / pl.Q;
     if ((t.n_tiles + tiles) * pl.n_groups > INT32_MAX)
       return fail(AE_EUNSUPPORTED, "too many resampler tiles in one call");
     t.n_tiles += tiles;
@@ -1409,9 +1412,11 @@ RsLayout rs_layout(int n_clips, const RsPlan &pl, int64_t total_in, int channels
   L.tile_off = off;
   off += al256(B1 * 4);
   L.lo = off;
-  off += equal ? 0 : al256((size_t)pl.NT * 4);
+  off += equal || pl.tc ? 0 : al256((size_t)pl.NT * 4);
   L.coef = off;
-  off += equal ? 0 : al256((size_t)pl.NT * pl.W_pad * pl.U * 4);
+  off += equal || pl.tc ? 0 : al256((size_t)pl.NT * pl.W_pad * pl.U * 4);
+  L.bmat = off;  // the tensor-core form's taps: bf16 high and low parts, [tcN][tcK] each
+  off += !equal && pl.tc ? al256((size_t)2 * pl.tcN * pl.tcK * 2) : 0;
   L.mono = off;
   off += (channels > 1 && !equal) ? al256((size_t)total_in * 4) : 0;
   L.total = off;
@@ -1500,6 +1505,7 @@ ae_status ae_resample(const float *d_x, int channels, int64_t ch_stride, const i
   int32_t *tile_off = reinterpret_cast<int32_t *>(w + L.tile_off);
   int32_t *lo = reinterpret_cast<int32_t *>(w + L.lo);
   float *coef = reinterpret_cast<float *>(w + L.coef);
+  void *bmat = w + L.bmat;
   const float *mono = d_x;
   if ((e = timed(AE_K_TABLES, 0.0, 0.0, s, [&] {
          cudaError_t r = launch_upload_bytes(T.in_off.data(), T.in_off.size() * 8, in_off, s);
@@ -1508,9 +1514,14 @@ ae_status ae_resample(const float *d_x, int channels, int64_t ch_stride, const i
          return r;
        })) != cudaSuccess)
     return cuda_fail(e, "table upload");
-  if ((e = timed(AE_K_RESAMPLE, 0.0, 4.0 * pl.U * pl.NT * pl.W_pad, s, [&] { return launch_rs_table(pl, coef, lo, s); })) !=
-      cudaSuccess)
+  if (pl.tc) {
+    if ((e = timed(AE_K_RESAMPLE, 0.0, 4.0 * pl.tcN * pl.tcK, s, [&] { return launch_rs_btc(pl, bmat, s); })) !=
+        cudaSuccess)
+      return cuda_fail(e, "resampler taps");
+  } else if ((e = timed(AE_K_RESAMPLE, 0.0, 4.0 * pl.U * pl.NT * pl.W_pad, s,
+                        [&] { return launch_rs_table(pl, coef, lo, s); })) != cudaSuccess) {
     return cuda_fail(e, "resampler taps");
+  }
   if (channels > 1) {
     float *m = reinterpret_cast<float *>(w + L.mono);
     if ((e = timed(AE_K_RESAMPLE, 0.0, in_bytes + 4.0 * T.total_in, s, [&] {
@@ -1521,6 +1532,7 @@ ae_status ae_resample(const float *d_x, int channels, int64_t ch_stride, const i
   }
   const double taps = (double)(2 * (int)std::ceil(pl.half) + 1);
   if ((e = timed(AE_K_RESAMPLE, 2.0 * taps * (double)T.total_out, 4.0 * (double)T.total_in + out_bytes, s, [&] {
+         if (pl.tc) return launch_rs_fir_tc(pl, mono, d_y, bmat, in_off, out_off, tile_off, n_clips, (int)T.n_tiles, s);
          return launch_rs_fir(pl, mono, d_y, coef, lo, in_off, out_off, tile_off, n_clips, (int)T.n_tiles, s);
        })) != cudaSuccess)
     return cuda_fail(e, "resampler");

@@ -41,6 +41,8 @@ constexpr int kRsThreads = 256;
 constexpr int kRsWarps = kRsThreads / 32;
 constexpr size_t kRsSmemMax = 200 * 1024;  // staged input + staged output per CTA
 constexpr size_t kRsPipeSmemMax = 220 * 1024;  // tap rows + two input spans (persistent form)
+constexpr int kRsTcMaxN = 160;   // outputs per row of the tensor-core form
+constexpr int kRsTcMaxK = 4096;  // inputs per row
 }  // namespace
 
 // I0(x) = sum_k ((x / 2)^2)^k / (k!)^2, summed while the terms still count.
@@ -401,9 +403,27 @@ static RsPlan rs_plan_u(int rate_in, int rate_out, int U, int items, int parts) 
 RsPlan rs_plan(int rate_in, int rate_out) {
   // eight outputs per unit in the persistent form when it fits (4 items of
   // 4 warps each), else four (8 items of 2 warps, or the per-tile form)
-  const RsPlan p8 = rs_plan_u(rate_in, rate_out, 8, 4, 4);
-  if (p8.pipe) return p8;
-  return rs_plan_u(rate_in, rate_out, 4, kRsWarps, 2);
+  RsPlan pl = rs_plan_u(rate_in, rate_out, 8, 4, 4);
+  if (!pl.pipe) pl = rs_plan_u(rate_in, rate_out, 4, kRsWarps, 2);
+  // the tensor-core form when a row of outputs that repeats the same taps
+  // (a multiple of p) holds at most 160 and a multiple of 16 of them
+  int g16 = 16;
+  while (pl.p % g16) g16 /= 2;
+  const int64_t N = (int64_t)pl.p * (16 / g16);
+  if (rate_in != rate_out && N <= kRsTcMaxN) {
+    const int64_t D = N * pl.o / pl.p;
+    const int lo = (int)std::floor(-pl.half) - 1;
+    const int hi = (int)std::ceil((double)(N - 1) * pl.o / pl.p + pl.half) + 1;
+    const int64_t K = ((int64_t)(hi - lo + 1) + 63) / 64 * 64;
+    if (D <= (1 << 20) && K <= kRsTcMaxK) {
+      pl.tc = true;
+      pl.tcN = (int)N;
+      pl.tcD = (int)D;
+      pl.tcLo = lo;
+      pl.tcK = (int)K;
+    }
+  }
+  return pl;
 }
 
 cudaError_t launch_rs_table(const RsPlan &pl, float *coef, int32_t *lo, cudaStream_t s) {
@@ -470,6 +490,283 @@ cudaError_t launch_rs_fir(const RsPlan &pl, const float *mono, float *y, const f
     if (e != cudaSuccess) return e;
   }
   return launch_k(k_rs_fir, dim3((unsigned)((int64_t)n_tiles * pl.n_groups)), dim3(kRsThreads), pl.smem, s, a);
+}
+
+// ------------------------------------------------------------------ tensor-core form
+
+// The FIR as a product: row r of outputs r N .. r N + N - 1 (N = tcN) reads
+// the inputs r D + lo .. r D + lo + K - 1 (D = tcD, lo = tcLo, K = tcK), with
+// the same taps for every row, so Y[rows][N] = X[rows][K] B^T with B[N][K]
+// the taps of each output of a row at each input offset (zero outside its 64
+// zero crossings). Both operands are split into bf16 parts (hi = bf16(v), lo =
+// bf16(v - hi), v = hi + lo to about 2^-18 relative) and the product is taken
+// as X_hi B_hi + X_hi B_lo + X_lo B_hi + X_lo B_lo, accumulated in float32 on
+// the tensor cores.
+
+// B's two parts, [N][K] bf16 each (hi first), the taps in float64 as the
+// other table's: t = (lo + k - j o / p) c for output j of a row, input k.
+__global__ void k_rs_btc(bf16 *__restrict__ bmat, int N, int K, int lo, int o, int p, double c, double i0b) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)N * K) return;
+  const int j = (int)(idx / K), k = (int)(idx % K);
+  const double t = ((double)(lo + k) - (double)j * (double)o / (double)p) * c;
+  double v = 0.0;
+  if (fabs(t) < kRsWidth) {
+    const double q = t / kRsWidth;
+    const double win = rs_bessel_i0(kRsBeta * sqrt(1.0 - q * q)) / i0b;
+    const double pt = M_PI * t;
+    v = (pt == 0.0 ? 1.0 : sin(pt) / pt) * win * c;
+  }
+  const bf16 hi = __double2bfloat16(v);
+  bmat[idx] = hi;
+  bmat[(int64_t)N * K + idx] = __double2bfloat16(v - (double)__bfloat162float(hi));
+}
+
+struct RsTcArgs {
+  const float *x;
+  float *y;
+  const int64_t *in_off, *out_off;
+  const int32_t *tile_off;  // [B + 1] tiles of 128 rows
+  int n_clips, n_tiles, N, D, lo, kb_n;
+};
+
+namespace {
+constexpr int kTcThreads = 256;
+constexpr uint32_t kTcA = 128 * 128;             // one part of A: 128 rows x 64 bf16
+constexpr uint32_t kTcB = kRsTcMaxN * 128;       // one part of B: up to 160 rows x 64 bf16
+constexpr uint32_t kTcOffB = 2 * 2 * kTcA;       // A: [2 stages][hi, lo]
+constexpr uint32_t kTcOffRaw = kTcOffB + 2 * 2 * kTcB;  // B: [2 stages][hi, lo]
+constexpr uint32_t kTcOffBar = kTcOffRaw + 2 * 128 * 64 * 4;  // raw inputs: [2][128 rows][64] float32
+constexpr size_t kTcSmem = kTcOffBar + 64 + 1024;
+static_assert(kTcOffB % 1024 == 0 && kTcOffRaw % 1024 == 0, "swizzle atoms");
+static_assert(kTcSmem <= 227 * 1024, "one CTA per SM");
+}  // namespace
+
+struct RsTcTile {
+  int64_t in0, n_in, out0, n_out, rows, r0;
+};
+__device__ __forceinline__ RsTcTile rs_tc_tile(const RsTcArgs &a, int tile) {
+  int l = 0, h = a.n_clips;
+  while (h - l > 1) {
+    const int mid = (l + h) >> 1;
+    if (a.tile_off[mid] <= tile) l = mid; else h = mid;
+  }
+  RsTcTile r;
+  r.in0 = a.in_off[l];
+  r.n_in = a.in_off[l + 1] - r.in0;
+  r.out0 = a.out_off[l];
+  r.n_out = a.out_off[l + 1] - r.out0;
+  r.rows = (r.n_out + a.N - 1) / a.N;
+  r.r0 = (int64_t)(tile - a.tile_off[l]) * 128;
+  return r;
+}
+
+// Persistent CTAs over tiles of 128 rows; per 64-input k-block: the raw inputs
+// of the next k-block are copied with cp.async while the current one is split
+// into A's two parts and B's two parts arrive by TMA; one thread issues the
+// four products into the tile's accumulator (N tensor-memory columns). All
+// threads drain it at the end of the tile.
+__global__ void __launch_bounds__(kTcThreads, 1) k_rs_fir_tc(const __grid_constant__ CUtensorMap tmB, const RsTcArgs a,
+                                                            unsigned *status) {
+  extern __shared__ uint8_t tc_raw_smem[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(tc_raw_smem) + 1023) & ~uintptr_t(1023));
+  float *raw = reinterpret_cast<float *>(smem + kTcOffRaw);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kTcOffBar), *empty = full + 2, *accb = full + 4;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(full + 5);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int N = a.N, D = a.D, kb_n = a.kb_n;
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(accb, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t idesc = idesc_bf16_f32(128, N);
+
+  // raw inputs of k-block kb of a tile into buffer b: row i (row r0 + i of the
+  // clip), input r D + lo + 64 kb + e; zero outside the clip and past its rows
+  auto stage = [&](const RsTcTile &T, int kb, int b) {
+    // thread tid copies column tid mod 64 of rows tid / 64 + 4 i; no checks when
+    // the whole block of 128 rows x 64 inputs lies inside the clip
+    float *dst = raw + b * 128 * 64 + tid;
+    int64_t r = T.r0 + (tid >> 6);
+    int64_t m = r * D + a.lo + 64 * kb + (tid & 63);
+    const float *xin = a.x + T.in0;
+    const int64_t first = T.r0 * D + a.lo + 64 * kb, last = (T.r0 + 127) * D + a.lo + 64 * kb + 63;
+    if (T.r0 + 127 < T.rows && first >= 0 && last < T.n_in) {
+      const float *src = xin + m;
+#pragma unroll 8
+      for (int i = 0; i < 128 * 64 / kTcThreads; ++i) cp_async4(dst + i * kTcThreads, src + (int64_t)i * 4 * D, true);
+    } else {
+#pragma unroll 4
+      for (int i = 0; i < 128 * 64 / kTcThreads; ++i, r += 4, m += 4 * (int64_t)D) {
+        const bool ok = r < T.rows && m >= 0 && m < T.n_in;
+        cp_async4(dst + i * kTcThreads, ok ? xin + m : a.x, ok);
+      }
+    }
+  };
+  int64_t g = 0;
+  int ntile = 0;
+  bool ok = true;
+  int t = blockIdx.x;
+  RsTcTile cur{};
+  if (t < a.n_tiles) {
+    cur = rs_tc_tile(a, t);
+    stage(cur, 0, 0);
+  }
+  cp_async_commit();
+  for (; t < a.n_tiles && ok; t += gridDim.x, ++ntile) {
+    for (int kb = 0; kb < kb_n; ++kb, ++g) {
+      const int st = (int)(g & 1);
+      // the next k-block's inputs (this tile's, or the next tile's first)
+      if (kb + 1 < kb_n) {
+        stage(cur, kb + 1, st ^ 1);
+      } else if (t + (int)gridDim.x < a.n_tiles) {
+        stage(rs_tc_tile(a, t + gridDim.x), 0, st ^ 1);
+      }
+      cp_async_commit();
+      cp_async_wait_1();  // this k-block's inputs (this thread's copies)
+      bool good = true;
+      if (tid == 0 && g >= 2) good = mbar_wait(&empty[st], (uint32_t)(((g >> 1) - 1) & 1));  // stage st is free
+      if (!__syncthreads_and(good)) {
+        ok = false;
+        break;
+      }
+      if (tid == 0) {
+        mbar_arrive_expect_tx(&full[st], 2u * (uint32_t)N * 128u);
+        tma_load_2d(smem + kTcOffB + (2 * st) * kTcB, &tmB, 64 * kb, 0, &full[st]);
+        tma_load_2d(smem + kTcOffB + (2 * st + 1) * kTcB, &tmB, 64 * kb, N, &full[st]);
+      }
+      {  // split the raw inputs into A's parts: thread = (row, quad of 4 inputs), 8 each;
+         // a warp reads two whole rows (conflict-free) and writes half-granules
+        const float *src = raw + st * 128 * 64;
+        uint8_t *ahi = smem + (2 * st) * kTcA, *alo = smem + (2 * st + 1) * kTcA;
+#pragma unroll
+        for (int rep = 0; rep < 8; ++rep) {
+          const int e = tid + rep * kTcThreads, row = e >> 4, quad = e & 15;
+          const float4 v = *reinterpret_cast<const float4 *>(src + row * 64 + quad * 4);
+          const float h0 = __bfloat162float(__float2bfloat16_rn(v.x)), h1 = __bfloat162float(__float2bfloat16_rn(v.y));
+          const float h2 = __bfloat162float(__float2bfloat16_rn(v.z)), h3 = __bfloat162float(__float2bfloat16_rn(v.w));
+          const uint32_t off = row * 128 + (((quad >> 1) ^ (row & 7)) << 4) + (quad & 1) * 8;
+          *reinterpret_cast<uint2 *>(ahi + off) = make_uint2(pack_bf16(h0, h1), pack_bf16(h2, h3));
+          *reinterpret_cast<uint2 *>(alo + off) = make_uint2(pack_bf16(v.x - h0, v.y - h1), pack_bf16(v.z - h2, v.w - h3));
+        }
+      }
+      fence_async_smem();
+      __syncthreads();  // A's parts are written
+      if (tid == 0) {
+        if (!mbar_wait(&full[st], (uint32_t)((g >> 1) & 1))) {
+          atomicOr(status, kStatusWaitTimeout);
+        } else {
+          tc_fence_after();
+          const uint32_t ahi = smem_u32(smem + (2 * st) * kTcA), alo = smem_u32(smem + (2 * st + 1) * kTcA);
+          const uint32_t bhi = smem_u32(smem + kTcOffB + (2 * st) * kTcB), blo = smem_u32(smem + kTcOffB + (2 * st + 1) * kTcB);
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            tc_mma_bf16(tmem, sw128_desc(ahi + ks * 32), sw128_desc(bhi + ks * 32), idesc, (kb | ks) != 0 ? 1u : 0u);
+            tc_mma_bf16(tmem, sw128_desc(ahi + ks * 32), sw128_desc(blo + ks * 32), idesc, 1u);
+            tc_mma_bf16(tmem, sw128_desc(alo + ks * 32), sw128_desc(bhi + ks * 32), idesc, 1u);
+            tc_mma_bf16(tmem, sw128_desc(alo + ks * 32), sw128_desc(blo + ks * 32), idesc, 1u);
+          }
+        }
+        tc_commit(&empty[st]);
+        if (kb + 1 == kb_n) tc_commit(accb);
+      }
+    }
+    if (!ok) break;
+    // drain: warp w reads lanes 32 (w & 3) .. + 31 (rows), columns of half w >> 2
+    const bool got = mbar_wait(accb, (uint32_t)(ntile & 1));
+    if (!__syncthreads_and(got)) {
+      ok = false;
+      break;
+    }
+    tc_fence_after();
+    {
+      const int q = warp & 3, half = warp >> 2, ncol = N / 2;  // N / 2 is a multiple of 8
+      const int64_t r = cur.r0 + 32 * q + lane;
+      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(half * ncol);
+      for (int c0 = 0; c0 < ncol; c0 += 8) {
+        uint32_t v[8];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+            : "r"(taddr + c0));
+        tmem_ld_wait();
+        if (r < cur.rows) {
+          const int64_t n0 = r * N + half * ncol + c0;
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            if (n0 + u < cur.n_out) a.y[cur.out0 + n0 + u] = __uint_as_float(v[u]);
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();  // the accumulator is read: the next tile's first product may overwrite it
+    if (t + (int)gridDim.x < a.n_tiles) cur = rs_tc_tile(a, t + gridDim.x);
+  }
+  if (!ok && tid == 0) atomicOr(status, kStatusWaitTimeout);
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+cudaError_t launch_rs_btc(const RsPlan &pl, void *bmat, cudaStream_t s) {
+  const int64_t n = (int64_t)pl.tcN * pl.tcK;
+  const double i0b = [] {
+    double q = 0.25 * kRsBeta * kRsBeta, term = 1.0, sum = 1.0;
+    for (int k = 1; k < 400; ++k) {
+      term *= q / ((double)k * (double)k);
+      sum += term;
+      if (term < sum * 1e-17) break;
+    }
+    return sum;
+  }();
+  return launch_k(k_rs_btc, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, static_cast<bf16 *>(bmat), pl.tcN,
+                  pl.tcK, pl.tcLo, pl.o, pl.p, pl.c, i0b);
+}
+
+cudaError_t launch_rs_fir_tc(const RsPlan &pl, const float *mono, float *y, void *bmat, const int64_t *in_off,
+                             const int64_t *out_off, const int32_t *tile_off, int n_clips, int n_tiles,
+                             cudaStream_t s) {
+  if (n_tiles <= 0) return cudaSuccess;
+  CUtensorMap tmB;  // both parts as one [2 N][K] bf16 matrix, boxes of 64 inputs x N rows
+  if (!make_tmap_2d_bf16(&tmB, bmat, (uint64_t)pl.tcK, (uint64_t)2 * pl.tcN, (uint64_t)pl.tcK * 2, 64,
+                         (uint32_t)pl.tcN))
+    return cudaErrorInvalidValue;
+  static std::atomic<uint64_t> attr{0};
+  if (const cudaError_t e = smem_attr(k_rs_fir_tc, kTcSmem, attr)) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  RsTcArgs a;
+  a.x = mono;
+  a.y = y;
+  a.in_off = in_off;
+  a.out_off = out_off;
+  a.tile_off = tile_off;
+  a.n_clips = n_clips;
+  a.n_tiles = n_tiles;
+  a.N = pl.tcN;
+  a.D = pl.tcD;
+  a.lo = pl.tcLo;
+  a.kb_n = pl.tcK / 64;
+  const int grid = n_tiles < sms ? n_tiles : sms;
+  return launch_k(k_rs_fir_tc, dim3((unsigned)grid), dim3(kTcThreads), kTcSmem, s, tmB, a, device_status_word());
 }
 
 }  // namespace ae
