@@ -535,10 +535,9 @@ constexpr int kTcThreads = 256;
 constexpr uint32_t kTcA = 128 * 128;             // one part of A: 128 rows x 64 bf16
 constexpr uint32_t kTcB = kRsTcMaxN * 128;       // one part of B: up to 160 rows x 64 bf16
 constexpr uint32_t kTcOffB = 2 * 2 * kTcA;       // A: [2 stages][hi, lo]
-constexpr uint32_t kTcOffRaw = kTcOffB + 2 * 2 * kTcB;  // B: [2 stages][hi, lo]
-constexpr uint32_t kTcOffBar = kTcOffRaw + 2 * 128 * 64 * 4;  // raw inputs: [2][128 rows][64] float32
+constexpr uint32_t kTcOffBar = kTcOffB + 2 * 2 * kTcB;  // B: [2 stages][hi, lo]
 constexpr size_t kTcSmem = kTcOffBar + 64 + 1024;
-static_assert(kTcOffB % 1024 == 0 && kTcOffRaw % 1024 == 0, "swizzle atoms");
+static_assert(kTcOffB % 1024 == 0 && kTcOffBar % 1024 == 0, "swizzle atoms");
 static_assert(kTcSmem <= 227 * 1024, "one CTA per SM");
 }  // namespace
 
@@ -561,16 +560,17 @@ __device__ __forceinline__ RsTcTile rs_tc_tile(const RsTcArgs &a, int tile) {
   return r;
 }
 
-// Persistent CTAs over tiles of 128 rows; per 64-input k-block: the raw inputs
-// of the next k-block are copied with cp.async while the current one is split
-// into A's two parts and B's two parts arrive by TMA; one thread issues the
-// four products into the tile's accumulator (N tensor-memory columns). All
-// threads drain it at the end of the tile.
+// Persistent CTAs over tiles of 128 rows, walked as one sequence of steps
+// (tile, 64-input k-block). Thread t owns inputs 4 (t mod 16) .. + 3 of rows
+// t / 16 + 16 i of every k-block: it loads them two steps ahead into one of
+// three register sets (the loop is unrolled three times, so no set is copied),
+// splits the current set into A's two parts, and B's two parts arrive by TMA;
+// one thread issues the four products into the tile's accumulator (N
+// tensor-memory columns), and all threads drain it after the tile's last step.
 __global__ void __launch_bounds__(kTcThreads, 1) k_rs_fir_tc(const __grid_constant__ CUtensorMap tmB, const RsTcArgs a,
                                                             unsigned *status) {
   extern __shared__ uint8_t tc_raw_smem[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(tc_raw_smem) + 1023) & ~uintptr_t(1023));
-  float *raw = reinterpret_cast<float *>(smem + kTcOffRaw);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + kTcOffBar), *empty = full + 2, *accb = full + 4;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(full + 5);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -593,108 +593,106 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_rs_fir_tc(const __grid_consta
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t idesc = idesc_bf16_f32(128, N);
+  const int my_tiles = (int)blockIdx.x < a.n_tiles ? (a.n_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int64_t n_steps = (int64_t)my_tiles * kb_n;
+  const int qd = tid & 15, rw0 = tid >> 4;
 
-  // raw inputs of k-block kb of a tile into buffer b: row i (row r0 + i of the
-  // clip), input r D + lo + 64 kb + e; zero outside the clip and past its rows
-  auto stage = [&](const RsTcTile &T, int kb, int b) {
-    // thread tid copies column tid mod 64 of rows tid / 64 + 4 i; no checks when
-    // the whole block of 128 rows x 64 inputs lies inside the clip
-    float *dst = raw + b * 128 * 64 + tid;
-    int64_t r = T.r0 + (tid >> 6);
-    int64_t m = r * D + a.lo + 64 * kb + (tid & 63);
-    const float *xin = a.x + T.in0;
+  // tile records of the step being computed and of the one being loaded
+  RsTcTile tc_cur{}, tc_ld{};
+  int ld_tile = -1;
+  auto tile_of_step = [&](int64_t st) { return (int)blockIdx.x + (int)(st / kb_n) * (int)gridDim.x; };
+  auto load = [&](int64_t st, float (&v)[32]) {
+    const int tile = tile_of_step(st), kb = (int)(st % kb_n);
+    if (tile != ld_tile) {
+      tc_ld = rs_tc_tile(a, tile);
+      ld_tile = tile;
+    }
+    const RsTcTile &T = tc_ld;
     const int64_t first = T.r0 * D + a.lo + 64 * kb, last = (T.r0 + 127) * D + a.lo + 64 * kb + 63;
+    const float *xin = a.x + T.in0;
+    int64_t m = (T.r0 + rw0) * D + a.lo + 64 * kb + 4 * qd;
     if (T.r0 + 127 < T.rows && first >= 0 && last < T.n_in) {
-      const float *src = xin + m;
-#pragma unroll 8
-      for (int i = 0; i < 128 * 64 / kTcThreads; ++i) cp_async4(dst + i * kTcThreads, src + (int64_t)i * 4 * D, true);
+#pragma unroll
+      for (int i = 0; i < 8; ++i, m += 16 * (int64_t)D) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[4 * i + u] = __ldg(xin + m + u);
+      }
     } else {
-#pragma unroll 4
-      for (int i = 0; i < 128 * 64 / kTcThreads; ++i, r += 4, m += 4 * (int64_t)D) {
-        const bool ok = r < T.rows && m >= 0 && m < T.n_in;
-        cp_async4(dst + i * kTcThreads, ok ? xin + m : a.x, ok);
+      int64_t r = T.r0 + rw0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i, m += 16 * (int64_t)D, r += 16) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const bool ok = r < T.rows && m + u >= 0 && m + u < T.n_in;
+          v[4 * i + u] = ok ? __ldg(xin + m + u) : 0.f;
+        }
       }
     }
   };
-  int64_t g = 0;
   int ntile = 0;
   bool ok = true;
-  int t = blockIdx.x;
-  RsTcTile cur{};
-  if (t < a.n_tiles) {
-    cur = rs_tc_tile(a, t);
-    stage(cur, 0, 0);
-  }
-  cp_async_commit();
-  for (; t < a.n_tiles && ok; t += gridDim.x, ++ntile) {
-    for (int kb = 0; kb < kb_n; ++kb, ++g) {
-      const int st = (int)(g & 1);
-      // the next k-block's inputs (this tile's, or the next tile's first)
-      if (kb + 1 < kb_n) {
-        stage(cur, kb + 1, st ^ 1);
-      } else if (t + (int)gridDim.x < a.n_tiles) {
-        stage(rs_tc_tile(a, t + gridDim.x), 0, st ^ 1);
-      }
-      cp_async_commit();
-      cp_async_wait_1();  // this k-block's inputs (this thread's copies)
-      bool good = true;
-      if (tid == 0 && g >= 2) good = mbar_wait(&empty[st], (uint32_t)(((g >> 1) - 1) & 1));  // stage st is free
-      if (!__syncthreads_and(good)) {
-        ok = false;
-        break;
-      }
-      if (tid == 0) {
-        mbar_arrive_expect_tx(&full[st], 2u * (uint32_t)N * 128u);
-        tma_load_2d(smem + kTcOffB + (2 * st) * kTcB, &tmB, 64 * kb, 0, &full[st]);
-        tma_load_2d(smem + kTcOffB + (2 * st + 1) * kTcB, &tmB, 64 * kb, N, &full[st]);
-      }
-      {  // split the raw inputs into A's parts: thread = (row, quad of 4 inputs), 8 each;
-         // a warp reads two whole rows (conflict-free) and writes half-granules
-        const float *src = raw + st * 128 * 64;
-        uint8_t *ahi = smem + (2 * st) * kTcA, *alo = smem + (2 * st + 1) * kTcA;
+  // one step: s's inputs are in `cur`; s + 2's are loaded into `nxt`
+  auto step = [&](int64_t sidx, float (&cur)[32], float (&nxt)[32]) {
+    if (!ok) return;
+    const int st = (int)(sidx & 1), kb = (int)(sidx % kb_n);
+    if (kb == 0) tc_cur = rs_tc_tile(a, tile_of_step(sidx));
+    if (sidx + 2 < n_steps) load(sidx + 2, nxt);
+    bool good = true;
+    if (tid == 0 && sidx >= 2) good = mbar_wait(&empty[st], (uint32_t)(((sidx >> 1) - 1) & 1));  // stage st is free
+    if (!__syncthreads_and(good)) {
+      ok = false;
+      return;
+    }
+    if (tid == 0) {
+      mbar_arrive_expect_tx(&full[st], 2u * (uint32_t)N * 128u);
+      tma_load_2d(smem + kTcOffB + (2 * st) * kTcB, &tmB, 64 * kb, 0, &full[st]);
+      tma_load_2d(smem + kTcOffB + (2 * st + 1) * kTcB, &tmB, 64 * kb, N, &full[st]);
+    }
+    {  // split into A's parts: row rw0 + 16 i, inputs 4 qd .. 4 qd + 3 (half a 16-byte granule)
+      uint8_t *ahi = smem + (2 * st) * kTcA, *alo = smem + (2 * st + 1) * kTcA;
 #pragma unroll
-        for (int rep = 0; rep < 8; ++rep) {
-          const int e = tid + rep * kTcThreads, row = e >> 4, quad = e & 15;
-          const float4 v = *reinterpret_cast<const float4 *>(src + row * 64 + quad * 4);
-          const float h0 = __bfloat162float(__float2bfloat16_rn(v.x)), h1 = __bfloat162float(__float2bfloat16_rn(v.y));
-          const float h2 = __bfloat162float(__float2bfloat16_rn(v.z)), h3 = __bfloat162float(__float2bfloat16_rn(v.w));
-          const uint32_t off = row * 128 + (((quad >> 1) ^ (row & 7)) << 4) + (quad & 1) * 8;
-          *reinterpret_cast<uint2 *>(ahi + off) = make_uint2(pack_bf16(h0, h1), pack_bf16(h2, h3));
-          *reinterpret_cast<uint2 *>(alo + off) = make_uint2(pack_bf16(v.x - h0, v.y - h1), pack_bf16(v.z - h2, v.w - h3));
-        }
-      }
-      fence_async_smem();
-      __syncthreads();  // A's parts are written
-      if (tid == 0) {
-        if (!mbar_wait(&full[st], (uint32_t)((g >> 1) & 1))) {
-          atomicOr(status, kStatusWaitTimeout);
-        } else {
-          tc_fence_after();
-          const uint32_t ahi = smem_u32(smem + (2 * st) * kTcA), alo = smem_u32(smem + (2 * st + 1) * kTcA);
-          const uint32_t bhi = smem_u32(smem + kTcOffB + (2 * st) * kTcB), blo = smem_u32(smem + kTcOffB + (2 * st + 1) * kTcB);
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            tc_mma_bf16(tmem, sw128_desc(ahi + ks * 32), sw128_desc(bhi + ks * 32), idesc, (kb | ks) != 0 ? 1u : 0u);
-            tc_mma_bf16(tmem, sw128_desc(ahi + ks * 32), sw128_desc(blo + ks * 32), idesc, 1u);
-            tc_mma_bf16(tmem, sw128_desc(alo + ks * 32), sw128_desc(bhi + ks * 32), idesc, 1u);
-            tc_mma_bf16(tmem, sw128_desc(alo + ks * 32), sw128_desc(blo + ks * 32), idesc, 1u);
-          }
-        }
-        tc_commit(&empty[st]);
-        if (kb + 1 == kb_n) tc_commit(accb);
+      for (int i = 0; i < 8; ++i) {
+        const int row = rw0 + 16 * i;
+        const float *v = cur + 4 * i;
+        const float h0 = __bfloat162float(__float2bfloat16_rn(v[0])), h1 = __bfloat162float(__float2bfloat16_rn(v[1]));
+        const float h2 = __bfloat162float(__float2bfloat16_rn(v[2])), h3 = __bfloat162float(__float2bfloat16_rn(v[3]));
+        const uint32_t off = row * 128 + (((qd >> 1) ^ (row & 7)) << 4) + (qd & 1) * 8;
+        *reinterpret_cast<uint2 *>(ahi + off) = make_uint2(pack_bf16(h0, h1), pack_bf16(h2, h3));
+        *reinterpret_cast<uint2 *>(alo + off) =
+            make_uint2(pack_bf16(v[0] - h0, v[1] - h1), pack_bf16(v[2] - h2, v[3] - h3));
       }
     }
-    if (!ok) break;
-    // drain: warp w reads lanes 32 (w & 3) .. + 31 (rows), columns of half w >> 2
+    fence_async_smem();
+    __syncthreads();  // A's parts are written
+    if (tid == 0) {
+      if (!mbar_wait(&full[st], (uint32_t)((sidx >> 1) & 1))) {
+        atomicOr(status, kStatusWaitTimeout);
+      } else {
+        tc_fence_after();
+        const uint32_t ahi = smem_u32(smem + (2 * st) * kTcA), alo = smem_u32(smem + (2 * st + 1) * kTcA);
+        const uint32_t bhi = smem_u32(smem + kTcOffB + (2 * st) * kTcB), blo = smem_u32(smem + kTcOffB + (2 * st + 1) * kTcB);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          tc_mma_bf16(tmem, sw128_desc(ahi + ks * 32), sw128_desc(bhi + ks * 32), idesc, (kb | ks) != 0 ? 1u : 0u);
+          tc_mma_bf16(tmem, sw128_desc(ahi + ks * 32), sw128_desc(blo + ks * 32), idesc, 1u);
+          tc_mma_bf16(tmem, sw128_desc(alo + ks * 32), sw128_desc(bhi + ks * 32), idesc, 1u);
+          tc_mma_bf16(tmem, sw128_desc(alo + ks * 32), sw128_desc(blo + ks * 32), idesc, 1u);
+        }
+      }
+      tc_commit(&empty[st]);
+      if (kb + 1 == kb_n) tc_commit(accb);
+    }
+    if (kb + 1 < kb_n) return;
+    // the tile's last step: drain (warp w reads lanes 32 (w & 3) .. + 31, columns of half w >> 2)
     const bool got = mbar_wait(accb, (uint32_t)(ntile & 1));
     if (!__syncthreads_and(got)) {
       ok = false;
-      break;
+      return;
     }
     tc_fence_after();
     {
       const int q = warp & 3, half = warp >> 2, ncol = N / 2;  // N / 2 is a multiple of 8
-      const int64_t r = cur.r0 + 32 * q + lane;
+      const int64_t r = tc_cur.r0 + 32 * q + lane;
       const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(half * ncol);
       for (int c0 = 0; c0 < ncol; c0 += 8) {
         uint32_t v[8];
@@ -703,20 +701,27 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_rs_fir_tc(const __grid_consta
             : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
             : "r"(taddr + c0));
         tmem_ld_wait();
-        if (r < cur.rows) {
+        if (r < tc_cur.rows) {
           const int64_t n0 = r * N + half * ncol + c0;
 #pragma unroll
           for (int u = 0; u < 8; ++u)
-            if (n0 + u < cur.n_out) a.y[cur.out0 + n0 + u] = __uint_as_float(v[u]);
+            if (n0 + u < tc_cur.n_out) a.y[tc_cur.out0 + n0 + u] = __uint_as_float(v[u]);
         }
       }
     }
     tc_fence_before();
     __syncthreads();  // the accumulator is read: the next tile's first product may overwrite it
-    if (t + (int)gridDim.x < a.n_tiles) cur = rs_tc_tile(a, t + gridDim.x);
+    ++ntile;
+  };
+  float va[32], vb[32], vc[32];
+  if (n_steps > 0) load(0, va);
+  if (n_steps > 1) load(1, vb);
+  for (int64_t sidx = 0; sidx < n_steps && ok; sidx += 3) {
+    step(sidx, va, vc);
+    if (sidx + 1 < n_steps) step(sidx + 1, vb, va);
+    if (sidx + 2 < n_steps) step(sidx + 2, vc, vb);
   }
   if (!ok && tid == 0) atomicOr(status, kStatusWaitTimeout);
-  asm volatile("cp.async.wait_all;" ::: "memory");
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
