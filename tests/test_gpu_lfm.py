@@ -71,3 +71,26 @@ def test_silence_and_zero_tail():
     assert np.all(got[0] == 0.0)  # constant log floor: zero variance, normalised to 0
     eff = L.effective_len(32000)
     assert eff == 200 and got[1].shape[0] == 201 and np.all(got[1][eff:] == 0.0)
+
+
+def test_wave_not_16_byte_aligned():
+    """With a waveform base 4 bytes off a 16-byte boundary the spectrum kernel
+    stages its samples 4 bytes at a time instead of 16: the same rows."""
+    clips = [synth.noise_tones_clip(n, 53, i) for i, n in enumerate([16000, 7777, 48123, 161])]
+    flat, off = synth.pack(clips)
+    cfg = ae.lfm_config()
+    frames = sum(ae.ae_lfm_num_frames(cfg, len(c)) for c in clips)
+    nb = ae.ae_lfm_workspace_size(cfg, len(clips))
+    outs = []
+    for shift in (0, 1):
+        base = torch.zeros(len(flat) + 8, device="cuda")
+        base[shift:shift + len(flat)] = dev(flat)
+        d_out = torch.full((frames, cfg.n_mels), float("nan"), device="cuda")
+        ws = workspace(nb)
+        ae.ae_lfm_logmel(cfg, base[shift:shift + len(flat)], off, d_out, ws, ws.numel())
+        torch.cuda.synchronize()
+        assert ae.ae_device_status() == ae.AE_OK
+        outs.append(d_out.cpu().numpy())
+    assert np.array_equal(outs[0], outs[1])
+    o = offsets([ae.ae_lfm_num_frames(cfg, len(c)) for c in clips])
+    _check(outs[1][o[2]:o[3]], L.features(clips[2]), "48123 samples from an unaligned base")

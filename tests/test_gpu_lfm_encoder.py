@@ -100,6 +100,27 @@ def test_stem_work_item_edges(m2, w2):
     assert_bf16(g, o, "LFM2A stem at work-item edges")
 
 
+def test_stem_mel_not_16_byte_aligned(m2):
+    """With a mel base 4 bytes off a 16-byte boundary the first stem kernel
+    stages its rows 4 bytes at a time instead of 16: the same rows."""
+    mels = _mels([16000, 2000, 10240], seed=44)
+    frames = [x.shape[0] for x in mels]
+    toks = [ae.ae_lenc_num_tokens(f) for f in frames]
+    off = offsets(frames)
+    flat = np.concatenate(mels)
+    outs = []
+    for shift in (0, 1):
+        base = torch.zeros(flat.size + 8, device="cuda")
+        base[shift:shift + flat.size] = dev(flat.ravel())
+        d_x = torch.full((sum(toks), 512), float("nan"), device="cuda")
+        ws = workspace(m2.workspace_size(off))
+        ae.ae_lenc_stem(m2, base[shift:shift + flat.size], off, d_x, ws, ws.numel())
+        _sync()
+        outs.append(d_x.cpu().numpy())
+    assert np.all(np.isfinite(outs[0]))
+    assert np.array_equal(outs[0], outs[1])
+
+
 @pytest.mark.parametrize("toks", [[1], [5, 128, 129, 3], [300, 7, 256]])
 def test_block_matches_oracle(m2, w2, toks):
     """One block from the same float32 input: the attention runs over whole clips
