@@ -26,6 +26,11 @@
 // spans do not fit: when the span does not fit (large D, as for co-prime
 // rates) it reads the input from global memory, and when the tap rows do not
 // fit it reads them from global memory too: correct, and slower.
+//
+// Rates whose repeating row of outputs is short (at most 160 outputs, a
+// multiple of 16: 44.1, 48, 32, 24, 8, 96 kHz ...) take the tensor-core form
+// instead (k_rs_btc builds its taps, k_rs_fir_tc computes; see the section
+// before launch_rs_btc): the same sums as products of bf16-split operands.
 #include <cmath>
 
 #include "ae_internal.h"
