@@ -1259,7 +1259,7 @@ ae_status ae_lfm_logmel(const ae_lfm_config *cfg, const float *d_wave, const int
   if (!cfg) return fail(AE_EINVAL, "cfg is null");
   if (!lfm_cfg_ok(cfg))
     return fail(AE_EUNSUPPORTED, "supported: n_fft 512, even win_length in [2, 512], even hop in [2, 320], n_mels "
-                                 "in [1, 128], sample_rate in [1000, 1e6], finite preemph, log_floor > 0, var_eps >= 0");
+                                 "in [1, 128], sample_rate in [1000, 1e6], finite preemph, log_floor > 0, var_eps > 0");
   if (n_clips < 0 || n_clips > kMaxClips) return fail(AE_EINVAL, "n_clips out of range");
   if (!h_sample_off) return fail(AE_EINVAL, "h_sample_off is null");
   if (h_sample_off[0] != 0) return fail(AE_EINVAL, "h_sample_off[0] must be 0");
