@@ -508,11 +508,17 @@ size_t ae_resample_workspace_size(const int64_t *h_sample_off, int n_clips, int3
  *          I0(12.8 sqrt(1 - (t/64)^2)) / I0(12.8),
  *   t = (m - n o / p) c, c = 0.958 min(o, p) / o, inputs outside the clip 0,
  * for n < ae_resample_len(N, rate_in, rate_out). The taps are evaluated in
- * float64 and applied in float32 with float32 accumulation in two
- * interleaved partial sums over L = 2 ceil(64 / c) + 3 taps: against the
- * float64 definition the error is below (L / 2 + 2) 2^-24 x 2.7 x max |mono|
- * (2.7 bounds the taps' absolute sum), 3e-5 x max |mono| from 48 kHz and
- * 6e-5 from 96 kHz. Equal rates copy mono.
+ * float64. Where a row of N = 16 p / gcd(p, 16) outputs (the taps repeat
+ * from one row to the next) holds at most 160 and its window at most 4096
+ * inputs (44.1, 48, 32, 24, 96 and 8 kHz among the common rates), the sums
+ * run on the tensor cores: inputs and taps each split into two bf16 parts
+ * (v = hi + lo to about 2^-18), the four products of the parts accumulated
+ * in float32. Other rates apply the taps in float32 with float32
+ * accumulation in two interleaved partial sums. Either way, against the
+ * float64 definition the error stays below (L / 2 + 2) 2^-24 x 2.7 x
+ * max |mono| with L = 2 ceil(64 / c) + 3 (2.7 bounds the taps' absolute
+ * sum): 3e-5 x max |mono| from 48 kHz, 6e-5 from 96 kHz. Equal rates copy
+ * mono.
  * d_x: float32, channel ch of the packed clips at d_x + ch * ch_stride
  * (ch_stride >= h_sample_off[n_clips] when channels > 1), clip k at
  * [h_sample_off[k], h_sample_off[k+1]) in every channel. channels 1 .. 64.

@@ -3,7 +3,9 @@ the C ABI) with the float64 oracle (``oracle/resample.py``), element by
 element, within the bound the arithmetic gives: float32 taps applied with
 float32 accumulation in two interleaved partial sums over L taps, error
 below (L / 2 + 2) 2^-24 x 2.7 x max |input|, 2.7 bounding the taps' absolute
-sum (computed from the definition for every rate used here)."""
+sum (computed from the definition for every rate used here, in
+``test_resample_pins.py``). The tensor-core form (bf16-split inputs and taps,
+four products, float32 accumulation) is held to the same bound."""
 import math
 
 import numpy as np
@@ -92,6 +94,25 @@ def test_ragged_stereo_batch_at_44k1():
 def test_other_rates(rate):
     rng = np.random.default_rng(rate)
     clips = [[rng.uniform(-1, 1, n).astype(np.float32)] for n in (rate // 3, 777)]
+    got = gpu_resample(clips, rate)
+    for k, clip in enumerate(clips):
+        _check(got[k], R.resample(clip[0], rate), float(np.max(np.abs(clip[0]))), rate, f"{rate} Hz clip {k}")
+
+
+# Each tile width the tensor-core form takes besides 16 and 160 (a row of
+# N = 32, 64, 80 and 128 outputs), its longest window (432 kHz: 4032 inputs
+# per row, the most it takes being 4096), and the per-tile FIR for the rates
+# past that window (448 kHz, taps staged in shared memory; 1 MHz, the highest
+# rate taken, taps read from global memory), each over several tiles and a
+# ragged tail, beside a short clip.
+TILE_EDGE_RATES = {10500: 10513, 15750: 15763, 12600: 12613, 5125: 15388, 432000: 108000, 448000: 112000,
+                   1000000: 60000}
+
+
+@pytest.mark.parametrize("rate", sorted(TILE_EDGE_RATES))
+def test_every_tile_width_and_the_widest_windows(rate):
+    rng = np.random.default_rng(rate + 1)
+    clips = [[rng.uniform(-1, 1, n).astype(np.float32)] for n in (TILE_EDGE_RATES[rate], 777)]
     got = gpu_resample(clips, rate)
     for k, clip in enumerate(clips):
         _check(got[k], R.resample(clip[0], rate), float(np.max(np.abs(clip[0]))), rate, f"{rate} Hz clip {k}")

@@ -146,3 +146,29 @@ def test_linear_and_shift_equivariant():
         a = R.resample(x, rate)
         b = R.resample(xs, rate)
         assert np.array_equal(b[p:p + len(a)], a) or np.max(np.abs(b[p:p + len(a)] - a)) < 1e-6
+
+
+# Every rate the GPU parity tests resample from (``tests/test_gpu_resample.py``).
+GPU_TEST_RATES = (8000, 44100, 48000, 22050, 96000, 11025, 32000, 24000, 44099, 10500, 15750, 12600, 5125, 432000,
+                  448000, 1000000)
+
+
+def test_tap_sums_stay_below_the_parity_bound():
+    """The GPU parity bound (L / 2 + 2) 2^-24 x 2.7 x max |input| takes 2.7 for
+    the absolute sum of one output's taps. Evaluated here from the page's
+    definition (numpy's I0, every phase of every rate the GPU tests use), the
+    largest sum is about 2.66 (upsampling) and 2.37 to 2.43 otherwise."""
+    for rate in GPU_TEST_RATES:
+        g = math.gcd(rate, 16000)
+        o, p = rate // g, 16000 // g
+        c = 0.958 * min(o, p) / o
+        half = 64.0 / c
+        worst = 0.0
+        for j in range(p):
+            frac = o * j / p
+            d = np.arange(math.floor(frac - half), math.ceil(frac + half) + 1)
+            t = (d - frac) * c
+            t = t[np.abs(t) < 64.0]
+            win = np.i0(12.8 * np.sqrt(1.0 - (t / 64.0) ** 2)) / np.i0(12.8)
+            worst = max(worst, float(np.sum(np.abs(np.sinc(t) * win * c))))
+        assert 2.0 < worst <= 2.7, (rate, worst)
