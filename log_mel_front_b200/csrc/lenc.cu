@@ -484,9 +484,12 @@ cudaError_t launch_lenc_dwconv(const void *g, const float *w, const float *db, c
                                void *out, const int32_t *tok_off, int n_clips, int64_t T, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
   const size_t smem = (size_t)(kDwRows + k - 1) * 256 * 4;
+  // the attribute is set once per device, so the generic form takes the size
+  // of the widest kernel it accepts (models of other widths may follow)
   static std::atomic<uint64_t> attr9{0}, attr0{0};
   auto kern = k == 9 ? k_lenc_dwconv<9> : k_lenc_dwconv<0>;
-  if (const cudaError_t e = smem_attr(kern, smem, k == 9 ? attr9 : attr0)) return e;
+  const size_t smem_max = k == 9 ? smem : (size_t)(kDwRows + kLencMaxConvK - 1) * 256 * 4;
+  if (const cudaError_t e = smem_attr(kern, smem_max, k == 9 ? attr9 : attr0)) return e;
   return launch_k(kern, dim3((unsigned)((T + kDwRows - 1) / kDwRows)), dim3(256), smem, s,
                   static_cast<const bf16 *>(g), w, db, aw, ab, k, static_cast<bf16 *>(out), tok_off, n_clips, T);
 }

@@ -190,6 +190,29 @@ def test_packed_batch_matches_single_clips(m2, w2):
         assert_bf16(g[off[i]:off[i + 1]], o, f"LFM2A encode in a split batch, clip {i} ({toks[i]} tokens)")
 
 
+def test_other_sizes_in_one_process():
+    """Models of other sizes one after another in one process: conv module
+    widths 4 (even: one tap of padding on the left, two on the right), 33 (the
+    widest taken) and 1, with smaller FFN and adapter widths. The widths other
+    than 9 take the generic depthwise kernel, whose shared memory grows with
+    the width; the narrow model runs first."""
+    lens = [64000, 2500, 20480]
+    mels = _mels(lens, seed=47)
+    for k, (n_ff, ad_ff, hidden) in ((4, (256, 512, 768)), (33, (512, 256, 512)), (1, (768, 1024, 256))):
+        shape = dict(synth.LENC_SHAPE, n_layers=2, conv_k=k, n_ff=n_ff, adapter_ff=ad_ff, llm_hidden=hidden)
+        w = synth.lfm_encoder_weights(shape=shape, seed=5100 + k)
+        m = ae.LencModel(w)
+        try:
+            g, toks = _gpu_encode(m, mels, hidden=hidden)
+        finally:
+            m.close()
+        off = offsets(toks)
+        for i, x in enumerate(mels):
+            o = E.encode(x.astype(np.float64), w)
+            assert o.shape == (toks[i], hidden)
+            assert_bf16(g[off[i]:off[i + 1]], o, f"LFM2A encode, conv_k {k}, n_ff {n_ff}, clip {i} ({toks[i]} tokens)")
+
+
 def test_refusals(m2):
     off = offsets([16])
     with pytest.raises(ae.AEError) as e:
