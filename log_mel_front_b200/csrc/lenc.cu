@@ -281,22 +281,40 @@ __global__ void __launch_bounds__(128) k_lenc_dw2(const bf16 *__restrict__ y, co
   for (int k = 0; k < 9; ++k) wk[k] = make_float2(__ldg(w + ch * 9 + k), __ldg(w + (ch + 1) * 9 + k));
   const float2 bias = make_float2(__ldg(b + ch), __ldg(b + ch + 1));
   const bf16 *src = y + (int64_t)t.s2_off[c] * (32 * kLencStemCh) + ch;
+  bool trok[3];  // input rows inside the clip
+#pragma unroll
+  for (int dt = 0; dt < 3; ++dt) trok[dt] = 2 * t3 + dt - 1 >= 0 && 2 * t3 + dt - 1 < T2;
+  // two output columns per step: their 18 loads are issued before the sums
 #pragma unroll 1
-  for (int f3 = 0; f3 < 16; ++f3) {
-    float2 a = bias;
+  for (int f3 = 0; f3 < 16; f3 += 2) {
+    uint32_t v[2][9];
 #pragma unroll
-    for (int dt = 0; dt < 3; ++dt) {
-      const int tr = 2 * t3 + dt - 1;
-      if (tr < 0 || tr >= T2) continue;
+    for (int h = 0; h < 2; ++h)
 #pragma unroll
-      for (int df = 0; df < 3; ++df) {
-        const int fr = 2 * f3 + df - 1;
-        if (fr < 0) continue;
-        const uint32_t v = *reinterpret_cast<const uint32_t *>(src + ((int64_t)tr * 32 + fr) * kLencStemCh);
-        ffma2(a, wk[dt * 3 + df], make_float2(bf16lo(v), bf16hi(v)));
+      for (int dt = 0; dt < 3; ++dt)
+#pragma unroll
+        for (int df = 0; df < 3; ++df) {
+          const int fr = 2 * (f3 + h) + df - 1;
+          v[h][dt * 3 + df] =
+              trok[dt] && fr >= 0
+                  ? *reinterpret_cast<const uint32_t *>(src + ((int64_t)(2 * t3 + dt - 1) * 32 + fr) * kLencStemCh)
+                  : 0u;
+        }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float2 a = bias;
+#pragma unroll
+      for (int dt = 0; dt < 3; ++dt) {
+        if (!trok[dt]) continue;
+#pragma unroll
+        for (int df = 0; df < 3; ++df) {
+          if (2 * (f3 + h) + df - 1 < 0) continue;
+          const uint32_t x = v[h][dt * 3 + df];
+          ffma2(a, wk[dt * 3 + df], make_float2(bf16lo(x), bf16hi(x)));
+        }
       }
+      *reinterpret_cast<uint32_t *>(out + (row * 16 + f3 + h) * (int64_t)kLencStemCh + ch) = pack_bf16(a.x, a.y);
     }
-    *reinterpret_cast<uint32_t *>(out + (row * 16 + f3) * (int64_t)kLencStemCh + ch) = pack_bf16(a.x, a.y);
   }
 }
 
@@ -405,23 +423,35 @@ __global__ void __launch_bounds__(256) k_lenc_dwconv(const bf16 *__restrict__ g,
   const float2 bias = make_float2(db[ch], db[ch + 1]), sc = make_float2(aw[ch], aw[ch + 1]),
                sh = make_float2(ab[ch], ab[ch + 1]);
   int c = lenc_clip_of(tok_off, n_clips, t0 < T ? t0 : T - 1);
+  int64_t s0 = tok_off[c], e = tok_off[c + 1];  // the current clip's rows, kept in registers
   asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
 #pragma unroll 1
   for (int r = 0; r < kDwRows; ++r) {
     const int64_t tt = t0 + r;
     if (tt >= T) break;
-    while (tok_off[c + 1] <= tt) ++c;  // rows are in order; clips may be empty
-    const int64_t s0 = tok_off[c], e = tok_off[c + 1];
+    while (e <= tt) {  // rows are in order; clips may be empty
+      ++c;
+      s0 = e;
+      e = tok_off[c + 1];
+    }
     const int m0 = (int)max((int64_t)0, s0 - (tt - lo)), m1 = (int)min((int64_t)k, e - (tt - lo));
     float2 a = bias;
     if (KT > 0) {
+      if (m0 == 0 && m1 == KT) {  // the whole window inside the clip: no per-tap test
 #pragma unroll
-      for (int m = 0; m < (KT > 0 ? KT : 1); ++m)
-        if (m >= m0 && m < m1) {
+        for (int m = 0; m < (KT > 0 ? KT : 1); ++m) {
           const uint32_t v = s_g[(r + m) * 256 + threadIdx.x];
           ffma2(a, wr[m], make_float2(bf16lo(v), bf16hi(v)));
         }
+      } else {
+#pragma unroll
+        for (int m = 0; m < (KT > 0 ? KT : 1); ++m)
+          if (m >= m0 && m < m1) {
+            const uint32_t v = s_g[(r + m) * 256 + threadIdx.x];
+            ffma2(a, wr[m], make_float2(bf16lo(v), bf16hi(v)));
+          }
+      }
     } else {
       for (int m = m0; m < m1; ++m) {
         const uint32_t v = s_g[(r + m) * 256 + threadIdx.x];
