@@ -383,7 +383,7 @@ __global__ void __launch_bounds__(256) k_lenc_ln(const LencLnArgs r) {
 // memory (bf16, 16-byte cp.async, zero fill outside the batch) and each
 // thread computes two channels of every row. SiLU is y / (1 + 2^(-y log2 e))
 // with the hardware's ex2 and reciprocal.
-constexpr int kDwRows = 32;
+constexpr int kDwRows = 16;
 
 __device__ __forceinline__ float lenc_silu(float y) {
   float e, r;
